@@ -1,0 +1,374 @@
+"""FwPKM retrieve + chunk-write loop: throughput on B200 against the HBM roofline.
+
+One step = one pass of the whole hot path (addressing, gather + gated output,
+sorted write, entropy key step) over one batch of the workload, i.e. one call of
+fwpkm_run_sequence over B sequences x H heads x T tokens.  Default workload: the
+paper-scale memory (n=1024 -> N=1,048,576 slots, d=d_v=256, k=32, C=256, B=4, H=2,
+T=4096, bf16 q/v, fp32 state, key update on).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload paper|mid|tiny|needle]
+    python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+Multi-GPU (torchrun): every rank runs its own independent memories (different
+sequences); there is no collective on the data path ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_weight_memory_chunk_b200.inputs import WORKLOADS, gen_keys, gen_qvg, gen_values  # noqa: E402
+
+BY_NAME = {w.name: (i, w) for i, w in WORKLOADS.items()}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="paper", choices=["tiny", "mid", "paper", "needle"])
+    ap.add_argument("--n-iter", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def describe(w, n_iter):
+    return (f"{w.name}: n={w.n} (N={w.N:,} slots), d={w.d}, d_v={w.d_v}, k={w.k}, C={w.C}, "
+            f"B={w.B} x H={w.H} memories, T={w.T}, {w.qv} q/v, fp32 V/K, key update "
+            f"{'on' if w.key_update else 'off'}, n_iter={n_iter}")
+
+
+# --------------------------------------------------------------------------- oracle leg
+_SAMPLE_CACHE = {}
+
+
+def oracle_sample(w, n_chunks):
+    """Time the CPU oracle (as it stands) on sequence 0's H memories, first n_chunks chunks.
+
+    The inputs are drawn once per process; every call starts from a fresh copy of the
+    initial state (the oracle updates it in place)."""
+    import oracle
+    from sparse_weight_memory_chunk_b200.inputs import bf16_to_f32
+    H = w.H
+    T = min(w.T, n_chunks * w.C)
+    key = (w.name, T)
+    if key not in _SAMPLE_CACHE:
+        q, v, g = gen_qvg(w, M=H)
+        q, v, g = q[:, :T], v[:, :T], g[:, :T]
+        K1, K2 = gen_keys(w, M=H)
+        V = np.stack([gen_values(w, m) for m in range(H)])
+        qf = (bf16_to_f32(q) if w.qv == "bf16" else q).astype(np.float64)
+        vf = (bf16_to_f32(v) if w.qv == "bf16" else v).astype(np.float64)
+        _SAMPLE_CACHE[key] = (qf, vf, g.astype(np.float64), K1, K2, V)
+        oracle.build()
+    qf, vf, gf, K1, K2, V = _SAMPLE_CACHE[key]
+    k1, k2, vv = K1.copy(), K2.copy(), V.copy()
+    cfg = oracle.make_cfg(w.n, w.d, w.d_v, w.k, w.C, key_update=w.key_update)
+    t0 = time.perf_counter()
+    _, used = oracle.run_sequence_multi(cfg, qf, vf, gf, k1, k2, vv, 1, nthreads=H)
+    dt = time.perf_counter() - t0
+    return dict(tokens=T, seconds=dt, threads=used,
+                sample=f"sequence 0 ({H} heads = {H} memories, full N={w.N:,} each), tokens 0..{T - 1} "
+                       f"({n_chunks} chunks), {used} threads")
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    n_chunks = 8 if w.name in ("paper", "needle") else 16
+    times = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        info = oracle_sample(w, n_chunks)
+        if i >= args.warmup:
+            times.append(info["seconds"])
+    ms = 1000.0 * sum(times) / len(times)
+    val = info["tokens"] / (ms / 1000.0)
+    line = {"metric": "FwPKM layer tokens/s (retrieve+chunk write) at 1M slots; % of HBM roofline",
+            "value": val, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(w, 1), "sample": info["sample"]},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": info["threads"], "kind": "oracle",
+                             "sample": info["sample"]},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- clocks
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], [], set()
+        for line in out.strip().splitlines():
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx.append(float(p[2]))
+            except ValueError:
+                continue
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"), p[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- ours
+def algorithmic_bytes(w, idx, T):
+    """B_VK of one step (each touched V row loaded once and stored once, K read + written)
+    and the gather kernel's bytes per launch.  idx: [M][T][k] final addressing."""
+    import torch
+    C, k, dv = w.C, w.k, w.d_v
+    U_total = 0
+    for t0 in range(0, T, C):
+        t1 = min(T, t0 + C)
+        npair = (t1 - t0) - (1 if t1 == T else 0)
+        blk = idx[:, t0:t0 + npair, :].reshape(idx.shape[0], -1)
+        s, _ = torch.sort(blk, dim=1)
+        U_total += int((s[:, 1:] != s[:, :-1]).sum().item()) + blk.shape[0]
+    key_bytes = (2 * 4 * w.n * w.d) * w.M * ((T + C - 1) // C) if w.key_update else 0
+    b_vk = 2 * U_total * dv * 4 + key_bytes
+    es = 2 if w.qv == "bf16" else 4
+    gather_per_token = k * dv * 4 + k * 8 + dv * es + dv * 4
+    return b_vk, gather_per_token, U_total
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from sparse_weight_memory_chunk_b200 import build, fwpkm
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks = {}
+    pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pp):
+        peaks = json.load(open(pp))
+    hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
+    tc_peak = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    peak_src = "measured" if peaks else "fallback"
+
+    # inputs (per-rank independent sequences: seed offset by rank)
+    from dataclasses import replace
+    wr = replace(w, seed=w.seed + 1000 * rank) if rank else w
+    q, v, g = gen_qvg(wr)
+    K1, K2 = gen_keys(wr)
+
+    def to_dev(x):
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(x).to(dev)
+
+    qd, vd, gd = to_dev(q), to_dev(v), to_dev(g)
+    K1d, K2d = to_dev(K1), to_dev(K2)
+    Vd = torch.empty(w.M, w.N, w.d_v, device=dev)
+    for m in range(w.M):
+        Vd[m].copy_(torch.from_numpy(gen_values(wr, m)))
+    cfg = fwpkm.make_config(w.n, w.d, w.d_v, w.k, w.C, w.M, w.qv == "bf16", key_update=w.key_update)
+    st = fwpkm.State(cfg, K1d, K2d, Vd, w.T)
+    o = torch.empty(w.M, w.T, w.d_v, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        st.run_sequence(qd, vd, gd, o, n_iter=args.n_iter)
+
+    # warm-up; find the dominant kernel kind by timing each kind once
+    for _ in range(max(args.warmup, 1)):
+        step()
+    kinds = {}
+    for name in ("gather", "write", "score", "cartesian", "sort", "address"):
+        st.profile_kernel(name)
+        step()
+        ms, n = st.kernel_time()
+        kinds[name] = (ms, n)
+    st.profile_kernel(0)
+    dominant = max(kinds, key=lambda k_: kinds[k_][0])
+    st.profile_kernel(dominant)
+    st.sync()
+
+    clocks = Clocks(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    l0 = fwpkm.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    launches = fwpkm.launch_count() - l0
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    dom_ms, dom_n = st.kernel_time()
+    st.profile_kernel(0)
+    st.sync()
+    ms_step = ms_total / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    tokens_per_step = w.B * w.T * args.n_iter
+    value = tokens_per_step * world / (ms_step / 1000.0)
+
+    # algorithmic traffic of the step (measured unique rows) and roofline
+    idx = torch.empty(w.M, w.T, w.k, dtype=torch.int32, device=dev)
+    st.last_addressing(w.T, idx_out=idx)
+    torch.cuda.synchronize()
+    b_vk, gather_per_token, U = algorithmic_bytes(w, idx, w.T)
+    b_vk *= args.n_iter
+    flops = 2 * w.n * w.d * w.M * w.T * args.n_iter * (2 if w.key_update else 1)
+    t_roof = max(b_vk / (hbm_peak * 1e9), flops / (tc_peak * 1e12))
+    step_frac = t_roof / (ms_step / 1000.0)
+    avg_launch_s = (dom_ms / 1000.0) / max(dom_n, 1)
+    if dominant == "gather":
+        per_launch = gather_per_token * w.M * w.C
+        achieved = per_launch / avg_launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": None}
+    elif dominant == "write":
+        per_launch = 2 * (U / max(1, (w.T + w.C - 1) // w.C)) * w.d_v * 4
+        achieved = per_launch / avg_launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": None}
+    else:
+        # contraction-shaped kernels: algorithmic FLOPs per launch against the tensor peak
+        nchunks = (w.T + w.C - 1) // w.C
+        launches_per_step = max(1, dom_n)
+        per_launch = flops / (args.n_iter * (2 if w.key_update else 1)) / (nchunks if w.key_update else 1)
+        if dominant == "address":
+            per_launch = 2 * w.n * w.d * w.M * w.C
+        achieved = per_launch / avg_launch_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": achieved / tc_peak, "traffic": None}
+        del launches_per_step
+    roof["kernel"] = dominant
+    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if roof['unit'] == 'GB/s' else 'bf16_tflops_sustained'})"
+    roof["avg_launch_us"] = avg_launch_s * 1e6
+    roof["launches_timed"] = dom_n
+
+    line = {"metric": "FwPKM layer tokens/s (retrieve+chunk write) at 1M slots; % of HBM roofline",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": describe(w, args.n_iter),
+                       "l2": "inputs larger than L2: V is 8 GiB per GPU and a step touches ~2.1 GB of V rows"
+                             if w.name == "paper" else "V state larger than L2" if w.N * w.d_v * 4 * w.M > 126e6
+                             else "L2-resident (tiny)",
+                       "parallelism": f"{world} GPU(s), independent memories per rank"},
+            "roofline": roof,
+            "step_roofline": {"t_roof_ms": t_roof * 1e3, "frac": step_frac, "bytes_VK": b_vk, "flops_tc": flops,
+                              "unique_rows": U, "definition": "max(F_tc/P_tc, B_VK/BW_HBM) / t_step"},
+            "kernel_ms_one_step": {k_: round(v_[0], 4) for k_, v_ in kinds.items()},
+            "clocks": clk, "gpu_launches": int(launches)}
+
+    # end to end through the public API with host buffers
+    if not args.no_e2e:
+        qh = torch.empty_like(qd, device="cpu").pin_memory()
+        vh = torch.empty_like(vd, device="cpu").pin_memory()
+        gh = torch.empty_like(gd, device="cpu").pin_memory()
+        oh = torch.empty_like(o, device="cpu").pin_memory()
+        qh.copy_(qd); vh.copy_(vd); gh.copy_(gd)
+        torch.cuda.synchronize()
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True); vd.copy_(vh, non_blocking=True); gd.copy_(gh, non_blocking=True)
+            st.run_sequence(qd, vd, gd, o, n_iter=args.n_iter)
+            oh.copy_(o, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1) / args.steps
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        bi = sum(x.numel() * x.element_size() for x in (qh, vh, gh))
+        line["e2e"] = {"value": tokens_per_step * world / (ems / 1000.0), "unit": "tokens/s",
+                       "h2d_bytes_per_step": bi, "d2h_bytes_per_step": oh.numel() * oh.element_size(),
+                       "ms_per_step": ems}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_chunks = 8 if w.name in ("paper", "needle") else 16
+        info = oracle_sample(w, n_chunks)
+        line["cpu_baseline"] = {"value": info["tokens"] / info["seconds"], "unit": "tokens/s",
+                                "cores": info["threads"], "kind": "oracle", "sample": info["sample"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    st.destroy()
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    _, w = BY_NAME[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * fwpkm.h -- C ABI of the B200 FwPKM retrieve + chunk-write library (libfwpkm.so).
+ *
+ * Fast-weight Product Key Memory keeps, per independent memory (one per sequence
+ * and head), a value table V of N = n*n rows and two sub-key codebooks K1, K2 of n
+ * keys each.  For every token of a chunk it reads the memory (product-key top-k
+ * with inverse-distance scores, softmax weights, weighted sum of k value rows,
+ * gated residual output); after the chunk it writes the memory (one gradient step
+ * of the gated lookahead reconstruction loss, averaged per row by its read count)
+ * and, optionally, takes an entropy gradient step on K1 and K2.
+ *
+ * Sources (page title, section):
+ *   "快速权重积键值记忆 Fast-weight Product Key Memory" (rainbus summary), method
+ *     steps 1-5 and the PKM prerequisite;
+ *   "Fast-weight Product Key Memory" (paperlayer summary of arXiv 2601.00671v2),
+ *     §2.2, §3.1-§3.5, §A.1-§A.5 and App. B.
+ *
+ * Conventions shared by every call:
+ *   - Every device buffer is allocated and owned by the caller.  The library never
+ *     allocates device memory; its scratch lives in the caller's workspace.
+ *   - Memories are independent and laid out memory-major: m = b*H + head.
+ *     Sequence inputs are [M][T][width] row-major; q's first d/2 entries are
+ *     half 1.  V is [M][n*n][d_v] fp32 with slot i = a*n + b (a: half-1 sub-key,
+ *     b: half-2 sub-key); K1, K2 are [M][n][d/2] fp32.
+ *   - q and v are fp32 or bf16 (cfg.qv_dtype); g, o and the state are fp32.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
+ *     enqueues work on it and returns; results are ready when the stream is.
+ *   - Calls return a status and never throw.  Argument checks run synchronously
+ *     before anything is enqueued (then nothing is enqueued).  Errors detected on
+ *     the device are latched in a status word returned by fwpkm_sync() and by the
+ *     next call on the same state.
+ *   - Results are deterministic: the same inputs give bit-identical outputs.
+ */
+#ifndef FWPKM_H
+#define FWPKM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FWPKM_OK = 0,
+  FWPKM_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned buffer            */
+  FWPKM_ERR_UNSUPPORTED = -2, /* valid but outside the supported shape limits          */
+  FWPKM_ERR_WORKSPACE = -3,   /* workspace smaller than fwpkm_workspace_size()         */
+  FWPKM_ERR_CUDA = -4,        /* a CUDA runtime call failed                            */
+  FWPKM_ERR_TIMEOUT = -5,     /* a bounded device-side wait gave up                    */
+  FWPKM_ERR_STATE = -6        /* call out of order (write_chunk without forward_chunk) */
+} fwpkm_status;
+
+typedef enum { FWPKM_F32 = 0, FWPKM_BF16 = 1 } fwpkm_dtype;
+
+/* cfg.flags */
+enum {
+  FWPKM_KEY_UPDATE = 1,  /* entropy step on K1, K2 after each chunk (rainbus step 5; paperlayer §3.4) */
+  FWPKM_TARGET_NORM = 2, /* z-score the reconstruction target per token (paperlayer §A.3)            */
+  FWPKM_LOOKAHEAD = 4,   /* target of token t is v_{t+1} (paperlayer §A.1); off: v_t (rainbus step 4) */
+  FWPKM_GATE_WEIGHT = 8  /* weight each token's loss by g_t (paperlayer §A.5)                        */
+};
+#define FWPKM_DEFAULT_FLAGS (FWPKM_TARGET_NORM | FWPKM_LOOKAHEAD | FWPKM_GATE_WEIGHT)
+
+/* Shape and hyper-parameters of M independent memories.
+ * Supported limits (else FWPKM_ERR_UNSUPPORTED):
+ *   1 <= k <= 32, k <= n <= 4096, d even with 8 <= d <= 512, d_v % 4 == 0 with
+ *   4 <= d_v <= 1024, 1 <= chunk <= 1024 with chunk*k <= 16384, num_mem >= 1. */
+typedef struct {
+  int n;         /* sub-keys per codebook; the memory has N = n*n slots              */
+  int d;         /* query width (two halves of d/2)                                  */
+  int d_v;       /* value width                                                      */
+  int k;         /* per-half top-k and final top-k                                   */
+  int chunk;     /* C, tokens per fast-weight update                                 */
+  int num_mem;   /* M independent memories                                           */
+  int qv_dtype;  /* fwpkm_dtype of q and v                                           */
+  float eps_idw; /* IDW score sigma = -log(eps_idw + ||q_j - K_j[a]||^2)              */
+  float eps_norm;/* z-score: (u - mean) / sqrt(var + eps_norm)                       */
+  float lr_key;  /* step size of the key update                                      */
+  unsigned flags;/* FWPKM_* flags                                                    */
+} fwpkm_config;
+
+/* Opaque host-side handle.  It records the caller's state pointers and the carved
+ * workspace; it owns no device memory (only CUDA streams/events/graphs). */
+typedef struct fwpkm_state fwpkm_state;
+
+/* Bytes of device workspace needed for sequences of up to max_T tokens.
+ * Returns FWPKM_ERR_INVALID_ARG / FWPKM_ERR_UNSUPPORTED for a bad config. */
+fwpkm_status fwpkm_workspace_size(const fwpkm_config* cfg, int max_T, size_t* bytes);
+
+/* Validate cfg, record the caller-owned state (K1, K2 [M][n][d/2] fp32 and
+ * V [M][n*n][d_v] fp32, all device pointers, 16-byte aligned) and carve the
+ * workspace (device, >= fwpkm_workspace_size(cfg, max_T), 256-byte aligned).
+ * The state tensors are read and written in place by later calls; the caller
+ * keeps them and the workspace alive until fwpkm_destroy_state().  Nothing is
+ * enqueued.  (Host-only; the state's memory can persist across sequences, which
+ * is how memory carries over sequence boundaries, paperlayer §E.1.) */
+fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, float* V, int max_T,
+                              void* workspace, size_t ws_bytes, fwpkm_state** out);
+
+/* Read phase of one chunk for all M memories (rainbus steps 2-3; paperlayer §2.2,
+ * §3.2, §A.2): per-half IDW top-k, restricted Cartesian top-k, softmax weights,
+ * vhat_t = sum_i s'_{t,i} V_i and o_t = g_t vhat_t + (1 - g_t) v_t, all against
+ * the state left by the previous chunk (paperlayer §3.1 causality).
+ *   q  device, element (m, t, e) at q[(m*seq_stride + t)*d + e]   (qv_dtype)
+ *   v  device, element (m, t, e) at v[(m*seq_stride + t)*d_v + e] (qv_dtype)
+ *   g  device fp32, (m, t) at g[m*seq_stride + t]
+ *   c_len tokens in this chunk, 1 <= c_len <= cfg.chunk; seq_stride >= c_len
+ *   o  device fp32 output, (m, t, e) at o[(m*seq_stride + t)*d_v + e]
+ *   idx_out [M][c_len][k] int32 and w_out [M][c_len][k] fp32 (device, nullable):
+ *      selected slots in rank order (score desc, slot asc) and their weights.
+ * q, v, g must stay valid until the matching fwpkm_write_chunk() has run. */
+fwpkm_status fwpkm_forward_chunk(fwpkm_state* st, const void* q, const void* v, const float* g,
+                                 int c_len, int seq_stride, float* o, int32_t* idx_out,
+                                 float* w_out, void* stream);
+
+/* Write phase of the chunk last passed to fwpkm_forward_chunk (rainbus steps 4-5;
+ * paperlayer §3.3, §3.4, §A.1-§A.5): for every slot i read by a token that has a
+ * target, V_i -= (sum_t s'_{t,i} g_t (vhat_t - z(u_t))) / N_read,i with u_t the
+ * lookahead value; then, if FWPKM_KEY_UPDATE, K_j -= lr_key * dL_addr/dK_j with
+ * L_addr = -H(pbar_1) - H(pbar_2) taken at the keys the chunk was read with.
+ *   v_next  device, value of the token after the chunk for each memory, element
+ *           (m, e) at v_next[m*seq_stride*d_v + e] (same seq_stride as the forward
+ *           call), or NULL when the chunk ends the sequence: its last token then has
+ *           no lookahead target and is left out of the write and of N_read.
+ * Returns FWPKM_ERR_STATE if no forward_chunk is pending. */
+fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream);
+
+/* The whole chunk-sequential loop over a sequence of T tokens (1 <= T <= max_T)
+ * for all M memories, repeated n_iter >= 1 times over the same input with the
+ * state carried across chunks and passes (paperlayer §3.1, §4.3 iterative
+ * reading).  Equivalent to forward_chunk/write_chunk over consecutive chunks with
+ * v_next = the following token (NULL for the last chunk), but scheduled as one
+ * stream-ordered program (addressing, which never depends on V, runs ahead of the
+ * value loop).  q, v, g, o use the forward_chunk layout with seq_stride = T;
+ * o receives the final pass.  T = 0 is a no-op. */
+fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, const float* g,
+                                int T, int n_iter, float* o, void* stream);
+
+/* Copy the slot indices and softmax weights that the most recent call computed for
+ * tokens [0, T) of every memory (final pass of fwpkm_run_sequence, or the chunk of
+ * fwpkm_forward_chunk with T <= c_len) into idx_out [M][T][k] int32 and
+ * w_out [M][T][k] fp32 (device, either nullable).  Enqueued on `stream`.  Used for
+ * inspection and for comparing selections against a reference. */
+fwpkm_status fwpkm_last_addressing(fwpkm_state* st, int T, int32_t* idx_out, float* w_out, void* stream);
+
+/* Wait for `stream` and return the latched device status (FWPKM_OK,
+ * FWPKM_ERR_TIMEOUT, ...), clearing it. */
+fwpkm_status fwpkm_sync(fwpkm_state* st, void* stream);
+
+/* Release the handle (streams, events, graphs).  Caller buffers are untouched. */
+void fwpkm_destroy_state(fwpkm_state* st);
+
+/* Static description of a status code. */
+const char* fwpkm_status_string(fwpkm_status s);
+
+/* Number of kernels this library has launched in this process (graph replays count
+ * every kernel node).  Used to report how many launches a timed region made. */
+uint64_t fwpkm_launch_count(void);
+
+/* Per-kernel timing with CUDA events recorded on the launching stream around every
+ * launch of the given kernel kind (0 = none).  Kinds: 1 gather, 2 write, 3 score,
+ * 4 cartesian, 5 sort, 6 address.  fwpkm_kernel_time() waits for the events and
+ * returns the summed duration (ms) and the number of timed launches since the last
+ * reset, then resets.  Graph replays overwrite their own events, so after graph
+ * replays it covers the last replay. */
+fwpkm_status fwpkm_profile_kernel(fwpkm_state* st, int kind);
+fwpkm_status fwpkm_kernel_time(fwpkm_state* st, double* total_ms, int* launches);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FWPKM_H */

@@ -1,0 +1,341 @@
+// fwpkm.cu -- the C ABI of libfwpkm.so: validation, workspace carve-up and the
+// chunk-sequential schedule (Fast-weight Product Key Memory (paperlayer summary)
+// §3.1: reads in a chunk use the fast weights left by earlier chunks; the write
+// follows the chunk; App. B: forward, then memorization, then addressing).
+//
+// Scheduling observation used by fwpkm_run_sequence: the addressing (scores,
+// top-k, Cartesian search, the pair sort) depends on q and the keys only, never on
+// V.  With the key update off the keys are constant, so the addressing of every
+// chunk and every pass is computed once, up front, in a few large launches, and only
+// the value loop (gather, write) stays chunk-sequential.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "fwpkm_internal.cuh"
+
+using namespace fwpkm;
+
+static std::atomic<uint64_t> g_launches{0};
+
+struct fwpkm_state {
+  fwpkm_config cfg;
+  Dims dm;
+  Work wk;
+  float *K1, *K2, *V;
+  // streaming (forward_chunk -> write_chunk)
+  int pending;
+  const void *q, *v;
+  const float* g;
+  int len;
+  long long stride;
+  // per-kernel timing
+  int prof_kind;
+  std::vector<cudaEvent_t> ev;
+  int ev_used;
+};
+
+namespace {
+
+constexpr size_t ALIGN = 256;
+
+size_t align_up(size_t x) { return (x + ALIGN - 1) & ~(ALIGN - 1); }
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+fwpkm_status check_cfg(const fwpkm_config* c) {
+  if (!c) return FWPKM_ERR_INVALID_ARG;
+  if (c->n <= 0 || c->d <= 0 || c->d_v <= 0 || c->k <= 0 || c->chunk <= 0 || c->num_mem <= 0)
+    return FWPKM_ERR_INVALID_ARG;
+  if (c->qv_dtype != FWPKM_F32 && c->qv_dtype != FWPKM_BF16) return FWPKM_ERR_INVALID_ARG;
+  if (!(c->eps_idw >= 0.f) || !(c->eps_norm >= 0.f)) return FWPKM_ERR_INVALID_ARG;
+  if (c->d % 2 != 0 || c->d_v % 4 != 0) return FWPKM_ERR_INVALID_ARG;
+  if (c->k > c->n) return FWPKM_ERR_INVALID_ARG;
+  if (c->k > 32 || c->n > 4096 || c->d < 8 || c->d > 512 || c->d_v > 1024 || c->chunk > 1024 ||
+      (long long)c->chunk * c->k > 16384)
+    return FWPKM_ERR_UNSUPPORTED;
+  return FWPKM_OK;
+}
+
+Dims make_dims(const fwpkm_config* c) {
+  Dims d;
+  d.n = c->n; d.h = c->d / 2; d.d = c->d; d.dv = c->d_v; d.k = c->k; d.C = c->chunk; d.M = c->num_mem;
+  d.N = (long long)c->n * c->n;
+  d.qv_bf16 = c->qv_dtype == FWPKM_BF16;
+  d.eps_idw = c->eps_idw; d.eps_norm = c->eps_norm; d.lr_key = c->lr_key; d.flags = c->flags;
+  return d;
+}
+
+size_t qv_size(const Dims& d) { return d.qv_bf16 ? 2 : 4; }
+
+const void* offs(const void* p, long long elems, size_t esize) {
+  return p ? (const void*)((const char*)p + elems * (long long)esize) : nullptr;
+}
+
+fwpkm_status last_cuda() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    fprintf(stderr, "fwpkm: CUDA error: %s\n", cudaGetErrorString(e));
+    return FWPKM_ERR_CUDA;
+  }
+  return FWPKM_OK;
+}
+
+template <class F>
+void run(fwpkm_state* st, int kind, cudaStream_t s, F&& f) {
+  const bool prof = st->prof_kind == kind && st->ev_used + 2 <= (int)st->ev.size();
+  if (prof) cudaEventRecord(st->ev[st->ev_used], s);
+  int nl = f();
+  if (prof) {
+    cudaEventRecord(st->ev[st->ev_used + 1], s);
+    st->ev_used += 2;
+  }
+  g_launches += (uint64_t)nl;
+}
+
+}  // namespace
+
+namespace fwpkm {
+
+size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
+  const size_t M = d.M, k = d.k, C = d.C, n = d.n, dv = d.dv;
+  const size_t T = max_T;
+  const size_t nch = (T + C - 1) / C;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return p;
+  };
+  Work x;
+  x.max_T = max_T;
+  x.max_chunks = (int)nch;
+  x.status = (int*)take(sizeof(int));
+  x.A = (int32_t*)take(4 * M * 2 * T * k);
+  x.Dsv = (float*)take(4 * M * 2 * T * k);
+  x.idx = (int32_t*)take(4 * M * T * k);
+  x.w = (float*)take(4 * M * T * k);
+  x.pair_tr = (uint32_t*)take(4 * M * nch * C * k);
+  x.seg_start = (int32_t*)take(4 * M * nch * (C * k + 1));
+  x.seg_slot = (int32_t*)take(4 * M * nch * C * k);
+  x.nseg = (int32_t*)take(4 * M * nch);
+  x.resid = (float*)take(4 * M * C * dv);
+  if (d.flags & FWPKM_KEY_UPDATE) {
+    x.Dfull = (float*)take(4 * M * 2 * C * n);
+    x.Z = (float*)take(4 * M * 2 * C);
+    x.lp = (float*)take(4 * M * 2 * n);
+    x.Lt = (float*)take(4 * M * 2 * C);
+  } else {
+    x.Dfull = nullptr; x.Z = nullptr; x.lp = nullptr; x.Lt = nullptr;
+  }
+  if (w) *w = x;
+  return off;
+}
+
+}  // namespace fwpkm
+
+extern "C" {
+
+const char* fwpkm_status_string(fwpkm_status s) {
+  switch (s) {
+    case FWPKM_OK: return "ok";
+    case FWPKM_ERR_INVALID_ARG: return "invalid argument";
+    case FWPKM_ERR_UNSUPPORTED: return "unsupported shape";
+    case FWPKM_ERR_WORKSPACE: return "workspace too small";
+    case FWPKM_ERR_CUDA: return "CUDA error";
+    case FWPKM_ERR_TIMEOUT: return "device wait timed out";
+    case FWPKM_ERR_STATE: return "call out of order";
+  }
+  return "unknown status";
+}
+
+uint64_t fwpkm_launch_count(void) { return g_launches.load(); }
+
+fwpkm_status fwpkm_workspace_size(const fwpkm_config* cfg, int max_T, size_t* bytes) {
+  fwpkm_status s = check_cfg(cfg);
+  if (s != FWPKM_OK) return s;
+  if (!bytes || max_T < 1) return FWPKM_ERR_INVALID_ARG;
+  *bytes = workspace_bytes(make_dims(cfg), max_T, nullptr, nullptr);
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, float* V, int max_T,
+                              void* workspace, size_t ws_bytes, fwpkm_state** out) {
+  fwpkm_status s = check_cfg(cfg);
+  if (s != FWPKM_OK) return s;
+  if (!out || !K1 || !K2 || !V || !workspace || max_T < 1) return FWPKM_ERR_INVALID_ARG;
+  if (!aligned(K1, 16) || !aligned(K2, 16) || !aligned(V, 16) || !aligned(workspace, ALIGN))
+    return FWPKM_ERR_INVALID_ARG;
+  Dims dm = make_dims(cfg);
+  if (ws_bytes < workspace_bytes(dm, max_T, nullptr, nullptr)) return FWPKM_ERR_WORKSPACE;
+  fwpkm_state* st = new (std::nothrow) fwpkm_state();
+  if (!st) return FWPKM_ERR_INVALID_ARG;
+  st->cfg = *cfg;
+  st->dm = dm;
+  workspace_bytes(dm, max_T, &st->wk, (char*)workspace);
+  st->K1 = K1; st->K2 = K2; st->V = V;
+  st->pending = 0;
+  st->prof_kind = 0;
+  st->ev_used = 0;
+  if (cudaMemset(st->wk.status, 0, sizeof(int)) != cudaSuccess) {
+    delete st;
+    return FWPKM_ERR_CUDA;
+  }
+  *out = st;
+  return FWPKM_OK;
+}
+
+void fwpkm_destroy_state(fwpkm_state* st) {
+  if (!st) return;
+  for (cudaEvent_t e : st->ev) cudaEventDestroy(e);
+  delete st;
+}
+
+static fwpkm_status peek_status(fwpkm_state* st) {
+  // A latched device error is reported by the next call (non-blocking check).
+  (void)st;
+  return last_cuda();
+}
+
+fwpkm_status fwpkm_forward_chunk(fwpkm_state* st, const void* q, const void* v, const float* g, int c_len,
+                                 int seq_stride, float* o, int32_t* idx_out, float* w_out, void* stream) {
+  if (!st || !q || !v || !g || !o) return FWPKM_ERR_INVALID_ARG;
+  const Dims& d = st->dm;
+  if (c_len < 1 || c_len > d.C || c_len > st->wk.max_T || seq_stride < c_len) return FWPKM_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4)) return FWPKM_ERR_INVALID_ARG;
+  fwpkm_status ps = peek_status(st);
+  if (ps != FWPKM_OK) return ps;
+  cudaStream_t s = (cudaStream_t)stream;
+  const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
+  run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, q, seq_stride, 0, c_len, ku, s); });
+  run(st, KK_CART, s, [&] { return launch_cartesian(d, st->wk, 0, c_len, idx_out, w_out, s); });
+  run(st, KK_GATHER, s, [&] {
+    return launch_gather(d, st->wk, st->V, v, g, seq_stride, 0, c_len, o, false, nullptr, s);
+  });
+  st->pending = 1;
+  st->q = q; st->v = v; st->g = g; st->len = c_len; st->stride = seq_stride;
+  return last_cuda();
+}
+
+fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream) {
+  if (!st) return FWPKM_ERR_INVALID_ARG;
+  if (!st->pending) return FWPKM_ERR_STATE;
+  if (v_next && !aligned(v_next, 4)) return FWPKM_ERR_INVALID_ARG;
+  const Dims& d = st->dm;
+  cudaStream_t s = (cudaStream_t)stream;
+  const bool last_has_target = (v_next != nullptr) || !(d.flags & FWPKM_LOOKAHEAD);
+  run(st, KK_OTHER, s, [&] { return launch_resid(d, st->wk, st->v, st->g, st->stride, st->len, v_next, s); });
+  run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, st->wk, 0, st->len, last_has_target, s); });
+  run(st, KK_WRITE, s, [&] { return launch_write(d, st->wk, st->V, 0, s); });
+  if (d.flags & FWPKM_KEY_UPDATE)
+    run(st, KK_ADDR, s, [&] { return launch_address(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, s); });
+  st->pending = 0;
+  return last_cuda();
+}
+
+fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, const float* g, int T,
+                                int n_iter, float* o, void* stream) {
+  if (!st) return FWPKM_ERR_INVALID_ARG;
+  if (T == 0) return FWPKM_OK;
+  if (!q || !v || !g || !o || T < 0 || T > st->wk.max_T || n_iter < 1) return FWPKM_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4)) return FWPKM_ERR_INVALID_ARG;
+  fwpkm_status ps = peek_status(st);
+  if (ps != FWPKM_OK) return ps;
+  st->pending = 0;
+  const Dims& d = st->dm;
+  const size_t es = qv_size(d);
+  const int C = d.C;
+  const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
+  const bool la = (d.flags & FWPKM_LOOKAHEAD) != 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int nch = (T + C - 1) / C;
+
+  auto value_chunk = [&](int c) {
+    const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
+    const void* vc = offs(v, (long long)t0 * d.dv, es);
+    const void* vn = (t0 + len < T) ? offs(v, (long long)(t0 + len) * d.dv, es) : nullptr;
+    run(st, KK_GATHER, s, [&] {
+      return launch_gather(d, st->wk, st->V, vc, g + t0, T, t0, len, o + (long long)t0 * d.dv, true, vn, s);
+    });
+    run(st, KK_WRITE, s, [&] { return launch_write(d, st->wk, st->V, t0, s); });
+  };
+
+  if (!ku) {
+    // keys are frozen: address every token once, for all passes
+    run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, q, T, 0, T, false, s); });
+    run(st, KK_CART, s, [&] { return launch_cartesian(d, st->wk, 0, T, nullptr, nullptr, s); });
+    run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, st->wk, 0, T, !la, s); });
+    for (int pass = 0; pass < n_iter; ++pass)
+      for (int c = 0; c < nch; ++c) value_chunk(c);
+  } else {
+    for (int pass = 0; pass < n_iter; ++pass) {
+      for (int c = 0; c < nch; ++c) {
+        const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
+        const void* qc = offs(q, (long long)t0 * d.d, es);
+        run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, qc, T, t0, len, true, s); });
+        run(st, KK_CART, s, [&] { return launch_cartesian(d, st->wk, t0, len, nullptr, nullptr, s); });
+        run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, st->wk, t0, len, !la || (t0 + len < T), s); });
+        value_chunk(c);
+        run(st, KK_ADDR, s, [&] { return launch_address(d, st->wk, st->K1, st->K2, qc, T, len, s); });
+      }
+    }
+  }
+  return last_cuda();
+}
+
+fwpkm_status fwpkm_last_addressing(fwpkm_state* st, int T, int32_t* idx_out, float* w_out, void* stream) {
+  if (!st || T < 1 || T > st->wk.max_T) return FWPKM_ERR_INVALID_ARG;
+  const Dims& d = st->dm;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t row = (size_t)T * d.k, src_pitch = (size_t)st->wk.max_T * d.k;
+  for (int m = 0; m < d.M; ++m) {
+    if (idx_out && cudaMemcpyAsync(idx_out + m * row, st->wk.idx + m * src_pitch, row * 4,
+                                   cudaMemcpyDeviceToDevice, s) != cudaSuccess) return last_cuda();
+    if (w_out && cudaMemcpyAsync(w_out + m * row, st->wk.w + m * src_pitch, row * 4,
+                                 cudaMemcpyDeviceToDevice, s) != cudaSuccess) return last_cuda();
+  }
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_sync(fwpkm_state* st, void* stream) {
+  if (!st) return FWPKM_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return last_cuda() == FWPKM_OK ? FWPKM_ERR_CUDA : FWPKM_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpy(&h, st->wk.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FWPKM_ERR_CUDA;
+  if (h != DEV_OK) {
+    cudaMemset(st->wk.status, 0, sizeof(int));
+    return h == DEV_TIMEOUT ? FWPKM_ERR_TIMEOUT : FWPKM_ERR_CUDA;
+  }
+  return last_cuda();
+}
+
+fwpkm_status fwpkm_profile_kernel(fwpkm_state* st, int kind) {
+  if (!st || kind < 0 || kind > KK_OTHER) return FWPKM_ERR_INVALID_ARG;
+  if (kind != 0 && st->ev.empty()) {
+    st->ev.resize(4096);
+    for (auto& e : st->ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return FWPKM_ERR_CUDA;
+  }
+  st->prof_kind = kind;
+  st->ev_used = 0;
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_kernel_time(fwpkm_state* st, double* total_ms, int* launches) {
+  if (!st || !total_ms || !launches) return FWPKM_ERR_INVALID_ARG;
+  double tot = 0.0;
+  for (int i = 0; i + 1 < st->ev_used; i += 2) {
+    if (cudaEventSynchronize(st->ev[i + 1]) != cudaSuccess) return FWPKM_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, st->ev[i], st->ev[i + 1]) != cudaSuccess) return FWPKM_ERR_CUDA;
+    tot += ms;
+  }
+  *total_ms = tot;
+  *launches = st->ev_used / 2;
+  st->ev_used = 0;
+  return FWPKM_OK;
+}
+
+}  // extern "C"

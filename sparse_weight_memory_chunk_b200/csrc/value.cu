@@ -1,0 +1,290 @@
+// value.cu -- the HBM-bound value path: sparse read + gated output, reconstruction
+// residuals, and the atomic-free fast-weight write.
+//
+// Fast-weight Product Key Memory (rainbus summary), method steps 2-4:
+//   vhat_t = sum_{i in I_t} s'_{t,i} V_i;  o_t = g_t vhat_t + (1 - g_t) v_t;
+//   L_mem = 1/2 sum_t g_t ||target_t - vhat_t||^2;  V_i -= (dL_mem/dV_i) / N_read,i.
+// (paperlayer summary) §A.1 target = v_{t+1}; §A.3 z-scored target, no clipping;
+// §A.4 summed (not averaged) loss, so the step is exactly the gradient; §A.5 gate
+// weighting; §3.3 read-count averaging.
+//
+// Rows are moved as 16-byte vectors: a warp covers 512 contiguous bytes per load.
+#include "fwpkm_internal.cuh"
+
+namespace fwpkm {
+
+constexpr int VAL_WARPS = 8;
+
+template <typename VT>
+__device__ __forceinline__ float4 load4(const VT* p, long long i4);
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* p, long long i4) {
+  return reinterpret_cast<const float4*>(p)[i4];
+}
+template <>
+__device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p, long long i4) {
+  const __nv_bfloat162* q = reinterpret_cast<const __nv_bfloat162*>(p) + 2 * i4;
+  float2 a = __bfloat1622float2(q[0]), b = __bfloat1622float2(q[1]);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// r = gw * (vhat - tau), tau = z(u) or u.  Shared by the fused and the streaming path
+// so both give the same bits.
+template <typename VT, int VPL>
+__device__ __forceinline__ void residual(const Dims& dm, const float4 (&vhat)[VPL], const VT* u,
+                                         float gw, float4 (&r)[VPL], int lane) {
+  const int dv4 = dm.dv >> 2;
+  float4 x[VPL];
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) {
+    int e4 = lane + 32 * c;
+    x[c] = e4 < dv4 ? load4<VT>(u, e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    s += (x[c].x + x[c].y) + (x[c].z + x[c].w);
+  }
+  if (dm.flags & FWPKM_TARGET_NORM) {
+    const float mean = warp_sum(s) / (float)dm.dv;
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) {
+      int e4 = lane + 32 * c;
+      if (e4 < dv4) {
+        float a = x[c].x - mean, b = x[c].y - mean, cc = x[c].z - mean, dd = x[c].w - mean;
+        ss += (a * a + b * b) + (cc * cc + dd * dd);
+      }
+    }
+    const float var = warp_sum(ss) / (float)dm.dv;
+    const float inv = 1.0f / sqrtf(var + dm.eps_norm);
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) {
+      x[c].x = (x[c].x - mean) * inv; x[c].y = (x[c].y - mean) * inv;
+      x[c].z = (x[c].z - mean) * inv; x[c].w = (x[c].w - mean) * inv;
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) {
+    r[c].x = gw * (vhat[c].x - x[c].x); r[c].y = gw * (vhat[c].y - x[c].y);
+    r[c].z = gw * (vhat[c].z - x[c].z); r[c].w = gw * (vhat[c].w - x[c].w);
+  }
+}
+
+// Lookahead source of local token i, or nullptr if it has no target.
+template <typename VT>
+__device__ __forceinline__ const VT* target_src(const Dims& dm, const VT* v, const VT* v_next,
+                                                long long stride, int m, int i, int len) {
+  if (!(dm.flags & FWPKM_LOOKAHEAD)) return v + ((long long)m * stride + i) * dm.dv;
+  if (i + 1 < len) return v + ((long long)m * stride + i + 1) * dm.dv;
+  if (v_next) return v_next + (long long)m * stride * dm.dv;
+  return nullptr;
+}
+
+// ---------------------------------------------------------------------------
+// Gather: one warp per (memory, token).  k rows of d_v fp32 are read in rank order
+// with 16-byte loads; vhat accumulates in fp32 in that order.
+// ---------------------------------------------------------------------------
+template <typename VT, int VPL>
+__global__ void __launch_bounds__(VAL_WARPS * 32)
+gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict__ v,
+              const float* __restrict__ g, long long stride, int wt0, int len, float* __restrict__ o,
+              int fuse_resid, const VT* __restrict__ v_next) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * VAL_WARPS + warp;
+  const int m = blockIdx.y;
+  if (i >= len) return;
+  const int k = dm.k, dv4 = dm.dv >> 2;
+  const long long tok = (long long)wt0 + i;
+  int myslot = 0;
+  float myw = 0.f;
+  if (lane < k) {
+    myslot = w.idx[((size_t)m * w.max_T + tok) * k + lane];
+    myw = w.w[((size_t)m * w.max_T + tok) * k + lane];
+  }
+  const float4* Vm = reinterpret_cast<const float4*>(V + (size_t)m * dm.N * dm.dv);
+  float4 acc[VPL];
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int r = 0; r < k; ++r) {
+    const int slot = __shfl_sync(0xffffffffu, myslot, r);
+    const float wr = __shfl_sync(0xffffffffu, myw, r);
+    const float4* row = Vm + (size_t)slot * dv4;
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) {
+      int e4 = lane + 32 * c;
+      if (e4 < dv4) {
+        float4 x = row[e4];
+        acc[c].x = fmaf(wr, x.x, acc[c].x); acc[c].y = fmaf(wr, x.y, acc[c].y);
+        acc[c].z = fmaf(wr, x.z, acc[c].z); acc[c].w = fmaf(wr, x.w, acc[c].w);
+      }
+    }
+  }
+  const float gt = g[(long long)m * stride + i];
+  const VT* vt = v + ((long long)m * stride + i) * dm.dv;
+  float4* orow = reinterpret_cast<float4*>(o + ((long long)m * stride + i) * dm.dv);
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) {
+    int e4 = lane + 32 * c;
+    if (e4 < dv4) {
+      float4 x = load4<VT>(vt, e4);
+      float4 y;
+      y.x = gt * acc[c].x + (1.f - gt) * x.x; y.y = gt * acc[c].y + (1.f - gt) * x.y;
+      y.z = gt * acc[c].z + (1.f - gt) * x.z; y.w = gt * acc[c].w + (1.f - gt) * x.w;
+      orow[e4] = y;
+    }
+  }
+  float4* rrow = reinterpret_cast<float4*>(w.resid + ((size_t)m * dm.C + i) * dm.dv);
+  if (fuse_resid) {
+    const VT* u = target_src<VT>(dm, v, v_next, stride, m, i, len);
+    if (u == nullptr) return;
+    const float gw = (dm.flags & FWPKM_GATE_WEIGHT) ? gt : 1.f;
+    float4 r[VPL];
+    residual<VT, VPL>(dm, acc, u, gw, r, lane);
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) {
+      int e4 = lane + 32 * c;
+      if (e4 < dv4) rrow[e4] = r[c];
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) {
+      int e4 = lane + 32 * c;
+      if (e4 < dv4) rrow[e4] = acc[c];
+    }
+  }
+}
+
+// Streaming path: resid holds vhat from the forward call; turn it into r_t in place.
+template <typename VT, int VPL>
+__global__ void __launch_bounds__(VAL_WARPS * 32)
+resid_kernel(Dims dm, Work w, const VT* __restrict__ v, const float* __restrict__ g, long long stride,
+             int len, const VT* __restrict__ v_next) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * VAL_WARPS + warp;
+  const int m = blockIdx.y;
+  if (i >= len) return;
+  const int dv4 = dm.dv >> 2;
+  const VT* u = target_src<VT>(dm, v, v_next, stride, m, i, len);
+  if (u == nullptr) return;
+  float4* rrow = reinterpret_cast<float4*>(w.resid + ((size_t)m * dm.C + i) * dm.dv);
+  float4 vh[VPL];
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) {
+    int e4 = lane + 32 * c;
+    vh[c] = e4 < dv4 ? rrow[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const float gt = g[(long long)m * stride + i];
+  const float gw = (dm.flags & FWPKM_GATE_WEIGHT) ? gt : 1.f;
+  float4 r[VPL];
+  residual<VT, VPL>(dm, vh, u, gw, r, lane);
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) {
+    int e4 = lane + 32 * c;
+    if (e4 < dv4) rrow[e4] = r[c];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Write: one warp per touched row (segment of the sorted pair list).  G_i sums
+// s'_{t,i} r_t in token order; V_i -= G_i / N_read,i.  Rows are disjoint, so there
+// are no atomics and the result does not depend on scheduling.
+// ---------------------------------------------------------------------------
+template <int VPL>
+__global__ void __launch_bounds__(VAL_WARPS * 32)
+write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = blockIdx.x * VAL_WARPS + warp;
+  const int m = blockIdx.y;
+  const int C = dm.C, k = dm.k, dv4 = dm.dv >> 2;
+  const int cslot = wt0 / C;
+  const size_t cbase = (size_t)m * w.max_chunks + cslot;
+  if (u >= w.nseg[cbase]) return;
+  const int32_t* seg_start = w.seg_start + cbase * (C * k + 1);
+  const int s0 = seg_start[u], s1 = seg_start[u + 1];
+  const int slot = w.seg_slot[cbase * (C * k) + u];
+  if (slot < 0 || (long long)slot >= dm.N) {
+    if (lane == 0) atomicExch(w.status, DEV_BAD_SLOT);
+    return;
+  }
+  const uint32_t* pair_tr = w.pair_tr + (size_t)m * w.max_chunks * C * k + (size_t)cslot * C * k;
+  float4 G[VPL];
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) G[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int p = s0; p < s1; ++p) {
+    const uint32_t tr = pair_tr[p];
+    const int t_local = (int)(tr / (uint32_t)k), r = (int)(tr - (uint32_t)t_local * k);
+    const float wt = w.w[((size_t)m * w.max_T + wt0 + t_local) * k + r];
+    const float4* rrow = reinterpret_cast<const float4*>(w.resid + ((size_t)m * C + t_local) * dm.dv);
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) {
+      int e4 = lane + 32 * c;
+      if (e4 < dv4) {
+        float4 x = rrow[e4];
+        G[c].x = fmaf(wt, x.x, G[c].x); G[c].y = fmaf(wt, x.y, G[c].y);
+        G[c].z = fmaf(wt, x.z, G[c].z); G[c].w = fmaf(wt, x.w, G[c].w);
+      }
+    }
+  }
+  const float nr = (float)(s1 - s0);
+  float4* row = reinterpret_cast<float4*>(V + ((size_t)m * dm.N + slot) * dm.dv);
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) {
+    int e4 = lane + 32 * c;
+    if (e4 < dv4) {
+      float4 x = row[e4];
+      x.x -= G[c].x / nr; x.y -= G[c].y / nr; x.z -= G[c].z / nr; x.w -= G[c].w / nr;
+      row[e4] = x;
+    }
+  }
+}
+
+// ---- launchers ----
+static int vpl_of(int dv) {
+  int v = (dv / 4 + 31) / 32;
+  return v <= 1 ? 1 : v <= 2 ? 2 : v <= 4 ? 4 : 8;
+}
+
+#define FWPKM_VPL_DISPATCH(VPLV, ...)            \
+  switch (VPLV) {                                \
+    case 1: { constexpr int VPL = 1; __VA_ARGS__; } break; \
+    case 2: { constexpr int VPL = 2; __VA_ARGS__; } break; \
+    case 4: { constexpr int VPL = 4; __VA_ARGS__; } break; \
+    default: { constexpr int VPL = 8; __VA_ARGS__; } break; \
+  }
+
+int launch_gather(const Dims& d, const Work& w, const float* V, const void* v, const float* g,
+                  long long stride, int wt0, int len, float* o, bool fuse_resid, const void* v_next,
+                  cudaStream_t s) {
+  if (len <= 0) return 0;
+  dim3 grid((len + VAL_WARPS - 1) / VAL_WARPS, d.M);
+  if (d.qv_bf16) {
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv), gather_kernel<__nv_bfloat16, VPL><<<grid, VAL_WARPS * 32, 0, s>>>(
+        d, w, V, (const __nv_bfloat16*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0,
+        (const __nv_bfloat16*)v_next));
+  } else {
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv), gather_kernel<float, VPL><<<grid, VAL_WARPS * 32, 0, s>>>(
+        d, w, V, (const float*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0, (const float*)v_next));
+  }
+  return 1;
+}
+
+int launch_resid(const Dims& d, const Work& w, const void* v, const float* g, long long stride, int len,
+                 const void* v_next, cudaStream_t s) {
+  if (len <= 0) return 0;
+  dim3 grid((len + VAL_WARPS - 1) / VAL_WARPS, d.M);
+  if (d.qv_bf16) {
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv), resid_kernel<__nv_bfloat16, VPL><<<grid, VAL_WARPS * 32, 0, s>>>(
+        d, w, (const __nv_bfloat16*)v, g, stride, len, (const __nv_bfloat16*)v_next));
+  } else {
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv), resid_kernel<float, VPL><<<grid, VAL_WARPS * 32, 0, s>>>(
+        d, w, (const float*)v, g, stride, len, (const float*)v_next));
+  }
+  return 1;
+}
+
+int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s) {
+  dim3 grid((d.C * d.k + VAL_WARPS - 1) / VAL_WARPS, d.M);
+  FWPKM_VPL_DISPATCH(vpl_of(d.dv), write_kernel<VPL><<<grid, VAL_WARPS * 32, 0, s>>>(d, w, V, wt0));
+  return 1;
+}
+
+}  // namespace fwpkm

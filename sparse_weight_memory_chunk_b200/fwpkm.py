@@ -1,0 +1,173 @@
+"""Thin ctypes binding of ``libfwpkm.so`` (declared in ``include/fwpkm.h``).
+
+Argument marshalling only: every step of the FwPKM hot path runs in the library's
+CUDA kernels.  Functions keep the C names without the ``fwpkm_`` prefix; device
+buffers are passed as torch tensors (their ``data_ptr``) and streams as
+``torch.cuda.Stream`` (default: the current stream).  A non-OK status raises
+``FwpkmError``.  If the library is missing, loading raises instead of falling back
+to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfwpkm.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_STATE = 0, -1, -2, -3, -4, -5, -6
+F32, BF16 = 0, 1
+KEY_UPDATE, TARGET_NORM, LOOKAHEAD, GATE_WEIGHT = 1, 2, 4, 8
+DEFAULT_FLAGS = TARGET_NORM | LOOKAHEAD | GATE_WEIGHT
+KIND = {"gather": 1, "write": 2, "score": 3, "cartesian": 4, "sort": 5, "address": 6, "other": 7}
+
+
+class FwpkmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int), ("d", ctypes.c_int), ("d_v", ctypes.c_int), ("k", ctypes.c_int),
+                ("chunk", ctypes.c_int), ("num_mem", ctypes.c_int), ("qv_dtype", ctypes.c_int),
+                ("eps_idw", ctypes.c_float), ("eps_norm", ctypes.c_float), ("lr_key", ctypes.c_float),
+                ("flags", ctypes.c_uint)]
+
+
+def make_config(n, d, d_v, k, chunk, num_mem, bf16, eps_idw=1e-3, eps_norm=1e-5, lr_key=1.0,
+                key_update=False, target_norm=True, lookahead=True, gate_weight=True) -> Config:
+    flags = ((KEY_UPDATE if key_update else 0) | (TARGET_NORM if target_norm else 0)
+             | (LOOKAHEAD if lookahead else 0) | (GATE_WEIGHT if gate_weight else 0))
+    return Config(n, d, d_v, k, chunk, num_mem, BF16 if bf16 else F32, eps_idw, eps_norm, lr_key, flags)
+
+
+_lib = None
+_P = ctypes.c_void_p
+
+
+def lib():
+    """Load libfwpkm.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python sparse_weight_memory_chunk_b200/build.py`")
+        L = ctypes.CDLL(LIB_PATH)
+        C = ctypes.POINTER(Config)
+        sig = {
+            "fwpkm_workspace_size": ([C, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+            "fwpkm_init_state": ([C, _P, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, ctypes.POINTER(_P)],
+                                 ctypes.c_int),
+            "fwpkm_forward_chunk": ([_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P], ctypes.c_int),
+            "fwpkm_write_chunk": ([_P, _P, _P], ctypes.c_int),
+            "fwpkm_run_sequence": ([_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P], ctypes.c_int),
+            "fwpkm_last_addressing": ([_P, ctypes.c_int, _P, _P, _P], ctypes.c_int),
+            "fwpkm_sync": ([_P, _P], ctypes.c_int),
+            "fwpkm_destroy_state": ([_P], None),
+            "fwpkm_status_string": ([ctypes.c_int], ctypes.c_char_p),
+            "fwpkm_launch_count": ([], ctypes.c_uint64),
+            "fwpkm_profile_kernel": ([_P, ctypes.c_int], ctypes.c_int),
+            "fwpkm_kernel_time": ([_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)],
+                                  ctypes.c_int),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise FwpkmError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def status_string(status: int) -> str:
+    return lib().fwpkm_status_string(status).decode()
+
+
+def launch_count() -> int:
+    return int(lib().fwpkm_launch_count())
+
+
+def workspace_size(cfg: Config, max_T: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().fwpkm_workspace_size(ctypes.byref(cfg), max_T, ctypes.byref(out)), "workspace_size")
+    return out.value
+
+
+class State:
+    """A handle from ``fwpkm_init_state``; keeps the caller's tensors alive."""
+
+    def __init__(self, cfg: Config, K1, K2, V, max_T: int, workspace=None):
+        import torch
+        self.cfg = cfg
+        self.max_T = max_T
+        nbytes = workspace_size(cfg, max_T)
+        if workspace is None:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=V.device)
+        for t in (K1, K2, V):
+            assert t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+        self.K1, self.K2, self.V, self.workspace = K1, K2, V, workspace
+        h = _P()
+        _check(lib().fwpkm_init_state(ctypes.byref(cfg), _ptr(K1), _ptr(K2), _ptr(V), max_T,
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      ctypes.byref(h)), "init_state")
+        self.handle = h
+        self._pending = None
+
+    def forward_chunk(self, q, v, g, o, c_len, seq_stride=None, idx_out=None, w_out=None, stream=None):
+        seq_stride = c_len if seq_stride is None else seq_stride
+        self._pending = (q, v, g)
+        _check(lib().fwpkm_forward_chunk(self.handle, _ptr(q), _ptr(v), _ptr(g), c_len, seq_stride, _ptr(o),
+                                         _ptr(idx_out), _ptr(w_out), _stream(stream)), "forward_chunk")
+
+    def write_chunk(self, v_next=None, stream=None):
+        _check(lib().fwpkm_write_chunk(self.handle, _ptr(v_next), _stream(stream)), "write_chunk")
+        self._pending = None
+
+    def run_sequence(self, q, v, g, o, T=None, n_iter=1, stream=None):
+        T = q.shape[1] if T is None else T
+        _check(lib().fwpkm_run_sequence(self.handle, _ptr(q), _ptr(v), _ptr(g), T, n_iter, _ptr(o),
+                                        _stream(stream)), "run_sequence")
+
+    def last_addressing(self, T, idx_out=None, w_out=None, stream=None):
+        _check(lib().fwpkm_last_addressing(self.handle, T, _ptr(idx_out), _ptr(w_out), _stream(stream)),
+               "last_addressing")
+
+    def sync(self, stream=None):
+        _check(lib().fwpkm_sync(self.handle, _stream(stream)), "sync")
+
+    def profile_kernel(self, kind):
+        kind = KIND.get(kind, kind) if isinstance(kind, str) else kind
+        _check(lib().fwpkm_profile_kernel(self.handle, int(kind)), "profile_kernel")
+
+    def kernel_time(self):
+        ms = ctypes.c_double(0.0)
+        n = ctypes.c_int(0)
+        _check(lib().fwpkm_kernel_time(self.handle, ctypes.byref(ms), ctypes.byref(n)), "kernel_time")
+        return ms.value, n.value
+
+    def destroy(self):
+        if getattr(self, "handle", None):
+            lib().fwpkm_destroy_state(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass

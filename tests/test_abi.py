@@ -1,0 +1,66 @@
+"""The C ABI library builds for sm_100a, loads without a GPU and exports every entry
+point that include/fwpkm.h declares.  Only host-side calls are made (no kernels)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_weight_memory_chunk_b200 import build, fwpkm
+    build.build()
+    return fwpkm
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(fwpkm_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    so = ctypes.CDLL(lib.LIB_PATH)
+    missing = [n for n in names if not hasattr(so, n)]
+    assert not missing, missing
+
+
+def test_library_is_built_for_sm100a(lib):
+    data = open(lib.LIB_PATH, "rb").read()
+    assert b"sm_100a" in data
+
+
+def test_status_strings(lib):
+    assert lib.status_string(0) == "ok"
+    assert lib.status_string(-3) == "workspace too small"
+    assert lib.status_string(-5) == "device wait timed out"
+
+
+def test_workspace_size_and_validation(lib):
+    cfg = lib.make_config(n=1024, d=256, d_v=256, k=32, chunk=256, num_mem=8, bf16=True, key_update=True)
+    ws = lib.workspace_size(cfg, 4096)
+    # idx + w + per-half survivors + pair lists dominate: O(M T k) + the chunk distance rows
+    assert 8 * 4096 * 32 * 4 * 6 < ws < 128 << 20
+    bad = [dict(k=33), dict(k=0), dict(n=16, k=32), dict(d=7), dict(d_v=6), dict(chunk=2048),
+           dict(num_mem=0), dict(n=8192)]
+    for over in bad:
+        c = dict(n=1024, d=256, d_v=256, k=32, chunk=256, num_mem=8, bf16=True)
+        c.update(over)
+        with pytest.raises(lib.FwpkmError) as e:
+            lib.workspace_size(lib.make_config(**c), 4096)
+        assert e.value.status in (lib.ERR_INVALID_ARG, lib.ERR_UNSUPPORTED)
+    with pytest.raises(lib.FwpkmError):
+        lib.workspace_size(cfg, 0)
+
+
+def test_launch_counter_starts_at_zero(lib):
+    assert lib.launch_count() == 0

@@ -1,0 +1,163 @@
+"""GPU (libfwpkm.so through the C ABI) against the CPU oracle on the same seeded inputs.
+
+Element-by-element, after every chunk, at sizes the oracle finishes in seconds: the
+five workload shapes (n, d, d_v, k, C, dtype) with reduced M and T, ragged tails,
+key update on and off.  The production entry point (fwpkm_run_sequence) is then
+checked bit-for-bit against the chunk-by-chunk entry points on the same inputs.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+from sparse_weight_memory_chunk_b200 import fwpkm  # noqa: E402
+from sparse_weight_memory_chunk_b200.inputs import Workload, gen_keys, gen_qvg, gen_values  # noqa: E402
+
+import oracle  # noqa: E402
+from parity import as_f64, assert_close, oracle_chunk_against_gpu, to_device  # noqa: E402
+
+# name: (n, d, d_v, k, C, M, T, qv, key_update, lr_key, v_init)
+CASES = {
+    "tiny": (64, 64, 64, 8, 64, 1, 256, "f32", False, 1.0, "zero"),
+    "tiny_key_ragged": (64, 64, 64, 8, 64, 2, 250, "f32", True, 100.0, "normal002"),
+    "mid": (256, 128, 128, 16, 128, 3, 300, "bf16", False, 1.0, "normal002"),
+    "mid_key": (256, 128, 128, 16, 128, 2, 300, "bf16", True, 100.0, "normal002"),
+    "paper": (1024, 256, 256, 32, 256, 2, 600, "bf16", True, 1.0, "normal002"),
+    "needle_chunk": (1024, 256, 256, 32, 512, 1, 1100, "bf16", False, 1.0, "normal002"),
+    "layer_shape": (512, 256, 256, 32, 256, 2, 520, "f32", True, 1.0, "normal002"),
+}
+
+
+def make_case(name, seed=10, **flags):
+    n, d, dv, k, C, M, T, qv, ku, lr, vinit = CASES[name]
+    w = Workload(name, n, d, dv, k, T, C, M, 1, qv, ku, seed, "sigmoid", vinit)
+    q, v, g = gen_qvg(w)
+    K1, K2 = gen_keys(w)
+    V = np.stack([gen_values(w, m) for m in range(M)])
+    gcfg = fwpkm.make_config(n, d, dv, k, C, M, qv == "bf16", lr_key=lr, key_update=ku, **flags)
+    ocfg = oracle.make_cfg(n, d, dv, k, C, lr_key=lr, key_update=ku, **flags)
+    return w, (q, v, g, K1, K2, V), gcfg, ocfg
+
+
+def device_state(w, data, gcfg, max_T):
+    q, v, g, K1, K2, V = data
+    dev = dict(q=to_device(q, w.qv, torch), v=to_device(v, w.qv, torch), g=torch.from_numpy(g).cuda(),
+               K1=torch.from_numpy(K1).cuda(), K2=torch.from_numpy(K2).cuda(), V=torch.from_numpy(V).cuda())
+    st = fwpkm.State(gcfg, dev["K1"], dev["K2"], dev["V"], max_T)
+    return st, dev
+
+
+def streaming_vs_oracle(name, **flags):
+    w, data, gcfg, ocfg = make_case(name, **flags)
+    q, v, g, K1, K2, V = data
+    M, T, C, k, dv, N = w.M, w.T, w.C, w.k, w.d_v, w.N
+    st, dev = device_state(w, data, gcfg, C)
+    o_d = torch.zeros(M, T, dv, device="cuda")
+    qf, vf = as_f64(q, w.qv), as_f64(v, w.qv)
+    V_orc = V.copy()
+    small = N * dv <= (1 << 22)
+    rng = np.random.default_rng(0)
+    ties = 0
+    for t0 in range(0, T, C):
+        ln = min(C, T - t0)
+        K1pre, K2pre = dev["K1"].cpu().numpy().copy(), dev["K2"].cpu().numpy().copy()
+        idx_d = torch.empty(M, ln, k, dtype=torch.int32, device="cuda")
+        w_d = torch.empty(M, ln, k, device="cuda")
+        st.forward_chunk(dev["q"][:, t0:], dev["v"][:, t0:], dev["g"][:, t0:], o_d[:, t0:], ln, seq_stride=T,
+                         idx_out=idx_d, w_out=w_d)
+        has_next = t0 + ln < T
+        st.write_chunk(dev["v"][:, t0 + ln] if has_next else None)
+        st.sync()
+        idx_g, w_g = idx_d.cpu().numpy(), w_d.cpu().numpy()
+        o_g = o_d[:, t0:t0 + ln].cpu().numpy()
+        for m in range(M):
+            k1, k2 = K1pre[m].copy(), K2pre[m].copy()
+            vn = vf[m, t0 + ln] if has_next else None
+            o_o, I_o, w_o, nt = oracle_chunk_against_gpu(ocfg, qf[m, t0:t0 + ln], vf[m, t0:t0 + ln],
+                                                         g[m, t0:t0 + ln].astype(np.float64), vn, k1, k2,
+                                                         V_orc[m], idx_g[m])
+            ties += nt
+            assert_close(o_g[m], o_o, f"{name} chunk@{t0} mem {m}: o")
+            assert_close(w_g[m], w_o, f"{name} chunk@{t0} mem {m}: w", atol=1e-6)
+            if w.key_update:
+                K1g, K2g = dev["K1"][m].cpu().numpy(), dev["K2"][m].cpu().numpy()
+                assert_close(K1g, k1, f"{name} chunk@{t0} mem {m}: K1")
+                assert_close(K2g, k2, f"{name} chunk@{t0} mem {m}: K2")
+                # the step itself (tiny next to K) must agree, not just the keys
+                for Kg, Ko, Kp in ((K1g, k1, K1pre[m]), (K2g, k2, K2pre[m])):
+                    dg = Kg.astype(np.float64) - Kp
+                    do = Ko.astype(np.float64) - Kp
+                    ulp = np.spacing(np.abs(Ko)).astype(np.float64)
+                    assert np.all(np.abs(dg - do) <= 2 * ulp + 2e-3 * np.abs(do) + 1e-9), f"{name}: dK"
+            if small:
+                rows = np.arange(N)
+            else:
+                touched = np.unique(idx_g[m].reshape(-1))
+                rows = np.unique(np.concatenate([touched, rng.integers(0, N, 2048)]))
+            Vg = dev["V"][m][torch.from_numpy(rows).cuda()].cpu().numpy()
+            assert_close(Vg, V_orc[m][rows], f"{name} chunk@{t0} mem {m}: V")
+    return dict(o=o_d.cpu(), V=dev["V"].cpu(), K1=dev["K1"].cpu(), K2=dev["K2"].cpu(), ties=ties,
+                w=w, data=data, gcfg=gcfg)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_streaming_matches_oracle_every_chunk(name):
+    res = streaming_vs_oracle(name)
+    print(f"{name}: near-ties {res['ties']}")
+    # the production schedule computes the same bits
+    w, data, gcfg = res["w"], res["data"], res["gcfg"]
+    st, dev = device_state(w, data, gcfg, w.T)
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    st.run_sequence(dev["q"], dev["v"], dev["g"], o)
+    st.sync()
+    assert torch.equal(o.cpu(), res["o"]), "run_sequence o differs from chunk-by-chunk"
+    assert torch.equal(dev["V"].cpu(), res["V"]), "run_sequence V differs"
+    assert torch.equal(dev["K1"].cpu(), res["K1"]) and torch.equal(dev["K2"].cpu(), res["K2"])
+
+
+@pytest.mark.parametrize("flags", [dict(lookahead=False), dict(target_norm=False), dict(gate_weight=False)])
+def test_flag_variants(flags):
+    streaming_vs_oracle("tiny_key_ragged", **flags)
+
+
+@pytest.mark.parametrize("name", ["mid", "mid_key"])
+def test_passes_compose_and_determinism(name):
+    w, data, gcfg, _ = make_case(name)
+    outs = []
+    for _ in range(2):
+        st, dev = device_state(w, data, gcfg, w.T)
+        o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+        st.run_sequence(dev["q"], dev["v"], dev["g"], o, n_iter=2)
+        st.sync()
+        outs.append((o.cpu(), dev["V"].cpu(), dev["K1"].cpu()))
+    assert all(torch.equal(a, b) for a, b in zip(*outs)), "two identical runs differ"
+    st, dev = device_state(w, data, gcfg, w.T)
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    st.run_sequence(dev["q"], dev["v"], dev["g"], o, n_iter=1)
+    st.run_sequence(dev["q"], dev["v"], dev["g"], o, n_iter=1)
+    st.sync()
+    assert torch.equal(o.cpu(), outs[0][0]) and torch.equal(dev["V"].cpu(), outs[0][1])
+    assert torch.equal(dev["K1"].cpu(), outs[0][2])
+
+
+def test_edge_cases():
+    w, data, gcfg, ocfg = make_case("tiny_key_ragged")
+    st, dev = device_state(w, data, gcfg, w.T)
+    V0, K10 = dev["V"].clone(), dev["K1"].clone()
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    st.run_sequence(dev["q"], dev["v"], dev["g"], o, T=0)  # no-op
+    st.sync()
+    assert torch.equal(dev["V"], V0)
+    # one token: nothing to write (no lookahead target) but the keys still take their step
+    st.run_sequence(dev["q"][:, :1].contiguous(), dev["v"][:, :1].contiguous(), dev["g"][:, :1].contiguous(),
+                    o[:, :1].contiguous(), T=1)
+    st.sync()
+    assert torch.equal(dev["V"], V0)
+    assert not torch.equal(dev["K1"], K10)
+    with pytest.raises(fwpkm.FwpkmError) as e:
+        st.write_chunk(None)
+    assert e.value.status == fwpkm.ERR_STATE
+    with pytest.raises(fwpkm.FwpkmError) as e:
+        st.run_sequence(dev["q"], dev["v"], dev["g"], o, T=w.T + 1)
+    assert e.value.status == fwpkm.ERR_INVALID_ARG
