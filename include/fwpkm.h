@@ -137,6 +137,23 @@ fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream
 fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, const float* g,
                                 int T, int n_iter, float* o, void* stream);
 
+/* One whole chunk step -- the read of fwpkm_forward_chunk followed by the write (and
+ * key step) of fwpkm_write_chunk -- that allocates nothing and needs no workspace.
+ * The paper has no counterpart: this exists for callers that cannot allocate device
+ * memory (host callbacks, loops under a no-allocation rule, plugins whose host owns
+ * the allocator, code that must not change the device memory map).  Arguments mean
+ * what they mean in fwpkm_forward_chunk / fwpkm_write_chunk (K1, K2, V are the
+ * caller's state, updated in place; v_next NULL = the chunk ends the sequence).
+ * Scratch is a fixed 16 MiB array inside the library that every GPU loading the
+ * library keeps until exit; shapes whose fwpkm_workspace_size(cfg, cfg->chunk)
+ * exceeds it are rejected with FWPKM_ERR_UNSUPPORTED.  The first call on a device
+ * looks up that array's device address (make it before any stream capture).  All
+ * calls share the array: calls that overlap on the GPU race and must be serialised
+ * by the caller.  Device-side errors are not reported by this entry point. */
+fwpkm_status fwpkm_chunk_step_noalloc(const fwpkm_config* cfg, float* K1, float* K2, float* V,
+                                      const void* q, const void* v, const float* g, const void* v_next,
+                                      int c_len, int seq_stride, float* o, void* stream);
+
 /* Copy the slot indices and softmax weights that the most recent call computed for
  * tokens [0, T) of every memory (final pass of fwpkm_run_sequence, or the chunk of
  * fwpkm_forward_chunk with T <= c_len) into idx_out [M][T][k] int32 and

@@ -63,6 +63,8 @@ def lib():
             "fwpkm_write_chunk": ([_P, _P, _P], ctypes.c_int),
             "fwpkm_run_sequence": ([_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P], ctypes.c_int),
             "fwpkm_last_addressing": ([_P, ctypes.c_int, _P, _P, _P], ctypes.c_int),
+            "fwpkm_chunk_step_noalloc": ([C, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P],
+                                         ctypes.c_int),
             "fwpkm_sync": ([_P, _P], ctypes.c_int),
             "fwpkm_destroy_state": ([_P], None),
             "fwpkm_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -107,6 +109,15 @@ def workspace_size(cfg: Config, max_T: int) -> int:
     out = ctypes.c_size_t(0)
     _check(lib().fwpkm_workspace_size(ctypes.byref(cfg), max_T, ctypes.byref(out)), "workspace_size")
     return out.value
+
+
+def chunk_step_noalloc(cfg: Config, K1, K2, V, q, v, g, o, c_len, seq_stride=None, v_next=None,
+                       stream=None):
+    """One chunk step (read + write + key step) with no workspace and no allocation."""
+    seq_stride = c_len if seq_stride is None else seq_stride
+    _check(lib().fwpkm_chunk_step_noalloc(ctypes.byref(cfg), _ptr(K1), _ptr(K2), _ptr(V), _ptr(q), _ptr(v),
+                                          _ptr(g), _ptr(v_next), c_len, seq_stride, _ptr(o), _stream(stream)),
+           "chunk_step_noalloc")
 
 
 class State:
