@@ -35,6 +35,7 @@ struct fwpkm_state {
   int prof_kind;
   std::vector<cudaEvent_t> ev;
   int ev_used;
+  int host_error;  // a launch could not be set up (e.g. tensor map encoding failed)
 };
 
 namespace {
@@ -92,12 +93,29 @@ void run(fwpkm_state* st, int kind, cudaStream_t s, F&& f) {
     cudaEventRecord(st->ev[st->ev_used + 1], s);
     st->ev_used += 2;
   }
-  g_launches += (uint64_t)nl;
+  if (nl < 0) st->host_error = 1;
+  else g_launches += (uint64_t)nl;
 }
 
 }  // namespace
 
 namespace fwpkm {
+
+// The tensor-core path needs bf16 queries (exact tcgen05 operands) and half widths that
+// are whole 64-element swizzle atoms no wider than one 128-column accumulator tile.
+bool use_tensor_cores(const Dims& d) {
+  return d.qv_bf16 && (d.h == 64 || d.h == 128) && d.n % 8 == 0 && d.n >= 64;
+}
+
+// Tokens addressed per batch when the keys are frozen: the distance rows of a batch are
+// kept (up to ~64 MiB) so that the per-half top-k can read them back.
+int addressing_window(const Dims& d, int max_T) {
+  const size_t per_tok = (size_t)d.M * 2 * d.n * 4;
+  size_t wtok = ((size_t)64 << 20) / per_tok / 128 * 128;
+  if (wtok < 128) wtok = 128;
+  const size_t need = ((size_t)max_T + 127) / 128 * 128;
+  return (int)(wtok < need ? wtok : need);
+}
 
 size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
   const size_t M = d.M, k = d.k, C = d.C, n = d.n, dv = d.dv;
@@ -122,13 +140,31 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
   x.seg_slot = (int32_t*)take(4 * M * nch * C * k);
   x.nseg = (int32_t*)take(4 * M * nch);
   x.resid = (float*)take(4 * M * C * dv);
-  if (d.flags & FWPKM_KEY_UPDATE) {
-    x.Dfull = (float*)take(4 * M * 2 * C * n);
+  const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
+  x.tc = use_tensor_cores(d) ? 1 : 0;
+  x.drows = ku ? (int)C : (x.tc ? addressing_window(d, max_T) : 0);
+  x.Dfull = x.drows ? (float*)take(4 * M * 2 * (size_t)x.drows * n) : nullptr;
+  if (ku) {
     x.Z = (float*)take(4 * M * 2 * C);
     x.lp = (float*)take(4 * M * 2 * n);
     x.Lt = (float*)take(4 * M * 2 * C);
   } else {
-    x.Dfull = nullptr; x.Z = nullptr; x.lp = nullptr; x.Lt = nullptr;
+    x.Z = nullptr; x.lp = nullptr; x.Lt = nullptr;
+  }
+  x.Kpc = nullptr; x.kn = nullptr; x.qn = nullptr; x.zpart = nullptr; x.ppart = nullptr;
+  x.Wt = nullptr; x.Qt = nullptr; x.wsum_part = nullptr;
+  if (x.tc) {
+    const size_t P = 2 * M, h = d.h, cpad = (C + 63) / 64 * 64, nt = (n + 127) / 128;
+    x.Kpc = (__nv_bfloat16*)take(2 * 3 * P * n * h);
+    x.kn = (float*)take(4 * P * n);
+    x.qn = (float*)take(4 * P * T);
+    if (ku) {
+      x.zpart = (float*)take(4 * P * C * nt);
+      x.ppart = (float*)take(4 * P * 8 * n);
+      x.Wt = (__nv_bfloat16*)take(2 * 3 * P * n * cpad);
+      x.Qt = (__nv_bfloat16*)take(2 * P * h * cpad);
+      x.wsum_part = (float*)take(4 * P * (cpad / 64) * n);
+    }
   }
   if (w) *w = x;
   return off;
@@ -209,13 +245,22 @@ fwpkm_status fwpkm_forward_chunk(fwpkm_state* st, const void* q, const void* v, 
   if (ps != FWPKM_OK) return ps;
   cudaStream_t s = (cudaStream_t)stream;
   const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
-  run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, q, seq_stride, 0, c_len, ku, s); });
+  st->host_error = 0;
+  if (st->wk.tc) {
+    run(st, KK_OTHER, s, [&] { return launch_qnorm(d, st->wk, q, seq_stride, 0, c_len, s); });
+    run(st, KK_OTHER, s, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, s); });
+    run(st, KK_SCORE, s, [&] { return launch_tc_score(d, st->wk, q, seq_stride, c_len, 0, 0, c_len, ku, s); });
+    run(st, KK_SCORE, s, [&] { return launch_topk_rows(d, st->wk, 0, c_len, s); });
+  } else {
+    run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, q, seq_stride, 0, c_len, ku, s); });
+  }
   run(st, KK_CART, s, [&] { return launch_cartesian(d, st->wk, 0, c_len, idx_out, w_out, s); });
   run(st, KK_GATHER, s, [&] {
     return launch_gather(d, st->wk, st->V, v, g, seq_stride, 0, c_len, o, false, nullptr, s);
   });
   st->pending = 1;
   st->q = q; st->v = v; st->g = g; st->len = c_len; st->stride = seq_stride;
+  if (st->host_error) return FWPKM_ERR_CUDA;
   return last_cuda();
 }
 
@@ -229,9 +274,14 @@ fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream
   run(st, KK_OTHER, s, [&] { return launch_resid(d, st->wk, st->v, st->g, st->stride, st->len, v_next, s); });
   run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, st->wk, 0, st->len, last_has_target, s); });
   run(st, KK_WRITE, s, [&] { return launch_write(d, st->wk, st->V, 0, s); });
+  st->host_error = 0;
   if (d.flags & FWPKM_KEY_UPDATE)
-    run(st, KK_ADDR, s, [&] { return launch_address(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, s); });
+    run(st, KK_ADDR, s, [&] {
+      return st->wk.tc ? launch_tc_address(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, s)
+                       : launch_address(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, s);
+    });
   st->pending = 0;
+  if (st->host_error) return FWPKM_ERR_CUDA;
   return last_cuda();
 }
 
@@ -262,9 +312,23 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
     run(st, KK_WRITE, s, [&] { return launch_write(d, st->wk, st->V, t0, s); });
   };
 
+  const bool tc = st->wk.tc != 0;
+  st->host_error = 0;
+  if (tc) {
+    run(st, KK_OTHER, s, [&] { return launch_qnorm(d, st->wk, q, T, 0, T, s); });
+    run(st, KK_OTHER, s, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, s); });
+  }
   if (!ku) {
     // keys are frozen: address every token once, for all passes
-    run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, q, T, 0, T, false, s); });
+    if (tc) {
+      for (int w0 = 0; w0 < T; w0 += st->wk.drows) {
+        const int wl = T - w0 < st->wk.drows ? T - w0 : st->wk.drows;
+        run(st, KK_SCORE, s, [&] { return launch_tc_score(d, st->wk, q, T, T, w0, w0, wl, false, s); });
+        run(st, KK_SCORE, s, [&] { return launch_topk_rows(d, st->wk, w0, wl, s); });
+      }
+    } else {
+      run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, q, T, 0, T, false, s); });
+    }
     run(st, KK_CART, s, [&] { return launch_cartesian(d, st->wk, 0, T, nullptr, nullptr, s); });
     run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, st->wk, 0, T, !la, s); });
     for (int pass = 0; pass < n_iter; ++pass)
@@ -274,14 +338,23 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
       for (int c = 0; c < nch; ++c) {
         const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
         const void* qc = offs(q, (long long)t0 * d.d, es);
-        run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, qc, T, t0, len, true, s); });
+        if (tc) {
+          run(st, KK_SCORE, s, [&] { return launch_tc_score(d, st->wk, q, T, T, t0, t0, len, true, s); });
+          run(st, KK_SCORE, s, [&] { return launch_topk_rows(d, st->wk, t0, len, s); });
+        } else {
+          run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, qc, T, t0, len, true, s); });
+        }
         run(st, KK_CART, s, [&] { return launch_cartesian(d, st->wk, t0, len, nullptr, nullptr, s); });
         run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, st->wk, t0, len, !la || (t0 + len < T), s); });
         value_chunk(c);
-        run(st, KK_ADDR, s, [&] { return launch_address(d, st->wk, st->K1, st->K2, qc, T, len, s); });
+        run(st, KK_ADDR, s, [&] {
+          return tc ? launch_tc_address(d, st->wk, st->K1, st->K2, qc, T, len, s)
+                    : launch_address(d, st->wk, st->K1, st->K2, qc, T, len, s);
+        });
       }
     }
   }
+  if (st->host_error) return FWPKM_ERR_CUDA;
   return last_cuda();
 }
 

@@ -1,6 +1,7 @@
 // fwpkm_internal.cuh -- shared declarations of the B200 FwPKM library (not part of the ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -42,7 +43,44 @@ struct Work {
   float* lp;         // [M][2][n]          key update: log pbar
   float* Lt;         // [M][2][C]          key update: sum_a P log pbar
   int* status;       // device status word
+  // tensor-core path (bf16 q, d/2 in {64, 128})
+  int tc;            // 1 if the tensor-core path is used
+  int drows;         // rows of Dfull per problem (C with the key step, else the addressing window)
+  __nv_bfloat16* Kpc;// [3][M*2][n][h]     bf16 pieces hi/mid/lo of the keys
+  float* kn;         // [M*2][n]           squared key norms
+  float* qn;         // [M*2][max_T]       squared half-query norms
+  float* zpart;      // [M*2][C][n/128]    per-tile partial sums of 1/(eps + D)
+  float* ppart;      // [M*2][8][n]        partial column sums for pbar
+  __nv_bfloat16* Wt; // [3][M*2][n][Cpad]  key-step weights, sub-key major, bf16 pieces
+  __nv_bfloat16* Qt; // [M*2][h][Cpad]     chunk half-queries, feature major
+  float* wsum_part;  // [M*2][Cpad/64][n]  per-token-tile sums of W
 };
+
+enum : int { TC_EPI_DIST = 0, TC_EPI_KEYSTEP = 1 };
+
+// One batched tensor-core contraction (see tc_gemm.cu).  Problem p (blockIdx.z) owns
+// A tiles at (x = (p % a_div) * a_xoff + 64 kb, y = a_y0 + 128 mt, z = p / a_div + pa * a_zpiece)
+// and B tiles at (x = 64 kb, y = 128 nt, z = p + pb * b_zpiece).
+struct TcGemm {
+  int P, k_blocks, n_tiles, tiles_per_cta;
+  int a_pieces, b_pieces;
+  int a_div, a_xoff, a_y0, a_zpiece, b_zpiece;
+  int m_valid, n_valid;
+  int epi;
+  // TC_EPI_DIST
+  float* out; long long out_pstride; int out_ld;
+  const float* rowv; long long rowv_pstride; int rowv_off;
+  const float* colv; long long colv_pstride;
+  float* zpart; long long zpart_pstride; float eps;
+  // TC_EPI_KEYSTEP
+  float* K1; float* K2; __nv_bfloat16* Kpc; float* kn;
+  const float* wsum_part; int wsum_tiles; float lr;
+  int* status;
+};
+
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z, uint64_t pitch_y,
+                       uint64_t pitch_z);
+int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g, int m_tiles, cudaStream_t s);
 
 size_t workspace_bytes(const Dims& d, int max_T, Work* carve, char* base);
 
@@ -78,6 +116,21 @@ int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s
 // Entropy key step for the chunk whose distances are in Dfull/Z (`len` tokens).
 int launch_address(const Dims& d, const Work& w, float* K1, float* K2, const void* q,
                    long long q_stride, int len, cudaStream_t s);
+
+// ---- tensor-core path ----
+// Squared norms of both halves of q for `len` tokens (workspace tokens wt0..).
+int launch_qnorm(const Dims& d, const Work& w, const void* q, long long q_stride, int wt0, int len, cudaStream_t s);
+// bf16 pieces + squared norms of the current keys.
+int launch_keyprep(const Dims& d, const Work& w, const float* K1, const float* K2, cudaStream_t s);
+// Distances of `len` tokens (workspace tokens wt0.., user q pointer at the range start,
+// q extent T_ext tokens per memory) into Dfull rows 0..len-1, plus zpart if key_update.
+int launch_tc_score(const Dims& d, const Work& w, const void* q_base, long long q_stride, int q_extent, int q_row0,
+                    int wt0, int len, bool key_update, cudaStream_t s);
+// Per-half top-k from Dfull rows 0..len-1 into A/Dsv at workspace tokens wt0..
+int launch_topk_rows(const Dims& d, const Work& w, int wt0, int len, cudaStream_t s);
+// Entropy key step from Dfull/zpart (tensor-core path).
+int launch_tc_address(const Dims& d, const Work& w, float* K1, float* K2, const void* q, long long q_stride, int len,
+                      cudaStream_t s);
 
 // ---- small device helpers ----
 __device__ __forceinline__ float load_qv(const float* p, long long i) { return p[i]; }

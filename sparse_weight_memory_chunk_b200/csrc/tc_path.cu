@@ -1,0 +1,303 @@
+// tc_path.cu -- kernels around the tensor-core contractions (bf16 queries, d/2 in {64, 128}).
+//
+// Scoring (Fast-weight Product Key Memory (paperlayer summary) §2.2, §A.2): the GEMM in
+// tc_gemm.cu writes the squared distances of a chunk's tokens to every sub-key; the
+// per-half top-k is taken here from those rows.
+// Entropy key step ((rainbus summary) method step 5; (paperlayer summary) §3.4): with
+// w = 1/(eps + D), Z_t = sum_a w, P = w / Z_t, pbar = mean_t P, lp = log pbar,
+// L_t = sum_a P lp, W[t][b] = (1/len) P[t][b] (lp[b] - L_t) w[t][b]; the key-step GEMM
+// then forms sum_t W[t][b] q_t and updates the keys in its epilogue.
+#include "fwpkm_internal.cuh"
+#include "sm100.cuh"
+
+namespace fwpkm {
+
+constexpr int TP_THREADS = 256;
+constexpr int PBAR_SLICES = 8;
+
+__device__ __forceinline__ void split3_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& mid, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(x);
+  float r = x - __bfloat162float(hi);
+  mid = __float2bfloat16_rn(r);
+  lo = __float2bfloat16_rn(r - __bfloat162float(mid));
+}
+
+// ||q_half||^2 per (memory, half, token): one warp per token, both halves.
+__global__ void __launch_bounds__(TP_THREADS)
+qnorm_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long q_stride, int wt0, int len) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (TP_THREADS / 32) + warp;
+  const int m = blockIdx.y;
+  if (i >= len) return;
+  const __nv_bfloat16* row = q + ((long long)m * q_stride + i) * dm.d;
+  for (int j = 0; j < 2; ++j) {
+    float s = 0.f;
+    for (int e = lane; e < dm.h; e += 32) {
+      float x = __bfloat162float(row[j * dm.h + e]);
+      s += x * x;
+    }
+    s = warp_sum(s);
+    if (lane == 0) w.qn[((size_t)m * 2 + j) * w.max_T + wt0 + i] = s;
+  }
+}
+
+// bf16 pieces and squared norm of every key: one thread per (problem, sub-key), features
+// in order (the key-step GEMM epilogue uses the same order, so both give the same bits).
+__global__ void __launch_bounds__(TP_THREADS)
+keyprep_kernel(Dims dm, Work w, const float* __restrict__ K1, const float* __restrict__ K2) {
+  const int P = dm.M * 2;
+  const long long idx = (long long)blockIdx.x * TP_THREADS + threadIdx.x;
+  if (idx >= (long long)P * dm.n) return;
+  const int p = (int)(idx / dm.n), b = (int)(idx - (long long)p * dm.n);
+  const int m = p >> 1, j = p & 1, h = dm.h;
+  const float* K = (j == 0 ? K1 : K2) + ((size_t)m * dm.n + b) * h;
+  const size_t pstride = (size_t)P * dm.n * h;
+  __nv_bfloat16* pc = w.Kpc + ((size_t)p * dm.n + b) * h;
+  float ss = 0.f;
+  for (int e = 0; e < h; e += 8) {
+    float4 k0 = *reinterpret_cast<const float4*>(K + e);
+    float4 k1 = *reinterpret_cast<const float4*>(K + e + 4);
+    float kin[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+    __align__(16) __nv_bfloat16 hi[8], mid[8], lo[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      ss += kin[u] * kin[u];
+      split3_bf16(kin[u], hi[u], mid[u], lo[u]);
+    }
+    *reinterpret_cast<uint4*>(pc + e) = *reinterpret_cast<uint4*>(hi);
+    *reinterpret_cast<uint4*>(pc + pstride + e) = *reinterpret_cast<uint4*>(mid);
+    *reinterpret_cast<uint4*>(pc + 2 * pstride + e) = *reinterpret_cast<uint4*>(lo);
+  }
+  w.kn[(size_t)p * dm.n + b] = ss;
+}
+
+// Per-half top-k from distance rows: one warp per (problem, token); the k smallest
+// (distance, index) keys, each round the winning lane advances past the last winner.
+__global__ void __launch_bounds__(TP_THREADS)
+topk_rows_kernel(Dims dm, Work w, int wt0, int len) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (TP_THREADS / 32) + warp;
+  const int p = blockIdx.y;
+  if (i >= len) return;
+  const int n = dm.n, k = dm.k;
+  const float* row = w.Dfull + ((size_t)p * w.drows + i) * n;
+  unsigned long long best = ~0ull;
+  for (int a = lane; a < n; a += 32) {
+    unsigned long long key = ((unsigned long long)orderable(row[a]) << 32) | (unsigned)a;
+    best = key < best ? key : best;
+  }
+  const size_t obase = ((size_t)p * w.max_T + wt0 + i) * k;
+  for (int r = 0; r < k; ++r) {
+    const unsigned long long win = warp_min_u64(best);
+    const int a = (int)(win & 0xffffffffu);
+    if (lane == 0) {
+      w.A[obase + r] = a;
+      w.Dsv[obase + r] = row[a];
+    }
+    if ((a & 31) == lane) {
+      best = ~0ull;
+      for (int b = lane; b < n; b += 32) {
+        unsigned long long key = ((unsigned long long)orderable(row[b]) << 32) | (unsigned)b;
+        if (key > win && key < best) best = key;
+      }
+    }
+  }
+}
+
+// Partial column sums sum_t w[t][a] / Z_t over one token slice; also Z_t itself.
+__global__ void __launch_bounds__(TP_THREADS)
+tc_pbar_kernel(Dims dm, Work w, int len) {
+  __shared__ float s_invz[1024 / PBAR_SLICES + 1];
+  const int p = blockIdx.y, sl = blockIdx.z;
+  const int t0 = (sl * len) / PBAR_SLICES, t1 = ((sl + 1) * len) / PBAR_SLICES;
+  const int nt = (dm.n + 127) / 128;
+  for (int t = t0 + threadIdx.x; t < t1; t += TP_THREADS) {
+    const float* zp = w.zpart + ((size_t)p * dm.C + t) * nt;
+    float z = 0.f;
+    for (int u = 0; u < nt; ++u) z += zp[u];
+    s_invz[t - t0] = 1.f / z;
+    if (blockIdx.x == 0) w.Z[(size_t)p * dm.C + t] = z;
+  }
+  __syncthreads();
+  const int a = blockIdx.x * TP_THREADS + threadIdx.x;
+  if (a >= dm.n) return;
+  const float* D = w.Dfull + (size_t)p * w.drows * dm.n;
+  float s = 0.f;
+  for (int t = t0; t < t1; ++t) s += (1.f / (dm.eps_idw + D[(size_t)t * dm.n + a])) * s_invz[t - t0];
+  w.ppart[((size_t)p * PBAR_SLICES + sl) * dm.n + a] = s;
+}
+
+__global__ void __launch_bounds__(TP_THREADS)
+tc_lp_kernel(Dims dm, Work w, int len) {
+  const long long idx = (long long)blockIdx.x * TP_THREADS + threadIdx.x;
+  if (idx >= (long long)dm.M * 2 * dm.n) return;
+  const int p = (int)(idx / dm.n), a = (int)(idx - (long long)p * dm.n);
+  float s = 0.f;
+  for (int sl = 0; sl < PBAR_SLICES; ++sl) s += w.ppart[((size_t)p * PBAR_SLICES + sl) * dm.n + a];
+  w.lp[idx] = logf(s / (float)len);
+}
+
+// L_t = sum_a P[t][a] log pbar[a]: one warp per (problem, token).
+__global__ void __launch_bounds__(TP_THREADS)
+tc_rowL_kernel(Dims dm, Work w, int len) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (TP_THREADS / 32) + warp;
+  const int p = blockIdx.y;
+  if (t >= len) return;
+  const float* D = w.Dfull + ((size_t)p * w.drows + t) * dm.n;
+  const float* lp = w.lp + (size_t)p * dm.n;
+  float s = 0.f;
+  for (int a = lane; a < dm.n; a += 32) s += lp[a] / (dm.eps_idw + D[a]);
+  s = warp_sum(s);
+  if (lane == 0) w.Lt[(size_t)p * dm.C + t] = s / w.Z[(size_t)p * dm.C + t];
+}
+
+// W for a 64-token x 64-sub-key tile, written sub-key major as three bf16 pieces (the
+// A operand of the key-step GEMM), plus the tile's per-sub-key sum of W.  CTAs of the
+// first sub-key tile also write their tokens' half-queries feature major (operand B).
+__global__ void __launch_bounds__(TP_THREADS)
+tc_wbuild_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long q_stride, int len, int cpad) {
+  __shared__ float s_W[64][65];
+  __shared__ float s_invz[64], s_L[64], s_lp[64];
+  __shared__ __nv_bfloat16 s_q[64][136];
+  const int p = blockIdx.z, m = p >> 1, j = p & 1;
+  const int b0 = blockIdx.x * 64, t0 = blockIdx.y * 64;
+  const int n = dm.n, h = dm.h, P = dm.M * 2;
+  const int tid = threadIdx.x;
+  if (tid < 64) {
+    const int t = t0 + tid;
+    s_invz[tid] = t < len ? 1.f / w.Z[(size_t)p * dm.C + t] : 0.f;
+    s_L[tid] = t < len ? w.Lt[(size_t)p * dm.C + t] : 0.f;
+  } else if (tid < 128) {
+    const int b = b0 + tid - 64;
+    s_lp[tid - 64] = b < n ? w.lp[(size_t)p * n + b] : 0.f;
+  }
+  __syncthreads();
+  const float inv_len = 1.f / (float)len;
+  const float* D = w.Dfull + (size_t)p * w.drows * n;
+  for (int idx = tid; idx < 64 * 64; idx += TP_THREADS) {
+    const int tl = idx >> 6, bl = idx & 63;
+    const int t = t0 + tl, b = b0 + bl;
+    float W = 0.f;
+    if (t < len && b < n) {
+      const float wv = 1.f / (dm.eps_idw + D[(size_t)t * n + b]);
+      const float P_ = wv * s_invz[tl];
+      W = inv_len * P_ * (s_lp[bl] - s_L[tl]) * wv;
+    }
+    s_W[bl][tl] = W;
+  }
+  __syncthreads();
+  const int ntt = gridDim.y;
+  if (tid < 64 && b0 + tid < n) {
+    float s = 0.f;
+    for (int tl = 0; tl < 64; ++tl) s += s_W[tid][tl];
+    w.wsum_part[((size_t)p * ntt + blockIdx.y) * n + b0 + tid] = s;
+  }
+  const size_t pstride = (size_t)P * n * cpad;
+  for (int idx = tid; idx < 64 * 8; idx += TP_THREADS) {
+    const int bl = idx >> 3, c8 = idx & 7;
+    const int b = b0 + bl;
+    if (b >= n) continue;
+    __align__(16) __nv_bfloat16 hi[8], mid[8], lo[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) split3_bf16(s_W[bl][c8 * 8 + u], hi[u], mid[u], lo[u]);
+    __nv_bfloat16* dst = w.Wt + ((size_t)p * n + b) * cpad + t0 + c8 * 8;
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(hi);
+    *reinterpret_cast<uint4*>(dst + pstride) = *reinterpret_cast<uint4*>(mid);
+    *reinterpret_cast<uint4*>(dst + 2 * pstride) = *reinterpret_cast<uint4*>(lo);
+  }
+  if (blockIdx.x == 0) {
+    // transpose this token tile's half-queries: Qt[p][e][t]
+    for (int idx = tid; idx < 64 * h; idx += TP_THREADS) {
+      const int tl = idx / h, e = idx - tl * h;
+      const int t = t0 + tl;
+      s_q[tl][e] = t < len ? q[((long long)m * q_stride + t) * dm.d + (long long)j * h + e] : __float2bfloat16(0.f);
+    }
+    __syncthreads();
+    for (int idx = tid; idx < h * 8; idx += TP_THREADS) {
+      const int e = idx >> 3, c8 = idx & 7;
+      __align__(16) __nv_bfloat16 v8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v8[u] = s_q[c8 * 8 + u][e];
+      *reinterpret_cast<uint4*>(w.Qt + ((size_t)p * h + e) * cpad + t0 + c8 * 8) = *reinterpret_cast<uint4*>(v8);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+int launch_qnorm(const Dims& d, const Work& w, const void* q, long long q_stride, int wt0, int len, cudaStream_t s) {
+  if (len <= 0) return 0;
+  dim3 grid((len + 7) / 8, d.M);
+  qnorm_kernel<<<grid, TP_THREADS, 0, s>>>(d, w, (const __nv_bfloat16*)q, q_stride, wt0, len);
+  return 1;
+}
+
+int launch_keyprep(const Dims& d, const Work& w, const float* K1, const float* K2, cudaStream_t s) {
+  const long long rows = (long long)d.M * 2 * d.n;
+  keyprep_kernel<<<(unsigned)((rows + TP_THREADS - 1) / TP_THREADS), TP_THREADS, 0, s>>>(d, w, K1, K2);
+  return 1;
+}
+
+int launch_tc_score(const Dims& d, const Work& w, const void* q_base, long long q_stride, int q_extent, int q_row0,
+                    int wt0, int len, bool key_update, cudaStream_t s) {
+  if (len <= 0) return 0;
+  const int P = d.M * 2;
+  CUtensorMap A, B;
+  if (!make_tmap_bf16_3d(&A, q_base, d.d, q_extent, d.M, (uint64_t)d.d * 2, (uint64_t)q_stride * d.d * 2)) return -1;
+  if (!make_tmap_bf16_3d(&B, w.Kpc, d.h, d.n, 3 * P, (uint64_t)d.h * 2, (uint64_t)d.n * d.h * 2)) return -1;
+  TcGemm g = {};
+  g.P = P;
+  g.k_blocks = d.h / 64;
+  g.n_tiles = (d.n + 127) / 128;
+  g.tiles_per_cta = 2;
+  g.a_pieces = 1; g.b_pieces = 3;
+  g.a_div = 2; g.a_xoff = d.h; g.a_y0 = q_row0; g.a_zpiece = 0; g.b_zpiece = P;
+  g.m_valid = len; g.n_valid = d.n;
+  g.epi = TC_EPI_DIST;
+  g.out = w.Dfull; g.out_pstride = (long long)w.drows * d.n; g.out_ld = d.n;
+  g.rowv = w.qn; g.rowv_pstride = w.max_T; g.rowv_off = wt0;
+  g.colv = w.kn; g.colv_pstride = d.n;
+  g.zpart = key_update ? w.zpart : nullptr; g.zpart_pstride = d.C; g.eps = d.eps_idw;
+  g.status = w.status;
+  return launch_tc_gemm(A, B, g, (len + 127) / 128, s);
+}
+
+int launch_topk_rows(const Dims& d, const Work& w, int wt0, int len, cudaStream_t s) {
+  if (len <= 0) return 0;
+  dim3 grid((len + 7) / 8, d.M * 2);
+  topk_rows_kernel<<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
+  return 1;
+}
+
+int launch_tc_address(const Dims& d, const Work& w, float* K1, float* K2, const void* q, long long q_stride, int len,
+                      cudaStream_t s) {
+  if (len <= 0) return 0;
+  const int P = d.M * 2;
+  const int cpad = (d.C + 63) / 64 * 64;
+  const int ntt = (len + 63) / 64;
+  tc_pbar_kernel<<<dim3((d.n + TP_THREADS - 1) / TP_THREADS, P, PBAR_SLICES), TP_THREADS, 0, s>>>(d, w, len);
+  tc_lp_kernel<<<(unsigned)(((long long)P * d.n + TP_THREADS - 1) / TP_THREADS), TP_THREADS, 0, s>>>(d, w, len);
+  tc_rowL_kernel<<<dim3((len + 7) / 8, P), TP_THREADS, 0, s>>>(d, w, len);
+  tc_wbuild_kernel<<<dim3((d.n + 63) / 64, ntt, P), TP_THREADS, 0, s>>>(d, w, (const __nv_bfloat16*)q, q_stride, len,
+                                                                         cpad);
+  CUtensorMap A, B;
+  if (!make_tmap_bf16_3d(&A, w.Wt, len, d.n, 3 * P, (uint64_t)cpad * 2, (uint64_t)d.n * cpad * 2)) return -1;
+  if (!make_tmap_bf16_3d(&B, w.Qt, len, d.h, P, (uint64_t)cpad * 2, (uint64_t)d.h * cpad * 2)) return -1;
+  TcGemm g = {};
+  g.P = P;
+  g.k_blocks = ntt;
+  g.n_tiles = 1;
+  g.tiles_per_cta = 1;
+  g.a_pieces = 3; g.b_pieces = 1;
+  g.a_div = 1; g.a_xoff = 0; g.a_y0 = 0; g.a_zpiece = P; g.b_zpiece = 0;
+  g.m_valid = d.n; g.n_valid = d.h;
+  g.epi = TC_EPI_KEYSTEP;
+  g.K1 = K1; g.K2 = K2; g.Kpc = w.Kpc; g.kn = w.kn;
+  g.wsum_part = w.wsum_part; g.wsum_tiles = ntt; g.lr = d.lr_key;
+  g.status = w.status;
+  return 4 + launch_tc_gemm(A, B, g, (d.n + 127) / 128, s);
+}
+
+}  // namespace fwpkm
