@@ -213,7 +213,7 @@ def run_ours(args, w, rank, world, local_rank):
     for _ in range(max(args.warmup, 1)):
         step()
     kinds = {}
-    for name in ("gather", "write", "score", "cartesian", "sort", "address"):
+    for name in ("gather", "write", "score", "topk", "cartesian", "sort", "address", "prep", "other"):
         st.profile_kernel(name)
         step()
         ms, n = st.kernel_time()

@@ -177,7 +177,7 @@ uint64_t fwpkm_launch_count(void);
 
 /* Per-kernel timing with CUDA events recorded on the launching stream around every
  * launch of the given kernel kind (0 = none).  Kinds: 1 gather, 2 write, 3 score,
- * 4 cartesian, 5 sort, 6 address.  fwpkm_kernel_time() waits for the events and
+ * 4 cartesian, 5 sort, 6 address (key step), 7 residual, 8 per-half top-k, 9 query/key prep.  fwpkm_kernel_time() waits for the events and
  * returns the summed duration (ms) and the number of timed launches since the last
  * reset, then resets.  Graph replays overwrite their own events, so after graph
  * replays it covers the last replay. */

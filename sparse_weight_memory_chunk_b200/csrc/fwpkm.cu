@@ -247,10 +247,10 @@ fwpkm_status fwpkm_forward_chunk(fwpkm_state* st, const void* q, const void* v, 
   const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
   st->host_error = 0;
   if (st->wk.tc) {
-    run(st, KK_OTHER, s, [&] { return launch_qnorm(d, st->wk, q, seq_stride, 0, c_len, s); });
-    run(st, KK_OTHER, s, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, s); });
+    run(st, KK_PREP, s, [&] { return launch_qnorm(d, st->wk, q, seq_stride, 0, c_len, s); });
+    run(st, KK_PREP, s, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, s); });
     run(st, KK_SCORE, s, [&] { return launch_tc_score(d, st->wk, q, seq_stride, c_len, 0, 0, c_len, ku, s); });
-    run(st, KK_SCORE, s, [&] { return launch_topk_rows(d, st->wk, 0, c_len, s); });
+    run(st, KK_TOPK, s, [&] { return launch_topk_rows(d, st->wk, 0, c_len, s); });
   } else {
     run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, q, seq_stride, 0, c_len, ku, s); });
   }
@@ -315,8 +315,8 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
   const bool tc = st->wk.tc != 0;
   st->host_error = 0;
   if (tc) {
-    run(st, KK_OTHER, s, [&] { return launch_qnorm(d, st->wk, q, T, 0, T, s); });
-    run(st, KK_OTHER, s, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, s); });
+    run(st, KK_PREP, s, [&] { return launch_qnorm(d, st->wk, q, T, 0, T, s); });
+    run(st, KK_PREP, s, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, s); });
   }
   if (!ku) {
     // keys are frozen: address every token once, for all passes
@@ -324,7 +324,7 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
       for (int w0 = 0; w0 < T; w0 += st->wk.drows) {
         const int wl = T - w0 < st->wk.drows ? T - w0 : st->wk.drows;
         run(st, KK_SCORE, s, [&] { return launch_tc_score(d, st->wk, q, T, T, w0, w0, wl, false, s); });
-        run(st, KK_SCORE, s, [&] { return launch_topk_rows(d, st->wk, w0, wl, s); });
+        run(st, KK_TOPK, s, [&] { return launch_topk_rows(d, st->wk, w0, wl, s); });
       }
     } else {
       run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, q, T, 0, T, false, s); });
@@ -340,7 +340,7 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
         const void* qc = offs(q, (long long)t0 * d.d, es);
         if (tc) {
           run(st, KK_SCORE, s, [&] { return launch_tc_score(d, st->wk, q, T, T, t0, t0, len, true, s); });
-          run(st, KK_SCORE, s, [&] { return launch_topk_rows(d, st->wk, t0, len, s); });
+          run(st, KK_TOPK, s, [&] { return launch_topk_rows(d, st->wk, t0, len, s); });
         } else {
           run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, qc, T, t0, len, true, s); });
         }
@@ -385,7 +385,7 @@ fwpkm_status fwpkm_sync(fwpkm_state* st, void* stream) {
 }
 
 fwpkm_status fwpkm_profile_kernel(fwpkm_state* st, int kind) {
-  if (!st || kind < 0 || kind > KK_OTHER) return FWPKM_ERR_INVALID_ARG;
+  if (!st || kind < 0 || kind > KK_LAST) return FWPKM_ERR_INVALID_ARG;
   if (kind != 0 && st->ev.empty()) {
     st->ev.resize(4096);
     for (auto& e : st->ev)

@@ -15,7 +15,7 @@ enum : int { DEV_OK = 0, DEV_BAD_SLOT = 1, DEV_TIMEOUT = 2 };
 
 // Kernel kinds for the launch counter / per-kernel timing.
 enum KernelKind : int { KK_NONE = 0, KK_GATHER = 1, KK_WRITE = 2, KK_SCORE = 3, KK_CART = 4,
-                        KK_SORT = 5, KK_ADDR = 6, KK_OTHER = 7 };
+                        KK_SORT = 5, KK_ADDR = 6, KK_OTHER = 7, KK_TOPK = 8, KK_PREP = 9, KK_LAST = 9 };
 
 struct Dims {
   int n, h, d, dv, k, C, M;

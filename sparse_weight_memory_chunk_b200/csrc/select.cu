@@ -4,6 +4,7 @@
 // Fast-weight Product Key Memory (rainbus summary), PKM prerequisite and method
 // step 2; (paperlayer summary) §2.2: the final top-k is searched in the Cartesian
 // product of the two halves' top-k, and the k selected slots get normalised weights.
+#include "bitonic.cuh"
 #include "fwpkm_internal.cuh"
 
 namespace fwpkm {
@@ -11,20 +12,30 @@ namespace fwpkm {
 // ---------------------------------------------------------------------------
 // Cartesian top-k: one warp per (memory, token).
 //
-// sigma_j = -log(eps + D_j) on the 2k survivors.  Each half is put in (sigma desc,
-// sub-key asc) order; then a pair of ranks (i, j) can only be in the final top-k if
-// (i+1)(j+1) <= k, because every pair (i' <= i, j' <= j) scores at least as high
-// and wins exact ties on the slot index.  Lane i owns row i of that staircase and
-// the k winners are extracted in (score desc, slot asc) order.  Weights are the
-// softmax of the k scores.
+// sigma_j = -log(eps + D_j) on the 2k survivors.  Each half is bitonic-sorted into
+// (sigma desc, sub-key asc) order; then a pair of ranks (i, j) can only be in the final
+// top-k if (i+1)(j+1) <= k, because every pair (i' <= i, j' <= j) scores at least as
+// high and wins exact ties on the slot index.  Those ~k ln k candidates are packed as
+// (score desc, slot asc) keys, bitonic-sorted, and the first k are the answer.  Weights
+// are the softmax of the k scores.
 // ---------------------------------------------------------------------------
 constexpr int CART_WARPS = 8;
 
+template <int VPT>
+__device__ __forceinline__ void sort_cand(u64* cand, int lane) {
+  u64 x[VPT];
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) x[u] = cand[lane * VPT + u];
+  warp_sort_asc<VPT>(x, lane);
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) cand[lane * VPT + u] = x[u];
+}
+
 __global__ void __launch_bounds__(CART_WARPS * 32)
-cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_out,
-                 float* __restrict__ w_out) {
+cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
   __shared__ float s_sig[CART_WARPS][2][32];
   __shared__ int s_sub[CART_WARPS][2][32];
+  __shared__ u64 s_cand[CART_WARPS][128];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i_tok = blockIdx.x * CART_WARPS + warp;
   const int m = blockIdx.y;
@@ -34,63 +45,58 @@ cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_ou
 
   for (int j = 0; j < 2; ++j) {
     const size_t base = (((size_t)m * 2 + j) * w.max_T + tok) * k;
-    float sig = 0.f;
-    int sub = 0;
-    unsigned long long key = ~0ull;
+    u64 key[1] = {~0ull};
     if (lane < k) {
-      sub = w.A[base + lane];
-      sig = -logf(dm.eps_idw + w.Dsv[base + lane]);
-      key = ((unsigned long long)(~orderable(sig)) << 32) | (unsigned)sub;  // sigma desc, sub asc
+      const int sub = w.A[base + lane];
+      const float sig = -logf(dm.eps_idw + w.Dsv[base + lane]);
+      key[0] = ((u64)(~float_key(sig)) << 32) | (unsigned)sub;  // sigma desc, sub asc
     }
-    int rank = 0;
-    for (int o = 0; o < 32; ++o) {
-      unsigned long long other = __shfl_sync(0xffffffffu, key, o);
-      rank += (other < key) ? 1 : 0;
-    }
+    warp_sort_asc<1>(key, lane);
     if (lane < k) {
-      s_sig[warp][j][rank] = sig;
-      s_sub[warp][j][rank] = sub;
+      s_sig[warp][j][lane] = key_float(~(uint32_t)(key[0] >> 32));
+      s_sub[warp][j][lane] = (int)(key[0] & 0xffffffffu);
     }
   }
   __syncwarp();
 
-  // candidate keys of row `lane`: (score desc, slot asc) packed so that smaller = better
+  // staircase candidates: lane i owns rank i of half 1 and pairs it with ranks
+  // 0 .. k/(i+1)-1 of half 2
   const int rowlen = lane < k ? k / (lane + 1) : 0;
-  const float sig1 = lane < k ? s_sig[warp][0][lane] : 0.f;
-  const int a = lane < k ? s_sub[warp][0][lane] : 0;
-  auto cand = [&](int jj) -> unsigned long long {
-    float S = sig1 + s_sig[warp][1][jj];
-    unsigned slot = (unsigned)(a * n + s_sub[warp][1][jj]);
-    return ((unsigned long long)(~orderable(S)) << 32) | slot;
-  };
-  unsigned long long best = ~0ull;
-  for (int jj = 0; jj < rowlen; ++jj) {
-    unsigned long long c = cand(jj);
-    best = c < best ? c : best;
+  int incl = rowlen;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
-  unsigned long long mine = ~0ull;  // lane r keeps the r-th winner
-  for (int r = 0; r < k; ++r) {
-    unsigned long long win = warp_min_u64(best);
-    if (lane == r) mine = win;
-    if (best == win) {
-      best = ~0ull;
-      for (int jj = 0; jj < rowlen; ++jj) {
-        unsigned long long c = cand(jj);
-        if (c > win && c < best) best = c;
-      }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  u64* cand = s_cand[warp];
+  if (rowlen > 0) {
+    const float sig1 = s_sig[warp][0][lane];
+    const unsigned a = (unsigned)s_sub[warp][0][lane];
+    int pos = incl - rowlen;
+    for (int jj = 0; jj < rowlen; ++jj) {
+      const float S = sig1 + s_sig[warp][1][jj];
+      const unsigned slot = a * (unsigned)n + (unsigned)s_sub[warp][1][jj];
+      cand[pos + jj] = ((u64)(~float_key(S)) << 32) | slot;
     }
   }
-  // unpack, softmax over the k scores (max is rank 0)
+  const int Sz = total <= 32 ? 32 : total <= 64 ? 64 : 128;
+  for (int jx = total + lane; jx < Sz; jx += 32) cand[jx] = ~0ull;
+  __syncwarp();
+  if (Sz == 32) sort_cand<1>(cand, lane);
+  else if (Sz == 64) sort_cand<2>(cand, lane);
+  else sort_cand<4>(cand, lane);
+  __syncwarp();
+
   float S = 0.f;
   int slot = 0;
   if (lane < k) {
-    uint32_t o = ~(uint32_t)(mine >> 32);
-    uint32_t u = (o & 0x80000000u) ? (o & 0x7fffffffu) : ~o;
-    S = __uint_as_float(u);
-    slot = (int)(mine & 0xffffffffu);
+    const u64 key = cand[lane];
+    S = key_float(~(uint32_t)(key >> 32));
+    slot = (int)(key & 0xffffffffu);
   }
   const float smax = __shfl_sync(0xffffffffu, S, 0);
-  float e = lane < k ? expf(S - smax) : 0.f;
+  const float e = lane < k ? expf(S - smax) : 0.f;
   const float z = warp_sum(e);
   if (lane < k) {
     const float wt = e / z;
@@ -115,14 +121,16 @@ int launch_cartesian(const Dims& d, const Work& w, int wt0, int len, int32_t* id
 //
 // Keys are (slot << 32) | (t_local * k + r); ascending order groups each slot's
 // readers in token order, which is the summation order of the write.  Segment
-// boundaries give N_read,i (paperlayer §3.3 read-count consensus).  Bitonic sort in
-// shared memory; all orders are fixed, so the result is deterministic.
+// boundaries give N_read,i (paperlayer §3.3 read-count consensus).  Register-resident
+// bitonic sort (VPT keys per thread); all orders are fixed, so the result is
+// deterministic.
 // ---------------------------------------------------------------------------
 constexpr int SORT_THREADS = 1024;
 
+template <int VPT>
 __global__ void __launch_bounds__(SORT_THREADS)
 sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) {
-  extern __shared__ unsigned long long s_keys[];
+  extern __shared__ u64 s_keys[];
   __shared__ int s_warp[SORT_THREADS / 32];
   __shared__ int s_base;
   const int m = blockIdx.y;
@@ -133,80 +141,70 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
   int npair = clen;
   if (!last_has_target && tc0 + clen == total_len) npair = clen - 1;
   const int P = npair * k;
-  int Ppad = 1;
+  int Ppad = 32 * VPT;
   while (Ppad < P) Ppad <<= 1;
   const int cslot = (wt0 + tc0) / C;
   const size_t cbase = (size_t)m * w.max_chunks + cslot;
+  const int tid = threadIdx.x;
 
-  for (int i = threadIdx.x; i < Ppad; i += SORT_THREADS) {
-    unsigned long long key = ~0ull;
+  u64 x[VPT];
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) {
+    const int i = tid * VPT + u;
+    u64 key = ~0ull;
     if (i < P) {
-      int t_local = i / k, r = i - t_local * k;
-      int slot = w.idx[((size_t)m * w.max_T + wt0 + tc0 + t_local) * k + r];
-      key = ((unsigned long long)(unsigned)slot << 32) | (unsigned)i;
+      const int t_local = i / k, r = i - t_local * k;
+      const int slot = w.idx[((size_t)m * w.max_T + wt0 + tc0 + t_local) * k + r];
+      key = ((u64)(unsigned)slot << 32) | (unsigned)i;
     }
-    s_keys[i] = key;
+    x[u] = key;
   }
+  block_sort_asc<VPT>(x, s_keys, Ppad);
+  if (tid * VPT < Ppad)
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) s_keys[tid * VPT + u] = x[u];
   __syncthreads();
-  for (int kk = 2; kk <= Ppad; kk <<= 1) {
-    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-      for (int i = threadIdx.x; i < Ppad; i += SORT_THREADS) {
-        int ixj = i ^ jj;
-        if (ixj > i) {
-          unsigned long long a = s_keys[i], b = s_keys[ixj];
-          bool up = (i & kk) == 0;
-          if ((a > b) == up) {
-            s_keys[i] = b;
-            s_keys[ixj] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
+
   // segments: compaction of the positions where the slot changes
   uint32_t* pair_tr = w.pair_tr + (size_t)m * w.max_chunks * C * k + (size_t)cslot * C * k;
   int32_t* seg_start = w.seg_start + cbase * (C * k + 1);
   int32_t* seg_slot = w.seg_slot + cbase * (C * k);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) s_base = 0;
+  const int warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) s_base = 0;
   __syncthreads();
   for (int i0 = 0; i0 < P; i0 += SORT_THREADS) {
-    const int i = i0 + threadIdx.x;
+    const int i = i0 + tid;
     bool head = false;
-    unsigned long long key = 0;
+    u64 key = 0;
     if (i < P) {
       key = s_keys[i];
       pair_tr[i] = (uint32_t)(key & 0xffffffffu);
       head = (i == 0) || ((s_keys[i - 1] >> 32) != (key >> 32));
     }
-    unsigned bal = __ballot_sync(0xffffffffu, head);
+    const unsigned bal = __ballot_sync(0xffffffffu, head);
     if (lane == 0) s_warp[warp] = __popc(bal);
     __syncthreads();
     if (warp == 0) {
-      int v = s_warp[lane];
+      const int v = s_warp[lane];
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
       s_warp[lane] = incl - v;  // exclusive
     }
     __syncthreads();
     if (head) {
-      int pos = s_base + s_warp[warp] + __popc(bal & ((1u << lane) - 1u));
+      const int pos = s_base + s_warp[warp] + __popc(bal & ((1u << lane) - 1u));
       seg_start[pos] = i;
       seg_slot[pos] = (int32_t)(key >> 32);
     }
     __syncthreads();
-    if (threadIdx.x == SORT_THREADS - 1) {
-      // last thread: total heads in this tile = exclusive prefix of last warp + its count
-      s_base += s_warp[SORT_THREADS / 32 - 1] + __popc(bal);
-    }
+    if (tid == SORT_THREADS - 1) s_base += s_warp[SORT_THREADS / 32 - 1] + __popc(bal);
     __syncthreads();
   }
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     seg_start[s_base] = P;
     w.nseg[cbase] = s_base;
   }
@@ -216,12 +214,21 @@ int launch_sort_pairs(const Dims& d, const Work& w, int wt0, int total_len, bool
                       cudaStream_t s) {
   if (total_len <= 0) return 0;
   const int nchunks = (total_len + d.C - 1) / d.C;
-  int Ppad = 1;
-  while (Ppad < d.C * d.k) Ppad <<= 1;
-  size_t smem = sizeof(unsigned long long) * (size_t)Ppad;
-  cudaFuncSetAttribute(sort_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int P = d.C * d.k;
   dim3 grid(nchunks, d.M);
-  sort_pairs_kernel<<<grid, SORT_THREADS, smem, s>>>(d, w, wt0, total_len, last_has_target ? 1 : 0);
+  if (P <= 8 * SORT_THREADS) {
+    int Ppad = 256;
+    while (Ppad < P) Ppad <<= 1;
+    const size_t smem = sizeof(u64) * (size_t)Ppad;
+    cudaFuncSetAttribute(sort_pairs_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    sort_pairs_kernel<8><<<grid, SORT_THREADS, smem, s>>>(d, w, wt0, total_len, last_has_target ? 1 : 0);
+  } else {
+    int Ppad = 512;
+    while (Ppad < P) Ppad <<= 1;
+    const size_t smem = sizeof(u64) * (size_t)Ppad;
+    cudaFuncSetAttribute(sort_pairs_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    sort_pairs_kernel<16><<<grid, SORT_THREADS, smem, s>>>(d, w, wt0, total_len, last_has_target ? 1 : 0);
+  }
   return 1;
 }
 

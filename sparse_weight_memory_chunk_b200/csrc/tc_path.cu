@@ -7,6 +7,7 @@
 // w = 1/(eps + D), Z_t = sum_a w, P = w / Z_t, pbar = mean_t P, lp = log pbar,
 // L_t = sum_a P lp, W[t][b] = (1/len) P[t][b] (lp[b] - L_t) w[t][b]; the key-step GEMM
 // then forms sum_t W[t][b] q_t and updates the keys in its epilogue.
+#include "bitonic.cuh"
 #include "fwpkm_internal.cuh"
 #include "sm100.cuh"
 
@@ -71,34 +72,106 @@ keyprep_kernel(Dims dm, Work w, const float* __restrict__ K1, const float* __res
   w.kn[(size_t)p * dm.n + b] = ss;
 }
 
-// Per-half top-k from distance rows: one warp per (problem, token); the k smallest
-// (distance, index) keys, each round the winning lane advances past the last winner.
+// Per-half top-k from distance rows: one warp per (problem, token).  Keys are
+// (distance, index) packed so that the k smallest keys are the k nearest sub-keys with
+// ties to the lower index.  The row sits in registers (NPL values per lane).  tau = the
+// k-th smallest of the 32 lane minima bounds the answer (at least k keys are <= tau);
+// the few keys <= tau are compacted into shared memory and bitonic-sorted, and the
+// first k are the result.  If unusually many keys pass (> 256) the warp falls back to
+// k rounds of warp-wide minimum extraction over its registers.
+template <int NPL>
 __global__ void __launch_bounds__(TP_THREADS)
 topk_rows_kernel(Dims dm, Work w, int wt0, int len) {
+  __shared__ u64 s_cand[TP_THREADS / 32][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * (TP_THREADS / 32) + warp;
   const int p = blockIdx.y;
   if (i >= len) return;
   const int n = dm.n, k = dm.k;
   const float* row = w.Dfull + ((size_t)p * w.drows + i) * n;
-  unsigned long long best = ~0ull;
-  for (int a = lane; a < n; a += 32) {
-    unsigned long long key = ((unsigned long long)orderable(row[a]) << 32) | (unsigned)a;
-    best = key < best ? key : best;
+  float v[NPL];
+#pragma unroll
+  for (int u = 0; u < NPL; ++u) {
+    const int a = lane + 32 * u;
+    v[u] = a < n ? row[a] : 0.f;
   }
+  auto key_of = [&](int u) -> u64 {
+    const int a = lane + 32 * u;
+    return a < n ? (((u64)float_key(v[u]) << 32) | (unsigned)a) : ~0ull;
+  };
+  u64 mn = ~0ull;
+#pragma unroll
+  for (int u = 0; u < NPL; ++u) mn = umin64(mn, key_of(u));
+  u64 lm[1] = {mn};
+  warp_sort_asc<1>(lm, lane);
+  const u64 tau = __shfl_sync(0xffffffffu, lm[0], k - 1);
+  int c = 0;
+#pragma unroll
+  for (int u = 0; u < NPL; ++u) c += key_of(u) <= tau ? 1 : 0;
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
   const size_t obase = ((size_t)p * w.max_T + wt0 + i) * k;
-  for (int r = 0; r < k; ++r) {
-    const unsigned long long win = warp_min_u64(best);
-    const int a = (int)(win & 0xffffffffu);
-    if (lane == 0) {
-      w.A[obase + r] = a;
-      w.Dsv[obase + r] = row[a];
+  u64* cand = s_cand[warp];
+  if (total <= 256) {
+    int pos = incl - c;
+#pragma unroll
+    for (int u = 0; u < NPL; ++u) {
+      const u64 key = key_of(u);
+      if (key <= tau) cand[pos++] = key;
     }
-    if ((a & 31) == lane) {
-      best = ~0ull;
-      for (int b = lane; b < n; b += 32) {
-        unsigned long long key = ((unsigned long long)orderable(row[b]) << 32) | (unsigned)b;
-        if (key > win && key < best) best = key;
+    const int S = total <= 32 ? 32 : total <= 64 ? 64 : total <= 128 ? 128 : 256;
+    for (int jx = total + lane; jx < S; jx += 32) cand[jx] = ~0ull;
+    __syncwarp();
+    if (S == 32) {
+      u64 x[1] = {cand[lane]};
+      warp_sort_asc<1>(x, lane);
+      cand[lane] = x[0];
+    } else if (S == 64) {
+      u64 x[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) x[u] = cand[lane * 2 + u];
+      warp_sort_asc<2>(x, lane);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) cand[lane * 2 + u] = x[u];
+    } else if (S == 128) {
+      u64 x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] = cand[lane * 4 + u];
+      warp_sort_asc<4>(x, lane);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) cand[lane * 4 + u] = x[u];
+    } else {
+      u64 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = cand[lane * 8 + u];
+      warp_sort_asc<8>(x, lane);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) cand[lane * 8 + u] = x[u];
+    }
+    __syncwarp();
+    if (lane < k) {
+      const u64 key = cand[lane];
+      w.A[obase + lane] = (int)(key & 0xffffffffu);
+      w.Dsv[obase + lane] = key_float((uint32_t)(key >> 32));
+    }
+  } else {
+    u64 last = 0;
+    for (int r = 0; r < k; ++r) {
+      u64 best = ~0ull;
+#pragma unroll
+      for (int u = 0; u < NPL; ++u) {
+        const u64 key = key_of(u);
+        if ((r == 0 || key > last) && key < best) best = key;
+      }
+      last = warp_min_u64(best);
+      if (lane == 0) {
+        w.A[obase + r] = (int)(last & 0xffffffffu);
+        w.Dsv[obase + r] = key_float((uint32_t)(last >> 32));
       }
     }
   }
@@ -267,7 +340,14 @@ int launch_tc_score(const Dims& d, const Work& w, const void* q_base, long long 
 int launch_topk_rows(const Dims& d, const Work& w, int wt0, int len, cudaStream_t s) {
   if (len <= 0) return 0;
   dim3 grid((len + 7) / 8, d.M * 2);
-  topk_rows_kernel<<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
+  const int npl = (d.n + 31) / 32;
+  if (npl <= 2) topk_rows_kernel<2><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
+  else if (npl <= 4) topk_rows_kernel<4><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
+  else if (npl <= 8) topk_rows_kernel<8><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
+  else if (npl <= 16) topk_rows_kernel<16><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
+  else if (npl <= 32) topk_rows_kernel<32><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
+  else if (npl <= 64) topk_rows_kernel<64><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
+  else topk_rows_kernel<128><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
   return 1;
 }
 

@@ -19,7 +19,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_
 F32, BF16 = 0, 1
 KEY_UPDATE, TARGET_NORM, LOOKAHEAD, GATE_WEIGHT = 1, 2, 4, 8
 DEFAULT_FLAGS = TARGET_NORM | LOOKAHEAD | GATE_WEIGHT
-KIND = {"gather": 1, "write": 2, "score": 3, "cartesian": 4, "sort": 5, "address": 6, "other": 7}
+KIND = {"gather": 1, "write": 2, "score": 3, "cartesian": 4, "sort": 5, "address": 6, "other": 7, "topk": 8,
+        "prep": 9}
 
 
 class FwpkmError(RuntimeError):
