@@ -10,6 +10,7 @@
 // the value loop (gather, write) stays chunk-sequential.
 #include <atomic>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -19,6 +20,14 @@
 using namespace fwpkm;
 
 static std::atomic<uint64_t> g_launches{0};
+
+struct SeqKey {
+  const void *q, *v, *g, *o;
+  int T, n_iter, prof_kind;
+  bool operator==(const SeqKey& x) const {
+    return q == x.q && v == x.v && g == x.g && o == x.o && T == x.T && n_iter == x.n_iter && prof_kind == x.prof_kind;
+  }
+};
 
 struct fwpkm_state {
   fwpkm_config cfg;
@@ -36,6 +45,15 @@ struct fwpkm_state {
   std::vector<cudaEvent_t> ev;
   int ev_used;
   int host_error;  // a launch could not be set up (e.g. tensor map encoding failed)
+  // run_sequence schedule: internal streams, dependency events and the cached graph
+  cudaStream_t sK, sS, sV, sCap;
+  std::vector<cudaEvent_t> sync_ev;
+  size_t ev_next;
+  int no_graph;
+  cudaGraphExec_t graph_exec;
+  SeqKey graph_key;
+  uint64_t graph_kernels;
+  int graph_ev_used;
 };
 
 namespace {
@@ -97,6 +115,15 @@ void run(fwpkm_state* st, int kind, cudaStream_t s, F&& f) {
   else g_launches += (uint64_t)nl;
 }
 
+cudaEvent_t next_event(fwpkm_state* st) {
+  if (st->ev_next == st->sync_ev.size()) {
+    cudaEvent_t e = nullptr;
+    cudaEventCreateWithFlags(&e, cudaEventDisableTiming);
+    st->sync_ev.push_back(e);
+  }
+  return st->sync_ev[st->ev_next++];
+}
+
 }  // namespace
 
 namespace fwpkm {
@@ -114,7 +141,10 @@ int addressing_window(const Dims& d, int max_T) {
   size_t wtok = ((size_t)64 << 20) / per_tok / 128 * 128;
   if (wtok < 128) wtok = 128;
   const size_t need = ((size_t)max_T + 127) / 128 * 128;
-  return (int)(wtok < need ? wtok : need);
+  if (wtok > need) wtok = need;
+  wtok = wtok / d.C * d.C;  // whole chunks, so a window's pairs can be sorted on their own
+  if (wtok < (size_t)d.C) wtok = d.C;
+  return (int)wtok;
 }
 
 size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
@@ -143,7 +173,9 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
   const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
   x.tc = use_tensor_cores(d) ? 1 : 0;
   x.drows = ku ? (int)C : (x.tc ? addressing_window(d, max_T) : 0);
-  x.Dfull = x.drows ? (float*)take(4 * M * 2 * (size_t)x.drows * n) : nullptr;
+  // with the key step the tensor-core path keeps two chunks of distance rows in flight
+  const size_t dbufs = (ku && x.tc) ? 2 : 1;
+  x.Dfull = x.drows ? (float*)take(4 * dbufs * M * 2 * (size_t)x.drows * n) : nullptr;
   if (ku) {
     x.Z = (float*)take(4 * M * 2 * C);
     x.lp = (float*)take(4 * M * 2 * n);
@@ -215,6 +247,22 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
   st->pending = 0;
   st->prof_kind = 0;
   st->ev_used = 0;
+  st->host_error = 0;
+  st->ev_next = 0;
+  st->graph_exec = nullptr;
+  st->graph_kernels = 0;
+  st->graph_ev_used = 0;
+  {
+    const char* e = getenv("FWPKM_NO_GRAPH");
+    st->no_graph = (e && e[0] == '1') ? 1 : 0;
+  }
+  if (cudaStreamCreateWithFlags(&st->sK, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&st->sS, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&st->sV, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&st->sCap, cudaStreamNonBlocking) != cudaSuccess) {
+    delete st;
+    return FWPKM_ERR_CUDA;
+  }
   if (cudaMemset(st->wk.status, 0, sizeof(int)) != cudaSuccess) {
     delete st;
     return FWPKM_ERR_CUDA;
@@ -225,6 +273,12 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
 
 void fwpkm_destroy_state(fwpkm_state* st) {
   if (!st) return;
+  if (st->graph_exec) cudaGraphExecDestroy(st->graph_exec);
+  for (cudaEvent_t e : st->sync_ev) cudaEventDestroy(e);
+  cudaStreamDestroy(st->sK);
+  cudaStreamDestroy(st->sS);
+  cudaStreamDestroy(st->sV);
+  cudaStreamDestroy(st->sCap);
   for (cudaEvent_t e : st->ev) cudaEventDestroy(e);
   delete st;
 }
@@ -285,6 +339,120 @@ fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream
   return last_cuda();
 }
 
+// Enqueue a whole sequence as three stream-ordered chains that fork from and join back
+// to `origin`:
+//   sK  addressing: q norms, key pieces, scoring GEMM, entropy key step (K-chain)
+//   sS  selection: per-half top-k, Cartesian search, pair sort
+//   sV  values: gather + gated output, sorted write
+// Addressing never reads V, so sK/sS run ahead of sV; sV only waits for the selection
+// of the chunk it is about to read.  The scoring GEMM writes its distance rows into one
+// of two buffers, so sK may start chunk c+1 while sS still reads chunk c's rows.  Across
+// passes, chunk c's selection waits for the previous pass's write of chunk c (its slot
+// lists and weights are overwritten).
+static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, const float* g, int T, int n_iter,
+                             float* o, cudaStream_t origin) {
+  const Dims& d = st->dm;
+  const size_t es = qv_size(d);
+  const int C = d.C;
+  const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
+  const bool la = (d.flags & FWPKM_LOOKAHEAD) != 0;
+  const bool tc = st->wk.tc != 0;
+  const int nch = (T + C - 1) / C;
+  cudaStream_t sK = st->sK, sS = st->sS, sV = st->sV;
+  st->ev_next = 0;
+  auto dep = [&](cudaStream_t from, cudaStream_t to) {
+    cudaEvent_t e = next_event(st);
+    cudaEventRecord(e, from);
+    cudaStreamWaitEvent(to, e, 0);
+  };
+  auto mark = [&](cudaStream_t s) {
+    cudaEvent_t e = next_event(st);
+    cudaEventRecord(e, s);
+    return e;
+  };
+  dep(origin, sK);
+  dep(origin, sS);
+  dep(origin, sV);
+
+  auto value_chunk = [&](int c) {
+    const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
+    const void* vc = offs(v, (long long)t0 * d.dv, es);
+    const void* vn = (t0 + len < T) ? offs(v, (long long)(t0 + len) * d.dv, es) : nullptr;
+    run(st, KK_GATHER, sV, [&] {
+      return launch_gather(d, st->wk, st->V, vc, g + t0, T, t0, len, o + (long long)t0 * d.dv, true, vn, sV);
+    });
+    run(st, KK_WRITE, sV, [&] { return launch_write(d, st->wk, st->V, t0, sV); });
+  };
+
+  if (tc) {
+    run(st, KK_PREP, sK, [&] { return launch_qnorm(d, st->wk, q, T, 0, T, sK); });
+    run(st, KK_PREP, sK, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, sK); });
+  }
+  if (!ku) {
+    // frozen keys: address window by window on sK; the value loop of a window starts as
+    // soon as its chunks are sorted.  The addressing serves every pass.
+    const int wtok = tc ? st->wk.drows : T;
+    std::vector<cudaEvent_t> ready;
+    for (int w0 = 0; w0 < T; w0 += wtok) {
+      const int wl = T - w0 < wtok ? T - w0 : wtok;
+      if (tc) {
+        run(st, KK_SCORE, sK, [&] { return launch_tc_score(d, st->wk, q, T, T, w0, w0, wl, false, sK); });
+        run(st, KK_TOPK, sK, [&] { return launch_topk_rows(d, st->wk, w0, wl, sK); });
+      } else {
+        run(st, KK_SCORE, sK, [&] {
+          return launch_score_topk(d, st->wk, st->K1, st->K2, offs(q, (long long)w0 * d.d, es), T, w0, wl, false, sK);
+        });
+      }
+      run(st, KK_CART, sK, [&] { return launch_cartesian(d, st->wk, w0, wl, nullptr, nullptr, sK); });
+      run(st, KK_SORT, sK, [&] { return launch_sort_pairs(d, st->wk, w0, wl, !la || (w0 + wl < T), sK); });
+      ready.push_back(mark(sK));
+    }
+    for (int pass = 0; pass < n_iter; ++pass)
+      for (int c = 0; c < nch; ++c) {
+        if (pass == 0 && (c * C) % wtok == 0) cudaStreamWaitEvent(sV, ready[(c * C) / wtok], 0);
+        value_chunk(c);
+      }
+  } else {
+    const size_t dbuf = (size_t)d.M * 2 * d.C * d.n;
+    std::vector<cudaEvent_t> topk_done(2, nullptr), sel_done(nch, nullptr), val_done(nch, nullptr);
+    int cnt = 0;
+    for (int pass = 0; pass < n_iter; ++pass) {
+      for (int c = 0; c < nch; ++c, ++cnt) {
+        const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
+        const void* qc = offs(q, (long long)t0 * d.d, es);
+        Work wb = st->wk;
+        if (tc) wb.Dfull = st->wk.Dfull + (size_t)(cnt & 1) * dbuf;
+        if (sel_done[c]) cudaStreamWaitEvent(sK, sel_done[c], 0);    // previous pass read A/Dsv
+        if (topk_done[cnt & 1]) cudaStreamWaitEvent(sK, topk_done[cnt & 1], 0);  // buffer reuse
+        if (tc) {
+          run(st, KK_SCORE, sK, [&] { return launch_tc_score(d, wb, q, T, T, t0, t0, len, true, sK); });
+        } else {
+          run(st, KK_SCORE, sK, [&] { return launch_score_topk(d, wb, st->K1, st->K2, qc, T, t0, len, true, sK); });
+        }
+        cudaStreamWaitEvent(sS, mark(sK), 0);
+        run(st, KK_ADDR, sK, [&] {
+          return tc ? launch_tc_address(d, wb, st->K1, st->K2, qc, T, len, sK)
+                    : launch_address(d, wb, st->K1, st->K2, qc, T, len, sK);
+        });
+        if (val_done[c]) cudaStreamWaitEvent(sS, val_done[c], 0);     // previous pass wrote chunk c
+        if (tc) {
+          run(st, KK_TOPK, sS, [&] { return launch_topk_rows(d, wb, t0, len, sS); });
+          topk_done[cnt & 1] = mark(sS);
+        }
+        run(st, KK_CART, sS, [&] { return launch_cartesian(d, wb, t0, len, nullptr, nullptr, sS); });
+        run(st, KK_SORT, sS, [&] { return launch_sort_pairs(d, wb, t0, len, !la || (t0 + len < T), sS); });
+        sel_done[c] = mark(sS);
+        cudaStreamWaitEvent(sV, sel_done[c], 0);
+        value_chunk(c);
+        val_done[c] = mark(sV);
+      }
+    }
+  }
+  dep(sK, origin);
+  dep(sS, origin);
+  dep(sV, origin);
+}
+
 fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, const float* g, int T,
                                 int n_iter, float* o, void* stream) {
   if (!st) return FWPKM_ERR_INVALID_ARG;
@@ -294,67 +462,45 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
   fwpkm_status ps = peek_status(st);
   if (ps != FWPKM_OK) return ps;
   st->pending = 0;
-  const Dims& d = st->dm;
-  const size_t es = qv_size(d);
-  const int C = d.C;
-  const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
-  const bool la = (d.flags & FWPKM_LOOKAHEAD) != 0;
-  cudaStream_t s = (cudaStream_t)stream;
-  const int nch = (T + C - 1) / C;
-
-  auto value_chunk = [&](int c) {
-    const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
-    const void* vc = offs(v, (long long)t0 * d.dv, es);
-    const void* vn = (t0 + len < T) ? offs(v, (long long)(t0 + len) * d.dv, es) : nullptr;
-    run(st, KK_GATHER, s, [&] {
-      return launch_gather(d, st->wk, st->V, vc, g + t0, T, t0, len, o + (long long)t0 * d.dv, true, vn, s);
-    });
-    run(st, KK_WRITE, s, [&] { return launch_write(d, st->wk, st->V, t0, s); });
-  };
-
-  const bool tc = st->wk.tc != 0;
   st->host_error = 0;
-  if (tc) {
-    run(st, KK_PREP, s, [&] { return launch_qnorm(d, st->wk, q, T, 0, T, s); });
-    run(st, KK_PREP, s, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, s); });
+  cudaStream_t user = (cudaStream_t)stream;
+  if (st->no_graph) {
+    enqueue_sequence(st, q, v, g, T, n_iter, o, user);
+    if (st->host_error) return FWPKM_ERR_CUDA;
+    return last_cuda();
   }
-  if (!ku) {
-    // keys are frozen: address every token once, for all passes
-    if (tc) {
-      for (int w0 = 0; w0 < T; w0 += st->wk.drows) {
-        const int wl = T - w0 < st->wk.drows ? T - w0 : st->wk.drows;
-        run(st, KK_SCORE, s, [&] { return launch_tc_score(d, st->wk, q, T, T, w0, w0, wl, false, s); });
-        run(st, KK_TOPK, s, [&] { return launch_topk_rows(d, st->wk, w0, wl, s); });
-      }
-    } else {
-      run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, q, T, 0, T, false, s); });
+  // One CUDA graph per distinct call: replayed while the arguments stay the same.
+  const SeqKey key = {q, v, g, o, T, n_iter, st->prof_kind};
+  if (!st->graph_exec || !(key == st->graph_key)) {
+    if (st->graph_exec) {
+      cudaGraphExecDestroy(st->graph_exec);
+      st->graph_exec = nullptr;
     }
-    run(st, KK_CART, s, [&] { return launch_cartesian(d, st->wk, 0, T, nullptr, nullptr, s); });
-    run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, st->wk, 0, T, !la, s); });
-    for (int pass = 0; pass < n_iter; ++pass)
-      for (int c = 0; c < nch; ++c) value_chunk(c);
-  } else {
-    for (int pass = 0; pass < n_iter; ++pass) {
-      for (int c = 0; c < nch; ++c) {
-        const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
-        const void* qc = offs(q, (long long)t0 * d.d, es);
-        if (tc) {
-          run(st, KK_SCORE, s, [&] { return launch_tc_score(d, st->wk, q, T, T, t0, t0, len, true, s); });
-          run(st, KK_TOPK, s, [&] { return launch_topk_rows(d, st->wk, t0, len, s); });
-        } else {
-          run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, qc, T, t0, len, true, s); });
-        }
-        run(st, KK_CART, s, [&] { return launch_cartesian(d, st->wk, t0, len, nullptr, nullptr, s); });
-        run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, st->wk, t0, len, !la || (t0 + len < T), s); });
-        value_chunk(c);
-        run(st, KK_ADDR, s, [&] {
-          return tc ? launch_tc_address(d, st->wk, st->K1, st->K2, qc, T, len, s)
-                    : launch_address(d, st->wk, st->K1, st->K2, qc, T, len, s);
-        });
-      }
+    const uint64_t before = g_launches.load();
+    if (cudaStreamBeginCapture(st->sCap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return last_cuda();
+    enqueue_sequence(st, q, v, g, T, n_iter, o, st->sCap);
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamEndCapture(st->sCap, &graph);
+    st->graph_kernels = g_launches.load() - before;
+    g_launches -= st->graph_kernels;  // counted per replay below
+    if (e != cudaSuccess || st->host_error) {
+      if (graph) cudaGraphDestroy(graph);
+      last_cuda();
+      return FWPKM_ERR_CUDA;
     }
+    e = cudaGraphInstantiate(&st->graph_exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (e != cudaSuccess) {
+      st->graph_exec = nullptr;
+      last_cuda();
+      return FWPKM_ERR_CUDA;
+    }
+    st->graph_key = key;
+    st->graph_ev_used = st->ev_used;
   }
-  if (st->host_error) return FWPKM_ERR_CUDA;
+  if (cudaGraphLaunch(st->graph_exec, user) != cudaSuccess) return last_cuda();
+  g_launches += st->graph_kernels;
+  st->ev_used = st->graph_ev_used;
   return last_cuda();
 }
 
