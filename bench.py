@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--n-iter", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--kernel", default=None,
+                    help="kernel kind timed for the roofline (default: the slowest kind, found by one timed step each)")
     return ap.parse_args()
 
 
@@ -213,13 +215,16 @@ def run_ours(args, w, rank, world, local_rank):
     for _ in range(max(args.warmup, 1)):
         step()
     kinds = {}
-    for name in ("gather", "write", "score", "topk", "cartesian", "sort", "address", "prep", "other"):
-        st.profile_kernel(name)
-        step()
-        ms, n = st.kernel_time()
-        kinds[name] = (ms, n)
-    st.profile_kernel(0)
-    dominant = max(kinds, key=lambda k_: kinds[k_][0])
+    if args.kernel is None:
+        for name in ("gather", "write", "score", "topk", "cartesian", "sort", "address", "prep", "other"):
+            st.profile_kernel(name)
+            step()
+            ms, n = st.kernel_time()
+            kinds[name] = (ms, n)
+        st.profile_kernel(0)
+        dominant = max(kinds, key=lambda k_: kinds[k_][0])
+    else:
+        dominant = args.kernel
     st.profile_kernel(dominant)
     st.sync()
 

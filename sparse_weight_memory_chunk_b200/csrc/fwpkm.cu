@@ -105,10 +105,15 @@ fwpkm_status last_cuda() {
 template <class F>
 void run(fwpkm_state* st, int kind, cudaStream_t s, F&& f) {
   const bool prof = st->prof_kind == kind && st->ev_used + 2 <= (int)st->ev.size();
-  if (prof) cudaEventRecord(st->ev[st->ev_used], s);
+  // Under stream capture a plain record is only a dependency marker; timing events must
+  // become event-record nodes of the graph.
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (prof) cudaStreamIsCapturing(s, &cs);
+  const unsigned rec_flags = cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+  if (prof) cudaEventRecordWithFlags(st->ev[st->ev_used], s, rec_flags);
   int nl = f();
   if (prof) {
-    cudaEventRecord(st->ev[st->ev_used + 1], s);
+    cudaEventRecordWithFlags(st->ev[st->ev_used + 1], s, rec_flags);
     st->ev_used += 2;
   }
   if (nl < 0) st->host_error = 1;
