@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--n-iter", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override the number of sequences B (profiling)")
+    ap.add_argument("--tokens", type=int, default=None, help="override T (profiling)")
     ap.add_argument("--kernel", default=None,
                     help="kernel kind timed for the roofline (default: the slowest kind, found by one timed step each)")
     return ap.parse_args()
@@ -357,6 +359,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     _, w = BY_NAME[args.workload]
+    if args.batch or args.tokens:
+        from dataclasses import replace
+        w = replace(w, B=args.batch or w.B, T=args.tokens or w.T)
     if args.impl == "reference":
         run_reference(args, w, rank)
         return
