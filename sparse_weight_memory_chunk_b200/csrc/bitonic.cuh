@@ -77,15 +77,19 @@ __device__ void block_sort_asc(u64 (&x)[VPT], u64* sm, int S) {
   for (int kk = 2; kk <= S; kk <<= 1) {
     int jj = kk >> 1;
     for (; jj >= warp_span; jj >>= 1) {  // partner in another warp: exchange through shared memory
+      // striped layout (slot u of thread t at u*nthr + t): conflict-free for both the
+      // stores and the partner loads, whose thread index differs only above the lane bits
+      const int nthr = S / VPT;
       if (active)
 #pragma unroll
-        for (int u = 0; u < VPT; ++u) sm[base + u] = x[u];
+        for (int u = 0; u < VPT; ++u) sm[u * nthr + tid] = x[u];
       __syncthreads();
       if (active) {
+        const int ptid = tid ^ (jj / VPT);
 #pragma unroll
         for (int u = 0; u < VPT; ++u) {
           const int i = base + u;
-          const u64 other = sm[i ^ jj];
+          const u64 other = sm[u * nthr + ptid];
           const bool up = (i & kk) == 0;
           const bool lower = (i & jj) == 0;
           x[u] = (lower == up) ? umin64(x[u], other) : umax64(x[u], other);

@@ -196,7 +196,7 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
     x.kn = (float*)take(4 * P * n);
     x.qn = (float*)take(4 * P * T);
     if (ku) {
-      x.zpart = (float*)take(4 * P * C * nt);
+      x.zpart = (float*)take(4 * P * C * nt * 4);
       x.ppart = (float*)take(4 * P * 8 * n);
       x.Wt = (__nv_bfloat16*)take(2 * 3 * P * n * cpad);
       x.Qt = (__nv_bfloat16*)take(2 * P * h * cpad);

@@ -49,7 +49,7 @@ struct Work {
   __nv_bfloat16* Kpc;// [3][M*2][n][h]     bf16 pieces hi/mid/lo of the keys
   float* kn;         // [M*2][n]           squared key norms
   float* qn;         // [M*2][max_T]       squared half-query norms
-  float* zpart;      // [M*2][C][n/128]    per-tile partial sums of 1/(eps + D)
+  float* zpart;      // [M*2][C][n/128][4] per-32-column partial sums of 1/(eps + D)
   float* ppart;      // [M*2][8][n]        partial column sums for pbar
   __nv_bfloat16* Wt; // [3][M*2][n][Cpad]  key-step weights, sub-key major, bf16 pieces
   __nv_bfloat16* Qt; // [M*2][h][Cpad]     chunk half-queries, feature major

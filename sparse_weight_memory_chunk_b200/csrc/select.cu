@@ -121,18 +121,26 @@ int launch_cartesian(const Dims& d, const Work& w, int wt0, int len, int32_t* id
 //
 // Keys are (slot << 32) | (t_local * k + r); ascending order groups each slot's
 // readers in token order, which is the summation order of the write.  Segment
-// boundaries give N_read,i (paperlayer §3.3 read-count consensus).  Register-resident
-// bitonic sort (VPT keys per thread); all orders are fixed, so the result is
-// deterministic.
+// boundaries give N_read,i (paperlayer §3.3 read-count consensus).
+//
+// The keys are first bucketed by the top bits of the slot (buckets follow slot order;
+// ~64 keys per bucket on average) and each warp then ranks the keys of its buckets by
+// comparing every key with every other key of the bucket, writing each to its rank.
+// The scatter into buckets may land keys in any order, but ranking by the full unique
+// key makes the result independent of it.  If a bucket is larger than 128 keys
+// (strongly skewed slot use) the CTA sorts all keys with a register bitonic network.
 // ---------------------------------------------------------------------------
 constexpr int SORT_THREADS = 1024;
+constexpr int SORT_BUCKET_KEYS = 64;   // average keys per bucket
+constexpr int SORT_BUCKET_CAP = 128;   // largest bucket the ranking path handles
 
 template <int VPT>
 __global__ void __launch_bounds__(SORT_THREADS)
 sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) {
   extern __shared__ u64 s_keys[];
+  __shared__ int s_cnt[512], s_off[513], s_cur[512];
   __shared__ int s_warp[SORT_THREADS / 32];
-  __shared__ int s_base;
+  __shared__ int s_base, s_max;
   const int m = blockIdx.y;
   const int cc = blockIdx.x;
   const int C = dm.C, k = dm.k;
@@ -143,33 +151,93 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
   const int P = npair * k;
   int Ppad = 32 * VPT;
   while (Ppad < P) Ppad <<= 1;
+  const int NB = Ppad / SORT_BUCKET_KEYS;  // <= 512
   const int cslot = (wt0 + tc0) / C;
   const size_t cbase = (size_t)m * w.max_chunks + cslot;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+  for (int b = tid; b < NB; b += SORT_THREADS) s_cnt[b] = 0;
+  __syncthreads();
   u64 x[VPT];
+  int bk[VPT];
 #pragma unroll
   for (int u = 0; u < VPT; ++u) {
     const int i = tid * VPT + u;
     u64 key = ~0ull;
+    bk[u] = -1;
     if (i < P) {
       const int t_local = i / k, r = i - t_local * k;
-      const int slot = w.idx[((size_t)m * w.max_T + wt0 + tc0 + t_local) * k + r];
-      key = ((u64)(unsigned)slot << 32) | (unsigned)i;
+      const unsigned slot = (unsigned)w.idx[((size_t)m * w.max_T + wt0 + tc0 + t_local) * k + r];
+      key = ((u64)slot << 32) | (unsigned)i;
+      bk[u] = (int)(((u64)slot * (u64)NB) / (u64)dm.N);
+      atomicAdd(&s_cnt[bk[u]], 1);
     }
     x[u] = key;
   }
-  block_sort_asc<VPT>(x, s_keys, Ppad);
-  if (tid * VPT < Ppad)
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of the bucket sizes, and the largest bucket
+    int run = 0, mx = 0;
+    for (int b0 = 0; b0 < NB; b0 += 32) {
+      const int v = b0 + lane < NB ? s_cnt[b0 + lane] : 0;
+      int incl = v, vm = v;
 #pragma unroll
-    for (int u = 0; u < VPT; ++u) s_keys[tid * VPT + u] = x[u];
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+        vm = max(vm, __shfl_xor_sync(0xffffffffu, vm, o));
+      }
+      if (b0 + lane < NB) {
+        s_off[b0 + lane] = run + incl - v;
+        s_cur[b0 + lane] = run + incl - v;
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
+      mx = max(mx, vm);
+    }
+    if (lane == 0) {
+      s_off[NB] = run;
+      s_max = mx;
+    }
+  }
+  __syncthreads();
+  if (s_max <= SORT_BUCKET_CAP) {
+#pragma unroll
+    for (int u = 0; u < VPT; ++u)
+      if (bk[u] >= 0) s_keys[atomicAdd(&s_cur[bk[u]], 1)] = x[u];
+    __syncthreads();
+    for (int b = warp; b < NB; b += SORT_THREADS / 32) {
+      const int base = s_off[b], cnt = s_off[b + 1] - base;
+      if (cnt == 0) continue;
+      u64 mine[SORT_BUCKET_CAP / 32];
+      int rk[SORT_BUCKET_CAP / 32];
+#pragma unroll
+      for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j) {
+        const int i = lane + 32 * j;
+        mine[j] = i < cnt ? s_keys[base + i] : ~0ull;
+        rk[j] = 0;
+      }
+      for (int t = 0; t < cnt; ++t) {
+        const u64 o = s_keys[base + t];
+#pragma unroll
+        for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j) rk[j] += o < mine[j] ? 1 : 0;
+      }
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j)
+        if (lane + 32 * j < cnt) s_keys[base + rk[j]] = mine[j];
+      __syncwarp();
+    }
+  } else {
+    block_sort_asc<VPT>(x, s_keys, Ppad);
+    if (tid * VPT < Ppad)
+#pragma unroll
+      for (int u = 0; u < VPT; ++u) s_keys[tid * VPT + u] = x[u];
+  }
   __syncthreads();
 
   // segments: compaction of the positions where the slot changes
   uint32_t* pair_tr = w.pair_tr + (size_t)m * w.max_chunks * C * k + (size_t)cslot * C * k;
   int32_t* seg_start = w.seg_start + cbase * (C * k + 1);
   int32_t* seg_slot = w.seg_slot + cbase * (C * k);
-  const int warp = tid >> 5, lane = tid & 31;
   if (tid == 0) s_base = 0;
   __syncthreads();
   for (int i0 = 0; i0 < P; i0 += SORT_THREADS) {

@@ -13,8 +13,9 @@
 // hi + mid + lo (~24 significant bits), each piece pair accumulating into one fp32 TMEM
 // accumulator, so the contraction matches fp32 arithmetic to ~1e-7 relative.
 //
-// CTA = 6 warps: warp 0 issues TMA loads, warp 1 owns TMEM and issues the MMAs (one
-// thread), warps 2-5 drain TMEM (warp w reads TMEM lanes 32*(w%4)..+31 = tile rows).
+// CTA = 18 warps: warp 0 issues TMA loads, warp 1 owns TMEM and issues the MMAs (one
+// thread), warps 2-17 drain TMEM: warp w reads TMEM lanes 32*(w%4)..+31 (tile rows) and
+// the 32 columns of column group (w-2)/4, so four warps share every lane quarter.
 // Accumulators are double-buffered (2 x 128 columns) so the epilogue of tile j overlaps
 // the MMAs of tile j+1.  Every wait is bounded (globaltimer); on timeout the CTA raises a
 // shared abort flag, drains its own in-flight copies and MMAs, frees TMEM and reports
@@ -31,7 +32,8 @@ using namespace sm100;
 constexpr int TC_BM = 128, TC_BN = 128, TC_BK = 64;
 constexpr int TC_TILE_BYTES = TC_BM * TC_BK * 2;  // 16 KiB, also the B tile (TC_BN == TC_BM)
 constexpr int TC_STAGES = 3;
-constexpr int TC_THREADS = 192;
+constexpr int TC_EPI_WARPS = 16;
+constexpr int TC_THREADS = (2 + TC_EPI_WARPS) * 32;
 constexpr uint32_t TC_TMEM_COLS = 256;
 constexpr uint64_t TC_TIMEOUT_NS = 200ull * 1000 * 1000;
 
@@ -63,8 +65,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* accf = empty + TC_STAGES;
   uint64_t* acce = accf + 2;
   uint64_t* drain = acce + 2;
-  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  uint64_t* normbar = drain + 1;
+  uint32_t* tmem_slot = (uint32_t*)(normbar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  __shared__ float s_norm[4][TC_BM];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = blockIdx.z, mt = blockIdx.y;
@@ -78,9 +82,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accf[b], 1);
-      mbar_init(&acce[b], 4);
+      mbar_init(&acce[b], TC_EPI_WARPS);
     }
     mbar_init(drain, 1);
+    mbar_init(normbar, TC_EPI_WARPS);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -158,8 +163,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     umma_commit(drain);  // completes once every MMA issued above has finished
     wait_deadline(drain, 0, deadline + TC_TIMEOUT_NS);
   } else if (ntiles > 0 && warp >= 2) {
-    // ---------------- epilogue: 4 warps, one tile row per thread ----------------
+    // ---------------- epilogue: 16 warps; warp w reads TMEM lane quarter w%4 (tile rows
+    // 32*(w%4)..+31, one per thread) and column group (w-2)/4 (32 columns) ----------------
     const int q = warp & 3;
+    const int cg = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const int m = p >> 1, jh = p & 1;
@@ -174,79 +181,96 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int nt = nt0 + j;
       const int r = mt * TC_BM + row;
       const bool rv = r < g.m_valid;
+      uint32_t v[32];
+      tmem_ld32(lane_base + (uint32_t)(b * TC_BN + cg * 32), v);
+      tmem_wait_ld();
+      // accumulator drained: hand the buffer back before the (longer) epilogue math
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[b]);
       if (g.epi == TC_EPI_DIST) {
+        const int c0 = nt * TC_BN + cg * 32;
         const float rq = rv ? g.rowv[(size_t)p * g.rowv_pstride + g.rowv_off + r] : 0.f;
         const float* kn = g.colv + (size_t)p * g.colv_pstride;
         float* out = g.out + ((size_t)p * g.out_pstride + (size_t)r * g.out_ld);
+        float dv[32];
         float zacc = 0.f;
-        for (int cc = 0; cc < TC_BN / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(lane_base + (uint32_t)(b * TC_BN + cc * 32), v);
-          tmem_wait_ld();
-          const int c0 = nt * TC_BN + cc * 32;
-          float dv[32];
+        if (c0 + 32 <= g.n_valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(kn + c0 + i);
+            const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              dv[i + u] = fmaxf((rq + kk[u]) - 2.f * __uint_as_float(v[i + u]), 0.f);
+              zacc += __fdividef(1.f, g.eps + dv[i + u]);
+            }
+          }
+          if (rv) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(out + c0 + i) = make_float4(dv[i], dv[i + 1], dv[i + 2], dv[i + 3]);
+          }
+        } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int c = c0 + i;
             const float kv = c < g.n_valid ? kn[c] : 0.f;
             dv[i] = fmaxf((rq + kv) - 2.f * __uint_as_float(v[i]), 0.f);
-            if (c < g.n_valid) zacc += 1.f / (g.eps + dv[i]);
-          }
-          if (rv) {
-            if (c0 + 32 <= g.n_valid) {
-#pragma unroll
-              for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4*>(out + c0 + i) = make_float4(dv[i], dv[i + 1], dv[i + 2], dv[i + 3]);
-            } else {
-              for (int i = 0; i < 32; ++i)
-                if (c0 + i < g.n_valid) out[c0 + i] = dv[i];
+            if (c < g.n_valid) {
+              zacc += __fdividef(1.f, g.eps + dv[i]);
+              if (rv) out[c] = dv[i];
             }
           }
         }
-        if (rv && g.zpart) g.zpart[((size_t)p * g.zpart_pstride + r) * g.n_tiles + nt] = zacc;
+        if (rv && g.zpart)
+          g.zpart[(((size_t)p * g.zpart_pstride + r) * g.n_tiles + nt) * 4 + cg] = zacc;
       } else {  // TC_EPI_KEYSTEP: row = sub-key b, columns = features e (one tile covers h)
         const int h = g.n_valid;
         const int n = g.m_valid;
-        float wsum = 0.f;
-        if (rv)
-          for (int tt = 0; tt < g.wsum_tiles; ++tt) wsum += g.wsum_part[((size_t)p * g.wsum_tiles + tt) * n + r];
-        float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h;
-        const size_t pstride = (size_t)g.P * n * h;
-        __nv_bfloat16* pc = g.Kpc + ((size_t)p * n + r) * h;
+        const int e0 = cg * 32;
         float ss = 0.f;
-        for (int cc = 0; cc < TC_BN / 32 && cc * 32 < h; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(lane_base + (uint32_t)(b * TC_BN + cc * 32), v);
-          tmem_wait_ld();
-          if (rv) {
+        if (rv && e0 < h) {
+          float wsum = 0.f;
+          for (int tt = 0; tt < g.wsum_tiles; ++tt) wsum += g.wsum_part[((size_t)p * g.wsum_tiles + tt) * n + r];
+          float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h;
+          const size_t pstride = (size_t)g.P * n * h;
+          __nv_bfloat16* pc = g.Kpc + ((size_t)p * n + r) * h;
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              const int e = cc * 32 + i;
-              float4 k0 = *reinterpret_cast<const float4*>(K + e);
-              float4 k1 = *reinterpret_cast<const float4*>(K + e + 4);
-              float kin[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-              float kout[8];
-              __align__(16) __nv_bfloat16 hi[8], mid[8], lo[8];
+          for (int i = 0; i < 32; i += 8) {
+            const int e = e0 + i;
+            const float4 k0 = *reinterpret_cast<const float4*>(K + e);
+            const float4 k1 = *reinterpret_cast<const float4*>(K + e + 4);
+            const float kin[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+            float kout[8];
+            __align__(16) __nv_bfloat16 hi[8], mid[8], lo[8];
 #pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                const float grad = 2.f * (__uint_as_float(v[i + u]) - wsum * kin[u]);
-                kout[u] = kin[u] - g.lr * grad;
-                ss += kout[u] * kout[u];
-                split3(kout[u], hi[u], mid[u], lo[u]);
-              }
-              *reinterpret_cast<float4*>(K + e) = make_float4(kout[0], kout[1], kout[2], kout[3]);
-              *reinterpret_cast<float4*>(K + e + 4) = make_float4(kout[4], kout[5], kout[6], kout[7]);
-              *reinterpret_cast<uint4*>(pc + e) = *reinterpret_cast<uint4*>(hi);
-              *reinterpret_cast<uint4*>(pc + pstride + e) = *reinterpret_cast<uint4*>(mid);
-              *reinterpret_cast<uint4*>(pc + 2 * pstride + e) = *reinterpret_cast<uint4*>(lo);
+            for (int u = 0; u < 8; ++u) {
+              const float grad = 2.f * (__uint_as_float(v[i + u]) - wsum * kin[u]);
+              kout[u] = kin[u] - g.lr * grad;
+              ss += kout[u] * kout[u];
+              split3(kout[u], hi[u], mid[u], lo[u]);
             }
+            *reinterpret_cast<float4*>(K + e) = make_float4(kout[0], kout[1], kout[2], kout[3]);
+            *reinterpret_cast<float4*>(K + e + 4) = make_float4(kout[4], kout[5], kout[6], kout[7]);
+            *reinterpret_cast<uint4*>(pc + e) = *reinterpret_cast<uint4*>(hi);
+            *reinterpret_cast<uint4*>(pc + pstride + e) = *reinterpret_cast<uint4*>(mid);
+            *reinterpret_cast<uint4*>(pc + 2 * pstride + e) = *reinterpret_cast<uint4*>(lo);
           }
         }
-        if (rv) g.kn[(size_t)p * n + r] = ss;
+        // squared norm of the new key: the four column groups' partials, summed in order
+        // by the column-group-0 warp once all 16 warps have published theirs (one tile per
+        // CTA in this mode, so the barrier has a single phase; the wait is bounded)
+        s_norm[cg][row] = ss;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(normbar);
+        if (cg == 0) {
+          int okn = lane == 0 ? (mbar_wait(normbar, 0, abort_flag, deadline) ? 1 : 0) : 0;
+          okn = __shfl_sync(0xffffffffu, okn, 0);
+          if (okn && rv)
+            g.kn[(size_t)p * n + r] = ((s_norm[0][row] + s_norm[1][row]) + s_norm[2][row]) + s_norm[3][row];
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[b]);
     }
   }
 

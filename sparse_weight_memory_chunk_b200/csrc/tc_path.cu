@@ -74,15 +74,20 @@ keyprep_kernel(Dims dm, Work w, const float* __restrict__ K1, const float* __res
 
 // Per-half top-k from distance rows: one warp per (problem, token).  Keys are
 // (distance, index) packed so that the k smallest keys are the k nearest sub-keys with
-// ties to the lower index.  The row sits in registers (NPL values per lane).  tau = the
-// k-th smallest of the 32 lane minima bounds the answer (at least k keys are <= tau);
-// the few keys <= tau are compacted into shared memory and bitonic-sorted, and the
-// first k are the result.  If unusually many keys pass (> 256) the warp falls back to
-// k rounds of warp-wide minimum extraction over its registers.
+// ties to the lower index.  The row sits in registers (NPL values per lane).
+//  1. every lane keeps its two smallest keys; tau = the k-th smallest of those 64
+//     distinct keys, so at least k keys of the row are <= tau (about 36 for k = 32);
+//  2. the keys <= tau are compacted into shared memory;
+//  3. each candidate's rank is counted by comparing it with every other candidate
+//     (independent compares, no dependent network), and the k smallest are written in
+//     rank order.
+// If unusually many keys pass (> 128) the warp falls back to k rounds of warp-wide
+// minimum extraction over its registers.
 template <int NPL>
 __global__ void __launch_bounds__(TP_THREADS)
 topk_rows_kernel(Dims dm, Work w, int wt0, int len) {
-  __shared__ u64 s_cand[TP_THREADS / 32][256];
+  __shared__ u64 s_cand[TP_THREADS / 32][128];
+  __shared__ u64 s_two[TP_THREADS / 32][64];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * (TP_THREADS / 32) + warp;
   const int p = blockIdx.y;
@@ -99,12 +104,29 @@ topk_rows_kernel(Dims dm, Work w, int wt0, int len) {
     const int a = lane + 32 * u;
     return a < n ? (((u64)float_key(v[u]) << 32) | (unsigned)a) : ~0ull;
   };
-  u64 mn = ~0ull;
+  u64 m1 = ~0ull, m2 = ~0ull;
 #pragma unroll
-  for (int u = 0; u < NPL; ++u) mn = umin64(mn, key_of(u));
-  u64 lm[1] = {mn};
-  warp_sort_asc<1>(lm, lane);
-  const u64 tau = __shfl_sync(0xffffffffu, lm[0], k - 1);
+  for (int u = 0; u < NPL; ++u) {
+    const u64 x = key_of(u);
+    m2 = umin64(m2, umax64(m1, x));
+    m1 = umin64(m1, x);
+  }
+  u64* two = s_two[warp];
+  two[lane] = m1;
+  two[32 + lane] = m2;
+  __syncwarp();
+  int r1 = 0, r2 = 0;
+#pragma unroll 8
+  for (int t = 0; t < 64; ++t) {
+    const u64 o = two[t];
+    r1 += o < m1 ? 1 : 0;
+    r2 += o < m2 ? 1 : 0;
+  }
+  // the key of rank k-1 among the 64 (ranks are unique where keys are; padding keys
+  // ~0 only appear when n < 64 and are never ranked below a real key)
+  const unsigned b1 = __ballot_sync(0xffffffffu, r1 == k - 1);
+  const unsigned b2 = __ballot_sync(0xffffffffu, r2 == k - 1);
+  const u64 tau = b1 ? __shfl_sync(0xffffffffu, m1, __ffs(b1) - 1) : __shfl_sync(0xffffffffu, m2, __ffs(b2) - 1);
   int c = 0;
 #pragma unroll
   for (int u = 0; u < NPL; ++u) c += key_of(u) <= tau ? 1 : 0;
@@ -117,48 +139,32 @@ topk_rows_kernel(Dims dm, Work w, int wt0, int len) {
   const int total = __shfl_sync(0xffffffffu, incl, 31);
   const size_t obase = ((size_t)p * w.max_T + wt0 + i) * k;
   u64* cand = s_cand[warp];
-  if (total <= 256) {
+  if (total <= 128) {
     int pos = incl - c;
 #pragma unroll
     for (int u = 0; u < NPL; ++u) {
       const u64 key = key_of(u);
       if (key <= tau) cand[pos++] = key;
     }
-    const int S = total <= 32 ? 32 : total <= 64 ? 64 : total <= 128 ? 128 : 256;
-    for (int jx = total + lane; jx < S; jx += 32) cand[jx] = ~0ull;
     __syncwarp();
-    if (S == 32) {
-      u64 x[1] = {cand[lane]};
-      warp_sort_asc<1>(x, lane);
-      cand[lane] = x[0];
-    } else if (S == 64) {
-      u64 x[2];
+    u64 mine[4];
+    int rk[4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) x[u] = cand[lane * 2 + u];
-      warp_sort_asc<2>(x, lane);
-#pragma unroll
-      for (int u = 0; u < 2; ++u) cand[lane * 2 + u] = x[u];
-    } else if (S == 128) {
-      u64 x[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) x[u] = cand[lane * 4 + u];
-      warp_sort_asc<4>(x, lane);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) cand[lane * 4 + u] = x[u];
-    } else {
-      u64 x[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = cand[lane * 8 + u];
-      warp_sort_asc<8>(x, lane);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) cand[lane * 8 + u] = x[u];
+    for (int j = 0; j < 4; ++j) {
+      mine[j] = lane + 32 * j < total ? cand[lane + 32 * j] : ~0ull;
+      rk[j] = 0;
     }
-    __syncwarp();
-    if (lane < k) {
-      const u64 key = cand[lane];
-      w.A[obase + lane] = (int)(key & 0xffffffffu);
-      w.Dsv[obase + lane] = key_float((uint32_t)(key >> 32));
+    for (int t = 0; t < total; ++t) {
+      const u64 o = cand[t];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) rk[j] += o < mine[j] ? 1 : 0;
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (lane + 32 * j < total && rk[j] < k) {
+        w.A[obase + rk[j]] = (int)(mine[j] & 0xffffffffu);
+        w.Dsv[obase + rk[j]] = key_float((uint32_t)(mine[j] >> 32));
+      }
   } else {
     u64 last = 0;
     for (int r = 0; r < k; ++r) {
@@ -183,7 +189,7 @@ tc_pbar_kernel(Dims dm, Work w, int len) {
   __shared__ float s_invz[1024 / PBAR_SLICES + 1];
   const int p = blockIdx.y, sl = blockIdx.z;
   const int t0 = (sl * len) / PBAR_SLICES, t1 = ((sl + 1) * len) / PBAR_SLICES;
-  const int nt = (dm.n + 127) / 128;
+  const int nt = (dm.n + 127) / 128 * 4;  // 4 column groups per 128-column tile
   for (int t = t0 + threadIdx.x; t < t1; t += TP_THREADS) {
     const float* zp = w.zpart + ((size_t)p * dm.C + t) * nt;
     float z = 0.f;
@@ -196,7 +202,8 @@ tc_pbar_kernel(Dims dm, Work w, int len) {
   if (a >= dm.n) return;
   const float* D = w.Dfull + (size_t)p * w.drows * dm.n;
   float s = 0.f;
-  for (int t = t0; t < t1; ++t) s += (1.f / (dm.eps_idw + D[(size_t)t * dm.n + a])) * s_invz[t - t0];
+#pragma unroll 8
+  for (int t = t0; t < t1; ++t) s += __fdividef(1.f, dm.eps_idw + D[(size_t)t * dm.n + a]) * s_invz[t - t0];
   w.ppart[((size_t)p * PBAR_SLICES + sl) * dm.n + a] = s;
 }
 
@@ -220,7 +227,8 @@ tc_rowL_kernel(Dims dm, Work w, int len) {
   const float* D = w.Dfull + ((size_t)p * w.drows + t) * dm.n;
   const float* lp = w.lp + (size_t)p * dm.n;
   float s = 0.f;
-  for (int a = lane; a < dm.n; a += 32) s += lp[a] / (dm.eps_idw + D[a]);
+#pragma unroll 8
+  for (int a = lane; a < dm.n; a += 32) s += __fdividef(lp[a], dm.eps_idw + D[a]);
   s = warp_sum(s);
   if (lane == 0) w.Lt[(size_t)p * dm.C + t] = s / w.Z[(size_t)p * dm.C + t];
 }
@@ -248,12 +256,13 @@ tc_wbuild_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long
   __syncthreads();
   const float inv_len = 1.f / (float)len;
   const float* D = w.Dfull + (size_t)p * w.drows * n;
+#pragma unroll 4
   for (int idx = tid; idx < 64 * 64; idx += TP_THREADS) {
     const int tl = idx >> 6, bl = idx & 63;
     const int t = t0 + tl, b = b0 + bl;
     float W = 0.f;
     if (t < len && b < n) {
-      const float wv = 1.f / (dm.eps_idw + D[(size_t)t * n + b]);
+      const float wv = __fdividef(1.f, dm.eps_idw + D[(size_t)t * n + b]);
       const float P_ = wv * s_invz[tl];
       W = inv_len * P_ * (s_lp[bl] - s_L[tl]) * wv;
     }

@@ -8,7 +8,9 @@
 // §A.4 summed (not averaged) loss, so the step is exactly the gradient; §A.5 gate
 // weighting; §3.3 read-count averaging.
 //
-// Rows are moved as 16-byte vectors: a warp covers 512 contiguous bytes per load.
+// Rows are moved as 16-byte vectors: a warp covers 512 contiguous bytes per load.  Both
+// kernels are bound by HBM latency x bytes in flight, so each warp keeps many row loads
+// outstanding before it consumes any of them.
 #include "fwpkm_internal.cuh"
 
 namespace fwpkm {
@@ -80,7 +82,8 @@ __device__ __forceinline__ const VT* target_src(const Dims& dm, const VT* v, con
 
 // ---------------------------------------------------------------------------
 // Gather: one warp per (memory, token).  k rows of d_v fp32 are read in rank order
-// with 16-byte loads; vhat accumulates in fp32 in that order.
+// with 16-byte loads (8 rows in flight per lane group); vhat accumulates in fp32 in
+// rank order.
 // ---------------------------------------------------------------------------
 template <typename VT, int VPL>
 __global__ void __launch_bounds__(VAL_WARPS * 32)
@@ -103,7 +106,7 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
   float4 acc[VPL];
 #pragma unroll
   for (int c = 0; c < VPL; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
+#pragma unroll 8
   for (int r = 0; r < k; ++r) {
     const int slot = __shfl_sync(0xffffffffu, myslot, r);
     const float wr = __shfl_sync(0xffffffffu, myw, r);
@@ -184,55 +187,86 @@ resid_kernel(Dims dm, Work w, const VT* __restrict__ v, const float* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// Write: one warp per touched row (segment of the sorted pair list).  G_i sums
-// s'_{t,i} r_t in token order; V_i -= G_i / N_read,i.  Rows are disjoint, so there
-// are no atomics and the result does not depend on scheduling.
+// Write: each warp owns G touched rows (segments of the sorted pair list).  It loads the
+// G segment descriptors with one coalesced load, issues all G value-row loads and the
+// first pair of every segment before consuming any of them, then for each row sums
+// G_i = sum s'_{t,i} r_t in token order and stores V_i - G_i / N_read,i.  Rows are
+// disjoint, so there are no atomics and the result does not depend on scheduling.
 // ---------------------------------------------------------------------------
-template <int VPL>
+template <int VPL, int G>
 __global__ void __launch_bounds__(VAL_WARPS * 32)
 write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u = blockIdx.x * VAL_WARPS + warp;
   const int m = blockIdx.y;
   const int C = dm.C, k = dm.k, dv4 = dm.dv >> 2;
   const int cslot = wt0 / C;
   const size_t cbase = (size_t)m * w.max_chunks + cslot;
-  if (u >= w.nseg[cbase]) return;
+  const int ns = w.nseg[cbase];
+  const int u0 = (blockIdx.x * VAL_WARPS + warp) * G;
+  if (u0 >= ns) return;
   const int32_t* seg_start = w.seg_start + cbase * (C * k + 1);
-  const int s0 = seg_start[u], s1 = seg_start[u + 1];
-  const int slot = w.seg_slot[cbase * (C * k) + u];
-  if (slot < 0 || (long long)slot >= dm.N) {
-    if (lane == 0) atomicExch(w.status, DEV_BAD_SLOT);
-    return;
-  }
+  const int32_t* seg_slot = w.seg_slot + cbase * (C * k);
   const uint32_t* pair_tr = w.pair_tr + (size_t)m * w.max_chunks * C * k + (size_t)cslot * C * k;
-  float4 G[VPL];
+  int my_slot = -1, my_s0 = 0, my_s1 = 0;
+  uint32_t my_tr = 0;
+  if (lane < G && u0 + lane < ns) {
+    my_slot = seg_slot[u0 + lane];
+    my_s0 = seg_start[u0 + lane];
+    my_s1 = seg_start[u0 + lane + 1];
+    my_tr = pair_tr[my_s0];
+  }
+  float* Vm = V + (size_t)m * dm.N * dm.dv;
+  float4 Vr[G][VPL];
 #pragma unroll
-  for (int c = 0; c < VPL; ++c) G[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int p = s0; p < s1; ++p) {
-    const uint32_t tr = pair_tr[p];
-    const int t_local = (int)(tr / (uint32_t)k), r = (int)(tr - (uint32_t)t_local * k);
-    const float wt = w.w[((size_t)m * w.max_T + wt0 + t_local) * k + r];
-    const float4* rrow = reinterpret_cast<const float4*>(w.resid + ((size_t)m * C + t_local) * dm.dv);
+  for (int gi = 0; gi < G; ++gi) {
+    const int slot = __shfl_sync(0xffffffffu, my_slot, gi);
+    const bool ok = slot >= 0 && (long long)slot < dm.N;
+    const float4* row = reinterpret_cast<const float4*>(Vm + (size_t)(ok ? slot : 0) * dm.dv);
 #pragma unroll
     for (int c = 0; c < VPL; ++c) {
-      int e4 = lane + 32 * c;
-      if (e4 < dv4) {
-        float4 x = rrow[e4];
-        G[c].x = fmaf(wt, x.x, G[c].x); G[c].y = fmaf(wt, x.y, G[c].y);
-        G[c].z = fmaf(wt, x.z, G[c].z); G[c].w = fmaf(wt, x.w, G[c].w);
-      }
+      const int e4 = lane + 32 * c;
+      Vr[gi][c] = (ok && e4 < dv4) ? row[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
-  const float nr = (float)(s1 - s0);
-  float4* row = reinterpret_cast<float4*>(V + ((size_t)m * dm.N + slot) * dm.dv);
 #pragma unroll
-  for (int c = 0; c < VPL; ++c) {
-    int e4 = lane + 32 * c;
-    if (e4 < dv4) {
-      float4 x = row[e4];
-      x.x -= G[c].x / nr; x.y -= G[c].y / nr; x.z -= G[c].z / nr; x.w -= G[c].w / nr;
-      row[e4] = x;
+  for (int gi = 0; gi < G; ++gi) {
+    const int slot = __shfl_sync(0xffffffffu, my_slot, gi);
+    const int s0 = __shfl_sync(0xffffffffu, my_s0, gi);
+    const int s1 = __shfl_sync(0xffffffffu, my_s1, gi);
+    const uint32_t tr0 = __shfl_sync(0xffffffffu, my_tr, gi);
+    if (u0 + gi >= ns) break;
+    if (slot < 0 || (long long)slot >= dm.N) {
+      if (lane == 0) atomicExch(w.status, DEV_BAD_SLOT);
+      continue;
+    }
+    float4 Gs[VPL];
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) Gs[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p = s0; p < s1; ++p) {
+      const uint32_t tr = p == s0 ? tr0 : pair_tr[p];
+      const int t_local = (int)(tr / (uint32_t)k), r = (int)(tr - (uint32_t)t_local * k);
+      const float wt = w.w[((size_t)m * w.max_T + wt0 + t_local) * k + r];
+      const float4* rrow = reinterpret_cast<const float4*>(w.resid + ((size_t)m * C + t_local) * dm.dv);
+#pragma unroll
+      for (int c = 0; c < VPL; ++c) {
+        const int e4 = lane + 32 * c;
+        if (e4 < dv4) {
+          const float4 x = rrow[e4];
+          Gs[c].x = fmaf(wt, x.x, Gs[c].x); Gs[c].y = fmaf(wt, x.y, Gs[c].y);
+          Gs[c].z = fmaf(wt, x.z, Gs[c].z); Gs[c].w = fmaf(wt, x.w, Gs[c].w);
+        }
+      }
+    }
+    const float nr = (float)(s1 - s0);
+    float4* row = reinterpret_cast<float4*>(Vm + (size_t)slot * dm.dv);
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) {
+      const int e4 = lane + 32 * c;
+      if (e4 < dv4) {
+        float4 x = Vr[gi][c];
+        x.x -= Gs[c].x / nr; x.y -= Gs[c].y / nr; x.z -= Gs[c].z / nr; x.w -= Gs[c].w / nr;
+        row[e4] = x;
+      }
     }
   }
 }
@@ -282,8 +316,15 @@ int launch_resid(const Dims& d, const Work& w, const void* v, const float* g, lo
 }
 
 int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s) {
-  dim3 grid((d.C * d.k + VAL_WARPS - 1) / VAL_WARPS, d.M);
-  FWPKM_VPL_DISPATCH(vpl_of(d.dv), write_kernel<VPL><<<grid, VAL_WARPS * 32, 0, s>>>(d, w, V, wt0));
+  const int vpl = vpl_of(d.dv);
+  const int G = vpl <= 2 ? 4 : vpl == 4 ? 2 : 1;  // rows per warp: ~8 float4 in flight per lane
+  dim3 grid((d.C * d.k + VAL_WARPS * G - 1) / (VAL_WARPS * G), d.M);
+  switch (vpl) {
+    case 1: write_kernel<1, 4><<<grid, VAL_WARPS * 32, 0, s>>>(d, w, V, wt0); break;
+    case 2: write_kernel<2, 4><<<grid, VAL_WARPS * 32, 0, s>>>(d, w, V, wt0); break;
+    case 4: write_kernel<4, 2><<<grid, VAL_WARPS * 32, 0, s>>>(d, w, V, wt0); break;
+    default: write_kernel<8, 1><<<grid, VAL_WARPS * 32, 0, s>>>(d, w, V, wt0); break;
+  }
   return 1;
 }
 
