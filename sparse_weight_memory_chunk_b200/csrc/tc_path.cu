@@ -54,8 +54,11 @@ keyprep_kernel(Dims dm, Work w, const float* __restrict__ K1, const float* __res
   const float* K = (j == 0 ? K1 : K2) + ((size_t)m * dm.n + b) * h;
   const size_t pstride = (size_t)P * dm.n * h;
   __nv_bfloat16* pc = w.Kpc + ((size_t)p * dm.n + b) * h;
-  float ss = 0.f;
+  // squared norm as four 32-feature partial sums combined in order, exactly as the
+  // key-step GEMM epilogue forms it
+  float part[4] = {0.f, 0.f, 0.f, 0.f};
   for (int e = 0; e < h; e += 8) {
+    float& ss = part[e >> 5];
     float4 k0 = *reinterpret_cast<const float4*>(K + e);
     float4 k1 = *reinterpret_cast<const float4*>(K + e + 4);
     float kin[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
@@ -69,7 +72,7 @@ keyprep_kernel(Dims dm, Work w, const float* __restrict__ K1, const float* __res
     *reinterpret_cast<uint4*>(pc + pstride + e) = *reinterpret_cast<uint4*>(mid);
     *reinterpret_cast<uint4*>(pc + 2 * pstride + e) = *reinterpret_cast<uint4*>(lo);
   }
-  w.kn[(size_t)p * dm.n + b] = ss;
+  w.kn[(size_t)p * dm.n + b] = ((part[0] + part[1]) + part[2]) + part[3];
 }
 
 // Per-half top-k from distance rows: one warp per (problem, token).  Keys are
