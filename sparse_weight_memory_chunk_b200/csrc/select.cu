@@ -123,12 +123,14 @@ int launch_cartesian(const Dims& d, const Work& w, int wt0, int len, int32_t* id
 // readers in token order, which is the summation order of the write.  Segment
 // boundaries give N_read,i (paperlayer §3.3 read-count consensus).
 //
-// The keys are first bucketed by the top bits of the slot (buckets follow slot order;
-// ~64 keys per bucket on average) and each warp then ranks the keys of its buckets by
-// comparing every key with every other key of the bucket, writing each to its rank.
-// The scatter into buckets may land keys in any order, but ranking by the full unique
-// key makes the result independent of it.  If a bucket is larger than 128 keys
-// (strongly skewed slot use) the CTA sorts all keys with a register bitonic network.
+// The write needs each slot's readers contiguous and in token order, not a global slot
+// order.  So keys are bucketed by a multiplicative hash of the slot (~64 keys per
+// bucket; a slot falls in exactly one bucket) and each warp ranks the keys of its
+// buckets by comparing every key with every other key of the bucket, writing each to
+// its rank.  The scatter into buckets may land keys in any order, but ranking by the
+// full unique key makes the result independent of it.  If a bucket is larger than 128
+// keys (strongly skewed slot use) the CTA sorts all keys with a register bitonic
+// network instead.
 // ---------------------------------------------------------------------------
 constexpr int SORT_THREADS = 1024;
 constexpr int SORT_BUCKET_KEYS = 64;   // average keys per bucket
@@ -151,7 +153,8 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
   const int P = npair * k;
   int Ppad = 32 * VPT;
   while (Ppad < P) Ppad <<= 1;
-  const int NB = Ppad / SORT_BUCKET_KEYS;  // <= 512
+  const int NB = Ppad / SORT_BUCKET_KEYS;  // <= 512, a power of two
+  const int nb_log2 = 31 - __clz(NB);
   const int cslot = (wt0 + tc0) / C;
   const size_t cbase = (size_t)m * w.max_chunks + cslot;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -169,7 +172,7 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
       const int t_local = i / k, r = i - t_local * k;
       const unsigned slot = (unsigned)w.idx[((size_t)m * w.max_T + wt0 + tc0 + t_local) * k + r];
       key = ((u64)slot << 32) | (unsigned)i;
-      bk[u] = (int)(((u64)slot * (u64)NB) / (u64)dm.N);
+      bk[u] = (int)((slot * 2654435761u) >> (32 - nb_log2));  // multiplicative hash
       atomicAdd(&s_cnt[bk[u]], 1);
     }
     x[u] = key;

@@ -75,117 +75,6 @@ keyprep_kernel(Dims dm, Work w, const float* __restrict__ K1, const float* __res
   w.kn[(size_t)p * dm.n + b] = ((part[0] + part[1]) + part[2]) + part[3];
 }
 
-// Per-half top-k from distance rows: one warp per (problem, token).  Keys are
-// (distance, index) packed so that the k smallest keys are the k nearest sub-keys with
-// ties to the lower index.  The row sits in registers (NPL values per lane).
-//  1. every lane keeps its two smallest keys; tau = the k-th smallest of those 64
-//     distinct keys, so at least k keys of the row are <= tau (about 36 for k = 32);
-//  2. the keys <= tau are compacted into shared memory;
-//  3. each candidate's rank is counted by comparing it with every other candidate
-//     (independent compares, no dependent network), and the k smallest are written in
-//     rank order.
-// If unusually many keys pass (> 128) the warp falls back to k rounds of warp-wide
-// minimum extraction over its registers.
-template <int NPL>
-__global__ void __launch_bounds__(TP_THREADS)
-topk_rows_kernel(Dims dm, Work w, int wt0, int len) {
-  __shared__ u64 s_cand[TP_THREADS / 32][128];
-  __shared__ u64 s_two[TP_THREADS / 32][64];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x * (TP_THREADS / 32) + warp;
-  const int p = blockIdx.y;
-  if (i >= len) return;
-  const int n = dm.n, k = dm.k;
-  const float* row = w.Dfull + ((size_t)p * w.drows + i) * n;
-  float v[NPL];
-#pragma unroll
-  for (int u = 0; u < NPL; ++u) {
-    const int a = lane + 32 * u;
-    v[u] = a < n ? row[a] : 0.f;
-  }
-  auto key_of = [&](int u) -> u64 {
-    const int a = lane + 32 * u;
-    return a < n ? (((u64)float_key(v[u]) << 32) | (unsigned)a) : ~0ull;
-  };
-  u64 m1 = ~0ull, m2 = ~0ull;
-#pragma unroll
-  for (int u = 0; u < NPL; ++u) {
-    const u64 x = key_of(u);
-    m2 = umin64(m2, umax64(m1, x));
-    m1 = umin64(m1, x);
-  }
-  u64* two = s_two[warp];
-  two[lane] = m1;
-  two[32 + lane] = m2;
-  __syncwarp();
-  int r1 = 0, r2 = 0;
-#pragma unroll 8
-  for (int t = 0; t < 64; ++t) {
-    const u64 o = two[t];
-    r1 += o < m1 ? 1 : 0;
-    r2 += o < m2 ? 1 : 0;
-  }
-  // the key of rank k-1 among the 64 (ranks are unique where keys are; padding keys
-  // ~0 only appear when n < 64 and are never ranked below a real key)
-  const unsigned b1 = __ballot_sync(0xffffffffu, r1 == k - 1);
-  const unsigned b2 = __ballot_sync(0xffffffffu, r2 == k - 1);
-  const u64 tau = b1 ? __shfl_sync(0xffffffffu, m1, __ffs(b1) - 1) : __shfl_sync(0xffffffffu, m2, __ffs(b2) - 1);
-  int c = 0;
-#pragma unroll
-  for (int u = 0; u < NPL; ++u) c += key_of(u) <= tau ? 1 : 0;
-  int incl = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  const int total = __shfl_sync(0xffffffffu, incl, 31);
-  const size_t obase = ((size_t)p * w.max_T + wt0 + i) * k;
-  u64* cand = s_cand[warp];
-  if (total <= 128) {
-    int pos = incl - c;
-#pragma unroll
-    for (int u = 0; u < NPL; ++u) {
-      const u64 key = key_of(u);
-      if (key <= tau) cand[pos++] = key;
-    }
-    __syncwarp();
-    u64 mine[4];
-    int rk[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      mine[j] = lane + 32 * j < total ? cand[lane + 32 * j] : ~0ull;
-      rk[j] = 0;
-    }
-    for (int t = 0; t < total; ++t) {
-      const u64 o = cand[t];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) rk[j] += o < mine[j] ? 1 : 0;
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (lane + 32 * j < total && rk[j] < k) {
-        w.A[obase + rk[j]] = (int)(mine[j] & 0xffffffffu);
-        w.Dsv[obase + rk[j]] = key_float((uint32_t)(mine[j] >> 32));
-      }
-  } else {
-    u64 last = 0;
-    for (int r = 0; r < k; ++r) {
-      u64 best = ~0ull;
-#pragma unroll
-      for (int u = 0; u < NPL; ++u) {
-        const u64 key = key_of(u);
-        if ((r == 0 || key > last) && key < best) best = key;
-      }
-      last = warp_min_u64(best);
-      if (lane == 0) {
-        w.A[obase + r] = (int)(last & 0xffffffffu);
-        w.Dsv[obase + r] = key_float((uint32_t)(last >> 32));
-      }
-    }
-  }
-}
-
 // Partial column sums sum_t w[t][a] / Z_t over one token slice; also Z_t itself.
 __global__ void __launch_bounds__(TP_THREADS)
 tc_pbar_kernel(Dims dm, Work w, int len) {
@@ -347,20 +236,6 @@ int launch_tc_score(const Dims& d, const Work& w, const void* q_base, long long 
   g.zpart = key_update ? w.zpart : nullptr; g.zpart_pstride = d.C; g.eps = d.eps_idw;
   g.status = w.status;
   return launch_tc_gemm(A, B, g, (len + 127) / 128, s);
-}
-
-int launch_topk_rows(const Dims& d, const Work& w, int wt0, int len, cudaStream_t s) {
-  if (len <= 0) return 0;
-  dim3 grid((len + 7) / 8, d.M * 2);
-  const int npl = (d.n + 31) / 32;
-  if (npl <= 2) topk_rows_kernel<2><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
-  else if (npl <= 4) topk_rows_kernel<4><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
-  else if (npl <= 8) topk_rows_kernel<8><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
-  else if (npl <= 16) topk_rows_kernel<16><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
-  else if (npl <= 32) topk_rows_kernel<32><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
-  else if (npl <= 64) topk_rows_kernel<64><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
-  else topk_rows_kernel<128><<<grid, TP_THREADS, 0, s>>>(d, w, wt0, len);
-  return 1;
 }
 
 int launch_tc_address(const Dims& d, const Work& w, float* K1, float* K2, const void* q, long long q_stride, int len,
