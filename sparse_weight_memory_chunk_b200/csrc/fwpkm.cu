@@ -170,10 +170,8 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
   x.Dsv = (float*)take(4 * M * 2 * T * k);
   x.idx = (int32_t*)take(4 * M * T * k);
   x.w = (float*)take(4 * M * T * k);
-  x.pair_tr = (uint32_t*)take(4 * M * nch * C * k);
-  x.seg_start = (int32_t*)take(4 * M * nch * (C * k + 1));
-  x.seg_slot = (int32_t*)take(4 * M * nch * C * k);
-  x.nseg = (int32_t*)take(4 * M * nch);
+  x.sk = (unsigned long long*)take(8 * M * nch * C * k);
+  x.npairs = (int32_t*)take(4 * M * nch);
   x.resid = (float*)take(4 * M * C * dv);
   const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
   x.tc = use_tensor_cores(d) ? 1 : 0;
@@ -189,7 +187,7 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
     x.Z = nullptr; x.lp = nullptr; x.Lt = nullptr;
   }
   x.Kpc = nullptr; x.kn = nullptr; x.qn = nullptr; x.zpart = nullptr; x.ppart = nullptr;
-  x.Wt = nullptr; x.Qt = nullptr; x.wsum_part = nullptr;
+  x.Wt = nullptr; x.Qt = nullptr; x.wsum_part = nullptr; x.qt_T = 0;
   if (x.tc) {
     const size_t P = 2 * M, h = d.h, cpad = (C + 63) / 64 * 64, nt = (n + 127) / 128;
     x.Kpc = (__nv_bfloat16*)take(2 * 3 * P * n * h);
@@ -199,7 +197,8 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
       x.zpart = (float*)take(4 * P * C * nt * 4);
       x.ppart = (float*)take(4 * P * 8 * n);
       x.Wt = (__nv_bfloat16*)take(2 * 3 * P * n * cpad);
-      x.Qt = (__nv_bfloat16*)take(2 * P * h * cpad);
+      x.qt_T = (int)((T > C ? T : C) + 63) / 64 * 64;
+      x.Qt = (__nv_bfloat16*)take(2 * P * h * (size_t)x.qt_T);
       x.wsum_part = (float*)take(4 * P * (cpad / 64) * n);
     }
   }
@@ -336,7 +335,7 @@ fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream
   st->host_error = 0;
   if (d.flags & FWPKM_KEY_UPDATE)
     run(st, KK_ADDR, s, [&] {
-      return st->wk.tc ? launch_tc_address(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, s)
+      return st->wk.tc ? launch_tc_address(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, -1, s)
                        : launch_address(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, s);
     });
   st->pending = 0;
@@ -363,6 +362,9 @@ static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, cons
   const bool la = (d.flags & FWPKM_LOOKAHEAD) != 0;
   const bool tc = st->wk.tc != 0;
   const int nch = (T + C - 1) / C;
+  // the key step reads every chunk's half-queries from one feature-major copy made up front
+  // (its TMA x offset, the chunk start, must be a multiple of 8 tokens)
+  const bool qt_whole = tc && ku && C % 8 == 0;
   cudaStream_t sK = st->sK, sS = st->sS, sV = st->sV;
   st->ev_next = 0;
   auto dep = [&](cudaStream_t from, cudaStream_t to) {
@@ -391,6 +393,7 @@ static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, cons
 
   if (tc) {
     run(st, KK_PREP, sK, [&] { return launch_qnorm(d, st->wk, q, T, 0, T, sK); });
+    if (qt_whole) run(st, KK_PREP, sK, [&] { return launch_qtrans(d, st->wk, q, T, 0, T, sK); });
     run(st, KK_PREP, sK, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, sK); });
   }
   if (!ku) {
@@ -436,7 +439,7 @@ static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, cons
         }
         cudaStreamWaitEvent(sS, mark(sK), 0);
         run(st, KK_ADDR, sK, [&] {
-          return tc ? launch_tc_address(d, wb, st->K1, st->K2, qc, T, len, sK)
+          return tc ? launch_tc_address(d, wb, st->K1, st->K2, qc, T, len, qt_whole ? t0 : -1, sK)
                     : launch_address(d, wb, st->K1, st->K2, qc, T, len, sK);
         });
         if (val_done[c]) cudaStreamWaitEvent(sS, val_done[c], 0);     // previous pass wrote chunk c

@@ -33,10 +33,9 @@ struct Work {
   float* Dsv;        // [M][2][max_T][k]   their squared distances
   int32_t* idx;      // [M][max_T][k]      final slots, rank order
   float* w;          // [M][max_T][k]      softmax weights
-  uint32_t* pair_tr; // [M][max_T*k]       sorted pairs: t_local*k + r, per chunk region of C*k
-  int32_t* seg_start;// [M][max_chunks][C*k + 1]
-  int32_t* seg_slot; // [M][max_chunks][C*k]
-  int32_t* nseg;     // [M][max_chunks]
+  unsigned long long* sk; // [M][max_chunks][C*k] read pairs (slot << 32 | t_local*k + r), each
+                          // slot's pairs contiguous and in token order
+  int32_t* npairs;   // [M][max_chunks]    pairs in the chunk's list
   float* resid;      // [M][C][dv]         vhat, then r_t = g_t (vhat_t - tau_t)
   float* Dfull;      // [M][2][C][n]       key update: all sub-key distances of the chunk
   float* Z;          // [M][2][C]          key update: sum_a 1/(eps + D)
@@ -52,7 +51,8 @@ struct Work {
   float* zpart;      // [M*2][C][n/128][4] per-32-column partial sums of 1/(eps + D)
   float* ppart;      // [M*2][8][n]        partial column sums for pbar
   __nv_bfloat16* Wt; // [3][M*2][n][Cpad]  key-step weights, sub-key major, bf16 pieces
-  __nv_bfloat16* Qt; // [M*2][h][Cpad]     chunk half-queries, feature major
+  __nv_bfloat16* Qt; // [M*2][h][qt_T]     half-queries, feature major (operand B of the key step)
+  int qt_T;          // token columns of Qt (a multiple of 64)
   float* wsum_part;  // [M*2][Cpad/64][n]  per-token-tile sums of W
 };
 
@@ -60,11 +60,11 @@ enum : int { TC_EPI_DIST = 0, TC_EPI_KEYSTEP = 1 };
 
 // One batched tensor-core contraction (see tc_gemm.cu).  Problem p (blockIdx.z) owns
 // A tiles at (x = (p % a_div) * a_xoff + 64 kb, y = a_y0 + 128 mt, z = p / a_div + pa * a_zpiece)
-// and B tiles at (x = 64 kb, y = 128 nt, z = p + pb * b_zpiece).
+// and B tiles at (x = b_x0 + 64 kb, y = 128 nt, z = p + pb * b_zpiece).
 struct TcGemm {
   int P, k_blocks, n_tiles, tiles_per_cta;
   int a_pieces, b_pieces;
-  int a_div, a_xoff, a_y0, a_zpiece, b_zpiece;
+  int a_div, a_xoff, a_y0, a_zpiece, b_zpiece, b_x0;
   int m_valid, n_valid;
   int epi;
   // TC_EPI_DIST
@@ -128,9 +128,13 @@ int launch_tc_score(const Dims& d, const Work& w, const void* q_base, long long 
                     int wt0, int len, bool key_update, cudaStream_t s);
 // Per-half top-k from Dfull rows 0..len-1 into A/Dsv at workspace tokens wt0..
 int launch_topk_rows(const Dims& d, const Work& w, int wt0, int len, cudaStream_t s);
-// Entropy key step from Dfull/zpart (tensor-core path).
+// Feature-major copy of both half-queries of `len` tokens into Qt columns qt0.. (the key
+// step's B operand).
+int launch_qtrans(const Dims& d, const Work& w, const void* q, long long q_stride, int qt0, int len, cudaStream_t s);
+// Entropy key step from Dfull/zpart (tensor-core path).  The chunk's half-queries are read
+// from Qt columns qt_t0..; qt_t0 < 0: transpose them first into columns 0.. .
 int launch_tc_address(const Dims& d, const Work& w, float* K1, float* K2, const void* q, long long q_stride, int len,
-                      cudaStream_t s);
+                      int qt_t0, cudaStream_t s);
 
 // ---- small device helpers ----
 __device__ __forceinline__ float load_qv(const float* p, long long i) { return p[i]; }

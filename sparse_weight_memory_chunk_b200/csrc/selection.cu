@@ -117,22 +117,25 @@ int launch_cartesian(const Dims& d, const Work& w, int wt0, int len, int32_t* id
 }
 
 // ---------------------------------------------------------------------------
-// Per-chunk sort of the (slot, token) read pairs: one CTA per (memory, chunk).
+// Per-chunk sort of the (slot, token) read pairs.
 //
-// Keys are (slot << 32) | (t_local * k + r); ascending order groups each slot's
-// readers in token order, which is the summation order of the write.  Segment
-// boundaries give N_read,i (paperlayer §3.3 read-count consensus).
+// Keys are (slot << 32) | (t_local * k + r).  The write needs every slot's readers
+// contiguous and in token order (its summation order); segment boundaries then give
+// N_read,i (paperlayer §3.3 read-count consensus).  A global slot order is not needed,
+// so keys are bucketed by a multiplicative hash of the slot (~64 keys per bucket; a slot
+// falls in exactly one bucket), laid out bucket after bucket, and ordered inside each
+// bucket by their full key.
 //
-// The write needs each slot's readers contiguous and in token order, not a global slot
-// order.  So keys are bucketed by a multiplicative hash of the slot (~64 keys per
-// bucket; a slot falls in exactly one bucket) and each warp ranks the keys of its
-// buckets by comparing every key with every other key of the bucket, writing each to
-// its rank.  The scatter into buckets may land keys in any order, but ranking by the
-// full unique key makes the result independent of it.  If a bucket is larger than 128
-// keys (strongly skewed slot use) the CTA sorts all keys with a register bitonic
-// network instead.
+// SORT_SPLIT CTAs share one (memory, chunk): each counts all buckets (so all agree on
+// the bucket offsets), keeps the keys of its own quarter of the buckets in shared
+// memory, and one warp per bucket ranks each key by comparing it with every other key
+// of the bucket and stores it at its rank.  The scatter into buckets may land keys in
+// any order; ranking by the full unique key makes the output independent of it.  If a
+// bucket holds more than 128 keys (strongly skewed slot use), the first CTA sorts all
+// keys with a register bitonic network instead and the others do nothing.
 // ---------------------------------------------------------------------------
 constexpr int SORT_THREADS = 1024;
+constexpr int SORT_SPLIT = 4;
 constexpr int SORT_BUCKET_KEYS = 64;   // average keys per bucket
 constexpr int SORT_BUCKET_CAP = 128;   // largest bucket the ranking path handles
 
@@ -141,10 +144,9 @@ __global__ void __launch_bounds__(SORT_THREADS)
 sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) {
   extern __shared__ u64 s_keys[];
   __shared__ int s_cnt[512], s_off[513], s_cur[512];
-  __shared__ int s_warp[SORT_THREADS / 32];
-  __shared__ int s_base, s_max;
+  __shared__ int s_max;
   const int m = blockIdx.y;
-  const int cc = blockIdx.x;
+  const int cc = blockIdx.x / SORT_SPLIT, part = blockIdx.x % SORT_SPLIT;
   const int C = dm.C, k = dm.k;
   const int tc0 = cc * C;  // relative to wt0
   const int clen = min(C, total_len - tc0);
@@ -153,10 +155,12 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
   const int P = npair * k;
   int Ppad = 32 * VPT;
   while (Ppad < P) Ppad <<= 1;
-  const int NB = Ppad / SORT_BUCKET_KEYS;  // <= 512, a power of two
+  const int NB = Ppad / SORT_BUCKET_KEYS;  // a power of two, <= 512
   const int nb_log2 = 31 - __clz(NB);
+  const int b_lo = part * NB / SORT_SPLIT, b_hi = (part + 1) * NB / SORT_SPLIT;
   const int cslot = (wt0 + tc0) / C;
   const size_t cbase = (size_t)m * w.max_chunks + cslot;
+  u64* out = w.sk + cbase * (size_t)(C * k);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   for (int b = tid; b < NB; b += SORT_THREADS) s_cnt[b] = 0;
@@ -172,7 +176,7 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
       const int t_local = i / k, r = i - t_local * k;
       const unsigned slot = (unsigned)w.idx[((size_t)m * w.max_T + wt0 + tc0 + t_local) * k + r];
       key = ((u64)slot << 32) | (unsigned)i;
-      bk[u] = (int)((slot * 2654435761u) >> (32 - nb_log2));  // multiplicative hash
+      bk[u] = NB > 1 ? (int)((slot * 2654435761u) >> (32 - nb_log2)) : 0;  // multiplicative hash
       atomicAdd(&s_cnt[bk[u]], 1);
     }
     x[u] = key;
@@ -202,13 +206,16 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
     }
   }
   __syncthreads();
+  if (part == 0 && tid == 0) w.npairs[cbase] = P;
   if (s_max <= SORT_BUCKET_CAP) {
+    // this CTA's buckets [b_lo, b_hi) occupy key positions [s_off[b_lo], s_off[b_hi])
+    const int base0 = s_off[b_lo];
 #pragma unroll
     for (int u = 0; u < VPT; ++u)
-      if (bk[u] >= 0) s_keys[atomicAdd(&s_cur[bk[u]], 1)] = x[u];
+      if (bk[u] >= b_lo && bk[u] < b_hi) s_keys[atomicAdd(&s_cur[bk[u]], 1) - base0] = x[u];
     __syncthreads();
-    for (int b = warp; b < NB; b += SORT_THREADS / 32) {
-      const int base = s_off[b], cnt = s_off[b + 1] - base;
+    for (int b = b_lo + warp; b < b_hi; b += SORT_THREADS / 32) {
+      const int base = s_off[b] - base0, cnt = s_off[b + 1] - s_off[b];
       if (cnt == 0) continue;
       u64 mine[SORT_BUCKET_CAP / 32];
       int rk[SORT_BUCKET_CAP / 32];
@@ -218,66 +225,32 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
         mine[j] = i < cnt ? s_keys[base + i] : ~0ull;
         rk[j] = 0;
       }
-      for (int t = 0; t < cnt; ++t) {
-        const u64 o = s_keys[base + t];
+      if (cnt <= 64) {
+        for (int t = 0; t < cnt; ++t) {
+          const u64 o = s_keys[base + t];
+          rk[0] += o < mine[0] ? 1 : 0;
+          rk[1] += o < mine[1] ? 1 : 0;
+        }
+      } else {
+        for (int t = 0; t < cnt; ++t) {
+          const u64 o = s_keys[base + t];
 #pragma unroll
-        for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j) rk[j] += o < mine[j] ? 1 : 0;
+          for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j) rk[j] += o < mine[j] ? 1 : 0;
+        }
       }
-      __syncwarp();
 #pragma unroll
       for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j)
-        if (lane + 32 * j < cnt) s_keys[base + rk[j]] = mine[j];
-      __syncwarp();
+        if (lane + 32 * j < cnt) out[s_off[b] + rk[j]] = mine[j];
     }
-  } else {
+  } else if (part == 0) {
     block_sort_asc<VPT>(x, s_keys, Ppad);
     if (tid * VPT < Ppad)
 #pragma unroll
-      for (int u = 0; u < VPT; ++u) s_keys[tid * VPT + u] = x[u];
-  }
-  __syncthreads();
-
-  // segments: compaction of the positions where the slot changes
-  uint32_t* pair_tr = w.pair_tr + (size_t)m * w.max_chunks * C * k + (size_t)cslot * C * k;
-  int32_t* seg_start = w.seg_start + cbase * (C * k + 1);
-  int32_t* seg_slot = w.seg_slot + cbase * (C * k);
-  if (tid == 0) s_base = 0;
-  __syncthreads();
-  for (int i0 = 0; i0 < P; i0 += SORT_THREADS) {
-    const int i = i0 + tid;
-    bool head = false;
-    u64 key = 0;
-    if (i < P) {
-      key = s_keys[i];
-      pair_tr[i] = (uint32_t)(key & 0xffffffffu);
-      head = (i == 0) || ((s_keys[i - 1] >> 32) != (key >> 32));
-    }
-    const unsigned bal = __ballot_sync(0xffffffffu, head);
-    if (lane == 0) s_warp[warp] = __popc(bal);
-    __syncthreads();
-    if (warp == 0) {
-      const int v = s_warp[lane];
-      int incl = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      s_warp[lane] = incl - v;  // exclusive
-    }
-    __syncthreads();
-    if (head) {
-      const int pos = s_base + s_warp[warp] + __popc(bal & ((1u << lane) - 1u));
-      seg_start[pos] = i;
-      seg_slot[pos] = (int32_t)(key >> 32);
-    }
-    __syncthreads();
-    if (tid == SORT_THREADS - 1) s_base += s_warp[SORT_THREADS / 32 - 1] + __popc(bal);
-    __syncthreads();
-  }
-  if (tid == 0) {
-    seg_start[s_base] = P;
-    w.nseg[cbase] = s_base;
+      for (int u = 0; u < VPT; ++u)
+        if (tid * VPT + u < P) out[tid * VPT + u] = x[u];
+  } else {
+    // the skewed fallback is handled by the first CTA; nothing to do here (the bitonic
+    // sort needs every thread of its CTA, so it is taken as a whole or not at all)
   }
 }
 
@@ -286,7 +259,7 @@ int launch_sort_pairs(const Dims& d, const Work& w, int wt0, int total_len, bool
   if (total_len <= 0) return 0;
   const int nchunks = (total_len + d.C - 1) / d.C;
   const int P = d.C * d.k;
-  dim3 grid(nchunks, d.M);
+  dim3 grid(nchunks * SORT_SPLIT, d.M);
   if (P <= 8 * SORT_THREADS) {
     int Ppad = 256;
     while (Ppad < P) Ppad <<= 1;

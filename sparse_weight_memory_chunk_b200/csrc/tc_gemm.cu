@@ -121,7 +121,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           tma_load_3d(st + pa * TC_TILE_BYTES, &tmA, &full[s], a_x0 + kb * TC_BK, g.a_y0 + mt * TC_BM,
                       a_z + pa * g.a_zpiece);
         for (int pb = 0; pb < g.b_pieces; ++pb)
-          tma_load_3d(st + (g.a_pieces + pb) * TC_TILE_BYTES, &tmB, &full[s], kb * TC_BK, nt * TC_BN,
+          tma_load_3d(st + (g.a_pieces + pb) * TC_TILE_BYTES, &tmB, &full[s], g.b_x0 + kb * TC_BK, nt * TC_BN,
                       p + pb * g.b_zpiece);
         ++issued;
       }

@@ -126,16 +126,14 @@ tc_rowL_kernel(Dims dm, Work w, int len) {
 }
 
 // W for a 64-token x 64-sub-key tile, written sub-key major as three bf16 pieces (the
-// A operand of the key-step GEMM), plus the tile's per-sub-key sum of W.  CTAs of the
-// first sub-key tile also write their tokens' half-queries feature major (operand B).
+// A operand of the key-step GEMM), plus the tile's per-sub-key sum of W.
 __global__ void __launch_bounds__(TP_THREADS)
-tc_wbuild_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long q_stride, int len, int cpad) {
+tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
   __shared__ float s_W[64][65];
   __shared__ float s_invz[64], s_L[64], s_lp[64];
-  __shared__ __nv_bfloat16 s_q[64][136];
-  const int p = blockIdx.z, m = p >> 1, j = p & 1;
+  const int p = blockIdx.z;
   const int b0 = blockIdx.x * 64, t0 = blockIdx.y * 64;
-  const int n = dm.n, h = dm.h, P = dm.M * 2;
+  const int n = dm.n, P = dm.M * 2;
   const int tid = threadIdx.x;
   if (tid < 64) {
     const int t = t0 + tid;
@@ -180,21 +178,31 @@ tc_wbuild_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long
     *reinterpret_cast<uint4*>(dst + pstride) = *reinterpret_cast<uint4*>(mid);
     *reinterpret_cast<uint4*>(dst + 2 * pstride) = *reinterpret_cast<uint4*>(lo);
   }
-  if (blockIdx.x == 0) {
-    // transpose this token tile's half-queries: Qt[p][e][t]
-    for (int idx = tid; idx < 64 * h; idx += TP_THREADS) {
-      const int tl = idx / h, e = idx - tl * h;
-      const int t = t0 + tl;
-      s_q[tl][e] = t < len ? q[((long long)m * q_stride + t) * dm.d + (long long)j * h + e] : __float2bfloat16(0.f);
-    }
-    __syncthreads();
-    for (int idx = tid; idx < h * 8; idx += TP_THREADS) {
-      const int e = idx >> 3, c8 = idx & 7;
-      __align__(16) __nv_bfloat16 v8[8];
+}
+
+// Feature-major copy of the half-queries of `len` tokens: Qt[p][e][qt0 + t].  One CTA
+// per (64-token tile, problem); 16-byte loads and stores through a shared-memory tile.
+// Token columns past `len` in the last tile are written as zeros (finite values, since the
+// key-step GEMM multiplies them by zero-filled weights).
+__global__ void __launch_bounds__(TP_THREADS)
+qtrans_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long q_stride, int qt0, int len) {
+  __shared__ __align__(16) __nv_bfloat16 s_q[64][128 + 8];
+  const int p = blockIdx.y, m = p >> 1, j = p & 1;
+  const int t0 = blockIdx.x * 64, h = dm.h, h8 = h / 8;
+  for (int idx = threadIdx.x; idx < 64 * h8; idx += TP_THREADS) {
+    const int tl = idx / h8, e8 = idx - tl * h8;
+    const int t = t0 + tl;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (t < len) val = *reinterpret_cast<const uint4*>(q + ((long long)m * q_stride + t) * dm.d + (long long)j * h + e8 * 8);
+    *reinterpret_cast<uint4*>(&s_q[tl][e8 * 8]) = val;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < h * 8; idx += TP_THREADS) {
+    const int e = idx >> 3, c8 = idx & 7;
+    __align__(16) __nv_bfloat16 v8[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v8[u] = s_q[c8 * 8 + u][e];
-      *reinterpret_cast<uint4*>(w.Qt + ((size_t)p * h + e) * cpad + t0 + c8 * 8) = *reinterpret_cast<uint4*>(v8);
-    }
+    for (int u = 0; u < 8; ++u) v8[u] = s_q[c8 * 8 + u][e];
+    *reinterpret_cast<uint4*>(w.Qt + ((size_t)p * h + e) * w.qt_T + qt0 + t0 + c8 * 8) = *reinterpret_cast<uint4*>(v8);
   }
 }
 
@@ -238,33 +246,46 @@ int launch_tc_score(const Dims& d, const Work& w, const void* q_base, long long 
   return launch_tc_gemm(A, B, g, (len + 127) / 128, s);
 }
 
+int launch_qtrans(const Dims& d, const Work& w, const void* q, long long q_stride, int qt0, int len, cudaStream_t s) {
+  if (len <= 0) return 0;
+  qtrans_kernel<<<dim3((len + 63) / 64, d.M * 2), TP_THREADS, 0, s>>>(d, w, (const __nv_bfloat16*)q, q_stride, qt0,
+                                                                       len);
+  return 1;
+}
+
 int launch_tc_address(const Dims& d, const Work& w, float* K1, float* K2, const void* q, long long q_stride, int len,
-                      cudaStream_t s) {
+                      int qt_t0, cudaStream_t s) {
   if (len <= 0) return 0;
   const int P = d.M * 2;
   const int cpad = (d.C + 63) / 64 * 64;
   const int ntt = (len + 63) / 64;
+  int launched = 5;
+  if (qt_t0 < 0) {
+    launch_qtrans(d, w, q, q_stride, 0, len, s);
+    qt_t0 = 0;
+    ++launched;
+  }
   tc_pbar_kernel<<<dim3((d.n + TP_THREADS - 1) / TP_THREADS, P, PBAR_SLICES), TP_THREADS, 0, s>>>(d, w, len);
   tc_lp_kernel<<<(unsigned)(((long long)P * d.n + TP_THREADS - 1) / TP_THREADS), TP_THREADS, 0, s>>>(d, w, len);
   tc_rowL_kernel<<<dim3((len + 7) / 8, P), TP_THREADS, 0, s>>>(d, w, len);
-  tc_wbuild_kernel<<<dim3((d.n + 63) / 64, ntt, P), TP_THREADS, 0, s>>>(d, w, (const __nv_bfloat16*)q, q_stride, len,
-                                                                         cpad);
+  tc_wbuild_kernel<<<dim3((d.n + 63) / 64, ntt, P), TP_THREADS, 0, s>>>(d, w, len, cpad);
   CUtensorMap A, B;
   if (!make_tmap_bf16_3d(&A, w.Wt, len, d.n, 3 * P, (uint64_t)cpad * 2, (uint64_t)d.n * cpad * 2)) return -1;
-  if (!make_tmap_bf16_3d(&B, w.Qt, len, d.h, P, (uint64_t)cpad * 2, (uint64_t)d.h * cpad * 2)) return -1;
+  if (!make_tmap_bf16_3d(&B, w.Qt, w.qt_T, d.h, P, (uint64_t)w.qt_T * 2, (uint64_t)d.h * w.qt_T * 2)) return -1;
   TcGemm g = {};
   g.P = P;
   g.k_blocks = ntt;
   g.n_tiles = 1;
   g.tiles_per_cta = 1;
   g.a_pieces = 3; g.b_pieces = 1;
-  g.a_div = 1; g.a_xoff = 0; g.a_y0 = 0; g.a_zpiece = P; g.b_zpiece = 0;
+  g.a_div = 1; g.a_xoff = 0; g.a_y0 = 0; g.a_zpiece = P; g.b_zpiece = 0; g.b_x0 = qt_t0;
   g.m_valid = d.n; g.n_valid = d.h;
   g.epi = TC_EPI_KEYSTEP;
   g.K1 = K1; g.K2 = K2; g.Kpc = w.Kpc; g.kn = w.kn;
   g.wsum_part = w.wsum_part; g.wsum_tiles = ntt; g.lr = d.lr_key;
   g.status = w.status;
-  return 4 + launch_tc_gemm(A, B, g, (d.n + 127) / 128, s);
+  launch_tc_gemm(A, B, g, (d.n + 127) / 128, s);
+  return launched;
 }
 
 }  // namespace fwpkm

@@ -187,11 +187,14 @@ resid_kernel(Dims dm, Work w, const VT* __restrict__ v, const float* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// Write: each warp owns G touched rows (segments of the sorted pair list).  It loads the
-// G segment descriptors with one coalesced load, issues all G value-row loads and the
-// first pair of every segment before consuming any of them, then for each row sums
-// G_i = sum s'_{t,i} r_t in token order and stores V_i - G_i / N_read,i.  Rows are
-// disjoint, so there are no atomics and the result does not depend on scheduling.
+// Write: the chunk's read pairs are sorted so that each touched row's pairs are
+// contiguous and in token order.  Each warp owns G consecutive list positions; a
+// position whose slot differs from its predecessor's starts a segment (one touched row)
+// and that segment belongs to the warp, even where it runs past the warp's positions.
+// The warp issues the value-row loads of all its segments before consuming any, then for
+// each row sums G_i = sum s'_{t,i} r_t in token order and stores V_i - G_i / N_read,i.
+// Rows are disjoint, so there are no atomics and the result does not depend on
+// scheduling.
 // ---------------------------------------------------------------------------
 template <int VPL, int G>
 __global__ void __launch_bounds__(VAL_WARPS * 32)
@@ -201,26 +204,25 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
   const int C = dm.C, k = dm.k, dv4 = dm.dv >> 2;
   const int cslot = wt0 / C;
   const size_t cbase = (size_t)m * w.max_chunks + cslot;
-  const int ns = w.nseg[cbase];
-  const int u0 = (blockIdx.x * VAL_WARPS + warp) * G;
-  if (u0 >= ns) return;
-  const int32_t* seg_start = w.seg_start + cbase * (C * k + 1);
-  const int32_t* seg_slot = w.seg_slot + cbase * (C * k);
-  const uint32_t* pair_tr = w.pair_tr + (size_t)m * w.max_chunks * C * k + (size_t)cslot * C * k;
-  int my_slot = -1, my_s0 = 0, my_s1 = 0;
-  uint32_t my_tr = 0;
-  if (lane < G && u0 + lane < ns) {
-    my_slot = seg_slot[u0 + lane];
-    my_s0 = seg_start[u0 + lane];
-    my_s1 = seg_start[u0 + lane + 1];
-    my_tr = pair_tr[my_s0];
+  const int P = w.npairs[cbase];
+  const int pos0 = (blockIdx.x * VAL_WARPS + warp) * G;
+  if (pos0 >= P) return;
+  const unsigned long long* sk = w.sk + cbase * (size_t)(C * k);
+  unsigned long long my_key = ~0ull;
+  bool head = false;
+  if (lane < G && pos0 + lane < P) {
+    const int pos = pos0 + lane;
+    my_key = sk[pos];
+    head = pos == 0 || (sk[pos - 1] >> 32) != (my_key >> 32);
   }
+  const unsigned heads = __ballot_sync(0xffffffffu, head);
+  const int my_slot = (int)(my_key >> 32);
   float* Vm = V + (size_t)m * dm.N * dm.dv;
   float4 Vr[G][VPL];
 #pragma unroll
   for (int gi = 0; gi < G; ++gi) {
     const int slot = __shfl_sync(0xffffffffu, my_slot, gi);
-    const bool ok = slot >= 0 && (long long)slot < dm.N;
+    const bool ok = ((heads >> gi) & 1u) && slot >= 0 && (long long)slot < dm.N;
     const float4* row = reinterpret_cast<const float4*>(Vm + (size_t)(ok ? slot : 0) * dm.dv);
 #pragma unroll
     for (int c = 0; c < VPL; ++c) {
@@ -230,11 +232,9 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
   }
 #pragma unroll
   for (int gi = 0; gi < G; ++gi) {
-    const int slot = __shfl_sync(0xffffffffu, my_slot, gi);
-    const int s0 = __shfl_sync(0xffffffffu, my_s0, gi);
-    const int s1 = __shfl_sync(0xffffffffu, my_s1, gi);
-    const uint32_t tr0 = __shfl_sync(0xffffffffu, my_tr, gi);
-    if (u0 + gi >= ns) break;
+    const unsigned long long key0 = __shfl_sync(0xffffffffu, my_key, gi);
+    if (!((heads >> gi) & 1u)) continue;
+    const int slot = (int)(key0 >> 32);
     if (slot < 0 || (long long)slot >= dm.N) {
       if (lane == 0) atomicExch(w.status, DEV_BAD_SLOT);
       continue;
@@ -242,8 +242,10 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
     float4 Gs[VPL];
 #pragma unroll
     for (int c = 0; c < VPL; ++c) Gs[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p = s0; p < s1; ++p) {
-      const uint32_t tr = p == s0 ? tr0 : pair_tr[p];
+    int p = pos0 + gi;
+    unsigned long long key = key0;
+    for (;;) {
+      const uint32_t tr = (uint32_t)(key & 0xffffffffu);
       const int t_local = (int)(tr / (uint32_t)k), r = (int)(tr - (uint32_t)t_local * k);
       const float wt = w.w[((size_t)m * w.max_T + wt0 + t_local) * k + r];
       const float4* rrow = reinterpret_cast<const float4*>(w.resid + ((size_t)m * C + t_local) * dm.dv);
@@ -256,8 +258,11 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
           Gs[c].z = fmaf(wt, x.z, Gs[c].z); Gs[c].w = fmaf(wt, x.w, Gs[c].w);
         }
       }
+      if (++p >= P) break;
+      key = sk[p];
+      if ((int)(key >> 32) != slot) break;
     }
-    const float nr = (float)(s1 - s0);
+    const float nr = (float)(p - (pos0 + gi));
     float4* row = reinterpret_cast<float4*>(Vm + (size_t)slot * dm.dv);
 #pragma unroll
     for (int c = 0; c < VPL; ++c) {
@@ -317,7 +322,7 @@ int launch_resid(const Dims& d, const Work& w, const void* v, const float* g, lo
 
 int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s) {
   const int vpl = vpl_of(d.dv);
-  const int G = vpl <= 2 ? 4 : vpl == 4 ? 2 : 1;  // rows per warp: ~8 float4 in flight per lane
+  const int G = vpl <= 2 ? 4 : vpl == 4 ? 2 : 1;  // list positions per warp: ~8 float4 in flight per lane
   dim3 grid((d.C * d.k + VAL_WARPS * G - 1) / (VAL_WARPS * G), d.M);
   switch (vpl) {
     case 1: write_kernel<1, 4><<<grid, VAL_WARPS * 32, 0, s>>>(d, w, V, wt0); break;
