@@ -50,6 +50,7 @@ struct fwpkm_state {
   std::vector<cudaEvent_t> sync_ev;
   size_t ev_next;
   int no_graph;
+  int serial;  // diagnostics: all three chains on one stream (per-kernel timing without overlap)
   cudaGraphExec_t graph_exec;
   SeqKey graph_key;
   uint64_t graph_kernels;
@@ -259,6 +260,8 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
   {
     const char* e = getenv("FWPKM_NO_GRAPH");
     st->no_graph = (e && e[0] == '1') ? 1 : 0;
+    const char* sv = getenv("FWPKM_SERIAL");
+    st->serial = (sv && sv[0] == '1') ? 1 : 0;
   }
   if (cudaStreamCreateWithFlags(&st->sK, cudaStreamNonBlocking) != cudaSuccess ||
       cudaStreamCreateWithFlags(&st->sS, cudaStreamNonBlocking) != cudaSuccess ||
@@ -365,7 +368,7 @@ static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, cons
   // the key step reads every chunk's half-queries from one feature-major copy made up front
   // (its TMA x offset, the chunk start, must be a multiple of 8 tokens)
   const bool qt_whole = tc && ku && C % 8 == 0;
-  cudaStream_t sK = st->sK, sS = st->sS, sV = st->sV;
+  cudaStream_t sK = st->sK, sS = st->serial ? st->sK : st->sS, sV = st->serial ? st->sK : st->sV;
   st->ev_next = 0;
   auto dep = [&](cudaStream_t from, cudaStream_t to) {
     cudaEvent_t e = next_event(st);

@@ -31,7 +31,8 @@ using namespace sm100;
 
 constexpr int TC_BM = 128, TC_BN = 128, TC_BK = 64;
 constexpr int TC_TILE_BYTES = TC_BM * TC_BK * 2;  // 16 KiB, also the B tile (TC_BN == TC_BM)
-constexpr int TC_STAGES = 3;
+// two stages (<= 128 KiB of tiles) leave room on the SM for the CTAs of the other chains
+constexpr int TC_STAGES = 2;
 constexpr int TC_EPI_WARPS = 16;
 constexpr int TC_THREADS = (2 + TC_EPI_WARPS) * 32;
 constexpr uint32_t TC_TMEM_COLS = 256;
