@@ -154,6 +154,78 @@ fwpkm_status fwpkm_chunk_step_noalloc(const fwpkm_config* cfg, float* K1, float*
                                       const void* q, const void* v, const float* g, const void* v_next,
                                       int c_len, int seq_stride, float* o, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Slow-weight projections around the memory ("快速权重积键值记忆 Fast-weight Product
+ * Key Memory" (rainbus summary), method steps 1 and 3):
+ *   q_t = Linear_q(RMSNorm_q(h_t)), v_t = Linear_v(RMSNorm_v(h_t)),
+ *   g_t = sigmoid(Linear_g(RMSNorm_g(h_t))), o'_t = Linear_o(RMSNorm_o(o_t)),
+ * with RMSNorm(x) = x / sqrt(mean(x^2) + eps_rms) * gamma and Linear(x) = x W^T + b.
+ * The rows (tokens) of h, q, v, g, o and o' are [rows][width] row-major; with one
+ * head per sequence the memory index is the sequence, so q, v, g and o are exactly
+ * the [M][T][width] inputs and output of the memory calls above.
+ * Precision: h and the weights W are bf16; the norm weights, biases, g and o fp32;
+ * q and v fp32 or bf16 (fwpkm_layer_config.qv_dtype); o' bf16.  gamma is folded into W in fp32 and held as two bf16 pieces (one
+ * when gamma is NULL); o enters the output GEMM as two bf16 pieces; accumulation is
+ * fp32 on the tensor cores and 1/rms scales the accumulator.
+ * ------------------------------------------------------------------------- */
+typedef struct fwpkm_layer fwpkm_layer;  /* opaque host handle */
+
+/* Supported limits (else FWPKM_ERR_UNSUPPORTED): d_model % 64 == 0 with
+ * 64 <= d_model <= 16384; d % 32 == 0, d_v % 64 == 0, 32 <= d, d_v <= 1024;
+ * max_rows >= 1. */
+typedef struct {
+  int d_model;   /* width of h and o'                                   */
+  int d;         /* query width                                         */
+  int d_v;       /* value width                                         */
+  int max_rows;  /* most rows (tokens) of one layer_in / layer_out call */
+  float eps_rms; /* RMSNorm epsilon                                     */
+  int qv_dtype;  /* fwpkm_dtype of the q and v that fwpkm_layer_in writes */
+} fwpkm_layer_config;
+
+/* Parameters (device pointers, read only during fwpkm_layer_set_params).  W_* are
+ * bf16 [out][in]: W_q [d][d_model], W_v [d_v][d_model], w_g [d_model],
+ * W_o [d_model][d_v].  gamma_* are fp32 [in] (NULL = ones); b_* fp32 [out]
+ * (NULL = zeros); b_g is the gate's scalar bias. */
+typedef struct {
+  const void* W_q; const float* gamma_q; const float* b_q;
+  const void* W_v; const float* gamma_v; const float* b_v;
+  const void* w_g; const float* gamma_g; float b_g;
+  const void* W_o; const float* gamma_o; const float* b_o;
+} fwpkm_layer_params;
+
+/* Bytes of device workspace (folded weights, biases and the output call's per-row
+ * scratch) for `cfg`.  The workspace must be 256-byte aligned. */
+fwpkm_status fwpkm_layer_workspace_size(const fwpkm_layer_config* cfg, size_t* bytes);
+
+/* Create a handle over the caller's workspace.  Nothing is enqueued. */
+fwpkm_status fwpkm_layer_init(const fwpkm_layer_config* cfg, void* workspace, size_t ws_bytes,
+                              fwpkm_layer** out);
+
+/* Fold the norm weights into the linear weights (fp32 product, split into bf16
+ * pieces) and copy the biases into the workspace.  Enqueued on `stream`; the
+ * parameters may be freed once the stream has passed this point. */
+fwpkm_status fwpkm_layer_set_params(fwpkm_layer* L, const fwpkm_layer_params* p, void* stream);
+
+/* Method step 1 for rows <= max_rows tokens: h bf16 [rows][d_model] (16-byte
+ * aligned) -> q [rows][d], v [rows][d_v] (cfg.qv_dtype: fp32, or bf16 rounded to
+ * nearest from the fp32 result; 16-byte aligned) and g fp32 [rows].  rows == 0 is a no-op.  One row-statistics kernel (1/rms and the gate)
+ * and one tensor-core GEMM with both outputs in its epilogue.  Uses the workspace's
+ * per-row scratch, so calls on one handle must not overlap on the GPU. */
+fwpkm_status fwpkm_layer_in(fwpkm_layer* L, const void* h, int rows, void* q, void* v, float* g,
+                            void* stream);
+
+/* Method step 3, output side, for rows <= max_rows tokens: o fp32 [rows][d_v] ->
+ * o' bf16 [rows][d_model] (both 16-byte aligned).  Uses the workspace's per-row
+ * scratch, so calls on one handle must not overlap on the GPU. */
+fwpkm_status fwpkm_layer_out(fwpkm_layer* L, const float* o, int rows, void* o_out, void* stream);
+
+/* Wait for `stream` and return the handle's latched device status (a GEMM wait
+ * that timed out gives FWPKM_ERR_TIMEOUT), clearing it. */
+fwpkm_status fwpkm_layer_sync(fwpkm_layer* L, void* stream);
+
+/* Release the handle (the workspace is the caller's). */
+void fwpkm_layer_destroy(fwpkm_layer* L);
+
 /* Copy the slot indices and softmax weights that the most recent call computed for
  * tokens [0, T) of every memory (final pass of fwpkm_run_sequence, or the chunk of
  * fwpkm_forward_chunk with T <= c_len) into idx_out [M][T][k] int32 and

@@ -46,7 +46,11 @@ struct fwpkm_state {
   int ev_used;
   int host_error;  // a launch could not be set up (e.g. tensor map encoding failed)
   // run_sequence schedule: internal streams, dependency events and the cached graph
-  cudaStream_t sK, sS, sV, sCap;
+  // Memories are split into `groups` contiguous groups; each group runs its own three
+  // chains, so one group's latency-bound kernels overlap another's.
+  static constexpr int MAX_GROUPS = 8;
+  int groups;
+  cudaStream_t sK[MAX_GROUPS], sS[MAX_GROUPS], sV[MAX_GROUPS], sCap;
   std::vector<cudaEvent_t> sync_ev;
   size_t ev_next;
   int no_graph;
@@ -203,8 +207,36 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
       x.wsum_part = (float*)take(4 * P * (cpad / 64) * n);
     }
   }
+  x.P_all = (int)(2 * M);
+  x.dfull_buf = (long long)(M * 2 * (size_t)x.drows * n);
   if (w) *w = x;
   return off;
+}
+
+Work group_work(const Dims& d, const Work& w, int m0) {
+  Work x = w;
+  const size_t M0 = m0, T = w.max_T, k = d.k, C = d.C, n = d.n, h = d.h, dv = d.dv, nch = w.max_chunks;
+  const size_t cpad = (C + 63) / 64 * 64, nt = (n + 127) / 128;
+  x.A += M0 * 2 * T * k;
+  x.Dsv += M0 * 2 * T * k;
+  x.idx += M0 * T * k;
+  x.w += M0 * T * k;
+  x.sk += M0 * nch * C * k;
+  x.npairs += M0 * nch;
+  x.resid += M0 * C * dv;
+  if (x.Dfull) x.Dfull += M0 * 2 * (size_t)w.drows * n;
+  if (x.Z) x.Z += M0 * 2 * C;
+  if (x.lp) x.lp += M0 * 2 * n;
+  if (x.Lt) x.Lt += M0 * 2 * C;
+  if (x.Kpc) x.Kpc += M0 * 2 * n * h;
+  if (x.kn) x.kn += M0 * 2 * n;
+  if (x.qn) x.qn += M0 * 2 * T;
+  if (x.zpart) x.zpart += M0 * 2 * C * nt * 4;
+  if (x.ppart) x.ppart += M0 * 2 * 8 * n;
+  if (x.Wt) x.Wt += M0 * 2 * n * cpad;
+  if (x.Qt) x.Qt += M0 * 2 * h * (size_t)w.qt_T;
+  if (x.wsum_part) x.wsum_part += M0 * 2 * (cpad / 64) * n;
+  return x;
 }
 
 }  // namespace fwpkm
@@ -263,11 +295,25 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
     const char* sv = getenv("FWPKM_SERIAL");
     st->serial = (sv && sv[0] == '1') ? 1 : 0;
   }
-  if (cudaStreamCreateWithFlags(&st->sK, cudaStreamNonBlocking) != cudaSuccess ||
-      cudaStreamCreateWithFlags(&st->sS, cudaStreamNonBlocking) != cudaSuccess ||
-      cudaStreamCreateWithFlags(&st->sV, cudaStreamNonBlocking) != cudaSuccess ||
-      cudaStreamCreateWithFlags(&st->sCap, cudaStreamNonBlocking) != cudaSuccess) {
-    delete st;
+  {
+    // default one group: on the paper-scale workload more groups were slower (every
+    // kernel keeps a fixed cost of several microseconds however little work it has,
+    // and the chains of one group already overlap), so the split is opt-in
+    int gr = 1;
+    const char* e = getenv("FWPKM_GROUPS");
+    if (e && atoi(e) > 0) gr = atoi(e);
+    if (gr > dm.M) gr = dm.M;
+    if (gr > fwpkm_state::MAX_GROUPS) gr = fwpkm_state::MAX_GROUPS;
+    st->groups = gr < 1 ? 1 : gr;
+  }
+  bool ok = cudaStreamCreateWithFlags(&st->sCap, cudaStreamNonBlocking) == cudaSuccess;
+  for (int gi = 0; gi < fwpkm_state::MAX_GROUPS; ++gi) st->sK[gi] = st->sS[gi] = st->sV[gi] = nullptr;
+  for (int gi = 0; gi < st->groups && ok; ++gi)
+    ok = cudaStreamCreateWithFlags(&st->sK[gi], cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&st->sS[gi], cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&st->sV[gi], cudaStreamNonBlocking) == cudaSuccess;
+  if (!ok) {
+    fwpkm_destroy_state(st);
     return FWPKM_ERR_CUDA;
   }
   if (cudaMemset(st->wk.status, 0, sizeof(int)) != cudaSuccess) {
@@ -282,10 +328,12 @@ void fwpkm_destroy_state(fwpkm_state* st) {
   if (!st) return;
   if (st->graph_exec) cudaGraphExecDestroy(st->graph_exec);
   for (cudaEvent_t e : st->sync_ev) cudaEventDestroy(e);
-  cudaStreamDestroy(st->sK);
-  cudaStreamDestroy(st->sS);
-  cudaStreamDestroy(st->sV);
-  cudaStreamDestroy(st->sCap);
+  for (int gi = 0; gi < fwpkm_state::MAX_GROUPS; ++gi) {
+    if (st->sK[gi]) cudaStreamDestroy(st->sK[gi]);
+    if (st->sS[gi]) cudaStreamDestroy(st->sS[gi]);
+    if (st->sV[gi]) cudaStreamDestroy(st->sV[gi]);
+  }
+  if (st->sCap) cudaStreamDestroy(st->sCap);
   for (cudaEvent_t e : st->ev) cudaEventDestroy(e);
   delete st;
 }
@@ -356,20 +404,20 @@ fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream
 // of two buffers, so sK may start chunk c+1 while sS still reads chunk c's rows.  Across
 // passes, chunk c's selection waits for the previous pass's write of chunk c (its slot
 // lists and weights are overwritten).
-static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, const float* g, int T, int n_iter,
-                             float* o, cudaStream_t origin) {
-  const Dims& d = st->dm;
+static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk, float* K1, float* K2, float* V,
+                          const void* q, const void* v, const float* g, int T, int n_iter, float* o,
+                          cudaStream_t origin) {
   const size_t es = qv_size(d);
   const int C = d.C;
   const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
   const bool la = (d.flags & FWPKM_LOOKAHEAD) != 0;
-  const bool tc = st->wk.tc != 0;
+  const bool tc = wk.tc != 0;
   const int nch = (T + C - 1) / C;
   // the key step reads every chunk's half-queries from one feature-major copy made up front
   // (its TMA x offset, the chunk start, must be a multiple of 8 tokens)
   const bool qt_whole = tc && ku && C % 8 == 0;
-  cudaStream_t sK = st->sK, sS = st->serial ? st->sK : st->sS, sV = st->serial ? st->sK : st->sV;
-  st->ev_next = 0;
+  cudaStream_t sK = st->serial ? st->sK[0] : st->sK[gi];
+  cudaStream_t sS = st->serial ? sK : st->sS[gi], sV = st->serial ? sK : st->sV[gi];
   auto dep = [&](cudaStream_t from, cudaStream_t to) {
     cudaEvent_t e = next_event(st);
     cudaEventRecord(e, from);
@@ -389,33 +437,33 @@ static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, cons
     const void* vc = offs(v, (long long)t0 * d.dv, es);
     const void* vn = (t0 + len < T) ? offs(v, (long long)(t0 + len) * d.dv, es) : nullptr;
     run(st, KK_GATHER, sV, [&] {
-      return launch_gather(d, st->wk, st->V, vc, g + t0, T, t0, len, o + (long long)t0 * d.dv, true, vn, sV);
+      return launch_gather(d, wk, V, vc, g + t0, T, t0, len, o + (long long)t0 * d.dv, true, vn, sV);
     });
-    run(st, KK_WRITE, sV, [&] { return launch_write(d, st->wk, st->V, t0, sV); });
+    run(st, KK_WRITE, sV, [&] { return launch_write(d, wk, V, t0, sV); });
   };
 
   if (tc) {
-    run(st, KK_PREP, sK, [&] { return launch_qnorm(d, st->wk, q, T, 0, T, sK); });
-    if (qt_whole) run(st, KK_PREP, sK, [&] { return launch_qtrans(d, st->wk, q, T, 0, T, sK); });
-    run(st, KK_PREP, sK, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, sK); });
+    run(st, KK_PREP, sK, [&] { return launch_qnorm(d, wk, q, T, 0, T, sK); });
+    if (qt_whole) run(st, KK_PREP, sK, [&] { return launch_qtrans(d, wk, q, T, 0, T, sK); });
+    run(st, KK_PREP, sK, [&] { return launch_keyprep(d, wk, K1, K2, sK); });
   }
   if (!ku) {
     // frozen keys: address window by window on sK; the value loop of a window starts as
     // soon as its chunks are sorted.  The addressing serves every pass.
-    const int wtok = tc ? st->wk.drows : T;
+    const int wtok = tc ? wk.drows : T;
     std::vector<cudaEvent_t> ready;
     for (int w0 = 0; w0 < T; w0 += wtok) {
       const int wl = T - w0 < wtok ? T - w0 : wtok;
       if (tc) {
-        run(st, KK_SCORE, sK, [&] { return launch_tc_score(d, st->wk, q, T, T, w0, w0, wl, false, sK); });
-        run(st, KK_TOPK, sK, [&] { return launch_topk_rows(d, st->wk, w0, wl, sK); });
+        run(st, KK_SCORE, sK, [&] { return launch_tc_score(d, wk, q, T, T, w0, w0, wl, false, sK); });
+        run(st, KK_TOPK, sK, [&] { return launch_topk_rows(d, wk, w0, wl, sK); });
       } else {
         run(st, KK_SCORE, sK, [&] {
-          return launch_score_topk(d, st->wk, st->K1, st->K2, offs(q, (long long)w0 * d.d, es), T, w0, wl, false, sK);
+          return launch_score_topk(d, wk, K1, K2, offs(q, (long long)w0 * d.d, es), T, w0, wl, false, sK);
         });
       }
-      run(st, KK_CART, sK, [&] { return launch_cartesian(d, st->wk, w0, wl, nullptr, nullptr, sK); });
-      run(st, KK_SORT, sK, [&] { return launch_sort_pairs(d, st->wk, w0, wl, !la || (w0 + wl < T), sK); });
+      run(st, KK_CART, sK, [&] { return launch_cartesian(d, wk, w0, wl, nullptr, nullptr, sK); });
+      run(st, KK_SORT, sK, [&] { return launch_sort_pairs(d, wk, w0, wl, !la || (w0 + wl < T), sK); });
       ready.push_back(mark(sK));
     }
     for (int pass = 0; pass < n_iter; ++pass)
@@ -424,26 +472,26 @@ static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, cons
         value_chunk(c);
       }
   } else {
-    const size_t dbuf = (size_t)d.M * 2 * d.C * d.n;
+    const size_t dbuf = (size_t)wk.dfull_buf;
     std::vector<cudaEvent_t> topk_done(2, nullptr), sel_done(nch, nullptr), val_done(nch, nullptr);
     int cnt = 0;
     for (int pass = 0; pass < n_iter; ++pass) {
       for (int c = 0; c < nch; ++c, ++cnt) {
         const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
         const void* qc = offs(q, (long long)t0 * d.d, es);
-        Work wb = st->wk;
-        if (tc) wb.Dfull = st->wk.Dfull + (size_t)(cnt & 1) * dbuf;
+        Work wb = wk;
+        if (tc) wb.Dfull = wk.Dfull + (size_t)(cnt & 1) * dbuf;
         if (sel_done[c]) cudaStreamWaitEvent(sK, sel_done[c], 0);    // previous pass read A/Dsv
         if (topk_done[cnt & 1]) cudaStreamWaitEvent(sK, topk_done[cnt & 1], 0);  // buffer reuse
         if (tc) {
           run(st, KK_SCORE, sK, [&] { return launch_tc_score(d, wb, q, T, T, t0, t0, len, true, sK); });
         } else {
-          run(st, KK_SCORE, sK, [&] { return launch_score_topk(d, wb, st->K1, st->K2, qc, T, t0, len, true, sK); });
+          run(st, KK_SCORE, sK, [&] { return launch_score_topk(d, wb, K1, K2, qc, T, t0, len, true, sK); });
         }
         cudaStreamWaitEvent(sS, mark(sK), 0);
         run(st, KK_ADDR, sK, [&] {
-          return tc ? launch_tc_address(d, wb, st->K1, st->K2, qc, T, len, qt_whole ? t0 : -1, sK)
-                    : launch_address(d, wb, st->K1, st->K2, qc, T, len, sK);
+          return tc ? launch_tc_address(d, wb, K1, K2, qc, T, len, qt_whole ? t0 : -1, sK)
+                    : launch_address(d, wb, K1, K2, qc, T, len, sK);
         });
         if (val_done[c]) cudaStreamWaitEvent(sS, val_done[c], 0);     // previous pass wrote chunk c
         if (tc) {
@@ -462,6 +510,26 @@ static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, cons
   dep(sK, origin);
   dep(sS, origin);
   dep(sV, origin);
+}
+
+// Split the memories into st->groups contiguous groups and enqueue each as its own set of
+// chains (all of them fork from and join back to `origin`).
+static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, const float* g, int T, int n_iter,
+                             float* o, cudaStream_t origin) {
+  const Dims& d = st->dm;
+  const size_t es = qv_size(d);
+  st->ev_next = 0;
+  const int G = st->groups;
+  for (int gi = 0; gi < G; ++gi) {
+    const int m0 = (int)((long long)gi * d.M / G), m1 = (int)((long long)(gi + 1) * d.M / G);
+    Dims dg = d;
+    dg.M = m1 - m0;
+    const Work wg = G == 1 ? st->wk : group_work(d, st->wk, m0);
+    const size_t kh = (size_t)m0 * d.n * d.h;
+    enqueue_group(st, gi, dg, wg, st->K1 + kh, st->K2 + kh, st->V + (size_t)m0 * d.N * d.dv,
+                  offs(q, (long long)m0 * T * d.d, es), offs(v, (long long)m0 * T * d.dv, es), g + (size_t)m0 * T,
+                  T, n_iter, o + (size_t)m0 * T * d.dv, origin);
+  }
 }
 
 fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, const float* g, int T,

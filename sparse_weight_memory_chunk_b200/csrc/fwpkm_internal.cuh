@@ -54,9 +54,14 @@ struct Work {
   __nv_bfloat16* Qt; // [M*2][h][qt_T]     half-queries, feature major (operand B of the key step)
   int qt_T;          // token columns of Qt (a multiple of 64)
   float* wsum_part;  // [M*2][Cpad/64][n]  per-token-tile sums of W
+  // Every array above is memory-major except the bf16 pieces (Kpc, Wt), whose piece
+  // stride is P_all problems; a Work for a group of memories is the same carve with its
+  // pointers advanced to the group's first memory (see group_work).
+  int P_all;         // problems between consecutive bf16 pieces of Kpc / Wt (2 * all memories)
+  long long dfull_buf; // elements between the two distance-row buffers
 };
 
-enum : int { TC_EPI_DIST = 0, TC_EPI_KEYSTEP = 1 };
+enum : int { TC_EPI_DIST = 0, TC_EPI_KEYSTEP = 1, TC_EPI_PROJ = 2 };
 
 // One batched tensor-core contraction (see tc_gemm.cu).  Problem p (blockIdx.z) owns
 // A tiles at (x = (p % a_div) * a_xoff + 64 kb, y = a_y0 + 128 mt, z = p / a_div + pa * a_zpiece)
@@ -73,8 +78,12 @@ struct TcGemm {
   const float* colv; long long colv_pstride;
   float* zpart; long long zpart_pstride; float eps;
   // TC_EPI_KEYSTEP
-  float* K1; float* K2; __nv_bfloat16* Kpc; float* kn;
+  float* K1; float* K2; __nv_bfloat16* Kpc; float* kn; int piece_P;
   const float* wsum_part; int wsum_tiles; float lr;
+  // TC_EPI_PROJ: y[r][c] = acc * rowscale[r] + bias[c] (n_valid and split multiples of 32)
+  // into pout0[r][c] (c < split) or pout1[r][c - split], fp32 or (out_bf16) bf16
+  const float* rowscale; const float* bias;
+  void* pout0; void* pout1; int split, ld0, ld1, out_bf16;
   int* status;
 };
 
@@ -83,6 +92,8 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t 
 int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g, int m_tiles, cudaStream_t s);
 
 size_t workspace_bytes(const Dims& d, int max_T, Work* carve, char* base);
+// The carve `w` of all memories seen from memory m0 on (kernels index it from 0).
+Work group_work(const Dims& d, const Work& w, int m0);
 
 // ---- launchers (each enqueues on `s` and returns the number of kernels launched) ----
 // Tokens are addressed two ways: user buffers are passed already offset to the first

@@ -226,6 +226,31 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         if (rv && g.zpart)
           g.zpart[(((size_t)p * g.zpart_pstride + r) * g.n_tiles + nt) * 4 + cg] = zacc;
+      } else if (g.epi == TC_EPI_PROJ) {
+        const int c0 = nt * TC_BN + cg * 32;
+        if (rv && c0 < g.n_valid) {
+          const float rs = g.rowscale[r];
+          float y[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]) * rs + (g.bias ? g.bias[c0 + i] : 0.f);
+          const bool first = c0 < g.split;
+          const size_t off = first ? (size_t)r * g.ld0 + c0 : (size_t)r * g.ld1 + (c0 - g.split);
+          if (g.out_bf16) {
+            __nv_bfloat16* dst = (__nv_bfloat16*)(first ? g.pout0 : g.pout1) + off;
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              __align__(16) __nv_bfloat16 yb[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) yb[u] = __float2bfloat16_rn(y[i + u]);
+              *reinterpret_cast<uint4*>(dst + i) = *reinterpret_cast<uint4*>(yb);
+            }
+          } else {
+            float* dst = (float*)(first ? g.pout0 : g.pout1) + off;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + i) = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
+          }
+        }
       } else {  // TC_EPI_KEYSTEP: row = sub-key b, columns = features e (one tile covers h)
         const int h = g.n_valid;
         const int n = g.m_valid;
@@ -235,7 +260,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           float wsum = 0.f;
           for (int tt = 0; tt < g.wsum_tiles; ++tt) wsum += g.wsum_part[((size_t)p * g.wsum_tiles + tt) * n + r];
           float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h;
-          const size_t pstride = (size_t)g.P * n * h;
+          const size_t pstride = (size_t)g.piece_P * n * h;
           __nv_bfloat16* pc = g.Kpc + ((size_t)p * n + r) * h;
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {

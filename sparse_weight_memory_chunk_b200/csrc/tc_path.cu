@@ -52,7 +52,7 @@ keyprep_kernel(Dims dm, Work w, const float* __restrict__ K1, const float* __res
   const int p = (int)(idx / dm.n), b = (int)(idx - (long long)p * dm.n);
   const int m = p >> 1, j = p & 1, h = dm.h;
   const float* K = (j == 0 ? K1 : K2) + ((size_t)m * dm.n + b) * h;
-  const size_t pstride = (size_t)P * dm.n * h;
+  const size_t pstride = (size_t)w.P_all * dm.n * h;
   __nv_bfloat16* pc = w.Kpc + ((size_t)p * dm.n + b) * h;
   // squared norm as four 32-feature partial sums combined in order, exactly as the
   // key-step GEMM epilogue forms it
@@ -133,7 +133,7 @@ tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
   __shared__ float s_invz[64], s_L[64], s_lp[64];
   const int p = blockIdx.z;
   const int b0 = blockIdx.x * 64, t0 = blockIdx.y * 64;
-  const int n = dm.n, P = dm.M * 2;
+  const int n = dm.n;
   const int tid = threadIdx.x;
   if (tid < 64) {
     const int t = t0 + tid;
@@ -165,7 +165,7 @@ tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
     for (int tl = 0; tl < 64; ++tl) s += s_W[tid][tl];
     w.wsum_part[((size_t)p * ntt + blockIdx.y) * n + b0 + tid] = s;
   }
-  const size_t pstride = (size_t)P * n * cpad;
+  const size_t pstride = (size_t)w.P_all * n * cpad;
   for (int idx = tid; idx < 64 * 8; idx += TP_THREADS) {
     const int bl = idx >> 3, c8 = idx & 7;
     const int b = b0 + bl;
@@ -228,14 +228,16 @@ int launch_tc_score(const Dims& d, const Work& w, const void* q_base, long long 
   const int P = d.M * 2;
   CUtensorMap A, B;
   if (!make_tmap_bf16_3d(&A, q_base, d.d, q_extent, d.M, (uint64_t)d.d * 2, (uint64_t)q_stride * d.d * 2)) return -1;
-  if (!make_tmap_bf16_3d(&B, w.Kpc, d.h, d.n, 3 * P, (uint64_t)d.h * 2, (uint64_t)d.n * d.h * 2)) return -1;
+  // pieces of problem p sit at z = p, p + P_all, p + 2 P_all
+  if (!make_tmap_bf16_3d(&B, w.Kpc, d.h, d.n, 2 * w.P_all + P, (uint64_t)d.h * 2, (uint64_t)d.n * d.h * 2))
+    return -1;
   TcGemm g = {};
   g.P = P;
   g.k_blocks = d.h / 64;
   g.n_tiles = (d.n + 127) / 128;
   g.tiles_per_cta = 2;
   g.a_pieces = 1; g.b_pieces = 3;
-  g.a_div = 2; g.a_xoff = d.h; g.a_y0 = q_row0; g.a_zpiece = 0; g.b_zpiece = P;
+  g.a_div = 2; g.a_xoff = d.h; g.a_y0 = q_row0; g.a_zpiece = 0; g.b_zpiece = w.P_all;
   g.m_valid = len; g.n_valid = d.n;
   g.epi = TC_EPI_DIST;
   g.out = w.Dfull; g.out_pstride = (long long)w.drows * d.n; g.out_ld = d.n;
@@ -270,7 +272,8 @@ int launch_tc_address(const Dims& d, const Work& w, float* K1, float* K2, const 
   tc_rowL_kernel<<<dim3((len + 7) / 8, P), TP_THREADS, 0, s>>>(d, w, len);
   tc_wbuild_kernel<<<dim3((d.n + 63) / 64, ntt, P), TP_THREADS, 0, s>>>(d, w, len, cpad);
   CUtensorMap A, B;
-  if (!make_tmap_bf16_3d(&A, w.Wt, len, d.n, 3 * P, (uint64_t)cpad * 2, (uint64_t)d.n * cpad * 2)) return -1;
+  if (!make_tmap_bf16_3d(&A, w.Wt, len, d.n, 2 * w.P_all + P, (uint64_t)cpad * 2, (uint64_t)d.n * cpad * 2))
+    return -1;
   if (!make_tmap_bf16_3d(&B, w.Qt, w.qt_T, d.h, P, (uint64_t)w.qt_T * 2, (uint64_t)d.h * w.qt_T * 2)) return -1;
   TcGemm g = {};
   g.P = P;
@@ -278,10 +281,10 @@ int launch_tc_address(const Dims& d, const Work& w, float* K1, float* K2, const 
   g.n_tiles = 1;
   g.tiles_per_cta = 1;
   g.a_pieces = 3; g.b_pieces = 1;
-  g.a_div = 1; g.a_xoff = 0; g.a_y0 = 0; g.a_zpiece = P; g.b_zpiece = 0; g.b_x0 = qt_t0;
+  g.a_div = 1; g.a_xoff = 0; g.a_y0 = 0; g.a_zpiece = w.P_all; g.b_zpiece = 0; g.b_x0 = qt_t0;
   g.m_valid = d.n; g.n_valid = d.h;
   g.epi = TC_EPI_KEYSTEP;
-  g.K1 = K1; g.K2 = K2; g.Kpc = w.Kpc; g.kn = w.kn;
+  g.K1 = K1; g.K2 = K2; g.Kpc = w.Kpc; g.kn = w.kn; g.piece_P = w.P_all;
   g.wsum_part = w.wsum_part; g.wsum_tiles = ntt; g.lr = d.lr_key;
   g.status = w.status;
   launch_tc_gemm(A, B, g, (d.n + 127) / 128, s);

@@ -191,12 +191,10 @@ resid_kernel(Dims dm, Work w, const VT* __restrict__ v, const float* __restrict_
 // contiguous and in token order.  Each warp owns G consecutive list positions; a
 // position whose slot differs from its predecessor's starts a segment (one touched row)
 // and that segment belongs to the warp, even where it runs past the warp's positions.
-// Before consuming anything the warp issues, for each of its segments, the loads of the
-// value row, of the first pair's weight and of the first pair's residual row; segment
-// ends come from keys the warp already holds, so the common one-reader row costs a single
-// round of independent loads.  It then stores V_i - G_i / N_read,i with
-// G_i = sum s'_{t,i} r_t in token order.  Rows are disjoint, so there are no atomics and
-// the result does not depend on scheduling.
+// The warp issues the value-row loads of all its segments before consuming any, then for
+// each row sums G_i = sum s'_{t,i} r_t in token order and stores V_i - G_i / N_read,i.
+// Rows are disjoint, so there are no atomics and the result does not depend on
+// scheduling.
 // ---------------------------------------------------------------------------
 template <int VPL, int G>
 __global__ void __launch_bounds__(VAL_WARPS * 32)
@@ -210,66 +208,43 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
   const int pos0 = (blockIdx.x * VAL_WARPS + warp) * G;
   if (pos0 >= P) return;
   const unsigned long long* sk = w.sk + cbase * (size_t)(C * k);
-  // lanes 0..G: keys at pos0 .. pos0+G (lane G: the first position after the range);
-  // lane 31: the key before the range
   unsigned long long my_key = ~0ull;
-  if (lane <= G && pos0 + lane < P) my_key = sk[pos0 + lane];
-  if (lane == 31 && pos0 > 0) my_key = sk[pos0 - 1];
-  const int my_slot = (int)(my_key >> 32);
-  const int prev_slot = __shfl_up_sync(0xffffffffu, my_slot, 1);
-  const int before = __shfl_sync(0xffffffffu, my_slot, 31);
-  const bool valid = lane < G && pos0 + lane < P;
-  const bool head = valid && (lane == 0 ? (pos0 == 0 || before != my_slot) : prev_slot != my_slot);
+  bool head = false;
+  if (lane < G && pos0 + lane < P) {
+    const int pos = pos0 + lane;
+    my_key = sk[pos];
+    head = pos == 0 || (sk[pos - 1] >> 32) != (my_key >> 32);
+  }
   const unsigned heads = __ballot_sync(0xffffffffu, head);
-  const uint32_t my_tr = (uint32_t)(my_key & 0xffffffffu);
-  const int my_t = (int)(my_tr / (uint32_t)k), my_r = (int)(my_tr - (uint32_t)my_t * k);
-  float my_wt = 0.f;
-  if (valid) my_wt = w.w[((size_t)m * w.max_T + wt0 + my_t) * k + my_r];
-
+  const int my_slot = (int)(my_key >> 32);
   float* Vm = V + (size_t)m * dm.N * dm.dv;
-  float4 Vr[G][VPL], R0[G][VPL];
+  float4 Vr[G][VPL];
 #pragma unroll
   for (int gi = 0; gi < G; ++gi) {
     const int slot = __shfl_sync(0xffffffffu, my_slot, gi);
-    const int t0 = __shfl_sync(0xffffffffu, my_t, gi);
     const bool ok = ((heads >> gi) & 1u) && slot >= 0 && (long long)slot < dm.N;
     const float4* row = reinterpret_cast<const float4*>(Vm + (size_t)(ok ? slot : 0) * dm.dv);
-    const float4* rr = reinterpret_cast<const float4*>(w.resid + ((size_t)m * C + (ok ? t0 : 0)) * dm.dv);
 #pragma unroll
     for (int c = 0; c < VPL; ++c) {
       const int e4 = lane + 32 * c;
       Vr[gi][c] = (ok && e4 < dv4) ? row[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
-      R0[gi][c] = (ok && e4 < dv4) ? rr[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
 #pragma unroll
   for (int gi = 0; gi < G; ++gi) {
-    const int slot = __shfl_sync(0xffffffffu, my_slot, gi);
-    const float wt0v = __shfl_sync(0xffffffffu, my_wt, gi);
+    const unsigned long long key0 = __shfl_sync(0xffffffffu, my_key, gi);
     if (!((heads >> gi) & 1u)) continue;
+    const int slot = (int)(key0 >> 32);
     if (slot < 0 || (long long)slot >= dm.N) {
       if (lane == 0) atomicExch(w.status, DEV_BAD_SLOT);
       continue;
     }
     float4 Gs[VPL];
 #pragma unroll
-    for (int c = 0; c < VPL; ++c) {
-      Gs[c].x = wt0v * R0[gi][c].x; Gs[c].y = wt0v * R0[gi][c].y;
-      Gs[c].z = wt0v * R0[gi][c].z; Gs[c].w = wt0v * R0[gi][c].w;
-    }
-    // further pairs of this row: inside the range they are the lanes up to the next head;
-    // past the range they are read from the list
-    int p = pos0 + gi + 1;
+    for (int c = 0; c < VPL; ++c) Gs[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    int p = pos0 + gi;
+    unsigned long long key = key0;
     for (;;) {
-      unsigned long long key;
-      if (p - pos0 <= G) {
-        key = __shfl_sync(0xffffffffu, my_key, (p - pos0) & 31);  // lane G holds pos0+G
-        if (p >= P) break;
-      } else {
-        if (p >= P) break;
-        key = sk[p];
-      }
-      if ((int)(key >> 32) != slot) break;
       const uint32_t tr = (uint32_t)(key & 0xffffffffu);
       const int t_local = (int)(tr / (uint32_t)k), r = (int)(tr - (uint32_t)t_local * k);
       const float wt = w.w[((size_t)m * w.max_T + wt0 + t_local) * k + r];
@@ -283,7 +258,9 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
           Gs[c].z = fmaf(wt, x.z, Gs[c].z); Gs[c].w = fmaf(wt, x.w, Gs[c].w);
         }
       }
-      ++p;
+      if (++p >= P) break;
+      key = sk[p];
+      if ((int)(key >> 32) != slot) break;
     }
     const float nr = (float)(p - (pos0 + gi));
     float4* row = reinterpret_cast<float4*>(Vm + (size_t)slot * dm.dv);

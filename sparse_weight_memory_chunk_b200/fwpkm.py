@@ -47,6 +47,18 @@ _lib = None
 _P = ctypes.c_void_p
 
 
+class LayerConfig(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int), ("d", ctypes.c_int), ("d_v", ctypes.c_int), ("max_rows", ctypes.c_int),
+                ("eps_rms", ctypes.c_float), ("qv_dtype", ctypes.c_int)]
+
+
+class LayerParams(ctypes.Structure):
+    _fields_ = [("W_q", _P), ("gamma_q", _P), ("b_q", _P),
+                ("W_v", _P), ("gamma_v", _P), ("b_v", _P),
+                ("w_g", _P), ("gamma_g", _P), ("b_g", ctypes.c_float),
+                ("W_o", _P), ("gamma_o", _P), ("b_o", _P)]
+
+
 def lib():
     """Load libfwpkm.so (raises if it has not been built)."""
     global _lib
@@ -73,6 +85,15 @@ def lib():
             "fwpkm_profile_kernel": ([_P, ctypes.c_int], ctypes.c_int),
             "fwpkm_kernel_time": ([_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)],
                                   ctypes.c_int),
+            "fwpkm_layer_workspace_size": ([ctypes.POINTER(LayerConfig), ctypes.POINTER(ctypes.c_size_t)],
+                                           ctypes.c_int),
+            "fwpkm_layer_init": ([ctypes.POINTER(LayerConfig), _P, ctypes.c_size_t, ctypes.POINTER(_P)],
+                                 ctypes.c_int),
+            "fwpkm_layer_set_params": ([_P, ctypes.POINTER(LayerParams), _P], ctypes.c_int),
+            "fwpkm_layer_in": ([_P, _P, ctypes.c_int, _P, _P, _P, _P], ctypes.c_int),
+            "fwpkm_layer_out": ([_P, _P, ctypes.c_int, _P, _P], ctypes.c_int),
+            "fwpkm_layer_sync": ([_P, _P], ctypes.c_int),
+            "fwpkm_layer_destroy": ([_P], None),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -176,6 +197,52 @@ class State:
     def destroy(self):
         if getattr(self, "handle", None):
             lib().fwpkm_destroy_state(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+class Layer:
+    """A handle from ``fwpkm_layer_init``: the slow-weight projections (method steps 1
+    and 3).  Weights are bf16 tensors [out][in]; norm weights and biases fp32 (None:
+    ones / zeros)."""
+
+    def __init__(self, d_model, d, d_v, max_rows, eps_rms=1e-6, qv_bf16=False, device="cuda"):
+        import torch
+        self.cfg = LayerConfig(d_model, d, d_v, max_rows, eps_rms, BF16 if qv_bf16 else F32)
+        out = ctypes.c_size_t(0)
+        _check(lib().fwpkm_layer_workspace_size(ctypes.byref(self.cfg), ctypes.byref(out)), "layer_workspace_size")
+        self.workspace = torch.empty(out.value, dtype=torch.uint8, device=device)
+        h = _P()
+        _check(lib().fwpkm_layer_init(ctypes.byref(self.cfg), _ptr(self.workspace), out.value, ctypes.byref(h)),
+               "layer_init")
+        self.handle = h
+
+    def set_params(self, W_q, W_v, w_g, W_o, gamma_q=None, gamma_v=None, gamma_g=None, gamma_o=None,
+                   b_q=None, b_v=None, b_g=0.0, b_o=None, stream=None):
+        p = LayerParams(_ptr(W_q), _ptr(gamma_q), _ptr(b_q), _ptr(W_v), _ptr(gamma_v), _ptr(b_v),
+                        _ptr(w_g), _ptr(gamma_g), float(b_g), _ptr(W_o), _ptr(gamma_o), _ptr(b_o))
+        _check(lib().fwpkm_layer_set_params(self.handle, ctypes.byref(p), _stream(stream)), "layer_set_params")
+
+    def project_in(self, h, q, v, g, rows=None, stream=None):
+        rows = h.shape[0] if rows is None else rows
+        _check(lib().fwpkm_layer_in(self.handle, _ptr(h), rows, _ptr(q), _ptr(v), _ptr(g), _stream(stream)),
+               "layer_in")
+
+    def project_out(self, o, o_out, rows=None, stream=None):
+        rows = o.shape[0] if rows is None else rows
+        _check(lib().fwpkm_layer_out(self.handle, _ptr(o), rows, _ptr(o_out), _stream(stream)), "layer_out")
+
+    def sync(self, stream=None):
+        _check(lib().fwpkm_layer_sync(self.handle, _stream(stream)), "layer_sync")
+
+    def destroy(self):
+        if getattr(self, "handle", None):
+            lib().fwpkm_layer_destroy(self.handle)
             self.handle = None
 
     def __del__(self):

@@ -174,8 +174,8 @@ def gen_layer(w: Workload, B: int | None = None, T: int | None = None):
 
     h [B][T][d_model] bf16 bits from 64 Gaussian clusters (centres N(0, I), cluster
     weights proportional to j^-1.1, x = centre + 0.1 N(0, I)); RMSNorm gains = 1;
-    W_q [d_model][d], W_v [d_model][d_v], w_g [d_model] and W_o [d_v][d_model] as
-    bf16 bits drawn N(0, 1/fan_in); gate bias 0."""
+    W_q [d][d_model], W_v [d_v][d_model], w_g [d_model] and W_o [d_model][d_v]
+    ([out][in]) as bf16 bits drawn N(0, 1/fan_in); gate bias 0."""
     B = w.B if B is None else B
     T = w.T if T is None else T
     ss = _streams(w.seed)
@@ -194,9 +194,9 @@ def gen_layer(w: Workload, B: int | None = None, T: int | None = None):
         x = np.random.Generator(np.random.PCG64(kid)).standard_normal(shape, dtype=np.float32)
         return f32_to_bf16(x * np.float32(1.0 / np.sqrt(fan_in)))
 
-    Wq = lin(kids[3], (w.d_model, w.d), w.d_model)
-    Wv = lin(kids[4], (w.d_model, w.d_v), w.d_model)
+    Wq = lin(kids[3], (w.d, w.d_model), w.d_model)
+    Wv = lin(kids[4], (w.d_v, w.d_model), w.d_model)
     kg, ko = kids[5].spawn(2)
     wg = lin(kg, (w.d_model,), w.d_model)
-    Wo = lin(ko, (w.d_v, w.d_model), w.d_v)
+    Wo = lin(ko, (w.d_model, w.d_v), w.d_v)
     return dict(h=np.ascontiguousarray(hid), Wq=Wq, Wv=Wv, wg=wg, Wo=Wo, assign=assign)

@@ -64,3 +64,23 @@ def test_workspace_size_and_validation(lib):
 
 def test_launch_counter_starts_at_zero(lib):
     assert lib.launch_count() == 0
+
+
+def test_layer_workspace_size_and_validation(lib):
+    import ctypes as C
+    so = lib.lib()
+    out = C.c_size_t(0)
+    cfg = lib.LayerConfig(2048, 256, 256, 65536, 1e-6, 0)
+    assert so.fwpkm_layer_workspace_size(C.byref(cfg), C.byref(out)) == lib.OK
+    # two bf16 pieces of both weight matrices + the per-row scratch of the output call
+    pieces = 2 * 2 * (512 * 2048 + 2048 * 256)
+    scratch = 4 * 65536 + 2 * 2 * 65536 * 256
+    assert pieces + scratch <= out.value < pieces + scratch + (1 << 20)
+    for bad, want in [((2048, 256, 256, 0, 1e-6), lib.ERR_INVALID_ARG), ((2000, 256, 256, 16, 1e-6), lib.ERR_UNSUPPORTED),
+                      ((2048, 48, 256, 16, 1e-6), lib.ERR_UNSUPPORTED), ((2048, 256, 96, 16, 1e-6), lib.ERR_UNSUPPORTED),
+                      ((2048, 256, 256, 16, -1.0), lib.ERR_INVALID_ARG)]:
+        c = lib.LayerConfig(*bad, 0)
+        assert so.fwpkm_layer_workspace_size(C.byref(c), C.byref(out)) == want, bad
+    assert so.fwpkm_layer_workspace_size(C.byref(cfg), None) == lib.ERR_INVALID_ARG
+    c = lib.LayerConfig(2048, 256, 256, 16, 1e-6, 7)
+    assert so.fwpkm_layer_workspace_size(C.byref(c), C.byref(out)) == lib.ERR_INVALID_ARG

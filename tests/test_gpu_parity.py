@@ -161,3 +161,20 @@ def test_edge_cases():
     with pytest.raises(fwpkm.FwpkmError) as e:
         st.run_sequence(dev["q"], dev["v"], dev["g"], o, T=w.T + 1)
     assert e.value.status == fwpkm.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name,groups", [("mid", 2), ("mid", 3), ("mid_key", 2), ("tiny_key_ragged", 2)])
+def test_memory_groups_give_the_same_bits(name, groups, monkeypatch):
+    """run_sequence splits the memories into groups with their own chains; the split
+    changes only the schedule, so every output bit equals the one-group run (which the
+    test above ties to the oracle through the chunk-by-chunk entry points)."""
+    w, data, gcfg, _ = make_case(name)
+    outs = []
+    for gr in (1, groups):
+        monkeypatch.setenv("FWPKM_GROUPS", str(gr))
+        st, dev = device_state(w, data, gcfg, w.T)
+        o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+        st.run_sequence(dev["q"], dev["v"], dev["g"], o, n_iter=2)
+        st.sync()
+        outs.append((o.cpu(), dev["V"].cpu(), dev["K1"].cpu(), dev["K2"].cpu()))
+    assert all(torch.equal(a, b) for a, b in zip(*outs)), f"{name}: {groups} groups differ from one"
