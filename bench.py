@@ -6,7 +6,7 @@ fwpkm_run_sequence over B sequences x H heads x T tokens.  Default workload: the
 paper-scale memory (n=1024 -> N=1,048,576 slots, d=d_v=256, k=32, C=256, B=4, H=2,
 T=4096, bf16 q/v, fp32 state, key update on).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload paper|mid|tiny|needle]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload paper|mid|tiny|needle|layer]
     python bench.py --impl reference ...   # the CPU oracle on a bounded sample
 
 Multi-GPU (torchrun): every rank runs its own independent memories (different
@@ -27,9 +27,15 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from sparse_weight_memory_chunk_b200.inputs import WORKLOADS, gen_keys, gen_qvg, gen_values  # noqa: E402
+from sparse_weight_memory_chunk_b200.inputs import (WORKLOADS, gen_keys, gen_layer, gen_needles, gen_qvg,  # noqa: E402
+                                                    gen_values)
 
 BY_NAME = {w.name: (i, w) for i, w in WORKLOADS.items()}
+
+# DRAM bytes (read + write) per launch and per memory of the paper-scale kernels, from one
+# ncu capture of a 2-memory case (profiles/ has the capture and its command); a full
+# launch scales with the memories it processes.  A kernel missing here reports null.
+TRAFFIC = {}
 
 
 def parse():
@@ -38,7 +44,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="paper", choices=["tiny", "mid", "paper", "needle"])
+    ap.add_argument("--workload", default="paper", choices=["tiny", "mid", "paper", "needle", "layer"])
     ap.add_argument("--n-iter", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -50,9 +56,12 @@ def parse():
 
 
 def describe(w, n_iter):
+    lay = (f", d_model={w.d_model} bf16 hidden states through RMSNorm+Linear in/out projections"
+           if w.d_model else "")
+    ndl = f", {w.needles} planted needles" if w.name == "needle" else ""
     return (f"{w.name}: n={w.n} (N={w.N:,} slots), d={w.d}, d_v={w.d_v}, k={w.k}, C={w.C}, "
             f"B={w.B} x H={w.H} memories, T={w.T}, {w.qv} q/v, fp32 V/K, key update "
-            f"{'on' if w.key_update else 'off'}, n_iter={n_iter}")
+            f"{'on' if w.key_update else 'off'}, n_iter={n_iter}{lay}{ndl}")
 
 
 # --------------------------------------------------------------------------- oracle leg
@@ -69,6 +78,18 @@ def oracle_sample(w, n_chunks):
     H = w.H
     T = min(w.T, n_chunks * w.C)
     key = (w.name, T)
+    if key not in _SAMPLE_CACHE and w.d_model:
+        # layer workload: the projections' oracle turns sequence 0's hidden states into q, v, g
+        from oracle import layer as orc_layer
+        L = gen_layer(w, B=1, T=T)
+        hf = bf16_to_f32(L["h"][0])
+        ones = np.ones(w.d_model)
+        qf, vf, gf = orc_layer.project_in(hf, ones, bf16_to_f32(L["Wq"]), None, ones, bf16_to_f32(L["Wv"]), None,
+                                          ones, bf16_to_f32(L["wg"]), 0.0)
+        K1, K2 = gen_keys(w, M=H)
+        V = np.stack([gen_values(w, m) for m in range(H)])
+        _SAMPLE_CACHE[key] = (qf[None], vf[None], gf[None], K1, K2, V, bf16_to_f32(L["Wo"]))
+        oracle.build()
     if key not in _SAMPLE_CACHE:
         q, v, g = gen_qvg(w, M=H)
         q, v, g = q[:, :T], v[:, :T], g[:, :T]
@@ -76,13 +97,16 @@ def oracle_sample(w, n_chunks):
         V = np.stack([gen_values(w, m) for m in range(H)])
         qf = (bf16_to_f32(q) if w.qv == "bf16" else q).astype(np.float64)
         vf = (bf16_to_f32(v) if w.qv == "bf16" else v).astype(np.float64)
-        _SAMPLE_CACHE[key] = (qf, vf, g.astype(np.float64), K1, K2, V)
+        _SAMPLE_CACHE[key] = (qf, vf, g.astype(np.float64), K1, K2, V, None)
         oracle.build()
-    qf, vf, gf, K1, K2, V = _SAMPLE_CACHE[key]
+    qf, vf, gf, K1, K2, V, Wo = _SAMPLE_CACHE[key]
     k1, k2, vv = K1.copy(), K2.copy(), V.copy()
     cfg = oracle.make_cfg(w.n, w.d, w.d_v, w.k, w.C, key_update=w.key_update)
     t0 = time.perf_counter()
-    _, used = oracle.run_sequence_multi(cfg, qf, vf, gf, k1, k2, vv, 1, nthreads=H)
+    res, used = oracle.run_sequence_multi(cfg, qf, vf, gf, k1, k2, vv, 1, nthreads=H)
+    if Wo is not None:
+        from oracle import layer as orc_layer
+        orc_layer.project_out(res[0], np.ones(w.d_v), Wo, None)
     dt = time.perf_counter() - t0
     return dict(tokens=T, seconds=dt, threads=used,
                 sample=f"sequence 0 ({H} heads = {H} memories, full N={w.N:,} each), tokens 0..{T - 1} "
@@ -168,7 +192,6 @@ def algorithmic_bytes(w, idx, T):
         U_total += int((s[:, 1:] != s[:, :-1]).sum().item()) + blk.shape[0]
     key_bytes = (2 * 4 * w.n * w.d) * w.M * ((T + C - 1) // C) if w.key_update else 0
     b_vk = 2 * U_total * dv * 4 + key_bytes
-    es = 2 if w.qv == "bf16" else 4
     gather_per_token = k * dv * 4 + k * 8 + dv * es + dv * 4
     return b_vk, gather_per_token, U_total
 
@@ -194,13 +217,13 @@ def run_ours(args, w, rank, world, local_rank):
     wr = replace(w, seed=w.seed + 1000 * rank) if rank else w
     q, v, g = gen_qvg(wr)
     K1, K2 = gen_keys(wr)
+    needles = gen_needles(wr, q, v) if w.name == "needle" else None
 
     def to_dev(x):
         if x.dtype == np.uint16:
             return torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
         return torch.from_numpy(x).to(dev)
 
-    qd, vd, gd = to_dev(q), to_dev(v), to_dev(g)
     K1d, K2d = to_dev(K1), to_dev(K2)
     Vd = torch.empty(w.M, w.N, w.d_v, device=dev)
     for m in range(w.M):
@@ -209,16 +232,38 @@ def run_ours(args, w, rank, world, local_rank):
     st = fwpkm.State(cfg, K1d, K2d, Vd, w.T)
     o = torch.empty(w.M, w.T, w.d_v, device=dev)
     stream = torch.cuda.current_stream()
+    layer = None
+    if w.d_model:
+        # full layer: h -> (RMSNorm + Linear) q, v, g -> memory -> (RMSNorm + Linear) o'
+        Ld = gen_layer(wr)
+        hd = to_dev(Ld["h"])
+        layer = fwpkm.Layer(w.d_model, w.d, w.d_v, w.M * w.T, qv_bf16=w.qv == "bf16", device=dev)
+        lw = {k_: to_dev(Ld[k_]) for k_ in ("Wq", "Wv", "wg", "Wo")}
+        layer.set_params(lw["Wq"], lw["Wv"], lw["wg"], lw["Wo"])
+        qdt = torch.bfloat16 if w.qv == "bf16" else torch.float32
+        qd = torch.empty(w.M, w.T, w.d, device=dev, dtype=qdt)
+        vd = torch.empty(w.M, w.T, w.d_v, device=dev, dtype=qdt)
+        gd = torch.empty(w.M, w.T, device=dev)
+        o_out = torch.empty(w.M * w.T, w.d_model, device=dev, dtype=torch.bfloat16)
 
-    def step():
-        st.run_sequence(qd, vd, gd, o, n_iter=args.n_iter)
+        def step():
+            layer.project_in(hd, qd, vd, gd, rows=w.M * w.T)
+            st.run_sequence(qd, vd, gd, o, n_iter=args.n_iter)
+            layer.project_out(o.view(-1, w.d_v), o_out)
+    else:
+        qd, vd, gd = to_dev(q), to_dev(v), to_dev(g)
+
+        def step():
+            st.run_sequence(qd, vd, gd, o, n_iter=args.n_iter)
+    state0 = (K1d.clone(), K2d.clone(), Vd.clone()) if needles is not None else None
 
     # warm-up; find the dominant kernel kind by timing each kind once
     for _ in range(max(args.warmup, 1)):
         step()
     kinds = {}
     if args.kernel is None:
-        for name in ("gather", "write", "score", "topk", "cartesian", "sort", "address", "prep", "other"):
+        for name in ("gather", "write", "score", "topk", "cartesian", "sort", "pbar", "wbuild", "address", "prep",
+                     "other"):
             st.profile_kernel(name)
             step()
             ms, n = st.kernel_time()
@@ -266,34 +311,51 @@ def run_ours(args, w, rank, world, local_rank):
     b_vk, gather_per_token, U = algorithmic_bytes(w, idx, w.T)
     b_vk *= args.n_iter
     flops = 2 * w.n * w.d * w.M * w.T * args.n_iter * (2 if w.key_update else 1)
+    if w.d_model:  # the slow-weight projections (in: q, v, gate; out: o')
+        flops += 2 * w.M * w.T * w.d_model * (w.d + w.d_v + 1 + w.d_v)
     t_roof = max(b_vk / (hbm_peak * 1e9), flops / (tc_peak * 1e12))
     step_frac = t_roof / (ms_step / 1000.0)
-    avg_launch_s = (dom_ms / 1000.0) / max(dom_n, 1)
-    if dominant == "gather":
-        per_launch = gather_per_token * w.M * w.C
-        achieved = per_launch / avg_launch_s / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": None}
-    elif dominant == "write":
-        per_launch = 2 * (U / max(1, (w.T + w.C - 1) // w.C)) * w.d_v * 4
-        achieved = per_launch / avg_launch_s / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": None}
-    else:
-        # contraction-shaped kernels: algorithmic FLOPs per launch against the tensor peak
-        nchunks = (w.T + w.C - 1) // w.C
-        launches_per_step = max(1, dom_n)
-        per_launch = flops / (args.n_iter * (2 if w.key_update else 1)) / (nchunks if w.key_update else 1)
-        if dominant == "address":
-            per_launch = 2 * w.n * w.d * w.M * w.C
-        achieved = per_launch / avg_launch_s / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": achieved / tc_peak, "traffic": None}
-        del launches_per_step
-    roof["kernel"] = dominant
-    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if roof['unit'] == 'GB/s' else 'bf16_tflops_sustained'})"
-    roof["avg_launch_us"] = avg_launch_s * 1e6
-    roof["launches_timed"] = dom_n
+    nchunks = (w.T + w.C - 1) // w.C
+    U_chunk = U / max(1, nchunks)  # unique touched rows per chunk launch (all memories)
+    tok = w.M * w.C  # token-memories per chunk launch
+    # algorithmic work of one launch of each kernel kind (bytes against HBM, FLOPs against
+    # the tensor peak, ALU ops against the fp32 lanes)
+    alu_peak = 148 * 128 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12  # Tops/s
+    cand = sum(w.k // (i + 1) for i in range(w.k))  # staircase candidates per token-memory
+    work = {
+        "gather": ("hbm", gather_per_token * tok),
+        "write": ("hbm", 2 * U_chunk * w.d_v * 4),
+        "score": ("tensor", 2 * w.n * w.d * tok),
+        "address": ("tensor", 2 * w.n * w.d * tok),
+        "topk": ("hbm", 2 * w.n * 4 * tok),                       # distance rows read
+        "pbar": ("hbm", 2 * w.n * 4 * tok),                       # distance rows read
+        "wbuild": ("hbm", 2 * w.n * 4 * tok * 2 + 2 * w.n * 2 * 3 * tok),  # rows read twice, 3 bf16 pieces written
+        "sort": ("hbm", w.k * tok * (4 + 8)),                      # slots read, pair keys written
+        "cartesian": ("alu", cand * 2 * tok),                      # one add + one compare per candidate
+    }
+
+    def kind_roofline(kind, ms, n):
+        if kind not in work or n == 0:
+            return None
+        bound, per_launch = work[kind]
+        avg_s = (ms / 1000.0) / n
+        if bound == "hbm":
+            ach, peak, unit, src = per_launch / avg_s / 1e9, hbm_peak, "GB/s", "hbm_gbs"
+        elif bound == "tensor":
+            ach, peak, unit, src = per_launch / avg_s / 1e12, tc_peak, "TFLOP/s", "bf16_tflops_sustained"
+        else:
+            ach, peak, unit, src = per_launch / avg_s / 1e12, alu_peak, "Tops/s", "148 SMs x 128 fp32 lanes x max clock"
+        return {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+                "traffic": TRAFFIC.get(kind, {}).get("per_mem", 0) * w.M or None,
+                "kernel": kind, "peak_source": f"{peak_src if bound != 'alu' else 'derived'} ({src})",
+                "avg_launch_us": avg_s * 1e6, "launches_timed": n,
+                "algorithmic_per_launch": per_launch}
+
+    roof = kind_roofline(dominant, dom_ms, dom_n) or {"bound": None, "kernel": dominant}
+    kind_table = {k_: {"ms_per_step": round(v_[0], 4),
+                       "frac": (round(r_["frac"], 4) if (r_ := kind_roofline(k_, v_[0], v_[1])) else None),
+                       "bound": r_["bound"] if r_ else None}
+                  for k_, v_ in kinds.items()}
 
     line = {"metric": "FwPKM layer tokens/s (retrieve+chunk write) at 1M slots; % of HBM roofline",
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -307,22 +369,24 @@ def run_ours(args, w, rank, world, local_rank):
             "roofline": roof,
             "step_roofline": {"t_roof_ms": t_roof * 1e3, "frac": step_frac, "bytes_VK": b_vk, "flops_tc": flops,
                               "unique_rows": U, "definition": "max(F_tc/P_tc, B_VK/BW_HBM) / t_step"},
-            "kernel_ms_one_step": {k_: round(v_[0], 4) for k_, v_ in kinds.items()},
+            "kernels_one_step": kind_table,
             "clocks": clk, "gpu_launches": int(launches)}
 
     # end to end through the public API with host buffers
     if not args.no_e2e:
-        qh = torch.empty_like(qd, device="cpu").pin_memory()
-        vh = torch.empty_like(vd, device="cpu").pin_memory()
-        gh = torch.empty_like(gd, device="cpu").pin_memory()
-        oh = torch.empty_like(o, device="cpu").pin_memory()
-        qh.copy_(qd); vh.copy_(vd); gh.copy_(gd)
+        dev_in = [hd] if layer is not None else [qd, vd, gd]
+        dev_out = o_out if layer is not None else o
+        host_in = [torch.empty_like(x, device="cpu").pin_memory() for x in dev_in]
+        host_out = torch.empty_like(dev_out, device="cpu").pin_memory()
+        for hx, dx in zip(host_in, dev_in):
+            hx.copy_(dx)
         torch.cuda.synchronize()
 
         def e2e_step():
-            qd.copy_(qh, non_blocking=True); vd.copy_(vh, non_blocking=True); gd.copy_(gh, non_blocking=True)
-            st.run_sequence(qd, vd, gd, o, n_iter=args.n_iter)
-            oh.copy_(o, non_blocking=True)
+            for hx, dx in zip(host_in, dev_in):
+                dx.copy_(hx, non_blocking=True)
+            step()
+            host_out.copy_(dev_out, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -338,10 +402,32 @@ def run_ours(args, w, rank, world, local_rank):
             t = torch.tensor([ems], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ems = float(t.item())
-        bi = sum(x.numel() * x.element_size() for x in (qh, vh, gh))
+        bi = sum(x.numel() * x.element_size() for x in host_in)
         line["e2e"] = {"value": tokens_per_step * world / (ems / 1000.0), "unit": "tokens/s",
-                       "h2d_bytes_per_step": bi, "d2h_bytes_per_step": oh.numel() * oh.element_size(),
+                       "h2d_bytes_per_step": bi, "d2h_bytes_per_step": host_out.numel() * host_out.element_size(),
                        "ms_per_step": ems}
+
+    if needles is not None:
+        # read-back: from the initial state, n_iter passes; vhat at each needle's query
+        # position recovered from o = g vhat + (1 - g) v, against the normalised needle value
+        from sparse_weight_memory_chunk_b200.inputs import bf16_to_f32
+        K1d.copy_(state0[0]); K2d.copy_(state0[1]); Vd.copy_(state0[2])
+        step()
+        st.sync()
+        pos, qpos, _, vs = needles
+        of = o[0].cpu().numpy().astype(np.float64)
+        vf = (bf16_to_f32(v[0]) if w.qv == "bf16" else v[0]).astype(np.float64)
+        gf = g[0].astype(np.float64)
+        vsf = (bf16_to_f32(vs) if w.qv == "bf16" else vs).astype(np.float64)
+        cos = []
+        for i, r in enumerate(qpos):
+            vhat = (of[r] - (1.0 - gf[r]) * vf[r]) / gf[r]
+            z = (vsf[i] - vsf[i].mean()) / np.sqrt(vsf[i].var() + 1e-5)
+            cos.append(float(vhat @ z / (np.linalg.norm(vhat) * np.linalg.norm(z) + 1e-30)))
+        line["needle_readback"] = {"n_iter": args.n_iter, "mean_cos": float(np.mean(cos)),
+                                   "min_cos": float(np.min(cos)), "needles": len(cos),
+                                   "definition": "cos(vhat_r, z(v*)) at each needle's query position r, final pass, "
+                                                 "run from the initial state"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_chunks = 8 if w.name in ("paper", "needle") else 16

@@ -164,9 +164,10 @@ fwpkm_status fwpkm_chunk_step_noalloc(const fwpkm_config* cfg, float* K1, float*
  * head per sequence the memory index is the sequence, so q, v, g and o are exactly
  * the [M][T][width] inputs and output of the memory calls above.
  * Precision: h and the weights W are bf16; the norm weights, biases, g and o fp32;
- * q and v fp32 or bf16 (fwpkm_layer_config.qv_dtype); o' bf16.  gamma is folded into W in fp32 and held as two bf16 pieces (one
- * when gamma is NULL); o enters the output GEMM as two bf16 pieces; accumulation is
- * fp32 on the tensor cores and 1/rms scales the accumulator.
+ * q and v fp32 or bf16 (fwpkm_layer_config.qv_dtype); o' bf16.  gamma is folded into
+ * W in fp32 (three bf16 pieces for the input GEMM, two for the output GEMM; one when
+ * gamma is NULL, as W is then exact); o enters the output GEMM as two bf16 pieces;
+ * accumulation is fp32 on the tensor cores and 1/rms scales the accumulator.
  * ------------------------------------------------------------------------- */
 typedef struct fwpkm_layer fwpkm_layer;  /* opaque host handle */
 
@@ -249,7 +250,9 @@ uint64_t fwpkm_launch_count(void);
 
 /* Per-kernel timing with CUDA events recorded on the launching stream around every
  * launch of the given kernel kind (0 = none).  Kinds: 1 gather, 2 write, 3 score,
- * 4 cartesian, 5 sort, 6 address (key step), 7 residual, 8 per-half top-k, 9 query/key prep.  fwpkm_kernel_time() waits for the events and
+ * 4 cartesian, 5 sort, 6 key-step GEMM (or the whole key step on the SIMT path),
+ * 7 residual, 8 per-half top-k, 9 query/key prep, 10 usage marginals (pbar, log pbar),
+ * 11 key-step weights W.  fwpkm_kernel_time() waits for the events and
  * returns the summed duration (ms) and the number of timed launches since the last
  * reset, then resets.  Graph replays overwrite their own events, so after graph
  * replays it covers the last replay. */

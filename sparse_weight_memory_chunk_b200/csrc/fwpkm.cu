@@ -138,6 +138,14 @@ cudaEvent_t next_event(fwpkm_state* st) {
 
 namespace fwpkm {
 
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("FWPKM_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
 // The tensor-core path needs bf16 queries (exact tcgen05 operands) and half widths that
 // are whole 64-element swizzle atoms no wider than one 128-column accumulator tile.
 bool use_tensor_cores(const Dims& d) {
@@ -192,7 +200,7 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
     x.Z = nullptr; x.lp = nullptr; x.Lt = nullptr;
   }
   x.Kpc = nullptr; x.kn = nullptr; x.qn = nullptr; x.zpart = nullptr; x.ppart = nullptr;
-  x.Wt = nullptr; x.Qt = nullptr; x.wsum_part = nullptr; x.qt_T = 0;
+  x.Wt = nullptr; x.Qt = nullptr; x.wsum_part = nullptr; x.pbar_cnt = nullptr; x.qt_T = 0;
   if (x.tc) {
     const size_t P = 2 * M, h = d.h, cpad = (C + 63) / 64 * 64, nt = (n + 127) / 128;
     x.Kpc = (__nv_bfloat16*)take(2 * 3 * P * n * h);
@@ -204,7 +212,8 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
       x.Wt = (__nv_bfloat16*)take(2 * 3 * P * n * cpad);
       x.qt_T = (int)((T > C ? T : C) + 63) / 64 * 64;
       x.Qt = (__nv_bfloat16*)take(2 * P * h * (size_t)x.qt_T);
-      x.wsum_part = (float*)take(4 * P * (cpad / 64) * n);
+      x.wsum_part = (float*)take(4 * P * (cpad / 16) * n);
+      x.pbar_cnt = (int*)take(4 * P * ((n + 255) / 256));
     }
   }
   x.P_all = (int)(2 * M);
@@ -235,7 +244,8 @@ Work group_work(const Dims& d, const Work& w, int m0) {
   if (x.ppart) x.ppart += M0 * 2 * 8 * n;
   if (x.Wt) x.Wt += M0 * 2 * n * cpad;
   if (x.Qt) x.Qt += M0 * 2 * h * (size_t)w.qt_T;
-  if (x.wsum_part) x.wsum_part += M0 * 2 * (cpad / 64) * n;
+  if (x.wsum_part) x.wsum_part += M0 * 2 * (cpad / 16) * n;
+  if (x.pbar_cnt) x.pbar_cnt += M0 * 2 * ((n + 255) / 256);
   return x;
 }
 
@@ -316,7 +326,9 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
     fwpkm_destroy_state(st);
     return FWPKM_ERR_CUDA;
   }
-  if (cudaMemset(st->wk.status, 0, sizeof(int)) != cudaSuccess) {
+  if (cudaMemset(st->wk.status, 0, sizeof(int)) != cudaSuccess ||
+      (st->wk.pbar_cnt &&
+       cudaMemset(st->wk.pbar_cnt, 0, sizeof(int) * 2 * (size_t)dm.M * ((dm.n + 255) / 256)) != cudaSuccess)) {
     delete st;
     return FWPKM_ERR_CUDA;
   }
@@ -384,11 +396,15 @@ fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream
   run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, st->wk, 0, st->len, last_has_target, s); });
   run(st, KK_WRITE, s, [&] { return launch_write(d, st->wk, st->V, 0, s); });
   st->host_error = 0;
-  if (d.flags & FWPKM_KEY_UPDATE)
+  if ((d.flags & FWPKM_KEY_UPDATE) && st->wk.tc) {
+    run(st, KK_PBAR, s, [&] { return launch_tc_pbar(d, st->wk, st->len, s); });
+    run(st, KK_WBUILD, s, [&] { return launch_tc_wbuild(d, st->wk, st->len, s); });
     run(st, KK_ADDR, s, [&] {
-      return st->wk.tc ? launch_tc_address(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, -1, s)
-                       : launch_address(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, s);
+      return launch_tc_keystep(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, -1, s);
     });
+  } else if (d.flags & FWPKM_KEY_UPDATE) {
+    run(st, KK_ADDR, s, [&] { return launch_address(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, s); });
+  }
   st->pending = 0;
   if (st->host_error) return FWPKM_ERR_CUDA;
   return last_cuda();
@@ -489,10 +505,13 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
           run(st, KK_SCORE, sK, [&] { return launch_score_topk(d, wb, K1, K2, qc, T, t0, len, true, sK); });
         }
         cudaStreamWaitEvent(sS, mark(sK), 0);
-        run(st, KK_ADDR, sK, [&] {
-          return tc ? launch_tc_address(d, wb, K1, K2, qc, T, len, qt_whole ? t0 : -1, sK)
-                    : launch_address(d, wb, K1, K2, qc, T, len, sK);
-        });
+        if (tc) {
+          run(st, KK_PBAR, sK, [&] { return launch_tc_pbar(d, wb, len, sK); });
+          run(st, KK_WBUILD, sK, [&] { return launch_tc_wbuild(d, wb, len, sK); });
+          run(st, KK_ADDR, sK, [&] { return launch_tc_keystep(d, wb, K1, K2, qc, T, len, qt_whole ? t0 : -1, sK); });
+        } else {
+          run(st, KK_ADDR, sK, [&] { return launch_address(d, wb, K1, K2, qc, T, len, sK); });
+        }
         if (val_done[c]) cudaStreamWaitEvent(sS, val_done[c], 0);     // previous pass wrote chunk c
         if (tc) {
           run(st, KK_TOPK, sS, [&] { return launch_topk_rows(d, wb, t0, len, sS); });

@@ -15,7 +15,8 @@ enum : int { DEV_OK = 0, DEV_BAD_SLOT = 1, DEV_TIMEOUT = 2 };
 
 // Kernel kinds for the launch counter / per-kernel timing.
 enum KernelKind : int { KK_NONE = 0, KK_GATHER = 1, KK_WRITE = 2, KK_SCORE = 3, KK_CART = 4,
-                        KK_SORT = 5, KK_ADDR = 6, KK_OTHER = 7, KK_TOPK = 8, KK_PREP = 9, KK_LAST = 9 };
+                        KK_SORT = 5, KK_ADDR = 6, KK_OTHER = 7, KK_TOPK = 8, KK_PREP = 9, KK_PBAR = 10,
+                        KK_WBUILD = 11, KK_LAST = 11 };
 
 struct Dims {
   int n, h, d, dv, k, C, M;
@@ -53,7 +54,8 @@ struct Work {
   __nv_bfloat16* Wt; // [3][M*2][n][Cpad]  key-step weights, sub-key major, bf16 pieces
   __nv_bfloat16* Qt; // [M*2][h][qt_T]     half-queries, feature major (operand B of the key step)
   int qt_T;          // token columns of Qt (a multiple of 64)
-  float* wsum_part;  // [M*2][Cpad/64][n]  per-token-tile sums of W
+  float* wsum_part;  // [M*2][Cpad/16][n]  per-16-token-block sums of W
+  int* pbar_cnt;     // [M*2][ceil(n/256)] arrival counters of the pbar column blocks (zero between launches)
   // Every array above is memory-major except the bf16 pieces (Kpc, Wt), whose piece
   // stride is P_all problems; a Work for a group of memories is the same carve with its
   // pointers advanced to the group's first memory (see group_work).
@@ -142,10 +144,44 @@ int launch_topk_rows(const Dims& d, const Work& w, int wt0, int len, cudaStream_
 // Feature-major copy of both half-queries of `len` tokens into Qt columns qt0.. (the key
 // step's B operand).
 int launch_qtrans(const Dims& d, const Work& w, const void* q, long long q_stride, int qt0, int len, cudaStream_t s);
-// Entropy key step from Dfull/zpart (tensor-core path).  The chunk's half-queries are read
-// from Qt columns qt_t0..; qt_t0 < 0: transpose them first into columns 0.. .
-int launch_tc_address(const Dims& d, const Work& w, float* K1, float* K2, const void* q, long long q_stride, int len,
+// Entropy key step from Dfull/zpart (tensor-core path), in three launches: pbar (Z,
+// column sums, lp), wbuild (L_t and the bf16 pieces of W), keystep (the GEMM and the key
+// update).  The chunk's half-queries are read from Qt columns qt_t0..; qt_t0 < 0:
+// keystep transposes them first into columns 0.. .
+int launch_tc_pbar(const Dims& d, const Work& w, int len, cudaStream_t s);
+int launch_tc_wbuild(const Dims& d, const Work& w, int len, cudaStream_t s);
+int launch_tc_keystep(const Dims& d, const Work& w, float* K1, float* K2, const void* q, long long q_stride, int len,
                       int qt_t0, cudaStream_t s);
+
+// ---- launches ----
+// Whether kernels are launched with programmatic dependent launch (default on; the
+// environment variable FWPKM_NO_PDL=1 turns it off for comparisons).
+bool pdl_enabled();
+
+// Launch `kern` on `s`, allowing it to start while the previous kernel of the same stream
+// finishes (programmatic stream serialization).  Every kernel launched this way calls
+// pdl_wait() before it touches memory that an earlier kernel writes, so the overlap
+// covers only its launch and set-up.
+template <typename... KArgs, typename... Args>
+inline void launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// Device side of programmatic dependent launch: wait until the preceding kernel of the
+// stream has completed and its writes are visible (a no-op without a programmatic
+// dependency), then let the next kernel of the stream begin its launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---- small device helpers ----
 __device__ __forceinline__ float load_qv(const float* p, long long i) { return p[i]; }

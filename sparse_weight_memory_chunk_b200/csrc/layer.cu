@@ -5,7 +5,7 @@
 //
 // Because RMSNorm is a per-row scale times a per-feature weight,
 //   Linear(RMSNorm(x)) = (1/rms(x)) * (x (gamma . W)^T) + b,
-// so gamma is folded into W once (fp32 product, kept as bf16 pieces hi + lo) and 1/rms
+// so gamma is folded into W once (fp32 product, kept as bf16 pieces) and 1/rms
 // scales the tensor-core accumulator in the GEMM epilogue.  The input side is one
 // row-statistics pass over h (1/rms and the gate's dot product; the gate is a single
 // output column, so it never reaches the tensor cores) and one GEMM whose epilogue writes
@@ -20,10 +20,10 @@ using namespace fwpkm;
 
 struct fwpkm_layer {
   fwpkm_layer_config cfg;
-  __nv_bfloat16* Wqv;   // [2][d + d_v][d_model]  folded q and v weights, bf16 pieces
+  __nv_bfloat16* Wqv;   // [3][d + d_v][d_model]  folded q and v weights, bf16 pieces
   float* wg;            // [d_model]              folded gate weights (fp32)
   float* bqv;           // [d + d_v]              q and v biases
-  __nv_bfloat16* Wo;    // [2][d_model][d_v]      folded output weights, bf16 pieces
+  __nv_bfloat16* Wo;    // [3][d_model][d_v]      folded output weights, bf16 pieces
   float* bo;            // [d_model]              output bias
   float* inv_rms;       // [max_rows]             per-row 1/rms scratch
   __nv_bfloat16* opc;   // [2][max_rows][d_v]     bf16 pieces of o
@@ -48,10 +48,10 @@ size_t layer_carve(const fwpkm_layer_config& c, fwpkm_layer* L, char* base) {
     return p;
   };
   int* status = (int*)take(sizeof(int));
-  __nv_bfloat16* Wqv = (__nv_bfloat16*)take(2 * 2 * nqv * D);
+  __nv_bfloat16* Wqv = (__nv_bfloat16*)take(2 * 3 * nqv * D);
   float* wg = (float*)take(4 * D);
   float* bqv = (float*)take(4 * nqv);
-  __nv_bfloat16* Wo = (__nv_bfloat16*)take(2 * 2 * D * dv);
+  __nv_bfloat16* Wo = (__nv_bfloat16*)take(2 * 3 * D * dv);
   float* bo = (float*)take(4 * D);
   float* inv = (float*)take(4 * R);
   __nv_bfloat16* opc = (__nv_bfloat16*)take(2 * 2 * R * dv);
@@ -87,8 +87,8 @@ fwpkm_status cuda_status() {
 
 namespace fwpkm {
 
-// W' = gamma[e] * W[j][e] in fp32, stored as bf16 pieces hi (and lo = W' - hi when
-// pieces == 2) at dst[piece][row0 + j][e].
+// W' = gamma[e] * W[j][e] in fp32, stored as `pieces` bf16 pieces at dst[piece][row0 + j][e]:
+// hi = bf16(W'), then mid = bf16(W' - hi), lo = bf16(W' - hi - mid) (~24 significant bits).
 __global__ void __launch_bounds__(LAYER_THREADS)
 fold_weights_kernel(const __nv_bfloat16* __restrict__ W, const float* __restrict__ gamma, int rows, int cols,
                     __nv_bfloat16* __restrict__ dst, long long piece_stride, int row0, int pieces) {
@@ -99,7 +99,12 @@ fold_weights_kernel(const __nv_bfloat16* __restrict__ W, const float* __restrict
   const __nv_bfloat16 hi = __float2bfloat16_rn(w);
   const size_t o = (size_t)(row0 + j) * cols + e;
   dst[o] = hi;
-  if (pieces == 2) dst[piece_stride + o] = __float2bfloat16_rn(w - __bfloat162float(hi));
+  if (pieces >= 2) {
+    const float r = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r);
+    dst[piece_stride + o] = mid;
+    if (pieces >= 3) dst[2 * piece_stride + o] = __float2bfloat16_rn(r - __bfloat162float(mid));
+  }
 }
 
 __global__ void __launch_bounds__(LAYER_THREADS)
@@ -223,9 +228,10 @@ fwpkm_status fwpkm_layer_set_params(fwpkm_layer* L, const fwpkm_layer_params* p,
   const fwpkm_layer_config& c = L->cfg;
   cudaStream_t s = (cudaStream_t)stream;
   const int D = c.d_model, nqv = c.d + c.d_v;
-  // one piece suffices when no norm weight is folded in (W is exact in bf16); the q and
-  // v weights share one GEMM, so they share its piece count
-  L->qv_pieces = (p->gamma_q || p->gamma_v) ? 2 : 1;
+  // one piece suffices when no norm weight is folded in (W is exact in bf16); else three
+  // pieces carry the fp32 product.  The q and v weights share one GEMM and its piece
+  // count; the output GEMM's result is rounded to bf16, so two pieces are enough there.
+  L->qv_pieces = (p->gamma_q || p->gamma_v) ? 3 : 1;
   L->o_pieces = p->gamma_o ? 2 : 1;
   const long long qv_ps = (long long)nqv * D, o_ps = (long long)D * c.d_v;
   auto blocks = [](long long n) { return (unsigned)((n + LAYER_THREADS - 1) / LAYER_THREADS); };
@@ -257,7 +263,7 @@ fwpkm_status fwpkm_layer_in(fwpkm_layer* L, const void* h, int rows, void* q, vo
                                                            L->b_g, L->inv_rms, g);
   CUtensorMap A, B;
   if (!make_tmap_bf16_3d(&A, h, D, rows, 1, (uint64_t)D * 2, (uint64_t)rows * D * 2)) return FWPKM_ERR_CUDA;
-  if (!make_tmap_bf16_3d(&B, L->Wqv, D, nqv, 2, (uint64_t)D * 2, (uint64_t)nqv * D * 2)) return FWPKM_ERR_CUDA;
+  if (!make_tmap_bf16_3d(&B, L->Wqv, D, nqv, 3, (uint64_t)D * 2, (uint64_t)nqv * D * 2)) return FWPKM_ERR_CUDA;
   TcGemm t = {};
   t.P = 1; t.k_blocks = D / 64; t.n_tiles = (nqv + 127) / 128; t.tiles_per_cta = 2;
   t.a_pieces = 1; t.b_pieces = L->qv_pieces;
@@ -285,7 +291,7 @@ fwpkm_status fwpkm_layer_out(fwpkm_layer* L, const float* o, int rows, void* o_o
   rms_split_kernel<<<(rows + 7) / 8, LAYER_THREADS, 0, s>>>(o, rows, dv, c.eps_rms, L->inv_rms, L->opc, ops);
   CUtensorMap A, B;
   if (!make_tmap_bf16_3d(&A, L->opc, dv, rows, 2, (uint64_t)dv * 2, (uint64_t)ops * 2)) return FWPKM_ERR_CUDA;
-  if (!make_tmap_bf16_3d(&B, L->Wo, dv, D, 2, (uint64_t)dv * 2, (uint64_t)D * dv * 2)) return FWPKM_ERR_CUDA;
+  if (!make_tmap_bf16_3d(&B, L->Wo, dv, D, 3, (uint64_t)dv * 2, (uint64_t)D * dv * 2)) return FWPKM_ERR_CUDA;
   TcGemm t = {};
   t.P = 1; t.k_blocks = dv / 64; t.n_tiles = (D + 127) / 128; t.tiles_per_cta = 4;
   t.a_pieces = 2; t.b_pieces = L->o_pieces;

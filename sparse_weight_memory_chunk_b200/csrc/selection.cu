@@ -1,4 +1,4 @@
-// select.cu -- restricted Cartesian top-k with softmax weights, and the per-chunk
+// selection.cu -- restricted Cartesian top-k with softmax weights, and the per-chunk
 // (slot, token) sort that drives the atomic-free write.
 //
 // Fast-weight Product Key Memory (rainbus summary), PKM prerequisite and method
@@ -33,6 +33,8 @@ __device__ __forceinline__ void sort_cand(u64* cand, int lane) {
 
 __global__ void __launch_bounds__(CART_WARPS * 32)
 cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float s_sig[CART_WARPS][2][32];
   __shared__ int s_sub[CART_WARPS][2][32];
   __shared__ u64 s_cand[CART_WARPS][128];
@@ -112,7 +114,7 @@ int launch_cartesian(const Dims& d, const Work& w, int wt0, int len, int32_t* id
                      cudaStream_t s) {
   if (len <= 0) return 0;
   dim3 grid((len + CART_WARPS - 1) / CART_WARPS, d.M);
-  cartesian_kernel<<<grid, CART_WARPS * 32, 0, s>>>(d, w, wt0, len, idx_out, w_out);
+  launch_k(cartesian_kernel, grid, CART_WARPS * 32, 0, s, d, w, wt0, len, idx_out, w_out);
   return 1;
 }
 
@@ -142,6 +144,8 @@ constexpr int SORT_BUCKET_CAP = 128;   // largest bucket the ranking path handle
 template <int VPT>
 __global__ void __launch_bounds__(SORT_THREADS)
 sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ u64 s_keys[];
   __shared__ int s_cnt[512], s_off[513], s_cur[512];
   __shared__ int s_max;
@@ -265,13 +269,13 @@ int launch_sort_pairs(const Dims& d, const Work& w, int wt0, int total_len, bool
     while (Ppad < P) Ppad <<= 1;
     const size_t smem = sizeof(u64) * (size_t)Ppad;
     cudaFuncSetAttribute(sort_pairs_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    sort_pairs_kernel<8><<<grid, SORT_THREADS, smem, s>>>(d, w, wt0, total_len, last_has_target ? 1 : 0);
+    launch_k(sort_pairs_kernel<8>, grid, SORT_THREADS, smem, s, d, w, wt0, total_len, last_has_target ? 1 : 0);
   } else {
     int Ppad = 512;
     while (Ppad < P) Ppad <<= 1;
     const size_t smem = sizeof(u64) * (size_t)Ppad;
     cudaFuncSetAttribute(sort_pairs_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    sort_pairs_kernel<16><<<grid, SORT_THREADS, smem, s>>>(d, w, wt0, total_len, last_has_target ? 1 : 0);
+    launch_k(sort_pairs_kernel<16>, grid, SORT_THREADS, smem, s, d, w, wt0, total_len, last_has_target ? 1 : 0);
   }
   return 1;
 }

@@ -1,4 +1,4 @@
-// tc_gemm.cu -- the two dense contractions of the hot path on the 5th-generation tensor
+// tc_gemm.cu -- the dense contractions of the hot path on the 5th-generation tensor
 // cores (tcgen05.mma, TMEM accumulators, TMA-fed 128-byte-swizzled tiles).
 //
 //  * scoring (Fast-weight Product Key Memory (paperlayer summary) §2.2, §A.2):
@@ -8,6 +8,9 @@
 //  * entropy key step ((rainbus summary) method step 5; (paperlayer summary) §3.4):
 //      G[b][e] = sum_t W[t][b] q_t[e]; epilogue applies K[b] -= lr * 2 (G[b] - Wsum[b] K[b])
 //      and refreshes the bf16 pieces and squared norms of the new keys.
+//  * slow-weight projections ((rainbus summary) method steps 1 and 3, see layer.cu):
+//      y[r][c] = (1/rms_r) sum_e x[r][e] W'[c][e] + b[c]; the epilogue applies the
+//      per-row scale and the bias and writes fp32 or bf16.
 //
 // Precision: q and v are bf16 (exact); fp32 operands (keys, W) enter as three bf16 pieces
 // hi + mid + lo (~24 significant bits), each piece pair accumulating into one fp32 TMEM
@@ -98,6 +101,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // barriers and TMEM are set up; from here on the CTA reads what earlier kernels wrote
+  pdl_wait();
+  pdl_trigger();
   const uint64_t deadline = globaltimer() + TC_TIMEOUT_NS;
   int issued = 0;  // producer: loads issued
 
@@ -356,7 +362,7 @@ int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g, 
   const size_t smem = tc_smem_bytes(g.a_pieces + g.b_pieces);
   cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((g.n_tiles + g.tiles_per_cta - 1) / g.tiles_per_cta, m_tiles, g.P);
-  tc_gemm_kernel<<<grid, TC_THREADS, smem, s>>>(A, B, g);
+  launch_k(tc_gemm_kernel, grid, TC_THREADS, smem, s, A, B, g);
   return 1;
 }
 

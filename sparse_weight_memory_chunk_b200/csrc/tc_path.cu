@@ -26,6 +26,8 @@ __device__ __forceinline__ void split3_bf16(float x, __nv_bfloat16& hi, __nv_bfl
 // ||q_half||^2 per (memory, half, token): one warp per token, both halves.
 __global__ void __launch_bounds__(TP_THREADS)
 qnorm_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long q_stride, int wt0, int len) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * (TP_THREADS / 32) + warp;
   const int m = blockIdx.y;
@@ -46,6 +48,8 @@ qnorm_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long q_s
 // in order (the key-step GEMM epilogue uses the same order, so both give the same bits).
 __global__ void __launch_bounds__(TP_THREADS)
 keyprep_kernel(Dims dm, Work w, const float* __restrict__ K1, const float* __restrict__ K2) {
+  pdl_wait();
+  pdl_trigger();
   const int P = dm.M * 2;
   const long long idx = (long long)blockIdx.x * TP_THREADS + threadIdx.x;
   if (idx >= (long long)P * dm.n) return;
@@ -75,10 +79,15 @@ keyprep_kernel(Dims dm, Work w, const float* __restrict__ K1, const float* __res
   w.kn[(size_t)p * dm.n + b] = ((part[0] + part[1]) + part[2]) + part[3];
 }
 
-// Partial column sums sum_t w[t][a] / Z_t over one token slice; also Z_t itself.
+// Partial column sums sum_t w[t][a] / Z_t over one token slice; also Z_t itself.  The
+// last of the PBAR_SLICES blocks of a column block to finish (arrival counter, reset by
+// that block) adds the slices in slice order and writes lp = log(pbar).
 __global__ void __launch_bounds__(TP_THREADS)
 tc_pbar_kernel(Dims dm, Work w, int len) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float s_invz[1024 / PBAR_SLICES + 1];
+  __shared__ int s_last;
   const int p = blockIdx.y, sl = blockIdx.z;
   const int t0 = (sl * len) / PBAR_SLICES, t1 = ((sl + 1) * len) / PBAR_SLICES;
   const int nt = (dm.n + 127) / 128 * 4;  // 4 column groups per 128-column tile
@@ -91,92 +100,93 @@ tc_pbar_kernel(Dims dm, Work w, int len) {
   }
   __syncthreads();
   const int a = blockIdx.x * TP_THREADS + threadIdx.x;
-  if (a >= dm.n) return;
-  const float* D = w.Dfull + (size_t)p * w.drows * dm.n;
-  float s = 0.f;
+  const bool av = a < dm.n;
+  if (av) {
+    const float* D = w.Dfull + (size_t)p * w.drows * dm.n;
+    float s = 0.f;
 #pragma unroll 8
-  for (int t = t0; t < t1; ++t) s += __fdividef(1.f, dm.eps_idw + D[(size_t)t * dm.n + a]) * s_invz[t - t0];
-  w.ppart[((size_t)p * PBAR_SLICES + sl) * dm.n + a] = s;
+    for (int t = t0; t < t1; ++t) s += __fdividef(1.f, dm.eps_idw + D[(size_t)t * dm.n + a]) * s_invz[t - t0];
+    w.ppart[((size_t)p * PBAR_SLICES + sl) * dm.n + a] = s;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int* c = w.pbar_cnt + (size_t)p * gridDim.x + blockIdx.x;
+    const int prev = atomicAdd(c, 1);
+    s_last = prev == PBAR_SLICES - 1;
+    if (s_last) *c = 0;  // every slice has arrived: ready for the next launch
+  }
+  __syncthreads();
+  if (s_last && av) {
+    __threadfence();
+    float s = 0.f;
+    for (int k = 0; k < PBAR_SLICES; ++k) s += __ldcg(w.ppart + ((size_t)p * PBAR_SLICES + k) * dm.n + a);
+    w.lp[(size_t)p * dm.n + a] = logf(s / (float)len);
+  }
 }
 
-__global__ void __launch_bounds__(TP_THREADS)
-tc_lp_kernel(Dims dm, Work w, int len) {
-  const long long idx = (long long)blockIdx.x * TP_THREADS + threadIdx.x;
-  if (idx >= (long long)dm.M * 2 * dm.n) return;
-  const int p = (int)(idx / dm.n), a = (int)(idx - (long long)p * dm.n);
-  float s = 0.f;
-  for (int sl = 0; sl < PBAR_SLICES; ++sl) s += w.ppart[((size_t)p * PBAR_SLICES + sl) * dm.n + a];
-  w.lp[idx] = logf(s / (float)len);
-}
-
-// L_t = sum_a P[t][a] log pbar[a]: one warp per (problem, token).
-__global__ void __launch_bounds__(TP_THREADS)
-tc_rowL_kernel(Dims dm, Work w, int len) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (TP_THREADS / 32) + warp;
-  const int p = blockIdx.y;
-  if (t >= len) return;
-  const float* D = w.Dfull + ((size_t)p * w.drows + t) * dm.n;
-  const float* lp = w.lp + (size_t)p * dm.n;
-  float s = 0.f;
-#pragma unroll 8
-  for (int a = lane; a < dm.n; a += 32) s += __fdividef(lp[a], dm.eps_idw + D[a]);
-  s = warp_sum(s);
-  if (lane == 0) w.Lt[(size_t)p * dm.C + t] = s / w.Z[(size_t)p * dm.C + t];
-}
-
-// W for a 64-token x 64-sub-key tile, written sub-key major as three bf16 pieces (the
-// A operand of the key-step GEMM), plus the tile's per-sub-key sum of W.
+// W for a block of WB_T tokens and every sub-key, written sub-key major as three bf16
+// pieces (the A operand of the key-step GEMM), plus the block's per-sub-key sum of W.
+// First L_t = sum_a P[t][a] lp[a] = (sum_a lp[a] w[t][a]) / Z_t for the block's tokens (one
+// warp per token), then W[t][b] = (1/len) (w/Z_t) (lp[b] - L_t) w with one thread per
+// sub-key (the rows are re-read from L1/L2).
+constexpr int WB_T = 16;
 __global__ void __launch_bounds__(TP_THREADS)
 tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
-  __shared__ float s_W[64][65];
-  __shared__ float s_invz[64], s_L[64], s_lp[64];
-  const int p = blockIdx.z;
-  const int b0 = blockIdx.x * 64, t0 = blockIdx.y * 64;
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float s_invz[WB_T], s_L[WB_T];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p = blockIdx.y, t0 = blockIdx.x * WB_T;
   const int n = dm.n;
-  const int tid = threadIdx.x;
-  if (tid < 64) {
-    const int t = t0 + tid;
-    s_invz[tid] = t < len ? 1.f / w.Z[(size_t)p * dm.C + t] : 0.f;
-    s_L[tid] = t < len ? w.Lt[(size_t)p * dm.C + t] : 0.f;
-  } else if (tid < 128) {
-    const int b = b0 + tid - 64;
-    s_lp[tid - 64] = b < n ? w.lp[(size_t)p * n + b] : 0.f;
+  const float* D = w.Dfull + (size_t)p * w.drows * n;
+  const float* lp = w.lp + (size_t)p * n;
+  for (int tl = warp; tl < WB_T; tl += TP_THREADS / 32) {
+    const int t = t0 + tl;
+    float L = 0.f, iz = 0.f;
+    if (t < len) {
+      const float* Dr = D + (size_t)t * n;
+      float s = 0.f;
+#pragma unroll 8
+      for (int a = lane; a < n; a += 32) s += __fdividef(lp[a], dm.eps_idw + Dr[a]);
+      s = warp_sum(s);
+      const float z = w.Z[(size_t)p * dm.C + t];
+      L = s / z;
+      iz = 1.f / z;
+    }
+    if (lane == 0) {
+      s_L[tl] = L;
+      s_invz[tl] = iz;
+    }
   }
   __syncthreads();
   const float inv_len = 1.f / (float)len;
-  const float* D = w.Dfull + (size_t)p * w.drows * n;
-#pragma unroll 4
-  for (int idx = tid; idx < 64 * 64; idx += TP_THREADS) {
-    const int tl = idx >> 6, bl = idx & 63;
-    const int t = t0 + tl, b = b0 + bl;
-    float W = 0.f;
-    if (t < len && b < n) {
-      const float wv = __fdividef(1.f, dm.eps_idw + D[(size_t)t * n + b]);
-      const float P_ = wv * s_invz[tl];
-      W = inv_len * P_ * (s_lp[bl] - s_L[tl]) * wv;
-    }
-    s_W[bl][tl] = W;
-  }
-  __syncthreads();
-  const int ntt = gridDim.y;
-  if (tid < 64 && b0 + tid < n) {
-    float s = 0.f;
-    for (int tl = 0; tl < 64; ++tl) s += s_W[tid][tl];
-    w.wsum_part[((size_t)p * ntt + blockIdx.y) * n + b0 + tid] = s;
-  }
   const size_t pstride = (size_t)w.P_all * n * cpad;
-  for (int idx = tid; idx < 64 * 8; idx += TP_THREADS) {
-    const int bl = idx >> 3, c8 = idx & 7;
-    const int b = b0 + bl;
-    if (b >= n) continue;
-    __align__(16) __nv_bfloat16 hi[8], mid[8], lo[8];
+  const int ntb = gridDim.x;
+  for (int b = threadIdx.x; b < n; b += TP_THREADS) {
+    const float lpb = lp[b];
+    __align__(16) __nv_bfloat16 hi[WB_T], mid[WB_T], lo[WB_T];
+    float wsum = 0.f;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) split3_bf16(s_W[bl][c8 * 8 + u], hi[u], mid[u], lo[u]);
-    __nv_bfloat16* dst = w.Wt + ((size_t)p * n + b) * cpad + t0 + c8 * 8;
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(hi);
-    *reinterpret_cast<uint4*>(dst + pstride) = *reinterpret_cast<uint4*>(mid);
-    *reinterpret_cast<uint4*>(dst + 2 * pstride) = *reinterpret_cast<uint4*>(lo);
+    for (int tl = 0; tl < WB_T; ++tl) {
+      const int t = t0 + tl;
+      float W = 0.f;
+      if (t < len) {
+        const float wv = __fdividef(1.f, dm.eps_idw + D[(size_t)t * n + b]);
+        const float P_ = wv * s_invz[tl];
+        W = inv_len * P_ * (lpb - s_L[tl]) * wv;
+      }
+      wsum += W;
+      split3_bf16(W, hi[tl], mid[tl], lo[tl]);
+    }
+    w.wsum_part[((size_t)p * ntb + blockIdx.x) * n + b] = wsum;
+    __nv_bfloat16* dst = w.Wt + ((size_t)p * n + b) * cpad + t0;
+#pragma unroll
+    for (int h8 = 0; h8 < WB_T / 8; ++h8) {
+      *reinterpret_cast<uint4*>(dst + h8 * 8) = *reinterpret_cast<uint4*>(hi + h8 * 8);
+      *reinterpret_cast<uint4*>(dst + pstride + h8 * 8) = *reinterpret_cast<uint4*>(mid + h8 * 8);
+      *reinterpret_cast<uint4*>(dst + 2 * pstride + h8 * 8) = *reinterpret_cast<uint4*>(lo + h8 * 8);
+    }
   }
 }
 
@@ -186,6 +196,8 @@ tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
 // key-step GEMM multiplies them by zero-filled weights).
 __global__ void __launch_bounds__(TP_THREADS)
 qtrans_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long q_stride, int qt0, int len) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ __align__(16) __nv_bfloat16 s_q[64][128 + 8];
   const int p = blockIdx.y, m = p >> 1, j = p & 1;
   const int t0 = blockIdx.x * 64, h = dm.h, h8 = h / 8;
@@ -212,13 +224,13 @@ qtrans_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long q_
 int launch_qnorm(const Dims& d, const Work& w, const void* q, long long q_stride, int wt0, int len, cudaStream_t s) {
   if (len <= 0) return 0;
   dim3 grid((len + 7) / 8, d.M);
-  qnorm_kernel<<<grid, TP_THREADS, 0, s>>>(d, w, (const __nv_bfloat16*)q, q_stride, wt0, len);
+  launch_k(qnorm_kernel, grid, TP_THREADS, 0, s, d, w, (const __nv_bfloat16*)q, q_stride, wt0, len);
   return 1;
 }
 
 int launch_keyprep(const Dims& d, const Work& w, const float* K1, const float* K2, cudaStream_t s) {
   const long long rows = (long long)d.M * 2 * d.n;
-  keyprep_kernel<<<(unsigned)((rows + TP_THREADS - 1) / TP_THREADS), TP_THREADS, 0, s>>>(d, w, K1, K2);
+  launch_k(keyprep_kernel, (unsigned)((rows + TP_THREADS - 1) / TP_THREADS), TP_THREADS, 0, s, d, w, K1, K2);
   return 1;
 }
 
@@ -250,27 +262,38 @@ int launch_tc_score(const Dims& d, const Work& w, const void* q_base, long long 
 
 int launch_qtrans(const Dims& d, const Work& w, const void* q, long long q_stride, int qt0, int len, cudaStream_t s) {
   if (len <= 0) return 0;
-  qtrans_kernel<<<dim3((len + 63) / 64, d.M * 2), TP_THREADS, 0, s>>>(d, w, (const __nv_bfloat16*)q, q_stride, qt0,
+  launch_k(qtrans_kernel, dim3((len + 63) / 64, d.M * 2), TP_THREADS, 0, s, d, w, (const __nv_bfloat16*)q, q_stride, qt0,
                                                                        len);
   return 1;
 }
 
-int launch_tc_address(const Dims& d, const Work& w, float* K1, float* K2, const void* q, long long q_stride, int len,
+int launch_tc_pbar(const Dims& d, const Work& w, int len, cudaStream_t s) {
+  if (len <= 0) return 0;
+  launch_k(tc_pbar_kernel, dim3((d.n + TP_THREADS - 1) / TP_THREADS, d.M * 2, PBAR_SLICES), TP_THREADS, 0, s, d, w,
+           len);
+  return 1;
+}
+
+int launch_tc_wbuild(const Dims& d, const Work& w, int len, cudaStream_t s) {
+  if (len <= 0) return 0;
+  const int cpad = (d.C + 63) / 64 * 64;
+  launch_k(tc_wbuild_kernel, dim3((len + WB_T - 1) / WB_T, d.M * 2), TP_THREADS, 0, s, d, w, len, cpad);
+  return 1;
+}
+
+int launch_tc_keystep(const Dims& d, const Work& w, float* K1, float* K2, const void* q, long long q_stride, int len,
                       int qt_t0, cudaStream_t s) {
   if (len <= 0) return 0;
   const int P = d.M * 2;
   const int cpad = (d.C + 63) / 64 * 64;
   const int ntt = (len + 63) / 64;
-  int launched = 5;
+  const int ntb = (len + WB_T - 1) / WB_T;
+  int launched = 1;
   if (qt_t0 < 0) {
     launch_qtrans(d, w, q, q_stride, 0, len, s);
     qt_t0 = 0;
     ++launched;
   }
-  tc_pbar_kernel<<<dim3((d.n + TP_THREADS - 1) / TP_THREADS, P, PBAR_SLICES), TP_THREADS, 0, s>>>(d, w, len);
-  tc_lp_kernel<<<(unsigned)(((long long)P * d.n + TP_THREADS - 1) / TP_THREADS), TP_THREADS, 0, s>>>(d, w, len);
-  tc_rowL_kernel<<<dim3((len + 7) / 8, P), TP_THREADS, 0, s>>>(d, w, len);
-  tc_wbuild_kernel<<<dim3((d.n + 63) / 64, ntt, P), TP_THREADS, 0, s>>>(d, w, len, cpad);
   CUtensorMap A, B;
   if (!make_tmap_bf16_3d(&A, w.Wt, len, d.n, 2 * w.P_all + P, (uint64_t)cpad * 2, (uint64_t)d.n * cpad * 2))
     return -1;
@@ -285,7 +308,7 @@ int launch_tc_address(const Dims& d, const Work& w, float* K1, float* K2, const 
   g.m_valid = d.n; g.n_valid = d.h;
   g.epi = TC_EPI_KEYSTEP;
   g.K1 = K1; g.K2 = K2; g.Kpc = w.Kpc; g.kn = w.kn; g.piece_P = w.P_all;
-  g.wsum_part = w.wsum_part; g.wsum_tiles = ntt; g.lr = d.lr_key;
+  g.wsum_part = w.wsum_part; g.wsum_tiles = ntb; g.lr = d.lr_key;
   g.status = w.status;
   launch_tc_gemm(A, B, g, (d.n + 127) / 128, s);
   return launched;

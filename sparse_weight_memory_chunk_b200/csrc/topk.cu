@@ -40,6 +40,8 @@ __device__ __forceinline__ float warp_sort32(float x, int lane) {
 template <int NPL>
 __global__ void __launch_bounds__(TK_THREADS, 3)
 topk_rows_kernel(Dims dm, Work w, int wt0, int len) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ u64 s_cand[TK_THREADS / 32][128];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * (TK_THREADS / 32) + warp;
@@ -154,13 +156,13 @@ int launch_topk_rows(const Dims& d, const Work& w, int wt0, int len, cudaStream_
   if (len <= 0) return 0;
   dim3 grid((len + 7) / 8, d.M * 2);
   const int npl = (d.n + 31) / 32;
-  if (npl <= 2) topk_rows_kernel<2><<<grid, TK_THREADS, 0, s>>>(d, w, wt0, len);
-  else if (npl <= 4) topk_rows_kernel<4><<<grid, TK_THREADS, 0, s>>>(d, w, wt0, len);
-  else if (npl <= 8) topk_rows_kernel<8><<<grid, TK_THREADS, 0, s>>>(d, w, wt0, len);
-  else if (npl <= 16) topk_rows_kernel<16><<<grid, TK_THREADS, 0, s>>>(d, w, wt0, len);
-  else if (npl <= 32) topk_rows_kernel<32><<<grid, TK_THREADS, 0, s>>>(d, w, wt0, len);
-  else if (npl <= 64) topk_rows_kernel<64><<<grid, TK_THREADS, 0, s>>>(d, w, wt0, len);
-  else topk_rows_kernel<128><<<grid, TK_THREADS, 0, s>>>(d, w, wt0, len);
+  if (npl <= 2) launch_k(topk_rows_kernel<2>, grid, TK_THREADS, 0, s, d, w, wt0, len);
+  else if (npl <= 4) launch_k(topk_rows_kernel<4>, grid, TK_THREADS, 0, s, d, w, wt0, len);
+  else if (npl <= 8) launch_k(topk_rows_kernel<8>, grid, TK_THREADS, 0, s, d, w, wt0, len);
+  else if (npl <= 16) launch_k(topk_rows_kernel<16>, grid, TK_THREADS, 0, s, d, w, wt0, len);
+  else if (npl <= 32) launch_k(topk_rows_kernel<32>, grid, TK_THREADS, 0, s, d, w, wt0, len);
+  else if (npl <= 64) launch_k(topk_rows_kernel<64>, grid, TK_THREADS, 0, s, d, w, wt0, len);
+  else launch_k(topk_rows_kernel<128>, grid, TK_THREADS, 0, s, d, w, wt0, len);
   return 1;
 }
 

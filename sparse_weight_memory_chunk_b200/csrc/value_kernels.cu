@@ -1,4 +1,4 @@
-// value.cu -- the HBM-bound value path: sparse read + gated output, reconstruction
+// value_kernels.cu -- the HBM-bound value path: sparse read + gated output, reconstruction
 // residuals, and the atomic-free fast-weight write.
 //
 // Fast-weight Product Key Memory (rainbus summary), method steps 2-4:
@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(VAL_WARPS * 32)
 gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict__ v,
               const float* __restrict__ g, long long stride, int wt0, int len, float* __restrict__ o,
               int fuse_resid, const VT* __restrict__ v_next) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * VAL_WARPS + warp;
   const int m = blockIdx.y;
@@ -161,6 +163,8 @@ template <typename VT, int VPL>
 __global__ void __launch_bounds__(VAL_WARPS * 32)
 resid_kernel(Dims dm, Work w, const VT* __restrict__ v, const float* __restrict__ g, long long stride,
              int len, const VT* __restrict__ v_next) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * VAL_WARPS + warp;
   const int m = blockIdx.y;
@@ -199,6 +203,8 @@ resid_kernel(Dims dm, Work w, const VT* __restrict__ v, const float* __restrict_
 template <int VPL, int G>
 __global__ void __launch_bounds__(VAL_WARPS * 32)
 write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = blockIdx.y;
   const int C = dm.C, k = dm.k, dv4 = dm.dv >> 2;
@@ -296,11 +302,11 @@ int launch_gather(const Dims& d, const Work& w, const float* V, const void* v, c
   if (len <= 0) return 0;
   dim3 grid((len + VAL_WARPS - 1) / VAL_WARPS, d.M);
   if (d.qv_bf16) {
-    FWPKM_VPL_DISPATCH(vpl_of(d.dv), gather_kernel<__nv_bfloat16, VPL><<<grid, VAL_WARPS * 32, 0, s>>>(
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(gather_kernel<__nv_bfloat16, VPL>, grid, VAL_WARPS * 32, 0, s, 
         d, w, V, (const __nv_bfloat16*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0,
         (const __nv_bfloat16*)v_next));
   } else {
-    FWPKM_VPL_DISPATCH(vpl_of(d.dv), gather_kernel<float, VPL><<<grid, VAL_WARPS * 32, 0, s>>>(
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(gather_kernel<float, VPL>, grid, VAL_WARPS * 32, 0, s, 
         d, w, V, (const float*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0, (const float*)v_next));
   }
   return 1;
@@ -311,10 +317,10 @@ int launch_resid(const Dims& d, const Work& w, const void* v, const float* g, lo
   if (len <= 0) return 0;
   dim3 grid((len + VAL_WARPS - 1) / VAL_WARPS, d.M);
   if (d.qv_bf16) {
-    FWPKM_VPL_DISPATCH(vpl_of(d.dv), resid_kernel<__nv_bfloat16, VPL><<<grid, VAL_WARPS * 32, 0, s>>>(
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(resid_kernel<__nv_bfloat16, VPL>, grid, VAL_WARPS * 32, 0, s, 
         d, w, (const __nv_bfloat16*)v, g, stride, len, (const __nv_bfloat16*)v_next));
   } else {
-    FWPKM_VPL_DISPATCH(vpl_of(d.dv), resid_kernel<float, VPL><<<grid, VAL_WARPS * 32, 0, s>>>(
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(resid_kernel<float, VPL>, grid, VAL_WARPS * 32, 0, s, 
         d, w, (const float*)v, g, stride, len, (const float*)v_next));
   }
   return 1;
@@ -325,10 +331,10 @@ int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s
   const int G = vpl <= 2 ? 4 : vpl == 4 ? 2 : 1;  // list positions per warp: ~8 float4 in flight per lane
   dim3 grid((d.C * d.k + VAL_WARPS * G - 1) / (VAL_WARPS * G), d.M);
   switch (vpl) {
-    case 1: write_kernel<1, 4><<<grid, VAL_WARPS * 32, 0, s>>>(d, w, V, wt0); break;
-    case 2: write_kernel<2, 4><<<grid, VAL_WARPS * 32, 0, s>>>(d, w, V, wt0); break;
-    case 4: write_kernel<4, 2><<<grid, VAL_WARPS * 32, 0, s>>>(d, w, V, wt0); break;
-    default: write_kernel<8, 1><<<grid, VAL_WARPS * 32, 0, s>>>(d, w, V, wt0); break;
+    case 1: launch_k(write_kernel<1, 4>, grid, VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
+    case 2: launch_k(write_kernel<2, 4>, grid, VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
+    case 4: launch_k(write_kernel<4, 2>, grid, VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
+    default: launch_k(write_kernel<8, 1>, grid, VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
   }
   return 1;
 }

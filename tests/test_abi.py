@@ -72,8 +72,8 @@ def test_layer_workspace_size_and_validation(lib):
     out = C.c_size_t(0)
     cfg = lib.LayerConfig(2048, 256, 256, 65536, 1e-6, 0)
     assert so.fwpkm_layer_workspace_size(C.byref(cfg), C.byref(out)) == lib.OK
-    # two bf16 pieces of both weight matrices + the per-row scratch of the output call
-    pieces = 2 * 2 * (512 * 2048 + 2048 * 256)
+    # three bf16 pieces of both weight matrices + the per-row scratch of the output call
+    pieces = 2 * 3 * (512 * 2048 + 2048 * 256)
     scratch = 4 * 65536 + 2 * 2 * 65536 * 256
     assert pieces + scratch <= out.value < pieces + scratch + (1 << 20)
     for bad, want in [((2048, 256, 256, 0, 1e-6), lib.ERR_INVALID_ARG), ((2000, 256, 256, 16, 1e-6), lib.ERR_UNSUPPORTED),

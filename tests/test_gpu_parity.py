@@ -48,8 +48,21 @@ def device_state(w, data, gcfg, max_T):
     return st, dev
 
 
+def workload_case(w):
+    """A benchmark workload at its full size, with the benchmark's own seed (same inputs)."""
+    q, v, g = gen_qvg(w)
+    K1, K2 = gen_keys(w)
+    V = np.stack([gen_values(w, m) for m in range(w.M)])
+    gcfg = fwpkm.make_config(w.n, w.d, w.d_v, w.k, w.C, w.M, w.qv == "bf16", key_update=w.key_update)
+    ocfg = oracle.make_cfg(w.n, w.d, w.d_v, w.k, w.C, key_update=w.key_update)
+    return w, (q, v, g, K1, K2, V), gcfg, ocfg
+
+
 def streaming_vs_oracle(name, **flags):
-    w, data, gcfg, ocfg = make_case(name, **flags)
+    return compare_streaming(name, *make_case(name, **flags))
+
+
+def compare_streaming(name, w, data, gcfg, ocfg):
     q, v, g, K1, K2, V = data
     M, T, C, k, dv, N = w.M, w.T, w.C, w.k, w.d_v, w.N
     st, dev = device_state(w, data, gcfg, C)
@@ -97,7 +110,8 @@ def streaming_vs_oracle(name, **flags):
                 rows = np.unique(np.concatenate([touched, rng.integers(0, N, 2048)]))
             Vg = dev["V"][m][torch.from_numpy(rows).cuda()].cpu().numpy()
             assert_close(Vg, V_orc[m][rows], f"{name} chunk@{t0} mem {m}: V")
-    return dict(o=o_d.cpu(), V=dev["V"].cpu(), K1=dev["K1"].cpu(), K2=dev["K2"].cpu(), ties=ties,
+    # full-size states stay on the device (8 GiB of V)
+    return dict(o=o_d.cpu(), V=dev["V"].cpu() if small else dev["V"], K1=dev["K1"].cpu(), K2=dev["K2"].cpu(), ties=ties,
                 w=w, data=data, gcfg=gcfg)
 
 
@@ -113,6 +127,25 @@ def test_streaming_matches_oracle_every_chunk(name):
     st.sync()
     assert torch.equal(o.cpu(), res["o"]), "run_sequence o differs from chunk-by-chunk"
     assert torch.equal(dev["V"].cpu(), res["V"]), "run_sequence V differs"
+    assert torch.equal(dev["K1"].cpu(), res["K1"]) and torch.equal(dev["K2"].cpu(), res["K2"])
+
+
+def test_paper_workload_full_size():
+    """The paper-scale workload at the benchmark's full size and seed (8 memories of
+    N = 1,048,576 slots, T = 4096, C = 256, key update on): every chunk's outputs, weights,
+    keys and sampled value rows against the oracle, then the benchmark's entry point
+    (fwpkm_run_sequence, one captured graph) bit-for-bit against the chunk-by-chunk run."""
+    from sparse_weight_memory_chunk_b200.inputs import WORKLOADS
+    w = WORKLOADS[3]
+    res = compare_streaming("paper_full", *workload_case(w))
+    print(f"paper full size: near-ties {res['ties']}")
+    data, gcfg = res["data"], res["gcfg"]
+    st, dev = device_state(w, data, gcfg, w.T)
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    st.run_sequence(dev["q"], dev["v"], dev["g"], o)
+    st.sync()
+    assert torch.equal(o.cpu(), res["o"]), "run_sequence o differs from chunk-by-chunk"
+    assert torch.equal(dev["V"], res["V"]), "run_sequence V differs from chunk-by-chunk"
     assert torch.equal(dev["K1"].cpu(), res["K1"]) and torch.equal(dev["K2"].cpu(), res["K2"])
 
 
