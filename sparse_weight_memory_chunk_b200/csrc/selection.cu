@@ -12,23 +12,27 @@ namespace fwpkm {
 // ---------------------------------------------------------------------------
 // Cartesian top-k: one warp per (memory, token).
 //
-// sigma_j = -log(eps + D_j) on the 2k survivors.  Each half is bitonic-sorted into
-// (sigma desc, sub-key asc) order; then a pair of ranks (i, j) can only be in the final
-// top-k if (i+1)(j+1) <= k, because every pair (i' <= i, j' <= j) scores at least as
-// high and wins exact ties on the slot index.  Those ~k ln k candidates are packed as
-// (score desc, slot asc) keys, bitonic-sorted, and the first k are the answer.  Weights
-// are the softmax of the k scores.
+// sigma_j = -log(eps + D_j) on the 2k survivors.  Each half must be in (sigma desc,
+// sub-key asc) order; the per-half top-k delivers its survivors by (D asc, sub-key asc),
+// which is that order unless two distances map to one sigma (or the logarithm's rounding
+// inverts a pair), so the warp checks neighbours and sorts only when the check fails.
+// Then a pair of ranks (i, j) can only be in the final top-k if (i+1)(j+1) <= k, because
+// every pair (i' <= i, j' <= j) scores at least as high and wins exact ties on the slot
+// index.  Those ~k ln k candidates (a table built once per CTA maps candidate c to its
+// (i, j)) are spread evenly over the lanes as (score desc, slot asc) keys,
+// bitonic-sorted, and the first k are the answer.  Weights are the softmax of the k
+// scores.
 // ---------------------------------------------------------------------------
 constexpr int CART_WARPS = 8;
 
 template <int VPT>
-__device__ __forceinline__ void sort_cand(u64* cand, int lane) {
-  u64 x[VPT];
+__device__ __forceinline__ void sort_cand(u64 (&x)[4], u64* cand, int lane) {
+  u64 y[VPT];
 #pragma unroll
-  for (int u = 0; u < VPT; ++u) x[u] = cand[lane * VPT + u];
-  warp_sort_asc<VPT>(x, lane);
+  for (int u = 0; u < VPT; ++u) y[u] = x[u];
+  warp_sort_asc<VPT>(y, lane);
 #pragma unroll
-  for (int u = 0; u < VPT; ++u) cand[lane * VPT + u] = x[u];
+  for (int u = 0; u < VPT; ++u) cand[lane * VPT + u] = y[u];
 }
 
 __global__ void __launch_bounds__(CART_WARPS * 32)
@@ -38,12 +42,28 @@ cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_ou
   __shared__ float s_sig[CART_WARPS][2][32];
   __shared__ int s_sub[CART_WARPS][2][32];
   __shared__ u64 s_cand[CART_WARPS][128];
+  __shared__ unsigned short s_tab[128];
+  __shared__ int s_total;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = dm.k, n = dm.n;
+  if (warp == 0) {
+    // staircase table: lane i owns rank i of half 1 and ranks 0 .. k/(i+1)-1 of half 2
+    const int rowlen = lane < k ? k / (lane + 1) : 0;
+    int incl = rowlen;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    for (int jj = 0; jj < rowlen; ++jj) s_tab[incl - rowlen + jj] = (unsigned short)((lane << 8) | jj);
+    if (lane == 31) s_total = incl;
+  }
+  __syncthreads();
   const int i_tok = blockIdx.x * CART_WARPS + warp;
   const int m = blockIdx.y;
   if (i_tok >= len) return;
-  const int k = dm.k, n = dm.n;
   const long long tok = (long long)wt0 + i_tok;
+  const int total = s_total;
 
   for (int j = 0; j < 2; ++j) {
     const size_t base = (((size_t)m * 2 + j) * w.max_T + tok) * k;
@@ -53,7 +73,8 @@ cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_ou
       const float sig = -logf(dm.eps_idw + w.Dsv[base + lane]);
       key[0] = ((u64)(~float_key(sig)) << 32) | (unsigned)sub;  // sigma desc, sub asc
     }
-    warp_sort_asc<1>(key, lane);
+    const u64 nxt = __shfl_down_sync(0xffffffffu, key[0], 1);
+    if (__any_sync(0xffffffffu, lane < 31 && nxt < key[0])) warp_sort_asc<1>(key, lane);
     if (lane < k) {
       s_sig[warp][j][lane] = key_float(~(uint32_t)(key[0] >> 32));
       s_sub[warp][j][lane] = (int)(key[0] & 0xffffffffu);
@@ -61,33 +82,34 @@ cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_ou
   }
   __syncwarp();
 
-  // staircase candidates: lane i owns rank i of half 1 and pairs it with ranks
-  // 0 .. k/(i+1)-1 of half 2
-  const int rowlen = lane < k ? k / (lane + 1) : 0;
-  int incl = rowlen;
+  u64 x[4];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  const int total = __shfl_sync(0xffffffffu, incl, 31);
-  u64* cand = s_cand[warp];
-  if (rowlen > 0) {
-    const float sig1 = s_sig[warp][0][lane];
-    const unsigned a = (unsigned)s_sub[warp][0][lane];
-    int pos = incl - rowlen;
-    for (int jj = 0; jj < rowlen; ++jj) {
-      const float S = sig1 + s_sig[warp][1][jj];
-      const unsigned slot = a * (unsigned)n + (unsigned)s_sub[warp][1][jj];
-      cand[pos + jj] = ((u64)(~float_key(S)) << 32) | slot;
+  for (int u = 0; u < 4; ++u) {
+    const int c = lane * 4 + u;
+    x[u] = ~0ull;
+    if (c < total) {
+      const int t = s_tab[c], i1 = t >> 8, i2 = t & 255;
+      const float S = s_sig[warp][0][i1] + s_sig[warp][1][i2];
+      const unsigned slot = (unsigned)s_sub[warp][0][i1] * (unsigned)n + (unsigned)s_sub[warp][1][i2];
+      x[u] = ((u64)(~float_key(S)) << 32) | slot;
     }
   }
+  // the sorts below take the elements lane * VPT + u, u < VPT: repack for VPT < 4
+  u64* cand = s_cand[warp];
   const int Sz = total <= 32 ? 32 : total <= 64 ? 64 : 128;
-  for (int jx = total + lane; jx < Sz; jx += 32) cand[jx] = ~0ull;
-  __syncwarp();
-  if (Sz == 32) sort_cand<1>(cand, lane);
-  else if (Sz == 64) sort_cand<2>(cand, lane);
-  else sort_cand<4>(cand, lane);
+  if (Sz == 128) {
+    sort_cand<4>(x, cand, lane);
+  } else {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) cand[lane * 4 + u] = x[u];
+    __syncwarp();
+    u64 y[4];
+    const int vpt = Sz / 32;
+    for (int u = 0; u < 4; ++u) y[u] = u < vpt ? cand[lane * vpt + u] : ~0ull;
+    __syncwarp();
+    if (Sz == 64) sort_cand<2>(y, cand, lane);
+    else sort_cand<1>(y, cand, lane);
+  }
   __syncwarp();
 
   float S = 0.f;
@@ -129,7 +151,7 @@ int launch_cartesian(const Dims& d, const Work& w, int wt0, int len, int32_t* id
 // bucket by their full key.
 //
 // SORT_SPLIT CTAs share one (memory, chunk): each counts all buckets (so all agree on
-// the bucket offsets), keeps the keys of its own quarter of the buckets in shared
+// the bucket offsets), keeps the keys of its own share of the buckets in shared
 // memory, and one warp per bucket ranks each key by comparing it with every other key
 // of the bucket and stores it at its rank.  The scatter into buckets may land keys in
 // any order; ranking by the full unique key makes the output independent of it.  If a
@@ -137,7 +159,7 @@ int launch_cartesian(const Dims& d, const Work& w, int wt0, int len, int32_t* id
 // keys with a register bitonic network instead and the others do nothing.
 // ---------------------------------------------------------------------------
 constexpr int SORT_THREADS = 1024;
-constexpr int SORT_SPLIT = 4;
+constexpr int SORT_SPLIT = 16;
 constexpr int SORT_BUCKET_KEYS = 64;   // average keys per bucket
 constexpr int SORT_BUCKET_CAP = 128;   // largest bucket the ranking path handles
 
@@ -177,8 +199,8 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
     u64 key = ~0ull;
     bk[u] = -1;
     if (i < P) {
-      const int t_local = i / k, r = i - t_local * k;
-      const unsigned slot = (unsigned)w.idx[((size_t)m * w.max_T + wt0 + tc0 + t_local) * k + r];
+      // pair i = t_local * k + r sits at offset i of the chunk's [C][k] slot block
+      const unsigned slot = (unsigned)w.idx[((size_t)m * w.max_T + wt0 + tc0) * k + i];
       key = ((u64)slot << 32) | (unsigned)i;
       bk[u] = NB > 1 ? (int)((slot * 2654435761u) >> (32 - nb_log2)) : 0;  // multiplicative hash
       atomicAdd(&s_cnt[bk[u]], 1);

@@ -11,6 +11,8 @@
 // Rows are moved as 16-byte vectors: a warp covers 512 contiguous bytes per load.  Both
 // kernels are bound by HBM latency x bytes in flight, so each warp keeps many row loads
 // outstanding before it consumes any of them.
+#include <mutex>
+
 #include "fwpkm_internal.cuh"
 
 namespace fwpkm {
@@ -208,75 +210,78 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = blockIdx.y;
   const int C = dm.C, k = dm.k, dv4 = dm.dv >> 2;
+  const int kshift = (k & (k - 1)) == 0 ? __popc(k - 1) : -1;  // t = pair / k by a shift when k is 2^s
   const int cslot = wt0 / C;
   const size_t cbase = (size_t)m * w.max_chunks + cslot;
   const int P = w.npairs[cbase];
-  const int pos0 = (blockIdx.x * VAL_WARPS + warp) * G;
-  if (pos0 >= P) return;
   const unsigned long long* sk = w.sk + cbase * (size_t)(C * k);
-  unsigned long long my_key = ~0ull;
-  bool head = false;
-  if (lane < G && pos0 + lane < P) {
-    const int pos = pos0 + lane;
-    my_key = sk[pos];
-    head = pos == 0 || (sk[pos - 1] >> 32) != (my_key >> 32);
-  }
-  const unsigned heads = __ballot_sync(0xffffffffu, head);
-  const int my_slot = (int)(my_key >> 32);
+  const float* wrow = w.w + ((size_t)m * w.max_T + wt0) * k;  // pair t*k + r of the chunk at wrow[t*k + r]
   float* Vm = V + (size_t)m * dm.N * dm.dv;
-  float4 Vr[G][VPL];
-#pragma unroll
-  for (int gi = 0; gi < G; ++gi) {
-    const int slot = __shfl_sync(0xffffffffu, my_slot, gi);
-    const bool ok = ((heads >> gi) & 1u) && slot >= 0 && (long long)slot < dm.N;
-    const float4* row = reinterpret_cast<const float4*>(Vm + (size_t)(ok ? slot : 0) * dm.dv);
-#pragma unroll
-    for (int c = 0; c < VPL; ++c) {
-      const int e4 = lane + 32 * c;
-      Vr[gi][c] = (ok && e4 < dv4) ? row[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+  // the CTAs of a memory cover its list in strides (grid sized to the resident CTAs)
+  for (int pos0 = (blockIdx.x * VAL_WARPS + warp) * G; pos0 < P; pos0 += gridDim.x * VAL_WARPS * G) {
+    unsigned long long my_key = ~0ull;
+    bool head = false;
+    if (lane < G && pos0 + lane < P) {
+      const int pos = pos0 + lane;
+      my_key = sk[pos];
+      head = pos == 0 || (sk[pos - 1] >> 32) != (my_key >> 32);
     }
-  }
+    const unsigned heads = __ballot_sync(0xffffffffu, head);
+    const int my_slot = (int)(my_key >> 32);
+    float4 Vr[G][VPL];
 #pragma unroll
-  for (int gi = 0; gi < G; ++gi) {
-    const unsigned long long key0 = __shfl_sync(0xffffffffu, my_key, gi);
-    if (!((heads >> gi) & 1u)) continue;
-    const int slot = (int)(key0 >> 32);
-    if (slot < 0 || (long long)slot >= dm.N) {
-      if (lane == 0) atomicExch(w.status, DEV_BAD_SLOT);
-      continue;
+    for (int gi = 0; gi < G; ++gi) {
+      const int slot = __shfl_sync(0xffffffffu, my_slot, gi);
+      const bool ok = ((heads >> gi) & 1u) && slot >= 0 && (long long)slot < dm.N;
+      const float4* row = reinterpret_cast<const float4*>(Vm + (size_t)(ok ? slot : 0) * dm.dv);
+#pragma unroll
+      for (int c = 0; c < VPL; ++c) {
+        const int e4 = lane + 32 * c;
+        Vr[gi][c] = (ok && e4 < dv4) ? row[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
-    float4 Gs[VPL];
 #pragma unroll
-    for (int c = 0; c < VPL; ++c) Gs[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-    int p = pos0 + gi;
-    unsigned long long key = key0;
-    for (;;) {
-      const uint32_t tr = (uint32_t)(key & 0xffffffffu);
-      const int t_local = (int)(tr / (uint32_t)k), r = (int)(tr - (uint32_t)t_local * k);
-      const float wt = w.w[((size_t)m * w.max_T + wt0 + t_local) * k + r];
-      const float4* rrow = reinterpret_cast<const float4*>(w.resid + ((size_t)m * C + t_local) * dm.dv);
+    for (int gi = 0; gi < G; ++gi) {
+      const unsigned long long key0 = __shfl_sync(0xffffffffu, my_key, gi);
+      if (!((heads >> gi) & 1u)) continue;
+      const int slot = (int)(key0 >> 32);
+      if (slot < 0 || (long long)slot >= dm.N) {
+        if (lane == 0) atomicExch(w.status, DEV_BAD_SLOT);
+        continue;
+      }
+      float4 Gs[VPL];
+#pragma unroll
+      for (int c = 0; c < VPL; ++c) Gs[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      int p = pos0 + gi;
+      unsigned long long key = key0;
+      for (;;) {
+        const uint32_t tr = (uint32_t)(key & 0xffffffffu);
+        const int t_local = kshift >= 0 ? (int)(tr >> kshift) : (int)(tr / (uint32_t)k);
+        const float wt = wrow[tr];
+        const float4* rrow = reinterpret_cast<const float4*>(w.resid + ((size_t)m * C + t_local) * dm.dv);
+#pragma unroll
+        for (int c = 0; c < VPL; ++c) {
+          const int e4 = lane + 32 * c;
+          if (e4 < dv4) {
+            const float4 x = rrow[e4];
+            Gs[c].x = fmaf(wt, x.x, Gs[c].x); Gs[c].y = fmaf(wt, x.y, Gs[c].y);
+            Gs[c].z = fmaf(wt, x.z, Gs[c].z); Gs[c].w = fmaf(wt, x.w, Gs[c].w);
+          }
+        }
+        if (++p >= P) break;
+        key = sk[p];
+        if ((int)(key >> 32) != slot) break;
+      }
+      const float nr = (float)(p - (pos0 + gi));
+      float4* row = reinterpret_cast<float4*>(Vm + (size_t)slot * dm.dv);
 #pragma unroll
       for (int c = 0; c < VPL; ++c) {
         const int e4 = lane + 32 * c;
         if (e4 < dv4) {
-          const float4 x = rrow[e4];
-          Gs[c].x = fmaf(wt, x.x, Gs[c].x); Gs[c].y = fmaf(wt, x.y, Gs[c].y);
-          Gs[c].z = fmaf(wt, x.z, Gs[c].z); Gs[c].w = fmaf(wt, x.w, Gs[c].w);
+          float4 x = Vr[gi][c];
+          x.x -= Gs[c].x / nr; x.y -= Gs[c].y / nr; x.z -= Gs[c].z / nr; x.w -= Gs[c].w / nr;
+          row[e4] = x;
         }
-      }
-      if (++p >= P) break;
-      key = sk[p];
-      if ((int)(key >> 32) != slot) break;
-    }
-    const float nr = (float)(p - (pos0 + gi));
-    float4* row = reinterpret_cast<float4*>(Vm + (size_t)slot * dm.dv);
-#pragma unroll
-    for (int c = 0; c < VPL; ++c) {
-      const int e4 = lane + 32 * c;
-      if (e4 < dv4) {
-        float4 x = Vr[gi][c];
-        x.x -= Gs[c].x / nr; x.y -= Gs[c].y / nr; x.z -= Gs[c].z / nr; x.w -= Gs[c].w / nr;
-        row[e4] = x;
       }
     }
   }
@@ -326,15 +331,40 @@ int launch_resid(const Dims& d, const Work& w, const void* v, const float* g, lo
   return 1;
 }
 
+// CTAs of one kernel that fit on the GPU at once (cached per kernel).
+static int resident_ctas(const void* kern, int threads) {
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  static const void* keys[8];
+  static int vals[8];
+  static int used = 0;
+  for (int i = 0; i < used; ++i)
+    if (keys[i] == kern) return vals[i];
+  int dev = 0, sms = 148, per_sm = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
+  const int v = sms * per_sm;
+  if (used < 8) {
+    keys[used] = kern;
+    vals[used++] = v;
+  }
+  return v;
+}
+
 int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s) {
   const int vpl = vpl_of(d.dv);
   const int G = vpl <= 2 ? 4 : vpl == 4 ? 2 : 1;  // list positions per warp: ~8 float4 in flight per lane
-  dim3 grid((d.C * d.k + VAL_WARPS * G - 1) / (VAL_WARPS * G), d.M);
+  const int need = (d.C * d.k + VAL_WARPS * G - 1) / (VAL_WARPS * G);  // CTAs per memory for one pass
+  auto grid_for = [&](int resident) {
+    const int per_mem = (resident + d.M - 1) / d.M;  // one resident wave over all memories
+    return dim3(need < per_mem ? need : per_mem, d.M);
+  };
   switch (vpl) {
-    case 1: launch_k(write_kernel<1, 4>, grid, VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
-    case 2: launch_k(write_kernel<2, 4>, grid, VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
-    case 4: launch_k(write_kernel<4, 2>, grid, VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
-    default: launch_k(write_kernel<8, 1>, grid, VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
+    case 1: launch_k(write_kernel<1, 4>, grid_for(resident_ctas((const void*)write_kernel<1, 4>, VAL_WARPS * 32)), VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
+    case 2: launch_k(write_kernel<2, 4>, grid_for(resident_ctas((const void*)write_kernel<2, 4>, VAL_WARPS * 32)), VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
+    case 4: launch_k(write_kernel<4, 2>, grid_for(resident_ctas((const void*)write_kernel<4, 2>, VAL_WARPS * 32)), VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
+    default: launch_k(write_kernel<8, 1>, grid_for(resident_ctas((const void*)write_kernel<8, 1>, VAL_WARPS * 32)), VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
   }
   return 1;
 }
