@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -55,10 +56,15 @@ struct fwpkm_state {
   size_t ev_next;
   int no_graph;
   int serial;  // diagnostics: all three chains on one stream (per-kernel timing without overlap)
-  cudaGraphExec_t graph_exec;
-  SeqKey graph_key;
-  uint64_t graph_kernels;
-  int graph_ev_used;
+  // two cached graphs (e.g. the plain step and the same step with timing events),
+  // least recently used replaced
+  static constexpr int NGRAPH = 2;
+  cudaGraphExec_t graph_exec[NGRAPH];
+  SeqKey graph_key[NGRAPH];
+  uint64_t graph_kernels[NGRAPH];
+  int graph_ev_used[NGRAPH];
+  uint64_t graph_used[NGRAPH];
+  uint64_t graph_clock;
 };
 
 namespace {
@@ -138,10 +144,25 @@ cudaEvent_t next_event(fwpkm_state* st) {
 
 namespace fwpkm {
 
+void set_carveout(const void* kern) {
+  static std::mutex mu;
+  static std::vector<const void*> done;
+  static const bool on = [] {
+    const char* e = getenv("FWPKM_CARVEOUT");
+    return !(e && e[0] == '0');
+  }();
+  if (!on) return;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const void* k : done)
+    if (k == kern) return;
+  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+  done.push_back(kern);
+}
+
 bool pdl_enabled() {
   static const bool on = [] {
-    const char* e = getenv("FWPKM_NO_PDL");
-    return !(e && e[0] == '1');
+    const char* e = getenv("FWPKM_PDL");
+    return e && e[0] == '1';
   }();
   return on;
 }
@@ -212,7 +233,7 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
       x.Wt = (__nv_bfloat16*)take(2 * 3 * P * n * cpad);
       x.qt_T = (int)((T > C ? T : C) + 63) / 64 * 64;
       x.Qt = (__nv_bfloat16*)take(2 * P * h * (size_t)x.qt_T);
-      x.wsum_part = (float*)take(4 * P * (cpad / 16) * n);
+      x.wsum_part = (float*)take(4 * P * (cpad / 8) * n);
       x.pbar_cnt = (int*)take(4 * P * ((n + 255) / 256));
     }
   }
@@ -244,7 +265,7 @@ Work group_work(const Dims& d, const Work& w, int m0) {
   if (x.ppart) x.ppart += M0 * 2 * 8 * n;
   if (x.Wt) x.Wt += M0 * 2 * n * cpad;
   if (x.Qt) x.Qt += M0 * 2 * h * (size_t)w.qt_T;
-  if (x.wsum_part) x.wsum_part += M0 * 2 * (cpad / 16) * n;
+  if (x.wsum_part) x.wsum_part += M0 * 2 * (cpad / 8) * n;
   if (x.pbar_cnt) x.pbar_cnt += M0 * 2 * ((n + 255) / 256);
   return x;
 }
@@ -296,9 +317,13 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
   st->ev_used = 0;
   st->host_error = 0;
   st->ev_next = 0;
-  st->graph_exec = nullptr;
-  st->graph_kernels = 0;
-  st->graph_ev_used = 0;
+  for (int i = 0; i < fwpkm_state::NGRAPH; ++i) {
+    st->graph_exec[i] = nullptr;
+    st->graph_kernels[i] = 0;
+    st->graph_ev_used[i] = 0;
+    st->graph_used[i] = 0;
+  }
+  st->graph_clock = 0;
   {
     const char* e = getenv("FWPKM_NO_GRAPH");
     st->no_graph = (e && e[0] == '1') ? 1 : 0;
@@ -338,7 +363,8 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
 
 void fwpkm_destroy_state(fwpkm_state* st) {
   if (!st) return;
-  if (st->graph_exec) cudaGraphExecDestroy(st->graph_exec);
+  for (int i = 0; i < fwpkm_state::NGRAPH; ++i)
+    if (st->graph_exec[i]) cudaGraphExecDestroy(st->graph_exec[i]);
   for (cudaEvent_t e : st->sync_ev) cudaEventDestroy(e);
   for (int gi = 0; gi < fwpkm_state::MAX_GROUPS; ++gi) {
     if (st->sK[gi]) cudaStreamDestroy(st->sK[gi]);
@@ -371,11 +397,11 @@ fwpkm_status fwpkm_forward_chunk(fwpkm_state* st, const void* q, const void* v, 
     run(st, KK_PREP, s, [&] { return launch_qnorm(d, st->wk, q, seq_stride, 0, c_len, s); });
     run(st, KK_PREP, s, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, s); });
     run(st, KK_SCORE, s, [&] { return launch_tc_score(d, st->wk, q, seq_stride, c_len, 0, 0, c_len, ku, s); });
-    run(st, KK_TOPK, s, [&] { return launch_topk_rows(d, st->wk, 0, c_len, s); });
+    run(st, KK_TOPK, s, [&] { return launch_select(d, st->wk, 0, c_len, idx_out, w_out, s); });
   } else {
     run(st, KK_SCORE, s, [&] { return launch_score_topk(d, st->wk, st->K1, st->K2, q, seq_stride, 0, c_len, ku, s); });
+    run(st, KK_CART, s, [&] { return launch_cartesian(d, st->wk, 0, c_len, idx_out, w_out, s); });
   }
-  run(st, KK_CART, s, [&] { return launch_cartesian(d, st->wk, 0, c_len, idx_out, w_out, s); });
   run(st, KK_GATHER, s, [&] {
     return launch_gather(d, st->wk, st->V, v, g, seq_stride, 0, c_len, o, false, nullptr, s);
   });
@@ -472,13 +498,13 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
       const int wl = T - w0 < wtok ? T - w0 : wtok;
       if (tc) {
         run(st, KK_SCORE, sK, [&] { return launch_tc_score(d, wk, q, T, T, w0, w0, wl, false, sK); });
-        run(st, KK_TOPK, sK, [&] { return launch_topk_rows(d, wk, w0, wl, sK); });
+        run(st, KK_TOPK, sK, [&] { return launch_select(d, wk, w0, wl, nullptr, nullptr, sK); });
       } else {
         run(st, KK_SCORE, sK, [&] {
           return launch_score_topk(d, wk, K1, K2, offs(q, (long long)w0 * d.d, es), T, w0, wl, false, sK);
         });
+        run(st, KK_CART, sK, [&] { return launch_cartesian(d, wk, w0, wl, nullptr, nullptr, sK); });
       }
-      run(st, KK_CART, sK, [&] { return launch_cartesian(d, wk, w0, wl, nullptr, nullptr, sK); });
       run(st, KK_SORT, sK, [&] { return launch_sort_pairs(d, wk, w0, wl, !la || (w0 + wl < T), sK); });
       ready.push_back(mark(sK));
     }
@@ -514,10 +540,11 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
         }
         if (val_done[c]) cudaStreamWaitEvent(sS, val_done[c], 0);     // previous pass wrote chunk c
         if (tc) {
-          run(st, KK_TOPK, sS, [&] { return launch_topk_rows(d, wb, t0, len, sS); });
+          run(st, KK_TOPK, sS, [&] { return launch_select(d, wb, t0, len, nullptr, nullptr, sS); });
           topk_done[cnt & 1] = mark(sS);
+        } else {
+          run(st, KK_CART, sS, [&] { return launch_cartesian(d, wb, t0, len, nullptr, nullptr, sS); });
         }
-        run(st, KK_CART, sS, [&] { return launch_cartesian(d, wb, t0, len, nullptr, nullptr, sS); });
         run(st, KK_SORT, sS, [&] { return launch_sort_pairs(d, wb, t0, len, !la || (t0 + len < T), sS); });
         sel_done[c] = mark(sS);
         cudaStreamWaitEvent(sV, sel_done[c], 0);
@@ -567,38 +594,46 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
     if (st->host_error) return FWPKM_ERR_CUDA;
     return last_cuda();
   }
-  // One CUDA graph per distinct call: replayed while the arguments stay the same.
+  // One CUDA graph per distinct call (arguments and timing kind), replayed while they stay
+  // the same; the last two are kept.
   const SeqKey key = {q, v, g, o, T, n_iter, st->prof_kind};
-  if (!st->graph_exec || !(key == st->graph_key)) {
-    if (st->graph_exec) {
-      cudaGraphExecDestroy(st->graph_exec);
-      st->graph_exec = nullptr;
+  int slot = -1;
+  for (int i = 0; i < fwpkm_state::NGRAPH; ++i)
+    if (st->graph_exec[i] && st->graph_key[i] == key) slot = i;
+  if (slot < 0) {
+    slot = 0;
+    for (int i = 1; i < fwpkm_state::NGRAPH; ++i)
+      if (st->graph_used[i] < st->graph_used[slot]) slot = i;
+    if (st->graph_exec[slot]) {
+      cudaGraphExecDestroy(st->graph_exec[slot]);
+      st->graph_exec[slot] = nullptr;
     }
     const uint64_t before = g_launches.load();
     if (cudaStreamBeginCapture(st->sCap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return last_cuda();
     enqueue_sequence(st, q, v, g, T, n_iter, o, st->sCap);
     cudaGraph_t graph = nullptr;
     cudaError_t e = cudaStreamEndCapture(st->sCap, &graph);
-    st->graph_kernels = g_launches.load() - before;
-    g_launches -= st->graph_kernels;  // counted per replay below
+    st->graph_kernels[slot] = g_launches.load() - before;
+    g_launches -= st->graph_kernels[slot];  // counted per replay below
     if (e != cudaSuccess || st->host_error) {
       if (graph) cudaGraphDestroy(graph);
       last_cuda();
       return FWPKM_ERR_CUDA;
     }
-    e = cudaGraphInstantiate(&st->graph_exec, graph, 0);
+    e = cudaGraphInstantiate(&st->graph_exec[slot], graph, 0);
     cudaGraphDestroy(graph);
     if (e != cudaSuccess) {
-      st->graph_exec = nullptr;
+      st->graph_exec[slot] = nullptr;
       last_cuda();
       return FWPKM_ERR_CUDA;
     }
-    st->graph_key = key;
-    st->graph_ev_used = st->ev_used;
+    st->graph_key[slot] = key;
+    st->graph_ev_used[slot] = st->ev_used;
   }
-  if (cudaGraphLaunch(st->graph_exec, user) != cudaSuccess) return last_cuda();
-  g_launches += st->graph_kernels;
-  st->ev_used = st->graph_ev_used;
+  st->graph_used[slot] = ++st->graph_clock;
+  if (cudaGraphLaunch(st->graph_exec[slot], user) != cudaSuccess) return last_cuda();
+  g_launches += st->graph_kernels[slot];
+  st->ev_used = st->graph_ev_used[slot];
   return last_cuda();
 }
 

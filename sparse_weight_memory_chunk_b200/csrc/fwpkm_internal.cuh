@@ -54,7 +54,7 @@ struct Work {
   __nv_bfloat16* Wt; // [3][M*2][n][Cpad]  key-step weights, sub-key major, bf16 pieces
   __nv_bfloat16* Qt; // [M*2][h][qt_T]     half-queries, feature major (operand B of the key step)
   int qt_T;          // token columns of Qt (a multiple of 64)
-  float* wsum_part;  // [M*2][Cpad/16][n]  per-16-token-block sums of W
+  float* wsum_part;  // [M*2][Cpad/8][n]   per-8-token-block sums of W
   int* pbar_cnt;     // [M*2][ceil(n/256)] arrival counters of the pbar column blocks (zero between launches)
   // Every array above is memory-major except the bf16 pieces (Kpc, Wt), whose piece
   // stride is P_all problems; a Work for a group of memories is the same carve with its
@@ -139,6 +139,9 @@ int launch_keyprep(const Dims& d, const Work& w, const float* K1, const float* K
 // q extent T_ext tokens per memory) into Dfull rows 0..len-1, plus zpart if key_update.
 int launch_tc_score(const Dims& d, const Work& w, const void* q_base, long long q_stride, int q_extent, int q_row0,
                     int wt0, int len, bool key_update, cudaStream_t s);
+// Fused per-half top-k + Cartesian search + softmax from Dfull rows 0..len-1 (workspace
+// tokens wt0..): writes idx, w and the optional user copies; A/Dsv are not written.
+int launch_select(const Dims& d, const Work& w, int wt0, int len, int32_t* idx_out, float* w_out, cudaStream_t s);
 // Per-half top-k from Dfull rows 0..len-1 into A/Dsv at workspace tokens wt0..
 int launch_topk_rows(const Dims& d, const Work& w, int wt0, int len, cudaStream_t s);
 // Feature-major copy of both half-queries of `len` tokens into Qt columns qt0.. (the key
@@ -154,9 +157,15 @@ int launch_tc_keystep(const Dims& d, const Work& w, float* K1, float* K2, const 
                       int qt_t0, cudaStream_t s);
 
 // ---- launches ----
-// Whether kernels are launched with programmatic dependent launch (default on; the
-// environment variable FWPKM_NO_PDL=1 turns it off for comparisons).
+// Whether kernels are launched with programmatic dependent launch (FWPKM_PDL=1; off by
+// default: on the paper-scale step the early-resident dependents held SM slots that the
+// other chains' kernels needed, 1.92 ms per step against 1.84 ms without).
 bool pdl_enabled();
+// Give `kern` the largest shared-memory carveout once per process (FWPKM_CARVEOUT=0 keeps
+// the driver's choice).  With every kernel on one carveout an SM never has to drain to
+// switch its L1/shared split before a CTA of another kernel (e.g. a GEMM needing 130 KB)
+// can start beside the running ones.
+void set_carveout(const void* kern);
 
 // Launch `kern` on `s`, allowing it to start while the previous kernel of the same stream
 // finishes (programmatic stream serialization).  Every kernel launched this way calls
@@ -174,6 +183,7 @@ inline void launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  set_carveout((const void*)kern);
   cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 

@@ -4,8 +4,7 @@
 // Fast-weight Product Key Memory (rainbus summary), PKM prerequisite and method
 // step 2; (paperlayer summary) §2.2: the final top-k is searched in the Cartesian
 // product of the two halves' top-k, and the k selected slots get normalised weights.
-#include "bitonic.cuh"
-#include "fwpkm_internal.cuh"
+#include "topk.cuh"
 
 namespace fwpkm {
 
@@ -35,49 +34,41 @@ __device__ __forceinline__ void sort_cand(u64 (&x)[4], u64* cand, int lane) {
   for (int u = 0; u < VPT; ++u) cand[lane * VPT + u] = y[u];
 }
 
-__global__ void __launch_bounds__(CART_WARPS * 32)
-cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
-  pdl_wait();
-  pdl_trigger();
-  __shared__ float s_sig[CART_WARPS][2][32];
-  __shared__ int s_sub[CART_WARPS][2][32];
-  __shared__ u64 s_cand[CART_WARPS][128];
-  __shared__ unsigned short s_tab[128];
-  __shared__ int s_total;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int k = dm.k, n = dm.n;
-  if (warp == 0) {
-    // staircase table: lane i owns rank i of half 1 and ranks 0 .. k/(i+1)-1 of half 2
-    const int rowlen = lane < k ? k / (lane + 1) : 0;
-    int incl = rowlen;
+// Staircase table, built by one warp: candidate c -> (i << 8) | j, where lane i owns rank
+// i of half 1 and ranks 0 .. k/(i+1)-1 of half 2.  Returns the candidate count in *total.
+__device__ __forceinline__ void build_staircase(int k, int lane, unsigned short* tab, int* total) {
+  const int rowlen = lane < k ? k / (lane + 1) : 0;
+  int incl = rowlen;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    for (int jj = 0; jj < rowlen; ++jj) s_tab[incl - rowlen + jj] = (unsigned short)((lane << 8) | jj);
-    if (lane == 31) s_total = incl;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
-  __syncthreads();
-  const int i_tok = blockIdx.x * CART_WARPS + warp;
-  const int m = blockIdx.y;
-  if (i_tok >= len) return;
-  const long long tok = (long long)wt0 + i_tok;
-  const int total = s_total;
+  for (int jj = 0; jj < rowlen; ++jj) tab[incl - rowlen + jj] = (unsigned short)((lane << 8) | jj);
+  if (lane == 31) *total = incl;
+}
 
+// Restricted Cartesian top-k + softmax of one token, by one warp.  Survivors of half j
+// arrive in rank order (D asc, sub-key asc) at sub[j][r], dist[j][r] (r < k).  Writes
+// slot/weight r of the token to idx_o[r], w_o[r] (and to the optional user copies).
+__device__ __noinline__ void cartesian_token(const Dims& dm, const int* const (&sub)[2],
+                                                const float* const (&dist)[2], float (*s_sig)[32],
+                                                int (*s_sub)[32], u64* cand, const unsigned short* tab,
+                                                int total, int lane, int32_t* idx_o, float* w_o,
+                                                int32_t* idx_u, float* w_u) {
+  const int k = dm.k, n = dm.n;
   for (int j = 0; j < 2; ++j) {
-    const size_t base = (((size_t)m * 2 + j) * w.max_T + tok) * k;
     u64 key[1] = {~0ull};
     if (lane < k) {
-      const int sub = w.A[base + lane];
-      const float sig = -logf(dm.eps_idw + w.Dsv[base + lane]);
-      key[0] = ((u64)(~float_key(sig)) << 32) | (unsigned)sub;  // sigma desc, sub asc
+      const float sig = -logf(dm.eps_idw + dist[j][lane]);
+      key[0] = ((u64)(~float_key(sig)) << 32) | (unsigned)sub[j][lane];  // sigma desc, sub asc
     }
     const u64 nxt = __shfl_down_sync(0xffffffffu, key[0], 1);
     if (__any_sync(0xffffffffu, lane < 31 && nxt < key[0])) warp_sort_asc<1>(key, lane);
+    __syncwarp();
     if (lane < k) {
-      s_sig[warp][j][lane] = key_float(~(uint32_t)(key[0] >> 32));
-      s_sub[warp][j][lane] = (int)(key[0] & 0xffffffffu);
+      s_sig[j][lane] = key_float(~(uint32_t)(key[0] >> 32));
+      s_sub[j][lane] = (int)(key[0] & 0xffffffffu);
     }
   }
   __syncwarp();
@@ -88,14 +79,13 @@ cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_ou
     const int c = lane * 4 + u;
     x[u] = ~0ull;
     if (c < total) {
-      const int t = s_tab[c], i1 = t >> 8, i2 = t & 255;
-      const float S = s_sig[warp][0][i1] + s_sig[warp][1][i2];
-      const unsigned slot = (unsigned)s_sub[warp][0][i1] * (unsigned)n + (unsigned)s_sub[warp][1][i2];
+      const int t = tab[c], i1 = t >> 8, i2 = t & 255;
+      const float S = s_sig[0][i1] + s_sig[1][i2];
+      const unsigned slot = (unsigned)s_sub[0][i1] * (unsigned)n + (unsigned)s_sub[1][i2];
       x[u] = ((u64)(~float_key(S)) << 32) | slot;
     }
   }
-  // the sorts below take the elements lane * VPT + u, u < VPT: repack for VPT < 4
-  u64* cand = s_cand[warp];
+  // the sorts take the elements lane * VPT + u, u < VPT: repack for VPT < 4
   const int Sz = total <= 32 ? 32 : total <= 64 ? 64 : 128;
   if (Sz == 128) {
     sort_cand<4>(x, cand, lane);
@@ -124,12 +114,90 @@ cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_ou
   const float z = warp_sum(e);
   if (lane < k) {
     const float wt = e / z;
-    const size_t o = ((size_t)m * w.max_T + tok) * k + lane;
-    w.idx[o] = slot;
-    w.w[o] = wt;
-    if (idx_out) idx_out[((size_t)m * len + i_tok) * k + lane] = slot;
-    if (w_out) w_out[((size_t)m * len + i_tok) * k + lane] = wt;
+    idx_o[lane] = slot;
+    w_o[lane] = wt;
+    if (idx_u) idx_u[lane] = slot;
+    if (w_u) w_u[lane] = wt;
   }
+}
+
+// Survivors from the per-half top-k arrays A/Dsv.
+__global__ void __launch_bounds__(CART_WARPS * 32)
+cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float s_sig[CART_WARPS][2][32];
+  __shared__ int s_sub[CART_WARPS][2][32];
+  __shared__ u64 s_cand[CART_WARPS][128];
+  __shared__ unsigned short s_tab[128];
+  __shared__ int s_total;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = dm.k;
+  if (warp == 0) build_staircase(k, lane, s_tab, &s_total);
+  __syncthreads();
+  const int i_tok = blockIdx.x * CART_WARPS + warp;
+  const int m = blockIdx.y;
+  if (i_tok >= len) return;
+  const long long tok = (long long)wt0 + i_tok;
+  const size_t b0 = (((size_t)m * 2 + 0) * w.max_T + tok) * k, b1 = (((size_t)m * 2 + 1) * w.max_T + tok) * k;
+  const int* const sub[2] = {w.A + b0, w.A + b1};
+  const float* const dist[2] = {w.Dsv + b0, w.Dsv + b1};
+  const size_t o = ((size_t)m * w.max_T + tok) * k;
+  const size_t ou = ((size_t)m * len + i_tok) * k;
+  cartesian_token(dm, sub, dist, s_sig[warp], s_sub[warp], s_cand[warp], s_tab, s_total, lane, w.idx + o, w.w + o,
+                  idx_out ? idx_out + ou : nullptr, w_out ? w_out + ou : nullptr);
+}
+
+// Fused per-half top-k + Cartesian search (tensor-core path): a CTA takes SEL_TOK tokens of
+// one memory; warps 2i and 2i+1 take the two halves of token i from the distance rows,
+// leave their survivors in shared memory, and warp 2i then finishes the token.
+constexpr int SEL_TOK = 4;
+template <int NPL>
+__global__ void __launch_bounds__(SEL_TOK * 64, 3)
+select_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ u64 s_cand[2 * SEL_TOK][128];
+  __shared__ int s_hsub[SEL_TOK][2][32];
+  __shared__ float s_hd[SEL_TOK][2][32];
+  __shared__ float s_sig[SEL_TOK][2][32];
+  __shared__ int s_sub[SEL_TOK][2][32];
+  __shared__ unsigned short s_tab[128];
+  __shared__ int s_total;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tl = warp >> 1, j = warp & 1;
+  const int i_tok = blockIdx.x * SEL_TOK + tl;
+  const int m = blockIdx.y;
+  const int k = dm.k;
+  if (warp == 0) build_staircase(k, lane, s_tab, &s_total);
+  if (i_tok < len) {
+    const float* row = w.Dfull + ((size_t)(m * 2 + j) * w.drows + i_tok) * dm.n;
+    row_topk<NPL>(row, dm.n, k, lane, s_cand[warp], s_hsub[tl][j], s_hd[tl][j]);
+  }
+  __syncthreads();
+  if (j != 0 || i_tok >= len) return;
+  const long long tok = (long long)wt0 + i_tok;
+  const int* const sub[2] = {s_hsub[tl][0], s_hsub[tl][1]};
+  const float* const dist[2] = {s_hd[tl][0], s_hd[tl][1]};
+  const size_t o = ((size_t)m * w.max_T + tok) * k;
+  const size_t ou = ((size_t)m * len + i_tok) * k;
+  cartesian_token(dm, sub, dist, s_sig[tl], s_sub[tl], s_cand[warp], s_tab, s_total, lane, w.idx + o, w.w + o,
+                  idx_out ? idx_out + ou : nullptr, w_out ? w_out + ou : nullptr);
+}
+
+int launch_select(const Dims& d, const Work& w, int wt0, int len, int32_t* idx_out, float* w_out, cudaStream_t s) {
+  if (len <= 0) return 0;
+  dim3 grid((len + SEL_TOK - 1) / SEL_TOK, d.M);
+  const int npl = (d.n + 31) / 32;
+  const int th = SEL_TOK * 64;
+  if (npl <= 2) launch_k(select_kernel<2>, grid, th, 0, s, d, w, wt0, len, idx_out, w_out);
+  else if (npl <= 4) launch_k(select_kernel<4>, grid, th, 0, s, d, w, wt0, len, idx_out, w_out);
+  else if (npl <= 8) launch_k(select_kernel<8>, grid, th, 0, s, d, w, wt0, len, idx_out, w_out);
+  else if (npl <= 16) launch_k(select_kernel<16>, grid, th, 0, s, d, w, wt0, len, idx_out, w_out);
+  else if (npl <= 32) launch_k(select_kernel<32>, grid, th, 0, s, d, w, wt0, len, idx_out, w_out);
+  else if (npl <= 64) launch_k(select_kernel<64>, grid, th, 0, s, d, w, wt0, len, idx_out, w_out);
+  else launch_k(select_kernel<128>, grid, th, 0, s, d, w, wt0, len, idx_out, w_out);
+  return 1;
 }
 
 int launch_cartesian(const Dims& d, const Work& w, int wt0, int len, int32_t* idx_out, float* w_out,

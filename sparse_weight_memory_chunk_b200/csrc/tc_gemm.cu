@@ -180,14 +180,45 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     for (int j = 0; j < ntiles; ++j) {
       const int b = j & 1;
       const uint32_t aph = (j >> 1) & 1;
+      const int nt = nt0 + j;
+      const int r = mt * TC_BM + row;
+      const bool rv = r < g.m_valid;
+      // operands of the epilogue that do not depend on the accumulator are loaded while
+      // the MMAs run: DIST the row norm and 32 column norms, KEYSTEP sum_t W and the key
+      float pre_s = 0.f, pre[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) pre[i] = 0.f;
+      if (g.epi == TC_EPI_DIST) {
+        const int c0 = nt * TC_BN + cg * 32;
+        pre_s = rv ? g.rowv[(size_t)p * g.rowv_pstride + g.rowv_off + r] : 0.f;
+        const float* kn = g.colv + (size_t)p * g.colv_pstride;
+        if (c0 + 32 <= g.n_valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(kn + c0 + i);
+            pre[i] = k4.x; pre[i + 1] = k4.y; pre[i + 2] = k4.z; pre[i + 3] = k4.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pre[i] = c0 + i < g.n_valid ? kn[c0 + i] : 0.f;
+        }
+      } else if (g.epi == TC_EPI_KEYSTEP) {
+        const int h = g.n_valid, n = g.m_valid, e0 = cg * 32;
+        if (rv && e0 < h) {
+          for (int tt = 0; tt < g.wsum_tiles; ++tt) pre_s += g.wsum_part[((size_t)p * g.wsum_tiles + tt) * n + r];
+          const float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h + e0;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(K + i);
+            pre[i] = k4.x; pre[i + 1] = k4.y; pre[i + 2] = k4.z; pre[i + 3] = k4.w;
+          }
+        }
+      }
       // one lane waits; the verdict is shared so the warp stays converged for tcgen05.ld
       int ok = lane == 0 ? (mbar_wait(&accf[b], aph, abort_flag, deadline) ? 1 : 0) : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const int nt = nt0 + j;
-      const int r = mt * TC_BM + row;
-      const bool rv = r < g.m_valid;
       uint32_t v[32];
       tmem_ld32(lane_base + (uint32_t)(b * TC_BN + cg * 32), v);
       tmem_wait_ld();
@@ -197,21 +228,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (lane == 0) mbar_arrive(&acce[b]);
       if (g.epi == TC_EPI_DIST) {
         const int c0 = nt * TC_BN + cg * 32;
-        const float rq = rv ? g.rowv[(size_t)p * g.rowv_pstride + g.rowv_off + r] : 0.f;
-        const float* kn = g.colv + (size_t)p * g.colv_pstride;
+        const float rq = pre_s;
         float* out = g.out + ((size_t)p * g.out_pstride + (size_t)r * g.out_ld);
         float dv[32];
         float zacc = 0.f;
         if (c0 + 32 <= g.n_valid) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float4 k4 = *reinterpret_cast<const float4*>(kn + c0 + i);
-            const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              dv[i + u] = fmaxf((rq + kk[u]) - 2.f * __uint_as_float(v[i + u]), 0.f);
-              zacc += __fdividef(1.f, g.eps + dv[i + u]);
-            }
+          for (int i = 0; i < 32; ++i) {
+            dv[i] = fmaxf((rq + pre[i]) - 2.f * __uint_as_float(v[i]), 0.f);
+            zacc += __fdividef(1.f, g.eps + dv[i]);
           }
           if (rv) {
 #pragma unroll
@@ -222,8 +247,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int c = c0 + i;
-            const float kv = c < g.n_valid ? kn[c] : 0.f;
-            dv[i] = fmaxf((rq + kv) - 2.f * __uint_as_float(v[i]), 0.f);
+            dv[i] = fmaxf((rq + pre[i]) - 2.f * __uint_as_float(v[i]), 0.f);
             if (c < g.n_valid) {
               zacc += __fdividef(1.f, g.eps + dv[i]);
               if (rv) out[c] = dv[i];
@@ -263,17 +287,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int e0 = cg * 32;
         float ss = 0.f;
         if (rv && e0 < h) {
-          float wsum = 0.f;
-          for (int tt = 0; tt < g.wsum_tiles; ++tt) wsum += g.wsum_part[((size_t)p * g.wsum_tiles + tt) * n + r];
+          const float wsum = pre_s;
           float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h;
           const size_t pstride = (size_t)g.piece_P * n * h;
           __nv_bfloat16* pc = g.Kpc + ((size_t)p * n + r) * h;
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
             const int e = e0 + i;
-            const float4 k0 = *reinterpret_cast<const float4*>(K + e);
-            const float4 k1 = *reinterpret_cast<const float4*>(K + e + 4);
-            const float kin[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+            float kin[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) kin[u] = pre[i + u];
             float kout[8];
             __align__(16) __nv_bfloat16 hi[8], mid[8], lo[8];
 #pragma unroll

@@ -104,7 +104,7 @@ tc_pbar_kernel(Dims dm, Work w, int len) {
   if (av) {
     const float* D = w.Dfull + (size_t)p * w.drows * dm.n;
     float s = 0.f;
-#pragma unroll 8
+#pragma unroll 16
     for (int t = t0; t < t1; ++t) s += __fdividef(1.f, dm.eps_idw + D[(size_t)t * dm.n + a]) * s_invz[t - t0];
     w.ppart[((size_t)p * PBAR_SLICES + sl) * dm.n + a] = s;
   }
@@ -128,10 +128,11 @@ tc_pbar_kernel(Dims dm, Work w, int len) {
 // W for a block of WB_T tokens and every sub-key, written sub-key major as three bf16
 // pieces (the A operand of the key-step GEMM), plus the block's per-sub-key sum of W.
 // First L_t = sum_a P[t][a] lp[a] = (sum_a lp[a] w[t][a]) / Z_t for the block's tokens (one
-// warp per token), then W[t][b] = (1/len) (w/Z_t) (lp[b] - L_t) w with one thread per
-// sub-key (the rows are re-read from L1/L2).
-constexpr int WB_T = 16;
-__global__ void __launch_bounds__(TP_THREADS)
+// warp per token, a row's loads all in flight), then W[t][b] = (1/len) (w/Z_t) (lp[b] -
+// L_t) w for WB_SUB sub-keys per thread (the block's rows re-read, all loads in flight).
+constexpr int WB_T = 8;
+constexpr int WB_SUB = 4;  // sub-keys per thread per pass: 256 threads x 4 = 1024
+__global__ void __launch_bounds__(TP_THREADS, 3)
 tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
   pdl_wait();
   pdl_trigger();
@@ -147,8 +148,17 @@ tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
     if (t < len) {
       const float* Dr = D + (size_t)t * n;
       float s = 0.f;
-#pragma unroll 8
-      for (int a = lane; a < n; a += 32) s += __fdividef(lp[a], dm.eps_idw + Dr[a]);
+      for (int a0 = 0; a0 < n; a0 += 32 * 16) {
+        float dd[16], ll[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int a = a0 + lane + 32 * u;
+          dd[u] = a < n ? Dr[a] : 0.f;
+          ll[u] = a < n ? lp[a] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) s += __fdividef(ll[u], dm.eps_idw + dd[u]);
+      }
       s = warp_sum(s);
       const float z = w.Z[(size_t)p * dm.C + t];
       L = s / z;
@@ -163,29 +173,37 @@ tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
   const float inv_len = 1.f / (float)len;
   const size_t pstride = (size_t)w.P_all * n * cpad;
   const int ntb = gridDim.x;
-  for (int b = threadIdx.x; b < n; b += TP_THREADS) {
-    const float lpb = lp[b];
-    __align__(16) __nv_bfloat16 hi[WB_T], mid[WB_T], lo[WB_T];
-    float wsum = 0.f;
+  for (int b0 = threadIdx.x; b0 < n; b0 += TP_THREADS * WB_SUB) {
+    float dd[WB_SUB][WB_T], lpb[WB_SUB];
 #pragma unroll
-    for (int tl = 0; tl < WB_T; ++tl) {
-      const int t = t0 + tl;
-      float W = 0.f;
-      if (t < len) {
-        const float wv = __fdividef(1.f, dm.eps_idw + D[(size_t)t * n + b]);
-        const float P_ = wv * s_invz[tl];
-        W = inv_len * P_ * (lpb - s_L[tl]) * wv;
-      }
-      wsum += W;
-      split3_bf16(W, hi[tl], mid[tl], lo[tl]);
+    for (int q = 0; q < WB_SUB; ++q) {
+      const int b = b0 + q * TP_THREADS;
+      lpb[q] = b < n ? lp[b] : 0.f;
+#pragma unroll
+      for (int tl = 0; tl < WB_T; ++tl) dd[q][tl] = (b < n && t0 + tl < len) ? D[(size_t)(t0 + tl) * n + b] : 0.f;
     }
-    w.wsum_part[((size_t)p * ntb + blockIdx.x) * n + b] = wsum;
-    __nv_bfloat16* dst = w.Wt + ((size_t)p * n + b) * cpad + t0;
 #pragma unroll
-    for (int h8 = 0; h8 < WB_T / 8; ++h8) {
-      *reinterpret_cast<uint4*>(dst + h8 * 8) = *reinterpret_cast<uint4*>(hi + h8 * 8);
-      *reinterpret_cast<uint4*>(dst + pstride + h8 * 8) = *reinterpret_cast<uint4*>(mid + h8 * 8);
-      *reinterpret_cast<uint4*>(dst + 2 * pstride + h8 * 8) = *reinterpret_cast<uint4*>(lo + h8 * 8);
+    for (int q = 0; q < WB_SUB; ++q) {
+      const int b = b0 + q * TP_THREADS;
+      if (b >= n) continue;
+      __align__(16) __nv_bfloat16 hi[WB_T], mid[WB_T], lo[WB_T];
+      float wsum = 0.f;
+#pragma unroll
+      for (int tl = 0; tl < WB_T; ++tl) {
+        float W = 0.f;
+        if (t0 + tl < len) {
+          const float wv = __fdividef(1.f, dm.eps_idw + dd[q][tl]);
+          const float P_ = wv * s_invz[tl];
+          W = inv_len * P_ * (lpb[q] - s_L[tl]) * wv;
+        }
+        wsum += W;
+        split3_bf16(W, hi[tl], mid[tl], lo[tl]);
+      }
+      w.wsum_part[((size_t)p * ntb + blockIdx.x) * n + b] = wsum;
+      __nv_bfloat16* dst = w.Wt + ((size_t)p * n + b) * cpad + t0;
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(hi);
+      *reinterpret_cast<uint4*>(dst + pstride) = *reinterpret_cast<uint4*>(mid);
+      *reinterpret_cast<uint4*>(dst + 2 * pstride) = *reinterpret_cast<uint4*>(lo);
     }
   }
 }

@@ -126,7 +126,7 @@ def test_streaming_matches_oracle_every_chunk(name):
     st.run_sequence(dev["q"], dev["v"], dev["g"], o)
     st.sync()
     assert torch.equal(o.cpu(), res["o"]), "run_sequence o differs from chunk-by-chunk"
-    assert torch.equal(dev["V"].cpu(), res["V"]), "run_sequence V differs"
+    assert torch.equal(dev["V"].cpu(), res["V"].cpu()), "run_sequence V differs"
     assert torch.equal(dev["K1"].cpu(), res["K1"]) and torch.equal(dev["K2"].cpu(), res["K2"])
 
 
