@@ -52,6 +52,9 @@ struct fwpkm_state {
   static constexpr int MAX_GROUPS = 8;
   int groups;
   cudaStream_t sK[MAX_GROUPS], sS[MAX_GROUPS], sV[MAX_GROUPS], sCap;
+  // scheduling priorities of the kernels of the three chains (the addressing chain is the
+  // critical path: highest); use_prio = 0 (FWPKM_PRIO=0) leaves them all at the default
+  int use_prio, prio_K, prio_S, prio_V;
   std::vector<cudaEvent_t> sync_ev;
   size_t ev_next;
   int no_graph;
@@ -113,8 +116,19 @@ fwpkm_status last_cuda() {
   return FWPKM_OK;
 }
 
+int stream_priority(const fwpkm_state* st, cudaStream_t s) {
+  for (int gi = 0; gi < st->groups; ++gi) {
+    if (s == st->sK[gi]) return st->prio_K;
+    if (s == st->sS[gi]) return st->prio_S;
+    if (s == st->sV[gi]) return st->prio_V;
+  }
+  return st->prio_V;
+}
+
 template <class F>
 void run(fwpkm_state* st, int kind, cudaStream_t s, F&& f) {
+  launch_priority_set = st->use_prio != 0 && !st->serial;
+  launch_priority = launch_priority_set ? stream_priority(st, s) : 0;
   const bool prof = st->prof_kind == kind && st->ev_used + 2 <= (int)st->ev.size();
   // Under stream capture a plain record is only a dependency marker; timing events must
   // become event-record nodes of the graph.
@@ -123,6 +137,7 @@ void run(fwpkm_state* st, int kind, cudaStream_t s, F&& f) {
   const unsigned rec_flags = cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
   if (prof) cudaEventRecordWithFlags(st->ev[st->ev_used], s, rec_flags);
   int nl = f();
+  launch_priority_set = false;
   if (prof) {
     cudaEventRecordWithFlags(st->ev[st->ev_used + 1], s, rec_flags);
     st->ev_used += 2;
@@ -149,7 +164,7 @@ void set_carveout(const void* kern) {
   static std::vector<const void*> done;
   static const bool on = [] {
     const char* e = getenv("FWPKM_CARVEOUT");
-    return !(e && e[0] == '0');
+    return e && e[0] == '1';
   }();
   if (!on) return;
   std::lock_guard<std::mutex> lock(mu);
@@ -158,6 +173,9 @@ void set_carveout(const void* kern) {
   cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
   done.push_back(kern);
 }
+
+thread_local int launch_priority = 0;
+thread_local bool launch_priority_set = false;
 
 bool pdl_enabled() {
   static const bool on = [] {
@@ -340,6 +358,15 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
     if (gr > dm.M) gr = dm.M;
     if (gr > fwpkm_state::MAX_GROUPS) gr = fwpkm_state::MAX_GROUPS;
     st->groups = gr < 1 ? 1 : gr;
+  }
+  {
+    const char* e = getenv("FWPKM_PRIO");
+    st->use_prio = (e && e[0] == '0') ? 0 : 1;
+    int least = 0, greatest = 0;
+    cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    st->prio_K = greatest;
+    st->prio_S = (least + greatest) / 2;
+    st->prio_V = least;
   }
   bool ok = cudaStreamCreateWithFlags(&st->sCap, cudaStreamNonBlocking) == cudaSuccess;
   for (int gi = 0; gi < fwpkm_state::MAX_GROUPS; ++gi) st->sK[gi] = st->sS[gi] = st->sV[gi] = nullptr;

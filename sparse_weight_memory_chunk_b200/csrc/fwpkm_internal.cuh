@@ -161,28 +161,40 @@ int launch_tc_keystep(const Dims& d, const Work& w, float* K1, float* K2, const 
 // default: on the paper-scale step the early-resident dependents held SM slots that the
 // other chains' kernels needed, 1.92 ms per step against 1.84 ms without).
 bool pdl_enabled();
-// Give `kern` the largest shared-memory carveout once per process (FWPKM_CARVEOUT=0 keeps
-// the driver's choice).  With every kernel on one carveout an SM never has to drain to
-// switch its L1/shared split before a CTA of another kernel (e.g. a GEMM needing 130 KB)
-// can start beside the running ones.
+// With FWPKM_CARVEOUT=1, give `kern` the largest shared-memory carveout once per process,
+// so that an SM never has to drain to switch its L1/shared split before a CTA of another
+// kernel can start beside the running ones.  Off by default: the smaller L1 it leaves
+// cost more than the switches (2.02 ms per paper-scale step against 1.73 ms without).
 void set_carveout(const void* kern);
 
 // Launch `kern` on `s`, allowing it to start while the previous kernel of the same stream
 // finishes (programmatic stream serialization).  Every kernel launched this way calls
 // pdl_wait() before it touches memory that an earlier kernel writes, so the overlap
 // covers only its launch and set-up.
+// Scheduling priority given to the kernels launched by this host thread (set around a
+// launcher call by the schedule; `launch_priority_set` false: the stream's own).
+extern thread_local int launch_priority;
+extern thread_local bool launch_priority_set;
+
 template <typename... KArgs, typename... Args>
 inline void launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  if (pdl_enabled()) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na++].val.programmaticStreamSerializationAllowed = 1;
+  }
+  if (launch_priority_set) {
+    attr[na].id = cudaLaunchAttributePriority;
+    attr[na++].val.priority = launch_priority;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cfg.numAttrs = na;
   set_carveout((const void*)kern);
   cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
