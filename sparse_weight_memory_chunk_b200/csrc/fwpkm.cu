@@ -248,10 +248,10 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
     if (ku) {
       x.zpart = (float*)take(4 * P * C * nt * 4);
       x.ppart = (float*)take(4 * P * 8 * n);
-      x.Wt = (__nv_bfloat16*)take(2 * 3 * P * n * cpad);
+      x.Wt = (__nv_bfloat16*)take(2 * 2 * P * n * cpad);
       x.qt_T = (int)((T > C ? T : C) + 63) / 64 * 64;
       x.Qt = (__nv_bfloat16*)take(2 * P * h * (size_t)x.qt_T);
-      x.wsum_part = (float*)take(4 * P * (cpad / 8) * n);
+      x.wsum_part = (float*)take(4 * P * (cpad / 16) * n);
       x.pbar_cnt = (int*)take(4 * P * ((n + 255) / 256));
     }
   }
@@ -283,7 +283,7 @@ Work group_work(const Dims& d, const Work& w, int m0) {
   if (x.ppart) x.ppart += M0 * 2 * 8 * n;
   if (x.Wt) x.Wt += M0 * 2 * n * cpad;
   if (x.Qt) x.Qt += M0 * 2 * h * (size_t)w.qt_T;
-  if (x.wsum_part) x.wsum_part += M0 * 2 * (cpad / 8) * n;
+  if (x.wsum_part) x.wsum_part += M0 * 2 * (cpad / 16) * n;
   if (x.pbar_cnt) x.pbar_cnt += M0 * 2 * ((n + 255) / 256);
   return x;
 }

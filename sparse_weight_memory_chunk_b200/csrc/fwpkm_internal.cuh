@@ -51,10 +51,10 @@ struct Work {
   float* qn;         // [M*2][max_T]       squared half-query norms
   float* zpart;      // [M*2][C][n/128][4] per-32-column partial sums of 1/(eps + D)
   float* ppart;      // [M*2][8][n]        partial column sums for pbar
-  __nv_bfloat16* Wt; // [3][M*2][n][Cpad]  key-step weights, sub-key major, bf16 pieces
+  __nv_bfloat16* Wt; // [2][M*2][n][Cpad]  key-step weights, sub-key major, bf16 pieces hi, lo
   __nv_bfloat16* Qt; // [M*2][h][qt_T]     half-queries, feature major (operand B of the key step)
   int qt_T;          // token columns of Qt (a multiple of 64)
-  float* wsum_part;  // [M*2][Cpad/8][n]   per-8-token-block sums of W
+  float* wsum_part;  // [M*2][Cpad/16][n]  per-16-token-block sums of W
   int* pbar_cnt;     // [M*2][ceil(n/256)] arrival counters of the pbar column blocks (zero between launches)
   // Every array above is memory-major except the bf16 pieces (Kpc, Wt), whose piece
   // stride is P_all problems; a Work for a group of memories is the same carve with its

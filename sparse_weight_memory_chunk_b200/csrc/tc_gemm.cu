@@ -12,9 +12,10 @@
 //      y[r][c] = (1/rms_r) sum_e x[r][e] W'[c][e] + b[c]; the epilogue applies the
 //      per-row scale and the bias and writes fp32 or bf16.
 //
-// Precision: q and v are bf16 (exact); fp32 operands (keys, W) enter as three bf16 pieces
-// hi + mid + lo (~24 significant bits), each piece pair accumulating into one fp32 TMEM
-// accumulator, so the contraction matches fp32 arithmetic to ~1e-7 relative.
+// Precision: q and v are bf16 (exact); the keys enter as three bf16 pieces hi + mid + lo
+// (~24 significant bits), each piece pair accumulating into one fp32 TMEM accumulator, so
+// the distances match fp32 arithmetic to ~1e-7 relative; the key-step weights W enter as
+// two pieces (~16 bits: the step they scale is then exact to ~1e-5 of itself).
 //
 // CTA = 18 warps: warp 0 issues TMA loads, warp 1 owns TMEM and issues the MMAs (one
 // thread), warps 2-17 drain TMEM: warp w reads TMEM lanes 32*(w%4)..+31 (tile rows) and
@@ -205,7 +206,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       } else if (g.epi == TC_EPI_KEYSTEP) {
         const int h = g.n_valid, n = g.m_valid, e0 = cg * 32;
         if (rv && e0 < h) {
-          for (int tt = 0; tt < g.wsum_tiles; ++tt) pre_s += g.wsum_part[((size_t)p * g.wsum_tiles + tt) * n + r];
+          // the partial sums are independent loads: four interleaved accumulators keep
+          // them in flight, combined in a fixed order
+          const float* wp = g.wsum_part + (size_t)p * g.wsum_tiles * n + r;
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          int tt = 0;
+          for (; tt + 4 <= g.wsum_tiles; tt += 4) {
+            a0 += wp[(size_t)tt * n];
+            a1 += wp[(size_t)(tt + 1) * n];
+            a2 += wp[(size_t)(tt + 2) * n];
+            a3 += wp[(size_t)(tt + 3) * n];
+          }
+          for (; tt < g.wsum_tiles; ++tt) a0 += wp[(size_t)tt * n];
+          pre_s = (a0 + a1) + (a2 + a3);
           const float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h + e0;
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {

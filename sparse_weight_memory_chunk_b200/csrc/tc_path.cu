@@ -125,13 +125,14 @@ tc_pbar_kernel(Dims dm, Work w, int len) {
   }
 }
 
-// W for a block of WB_T tokens and every sub-key, written sub-key major as three bf16
+// W for a block of WB_T tokens and every sub-key, written sub-key major as two bf16
 // pieces (the A operand of the key-step GEMM), plus the block's per-sub-key sum of W.
 // First L_t = sum_a P[t][a] lp[a] = (sum_a lp[a] w[t][a]) / Z_t for the block's tokens (one
 // warp per token, a row's loads all in flight), then W[t][b] = (1/len) (w/Z_t) (lp[b] -
 // L_t) w for WB_SUB sub-keys per thread (the block's rows re-read, all loads in flight).
-constexpr int WB_T = 8;
-constexpr int WB_SUB = 4;  // sub-keys per thread per pass: 256 threads x 4 = 1024
+constexpr int WB_T = 16;  // tokens per CTA (one wave of CTAs at the paper-scale shapes)
+constexpr int WB_G = 8;   // tokens per pass of the W phase (one 16-byte store per piece)
+constexpr int WB_SUB = 4; // sub-keys per thread per pass: 256 threads x 4 = 1024
 __global__ void __launch_bounds__(TP_THREADS, 3)
 tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
   pdl_wait();
@@ -174,36 +175,48 @@ tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
   const size_t pstride = (size_t)w.P_all * n * cpad;
   const int ntb = gridDim.x;
   for (int b0 = threadIdx.x; b0 < n; b0 += TP_THREADS * WB_SUB) {
-    float dd[WB_SUB][WB_T], lpb[WB_SUB];
+    float wsum[WB_SUB];
 #pragma unroll
-    for (int q = 0; q < WB_SUB; ++q) {
-      const int b = b0 + q * TP_THREADS;
-      lpb[q] = b < n ? lp[b] : 0.f;
+    for (int q = 0; q < WB_SUB; ++q) wsum[q] = 0.f;
+    for (int g0 = 0; g0 < WB_T; g0 += WB_G) {
+      const int tg = t0 + g0;
+      if (tg >= len) break;
+      float dd[WB_SUB][WB_G], lpb[WB_SUB];
 #pragma unroll
-      for (int tl = 0; tl < WB_T; ++tl) dd[q][tl] = (b < n && t0 + tl < len) ? D[(size_t)(t0 + tl) * n + b] : 0.f;
+      for (int q = 0; q < WB_SUB; ++q) {
+        const int b = b0 + q * TP_THREADS;
+        lpb[q] = b < n ? lp[b] : 0.f;
+#pragma unroll
+        for (int tl = 0; tl < WB_G; ++tl) dd[q][tl] = (b < n && tg + tl < len) ? D[(size_t)(tg + tl) * n + b] : 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < WB_SUB; ++q) {
+        const int b = b0 + q * TP_THREADS;
+        if (b >= n) continue;
+        __align__(16) __nv_bfloat16 hi[WB_G], lo[WB_G];
+#pragma unroll
+        for (int tl = 0; tl < WB_G; ++tl) {
+          float W = 0.f;
+          if (tg + tl < len) {
+            const float wv = __fdividef(1.f, dm.eps_idw + dd[q][tl]);
+            const float P_ = wv * s_invz[g0 + tl];
+            W = inv_len * P_ * (lpb[q] - s_L[g0 + tl]) * wv;
+          }
+          wsum[q] += W;
+          // two bf16 pieces (~16 significant bits): W only scales the key step, whose
+          // error this leaves at ~1e-5 of the step
+          hi[tl] = __float2bfloat16_rn(W);
+          lo[tl] = __float2bfloat16_rn(W - __bfloat162float(hi[tl]));
+        }
+        __nv_bfloat16* dst = w.Wt + ((size_t)p * n + b) * cpad + tg;
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(hi);
+        *reinterpret_cast<uint4*>(dst + pstride) = *reinterpret_cast<uint4*>(lo);
+      }
     }
 #pragma unroll
     for (int q = 0; q < WB_SUB; ++q) {
       const int b = b0 + q * TP_THREADS;
-      if (b >= n) continue;
-      __align__(16) __nv_bfloat16 hi[WB_T], mid[WB_T], lo[WB_T];
-      float wsum = 0.f;
-#pragma unroll
-      for (int tl = 0; tl < WB_T; ++tl) {
-        float W = 0.f;
-        if (t0 + tl < len) {
-          const float wv = __fdividef(1.f, dm.eps_idw + dd[q][tl]);
-          const float P_ = wv * s_invz[tl];
-          W = inv_len * P_ * (lpb[q] - s_L[tl]) * wv;
-        }
-        wsum += W;
-        split3_bf16(W, hi[tl], mid[tl], lo[tl]);
-      }
-      w.wsum_part[((size_t)p * ntb + blockIdx.x) * n + b] = wsum;
-      __nv_bfloat16* dst = w.Wt + ((size_t)p * n + b) * cpad + t0;
-      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(hi);
-      *reinterpret_cast<uint4*>(dst + pstride) = *reinterpret_cast<uint4*>(mid);
-      *reinterpret_cast<uint4*>(dst + 2 * pstride) = *reinterpret_cast<uint4*>(lo);
+      if (b < n) w.wsum_part[((size_t)p * ntb + blockIdx.x) * n + b] = wsum[q];
     }
   }
 }
@@ -313,7 +326,7 @@ int launch_tc_keystep(const Dims& d, const Work& w, float* K1, float* K2, const 
     ++launched;
   }
   CUtensorMap A, B;
-  if (!make_tmap_bf16_3d(&A, w.Wt, len, d.n, 2 * w.P_all + P, (uint64_t)cpad * 2, (uint64_t)d.n * cpad * 2))
+  if (!make_tmap_bf16_3d(&A, w.Wt, len, d.n, w.P_all + P, (uint64_t)cpad * 2, (uint64_t)d.n * cpad * 2))
     return -1;
   if (!make_tmap_bf16_3d(&B, w.Qt, w.qt_T, d.h, P, (uint64_t)w.qt_T * 2, (uint64_t)d.h * w.qt_T * 2)) return -1;
   TcGemm g = {};
@@ -321,7 +334,7 @@ int launch_tc_keystep(const Dims& d, const Work& w, float* K1, float* K2, const 
   g.k_blocks = ntt;
   g.n_tiles = 1;
   g.tiles_per_cta = 1;
-  g.a_pieces = 3; g.b_pieces = 1;
+  g.a_pieces = 2; g.b_pieces = 1;
   g.a_div = 1; g.a_xoff = 0; g.a_y0 = 0; g.a_zpiece = w.P_all; g.b_zpiece = 0; g.b_x0 = qt_t0;
   g.m_valid = d.n; g.n_valid = d.h;
   g.epi = TC_EPI_KEYSTEP;
