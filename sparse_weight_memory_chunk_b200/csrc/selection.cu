@@ -153,7 +153,7 @@ cartesian_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_ou
 // leave their survivors in shared memory, and warp 2i then finishes the token.
 constexpr int SEL_TOK = 4;
 template <int NPL>
-__global__ void __launch_bounds__(SEL_TOK * 64, 4)
+__global__ void __launch_bounds__(SEL_TOK * 64, 3)
 select_kernel(Dims dm, Work w, int wt0, int len, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
   pdl_wait();
   pdl_trigger();

@@ -35,17 +35,23 @@ __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p, l
 // r = gw * (vhat - tau), tau = z(u) or u.  Shared by the fused and the streaming path
 // so both give the same bits.
 template <typename VT, int VPL>
-__device__ __forceinline__ void residual(const Dims& dm, const float4 (&vhat)[VPL], const VT* u,
-                                         float gw, float4 (&r)[VPL], int lane) {
+__device__ __forceinline__ void load_row(const Dims& dm, const VT* u, float4 (&x)[VPL], int lane) {
   const int dv4 = dm.dv >> 2;
-  float4 x[VPL];
-  float s = 0.f;
 #pragma unroll
   for (int c = 0; c < VPL; ++c) {
     int e4 = lane + 32 * c;
-    x[c] = e4 < dv4 ? load4<VT>(u, e4) : make_float4(0.f, 0.f, 0.f, 0.f);
-    s += (x[c].x + x[c].y) + (x[c].z + x[c].w);
+    x[c] = (u && e4 < dv4) ? load4<VT>(u, e4) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+}
+
+// r from vhat and the target row already in registers (x, overwritten).
+template <int VPL>
+__device__ __forceinline__ void residual_of(const Dims& dm, const float4 (&vhat)[VPL], float4 (&x)[VPL],
+                                            float gw, float4 (&r)[VPL], int lane) {
+  const int dv4 = dm.dv >> 2;
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) s += (x[c].x + x[c].y) + (x[c].z + x[c].w);
   if (dm.flags & FWPKM_TARGET_NORM) {
     const float mean = warp_sum(s) / (float)dm.dv;
     float ss = 0.f;
@@ -72,6 +78,14 @@ __device__ __forceinline__ void residual(const Dims& dm, const float4 (&vhat)[VP
   }
 }
 
+template <typename VT, int VPL>
+__device__ __forceinline__ void residual(const Dims& dm, const float4 (&vhat)[VPL], const VT* u,
+                                         float gw, float4 (&r)[VPL], int lane) {
+  float4 x[VPL];
+  load_row<VT, VPL>(dm, u, x, lane);
+  residual_of<VPL>(dm, vhat, x, gw, r, lane);
+}
+
 // Lookahead source of local token i, or nullptr if it has no target.
 template <typename VT>
 __device__ __forceinline__ const VT* target_src(const Dims& dm, const VT* v, const VT* v_next,
@@ -83,56 +97,80 @@ __device__ __forceinline__ const VT* target_src(const Dims& dm, const VT* v, con
 }
 
 // ---------------------------------------------------------------------------
-// Gather: one warp per (memory, token).  k rows of d_v fp32 are read in rank order
-// with 16-byte loads (16 rows in flight per lane group); vhat accumulates in fp32 in
-// rank order.
+// Gather: two warps per (memory, token), GATHER_TOK tokens per CTA.  Warp half h reads the
+// rows of ranks [16h, 16h + 16) with 16-byte loads, all in flight at once, and sums them in
+// rank order; warp half 0 adds half 1's sum (a fixed order), then forms o and the residual.
+// The token's own value row and gate are loaded before the rows so that their latency
+// overlaps the gather.
 // ---------------------------------------------------------------------------
+constexpr int GATHER_TOK = VAL_WARPS / 2;
 template <typename VT, int VPL>
-__global__ void __launch_bounds__(VAL_WARPS * 32)
+__global__ void __launch_bounds__(VAL_WARPS * 32, 4)
 gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict__ v,
               const float* __restrict__ g, long long stride, int wt0, int len, float* __restrict__ o,
               int fuse_resid, const VT* __restrict__ v_next) {
   pdl_wait();
   pdl_trigger();
+  __shared__ float4 s_part[GATHER_TOK][VPL][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x * VAL_WARPS + warp;
+  const int tl = warp >> 1, half = warp & 1;
+  const int i = blockIdx.x * GATHER_TOK + tl;
   const int m = blockIdx.y;
-  if (i >= len) return;
+  const bool active = i < len;
   const int k = dm.k, dv4 = dm.dv >> 2;
   const long long tok = (long long)wt0 + i;
   int myslot = 0;
   float myw = 0.f;
-  if (lane < k) {
+  if (active && lane < k) {
     myslot = w.idx[((size_t)m * w.max_T + tok) * k + lane];
     myw = w.w[((size_t)m * w.max_T + tok) * k + lane];
+  }
+  // half 0 prefetches the token's value row and gate
+  float4 xv[VPL];
+  float gt = 0.f;
+  if (active && half == 0) {
+    gt = g[(long long)m * stride + i];
+    load_row<VT, VPL>(dm, v + ((long long)m * stride + i) * dm.dv, xv, lane);
   }
   const float4* Vm = reinterpret_cast<const float4*>(V + (size_t)m * dm.N * dm.dv);
   float4 acc[VPL];
 #pragma unroll
   for (int c = 0; c < VPL; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int r0 = half * 16, r1 = min(k, r0 + 16);
+  if (active) {
 #pragma unroll 16
-  for (int r = 0; r < k; ++r) {
-    const int slot = __shfl_sync(0xffffffffu, myslot, r);
-    const float wr = __shfl_sync(0xffffffffu, myw, r);
-    const float4* row = Vm + (size_t)slot * dv4;
+    for (int r = r0; r < r1; ++r) {
+      const int slot = __shfl_sync(0xffffffffu, myslot, r);
+      const float wr = __shfl_sync(0xffffffffu, myw, r);
+      const float4* row = Vm + (size_t)slot * dv4;
 #pragma unroll
-    for (int c = 0; c < VPL; ++c) {
-      int e4 = lane + 32 * c;
-      if (e4 < dv4) {
-        float4 x = row[e4];
-        acc[c].x = fmaf(wr, x.x, acc[c].x); acc[c].y = fmaf(wr, x.y, acc[c].y);
-        acc[c].z = fmaf(wr, x.z, acc[c].z); acc[c].w = fmaf(wr, x.w, acc[c].w);
+      for (int c = 0; c < VPL; ++c) {
+        int e4 = lane + 32 * c;
+        if (e4 < dv4) {
+          float4 x = row[e4];
+          acc[c].x = fmaf(wr, x.x, acc[c].x); acc[c].y = fmaf(wr, x.y, acc[c].y);
+          acc[c].z = fmaf(wr, x.z, acc[c].z); acc[c].w = fmaf(wr, x.w, acc[c].w);
+        }
       }
     }
   }
-  const float gt = g[(long long)m * stride + i];
-  const VT* vt = v + ((long long)m * stride + i) * dm.dv;
+  if (half == 1) {
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) s_part[tl][c][lane] = acc[c];
+  }
+  __syncthreads();
+  if (half == 1 || !active) return;
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) {
+    const float4 b = s_part[tl][c][lane];
+    acc[c].x += b.x; acc[c].y += b.y; acc[c].z += b.z; acc[c].w += b.w;
+  }
   float4* orow = reinterpret_cast<float4*>(o + ((long long)m * stride + i) * dm.dv);
 #pragma unroll
   for (int c = 0; c < VPL; ++c) {
     int e4 = lane + 32 * c;
     if (e4 < dv4) {
-      float4 x = load4<VT>(vt, e4);
+      const float4 x = xv[c];
       float4 y;
       y.x = gt * acc[c].x + (1.f - gt) * x.x; y.y = gt * acc[c].y + (1.f - gt) * x.y;
       y.z = gt * acc[c].z + (1.f - gt) * x.z; y.w = gt * acc[c].w + (1.f - gt) * x.w;
@@ -305,7 +343,7 @@ int launch_gather(const Dims& d, const Work& w, const float* V, const void* v, c
                   long long stride, int wt0, int len, float* o, bool fuse_resid, const void* v_next,
                   cudaStream_t s) {
   if (len <= 0) return 0;
-  dim3 grid((len + VAL_WARPS - 1) / VAL_WARPS, d.M);
+  dim3 grid((len + GATHER_TOK - 1) / GATHER_TOK, d.M);
   if (d.qv_bf16) {
     FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(gather_kernel<__nv_bfloat16, VPL>, grid, VAL_WARPS * 32, 0, s, 
         d, w, V, (const __nv_bfloat16*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0,
