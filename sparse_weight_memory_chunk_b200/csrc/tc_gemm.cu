@@ -42,14 +42,8 @@ constexpr int TC_THREADS = (2 + TC_EPI_WARPS) * 32;
 constexpr uint32_t TC_TMEM_COLS = 256;
 constexpr uint64_t TC_TIMEOUT_NS = 200ull * 1000 * 1000;
 
-// Epilogue staging: per epilogue warp a 32 x 32 fp32 block with rows padded to 36 floats
-// (16-byte aligned, conflict-free float4 access by quarter-warps), so that the distance
-// rows leave as whole 128-byte lines instead of one 16-byte piece per row and lane.
-constexpr int TC_STAGE_LD = 36;
-constexpr size_t TC_STAGE_BYTES = (size_t)TC_EPI_WARPS * 32 * TC_STAGE_LD * 4;
-
 size_t tc_smem_bytes(int npieces) {
-  return 1024 + (size_t)TC_STAGES * npieces * TC_TILE_BYTES + 256 + TC_STAGE_BYTES;
+  return 1024 + (size_t)TC_STAGES * npieces * TC_TILE_BYTES + 256;
 }
 
 __device__ __forceinline__ bool wait_deadline(uint64_t* bar, uint32_t parity, uint64_t deadline) {
@@ -79,7 +73,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* normbar = drain + 1;
   uint32_t* tmem_slot = (uint32_t*)(normbar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  float* stage_all = (float*)(tiles + (size_t)TC_STAGES * npc * TC_TILE_BYTES + 256);
   __shared__ float s_norm[4][TC_BM];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -212,41 +205,26 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
       } else if (g.epi == TC_EPI_KEYSTEP) {
         const int h = g.n_valid, n = g.m_valid, e0 = cg * 32;
-        if (e0 < h) {  // warp-uniform
-          if (rv) {
-            // the partial sums are independent loads: four interleaved accumulators keep
-            // them in flight, combined in a fixed order
-            const float* wp = g.wsum_part + (size_t)p * g.wsum_tiles * n + r;
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-            int tt = 0;
-            for (; tt + 4 <= g.wsum_tiles; tt += 4) {
-              a0 += wp[(size_t)tt * n];
-              a1 += wp[(size_t)(tt + 1) * n];
-              a2 += wp[(size_t)(tt + 2) * n];
-              a3 += wp[(size_t)(tt + 3) * n];
-            }
-            for (; tt < g.wsum_tiles; ++tt) a0 += wp[(size_t)tt * n];
-            pre_s = (a0 + a1) + (a2 + a3);
+        if (rv && e0 < h) {
+          // the partial sums are independent loads: four interleaved accumulators keep
+          // them in flight, combined in a fixed order
+          const float* wp = g.wsum_part + (size_t)p * g.wsum_tiles * n + r;
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          int tt = 0;
+          for (; tt + 4 <= g.wsum_tiles; tt += 4) {
+            a0 += wp[(size_t)tt * n];
+            a1 += wp[(size_t)(tt + 1) * n];
+            a2 += wp[(size_t)(tt + 2) * n];
+            a3 += wp[(size_t)(tt + 3) * n];
           }
-          // the warp's 32 keys x 32 features, read as whole lines and transposed through
-          // shared memory to one key per lane
-          float* stg = stage_all + (size_t)(warp - 2) * 32 * TC_STAGE_LD;
-          const float* Kb = (jh == 0 ? g.K1 : g.K2) + (size_t)m * n * h + e0;
-          const int rsub = lane >> 3, csub = (lane & 7) * 4;
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int rl = it * 4 + rsub, rr = mt * TC_BM + q * 32 + rl;
-            const float4 k4 = rr < n ? *reinterpret_cast<const float4*>(Kb + (size_t)rr * h + csub)
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4*>(stg + rl * TC_STAGE_LD + csub) = k4;
-          }
-          __syncwarp();
+          for (; tt < g.wsum_tiles; ++tt) a0 += wp[(size_t)tt * n];
+          pre_s = (a0 + a1) + (a2 + a3);
+          const float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h + e0;
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
-            const float4 k4 = *reinterpret_cast<const float4*>(stg + lane * TC_STAGE_LD + i);
+            const float4 k4 = *reinterpret_cast<const float4*>(K + i);
             pre[i] = k4.x; pre[i + 1] = k4.y; pre[i + 2] = k4.z; pre[i + 3] = k4.w;
           }
-          __syncwarp();
         }
       }
       // one lane waits; the verdict is shared so the warp stays converged for tcgen05.ld
@@ -273,24 +251,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             dv[i] = fmaxf((rq + pre[i]) - 2.f * __uint_as_float(v[i]), 0.f);
             zacc += __fdividef(1.f, g.eps + dv[i]);
           }
-          // transpose through shared memory: lane `lane` holds row q*32 + lane; each store
-          // below writes four rows x 32 columns (four full 128-byte lines)
-          float* stg = stage_all + (size_t)(warp - 2) * 32 * TC_STAGE_LD;
+          if (rv) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(stg + lane * TC_STAGE_LD + i) = make_float4(dv[i], dv[i + 1], dv[i + 2], dv[i + 3]);
-          __syncwarp();
-          const int rsub = lane >> 3, csub = (lane & 7) * 4;
-          float* obase = g.out + (size_t)p * g.out_pstride + c0 + csub;
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int rl = it * 4 + rsub;
-            const int rr = mt * TC_BM + q * 32 + rl;
-            if (rr < g.m_valid)
-              *reinterpret_cast<float4*>(obase + (size_t)rr * g.out_ld) =
-                  *reinterpret_cast<const float4*>(stg + rl * TC_STAGE_LD + csub);
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(out + c0 + i) = make_float4(dv[i], dv[i + 1], dv[i + 2], dv[i + 3]);
           }
-          __syncwarp();
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -334,45 +299,32 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int n = g.m_valid;
         const int e0 = cg * 32;
         float ss = 0.f;
-        if (e0 < h) {  // warp-uniform
+        if (rv && e0 < h) {
           const float wsum = pre_s;
+          float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h;
           const size_t pstride = (size_t)g.piece_P * n * h;
           __nv_bfloat16* pc = g.Kpc + ((size_t)p * n + r) * h;
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
+            const int e = e0 + i;
+            float kin[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) kin[u] = pre[i + u];
+            float kout[8];
             __align__(16) __nv_bfloat16 hi[8], mid[8], lo[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-              const float kin = pre[i + u];
-              const float grad = 2.f * (__uint_as_float(v[i + u]) - wsum * kin);
-              pre[i + u] = kin - g.lr * grad;  // the new key
-              ss += pre[i + u] * pre[i + u];
-              split3(pre[i + u], hi[u], mid[u], lo[u]);
+              const float grad = 2.f * (__uint_as_float(v[i + u]) - wsum * kin[u]);
+              kout[u] = kin[u] - g.lr * grad;
+              ss += kout[u] * kout[u];
+              split3(kout[u], hi[u], mid[u], lo[u]);
             }
-            if (rv) {
-              const int e = e0 + i;
-              *reinterpret_cast<uint4*>(pc + e) = *reinterpret_cast<uint4*>(hi);
-              *reinterpret_cast<uint4*>(pc + pstride + e) = *reinterpret_cast<uint4*>(mid);
-              *reinterpret_cast<uint4*>(pc + 2 * pstride + e) = *reinterpret_cast<uint4*>(lo);
-            }
+            *reinterpret_cast<float4*>(K + e) = make_float4(kout[0], kout[1], kout[2], kout[3]);
+            *reinterpret_cast<float4*>(K + e + 4) = make_float4(kout[4], kout[5], kout[6], kout[7]);
+            *reinterpret_cast<uint4*>(pc + e) = *reinterpret_cast<uint4*>(hi);
+            *reinterpret_cast<uint4*>(pc + pstride + e) = *reinterpret_cast<uint4*>(mid);
+            *reinterpret_cast<uint4*>(pc + 2 * pstride + e) = *reinterpret_cast<uint4*>(lo);
           }
-          // the new keys leave through shared memory as whole lines
-          float* stg = stage_all + (size_t)(warp - 2) * 32 * TC_STAGE_LD;
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(stg + lane * TC_STAGE_LD + i) = make_float4(pre[i], pre[i + 1], pre[i + 2], pre[i + 3]);
-          __syncwarp();
-          float* Kb = (jh == 0 ? g.K1 : g.K2) + (size_t)m * n * h + e0;
-          const int rsub = lane >> 3, csub = (lane & 7) * 4;
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int rl = it * 4 + rsub, rr = mt * TC_BM + q * 32 + rl;
-            if (rr < n)
-              *reinterpret_cast<float4*>(Kb + (size_t)rr * h + csub) =
-                  *reinterpret_cast<const float4*>(stg + rl * TC_STAGE_LD + csub);
-          }
-          __syncwarp();
-          if (!rv) ss = 0.f;
         }
         // squared norm of the new key: the four column groups' partials, summed in order
         // by the column-group-0 warp once all 16 warps have published theirs (one tile per
