@@ -257,8 +257,15 @@ uint64_t fwpkm_launch_count(void);
  * returns the summed duration (ms) and the number of timed launches since the last
  * reset, then resets.  Graph replays overwrite their own events, so after graph
  * replays it covers the last replay. */
+#define FWPKM_PROFILE_ALL 100 /* fwpkm_profile_kernel kind: time every launch */
 fwpkm_status fwpkm_profile_kernel(fwpkm_state* st, int kind);
 fwpkm_status fwpkm_kernel_time(fwpkm_state* st, double* total_ms, int* launches);
+
+/* The timed launches of the last call (in enqueue order, at most `max`): kind, start and
+ * end in ms from the earliest start.  *n receives the number of timed launches.  Waits
+ * for the events.  A diagnostic of the schedule (events themselves add some latency). */
+fwpkm_status fwpkm_kernel_timeline(fwpkm_state* st, int max, int* kinds, float* start_ms, float* end_ms,
+                                   int* n);
 
 #ifdef __cplusplus
 }

@@ -42,7 +42,8 @@ struct fwpkm_state {
   int len;
   long long stride;
   // per-kernel timing
-  int prof_kind;
+  int prof_kind;  // kernel kind timed with events; FWPKM_PROFILE_ALL: every kind
+  std::vector<int> ev_kind;  // kind of each timed launch (event pair)
   std::vector<cudaEvent_t> ev;
   int ev_used;
   int host_error;  // a launch could not be set up (e.g. tensor map encoding failed)
@@ -129,7 +130,8 @@ template <class F>
 void run(fwpkm_state* st, int kind, cudaStream_t s, F&& f) {
   launch_priority_set = st->use_prio != 0 && !st->serial;
   launch_priority = launch_priority_set ? stream_priority(st, s) : 0;
-  const bool prof = st->prof_kind == kind && st->ev_used + 2 <= (int)st->ev.size();
+  const bool prof = (st->prof_kind == kind || st->prof_kind == FWPKM_PROFILE_ALL) &&
+                    st->ev_used + 2 <= (int)st->ev.size();
   // Under stream capture a plain record is only a dependency marker; timing events must
   // become event-record nodes of the graph.
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
@@ -140,6 +142,7 @@ void run(fwpkm_state* st, int kind, cudaStream_t s, F&& f) {
   launch_priority_set = false;
   if (prof) {
     cudaEventRecordWithFlags(st->ev[st->ev_used + 1], s, rec_flags);
+    st->ev_kind[st->ev_used / 2] = kind;
     st->ev_used += 2;
   }
   if (nl < 0) st->host_error = 1;
@@ -691,14 +694,41 @@ fwpkm_status fwpkm_sync(fwpkm_state* st, void* stream) {
 }
 
 fwpkm_status fwpkm_profile_kernel(fwpkm_state* st, int kind) {
-  if (!st || kind < 0 || kind > KK_LAST) return FWPKM_ERR_INVALID_ARG;
+  if (!st || ((kind < 0 || kind > KK_LAST) && kind != FWPKM_PROFILE_ALL)) return FWPKM_ERR_INVALID_ARG;
   if (kind != 0 && st->ev.empty()) {
     st->ev.resize(4096);
+    st->ev_kind.assign(2048, 0);
     for (auto& e : st->ev)
       if (cudaEventCreate(&e) != cudaSuccess) return FWPKM_ERR_CUDA;
   }
   st->prof_kind = kind;
   st->ev_used = 0;
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_kernel_timeline(fwpkm_state* st, int max, int* kinds, float* start_ms, float* end_ms,
+                                   int* n) {
+  if (!st || !n || max < 0 || (max > 0 && (!kinds || !start_ms || !end_ms))) return FWPKM_ERR_INVALID_ARG;
+  const int pairs = st->ev_used / 2;
+  *n = pairs;
+  if (pairs == 0) return FWPKM_OK;
+  if (cudaEventSynchronize(st->ev[st->ev_used - 1]) != cudaSuccess) return FWPKM_ERR_CUDA;
+  // the earliest start is the origin
+  int first = 0;
+  for (int i = 1; i < pairs; ++i) {
+    float d = 0.f;
+    if (cudaEventElapsedTime(&d, st->ev[2 * first], st->ev[2 * i]) != cudaSuccess) return FWPKM_ERR_CUDA;
+    if (d < 0.f) first = i;
+  }
+  for (int i = 0; i < pairs && i < max; ++i) {
+    float a = 0.f, b = 0.f;
+    if (cudaEventElapsedTime(&a, st->ev[2 * first], st->ev[2 * i]) != cudaSuccess ||
+        cudaEventElapsedTime(&b, st->ev[2 * first], st->ev[2 * i + 1]) != cudaSuccess)
+      return FWPKM_ERR_CUDA;
+    kinds[i] = st->ev_kind[i];
+    start_ms[i] = a;
+    end_ms[i] = b;
+  }
   return FWPKM_OK;
 }
 

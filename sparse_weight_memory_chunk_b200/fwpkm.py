@@ -20,7 +20,8 @@ F32, BF16 = 0, 1
 KEY_UPDATE, TARGET_NORM, LOOKAHEAD, GATE_WEIGHT = 1, 2, 4, 8
 DEFAULT_FLAGS = TARGET_NORM | LOOKAHEAD | GATE_WEIGHT
 KIND = {"gather": 1, "write": 2, "score": 3, "cartesian": 4, "sort": 5, "address": 6, "other": 7, "topk": 8,
-        "prep": 9, "pbar": 10, "wbuild": 11}
+        "prep": 9, "pbar": 10, "wbuild": 11, "all": 100}
+KIND_NAME = {v: k for k, v in KIND.items()}
 
 
 class FwpkmError(RuntimeError):
@@ -85,6 +86,7 @@ def lib():
             "fwpkm_profile_kernel": ([_P, ctypes.c_int], ctypes.c_int),
             "fwpkm_kernel_time": ([_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)],
                                   ctypes.c_int),
+            "fwpkm_kernel_timeline": ([_P, ctypes.c_int, _P, _P, _P, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
             "fwpkm_layer_workspace_size": ([ctypes.POINTER(LayerConfig), ctypes.POINTER(ctypes.c_size_t)],
                                            ctypes.c_int),
             "fwpkm_layer_init": ([ctypes.POINTER(LayerConfig), _P, ctypes.c_size_t, ctypes.POINTER(_P)],
@@ -187,6 +189,18 @@ class State:
     def profile_kernel(self, kind):
         kind = KIND.get(kind, kind) if isinstance(kind, str) else kind
         _check(lib().fwpkm_profile_kernel(self.handle, int(kind)), "profile_kernel")
+
+    def kernel_timeline(self, max_launches=4096):
+        """[(kind name, start ms, end ms)] of the launches timed in the last call."""
+        import numpy as np
+        kinds = np.zeros(max_launches, dtype=np.int32)
+        t0 = np.zeros(max_launches, dtype=np.float32)
+        t1 = np.zeros(max_launches, dtype=np.float32)
+        n = ctypes.c_int(0)
+        _check(lib().fwpkm_kernel_timeline(self.handle, max_launches, kinds.ctypes.data_as(_P), t0.ctypes.data_as(_P),
+                                           t1.ctypes.data_as(_P), ctypes.byref(n)), "kernel_timeline")
+        m = min(n.value, max_launches)
+        return [(KIND_NAME.get(int(kinds[i]), str(int(kinds[i]))), float(t0[i]), float(t1[i])) for i in range(m)]
 
     def kernel_time(self):
         ms = ctypes.c_double(0.0)
