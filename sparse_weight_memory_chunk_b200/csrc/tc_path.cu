@@ -92,9 +92,17 @@ tc_pbar_kernel(Dims dm, Work w, int len) {
   const int t0 = (sl * len) / PBAR_SLICES, t1 = ((sl + 1) * len) / PBAR_SLICES;
   const int nt = (dm.n + 127) / 128 * 4;  // 4 column groups per 128-column tile
   for (int t = t0 + threadIdx.x; t < t1; t += TP_THREADS) {
-    const float* zp = w.zpart + ((size_t)p * dm.C + t) * nt;
+    // Z_t from the scoring epilogue's nt partial sums (a multiple of 4, 16-byte aligned):
+    // all loads issued together, summed in order
+    const float4* zp = reinterpret_cast<const float4*>(w.zpart + ((size_t)p * dm.C + t) * nt);
     float z = 0.f;
-    for (int u = 0; u < nt; ++u) z += zp[u];
+    for (int u0 = 0; u0 < nt / 4; u0 += 8) {
+      float4 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = u0 + u < nt / 4 ? zp[u0 + u] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) z = (((z + x[u].x) + x[u].y) + x[u].z) + x[u].w;
+    }
     s_invz[t - t0] = 1.f / z;
     if (blockIdx.x == 0) w.Z[(size_t)p * dm.C + t] = z;
   }
