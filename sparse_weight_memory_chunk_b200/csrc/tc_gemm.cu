@@ -35,23 +35,15 @@ using namespace sm100;
 
 constexpr int TC_BM = 128, TC_BN = 128, TC_BK = 64;
 constexpr int TC_TILE_BYTES = TC_BM * TC_BK * 2;  // 16 KiB, also the B tile (TC_BN == TC_BM)
-constexpr int TC_MAX_STAGES = 2;
+// two stages (<= 128 KiB of tiles) leave room on the SM for the CTAs of the other chains
+constexpr int TC_STAGES = 2;
 constexpr int TC_EPI_WARPS = 16;
 constexpr int TC_THREADS = (2 + TC_EPI_WARPS) * 32;
 constexpr uint32_t TC_TMEM_COLS = 256;
 constexpr uint64_t TC_TIMEOUT_NS = 200ull * 1000 * 1000;
-// Two CTAs share an SM (registers: 576 threads x <= 56; TMEM: 2 x 256 columns); the
-// shared-memory request never goes below this, so that a third CTA never fits and waits
-// for TMEM.
-constexpr size_t TC_MIN_SMEM = 80 * 1024;
-
-// Pipeline stages for `npieces` operand tiles per k-block: two while they fit in half an
-// SM's shared memory, else one (the second CTA on the SM overlaps it).
-int tc_stages(int npieces) { return 2 * npieces * TC_TILE_BYTES <= 100 * 1024 ? 2 : 1; }
 
 size_t tc_smem_bytes(int npieces) {
-  const size_t b = 1024 + (size_t)tc_stages(npieces) * npieces * TC_TILE_BYTES + 256;
-  return b < TC_MIN_SMEM ? TC_MIN_SMEM : b;
+  return 1024 + (size_t)TC_STAGES * npieces * TC_TILE_BYTES + 256;
 }
 
 __device__ __forceinline__ bool wait_deadline(uint64_t* bar, uint32_t parity, uint64_t deadline) {
@@ -67,16 +59,15 @@ __device__ __forceinline__ void split3(float x, __nv_bfloat16& hi, __nv_bfloat16
   lo = __float2bfloat16_rn(r - __bfloat162float(mid));
 }
 
-__global__ void __launch_bounds__(TC_THREADS, 2)
+__global__ void __launch_bounds__(TC_THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcGemm g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int npc = g.a_pieces + g.b_pieces;
-  const int S = g.stages;
   uint8_t* tiles = smem;
-  uint64_t* full = (uint64_t*)(tiles + (size_t)S * npc * TC_TILE_BYTES);
-  uint64_t* empty = full + TC_MAX_STAGES;
-  uint64_t* accf = empty + TC_MAX_STAGES;
+  uint64_t* full = (uint64_t*)(tiles + (size_t)TC_STAGES * npc * TC_TILE_BYTES);
+  uint64_t* empty = full + TC_STAGES;
+  uint64_t* accf = empty + TC_STAGES;
   uint64_t* acce = accf + 2;
   uint64_t* drain = acce + 2;
   uint64_t* normbar = drain + 1;
@@ -90,7 +81,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int ntiles = min(g.n_tiles, nt0 + g.tiles_per_cta) - nt0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < TC_STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -126,9 +117,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int nt = nt0 + j;
       bool ok = true;
       for (int kb = 0; kb < g.k_blocks; ++kb) {
-        const int s = issued % S;
-        const uint32_t ph = (issued / S) & 1;
-        if (issued >= S && !mbar_wait(&empty[s], ph ^ 1, abort_flag, deadline)) {
+        const int s = issued % TC_STAGES;
+        const uint32_t ph = (issued / TC_STAGES) & 1;
+        if (issued >= TC_STAGES && !mbar_wait(&empty[s], ph ^ 1, abort_flag, deadline)) {
           ok = false;
           break;
         }
@@ -156,8 +147,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t dt = tmem + (uint32_t)(b * TC_BN);
       bool ok = true;
       for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1;
+        const int s = it % TC_STAGES;
+        const uint32_t ph = (it / TC_STAGES) & 1;
         if (!mbar_wait(&full[s], ph, abort_flag, deadline)) {
           ok = false;
           break;
@@ -181,8 +172,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     wait_deadline(drain, 0, deadline + TC_TIMEOUT_NS);
   } else if (ntiles > 0 && warp >= 2) {
     // ---------------- epilogue: 16 warps; warp w reads TMEM lane quarter w%4 (tile rows
-    // 32*(w%4)..+31, one per thread) and column group (w-2)/4 (32 columns), in two halves
-    // of 16 columns (register budget of two CTAs per SM) ----------------
+    // 32*(w%4)..+31, one per thread) and column group (w-2)/4 (32 columns) ----------------
     const int q = warp & 3;
     const int cg = (warp - 2) >> 2;
     const int row = q * 32 + lane;
@@ -194,141 +184,151 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int nt = nt0 + j;
       const int r = mt * TC_BM + row;
       const bool rv = r < g.m_valid;
-      // operands that do not depend on the accumulator are loaded while the MMAs run
-      float pre_s = 0.f;
+      // operands of the epilogue that do not depend on the accumulator are loaded while
+      // the MMAs run: DIST the row norm and 32 column norms, KEYSTEP sum_t W and the key
+      float pre_s = 0.f, pre[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) pre[i] = 0.f;
       if (g.epi == TC_EPI_DIST) {
+        const int c0 = nt * TC_BN + cg * 32;
         pre_s = rv ? g.rowv[(size_t)p * g.rowv_pstride + g.rowv_off + r] : 0.f;
-      } else if (g.epi == TC_EPI_KEYSTEP && rv && cg * 32 < g.n_valid) {
-        // the partial sums are independent loads: four interleaved accumulators keep
-        // them in flight, combined in a fixed order
-        const int n = g.m_valid;
-        const float* wp = g.wsum_part + (size_t)p * g.wsum_tiles * n + r;
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-        int tt = 0;
-        for (; tt + 4 <= g.wsum_tiles; tt += 4) {
-          a0 += wp[(size_t)tt * n];
-          a1 += wp[(size_t)(tt + 1) * n];
-          a2 += wp[(size_t)(tt + 2) * n];
-          a3 += wp[(size_t)(tt + 3) * n];
+        const float* kn = g.colv + (size_t)p * g.colv_pstride;
+        if (c0 + 32 <= g.n_valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(kn + c0 + i);
+            pre[i] = k4.x; pre[i + 1] = k4.y; pre[i + 2] = k4.z; pre[i + 3] = k4.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pre[i] = c0 + i < g.n_valid ? kn[c0 + i] : 0.f;
         }
-        for (; tt < g.wsum_tiles; ++tt) a0 += wp[(size_t)tt * n];
-        pre_s = (a0 + a1) + (a2 + a3);
+      } else if (g.epi == TC_EPI_KEYSTEP) {
+        const int h = g.n_valid, n = g.m_valid, e0 = cg * 32;
+        if (rv && e0 < h) {
+          // the partial sums are independent loads: four interleaved accumulators keep
+          // them in flight, combined in a fixed order
+          const float* wp = g.wsum_part + (size_t)p * g.wsum_tiles * n + r;
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          int tt = 0;
+          for (; tt + 4 <= g.wsum_tiles; tt += 4) {
+            a0 += wp[(size_t)tt * n];
+            a1 += wp[(size_t)(tt + 1) * n];
+            a2 += wp[(size_t)(tt + 2) * n];
+            a3 += wp[(size_t)(tt + 3) * n];
+          }
+          for (; tt < g.wsum_tiles; ++tt) a0 += wp[(size_t)tt * n];
+          pre_s = (a0 + a1) + (a2 + a3);
+          const float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h + e0;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(K + i);
+            pre[i] = k4.x; pre[i + 1] = k4.y; pre[i + 2] = k4.z; pre[i + 3] = k4.w;
+          }
+        }
       }
       // one lane waits; the verdict is shared so the warp stays converged for tcgen05.ld
       int ok = lane == 0 ? (mbar_wait(&accf[b], aph, abort_flag, deadline) ? 1 : 0) : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      float zacc = 0.f, ss = 0.f;
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t v[16];
-        tmem_ld16(lane_base + (uint32_t)(b * TC_BN + cg * 32 + hh * 16), v);
-        tmem_wait_ld();
-        if (hh == 1) {
-          // accumulator drained: hand the buffer back before the (longer) epilogue math
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acce[b]);
-        }
-        if (g.epi == TC_EPI_DIST) {
-          const int c0 = nt * TC_BN + cg * 32 + hh * 16;
-          const float rq = pre_s;
-          const float* kn = g.colv + (size_t)p * g.colv_pstride;
-          float* out = g.out + ((size_t)p * g.out_pstride + (size_t)r * g.out_ld);
-          if (c0 + 16 <= g.n_valid) {
-            float dv[16];
+      uint32_t v[32];
+      tmem_ld32(lane_base + (uint32_t)(b * TC_BN + cg * 32), v);
+      tmem_wait_ld();
+      // accumulator drained: hand the buffer back before the (longer) epilogue math
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[b]);
+      if (g.epi == TC_EPI_DIST) {
+        const int c0 = nt * TC_BN + cg * 32;
+        const float rq = pre_s;
+        float* out = g.out + ((size_t)p * g.out_pstride + (size_t)r * g.out_ld);
+        float dv[32];
+        float zacc = 0.f;
+        if (c0 + 32 <= g.n_valid) {
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-              const float4 k4 = *reinterpret_cast<const float4*>(kn + c0 + i);
-              const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+          for (int i = 0; i < 32; ++i) {
+            dv[i] = fmaxf((rq + pre[i]) - 2.f * __uint_as_float(v[i]), 0.f);
+            zacc += __fdividef(1.f, g.eps + dv[i]);
+          }
+          if (rv) {
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                dv[i + u] = fmaxf((rq + kk[u]) - 2.f * __uint_as_float(v[i + u]), 0.f);
-                zacc += __fdividef(1.f, g.eps + dv[i + u]);
-              }
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(out + c0 + i) = make_float4(dv[i], dv[i + 1], dv[i + 2], dv[i + 3]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int c = c0 + i;
+            dv[i] = fmaxf((rq + pre[i]) - 2.f * __uint_as_float(v[i]), 0.f);
+            if (c < g.n_valid) {
+              zacc += __fdividef(1.f, g.eps + dv[i]);
+              if (rv) out[c] = dv[i];
             }
-            if (rv) {
+          }
+        }
+        if (rv && g.zpart)
+          g.zpart[(((size_t)p * g.zpart_pstride + r) * g.n_tiles + nt) * 4 + cg] = zacc;
+      } else if (g.epi == TC_EPI_PROJ) {
+        const int c0 = nt * TC_BN + cg * 32;
+        if (rv && c0 < g.n_valid) {
+          const float rs = g.rowscale[r];
+          float y[32];
 #pragma unroll
-              for (int i = 0; i < 16; i += 4)
-                *reinterpret_cast<float4*>(out + c0 + i) = make_float4(dv[i], dv[i + 1], dv[i + 2], dv[i + 3]);
+          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]) * rs + (g.bias ? g.bias[c0 + i] : 0.f);
+          const bool first = c0 < g.split;
+          const size_t off = first ? (size_t)r * g.ld0 + c0 : (size_t)r * g.ld1 + (c0 - g.split);
+          if (g.out_bf16) {
+            __nv_bfloat16* dst = (__nv_bfloat16*)(first ? g.pout0 : g.pout1) + off;
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              __align__(16) __nv_bfloat16 yb[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) yb[u] = __float2bfloat16_rn(y[i + u]);
+              *reinterpret_cast<uint4*>(dst + i) = *reinterpret_cast<uint4*>(yb);
             }
           } else {
+            float* dst = (float*)(first ? g.pout0 : g.pout1) + off;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int c = c0 + i;
-              const float kv = c < g.n_valid ? kn[c] : 0.f;
-              const float dd = fmaxf((rq + kv) - 2.f * __uint_as_float(v[i]), 0.f);
-              if (c < g.n_valid) {
-                zacc += __fdividef(1.f, g.eps + dd);
-                if (rv) out[c] = dd;
-              }
-            }
-          }
-        } else if (g.epi == TC_EPI_PROJ) {
-          const int c0 = nt * TC_BN + cg * 32 + hh * 16;
-          if (rv && c0 < g.n_valid) {
-            const float rs = g.rowscale[r];
-            float y[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) y[i] = __uint_as_float(v[i]) * rs + (g.bias ? g.bias[c0 + i] : 0.f);
-            const bool first = c0 < g.split;
-            const size_t off = first ? (size_t)r * g.ld0 + c0 : (size_t)r * g.ld1 + (c0 - g.split);
-            if (g.out_bf16) {
-              __nv_bfloat16* dst = (__nv_bfloat16*)(first ? g.pout0 : g.pout1) + off;
-#pragma unroll
-              for (int i = 0; i < 16; i += 8) {
-                __align__(16) __nv_bfloat16 yb[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) yb[u] = __float2bfloat16_rn(y[i + u]);
-                *reinterpret_cast<uint4*>(dst + i) = *reinterpret_cast<uint4*>(yb);
-              }
-            } else {
-              float* dst = (float*)(first ? g.pout0 : g.pout1) + off;
-#pragma unroll
-              for (int i = 0; i < 16; i += 4)
-                *reinterpret_cast<float4*>(dst + i) = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
-            }
-          }
-        } else {  // TC_EPI_KEYSTEP: row = sub-key b, columns = features e (one tile covers h)
-          const int h = g.n_valid;
-          const int n = g.m_valid;
-          const int e0 = cg * 32 + hh * 16;
-          if (rv && e0 < h) {
-            const float wsum = pre_s;
-            float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h;
-            const size_t pstride = (size_t)g.piece_P * n * h;
-            __nv_bfloat16* pc = g.Kpc + ((size_t)p * n + r) * h;
-#pragma unroll
-            for (int i = 0; i < 16; i += 8) {
-              const int e = e0 + i;
-              const float4 k0 = *reinterpret_cast<const float4*>(K + e);
-              const float4 k1 = *reinterpret_cast<const float4*>(K + e + 4);
-              const float kin[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-              float kout[8];
-              __align__(16) __nv_bfloat16 hi[8], mid[8], lo[8];
-#pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                const float grad = 2.f * (__uint_as_float(v[i + u]) - wsum * kin[u]);
-                kout[u] = kin[u] - g.lr * grad;
-                ss += kout[u] * kout[u];
-                split3(kout[u], hi[u], mid[u], lo[u]);
-              }
-              *reinterpret_cast<float4*>(K + e) = make_float4(kout[0], kout[1], kout[2], kout[3]);
-              *reinterpret_cast<float4*>(K + e + 4) = make_float4(kout[4], kout[5], kout[6], kout[7]);
-              *reinterpret_cast<uint4*>(pc + e) = *reinterpret_cast<uint4*>(hi);
-              *reinterpret_cast<uint4*>(pc + pstride + e) = *reinterpret_cast<uint4*>(mid);
-              *reinterpret_cast<uint4*>(pc + 2 * pstride + e) = *reinterpret_cast<uint4*>(lo);
-            }
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + i) = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
           }
         }
-      }
-      if (g.epi == TC_EPI_DIST) {
-        if (rv && g.zpart) g.zpart[(((size_t)p * g.zpart_pstride + r) * g.n_tiles + nt) * 4 + cg] = zacc;
-      } else if (g.epi == TC_EPI_KEYSTEP) {
+      } else {  // TC_EPI_KEYSTEP: row = sub-key b, columns = features e (one tile covers h)
+        const int h = g.n_valid;
+        const int n = g.m_valid;
+        const int e0 = cg * 32;
+        float ss = 0.f;
+        if (rv && e0 < h) {
+          const float wsum = pre_s;
+          float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h;
+          const size_t pstride = (size_t)g.piece_P * n * h;
+          __nv_bfloat16* pc = g.Kpc + ((size_t)p * n + r) * h;
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            const int e = e0 + i;
+            float kin[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) kin[u] = pre[i + u];
+            float kout[8];
+            __align__(16) __nv_bfloat16 hi[8], mid[8], lo[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float grad = 2.f * (__uint_as_float(v[i + u]) - wsum * kin[u]);
+              kout[u] = kin[u] - g.lr * grad;
+              ss += kout[u] * kout[u];
+              split3(kout[u], hi[u], mid[u], lo[u]);
+            }
+            *reinterpret_cast<float4*>(K + e) = make_float4(kout[0], kout[1], kout[2], kout[3]);
+            *reinterpret_cast<float4*>(K + e + 4) = make_float4(kout[4], kout[5], kout[6], kout[7]);
+            *reinterpret_cast<uint4*>(pc + e) = *reinterpret_cast<uint4*>(hi);
+            *reinterpret_cast<uint4*>(pc + pstride + e) = *reinterpret_cast<uint4*>(mid);
+            *reinterpret_cast<uint4*>(pc + 2 * pstride + e) = *reinterpret_cast<uint4*>(lo);
+          }
+        }
         // squared norm of the new key: the four column groups' partials, summed in order
         // by the column-group-0 warp once all 16 warps have published theirs (one tile per
         // CTA in this mode, so the barrier has a single phase; the wait is bounded)
-        const int n = g.m_valid;
         s_norm[cg][row] = ss;
         __syncwarp();
         if (lane == 0) mbar_arrive(normbar);
@@ -346,8 +346,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   __syncwarp();
   if (warp == 0 && lane == 0 && *abort_flag) {
     // let the copies this CTA issued land before its shared memory goes away
-    for (int i = issued - S < 0 ? 0 : issued - S; i < issued; ++i)
-      wait_deadline(&full[i % S], (i / S) & 1, deadline + TC_TIMEOUT_NS);
+    for (int i = issued - TC_STAGES < 0 ? 0 : issued - TC_STAGES; i < issued; ++i)
+      wait_deadline(&full[i % TC_STAGES], (i / TC_STAGES) & 1, deadline + TC_TIMEOUT_NS);
   }
   tc_fence_before();
   __syncthreads();
@@ -394,9 +394,7 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
-int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g0, int m_tiles, cudaStream_t s) {
-  TcGemm g = g0;
-  g.stages = tc_stages(g.a_pieces + g.b_pieces);
+int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g, int m_tiles, cudaStream_t s) {
   const size_t smem = tc_smem_bytes(g.a_pieces + g.b_pieces);
   cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((g.n_tiles + g.tiles_per_cta - 1) / g.tiles_per_cta, m_tiles, g.P);
