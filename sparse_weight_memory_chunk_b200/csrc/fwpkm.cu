@@ -575,19 +575,14 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
         } else {
           run(st, KK_CART, sS, [&] { return launch_cartesian(d, wb, t0, len, nullptr, nullptr, sS); });
         }
-        // the gather needs the slots and weights only; the write also needs the pair sort
-        cudaStreamWaitEvent(sV, mark(sS), 0);
-        {
-          const void* vc = offs(v, (long long)t0 * d.dv, es);
-          const void* vn = (t0 + len < T) ? offs(v, (long long)(t0 + len) * d.dv, es) : nullptr;
-          run(st, KK_GATHER, sV, [&] {
-            return launch_gather(d, wk, V, vc, g + t0, T, t0, len, o + (long long)t0 * d.dv, true, vn, sV);
-          });
-        }
         run(st, KK_SORT, sS, [&] { return launch_sort_pairs(d, wb, t0, len, !la || (t0 + len < T), sS); });
         sel_done[c] = mark(sS);
+        // the values chain starts a chunk only once its whole selection (slots, weights and
+        // the pair sort) is done: starting the gather right after the slots were chosen
+        // made it overlap the scoring and key-step GEMMs, which slowed them (1.82 against
+        // 1.62 ms per step)
         cudaStreamWaitEvent(sV, sel_done[c], 0);
-        run(st, KK_WRITE, sV, [&] { return launch_write(d, wk, V, t0, sV); });
+        value_chunk(c);
         val_done[c] = mark(sV);
       }
     }

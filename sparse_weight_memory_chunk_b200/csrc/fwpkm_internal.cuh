@@ -70,6 +70,7 @@ enum : int { TC_EPI_DIST = 0, TC_EPI_KEYSTEP = 1, TC_EPI_PROJ = 2 };
 // and B tiles at (x = b_x0 + 64 kb, y = 128 nt, z = p + pb * b_zpiece).
 struct TcGemm {
   int P, k_blocks, n_tiles, tiles_per_cta;
+  int stages;  // pipeline stages (set by launch_tc_gemm)
   int a_pieces, b_pieces;
   int a_div, a_xoff, a_y0, a_zpiece, b_zpiece, b_x0;
   int m_valid, n_valid;

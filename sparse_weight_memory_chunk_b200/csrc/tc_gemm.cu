@@ -35,15 +35,24 @@ using namespace sm100;
 
 constexpr int TC_BM = 128, TC_BN = 128, TC_BK = 64;
 constexpr int TC_TILE_BYTES = TC_BM * TC_BK * 2;  // 16 KiB, also the B tile (TC_BN == TC_BM)
-// two stages (<= 128 KiB of tiles) leave room on the SM for the CTAs of the other chains
-constexpr int TC_STAGES = 2;
+// Pipeline depth: as many stages (<= TC_MAX_STAGES) as fit in ~200 KiB of tiles and are
+// useful (a CTA's k-blocks); the CTA already holds most of the SM's registers, so the
+// shared memory it takes keeps no other kernel out.
+constexpr int TC_MAX_STAGES = 4;
 constexpr int TC_EPI_WARPS = 16;
 constexpr int TC_THREADS = (2 + TC_EPI_WARPS) * 32;
 constexpr uint32_t TC_TMEM_COLS = 256;
 constexpr uint64_t TC_TIMEOUT_NS = 200ull * 1000 * 1000;
 
-size_t tc_smem_bytes(int npieces) {
-  return 1024 + (size_t)TC_STAGES * npieces * TC_TILE_BYTES + 256;
+int tc_stages(int npieces, int kblocks_per_cta) {
+  int st = (200 * 1024) / (npieces * TC_TILE_BYTES);
+  if (st > TC_MAX_STAGES) st = TC_MAX_STAGES;
+  if (st > kblocks_per_cta) st = kblocks_per_cta;
+  return st < 1 ? 1 : st;
+}
+
+size_t tc_smem_bytes(int npieces, int stages) {
+  return 1024 + (size_t)stages * npieces * TC_TILE_BYTES + 256;
 }
 
 __device__ __forceinline__ bool wait_deadline(uint64_t* bar, uint32_t parity, uint64_t deadline) {
@@ -65,9 +74,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int npc = g.a_pieces + g.b_pieces;
   uint8_t* tiles = smem;
-  uint64_t* full = (uint64_t*)(tiles + (size_t)TC_STAGES * npc * TC_TILE_BYTES);
-  uint64_t* empty = full + TC_STAGES;
-  uint64_t* accf = empty + TC_STAGES;
+  const int S = g.stages;
+  uint64_t* full = (uint64_t*)(tiles + (size_t)S * npc * TC_TILE_BYTES);
+  uint64_t* empty = full + TC_MAX_STAGES;
+  uint64_t* accf = empty + TC_MAX_STAGES;
   uint64_t* acce = accf + 2;
   uint64_t* drain = acce + 2;
   uint64_t* normbar = drain + 1;
@@ -81,7 +91,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int ntiles = min(g.n_tiles, nt0 + g.tiles_per_cta) - nt0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < TC_STAGES; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -117,9 +127,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int nt = nt0 + j;
       bool ok = true;
       for (int kb = 0; kb < g.k_blocks; ++kb) {
-        const int s = issued % TC_STAGES;
-        const uint32_t ph = (issued / TC_STAGES) & 1;
-        if (issued >= TC_STAGES && !mbar_wait(&empty[s], ph ^ 1, abort_flag, deadline)) {
+        const int s = issued % S;
+        const uint32_t ph = (issued / S) & 1;
+        if (issued >= S && !mbar_wait(&empty[s], ph ^ 1, abort_flag, deadline)) {
           ok = false;
           break;
         }
@@ -147,8 +157,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t dt = tmem + (uint32_t)(b * TC_BN);
       bool ok = true;
       for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
-        const int s = it % TC_STAGES;
-        const uint32_t ph = (it / TC_STAGES) & 1;
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1;
         if (!mbar_wait(&full[s], ph, abort_flag, deadline)) {
           ok = false;
           break;
@@ -346,8 +356,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   __syncwarp();
   if (warp == 0 && lane == 0 && *abort_flag) {
     // let the copies this CTA issued land before its shared memory goes away
-    for (int i = issued - TC_STAGES < 0 ? 0 : issued - TC_STAGES; i < issued; ++i)
-      wait_deadline(&full[i % TC_STAGES], (i / TC_STAGES) & 1, deadline + TC_TIMEOUT_NS);
+    for (int i = issued - S < 0 ? 0 : issued - S; i < issued; ++i)
+      wait_deadline(&full[i % S], (i / S) & 1, deadline + TC_TIMEOUT_NS);
   }
   tc_fence_before();
   __syncthreads();
@@ -394,8 +404,11 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
-int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g, int m_tiles, cudaStream_t s) {
-  const size_t smem = tc_smem_bytes(g.a_pieces + g.b_pieces);
+int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g0, int m_tiles, cudaStream_t s) {
+  TcGemm g = g0;
+  const int npc = g.a_pieces + g.b_pieces;
+  g.stages = tc_stages(npc, g.k_blocks * g.tiles_per_cta);
+  const size_t smem = tc_smem_bytes(npc, g.stages);
   cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((g.n_tiles + g.tiles_per_cta - 1) / g.tiles_per_cta, m_tiles, g.P);
   launch_k(tc_gemm_kernel, grid, TC_THREADS, smem, s, A, B, g);

@@ -151,31 +151,37 @@ tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
   const int n = dm.n;
   const float* D = w.Dfull + (size_t)p * w.drows * n;
   const float* lp = w.lp + (size_t)p * n;
-  for (int tl = warp; tl < WB_T; tl += TP_THREADS / 32) {
-    const int t = t0 + tl;
-    float L = 0.f, iz = 0.f;
-    if (t < len) {
-      const float* Dr = D + (size_t)t * n;
-      float s = 0.f;
-      for (int a0 = 0; a0 < n; a0 += 32 * 16) {
-        float dd[16], ll[16];
+  // two tokens per warp, their row loads and the shared log-marginal loads in flight together
+  static_assert(WB_T == 2 * (TP_THREADS / 32), "two tokens per warp");
+  {
+    const int ta = t0 + 2 * warp, tb = ta + 1;
+    const bool va = ta < len, vb = tb < len;
+    const float* Da = D + (size_t)(va ? ta : 0) * n;
+    const float* Db = D + (size_t)(vb ? tb : 0) * n;
+    float sa = 0.f, sb = 0.f;
+    for (int a0 = 0; a0 < n; a0 += 32 * 16) {
+      float da[16], db[16], ll[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int a = a0 + lane + 32 * u;
-          dd[u] = a < n ? Dr[a] : 0.f;
-          ll[u] = a < n ? lp[a] : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) s += __fdividef(ll[u], dm.eps_idw + dd[u]);
+      for (int u = 0; u < 16; ++u) {
+        const int a = a0 + lane + 32 * u;
+        ll[u] = a < n ? lp[a] : 0.f;
+        da[u] = (va && a < n) ? Da[a] : 0.f;
+        db[u] = (vb && a < n) ? Db[a] : 0.f;
       }
-      s = warp_sum(s);
-      const float z = w.Z[(size_t)p * dm.C + t];
-      L = s / z;
-      iz = 1.f / z;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        sa += __fdividef(ll[u], dm.eps_idw + da[u]);
+        sb += __fdividef(ll[u], dm.eps_idw + db[u]);
+      }
     }
+    sa = warp_sum(sa);
+    sb = warp_sum(sb);
     if (lane == 0) {
-      s_L[tl] = L;
-      s_invz[tl] = iz;
+      const float za = va ? w.Z[(size_t)p * dm.C + ta] : 1.f, zb = vb ? w.Z[(size_t)p * dm.C + tb] : 1.f;
+      s_L[2 * warp] = va ? sa / za : 0.f;
+      s_invz[2 * warp] = va ? 1.f / za : 0.f;
+      s_L[2 * warp + 1] = vb ? sb / zb : 0.f;
+      s_invz[2 * warp + 1] = vb ? 1.f / zb : 0.f;
     }
   }
   __syncthreads();
