@@ -198,6 +198,30 @@ def algorithmic_bytes(w, idx, T):
     return b_vk, gather_per_token, U_total
 
 
+# --------------------------------------------------------------------------- ranks
+def rank_workload(w, rank):
+    """Each rank runs its own independent memories: rank r draws its sequences with seed
+    offset 1000 r (rank 0 is the workload itself)."""
+    from dataclasses import replace
+    return replace(w, seed=w.seed + 1000 * rank) if rank else w
+
+
+def max_over_ranks(x, world, device):
+    """The largest of the ranks' values (the job's time is its slowest rank's)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step, world, ms_step):
+    """Whole-job units per second: every rank processes units_per_rank_step per step."""
+    return units_per_rank_step * world / (ms_step / 1000.0)
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -215,8 +239,7 @@ def run_ours(args, w, rank, world, local_rank):
     peak_src = "measured" if peaks else "fallback"
 
     # inputs (per-rank independent sequences: seed offset by rank)
-    from dataclasses import replace
-    wr = replace(w, seed=w.seed + 1000 * rank) if rank else w
+    wr = rank_workload(w, rank)
     q, v, g = gen_qvg(wr)
     K1, K2 = gen_keys(wr)
     needles = gen_needles(wr, q, v) if w.name == "needle" else None
@@ -305,13 +328,9 @@ def run_ours(args, w, rank, world, local_rank):
     dom_ms, dom_n = st.kernel_time()
     st.profile_kernel(0)
     st.sync()
-    ms_step = ms_total / args.steps
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = max_over_ranks(ms_total / args.steps, world, dev)
     tokens_per_step = w.B * w.T * args.n_iter
-    value = tokens_per_step * world / (ms_step / 1000.0)
+    value = job_throughput(tokens_per_step, world, ms_step)
 
     # algorithmic traffic of the step (measured unique rows) and roofline
     idx = torch.empty(w.M, w.T, w.k, dtype=torch.int32, device=dev)
@@ -406,13 +425,9 @@ def run_ours(args, w, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1) / args.steps
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
         bi = sum(x.numel() * x.element_size() for x in host_in)
-        line["e2e"] = {"value": tokens_per_step * world / (ems / 1000.0), "unit": "tokens/s",
+        line["e2e"] = {"value": job_throughput(tokens_per_step, world, ems), "unit": "tokens/s",
                        "h2d_bytes_per_step": bi, "d2h_bytes_per_step": host_out.numel() * host_out.element_size(),
                        "ms_per_step": ems}
 
