@@ -35,10 +35,9 @@ using namespace sm100;
 
 constexpr int TC_BM = 128, TC_BN = 128, TC_BK = 64;
 constexpr int TC_TILE_BYTES = TC_BM * TC_BK * 2;  // 16 KiB, also the B tile (TC_BN == TC_BM)
-// Pipeline depth: as many stages (<= TC_MAX_STAGES) as fit in ~200 KiB of tiles and are
-// useful (a CTA's k-blocks); the CTA already holds most of the SM's registers, so the
-// shared memory it takes keeps no other kernel out.
-constexpr int TC_MAX_STAGES = 4;
+// Pipeline depth: two stages (up to four were measured slower: the larger shared-memory
+// carve-out leaves the epilogue's loads and stores less L1).
+constexpr int TC_MAX_STAGES = 2;
 constexpr int TC_EPI_WARPS = 16;
 constexpr int TC_THREADS = (2 + TC_EPI_WARPS) * 32;
 constexpr uint32_t TC_TMEM_COLS = 256;
