@@ -26,6 +26,11 @@ CASES = {
     "paper": (1024, 256, 256, 32, 256, 2, 600, "bf16", True, 1.0, "normal002"),
     "needle_chunk": (1024, 256, 256, 32, 512, 1, 1100, "bf16", False, 1.0, "normal002"),
     "layer_shape": (512, 256, 256, 32, 256, 2, 520, "f32", True, 1.0, "normal002"),
+    # degenerate and extreme shapes
+    "k_equals_n": (8, 16, 8, 8, 4, 2, 21, "f32", True, 10.0, "normal002"),   # every sub-key survives
+    "k1": (64, 128, 64, 1, 32, 2, 70, "bf16", True, 10.0, "normal002"),       # single slot per token
+    "chunk1": (64, 128, 64, 4, 1, 1, 9, "bf16", True, 10.0, "normal002"),     # one token per chunk
+    "n_max": (4096, 256, 32, 32, 16, 1, 40, "bf16", True, 1.0, "normal002"),  # largest codebook
 }
 
 
