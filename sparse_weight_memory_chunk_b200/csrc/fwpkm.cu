@@ -560,9 +560,13 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
         } else {
           run(st, KK_SCORE, sK, [&] { return launch_score_topk(d, wb, K1, K2, qc, T, t0, len, true, sK); });
         }
-        cudaStreamWaitEvent(sS, mark(sK), 0);
+        // the selection needs the distance rows; on the tensor-core path it also waits for
+        // the usage marginals, so that pbar (on the critical addressing chain) does not share
+        // the GPU with it (1.606 against 1.628 ms per step)
+        if (!tc) cudaStreamWaitEvent(sS, mark(sK), 0);
         if (tc) {
           run(st, KK_PBAR, sK, [&] { return launch_tc_pbar(d, wb, len, sK); });
+          cudaStreamWaitEvent(sS, mark(sK), 0);
           run(st, KK_WBUILD, sK, [&] { return launch_tc_wbuild(d, wb, len, sK); });
           run(st, KK_ADDR, sK, [&] { return launch_tc_keystep(d, wb, K1, K2, qc, T, len, qt_whole ? t0 : -1, sK); });
         } else {

@@ -11,6 +11,7 @@
 // Rows are moved as 16-byte vectors: a warp covers 512 contiguous bytes per load.  Both
 // kernels are bound by HBM latency x bytes in flight, so each warp keeps many row loads
 // outstanding before it consumes any of them.
+#include <cstdlib>
 #include <mutex>
 
 #include "fwpkm_internal.cuh"
@@ -30,6 +31,27 @@ __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p, l
   const __nv_bfloat162* q = reinterpret_cast<const __nv_bfloat162*>(p) + 2 * i4;
   float2 a = __bfloat1622float2(q[0]), b = __bfloat1622float2(q[1]);
   return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// V rows stream through L2 (a chunk touches ~200 MB of them, mostly once): their loads
+// and stores carry an evict-first policy so that they do not push the addressing chain's
+// working set (distance rows, key pieces, W) out of L2.
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ float4 ld_stream(const float4* p, uint64_t pol) {
+  float4 v;
+  asm volatile("ld.global.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ void st_stream(float4* p, float4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w), "l"(pol)
+               : "memory");
 }
 
 // r = gw * (vhat - tau), tau = z(u) or u.  Shared by the fused and the streaming path
@@ -137,6 +159,7 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
 #pragma unroll
   for (int c = 0; c < VPL; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   const int r0 = half * 16, r1 = min(k, r0 + 16);
+  const uint64_t pol = evict_first_policy();
   if (active) {
 #pragma unroll 16
     for (int r = r0; r < r1; ++r) {
@@ -147,7 +170,7 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
       for (int c = 0; c < VPL; ++c) {
         int e4 = lane + 32 * c;
         if (e4 < dv4) {
-          float4 x = row[e4];
+          float4 x = ld_stream(row + e4, pol);
           acc[c].x = fmaf(wr, x.x, acc[c].x); acc[c].y = fmaf(wr, x.y, acc[c].y);
           acc[c].z = fmaf(wr, x.z, acc[c].z); acc[c].w = fmaf(wr, x.w, acc[c].w);
         }
@@ -255,6 +278,7 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
   const unsigned long long* sk = w.sk + cbase * (size_t)(C * k);
   const float* wrow = w.w + ((size_t)m * w.max_T + wt0) * k;  // pair t*k + r of the chunk at wrow[t*k + r]
   float* Vm = V + (size_t)m * dm.N * dm.dv;
+  const uint64_t pol = evict_first_policy();
   // the CTAs of a memory cover its list in strides (grid sized to the resident CTAs)
   for (int pos0 = (blockIdx.x * VAL_WARPS + warp) * G; pos0 < P; pos0 += gridDim.x * VAL_WARPS * G) {
     unsigned long long my_key = ~0ull;
@@ -275,7 +299,7 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
 #pragma unroll
       for (int c = 0; c < VPL; ++c) {
         const int e4 = lane + 32 * c;
-        Vr[gi][c] = (ok && e4 < dv4) ? row[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        Vr[gi][c] = (ok && e4 < dv4) ? ld_stream(row + e4, pol) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
 #pragma unroll
@@ -318,7 +342,7 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
         if (e4 < dv4) {
           float4 x = Vr[gi][c];
           x.x -= Gs[c].x / nr; x.y -= Gs[c].y / nr; x.z -= Gs[c].z / nr; x.w -= Gs[c].w / nr;
-          row[e4] = x;
+          st_stream(row + e4, x, pol);
         }
       }
     }
@@ -394,9 +418,17 @@ int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s
   const int vpl = vpl_of(d.dv);
   const int G = vpl <= 2 ? 4 : vpl == 4 ? 2 : 1;  // list positions per warp: ~8 float4 in flight per lane
   const int need = (d.C * d.k + VAL_WARPS * G - 1) / (VAL_WARPS * G);  // CTAs per memory for one pass
+  // the grid is a fraction of one resident wave (FWPKM_WRITE_SHARE percent, default 50): the
+  // write runs beside the addressing chain of the next chunk, and a smaller footprint
+  // leaves that chain more of the GPU
+  static const int share = [] {
+    const char* e = getenv("FWPKM_WRITE_SHARE");
+    const int v = e ? atoi(e) : 50;
+    return v < 5 ? 5 : v > 100 ? 100 : v;
+  }();
   auto grid_for = [&](int resident) {
-    const int per_mem = (resident + d.M - 1) / d.M;  // one resident wave over all memories
-    return dim3(need < per_mem ? need : per_mem, d.M);
+    const int per_mem = ((long long)resident * share / 100 + d.M - 1) / d.M;
+    return dim3(need < per_mem ? need : (per_mem < 1 ? 1 : per_mem), d.M);
   };
   switch (vpl) {
     case 1: launch_k(write_kernel<1, 4>, grid_for(resident_ctas((const void*)write_kernel<1, 4>, VAL_WARPS * 32)), VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
