@@ -515,9 +515,15 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
   };
 
   if (tc) {
-    run(st, KK_PREP, sK, [&] { return launch_qnorm(d, wk, q, T, 0, T, sK); });
-    if (qt_whole) run(st, KK_PREP, sK, [&] { return launch_qtrans(d, wk, q, T, 0, T, sK); });
+    // the three per-call preparations are independent: query norms (selection stream),
+    // query transpose (values stream) and key pieces (addressing stream) run side by side
+    run(st, KK_PREP, sS, [&] { return launch_qnorm(d, wk, q, T, 0, T, sS); });
+    const cudaEvent_t qn_done = mark(sS);
+    if (qt_whole) run(st, KK_PREP, sV, [&] { return launch_qtrans(d, wk, q, T, 0, T, sV); });
+    const cudaEvent_t qt_done = mark(sV);
     run(st, KK_PREP, sK, [&] { return launch_keyprep(d, wk, K1, K2, sK); });
+    cudaStreamWaitEvent(sK, qn_done, 0);
+    cudaStreamWaitEvent(sK, qt_done, 0);
   }
   if (!ku) {
     // frozen keys: address window by window on sK; the value loop of a window starts as

@@ -33,9 +33,10 @@ __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p, l
   return make_float4(a.x, a.y, b.x, b.y);
 }
 
-// V rows stream through L2 (a chunk touches ~200 MB of them, mostly once): their loads
-// and stores carry an evict-first policy so that they do not push the addressing chain's
-// working set (distance rows, key pieces, W) out of L2.
+// The gather streams V rows through L2 (64 MB per chunk, mostly read once): its loads
+// carry an evict-first policy so that they do not push the addressing chain's working set
+// (distance rows, key pieces, W) out of L2.  (The write's rows are left at the default:
+// with the policy on its loads and stores the step was slower.)
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -48,12 +49,6 @@ __device__ __forceinline__ float4 ld_stream(const float4* p, uint64_t pol) {
                : "l"(p), "l"(pol));
   return v;
 }
-__device__ __forceinline__ void st_stream(float4* p, float4 v, uint64_t pol) {
-  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y),
-               "f"(v.z), "f"(v.w), "l"(pol)
-               : "memory");
-}
-
 // r = gw * (vhat - tau), tau = z(u) or u.  Shared by the fused and the streaming path
 // so both give the same bits.
 template <typename VT, int VPL>
@@ -278,7 +273,6 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
   const unsigned long long* sk = w.sk + cbase * (size_t)(C * k);
   const float* wrow = w.w + ((size_t)m * w.max_T + wt0) * k;  // pair t*k + r of the chunk at wrow[t*k + r]
   float* Vm = V + (size_t)m * dm.N * dm.dv;
-  const uint64_t pol = evict_first_policy();
   // the CTAs of a memory cover its list in strides (grid sized to the resident CTAs)
   for (int pos0 = (blockIdx.x * VAL_WARPS + warp) * G; pos0 < P; pos0 += gridDim.x * VAL_WARPS * G) {
     unsigned long long my_key = ~0ull;
@@ -299,7 +293,7 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
 #pragma unroll
       for (int c = 0; c < VPL; ++c) {
         const int e4 = lane + 32 * c;
-        Vr[gi][c] = (ok && e4 < dv4) ? ld_stream(row + e4, pol) : make_float4(0.f, 0.f, 0.f, 0.f);
+        Vr[gi][c] = (ok && e4 < dv4) ? row[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
 #pragma unroll
@@ -342,7 +336,7 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
         if (e4 < dv4) {
           float4 x = Vr[gi][c];
           x.x -= Gs[c].x / nr; x.y -= Gs[c].y / nr; x.z -= Gs[c].z / nr; x.w -= Gs[c].w / nr;
-          st_stream(row + e4, x, pol);
+          row[e4] = x;
         }
       }
     }
