@@ -177,6 +177,23 @@ void set_carveout(const void* kern) {
   done.push_back(kern);
 }
 
+bool raise_smem_limit(const void* kern, size_t bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, size_t>> lim;
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto& e : lim)
+    if (e.first == kern) {
+      if (bytes <= e.second) return true;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return false;
+      e.second = bytes;
+      return true;
+    }
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) return false;
+  lim.emplace_back(kern, bytes);
+  return true;
+}
+
 thread_local int launch_priority = 0;
 thread_local bool launch_priority_set = false;
 
@@ -250,7 +267,7 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
     x.qn = (float*)take(4 * P * T);
     if (ku) {
       x.zpart = (float*)take(4 * P * C * nt * 4);
-      x.ppart = (float*)take(4 * P * 8 * n);
+      x.ppart = (float*)take(4 * P * PBAR_SLICES * n);
       x.Wt = (__nv_bfloat16*)take(2 * 2 * P * n * cpad);
       x.qt_T = (int)((T > C ? T : C) + 63) / 64 * 64;
       x.Qt = (__nv_bfloat16*)take(2 * P * h * (size_t)x.qt_T);
@@ -283,7 +300,7 @@ Work group_work(const Dims& d, const Work& w, int m0) {
   if (x.kn) x.kn += M0 * 2 * n;
   if (x.qn) x.qn += M0 * 2 * T;
   if (x.zpart) x.zpart += M0 * 2 * C * nt * 4;
-  if (x.ppart) x.ppart += M0 * 2 * 8 * n;
+  if (x.ppart) x.ppart += M0 * 2 * PBAR_SLICES * n;
   if (x.Wt) x.Wt += M0 * 2 * n * cpad;
   if (x.Qt) x.Qt += M0 * 2 * h * (size_t)w.qt_T;
   if (x.wsum_part) x.wsum_part += M0 * 2 * (cpad / 16) * n;

@@ -50,7 +50,7 @@ struct Work {
   float* kn;         // [M*2][n]           squared key norms
   float* qn;         // [M*2][max_T]       squared half-query norms
   float* zpart;      // [M*2][C][n/128][4] per-32-column partial sums of 1/(eps + D)
-  float* ppart;      // [M*2][8][n]        partial column sums for pbar
+  float* ppart;      // [M*2][PBAR_SLICES][n] partial column sums for pbar
   __nv_bfloat16* Wt; // [2][M*2][n][Cpad]  key-step weights, sub-key major, bf16 pieces hi, lo
   __nv_bfloat16* Qt; // [M*2][h][qt_T]     half-queries, feature major (operand B of the key step)
   int qt_T;          // token columns of Qt (a multiple of 64)
@@ -64,6 +64,10 @@ struct Work {
 };
 
 enum : int { TC_EPI_DIST = 0, TC_EPI_KEYSTEP = 1, TC_EPI_PROJ = 2 };
+
+// Token slices of the usage-marginal pass (pbar): each column's sum is formed in this many
+// partial sums, one per CTA slice.
+constexpr int PBAR_SLICES = 16;
 
 // One batched tensor-core contraction (see tc_gemm.cu).  Problem p (blockIdx.z) owns
 // A tiles at (x = (p % a_div) * a_xoff + 64 kb, y = a_y0 + 128 mt, z = p / a_div + pa * a_zpiece)
@@ -167,6 +171,10 @@ bool pdl_enabled();
 // kernel can start beside the running ones.  Off by default: the smaller L1 it leaves
 // cost more than the switches (2.02 ms per paper-scale step against 1.73 ms without).
 void set_carveout(const void* kern);
+// Raise `kern`'s dynamic shared-memory limit to at least `bytes` (never lowered, so that a
+// launch captured earlier with more never finds the function's limit below its own need).
+// Returns false if the attribute cannot be set.
+bool raise_smem_limit(const void* kern, size_t bytes);
 
 // Launch `kern` on `s`, allowing it to start while the previous kernel of the same stream
 // finishes (programmatic stream serialization).  Every kernel launched this way calls

@@ -88,13 +88,14 @@ extern "C" fwpkm_status fwpkm_chunk_step_noalloc(const fwpkm_config* cfg, float*
   }
   const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
   const bool last_has_target = (v_next != nullptr) || !(d.flags & FWPKM_LOOKAHEAD);
-  launch_score_topk(d, w, K1, K2, q, seq_stride, 0, c_len, ku, st);
-  launch_cartesian(d, w, 0, c_len, nullptr, nullptr, st);
-  launch_gather(d, w, V, v, g, seq_stride, 0, c_len, o, true, v_next, st);
-  launch_sort_pairs(d, w, 0, c_len, last_has_target, st);
-  launch_write(d, w, V, 0, st);
-  if (ku) launch_address(d, w, K1, K2, q, seq_stride, c_len, st);
+  bool ok = launch_score_topk(d, w, K1, K2, q, seq_stride, 0, c_len, ku, st) >= 0;
+  ok = ok && launch_cartesian(d, w, 0, c_len, nullptr, nullptr, st) >= 0;
+  ok = ok && launch_gather(d, w, V, v, g, seq_stride, 0, c_len, o, true, v_next, st) >= 0;
+  ok = ok && launch_sort_pairs(d, w, 0, c_len, last_has_target, st) >= 0;
+  ok = ok && launch_write(d, w, V, 0, st) >= 0;
+  if (ok && ku) ok = launch_address(d, w, K1, K2, q, seq_stride, c_len, st) >= 0;
   cudaError_t e = cudaGetLastError();
+  if (!ok && e == cudaSuccess) return FWPKM_ERR_CUDA;
   if (e != cudaSuccess) {
     fprintf(stderr, "fwpkm_chunk_step_noalloc: %s\n", cudaGetErrorString(e));
     return FWPKM_ERR_CUDA;

@@ -109,14 +109,15 @@ score_topk_simt(Dims dm, Work w, const float* __restrict__ K1, const float* __re
 }
 
 template <typename QT, int TQ>
-static void launch_tq(const Dims& d, const Work& w, const float* K1, const float* K2, const void* q,
-                      long long q_stride, int wt0, int len, bool key_update, cudaStream_t s) {
+static int launch_tq(const Dims& d, const Work& w, const float* K1, const float* K2, const void* q,
+                     long long q_stride, int wt0, int len, bool key_update, cudaStream_t s) {
   size_t smem = sizeof(float) * ((size_t)TQ * d.h + (size_t)SCORE_KT * (d.h + 1) + (size_t)TQ * d.n);
   auto kern = score_topk_simt<QT, TQ>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (!raise_smem_limit((const void*)kern, smem)) return -1;
   dim3 grid((len + TQ - 1) / TQ, d.M * 2);
   kern<<<grid, SCORE_THREADS, smem, s>>>(d, w, K1, K2, (const QT*)q, q_stride, wt0, len,
                                         key_update ? 1 : 0);
+  return 1;
 }
 
 int launch_score_topk(const Dims& d, const Work& w, const float* K1, const float* K2, const void* q,
@@ -127,17 +128,15 @@ int launch_score_topk(const Dims& d, const Work& w, const float* K1, const float
   while (tq > 4 && (size_t)tq * d.n * 4 + (size_t)tq * d.h * 4 + (size_t)SCORE_KT * (d.h + 1) * 4 > 200 * 1024)
     tq >>= 1;
   if (d.qv_bf16) {
-    if (tq == 32) launch_tq<__nv_bfloat16, 32>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
-    else if (tq == 16) launch_tq<__nv_bfloat16, 16>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
-    else if (tq == 8) launch_tq<__nv_bfloat16, 8>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
-    else launch_tq<__nv_bfloat16, 4>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
-  } else {
-    if (tq == 32) launch_tq<float, 32>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
-    else if (tq == 16) launch_tq<float, 16>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
-    else if (tq == 8) launch_tq<float, 8>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
-    else launch_tq<float, 4>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
+    if (tq == 32) return launch_tq<__nv_bfloat16, 32>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
+    if (tq == 16) return launch_tq<__nv_bfloat16, 16>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
+    if (tq == 8) return launch_tq<__nv_bfloat16, 8>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
+    return launch_tq<__nv_bfloat16, 4>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
   }
-  return 1;
+  if (tq == 32) return launch_tq<float, 32>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
+  if (tq == 16) return launch_tq<float, 16>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
+  if (tq == 8) return launch_tq<float, 8>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
+  return launch_tq<float, 4>(d, w, K1, K2, q, q_stride, wt0, len, key_update, s);
 }
 
 }  // namespace fwpkm

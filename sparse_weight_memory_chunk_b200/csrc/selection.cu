@@ -358,13 +358,13 @@ int launch_sort_pairs(const Dims& d, const Work& w, int wt0, int total_len, bool
     int Ppad = 256;
     while (Ppad < P) Ppad <<= 1;
     const size_t smem = sizeof(u64) * (size_t)Ppad;
-    cudaFuncSetAttribute(sort_pairs_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (!raise_smem_limit((const void*)sort_pairs_kernel<8>, smem)) return -1;
     launch_k(sort_pairs_kernel<8>, grid, SORT_THREADS, smem, s, d, w, wt0, total_len, last_has_target ? 1 : 0);
   } else {
     int Ppad = 512;
     while (Ppad < P) Ppad <<= 1;
     const size_t smem = sizeof(u64) * (size_t)Ppad;
-    cudaFuncSetAttribute(sort_pairs_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (!raise_smem_limit((const void*)sort_pairs_kernel<16>, smem)) return -1;
     launch_k(sort_pairs_kernel<16>, grid, SORT_THREADS, smem, s, d, w, wt0, total_len, last_has_target ? 1 : 0);
   }
   return 1;

@@ -408,7 +408,11 @@ int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g0,
   const int npc = g.a_pieces + g.b_pieces;
   g.stages = tc_stages(npc, g.k_blocks * g.tiles_per_cta);
   const size_t smem = tc_smem_bytes(npc, g.stages);
-  cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // The kernel's dynamic shared-memory limit is one attribute of the function, while its
+  // launches need different amounts (scoring 129 KiB, key step 97 KiB, ...): it is only
+  // ever raised, so that no captured launch is above it (a replay that launches graph
+  // nodes one by one checks each node against the function's current limit).
+  if (!raise_smem_limit((const void*)tc_gemm_kernel, smem)) return -1;
   dim3 grid((g.n_tiles + g.tiles_per_cta - 1) / g.tiles_per_cta, m_tiles, g.P);
   launch_k(tc_gemm_kernel, grid, TC_THREADS, smem, s, A, B, g);
   return 1;

@@ -14,7 +14,6 @@
 namespace fwpkm {
 
 constexpr int TP_THREADS = 256;
-constexpr int PBAR_SLICES = 8;
 
 __device__ __forceinline__ void split3_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& mid, __nv_bfloat16& lo) {
   hi = __float2bfloat16_rn(x);
