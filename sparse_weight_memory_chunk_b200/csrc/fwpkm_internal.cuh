@@ -147,8 +147,6 @@ int launch_tc_score(const Dims& d, const Work& w, const void* q_base, long long 
 // Fused per-half top-k + Cartesian search + softmax from Dfull rows 0..len-1 (workspace
 // tokens wt0..): writes idx, w and the optional user copies; A/Dsv are not written.
 int launch_select(const Dims& d, const Work& w, int wt0, int len, int32_t* idx_out, float* w_out, cudaStream_t s);
-// Per-half top-k from Dfull rows 0..len-1 into A/Dsv at workspace tokens wt0..
-int launch_topk_rows(const Dims& d, const Work& w, int wt0, int len, cudaStream_t s);
 // Feature-major copy of both half-queries of `len` tokens into Qt columns qt0.. (the key
 // step's B operand).
 int launch_qtrans(const Dims& d, const Work& w, const void* q, long long q_stride, int qt0, int len, cudaStream_t s);

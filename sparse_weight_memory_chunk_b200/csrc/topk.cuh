@@ -1,5 +1,5 @@
-// topk.cuh -- per-half top-k of one distance row by one warp (used by the top-k kernel and
-// by the fused selection kernel).
+// topk.cuh -- per-half top-k of one distance row by one warp (used by the fused selection
+// kernel).
 //
 // Fast-weight Product Key Memory (paperlayer summary) §2.2: each half keeps the k
 // sub-keys nearest to its half-query; (rainbus summary) PKM prerequisite.  Order: distance
