@@ -85,7 +85,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   __shared__ float s_norm[4][TC_BM];
   __shared__ float s_wsum[4][TC_BM];  // a_build: per-row partial sums of W by token quarter
-  __shared__ float s_tok[2][1024];     // a_build: 1/Z_t and L_t of the chunk's tokens
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = blockIdx.z, mt = blockIdx.y;
@@ -205,13 +204,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const float* D = g.bD + (size_t)p * g.bD_pstride;
       const float lpb = bvalid ? g.blp[(size_t)p * n + bsub] : 0.f;
       const float inv_len = 1.f / (float)g.blen;
-      // per-token 1/Z_t and L_t, once per CTA (the epilogue warps' own named barrier: the
-      // producer and MMA warps do not take part)
-      for (int t = et; t < g.blen; t += TC_EPI_WARPS * 32) {
-        s_tok[0][t] = 1.f / g.bZ[(size_t)p * g.bC + t];
-        s_tok[1][t] = g.bL[(size_t)p * g.bC + t];
-      }
-      asm volatile("bar.sync 1, %0;" ::"r"(TC_EPI_WARPS * 32) : "memory");
       float wacc = 0.f;
       for (int kb = 0; kb < g.k_blocks && built; ++kb) {
         const int s = kb % S;
@@ -239,8 +231,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           float W = 0.f;
           if (bvalid && t < g.blen) {
             const float wv = __fdividef(1.f, g.beps + dd[u]);
-            const float P_ = wv * s_tok[0][t];
-            W = inv_len * P_ * (lpb - s_tok[1][t]) * wv;
+            const float P_ = wv * (1.f / g.bZ[(size_t)p * g.bC + t]);
+            W = inv_len * P_ * (lpb - g.bL[(size_t)p * g.bC + t]) * wv;
           }
           wacc += W;
           hi[u] = __float2bfloat16_rn(W);
