@@ -261,17 +261,17 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
   x.Kpc = nullptr; x.kn = nullptr; x.qn = nullptr; x.zpart = nullptr; x.ppart = nullptr;
   x.Wt = nullptr; x.Qt = nullptr; x.wsum_part = nullptr; x.pbar_cnt = nullptr; x.qt_T = 0;
   if (x.tc) {
-    const size_t P = 2 * M, h = d.h, nt = (n + 127) / 128;
+    const size_t P = 2 * M, h = d.h, cpad = (C + 63) / 64 * 64, nt = (n + 127) / 128;
     x.Kpc = (__nv_bfloat16*)take(2 * 3 * P * n * h);
     x.kn = (float*)take(4 * P * n);
     x.qn = (float*)take(4 * P * T);
     if (ku) {
       x.zpart = (float*)take(4 * P * C * nt * 4);
       x.ppart = (float*)take(4 * P * PBAR_SLICES * n);
-      x.Wt = nullptr;  // W is built inside the key-step GEMM
+      x.Wt = (__nv_bfloat16*)take(2 * 2 * P * n * cpad);
       x.qt_T = (int)((T > C ? T : C) + 63) / 64 * 64;
       x.Qt = (__nv_bfloat16*)take(2 * P * h * (size_t)x.qt_T);
-      x.wsum_part = nullptr;
+      x.wsum_part = (float*)take(4 * P * (cpad / 16) * n);
       x.pbar_cnt = (int*)take(4 * P * ((n + 255) / 256));
     }
   }

@@ -51,10 +51,10 @@ struct Work {
   float* qn;         // [M*2][max_T]       squared half-query norms
   float* zpart;      // [M*2][C][n/128][4] per-32-column partial sums of 1/(eps + D)
   float* ppart;      // [M*2][PBAR_SLICES][n] partial column sums for pbar
-  __nv_bfloat16* Wt; // unused on the current path (W is built inside the key-step GEMM): null
+  __nv_bfloat16* Wt; // [2][M*2][n][Cpad]  key-step weights, sub-key major, bf16 pieces hi, lo
   __nv_bfloat16* Qt; // [M*2][h][qt_T]     half-queries, feature major (operand B of the key step)
   int qt_T;          // token columns of Qt (a multiple of 64)
-  float* wsum_part;  // unused on the current path (sum_t W is formed with W): null
+  float* wsum_part;  // [M*2][Cpad/16][n]  per-16-token-block sums of W
   int* pbar_cnt;     // [M*2][ceil(n/256)] arrival counters of the pbar column blocks (zero between launches)
   // Every array above is memory-major except the bf16 pieces (Kpc, Wt), whose piece
   // stride is P_all problems; a Work for a group of memories is the same carve with its
@@ -87,14 +87,6 @@ struct TcGemm {
   // TC_EPI_KEYSTEP
   float* K1; float* K2; __nv_bfloat16* Kpc; float* kn; int piece_P;
   const float* wsum_part; int wsum_tiles; float lr;
-  // KEYSTEP with a_build: the epilogue warps build the A operand (W, two bf16 pieces) in
-  // shared memory from the distance rows instead of loading it:
-  // W[t][b] = (1/len) (w / Z_t) (lp[b] - L_t) w with w = 1/(eps + D[t][b]), and sum_t W
-  int a_build;
-  const float* bD; long long bD_pstride;  // distance rows [P][C][n]
-  const float* bZ; const float* bL; int bC; // Z_t, L_t [P][C]
-  const float* blp;                         // log pbar [P][n]
-  int blen; float beps;
   // TC_EPI_PROJ: y[r][c] = acc * rowscale[r] + bias[c] (n_valid and split multiples of 32)
   // into pout0[r][c] (c < split) or pout1[r][c - split], fp32 or (out_bf16) bf16
   const float* rowscale; const float* bias;

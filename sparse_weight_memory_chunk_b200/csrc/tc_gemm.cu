@@ -80,11 +80,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* acce = accf + 2;
   uint64_t* drain = acce + 2;
   uint64_t* normbar = drain + 1;
-  uint64_t* wsbar = normbar + 1;
-  uint32_t* tmem_slot = (uint32_t*)(wsbar + 1);
+  uint32_t* tmem_slot = (uint32_t*)(normbar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   __shared__ float s_norm[4][TC_BM];
-  __shared__ float s_wsum[4][TC_BM];  // a_build: per-row partial sums of W by token quarter
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = blockIdx.z, mt = blockIdx.y;
@@ -93,8 +91,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      // built A operand: the TMA producer's arrival plus one per epilogue warp
-      mbar_init(&full[s], g.a_build ? 1 + TC_EPI_WARPS : 1);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -103,7 +100,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     mbar_init(drain, 1);
     mbar_init(normbar, TC_EPI_WARPS);
-    mbar_init(wsbar, TC_EPI_WARPS);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -123,7 +119,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   if (ntiles > 0 && warp == 0 && lane == 0) {
     // ---------------- TMA producer ----------------
-    if (!g.a_build) tma_prefetch(&tmA);
+    tma_prefetch(&tmA);
     tma_prefetch(&tmB);
     const int a_z = p / g.a_div, a_x0 = (p % g.a_div) * g.a_xoff;
     for (int j = 0; j < ntiles && !*abort_flag; ++j) {
@@ -136,12 +132,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           ok = false;
           break;
         }
-        mbar_expect_tx(&full[s], (uint32_t)((g.a_build ? g.b_pieces : npc) * TC_TILE_BYTES));
+        mbar_expect_tx(&full[s], (uint32_t)(npc * TC_TILE_BYTES));
         uint8_t* st = tiles + (size_t)s * npc * TC_TILE_BYTES;
-        if (!g.a_build)
-          for (int pa = 0; pa < g.a_pieces; ++pa)
-            tma_load_3d(st + pa * TC_TILE_BYTES, &tmA, &full[s], a_x0 + kb * TC_BK, g.a_y0 + mt * TC_BM,
-                        a_z + pa * g.a_zpiece);
+        for (int pa = 0; pa < g.a_pieces; ++pa)
+          tma_load_3d(st + pa * TC_TILE_BYTES, &tmA, &full[s], a_x0 + kb * TC_BK, g.a_y0 + mt * TC_BM,
+                      a_z + pa * g.a_zpiece);
         for (int pb = 0; pb < g.b_pieces; ++pb)
           tma_load_3d(st + (g.a_pieces + pb) * TC_TILE_BYTES, &tmB, &full[s], g.b_x0 + kb * TC_BK, nt * TC_BN,
                       p + pb * g.b_zpiece);
@@ -192,70 +187,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int row = q * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const int m = p >> 1, jh = p & 1;
-    bool built = true;
-    if (g.a_build) {
-      // ---- build the A operand (one tile per CTA in this mode): thread -> A row rl
-      // (sub-key mt*128 + rl), token quarter tq (16 tokens of each 64-token k-block) ----
-      const int et = threadIdx.x - 64;
-      const int rl = et & (TC_BM - 1), tq = et >> 7;
-      const int bsub = mt * TC_BM + rl;
-      const bool bvalid = bsub < g.m_valid;
-      const int n = g.m_valid;
-      const float* D = g.bD + (size_t)p * g.bD_pstride;
-      const float lpb = bvalid ? g.blp[(size_t)p * n + bsub] : 0.f;
-      const float inv_len = 1.f / (float)g.blen;
-      float wacc = 0.f;
-      for (int kb = 0; kb < g.k_blocks && built; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (kb >= S) {
-          int okw = lane == 0 ? (mbar_wait(&empty[s], ph ^ 1, abort_flag, deadline) ? 1 : 0) : 0;
-          okw = __shfl_sync(0xffffffffu, okw, 0);
-          if (!okw) {
-            built = false;
-            break;
-          }
-        }
-        uint8_t* st = tiles + (size_t)s * npc * TC_TILE_BYTES;
-        const int t0 = kb * TC_BK + tq * 16;
-        float dd[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int t = t0 + u;
-          dd[u] = (bvalid && t < g.blen) ? D[(size_t)t * n + bsub] : 0.f;
-        }
-        __align__(16) __nv_bfloat16 hi[16], lo[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int t = t0 + u;
-          float W = 0.f;
-          if (bvalid && t < g.blen) {
-            const float wv = __fdividef(1.f, g.beps + dd[u]);
-            const float P_ = wv * (1.f / g.bZ[(size_t)p * g.bC + t]);
-            W = inv_len * P_ * (lpb - g.bL[(size_t)p * g.bC + t]) * wv;
-          }
-          wacc += W;
-          hi[u] = __float2bfloat16_rn(W);
-          lo[u] = __float2bfloat16_rn(W - __bfloat162float(hi[u]));
-        }
-        // 128-byte-swizzled K-major tile: row rl holds 64 tokens in eight 16-byte chunks,
-        // chunk c stored at position c ^ (rl % 8)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int c = tq * 2 + hf;
-          const size_t off = (size_t)rl * 128 + (size_t)((c ^ (rl & 7)) << 4);
-          *reinterpret_cast<uint4*>(st + off) = *reinterpret_cast<const uint4*>(hi + hf * 8);
-          *reinterpret_cast<uint4*>(st + TC_TILE_BYTES + off) = *reinterpret_cast<const uint4*>(lo + hf * 8);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[s]);
-      }
-      s_wsum[tq][rl] = wacc;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(wsbar);
-    }
-    for (int j = 0; j < ntiles && built; ++j) {
+    for (int j = 0; j < ntiles; ++j) {
       const int b = j & 1;
       const uint32_t aph = (j >> 1) & 1;
       const int nt = nt0 + j;
@@ -282,29 +214,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
       } else if (g.epi == TC_EPI_KEYSTEP) {
         const int h = g.n_valid, n = g.m_valid, e0 = cg * 32;
-        if (g.a_build) {
-          // the four token quarters' partial sums of W, once every builder has published
-          int okw = lane == 0 ? (mbar_wait(wsbar, 0, abort_flag, deadline) ? 1 : 0) : 0;
-          okw = __shfl_sync(0xffffffffu, okw, 0);
-          if (okw) pre_s = ((s_wsum[0][row] + s_wsum[1][row]) + s_wsum[2][row]) + s_wsum[3][row];
-        }
         if (rv && e0 < h) {
-          // the key row is loaded while the MMAs run
-          if (!g.a_build) {
-            // the partial sums are independent loads: four interleaved accumulators keep
-            // them in flight, combined in a fixed order
-            const float* wp = g.wsum_part + (size_t)p * g.wsum_tiles * n + r;
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-            int tt = 0;
-            for (; tt + 4 <= g.wsum_tiles; tt += 4) {
-              a0 += wp[(size_t)tt * n];
-              a1 += wp[(size_t)(tt + 1) * n];
-              a2 += wp[(size_t)(tt + 2) * n];
-              a3 += wp[(size_t)(tt + 3) * n];
-            }
-            for (; tt < g.wsum_tiles; ++tt) a0 += wp[(size_t)tt * n];
-            pre_s = (a0 + a1) + (a2 + a3);
+          // the partial sums are independent loads: four interleaved accumulators keep
+          // them in flight, combined in a fixed order
+          const float* wp = g.wsum_part + (size_t)p * g.wsum_tiles * n + r;
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          int tt = 0;
+          for (; tt + 4 <= g.wsum_tiles; tt += 4) {
+            a0 += wp[(size_t)tt * n];
+            a1 += wp[(size_t)(tt + 1) * n];
+            a2 += wp[(size_t)(tt + 2) * n];
+            a3 += wp[(size_t)(tt + 3) * n];
           }
+          for (; tt < g.wsum_tiles; ++tt) a0 += wp[(size_t)tt * n];
+          pre_s = (a0 + a1) + (a2 + a3);
           const float* K = (jh == 0 ? g.K1 : g.K2) + ((size_t)m * n + r) * h + e0;
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {

@@ -132,46 +132,105 @@ tc_pbar_kernel(Dims dm, Work w, int len) {
   }
 }
 
-// L_t = sum_a P[t][a] lp[a] = (sum_a lp[a] w[t][a]) / Z_t for RL_T tokens per CTA: two
-// tokens per warp, their row loads and the shared log-marginal loads in flight together.
-// (W itself is formed by the key-step GEMM's epilogue warps as its A operand.)
-constexpr int RL_T = 16;
-__global__ void __launch_bounds__(TP_THREADS)
-tc_rowL_kernel(Dims dm, Work w, int len) {
+// W for a block of WB_T tokens and every sub-key, written sub-key major as two bf16
+// pieces (the A operand of the key-step GEMM), plus the block's per-sub-key sum of W.
+// First L_t = sum_a P[t][a] lp[a] = (sum_a lp[a] w[t][a]) / Z_t for the block's tokens (one
+// warp per token, a row's loads all in flight), then W[t][b] = (1/len) (w/Z_t) (lp[b] -
+// L_t) w for WB_SUB sub-keys per thread (the block's rows re-read, all loads in flight).
+constexpr int WB_T = 16;  // tokens per CTA (one wave of CTAs at the paper-scale shapes)
+constexpr int WB_G = 8;   // tokens per pass of the W phase (one 16-byte store per piece)
+constexpr int WB_SUB = 4; // sub-keys per thread per pass: 256 threads x 4 = 1024
+__global__ void __launch_bounds__(TP_THREADS, 3)
+tc_wbuild_kernel(Dims dm, Work w, int len, int cpad) {
   pdl_wait();
   pdl_trigger();
-  static_assert(RL_T == 2 * (TP_THREADS / 32), "two tokens per warp");
+  __shared__ float s_invz[WB_T], s_L[WB_T];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p = blockIdx.y, t0 = blockIdx.x * RL_T;
+  const int p = blockIdx.y, t0 = blockIdx.x * WB_T;
   const int n = dm.n;
   const float* D = w.Dfull + (size_t)p * w.drows * n;
   const float* lp = w.lp + (size_t)p * n;
-  const int ta = t0 + 2 * warp, tb = ta + 1;
-  const bool va = ta < len, vb = tb < len;
-  if (!va) return;
-  const float* Da = D + (size_t)ta * n;
-  const float* Db = D + (size_t)(vb ? tb : ta) * n;
-  float sa = 0.f, sb = 0.f;
-  for (int a0 = 0; a0 < n; a0 += 32 * 16) {
-    float da[16], db[16], ll[16];
+  // two tokens per warp, their row loads and the shared log-marginal loads in flight together
+  static_assert(WB_T == 2 * (TP_THREADS / 32), "two tokens per warp");
+  {
+    const int ta = t0 + 2 * warp, tb = ta + 1;
+    const bool va = ta < len, vb = tb < len;
+    const float* Da = D + (size_t)(va ? ta : 0) * n;
+    const float* Db = D + (size_t)(vb ? tb : 0) * n;
+    float sa = 0.f, sb = 0.f;
+    for (int a0 = 0; a0 < n; a0 += 32 * 16) {
+      float da[16], db[16], ll[16];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int a = a0 + lane + 32 * u;
-      ll[u] = a < n ? lp[a] : 0.f;
-      da[u] = a < n ? Da[a] : 0.f;
-      db[u] = a < n ? Db[a] : 0.f;
+      for (int u = 0; u < 16; ++u) {
+        const int a = a0 + lane + 32 * u;
+        ll[u] = a < n ? lp[a] : 0.f;
+        da[u] = (va && a < n) ? Da[a] : 0.f;
+        db[u] = (vb && a < n) ? Db[a] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        sa += __fdividef(ll[u], dm.eps_idw + da[u]);
+        sb += __fdividef(ll[u], dm.eps_idw + db[u]);
+      }
     }
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      sa += __fdividef(ll[u], dm.eps_idw + da[u]);
-      sb += __fdividef(ll[u], dm.eps_idw + db[u]);
+    sa = warp_sum(sa);
+    sb = warp_sum(sb);
+    if (lane == 0) {
+      const float za = va ? w.Z[(size_t)p * dm.C + ta] : 1.f, zb = vb ? w.Z[(size_t)p * dm.C + tb] : 1.f;
+      s_L[2 * warp] = va ? sa / za : 0.f;
+      s_invz[2 * warp] = va ? 1.f / za : 0.f;
+      s_L[2 * warp + 1] = vb ? sb / zb : 0.f;
+      s_invz[2 * warp + 1] = vb ? 1.f / zb : 0.f;
     }
   }
-  sa = warp_sum(sa);
-  sb = warp_sum(sb);
-  if (lane == 0) {
-    w.Lt[(size_t)p * dm.C + ta] = sa / w.Z[(size_t)p * dm.C + ta];
-    if (vb) w.Lt[(size_t)p * dm.C + tb] = sb / w.Z[(size_t)p * dm.C + tb];
+  __syncthreads();
+  const float inv_len = 1.f / (float)len;
+  const size_t pstride = (size_t)w.P_all * n * cpad;
+  const int ntb = gridDim.x;
+  for (int b0 = threadIdx.x; b0 < n; b0 += TP_THREADS * WB_SUB) {
+    float wsum[WB_SUB];
+#pragma unroll
+    for (int q = 0; q < WB_SUB; ++q) wsum[q] = 0.f;
+    for (int g0 = 0; g0 < WB_T; g0 += WB_G) {
+      const int tg = t0 + g0;
+      if (tg >= len) break;
+      float dd[WB_SUB][WB_G], lpb[WB_SUB];
+#pragma unroll
+      for (int q = 0; q < WB_SUB; ++q) {
+        const int b = b0 + q * TP_THREADS;
+        lpb[q] = b < n ? lp[b] : 0.f;
+#pragma unroll
+        for (int tl = 0; tl < WB_G; ++tl) dd[q][tl] = (b < n && tg + tl < len) ? D[(size_t)(tg + tl) * n + b] : 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < WB_SUB; ++q) {
+        const int b = b0 + q * TP_THREADS;
+        if (b >= n) continue;
+        __align__(16) __nv_bfloat16 hi[WB_G], lo[WB_G];
+#pragma unroll
+        for (int tl = 0; tl < WB_G; ++tl) {
+          float W = 0.f;
+          if (tg + tl < len) {
+            const float wv = __fdividef(1.f, dm.eps_idw + dd[q][tl]);
+            const float P_ = wv * s_invz[g0 + tl];
+            W = inv_len * P_ * (lpb[q] - s_L[g0 + tl]) * wv;
+          }
+          wsum[q] += W;
+          // two bf16 pieces (~16 significant bits): W only scales the key step, whose
+          // error this leaves at ~1e-5 of the step
+          hi[tl] = __float2bfloat16_rn(W);
+          lo[tl] = __float2bfloat16_rn(W - __bfloat162float(hi[tl]));
+        }
+        __nv_bfloat16* dst = w.Wt + ((size_t)p * n + b) * cpad + tg;
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(hi);
+        *reinterpret_cast<uint4*>(dst + pstride) = *reinterpret_cast<uint4*>(lo);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < WB_SUB; ++q) {
+      const int b = b0 + q * TP_THREADS;
+      if (b < n) w.wsum_part[((size_t)p * ntb + blockIdx.x) * n + b] = wsum[q];
+    }
   }
 }
 
@@ -261,7 +320,8 @@ int launch_tc_pbar(const Dims& d, const Work& w, int len, cudaStream_t s) {
 
 int launch_tc_wbuild(const Dims& d, const Work& w, int len, cudaStream_t s) {
   if (len <= 0) return 0;
-  launch_k(tc_rowL_kernel, dim3((len + RL_T - 1) / RL_T, d.M * 2), TP_THREADS, 0, s, d, w, len);
+  const int cpad = (d.C + 63) / 64 * 64;
+  launch_k(tc_wbuild_kernel, dim3((len + WB_T - 1) / WB_T, d.M * 2), TP_THREADS, 0, s, d, w, len, cpad);
   return 1;
 }
 
@@ -269,32 +329,30 @@ int launch_tc_keystep(const Dims& d, const Work& w, float* K1, float* K2, const 
                       int qt_t0, cudaStream_t s) {
   if (len <= 0) return 0;
   const int P = d.M * 2;
+  const int cpad = (d.C + 63) / 64 * 64;
   const int ntt = (len + 63) / 64;
+  const int ntb = (len + WB_T - 1) / WB_T;
   int launched = 1;
   if (qt_t0 < 0) {
     launch_qtrans(d, w, q, q_stride, 0, len, s);
     qt_t0 = 0;
     ++launched;
   }
-  // A (W, two bf16 pieces) is built in shared memory by the GEMM's epilogue warps; only B
-  // (the half-queries) is loaded, so the B map stands in for the unused A map
-  CUtensorMap B;
+  CUtensorMap A, B;
+  if (!make_tmap_bf16_3d(&A, w.Wt, len, d.n, w.P_all + P, (uint64_t)cpad * 2, (uint64_t)d.n * cpad * 2))
+    return -1;
   if (!make_tmap_bf16_3d(&B, w.Qt, w.qt_T, d.h, P, (uint64_t)w.qt_T * 2, (uint64_t)d.h * w.qt_T * 2)) return -1;
-  const CUtensorMap& A = B;
   TcGemm g = {};
   g.P = P;
   g.k_blocks = ntt;
   g.n_tiles = 1;
   g.tiles_per_cta = 1;
   g.a_pieces = 2; g.b_pieces = 1;
-  g.a_div = 1; g.a_xoff = 0; g.a_y0 = 0; g.a_zpiece = 0; g.b_zpiece = 0; g.b_x0 = qt_t0;
+  g.a_div = 1; g.a_xoff = 0; g.a_y0 = 0; g.a_zpiece = w.P_all; g.b_zpiece = 0; g.b_x0 = qt_t0;
   g.m_valid = d.n; g.n_valid = d.h;
   g.epi = TC_EPI_KEYSTEP;
   g.K1 = K1; g.K2 = K2; g.Kpc = w.Kpc; g.kn = w.kn; g.piece_P = w.P_all;
-  g.lr = d.lr_key;
-  g.a_build = 1;
-  g.bD = w.Dfull; g.bD_pstride = (long long)w.drows * d.n;
-  g.bZ = w.Z; g.bL = w.Lt; g.bC = d.C; g.blp = w.lp; g.blen = len; g.beps = d.eps_idw;
+  g.wsum_part = w.wsum_part; g.wsum_tiles = ntb; g.lr = d.lr_key;
   g.status = w.status;
   launch_tc_gemm(A, B, g, (d.n + 127) / 128, s);
   return launched;
