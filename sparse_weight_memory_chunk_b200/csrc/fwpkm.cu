@@ -197,6 +197,14 @@ bool raise_smem_limit(const void* kern, size_t bytes) {
 thread_local int launch_priority = 0;
 thread_local bool launch_priority_set = false;
 
+int pbar_slices() {
+  static const int v = [] {
+    const char* e = getenv("FWPKM_PBAR_SLICES");
+    return (e && atoi(e) == 8) ? 8 : 16;
+  }();
+  return v;
+}
+
 bool pdl_enabled() {
   static const bool on = [] {
     const char* e = getenv("FWPKM_PDL");

@@ -65,9 +65,10 @@ struct Work {
 
 enum : int { TC_EPI_DIST = 0, TC_EPI_KEYSTEP = 1, TC_EPI_PROJ = 2 };
 
-// Token slices of the usage-marginal pass (pbar): each column's sum is formed in this many
-// partial sums, one per CTA slice.
+// Token slices of the usage-marginal pass (pbar): each column's sum is formed in up to
+// this many partial sums, one per CTA slice (FWPKM_PBAR_SLICES picks 8 or 16 at run time).
 constexpr int PBAR_SLICES = 16;
+int pbar_slices();
 
 // One batched tensor-core contraction (see tc_gemm.cu).  Problem p (blockIdx.z) owns
 // A tiles at (x = (p % a_div) * a_xoff + 64 kb, y = a_y0 + 128 mt, z = p / a_div + pa * a_zpiece)

@@ -79,16 +79,17 @@ keyprep_kernel(Dims dm, Work w, const float* __restrict__ K1, const float* __res
 }
 
 // Partial column sums sum_t w[t][a] / Z_t over one token slice; also Z_t itself.  The
-// last of the PBAR_SLICES blocks of a column block to finish (arrival counter, reset by
+// last of the slice blocks of a column block to finish (arrival counter, reset by
 // that block) adds the slices in slice order and writes lp = log(pbar).
 __global__ void __launch_bounds__(TP_THREADS)
 tc_pbar_kernel(Dims dm, Work w, int len) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float s_invz[1024 / PBAR_SLICES + 1];
+  __shared__ float s_invz[1024 / 8 + 1];  // tokens of one slice (at least 8 slices)
   __shared__ int s_last;
   const int p = blockIdx.y, sl = blockIdx.z;
-  const int t0 = (sl * len) / PBAR_SLICES, t1 = ((sl + 1) * len) / PBAR_SLICES;
+  const int ns = gridDim.z;
+  const int t0 = (sl * len) / ns, t1 = ((sl + 1) * len) / ns;
   const int nt = (dm.n + 127) / 128 * 4;  // 4 column groups per 128-column tile
   for (int t = t0 + threadIdx.x; t < t1; t += TP_THREADS) {
     // Z_t from the scoring epilogue's nt partial sums (a multiple of 4, 16-byte aligned):
@@ -113,21 +114,21 @@ tc_pbar_kernel(Dims dm, Work w, int len) {
     float s = 0.f;
 #pragma unroll 16
     for (int t = t0; t < t1; ++t) s += __fdividef(1.f, dm.eps_idw + D[(size_t)t * dm.n + a]) * s_invz[t - t0];
-    w.ppart[((size_t)p * PBAR_SLICES + sl) * dm.n + a] = s;
+    w.ppart[((size_t)p * ns + sl) * dm.n + a] = s;
   }
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
     int* c = w.pbar_cnt + (size_t)p * gridDim.x + blockIdx.x;
     const int prev = atomicAdd(c, 1);
-    s_last = prev == PBAR_SLICES - 1;
+    s_last = prev == ns - 1;
     if (s_last) *c = 0;  // every slice has arrived: ready for the next launch
   }
   __syncthreads();
   if (s_last && av) {
     __threadfence();
     float s = 0.f;
-    for (int k = 0; k < PBAR_SLICES; ++k) s += __ldcg(w.ppart + ((size_t)p * PBAR_SLICES + k) * dm.n + a);
+    for (int k = 0; k < ns; ++k) s += __ldcg(w.ppart + ((size_t)p * ns + k) * dm.n + a);
     w.lp[(size_t)p * dm.n + a] = logf(s / (float)len);
   }
 }
@@ -313,7 +314,7 @@ int launch_qtrans(const Dims& d, const Work& w, const void* q, long long q_strid
 
 int launch_tc_pbar(const Dims& d, const Work& w, int len, cudaStream_t s) {
   if (len <= 0) return 0;
-  launch_k(tc_pbar_kernel, dim3((d.n + TP_THREADS - 1) / TP_THREADS, d.M * 2, PBAR_SLICES), TP_THREADS, 0, s, d, w,
+  launch_k(tc_pbar_kernel, dim3((d.n + TP_THREADS - 1) / TP_THREADS, d.M * 2, pbar_slices()), TP_THREADS, 0, s, d, w,
            len);
   return 1;
 }
