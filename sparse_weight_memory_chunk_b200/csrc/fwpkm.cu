@@ -200,7 +200,7 @@ thread_local bool launch_priority_set = false;
 int pbar_slices() {
   static const int v = [] {
     const char* e = getenv("FWPKM_PBAR_SLICES");
-    return (e && atoi(e) == 8) ? 8 : 16;
+    return (e && atoi(e) == 16) ? 16 : 8;  // 8 measured faster (1.597 against 1.625 ms per step)
   }();
   return v;
 }

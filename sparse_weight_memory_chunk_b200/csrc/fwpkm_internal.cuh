@@ -66,7 +66,7 @@ struct Work {
 enum : int { TC_EPI_DIST = 0, TC_EPI_KEYSTEP = 1, TC_EPI_PROJ = 2 };
 
 // Token slices of the usage-marginal pass (pbar): each column's sum is formed in up to
-// this many partial sums, one per CTA slice (FWPKM_PBAR_SLICES picks 8 or 16 at run time).
+// this many partial sums, one per CTA slice (8 by default; FWPKM_PBAR_SLICES=16 for 16).
 constexpr int PBAR_SLICES = 16;
 int pbar_slices();
 
