@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--n-iter", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-metrics", action="store_true", help="skip the addressing-metrics measurement")
     ap.add_argument("--batch", type=int, default=None, help="override the number of sequences B (profiling)")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling)")
     ap.add_argument("--kernel", default=None,
@@ -399,6 +400,32 @@ def run_ours(args, w, rank, world, local_rank):
                               "unique_rows": U, "definition": "max(F_tc/P_tc, B_VK/BW_HBM) / t_step"},
             "kernels_one_step": kind_table,
             "clocks": clk, "gpu_launches": int(launches)}
+
+    # addressing metrics of the final pass's selections (windows of 32K tokens per memory),
+    # timed apart from the step
+    if not args.no_metrics:
+        mwin = 32768
+        mws = torch.empty(fwpkm.metrics_workspace_size(w.M, w.T, w.N, mwin), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            met, mcnt = fwpkm.addressing_metrics(idx, w.N, mwin, workspace=mws, stream=stream)
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        m0.record(stream)
+        for _ in range(reps):
+            fwpkm.addressing_metrics(idx, w.N, mwin, workspace=mws, stream=stream)
+        m1.record(stream)
+        torch.cuda.synchronize()
+        mms = m0.elapsed_time(m1) / reps
+        nwin = met.shape[0] * met.shape[1]
+        mbytes = idx.numel() * 4 + nwin * w.N * 4 * 2  # selections read; counters zero-filled and read once
+        mv = met.cpu().numpy().reshape(-1, 3)
+        line["addressing_metrics"] = {
+            "window_tokens": mwin, "windows": int(nwin), "ms": mms,
+            "coverage_mean": float(mv[:, 0].mean()), "collision_mean": float(mv[:, 1].mean()),
+            "kld_mean": float(mv[:, 2].mean()),
+            "roofline": {"bound": "hbm", "achieved": mbytes / (mms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": mbytes / (mms / 1e3) / 1e9 / hbm_peak, "algorithmic_bytes": mbytes,
+                         "definition": "selections read once + N 32-bit counters per window written and read once"}}
 
     # end to end through the public API with host buffers
     if not args.no_e2e:

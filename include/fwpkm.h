@@ -234,6 +234,42 @@ void fwpkm_layer_destroy(fwpkm_layer* L);
  * inspection and for comparing selections against a reference. */
 fwpkm_status fwpkm_last_addressing(fwpkm_state* st, int T, int32_t* idx_out, float* w_out, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Addressing metrics ("Fast-weight Product Key Memory" (paperlayer summary), §D.3
+ * Addressing Metrics): slot-use balance of the reads over windows of tokens.
+ * The row contribution c_i of slot i is how many accesses it receives in a window,
+ * an access being one (token, selected slot) pair; windows are consecutive blocks of
+ * `window` tokens of each memory (the paper uses 32768; the last window may be
+ * shorter).  Per (memory, window):
+ *   coverage  = #{i : c_i > 0} / N
+ *   collision = (accesses whose slot receives >= 2 accesses in the window) / (accesses)
+ *   KLD       = sum_i p_i log(p_i N), p_i = c_i / sum c   (KL to uniform, natural log)
+ * (all three 0 for a window without accesses).  Entries outside [0, N) are not
+ * accesses and are counted apart.
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of device workspace that lets fwpkm_addressing_metrics histogram up to 32
+ * windows at once (4 * N bytes plus 8 KiB per window).  Any workspace that holds
+ * one window works; a smaller one only processes fewer windows at a time. */
+fwpkm_status fwpkm_metrics_workspace_size(int num_mem, int T, int N, int window, size_t* bytes);
+
+/* Metrics of every (memory, window) of the selections idx.
+ *   idx      device int32 [num_mem][T][k] (4-byte aligned): selected slots, as written by
+ *            fwpkm_forward_chunk (idx_out) or fwpkm_last_addressing; read only.
+ *   N        slots per memory (n*n); window >= 1 tokens; k >= 1.
+ *   workspace device, 256-byte aligned, ws_bytes >= the one-window size (else
+ *            FWPKM_ERR_WORKSPACE); scratch, contents need not be initialised.
+ *   metrics  device fp64 [num_mem][W][3] (coverage, collision, KLD), W = ceil(T/window).
+ *   counts   device int64 [num_mem][W][4] or NULL: rows accessed, accesses, competitive
+ *            accesses, invalid entries -- exact integers.
+ * Coverage and collision are exact ratios of those integers (fp64 division); KLD is
+ * (sum_i c_i log c_i) / S + log(N / S) in fp64 with a fixed summation order, so the
+ * call is deterministic.  T == 0 is a no-op.  Enqueued on `stream`; the workspace must
+ * not be shared with a concurrent call. */
+fwpkm_status fwpkm_addressing_metrics(const int32_t* idx, int num_mem, int T, int k, int N, int window,
+                                      void* workspace, size_t ws_bytes, double* metrics, int64_t* counts,
+                                      void* stream);
+
 /* Wait for `stream` and return the latched device status (FWPKM_OK,
  * FWPKM_ERR_TIMEOUT, ...), clearing it. */
 fwpkm_status fwpkm_sync(fwpkm_state* st, void* stream);

@@ -194,6 +194,8 @@ bool raise_smem_limit(const void* kern, size_t bytes) {
   return true;
 }
 
+void count_launches(int n) { g_launches += (uint64_t)n; }
+
 thread_local int launch_priority = 0;
 thread_local bool launch_priority_set = false;
 

@@ -179,6 +179,10 @@ bool raise_smem_limit(const void* kern, size_t bytes);
 // finishes (programmatic stream serialization).  Every kernel launched this way calls
 // pdl_wait() before it touches memory that an earlier kernel writes, so the overlap
 // covers only its launch and set-up.
+// Adds kernel launches made outside a state's schedule (layer projections, metrics) to
+// the count fwpkm_launch_count() reports.
+void count_launches(int n);
+
 // Scheduling priority given to the kernels launched by this host thread (set around a
 // launcher call by the schedule; `launch_priority_set` false: the stream's own).
 extern thread_local int launch_priority;

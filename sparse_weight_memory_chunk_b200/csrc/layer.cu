@@ -245,6 +245,7 @@ fwpkm_status fwpkm_layer_set_params(fwpkm_layer* L, const fwpkm_layer_params* p,
   fold_weights_kernel<<<blocks((long long)D * c.d_v), LAYER_THREADS, 0, s>>>(
       (const __nv_bfloat16*)p->W_o, p->gamma_o, D, c.d_v, L->Wo, o_ps, 0, L->o_pieces);
   copy_bias_kernel<<<blocks(D), LAYER_THREADS, 0, s>>>(p->b_o, D, L->bo);
+  count_launches(7);
   L->b_g = p->b_g;
   L->have_params = 1;
   return cuda_status();
@@ -275,6 +276,7 @@ fwpkm_status fwpkm_layer_in(fwpkm_layer* L, const void* h, int rows, void* q, vo
   t.out_bf16 = c.qv_dtype == FWPKM_BF16;
   t.status = L->status;
   launch_tc_gemm(A, B, t, (rows + 127) / 128, s);
+  count_launches(2);
   return cuda_status();
 }
 
@@ -303,6 +305,7 @@ fwpkm_status fwpkm_layer_out(fwpkm_layer* L, const float* o, int rows, void* o_o
   t.out_bf16 = 1;
   t.status = L->status;
   launch_tc_gemm(A, B, t, (rows + 127) / 128, s);
+  count_launches(2);
   return cuda_status();
 }
 

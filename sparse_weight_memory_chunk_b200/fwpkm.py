@@ -96,6 +96,10 @@ def lib():
             "fwpkm_layer_out": ([_P, _P, ctypes.c_int, _P, _P], ctypes.c_int),
             "fwpkm_layer_sync": ([_P, _P], ctypes.c_int),
             "fwpkm_layer_destroy": ([_P], None),
+            "fwpkm_metrics_workspace_size": ([ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+            "fwpkm_addressing_metrics": ([_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          _P, ctypes.c_size_t, _P, _P, _P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -142,6 +146,30 @@ def chunk_step_noalloc(cfg: Config, K1, K2, V, q, v, g, o, c_len, seq_stride=Non
     _check(lib().fwpkm_chunk_step_noalloc(ctypes.byref(cfg), _ptr(K1), _ptr(K2), _ptr(V), _ptr(q), _ptr(v),
                                           _ptr(g), _ptr(v_next), c_len, seq_stride, _ptr(o), _stream(stream)),
            "chunk_step_noalloc")
+
+
+def metrics_workspace_size(num_mem: int, T: int, N: int, window: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().fwpkm_metrics_workspace_size(num_mem, T, N, window, ctypes.byref(out)), "metrics_workspace_size")
+    return out.value
+
+
+def addressing_metrics(idx, N: int, window: int = 32768, workspace=None, stream=None):
+    """Addressing metrics of selections idx (int32 CUDA tensor [M][T][k]) per window of tokens.
+
+    Returns (metrics fp64 [M][W][3]: coverage, collision rate, KLD; counts int64 [M][W][4]:
+    rows accessed, accesses, competitive accesses, invalid entries), W = ceil(T / window).
+    """
+    import torch
+    M, T, k = idx.shape
+    W = (T + window - 1) // window
+    met = torch.zeros(M, W, 3, dtype=torch.float64, device=idx.device)
+    cnt = torch.zeros(M, W, 4, dtype=torch.int64, device=idx.device)
+    if workspace is None:
+        workspace = torch.empty(metrics_workspace_size(M, T, N, window), dtype=torch.uint8, device=idx.device)
+    _check(lib().fwpkm_addressing_metrics(_ptr(idx), M, T, k, N, window, _ptr(workspace), workspace.numel(),
+                                          _ptr(met), _ptr(cnt), _stream(stream)), "addressing_metrics")
+    return met, cnt
 
 
 class State:

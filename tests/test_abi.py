@@ -84,3 +84,24 @@ def test_layer_workspace_size_and_validation(lib):
     assert so.fwpkm_layer_workspace_size(C.byref(cfg), None) == lib.ERR_INVALID_ARG
     c = lib.LayerConfig(2048, 256, 256, 16, 1e-6, 7)
     assert so.fwpkm_layer_workspace_size(C.byref(c), C.byref(out)) == lib.ERR_INVALID_ARG
+
+
+def test_metrics_workspace_size_and_validation(lib):
+    import ctypes as C
+    so = lib.lib()
+    N = 1024 * 1024
+    # one window per memory: 8 windows of N 32-bit counters, plus 8 KiB of partials per window
+    ws = lib.metrics_workspace_size(8, 4096, N, 32768)
+    assert 8 * N * 4 <= ws < 8 * N * 4 + (1 << 17)
+    # at most 32 windows at once, however long the sequence
+    assert lib.metrics_workspace_size(8, 1 << 22, N, 32768) < 33 * N * 4
+    out = C.c_size_t(0)
+    for args in [(0, 16, 64, 8), (1, -1, 64, 8), (1, 16, 0, 8), (1, 16, 64, 0)]:
+        assert so.fwpkm_metrics_workspace_size(*args, C.byref(out)) == lib.ERR_INVALID_ARG
+    fake = C.c_void_p(1 << 20)  # aligned, never dereferenced: every call below returns before any launch
+    assert so.fwpkm_addressing_metrics(fake, 1, 0, 4, 64, 8, fake, 0, fake, None, None) == lib.OK  # T = 0
+    assert so.fwpkm_addressing_metrics(None, 1, 16, 4, 64, 8, fake, 1 << 20, fake, None, None) == lib.ERR_INVALID_ARG
+    assert so.fwpkm_addressing_metrics(fake, 1, 16, 0, 64, 8, fake, 1 << 20, fake, None, None) == lib.ERR_INVALID_ARG
+    assert so.fwpkm_addressing_metrics(fake, 1, 16, 4, 64, 8, C.c_void_p((1 << 20) + 16), 1 << 20, fake, None,
+                                       None) == lib.ERR_INVALID_ARG  # workspace not 256-byte aligned
+    assert so.fwpkm_addressing_metrics(fake, 1, 16, 4, 64, 8, fake, 64, fake, None, None) == lib.ERR_WORKSPACE
