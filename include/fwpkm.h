@@ -137,6 +137,31 @@ fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream
 fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, const float* g,
                                 int T, int n_iter, float* o, void* stream);
 
+/* Token-at-a-time inference ("Fast-weight Product Key Memory" (paperlayer summary),
+ * §A.1: at inference the memory accumulates (q_t, v_{t+1}) pairs and writes once a
+ * chunk's worth is ready).  Each call reads n_tok >= 1 new tokens of every memory at once,
+ * in order, against the state left by the last write, and writes o for them; the tokens
+ * are staged in the workspace.  A chunk of cfg.chunk pending tokens is written as soon as
+ * the token after it arrives (that token's v is the lookahead target of the chunk's last
+ * token), before that token is read; fwpkm_stream_flush() writes a partial or full
+ * pending chunk with no lookahead (end of the sequence).  The tokens of a sequence fed in
+ * any grouping followed by a flush give the outputs and final state of
+ * fwpkm_run_sequence over the same tokens (n_iter = 1).
+ *   q, v, g, o  device, element (m, t, e) of the call's tokens at q[(m*seq_stride + t)*d + e]
+ *               etc., as in fwpkm_forward_chunk (seq_stride >= n_tok); read/written by work
+ *               enqueued on `stream` (keep them until the stream passes the call).
+ * The state must have been initialised with max_T >= cfg.chunk (else
+ * FWPKM_ERR_UNSUPPORTED).  While tokens are pending, fwpkm_forward_chunk and
+ * fwpkm_run_sequence return FWPKM_ERR_STATE, and the caller must not change K1, K2, V
+ * (between chunks it may).  The keys are re-read at the start of every call.  With the
+ * key update, a chunk's write recomputes its distance rows from the staged queries. */
+fwpkm_status fwpkm_stream_tokens(fwpkm_state* st, const void* q, const void* v, const float* g, int n_tok,
+                                 int seq_stride, float* o, void* stream);
+
+/* End of a token-at-a-time sequence: write the pending tokens (if any) with no lookahead
+ * target for the last one.  No-op when nothing is pending. */
+fwpkm_status fwpkm_stream_flush(fwpkm_state* st, void* stream);
+
 /* One whole chunk step -- the read of fwpkm_forward_chunk followed by the write (and
  * key step) of fwpkm_write_chunk -- that allocates nothing and needs no workspace.
  * The paper has no counterpart: this exists for callers that cannot allocate device
@@ -145,8 +170,9 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
  * what they mean in fwpkm_forward_chunk / fwpkm_write_chunk (K1, K2, V are the
  * caller's state, updated in place; v_next NULL = the chunk ends the sequence).
  * Scratch is a fixed 16 MiB array inside the library that every GPU loading the
- * library keeps until exit; shapes whose fwpkm_workspace_size(cfg, cfg->chunk)
- * exceeds it are rejected with FWPKM_ERR_UNSUPPORTED.  The first call on a device
+ * library keeps until exit; shapes whose scratch for one chunk (fwpkm_workspace_size(cfg,
+ * cfg->chunk) less the staging rows of token-at-a-time inference) exceeds it are rejected
+ * with FWPKM_ERR_UNSUPPORTED.  The first call on a device
  * looks up that array's device address (make it before any stream capture).  All
  * calls share the array: calls that overlap on the GPU race and must be serialised
  * by the caller.  Device-side errors are not reported by this entry point. */

@@ -8,6 +8,7 @@
 // V.  With the key update off the keys are constant, so the addressing of every
 // chunk and every pass is computed once, up front, in a few large launches, and only
 // the value loop (gather, write) stays chunk-sequential.
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <cstdlib>
@@ -41,6 +42,9 @@ struct fwpkm_state {
   const float* g;
   int len;
   long long stride;
+  // token-at-a-time inference: tokens of the pending chunk read so far (staged in the
+  // workspace); its write waits for the next token (the lookahead) or a flush
+  int spos;
   // per-kernel timing
   int prof_kind;  // kernel kind timed with events; FWPKM_PROFILE_ALL: every kind
   std::vector<int> ev_kind;  // kind of each timed launch (event pair)
@@ -234,7 +238,7 @@ int addressing_window(const Dims& d, int max_T) {
   return (int)wtok;
 }
 
-size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
+size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base, bool stream_stage) {
   const size_t M = d.M, k = d.k, C = d.C, n = d.n, dv = d.dv;
   const size_t T = max_T;
   const size_t nch = (T + C - 1) / C;
@@ -287,6 +291,14 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base) {
   }
   x.P_all = (int)(2 * M);
   x.dfull_buf = (long long)(M * 2 * (size_t)x.drows * n);
+  x.stage_q = x.stage_v = nullptr;
+  x.stage_g = nullptr;
+  if (stream_stage) {
+    const size_t es = d.qv_bf16 ? 2 : 4;
+    x.stage_q = take(es * M * C * d.d);
+    x.stage_v = take(es * M * (C + 1) * dv);
+    x.stage_g = (float*)take(4 * M * (C + 1));
+  }
   if (w) *w = x;
   return off;
 }
@@ -361,6 +373,7 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
   workspace_bytes(dm, max_T, &st->wk, (char*)workspace);
   st->K1 = K1; st->K2 = K2; st->V = V;
   st->pending = 0;
+  st->spos = 0;
   st->prof_kind = 0;
   st->ev_used = 0;
   st->host_error = 0;
@@ -445,6 +458,7 @@ fwpkm_status fwpkm_forward_chunk(fwpkm_state* st, const void* q, const void* v, 
   const Dims& d = st->dm;
   if (c_len < 1 || c_len > d.C || c_len > st->wk.max_T || seq_stride < c_len) return FWPKM_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4)) return FWPKM_ERR_INVALID_ARG;
+  if (st->spos) return FWPKM_ERR_STATE;  // token-at-a-time chunk pending
   fwpkm_status ps = peek_status(st);
   if (ps != FWPKM_OK) return ps;
   cudaStream_t s = (cudaStream_t)stream;
@@ -489,6 +503,117 @@ fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream
     run(st, KK_ADDR, s, [&] { return launch_address(d, st->wk, st->K1, st->K2, st->q, st->stride, st->len, s); });
   }
   st->pending = 0;
+  if (st->host_error) return FWPKM_ERR_CUDA;
+  return last_cuda();
+}
+
+// ---- token-at-a-time inference ----
+// The pending chunk's q, v, g are staged in the workspace as they arrive (chunk-local
+// rows 0..spos-1), and each arriving group of tokens is read at once against the state
+// left by the last write: the reads are per token, so reading a chunk in pieces gives
+// the bits of reading it whole.  The chunk is written when the token after it arrives
+// (its v is the lookahead target of the chunk's last token) or at a flush (no target).
+// The key step needs every token's distance row, so the write recomputes the chunk's
+// distances from the staged queries with the same kernel (the keys have not changed
+// since the reads).
+
+// Read tokens [spos, spos + len) of the pending chunk (already staged); v, g, o are the
+// caller's rows of those tokens.
+static void stream_read(fwpkm_state* st, const void* v, const float* g, long long stride, int len, float* o,
+                        cudaStream_t s) {
+  const Dims& d = st->dm;
+  const Work& wk = st->wk;
+  const size_t es = qv_size(d);
+  const int p = st->spos;
+  const void* qs = offs(wk.stage_q, (long long)p * d.d, es);
+  if (wk.tc) {
+    run(st, KK_PREP, s, [&] { return launch_qnorm(d, wk, qs, d.C, p, len, s); });
+    run(st, KK_SCORE, s, [&] { return launch_tc_score(d, wk, wk.stage_q, d.C, d.C, p, p, len, false, s); });
+    run(st, KK_TOPK, s, [&] { return launch_select(d, wk, p, len, nullptr, nullptr, s); });
+  } else {
+    run(st, KK_SCORE, s, [&] { return launch_score_topk(d, wk, st->K1, st->K2, qs, d.C, p, len, false, s); });
+    run(st, KK_CART, s, [&] { return launch_cartesian(d, wk, p, len, nullptr, nullptr, s); });
+  }
+  run(st, KK_GATHER, s, [&] { return launch_gather(d, wk, st->V, v, g, stride, p, len, o, false, nullptr, s); });
+}
+
+// Write the pending chunk (spos tokens); has_next: staged row C holds the lookahead v.
+static void stream_write(fwpkm_state* st, bool has_next, cudaStream_t s) {
+  const Dims& d = st->dm;
+  const Work& wk = st->wk;
+  const size_t es = qv_size(d);
+  const int len = st->spos;
+  const void* vn = has_next ? offs(wk.stage_v, (long long)d.C * d.dv, es) : nullptr;
+  const bool last_has_target = has_next || !(d.flags & FWPKM_LOOKAHEAD);
+  run(st, KK_OTHER, s, [&] { return launch_resid(d, wk, wk.stage_v, wk.stage_g, d.C + 1, len, vn, s); });
+  run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, wk, 0, len, last_has_target, s); });
+  run(st, KK_WRITE, s, [&] { return launch_write(d, wk, st->V, 0, s); });
+  if (d.flags & FWPKM_KEY_UPDATE) {
+    if (wk.tc) {
+      run(st, KK_SCORE, s, [&] { return launch_tc_score(d, wk, wk.stage_q, d.C, d.C, 0, 0, len, true, s); });
+      run(st, KK_PBAR, s, [&] { return launch_tc_pbar(d, wk, len, s); });
+      run(st, KK_WBUILD, s, [&] { return launch_tc_wbuild(d, wk, len, s); });
+      run(st, KK_ADDR, s, [&] { return launch_tc_keystep(d, wk, st->K1, st->K2, wk.stage_q, d.C, len, -1, s); });
+      run(st, KK_PREP, s, [&] { return launch_keyprep(d, wk, st->K1, st->K2, s); });
+    } else {
+      run(st, KK_SCORE, s, [&] {
+        return launch_score_topk(d, wk, st->K1, st->K2, wk.stage_q, d.C, 0, len, true, s);
+      });
+      run(st, KK_ADDR, s, [&] { return launch_address(d, wk, st->K1, st->K2, wk.stage_q, d.C, len, s); });
+    }
+  }
+  st->spos = 0;
+}
+
+fwpkm_status fwpkm_stream_tokens(fwpkm_state* st, const void* q, const void* v, const float* g, int n_tok,
+                                 int seq_stride, float* o, void* stream) {
+  if (!st || !q || !v || !g || !o) return FWPKM_ERR_INVALID_ARG;
+  const Dims& d = st->dm;
+  if (n_tok < 1 || seq_stride < n_tok) return FWPKM_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4)) return FWPKM_ERR_INVALID_ARG;
+  if (st->pending) return FWPKM_ERR_STATE;
+  if (st->wk.max_T < d.C || !st->wk.stage_q) return FWPKM_ERR_UNSUPPORTED;
+  fwpkm_status ps = peek_status(st);
+  if (ps != FWPKM_OK) return ps;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t es = qv_size(d);
+  const Work& wk = st->wk;
+  st->host_error = 0;
+  // the caller may have changed the keys since the last call
+  if (wk.tc) run(st, KK_PREP, s, [&] { return launch_keyprep(d, wk, st->K1, st->K2, s); });
+  int j = 0;
+  while (j < n_tok) {
+    if (st->spos == d.C) {
+      // token j completes the pending chunk's last pair: stage its v as the lookahead, write
+      const StageJob la[3] = {{nullptr, nullptr, 0, 0, 0},
+                              {offs(v, (long long)j * d.dv, es), wk.stage_v, seq_stride, d.C + 1,
+                               (int)(d.dv * es / 4)},
+                              {nullptr, nullptr, 0, 0, 0}};
+      run(st, KK_PREP, s, [&] { return launch_stage(d, la, d.C, 1, s); });
+      stream_write(st, true, s);
+    }
+    const int len = std::min(d.C - st->spos, n_tok - j);
+    const StageJob in[3] = {
+        {offs(q, (long long)j * d.d, es), wk.stage_q, seq_stride, d.C, (int)(d.d * es / 4)},
+        {offs(v, (long long)j * d.dv, es), wk.stage_v, seq_stride, d.C + 1, (int)(d.dv * es / 4)},
+        {g + j, wk.stage_g, seq_stride, d.C + 1, 1}};
+    run(st, KK_PREP, s, [&] { return launch_stage(d, in, st->spos, len, s); });
+    stream_read(st, offs(v, (long long)j * d.dv, es), g + j, seq_stride, len, o + (long long)j * d.dv, s);
+    st->spos += len;
+    j += len;
+  }
+  if (st->host_error) return FWPKM_ERR_CUDA;
+  return last_cuda();
+}
+
+fwpkm_status fwpkm_stream_flush(fwpkm_state* st, void* stream) {
+  if (!st) return FWPKM_ERR_INVALID_ARG;
+  if (st->pending) return FWPKM_ERR_STATE;
+  fwpkm_status ps = peek_status(st);
+  if (ps != FWPKM_OK) return ps;
+  if (st->spos == 0) return FWPKM_OK;
+  st->host_error = 0;
+  stream_write(st, false, (cudaStream_t)stream);
   if (st->host_error) return FWPKM_ERR_CUDA;
   return last_cuda();
 }
@@ -655,6 +780,7 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
   if (T == 0) return FWPKM_OK;
   if (!q || !v || !g || !o || T < 0 || T > st->wk.max_T || n_iter < 1) return FWPKM_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4)) return FWPKM_ERR_INVALID_ARG;
+  if (st->spos) return FWPKM_ERR_STATE;  // token-at-a-time chunk pending
   fwpkm_status ps = peek_status(st);
   if (ps != FWPKM_OK) return ps;
   st->pending = 0;

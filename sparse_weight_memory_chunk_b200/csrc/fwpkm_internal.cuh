@@ -61,6 +61,10 @@ struct Work {
   // pointers advanced to the group's first memory (see group_work).
   int P_all;         // problems between consecutive bf16 pieces of Kpc / Wt (2 * all memories)
   long long dfull_buf; // elements between the two distance-row buffers
+  // token-at-a-time inference: the pending chunk's inputs (nullptr when not carved)
+  void* stage_q;     // [M][C][d]     q of the pending chunk (qv dtype)
+  void* stage_v;     // [M][C+1][dv]  v of the pending chunk; row C: the lookahead token's v
+  float* stage_g;    // [M][C+1]      g of the pending chunk
 };
 
 enum : int { TC_EPI_DIST = 0, TC_EPI_KEYSTEP = 1, TC_EPI_PROJ = 2 };
@@ -99,7 +103,8 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t 
                        uint64_t pitch_z);
 int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g, int m_tiles, cudaStream_t s);
 
-size_t workspace_bytes(const Dims& d, int max_T, Work* carve, char* base);
+// stream_stage: also carve the staging rows of token-at-a-time inference (at the end).
+size_t workspace_bytes(const Dims& d, int max_T, Work* carve, char* base, bool stream_stage = true);
 // The carve `w` of all memories seen from memory m0 on (kernels index it from 0).
 Work group_work(const Dims& d, const Work& w, int m0);
 
@@ -127,6 +132,16 @@ int launch_sort_pairs(const Dims& d, const Work& w, int wt0, int total_len, bool
 int launch_gather(const Dims& d, const Work& w, const float* V, const void* v, const float* g,
                   long long stride, int wt0, int len, float* o, bool fuse_resid,
                   const void* v_next, cudaStream_t s);
+// Token-at-a-time inference: copy `len` tokens (rows of `words` 32-bit words, per memory
+// `src_stride` rows apart) of up to three inputs into staging rows r0.. (`dst_stride` rows
+// per memory).  A job with a null source is skipped.
+struct StageJob {
+  const void* src;
+  void* dst;
+  long long src_stride, dst_stride;
+  int words;
+};
+int launch_stage(const Dims& d, const StageJob (&jobs)[3], int r0, int len, cudaStream_t s);
 // Streaming write path: turn the stored vhat of a chunk into residuals.
 int launch_resid(const Dims& d, const Work& w, const void* v, const float* g, long long stride,
                  int len, const void* v_next, cudaStream_t s);

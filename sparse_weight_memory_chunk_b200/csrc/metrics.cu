@@ -133,17 +133,24 @@ metric_reduce_kernel(uint32_t* __restrict__ cnt, long long np_, int rezero, Metr
   }
 }
 
-// One thread per window of the batch: fixed-order sum of the partials, then the metrics.
-__global__ void metric_final_kernel(const MetricPart* __restrict__ part, unsigned long long* __restrict__ bad,
-                                    long long w0, int nb, long long N, double* __restrict__ out,
-                                    long long* __restrict__ counts) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+// One warp per window of the batch: each lane sums a fixed stride of the partials, then a
+// fixed butterfly combines the lanes (the order never changes, so neither do the bits).
+__global__ void __launch_bounds__(128) metric_final_kernel(const MetricPart* __restrict__ part,
+                                                           unsigned long long* __restrict__ bad, long long w0, int nb,
+                                                           long long N, double* __restrict__ out,
+                                                           long long* __restrict__ counts) {
+  const int b = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (b >= nb) return;
-  MetricPart t = part[(long long)b * MT_RED_BLOCKS];
-  for (int i = 1; i < MT_RED_BLOCKS; ++i) {
+  MetricPart t{0ull, 0ull, 0ull, 0.0};
+  for (int i = lane; i < MT_RED_BLOCKS; i += 32) {
     const MetricPart& p = part[(long long)b * MT_RED_BLOCKS + i];
     t.rows += p.rows; t.acc += p.acc; t.comp += p.comp; t.clogc += p.clogc;
   }
+  t.rows = warp_sum_u64(t.rows);
+  t.acc = warp_sum_u64(t.acc);
+  t.comp = warp_sum_u64(t.comp);
+  t.clogc = warp_sum_f64(t.clogc);
+  if (lane != 0) return;
   const unsigned long long nbad = bad[b];
   bad[b] = 0ull;  // ready for the next batch
   double cov = 0.0, col = 0.0, kld = 0.0;
@@ -219,7 +226,7 @@ fwpkm_status fwpkm_addressing_metrics(const int32_t* idx, int num_mem, int T, in
                                                                                   np_, bad);
     const int rezero = w0 + nb < total ? 1 : 0;
     metric_reduce_kernel<<<dim3(MT_RED_BLOCKS, (unsigned)nb), MT_THREADS, 0, s>>>(cnt, np_, rezero, part);
-    metric_final_kernel<<<(nb + 63) / 64, 64, 0, s>>>(part, bad, w0, nb, N, metrics, (long long*)counts);
+    metric_final_kernel<<<(nb + 3) / 4, 128, 0, s>>>(part, bad, w0, nb, N, metrics, (long long*)counts);
     launches += 3;
   }
   count_launches(launches);

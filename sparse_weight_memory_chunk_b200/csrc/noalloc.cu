@@ -56,8 +56,13 @@ extern "C" fwpkm_status fwpkm_chunk_step_noalloc(const fwpkm_config* cfg, float*
                                                  void* stream) {
   if (!cfg || !K1 || !K2 || !V || !q || !v || !g || !o) return FWPKM_ERR_INVALID_ARG;
   size_t need = 0;
-  fwpkm_status s = fwpkm_workspace_size(cfg, cfg->chunk, &need);
+  fwpkm_status s = fwpkm_workspace_size(cfg, cfg->chunk, &need);  // validates cfg
   if (s != FWPKM_OK) return s;
+  Dims d;
+  d.n = cfg->n; d.h = cfg->d / 2; d.d = cfg->d; d.dv = cfg->d_v; d.k = cfg->k; d.C = cfg->chunk;
+  d.M = cfg->num_mem; d.N = (long long)cfg->n * cfg->n; d.qv_bf16 = cfg->qv_dtype == FWPKM_BF16;
+  d.eps_idw = cfg->eps_idw; d.eps_norm = cfg->eps_norm; d.lr_key = cfg->lr_key; d.flags = cfg->flags;
+  need = workspace_bytes(d, cfg->chunk, nullptr, nullptr, false);  // no token-at-a-time staging
   if (need > FWPKM_NOALLOC_SCRATCH_BYTES) {
     fprintf(stderr, "fwpkm_chunk_step_noalloc: this shape needs %zu bytes of scratch; the built-in "
                     "array holds %u\n", need, FWPKM_NOALLOC_SCRATCH_BYTES);
@@ -72,12 +77,8 @@ extern "C" fwpkm_status fwpkm_chunk_step_noalloc(const fwpkm_config* cfg, float*
   s = scratch_address(&base);
   if (s != FWPKM_OK) return s;
 
-  Dims d;
-  d.n = cfg->n; d.h = cfg->d / 2; d.d = cfg->d; d.dv = cfg->d_v; d.k = cfg->k; d.C = cfg->chunk;
-  d.M = cfg->num_mem; d.N = (long long)cfg->n * cfg->n; d.qv_bf16 = cfg->qv_dtype == FWPKM_BF16;
-  d.eps_idw = cfg->eps_idw; d.eps_norm = cfg->eps_norm; d.lr_key = cfg->lr_key; d.flags = cfg->flags;
   Work w;
-  workspace_bytes(d, cfg->chunk, &w, (char*)base);
+  workspace_bytes(d, cfg->chunk, &w, (char*)base, false);
 
   cudaStream_t st = (cudaStream_t)stream;
   // The array keeps the previous call's contents: only the status word is read

@@ -195,7 +195,8 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
       orow[e4] = y;
     }
   }
-  float4* rrow = reinterpret_cast<float4*>(w.resid + ((size_t)m * dm.C + i) * dm.dv);
+  // resid rows are chunk-local: a call may start inside a chunk (token-at-a-time reads)
+  float4* rrow = reinterpret_cast<float4*>(w.resid + ((size_t)m * dm.C + wt0 % dm.C + i) * dm.dv);
   if (fuse_resid) {
     const VT* u = target_src<VT>(dm, v, v_next, stride, m, i, len);
     if (u == nullptr) return;
@@ -384,6 +385,39 @@ int launch_resid(const Dims& d, const Work& w, const void* v, const float* g, lo
     FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(resid_kernel<float, VPL>, grid, VAL_WARPS * 32, 0, s, 
         d, w, (const float*)v, g, stride, len, (const float*)v_next));
   }
+  return 1;
+}
+
+// Token-at-a-time inference: copy rows of up to three inputs into the staging buffers.
+struct StageJobs {
+  StageJob j[3];
+  int r0, len;
+};
+
+__global__ void __launch_bounds__(256) stage_kernel(StageJobs jobs) {
+  const StageJob& J = jobs.j[blockIdx.z];
+  if (J.src == nullptr) return;
+  const int m = blockIdx.y;
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(J.src) + (long long)m * J.src_stride * J.words;
+  uint32_t* dst = reinterpret_cast<uint32_t*>(J.dst) + ((long long)m * J.dst_stride + jobs.r0) * J.words;
+  const long long total = (long long)jobs.len * J.words;  // rows are contiguous on both sides
+  for (long long i = (long long)blockIdx.x * 256 + threadIdx.x; i < total; i += (long long)gridDim.x * 256)
+    dst[i] = src[i];
+}
+
+int launch_stage(const Dims& d, const StageJob (&jobs)[3], int r0, int len, cudaStream_t s) {
+  if (len <= 0) return 0;
+  StageJobs J;
+  int words = 1;
+  for (int i = 0; i < 3; ++i) {
+    J.j[i] = jobs[i];
+    if (jobs[i].src && jobs[i].words > words) words = jobs[i].words;
+  }
+  J.r0 = r0;
+  J.len = len;
+  long long bx = ((long long)len * words + 255) / 256;
+  if (bx > 64) bx = 64;
+  launch_k(stage_kernel, dim3((unsigned)bx, d.M, 3), 256, 0, s, J);
   return 1;
 }
 

@@ -79,6 +79,8 @@ def lib():
             "fwpkm_last_addressing": ([_P, ctypes.c_int, _P, _P, _P], ctypes.c_int),
             "fwpkm_chunk_step_noalloc": ([C, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P],
                                          ctypes.c_int),
+            "fwpkm_stream_tokens": ([_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P], ctypes.c_int),
+            "fwpkm_stream_flush": ([_P, _P], ctypes.c_int),
             "fwpkm_sync": ([_P, _P], ctypes.c_int),
             "fwpkm_destroy_state": ([_P], None),
             "fwpkm_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -206,6 +208,17 @@ class State:
         T = q.shape[1] if T is None else T
         _check(lib().fwpkm_run_sequence(self.handle, _ptr(q), _ptr(v), _ptr(g), T, n_iter, _ptr(o),
                                         _stream(stream)), "run_sequence")
+
+    def stream_tokens(self, q, v, g, o, n_tok=None, seq_stride=None, stream=None):
+        """Read n_tok new tokens of every memory ([M][seq_stride][..] rows); writes o for them."""
+        n_tok = q.shape[1] if n_tok is None else n_tok
+        seq_stride = q.shape[1] if seq_stride is None else seq_stride
+        _check(lib().fwpkm_stream_tokens(self.handle, _ptr(q), _ptr(v), _ptr(g), n_tok, seq_stride, _ptr(o),
+                                         _stream(stream)), "stream_tokens")
+
+    def stream_flush(self, stream=None):
+        """Write the pending tokens of a token-at-a-time sequence (no lookahead for the last)."""
+        _check(lib().fwpkm_stream_flush(self.handle, _stream(stream)), "stream_flush")
 
     def last_addressing(self, T, idx_out=None, w_out=None, stream=None):
         _check(lib().fwpkm_last_addressing(self.handle, T, _ptr(idx_out), _ptr(w_out), _stream(stream)),

@@ -1,0 +1,92 @@
+"""Token-at-a-time inference on the GPU (fwpkm_stream_tokens / fwpkm_stream_flush through
+the C ABI).
+
+Feeding a sequence in arbitrary groups of tokens, then flushing, must give the bits of the
+production entry point (fwpkm_run_sequence) on the same inputs: the reads are per token
+and the writes are the same kernels on the same chunk contents.  fwpkm_run_sequence is
+checked against the oracle chunk by chunk in test_gpu_parity.py, and the oracle's own
+token-at-a-time loop against its chunked loop in test_oracle_stream_pins.py.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+from sparse_weight_memory_chunk_b200 import fwpkm  # noqa: E402
+
+from test_gpu_parity import device_state, make_case  # noqa: E402
+
+
+def groups_for(T, C, seed):
+    rng = np.random.default_rng(seed)
+    sizes = [1, 2, 3, max(1, C - 1), C, C + 1, 2 * C + 3]
+    out, t = [], 0
+    while t < T:
+        n = min(T - t, int(rng.choice(sizes)))
+        out.append(n)
+        t += n
+    return out
+
+
+def reference(w, data, gcfg):
+    st, dev = device_state(w, data, gcfg, w.T)
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    st.run_sequence(dev["q"], dev["v"], dev["g"], o)
+    st.sync()
+    return o, dev
+
+
+@pytest.mark.parametrize("name", ["tiny_key_ragged", "mid", "mid_key", "k1", "chunk1", "k_equals_n", "paper"])
+def test_token_stream_gives_the_bits_of_run_sequence(name):
+    w, data, gcfg, _ = make_case(name)
+    o_ref, dev_ref = reference(w, data, gcfg)
+    st, dev = device_state(w, data, gcfg, w.C)  # a chunk of workspace is enough
+    o = torch.full((w.M, w.T, w.d_v), float("nan"), device="cuda")
+    t = 0
+    for n in groups_for(w.T, w.C, seed=len(name)):
+        st.stream_tokens(dev["q"][:, t:], dev["v"][:, t:], dev["g"][:, t:], o[:, t:], n_tok=n, seq_stride=w.T)
+        t += n
+        if t == w.C + 3 or (t > w.C + 3 and t - n < w.C + 3):
+            # outputs are final as soon as their tokens are read
+            st.sync()
+            assert torch.equal(o[:, :t], o_ref[:, :t]), f"{name}: o of the first {t} tokens"
+    st.stream_flush()
+    st.sync()
+    assert torch.equal(o, o_ref), f"{name}: o differs from run_sequence"
+    for key in ("V", "K1", "K2"):
+        assert torch.equal(dev[key], dev_ref[key]), f"{name}: {key} differs from run_sequence"
+
+
+def test_one_token_at_a_time_and_state_rules():
+    w, data, gcfg, _ = make_case("mid_key")
+    o_ref, dev_ref = reference(w, data, gcfg)
+    st, dev = device_state(w, data, gcfg, w.T)
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    st.stream_flush()  # nothing pending: no-op
+    for t in range(w.T):
+        st.stream_tokens(dev["q"][:, t:], dev["v"][:, t:], dev["g"][:, t:], o[:, t:], n_tok=1, seq_stride=w.T)
+        if t == 5:
+            with pytest.raises(fwpkm.FwpkmError) as e:  # chunk mode while tokens are pending
+                st.run_sequence(dev["q"], dev["v"], dev["g"], o)
+            assert e.value.status == fwpkm.ERR_STATE
+            with pytest.raises(fwpkm.FwpkmError) as e:
+                st.forward_chunk(dev["q"], dev["v"], dev["g"], o, 4, seq_stride=w.T)
+            assert e.value.status == fwpkm.ERR_STATE
+    st.stream_flush()
+    st.sync()
+    assert torch.equal(o, o_ref)
+    assert torch.equal(dev["V"], dev_ref["V"]) and torch.equal(dev["K1"], dev_ref["K1"])
+    # after the flush the state takes chunk-mode calls again
+    o2 = torch.zeros_like(o)
+    st.run_sequence(dev["q"], dev["v"], dev["g"], o2, T=w.C)
+    st.sync()
+
+
+def test_stream_needs_a_chunk_of_workspace():
+    w, data, gcfg, _ = make_case("mid")
+    st, dev = device_state(w, data, gcfg, w.C - 1)
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    with pytest.raises(fwpkm.FwpkmError) as e:
+        st.stream_tokens(dev["q"], dev["v"], dev["g"], o, n_tok=1, seq_stride=w.T)
+    assert e.value.status == fwpkm.ERR_UNSUPPORTED
