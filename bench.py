@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-metrics", action="store_true", help="skip the addressing-metrics measurement")
+    ap.add_argument("--no-stream", action="store_true", help="skip the token-at-a-time measurement")
     ap.add_argument("--batch", type=int, default=None, help="override the number of sequences B (profiling)")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling)")
     ap.add_argument("--kernel", default=None,
@@ -479,6 +480,42 @@ def run_ours(args, w, rank, world, local_rank):
                                    "min_cos": float(np.min(cos)), "needles": len(cos),
                                    "definition": "cos(vhat_r, z(v*)) at each needle's query position r, final pass, "
                                                  "run from the initial state"}
+
+    if not args.no_stream:
+        # token-at-a-time inference: the first 2C + 1 tokens of every memory fed 1 (then 16)
+        # per call through fwpkm_stream_tokens (two chunk writes, each when its lookahead
+        # arrives), then a flush; timed with events on the launching stream
+        S = min(w.T, 2 * w.C + 1)
+        for t_ in range(0, 8, 4):  # warm-up of the streaming launches
+            st.stream_tokens(qd[:, t_:], vd[:, t_:], gd[:, t_:], o[:, t_:], n_tok=4, seq_stride=w.T, stream=stream)
+        st.stream_flush(stream=stream)
+        torch.cuda.synchronize()
+        per = {}
+        for per_call in (1, 16):
+            l0s = fwpkm.launch_count()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            t_ = 0
+            while t_ < S:
+                n_ = min(per_call, S - t_)
+                st.stream_tokens(qd[:, t_:], vd[:, t_:], gd[:, t_:], o[:, t_:], n_tok=n_, seq_stride=w.T,
+                                 stream=stream)
+                t_ += n_
+            st.stream_flush(stream=stream)
+            s1.record(stream)
+            torch.cuda.synchronize()
+            sms = s0.elapsed_time(s1)
+            per[str(per_call)] = {"us_per_token": sms * 1e3 / S, "tokens_per_s": w.B * S / (sms / 1e3),
+                                  "launches_per_token": (fwpkm.launch_count() - l0s) / S}
+        st.sync()
+        line["token_stream"] = {
+            "tokens": S, "per_call": per,
+            "hbm_bytes_per_token_max": w.M * 3 * w.k * w.d_v * 4,
+            "definition": "tokens of the first 2C+1 positions of every sequence fed n per fwpkm_stream_tokens call, "
+                          "then fwpkm_stream_flush; tokens/s counts sequence tokens (B per position); "
+                          "hbm_bytes_per_token_max: gathered rows + the same rows read and written by the chunk "
+                          "write (unique rows), all memories; latency-bound: a token's read is a chain of about "
+                          "six dependent launches"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_chunks = 8 if w.name in ("paper", "needle") else 16

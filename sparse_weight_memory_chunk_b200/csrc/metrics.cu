@@ -17,7 +17,8 @@
 // the result is deterministic.  KLD = (sum c log c) / S + log(N / S) with S = sum c.
 // Several windows are histogrammed at once (up to MT_MAX_BATCH, as the workspace
 // allows); the counters of a batch are zeroed while they are read when another batch
-// follows, so the whole call zero-fills them only once.
+// follows, so the whole call zero-fills them only once.  Launches: one zero-fill, then
+// per batch a histogram pass and a reduction pass whose last CTA per window finishes it.
 #include "fwpkm_internal.cuh"
 
 namespace fwpkm {
@@ -36,27 +37,34 @@ long long padded_slots(long long N) { return (N + 3) / 4 * 4; }  // uint4 rows o
 
 size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace of a batch of B windows: counters [B][Np] u32 | parts [B][MT_RED_BLOCKS] | invalid [B] u64.
+// Workspace of a batch of B windows: counters [B][Np] u32 | parts [B][MT_RED_BLOCKS] |
+// invalid entries [B] u64 | reduction CTAs arrived [B] u32.
 size_t metrics_carve(long long N, int B, char* base, uint32_t** cnt, MetricPart** part,
-                     unsigned long long** bad) {
+                     unsigned long long** bad, unsigned** arrive) {
   const size_t c_bytes = al256((size_t)B * padded_slots(N) * 4);
   const size_t p_bytes = al256((size_t)B * MT_RED_BLOCKS * sizeof(MetricPart));
   const size_t b_bytes = al256((size_t)B * 8);
+  const size_t a_bytes = al256((size_t)B * 4);
   if (base) {
     *cnt = (uint32_t*)base;
     *part = (MetricPart*)(base + c_bytes);
     *bad = (unsigned long long*)(base + c_bytes + p_bytes);
+    *arrive = (unsigned*)(base + c_bytes + p_bytes + b_bytes);
   }
-  return c_bytes + p_bytes + b_bytes;
+  return c_bytes + p_bytes + b_bytes + a_bytes;
 }
 
 __global__ void __launch_bounds__(MT_THREADS)
-metric_zero_kernel(uint4* __restrict__ cnt, long long n_vec, unsigned long long* __restrict__ bad, int nb) {
+metric_zero_kernel(uint4* __restrict__ cnt, long long n_vec, unsigned long long* __restrict__ bad,
+                   unsigned* __restrict__ arrive, int nb) {
   const long long stride = (long long)gridDim.x * MT_THREADS;
   for (long long i = (long long)blockIdx.x * MT_THREADS + threadIdx.x; i < n_vec; i += stride)
     cnt[i] = make_uint4(0u, 0u, 0u, 0u);
   if (blockIdx.x == 0)
-    for (int b = threadIdx.x; b < nb; b += MT_THREADS) bad[b] = 0ull;
+    for (int b = threadIdx.x; b < nb; b += MT_THREADS) {
+      bad[b] = 0ull;
+      arrive[b] = 0u;
+    }
 }
 
 // Histogram of the accesses of window (w0 + blockIdx.y): the window's indices are one
@@ -95,10 +103,16 @@ __device__ __forceinline__ double warp_sum_f64(double x) {
   return x;
 }
 
-// Partial statistics of the counters of window blockIdx.y over a fixed slice pattern.
+// Partial statistics of the counters of window blockIdx.y over a fixed slice pattern; the
+// last CTA of the window to finish (arrival counter, after a fence) sums the partials --
+// each lane a fixed stride, then a fixed butterfly, so the bits never depend on which CTA
+// is last -- and writes the window's metrics.
 __global__ void __launch_bounds__(MT_THREADS)
-metric_reduce_kernel(uint32_t* __restrict__ cnt, long long np_, int rezero, MetricPart* __restrict__ part) {
+metric_reduce_kernel(uint32_t* __restrict__ cnt, long long np_, int rezero, MetricPart* __restrict__ part,
+                     unsigned long long* __restrict__ bad, unsigned* __restrict__ arrive, long long w0, long long N,
+                     double* __restrict__ out, long long* __restrict__ counts) {
   __shared__ MetricPart s_part[MT_THREADS / 32];
+  __shared__ bool s_last;
   uint4* c = reinterpret_cast<uint4*>(cnt + (long long)blockIdx.y * np_);
   const long long nv = np_ / 4;
   unsigned long long rows = 0, acc = 0, comp = 0;
@@ -121,38 +135,38 @@ metric_reduce_kernel(uint32_t* __restrict__ cnt, long long np_, int rezero, Metr
   acc = warp_sum_u64(acc);
   comp = warp_sum_u64(comp);
   clogc = warp_sum_f64(clogc);
-  const int warp = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) s_part[warp] = MetricPart{rows, acc, comp, clogc};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) s_part[warp] = MetricPart{rows, acc, comp, clogc};
   __syncthreads();
+  MetricPart* wpart = part + (long long)blockIdx.y * MT_RED_BLOCKS;
   if (threadIdx.x == 0) {
     MetricPart t = s_part[0];
     for (int i = 1; i < MT_THREADS / 32; ++i) {
       t.rows += s_part[i].rows; t.acc += s_part[i].acc; t.comp += s_part[i].comp; t.clogc += s_part[i].clogc;
     }
-    part[(long long)blockIdx.y * MT_RED_BLOCKS + blockIdx.x] = t;
+    wpart[blockIdx.x] = t;
+    __threadfence();
+    s_last = atomicAdd(arrive + blockIdx.y, 1u) == MT_RED_BLOCKS - 1;
   }
-}
-
-// One warp per window of the batch: each lane sums a fixed stride of the partials, then a
-// fixed butterfly combines the lanes (the order never changes, so neither do the bits).
-__global__ void __launch_bounds__(128) metric_final_kernel(const MetricPart* __restrict__ part,
-                                                           unsigned long long* __restrict__ bad, long long w0, int nb,
-                                                           long long N, double* __restrict__ out,
-                                                           long long* __restrict__ counts) {
-  const int b = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (b >= nb) return;
+  __syncthreads();
+  if (!s_last || warp != 0) return;
+  __threadfence();
   MetricPart t{0ull, 0ull, 0ull, 0.0};
   for (int i = lane; i < MT_RED_BLOCKS; i += 32) {
-    const MetricPart& p = part[(long long)b * MT_RED_BLOCKS + i];
-    t.rows += p.rows; t.acc += p.acc; t.comp += p.comp; t.clogc += p.clogc;
+    t.rows += __ldcg(&wpart[i].rows);
+    t.acc += __ldcg(&wpart[i].acc);
+    t.comp += __ldcg(&wpart[i].comp);
+    t.clogc += __ldcg(&wpart[i].clogc);
   }
   t.rows = warp_sum_u64(t.rows);
   t.acc = warp_sum_u64(t.acc);
   t.comp = warp_sum_u64(t.comp);
   t.clogc = warp_sum_f64(t.clogc);
   if (lane != 0) return;
-  const unsigned long long nbad = bad[b];
-  bad[b] = 0ull;  // ready for the next batch
+  const int b = blockIdx.y;
+  const unsigned long long nbad = __ldcg(bad + b);
+  bad[b] = 0ull;     // ready for the next batch
+  arrive[b] = 0u;
   double cov = 0.0, col = 0.0, kld = 0.0;
   if (t.acc > 0) {
     const double S = (double)t.acc;
@@ -185,7 +199,7 @@ fwpkm_status fwpkm_metrics_workspace_size(int num_mem, int T, int N, int window,
   if (!bytes || num_mem < 1 || T < 0 || N < 1 || window < 1) return FWPKM_ERR_INVALID_ARG;
   const long long total = (long long)num_mem * (((long long)T + window - 1) / window);
   const int B = (int)(total < 1 ? 1 : (total < MT_MAX_BATCH ? total : MT_MAX_BATCH));
-  *bytes = metrics_carve(N, B, nullptr, nullptr, nullptr, nullptr);
+  *bytes = metrics_carve(N, B, nullptr, nullptr, nullptr, nullptr, nullptr);
   return FWPKM_OK;
 }
 
@@ -201,18 +215,19 @@ fwpkm_status fwpkm_addressing_metrics(const int32_t* idx, int num_mem, int T, in
   const long long W = ((long long)T + window - 1) / window;
   const long long total = (long long)num_mem * W;
   int B = (int)(total < MT_MAX_BATCH ? total : MT_MAX_BATCH);
-  while (B > 1 && metrics_carve(N, B, nullptr, nullptr, nullptr, nullptr) > ws_bytes) --B;
-  if (metrics_carve(N, B, nullptr, nullptr, nullptr, nullptr) > ws_bytes) return FWPKM_ERR_WORKSPACE;
+  while (B > 1 && metrics_carve(N, B, nullptr, nullptr, nullptr, nullptr, nullptr) > ws_bytes) --B;
+  if (metrics_carve(N, B, nullptr, nullptr, nullptr, nullptr, nullptr) > ws_bytes) return FWPKM_ERR_WORKSPACE;
   uint32_t* cnt;
   MetricPart* part;
   unsigned long long* bad;
-  metrics_carve(N, B, (char*)workspace, &cnt, &part, &bad);
+  unsigned* arrive;
+  metrics_carve(N, B, (char*)workspace, &cnt, &part, &bad, &arrive);
   cudaStream_t s = (cudaStream_t)stream;
   const long long np_ = padded_slots(N);
   const long long n_vec = (long long)B * np_ / 4;
   const long long zb = (n_vec + MT_THREADS - 1) / MT_THREADS;
   metric_zero_kernel<<<(unsigned)(zb < 1184 ? (zb < 1 ? 1 : zb) : 1184), MT_THREADS, 0, s>>>(
-      reinterpret_cast<uint4*>(cnt), n_vec, bad, B);
+      reinterpret_cast<uint4*>(cnt), n_vec, bad, arrive, B);
   int launches = 1;
   const long long max_len = (window < T ? (long long)window : (long long)T) * k;
   for (long long w0 = 0; w0 < total; w0 += B) {
@@ -225,9 +240,9 @@ fwpkm_status fwpkm_addressing_metrics(const int32_t* idx, int num_mem, int T, in
     metric_count_kernel<<<dim3((unsigned)gx, (unsigned)nb), MT_THREADS, 0, s>>>(idx, T, k, N, window, W, w0, cnt,
                                                                                   np_, bad);
     const int rezero = w0 + nb < total ? 1 : 0;
-    metric_reduce_kernel<<<dim3(MT_RED_BLOCKS, (unsigned)nb), MT_THREADS, 0, s>>>(cnt, np_, rezero, part);
-    metric_final_kernel<<<(nb + 3) / 4, 128, 0, s>>>(part, bad, w0, nb, N, metrics, (long long*)counts);
-    launches += 3;
+    metric_reduce_kernel<<<dim3(MT_RED_BLOCKS, (unsigned)nb), MT_THREADS, 0, s>>>(
+        cnt, np_, rezero, part, bad, arrive, w0, N, metrics, (long long*)counts);
+    launches += 2;
   }
   count_launches(launches);
   const cudaError_t e = cudaGetLastError();
