@@ -153,7 +153,7 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
  * The state must have been initialised with max_T >= cfg.chunk (else
  * FWPKM_ERR_UNSUPPORTED).  While tokens are pending, fwpkm_forward_chunk and
  * fwpkm_run_sequence return FWPKM_ERR_STATE, and the caller must not change K1, K2, V
- * (between chunks it may).  The keys are re-read at the start of every call.  With the
+ * (between chunks it may: the keys are re-read at the start of every chunk).  With the
  * key update, a chunk's write recomputes its distance rows from the staged queries. */
 fwpkm_status fwpkm_stream_tokens(fwpkm_state* st, const void* q, const void* v, const float* g, int n_tok,
                                  int seq_stride, float* o, void* stream);

@@ -579,8 +579,9 @@ fwpkm_status fwpkm_stream_tokens(fwpkm_state* st, const void* q, const void* v, 
   const size_t es = qv_size(d);
   const Work& wk = st->wk;
   st->host_error = 0;
-  // the caller may have changed the keys since the last call
-  if (wk.tc) run(st, KK_PREP, s, [&] { return launch_keyprep(d, wk, st->K1, st->K2, s); });
+  // bf16 pieces of the keys for the scoring GEMM: made at the start of every chunk (the
+  // caller may change the keys between chunks, never inside one) and after a key step
+  if (wk.tc && st->spos == 0) run(st, KK_PREP, s, [&] { return launch_keyprep(d, wk, st->K1, st->K2, s); });
   int j = 0;
   while (j < n_tok) {
     if (st->spos == d.C) {

@@ -14,7 +14,9 @@
 // are exact and independent of the order of arrival), then one pass over the counters
 // that forms rows / accesses / competitive accesses exactly in 64-bit integers and
 // sum c log c (c >= 2) in fp64 over a fixed partition with a fixed reduction tree, so
-// the result is deterministic.  KLD = (sum c log c) / S + log(N / S) with S = sum c.
+// the result is deterministic.  Counts below 256 are tallied per CTA in shared memory
+// (integer atomics) and their c log c taken once per count value, so the scan evaluates
+// no logarithm per row (a divergent fp64 log per row was most of the pass's time).  KLD = (sum c log c) / S + log(N / S) with S = sum c.
 // Several windows are histogrammed at once (up to MT_MAX_BATCH, as the workspace
 // allows); the counters of a batch are zeroed while they are read when another batch
 // follows, so the whole call zero-fills them only once.  Launches: one zero-fill, then
@@ -27,6 +29,8 @@ namespace {
 constexpr int MT_THREADS = 256;
 constexpr int MT_RED_BLOCKS = 256;  // reduction CTAs per window (fixes the fp64 summation order)
 constexpr int MT_MAX_BATCH = 32;    // windows histogrammed together at most
+constexpr int MT_HIST = 256;        // counts below this are tallied per CTA (one log per count value)
+static_assert(MT_HIST == MT_THREADS, "one thread per tallied count value");
 
 struct MetricPart {
   unsigned long long rows, acc, comp;
@@ -112,7 +116,10 @@ metric_reduce_kernel(uint32_t* __restrict__ cnt, long long np_, int rezero, Metr
                      unsigned long long* __restrict__ bad, unsigned* __restrict__ arrive, long long w0, long long N,
                      double* __restrict__ out, long long* __restrict__ counts) {
   __shared__ MetricPart s_part[MT_THREADS / 32];
+  __shared__ unsigned s_hist[MT_HIST];  // rows of this CTA's slice with count c (2 <= c < MT_HIST)
   __shared__ bool s_last;
+  s_hist[threadIdx.x] = 0u;
+  __syncthreads();
   uint4* c = reinterpret_cast<uint4*>(cnt + (long long)blockIdx.y * np_);
   const long long nv = np_ / 4;
   unsigned long long rows = 0, acc = 0, comp = 0;
@@ -127,9 +134,15 @@ metric_reduce_kernel(uint32_t* __restrict__ cnt, long long np_, int rezero, Metr
       acc += x[e];
       if (x[e] >= 2u) {
         comp += x[e];
-        clogc += (double)x[e] * log((double)x[e]);
+        if (x[e] < (uint32_t)MT_HIST) atomicAdd(&s_hist[x[e]], 1u);  // exact integer tally
+        else clogc += (double)x[e] * log((double)x[e]);
       }
     }
+  }
+  __syncthreads();
+  {  // c log c of the tallied rows: thread c takes count value c (a fixed assignment)
+    const unsigned hc = s_hist[threadIdx.x];
+    if (hc != 0u) clogc += (double)hc * ((double)threadIdx.x * log((double)threadIdx.x));
   }
   rows = warp_sum_u64(rows);
   acc = warp_sum_u64(acc);
