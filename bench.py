@@ -413,7 +413,7 @@ def run_ours(args, w, rank, world, local_rank):
         reps = 10
         m0.record(stream)
         for _ in range(reps):
-            fwpkm.addressing_metrics(idx, w.N, mwin, workspace=mws, stream=stream)
+            fwpkm.addressing_metrics(idx, w.N, mwin, workspace=mws, stream=stream, out=(met, mcnt))
         m1.record(stream)
         torch.cuda.synchronize()
         mms = m0.elapsed_time(m1) / reps

@@ -156,17 +156,24 @@ def metrics_workspace_size(num_mem: int, T: int, N: int, window: int) -> int:
     return out.value
 
 
-def addressing_metrics(idx, N: int, window: int = 32768, workspace=None, stream=None):
+def addressing_metrics(idx, N: int, window: int = 32768, workspace=None, stream=None, out=None):
     """Addressing metrics of selections idx (int32 CUDA tensor [M][T][k]) per window of tokens.
 
     Returns (metrics fp64 [M][W][3]: coverage, collision rate, KLD; counts int64 [M][W][4]:
-    rows accessed, accesses, competitive accesses, invalid entries), W = ceil(T / window).
+    rows accessed, accesses, competitive accesses, invalid entries), W = ceil(T / window);
+    `out` = (metrics, counts) tensors of those shapes to fill instead of new ones.
     """
     import torch
     M, T, k = idx.shape
     W = (T + window - 1) // window
-    met = torch.zeros(M, W, 3, dtype=torch.float64, device=idx.device)
-    cnt = torch.zeros(M, W, 4, dtype=torch.int64, device=idx.device)
+    if out is None:
+        met = torch.zeros(M, W, 3, dtype=torch.float64, device=idx.device)
+        cnt = torch.zeros(M, W, 4, dtype=torch.int64, device=idx.device)
+    else:
+        met, cnt = out
+        if tuple(met.shape) != (M, W, 3) or tuple(cnt.shape) != (M, W, 4) or met.dtype != torch.float64 \
+                or cnt.dtype != torch.int64 or not (met.is_contiguous() and cnt.is_contiguous()):
+            raise ValueError("out must be contiguous fp64 [M][W][3] and int64 [M][W][4] tensors")
     if workspace is None:
         workspace = torch.empty(metrics_workspace_size(M, T, N, window), dtype=torch.uint8, device=idx.device)
     _check(lib().fwpkm_addressing_metrics(_ptr(idx), M, T, k, N, window, _ptr(workspace), workspace.numel(),

@@ -105,3 +105,14 @@ def test_metrics_workspace_size_and_validation(lib):
     assert so.fwpkm_addressing_metrics(fake, 1, 16, 4, 64, 8, C.c_void_p((1 << 20) + 16), 1 << 20, fake, None,
                                        None) == lib.ERR_INVALID_ARG  # workspace not 256-byte aligned
     assert so.fwpkm_addressing_metrics(fake, 1, 16, 4, 64, 8, fake, 64, fake, None, None) == lib.ERR_WORKSPACE
+
+
+def test_metrics_binding_checks_given_outputs(lib):
+    import torch
+    idx = torch.zeros(2, 10, 4, dtype=torch.int32)
+    bad = (torch.zeros(2, 1, 3, dtype=torch.float32), torch.zeros(2, 1, 4, dtype=torch.int64))
+    with pytest.raises(ValueError):
+        lib.addressing_metrics(idx, 64, 16, workspace=torch.zeros(1), out=bad)
+    bad = (torch.zeros(2, 2, 3, dtype=torch.float64), torch.zeros(2, 2, 4, dtype=torch.int64))  # W = 1
+    with pytest.raises(ValueError):
+        lib.addressing_metrics(idx, 64, 16, workspace=torch.zeros(1), out=bad)
