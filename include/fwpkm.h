@@ -254,8 +254,9 @@ fwpkm_status fwpkm_layer_sync(fwpkm_layer* L, void* stream);
 void fwpkm_layer_destroy(fwpkm_layer* L);
 
 /* Copy the slot indices and softmax weights that the most recent call computed for
- * tokens [0, T) of every memory (final pass of fwpkm_run_sequence, or the chunk of
- * fwpkm_forward_chunk with T <= c_len) into idx_out [M][T][k] int32 and
+ * tokens [0, T) of every memory (final pass of fwpkm_run_sequence, the chunk of
+ * fwpkm_forward_chunk with T <= c_len, or -- after fwpkm_stream_tokens -- the positions
+ * 0..T-1 of the current or last written chunk) into idx_out [M][T][k] int32 and
  * w_out [M][T][k] fp32 (device, either nullable).  Enqueued on `stream`.  Used for
  * inspection and for comparing selections against a reference. */
 fwpkm_status fwpkm_last_addressing(fwpkm_state* st, int T, int32_t* idx_out, float* w_out, void* stream);
