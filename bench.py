@@ -33,9 +33,19 @@ from sparse_weight_memory_chunk_b200.inputs import (WORKLOADS, gen_keys, gen_lay
 BY_NAME = {w.name: (i, w) for i, w in WORKLOADS.items()}
 
 # DRAM bytes (read + write) per launch and per memory of the paper-scale kernels, from one
-# ncu capture of a 2-memory case (profiles/ has the capture and its command); a full
-# launch scales with the memories it processes.  A kernel missing here reports null.
-TRAFFIC = {}
+# ncu capture of a 2-memory case of the paper shapes (profiles/kernel_counters_paper_workload_2mem.md
+# has the capture and its command): dram__bytes_read.sum + dram__bytes_write.sum of the
+# captured launch / 2; a full launch scales with the memories it processes (each memory's
+# work is the same).  A kernel changed since that capture is missing here and reports null.
+TRAFFIC = {
+    "score": {"per_mem": (3_493_376 + 512) / 2},
+    "pbar": {"per_mem": 4_345_856 / 2},
+    "wbuild": {"per_mem": 4_244_736 / 2},
+    "address": {"per_mem": 6_880_000 / 2},
+    "topk": {"per_mem": 4_262_400 / 2},
+    "sort": {"per_mem": 107_008 / 2},
+    "write": {"per_mem": (16_262_656 + 8_704) / 2},
+}
 
 
 def parse():
