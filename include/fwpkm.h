@@ -162,6 +162,13 @@ fwpkm_status fwpkm_stream_tokens(fwpkm_state* st, const void* q, const void* v, 
  * target for the last one.  No-op when nothing is pending. */
 fwpkm_status fwpkm_stream_flush(fwpkm_state* st, void* stream);
 
+/* Tokens read by fwpkm_stream_tokens and not yet written (0 .. cfg.chunk), host-only.
+ * Checkpoint/resume of a token-at-a-time sequence: save K1, K2, V (the caller's tensors)
+ * after the last write together with the inputs of the pending tokens; on resume, feed
+ * those tokens again -- the reads depend only on the saved state, so the outputs and the
+ * staged chunk come back bit for bit. */
+fwpkm_status fwpkm_stream_pending(const fwpkm_state* st, int* n_pending);
+
 /* One whole chunk step -- the read of fwpkm_forward_chunk followed by the write (and
  * key step) of fwpkm_write_chunk -- that allocates nothing and needs no workspace.
  * The paper has no counterpart: this exists for callers that cannot allocate device

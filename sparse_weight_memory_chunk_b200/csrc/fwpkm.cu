@@ -454,6 +454,7 @@ static fwpkm_status peek_status(fwpkm_state* st) {
 
 fwpkm_status fwpkm_forward_chunk(fwpkm_state* st, const void* q, const void* v, const float* g, int c_len,
                                  int seq_stride, float* o, int32_t* idx_out, float* w_out, void* stream) {
+  NvtxRange nvtx_range("fwpkm_forward_chunk");
   if (!st || !q || !v || !g || !o) return FWPKM_ERR_INVALID_ARG;
   const Dims& d = st->dm;
   if (c_len < 1 || c_len > d.C || c_len > st->wk.max_T || seq_stride < c_len) return FWPKM_ERR_INVALID_ARG;
@@ -483,6 +484,7 @@ fwpkm_status fwpkm_forward_chunk(fwpkm_state* st, const void* q, const void* v, 
 }
 
 fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream) {
+  NvtxRange nvtx_range("fwpkm_write_chunk");
   if (!st) return FWPKM_ERR_INVALID_ARG;
   if (!st->pending) return FWPKM_ERR_STATE;
   if (v_next && !aligned(v_next, 4)) return FWPKM_ERR_INVALID_ARG;
@@ -567,6 +569,7 @@ static void stream_write(fwpkm_state* st, bool has_next, cudaStream_t s) {
 
 fwpkm_status fwpkm_stream_tokens(fwpkm_state* st, const void* q, const void* v, const float* g, int n_tok,
                                  int seq_stride, float* o, void* stream) {
+  NvtxRange nvtx_range("fwpkm_stream_tokens");
   if (!st || !q || !v || !g || !o) return FWPKM_ERR_INVALID_ARG;
   const Dims& d = st->dm;
   if (n_tok < 1 || seq_stride < n_tok) return FWPKM_ERR_INVALID_ARG;
@@ -607,7 +610,14 @@ fwpkm_status fwpkm_stream_tokens(fwpkm_state* st, const void* q, const void* v, 
   return last_cuda();
 }
 
+fwpkm_status fwpkm_stream_pending(const fwpkm_state* st, int* n_pending) {
+  if (!st || !n_pending) return FWPKM_ERR_INVALID_ARG;
+  *n_pending = st->spos;
+  return FWPKM_OK;
+}
+
 fwpkm_status fwpkm_stream_flush(fwpkm_state* st, void* stream) {
+  NvtxRange nvtx_range("fwpkm_stream_flush");
   if (!st) return FWPKM_ERR_INVALID_ARG;
   if (st->pending) return FWPKM_ERR_STATE;
   fwpkm_status ps = peek_status(st);
@@ -777,6 +787,7 @@ static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, cons
 
 fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, const float* g, int T,
                                 int n_iter, float* o, void* stream) {
+  NvtxRange nvtx_range("fwpkm_run_sequence");
   if (!st) return FWPKM_ERR_INVALID_ARG;
   if (T == 0) return FWPKM_OK;
   if (!q || !v || !g || !o || T < 0 || T > st->wk.max_T || n_iter < 1) return FWPKM_ERR_INVALID_ARG;
@@ -850,6 +861,7 @@ fwpkm_status fwpkm_last_addressing(fwpkm_state* st, int T, int32_t* idx_out, flo
 }
 
 fwpkm_status fwpkm_sync(fwpkm_state* st, void* stream) {
+  NvtxRange nvtx_range("fwpkm_sync");
   if (!st) return FWPKM_ERR_INVALID_ARG;
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return last_cuda() == FWPKM_OK ? FWPKM_ERR_CUDA : FWPKM_ERR_CUDA;
   int h = 0;

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "fwpkm.h"
 
 namespace fwpkm {
@@ -194,6 +196,15 @@ bool raise_smem_limit(const void* kern, size_t bytes);
 // finishes (programmatic stream serialization).  Every kernel launched this way calls
 // pdl_wait() before it touches memory that an earlier kernel writes, so the overlap
 // covers only its launch and set-up.
+// An NVTX range named after the C-ABI call that opens it, for the Nsight tools' timelines
+// (a no-op when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Adds kernel launches made outside a state's schedule (layer projections, metrics) to
 // the count fwpkm_launch_count() reports.
 void count_launches(int n);

@@ -224,6 +224,7 @@ fwpkm_status fwpkm_layer_sync(fwpkm_layer* L, void* stream) {
 void fwpkm_layer_destroy(fwpkm_layer* L) { delete L; }
 
 fwpkm_status fwpkm_layer_set_params(fwpkm_layer* L, const fwpkm_layer_params* p, void* stream) {
+  NvtxRange nvtx_range("fwpkm_layer_set_params");
   if (!L || !p || !p->W_q || !p->W_v || !p->w_g || !p->W_o) return FWPKM_ERR_INVALID_ARG;
   const fwpkm_layer_config& c = L->cfg;
   cudaStream_t s = (cudaStream_t)stream;
@@ -252,6 +253,7 @@ fwpkm_status fwpkm_layer_set_params(fwpkm_layer* L, const fwpkm_layer_params* p,
 }
 
 fwpkm_status fwpkm_layer_in(fwpkm_layer* L, const void* h, int rows, void* q, void* v, float* g, void* stream) {
+  NvtxRange nvtx_range("fwpkm_layer_in");
   if (!L) return FWPKM_ERR_INVALID_ARG;
   if (rows == 0) return FWPKM_OK;
   const fwpkm_layer_config& c = L->cfg;
@@ -281,6 +283,7 @@ fwpkm_status fwpkm_layer_in(fwpkm_layer* L, const void* h, int rows, void* q, vo
 }
 
 fwpkm_status fwpkm_layer_out(fwpkm_layer* L, const float* o, int rows, void* o_out, void* stream) {
+  NvtxRange nvtx_range("fwpkm_layer_out");
   if (!L) return FWPKM_ERR_INVALID_ARG;
   if (rows == 0) return FWPKM_OK;
   const fwpkm_layer_config& c = L->cfg;

@@ -219,6 +219,7 @@ fwpkm_status fwpkm_metrics_workspace_size(int num_mem, int T, int N, int window,
 fwpkm_status fwpkm_addressing_metrics(const int32_t* idx, int num_mem, int T, int k, int N, int window,
                                       void* workspace, size_t ws_bytes, double* metrics, int64_t* counts,
                                       void* stream) {
+  NvtxRange nvtx_range("fwpkm_addressing_metrics");
   if (num_mem < 1 || T < 0 || k < 1 || N < 1 || window < 1) return FWPKM_ERR_INVALID_ARG;
   if (T == 0) return FWPKM_OK;
   if (!idx || !workspace || !metrics) return FWPKM_ERR_INVALID_ARG;

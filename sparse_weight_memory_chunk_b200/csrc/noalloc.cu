@@ -54,6 +54,7 @@ extern "C" fwpkm_status fwpkm_chunk_step_noalloc(const fwpkm_config* cfg, float*
                                                  const void* q, const void* v, const float* g,
                                                  const void* v_next, int c_len, int seq_stride, float* o,
                                                  void* stream) {
+  NvtxRange nvtx_range("fwpkm_chunk_step_noalloc");
   if (!cfg || !K1 || !K2 || !V || !q || !v || !g || !o) return FWPKM_ERR_INVALID_ARG;
   size_t need = 0;
   fwpkm_status s = fwpkm_workspace_size(cfg, cfg->chunk, &need);  // validates cfg

@@ -81,6 +81,7 @@ def lib():
                                          ctypes.c_int),
             "fwpkm_stream_tokens": ([_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P], ctypes.c_int),
             "fwpkm_stream_flush": ([_P, _P], ctypes.c_int),
+            "fwpkm_stream_pending": ([_P, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
             "fwpkm_sync": ([_P, _P], ctypes.c_int),
             "fwpkm_destroy_state": ([_P], None),
             "fwpkm_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -226,6 +227,12 @@ class State:
     def stream_flush(self, stream=None):
         """Write the pending tokens of a token-at-a-time sequence (no lookahead for the last)."""
         _check(lib().fwpkm_stream_flush(self.handle, _stream(stream)), "stream_flush")
+
+    def stream_pending(self) -> int:
+        """Tokens read by stream_tokens and not yet written (host-side count)."""
+        n = ctypes.c_int(0)
+        _check(lib().fwpkm_stream_pending(self.handle, ctypes.byref(n)), "stream_pending")
+        return n.value
 
     def last_addressing(self, T, idx_out=None, w_out=None, stream=None):
         _check(lib().fwpkm_last_addressing(self.handle, T, _ptr(idx_out), _ptr(w_out), _stream(stream)),

@@ -66,6 +66,7 @@ def test_one_token_at_a_time_and_state_rules():
     st.stream_flush()  # nothing pending: no-op
     for t in range(w.T):
         st.stream_tokens(dev["q"][:, t:], dev["v"][:, t:], dev["g"][:, t:], o[:, t:], n_tok=1, seq_stride=w.T)
+        assert st.stream_pending() == t % w.C + 1
         if t == 5:
             with pytest.raises(fwpkm.FwpkmError) as e:  # chunk mode while tokens are pending
                 st.run_sequence(dev["q"], dev["v"], dev["g"], o)
@@ -74,6 +75,7 @@ def test_one_token_at_a_time_and_state_rules():
                 st.forward_chunk(dev["q"], dev["v"], dev["g"], o, 4, seq_stride=w.T)
             assert e.value.status == fwpkm.ERR_STATE
     st.stream_flush()
+    assert st.stream_pending() == 0
     st.sync()
     assert torch.equal(o, o_ref)
     assert torch.equal(dev["V"], dev_ref["V"]) and torch.equal(dev["K1"], dev_ref["K1"])
@@ -81,6 +83,29 @@ def test_one_token_at_a_time_and_state_rules():
     o2 = torch.zeros_like(o)
     st.run_sequence(dev["q"], dev["v"], dev["g"], o2, T=w.C)
     st.sync()
+
+
+def test_resume_from_a_checkpoint_mid_chunk():
+    w, data, gcfg, _ = make_case("mid_key")
+    o_ref, dev_ref = reference(w, data, gcfg)
+    st, dev = device_state(w, data, gcfg, w.C)
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    t0 = w.C + 37  # inside the second chunk
+    st.stream_tokens(dev["q"], dev["v"], dev["g"], o, n_tok=t0, seq_stride=w.T)
+    pend = st.stream_pending()
+    assert pend == 37
+    st.sync()
+    ck = {key: dev[key].clone() for key in ("K1", "K2", "V")}  # the state after the last write
+    # a new handle from the checkpoint: the pending tokens again, then the rest
+    st2 = fwpkm.State(gcfg, ck["K1"], ck["K2"], ck["V"], w.C)
+    o2 = torch.zeros_like(o)
+    a = t0 - pend
+    st2.stream_tokens(dev["q"][:, a:], dev["v"][:, a:], dev["g"][:, a:], o2[:, a:], n_tok=w.T - a, seq_stride=w.T)
+    st2.stream_flush()
+    st2.sync()
+    assert torch.equal(o2[:, a:], o_ref[:, a:])
+    for key in ("K1", "K2", "V"):
+        assert torch.equal(ck[key], dev_ref[key]), key
 
 
 def test_stream_needs_a_chunk_of_workspace():
