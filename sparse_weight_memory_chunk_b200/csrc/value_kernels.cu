@@ -395,6 +395,8 @@ struct StageJobs {
 };
 
 __global__ void __launch_bounds__(256) stage_kernel(StageJobs jobs) {
+  pdl_wait();  // the previous chunk's write may still read the staging rows
+  pdl_trigger();
   const StageJob& J = jobs.j[blockIdx.z];
   if (J.src == nullptr) return;
   const int m = blockIdx.y;
