@@ -243,6 +243,42 @@ def test_key_step_is_entropy_gradient(seed):
         np.testing.assert_allclose(got, G, rtol=2e-5, atol=2e-6 * np.abs(G).max())
 
 
+@pytest.mark.parametrize("seed", [4, 5])
+def test_key_step_factors_through_inverse_square_distances(seed):
+    """The key gradient rebuilt from u = (eps + D)^-2, which does not depend on the usage
+    marginals, and the small per-token factors 1/Z_t and L_t/Z_t:
+    dL/dK[b] = (2/C) (lp[b] sum_t u q_t / Z_t - sum_t u L_t q_t / Z_t
+                      - (lp[b] sum_t u / Z_t - sum_t u L_t / Z_t) K[b]),
+    at a size the finite-difference check cannot afford (n = 64, C = 40)."""
+    rng = np.random.default_rng(seed)
+    n, h, C, eps, lr = 64, 16, 40, 1e-3, 3.0
+    q = rng.standard_normal((C, 2 * h))
+    K1 = rng.standard_normal((n, h)).astype(np.float32)
+    K2 = rng.standard_normal((n, h)).astype(np.float32)
+    cfg = oracle.make_cfg(n=n, d=2 * h, d_v=2, k=4, chunk=C, eps_idw=eps, lr_key=lr, key_update=True)
+    K1n, K2n = K1.copy(), K2.copy()
+    oracle.chunk(cfg, q, rng.standard_normal((C, 2)), np.ones(C), None, K1n, K2n,
+                 np.zeros((n * n, 2), np.float32))
+    for j, (K0, Kn) in enumerate(((K1, K1n), (K2, K2n))):
+        K = K0.astype(np.float64)
+        qj = q[:, j * h:(j + 1) * h]
+        D = cdist(qj, K, "sqeuclidean")
+        Z = (1.0 / (eps + D)).sum(axis=1)
+        P = (1.0 / (eps + D)) / Z[:, None]
+        lp = np.log(P.mean(axis=0))
+        L = P @ lp
+        u = (eps + D) ** -2
+        A1 = u.T @ (qj / Z[:, None])
+        A2 = u.T @ (qj * (L / Z)[:, None])
+        s1 = u.T @ (1.0 / Z)
+        s2 = u.T @ (L / Z)
+        grad = (2.0 / C) * (lp[:, None] * A1 - A2 - (lp * s1 - s2)[:, None] * K)
+        step = Kn.astype(np.float64) - K  # the oracle's update, stored in fp32
+        ulp = np.spacing(np.abs(Kn)).astype(np.float64)
+        assert np.abs(lr * grad).max() > 1e3 * ulp.max()  # a step far above the storage rounding
+        assert np.all(np.abs(step + lr * grad) <= ulp)
+
+
 def test_uniform_usage_gives_zero_key_step():
     """Two tokens mirrored about symmetric keys: pbar is uniform, so the entropy is maximal."""
     cfg = oracle.make_cfg(n=2, d=2, d_v=2, k=1, chunk=2, key_update=True, lr_key=10.0)
