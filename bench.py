@@ -369,7 +369,7 @@ def run_ours(args, w, rank, world, local_rank):
         "address": ("tensor", 2 * w.n * w.d * tok),
         "topk": ("hbm", 2 * w.n * 4 * tok),                       # distance rows read
         "pbar": ("hbm", 2 * w.n * 4 * tok),                       # distance rows read
-        "wbuild": ("hbm", 2 * w.n * 4 * tok * 2 + 2 * w.n * 2 * 3 * tok),  # rows read twice, 3 bf16 pieces written
+        "wbuild": ("hbm", 2 * w.n * 4 * tok * 2 + 2 * w.n * 2 * 2 * tok),  # rows read twice, 2 bf16 pieces written
         "sort": ("hbm", w.k * tok * (4 + 8)),                      # slots read, pair keys written
         "cartesian": ("alu", cand * 2 * tok),                      # one add + one compare per candidate
     }
