@@ -33,12 +33,14 @@ import numpy as np
 
 
 def window_count(T: int, window: int) -> int:
-    """Windows of `window` tokens covering T tokens (the last one may be shorter)."""
+    """Windows of `window` tokens covering T tokens (the last one may be shorter; §D.3
+    measures every 32K tokens)."""
     return (T + window - 1) // window
 
 
 def addressing_metrics(idx, N: int, window: int):
-    """Metrics of every (memory, window).
+    """Metrics of every (memory, window), paperlayer §D.3: row contributions c_i per window,
+    then coverage, collision rate and KL divergence from uniform slot use.
 
     idx: int array [M][T][k] of selected slots.  Returns (metrics, counts):
       metrics fp64 [M][W][3]: coverage, collision rate, KLD;

@@ -26,7 +26,8 @@ from . import chunk, read_values, select, subkey_dist
 
 
 def read_token(cfg, q_t, v_t, g_t, K1, K2, V):
-    """The read of one token against the state (K1, K2, V): returns (o_t, I_t, s'_t)."""
+    """The read of one token against the state (K1, K2, V) -- method steps 2-3 of the
+    rainbus summary, the scores of paperlayer §A.2: returns (o_t, I_t, s'_t)."""
     q_t = np.asarray(q_t, dtype=np.float64)
     D1 = subkey_dist(cfg, q_t[:cfg.h], K1)
     D2 = subkey_dist(cfg, q_t[cfg.h:], K2)
@@ -37,7 +38,8 @@ def read_token(cfg, q_t, v_t, g_t, K1, K2, V):
 
 def stream_sequence(cfg, q, v, g, K1, K2, V, groups):
     """Feed the tokens of one memory in arrival groups of the given sizes (summing to T),
-    then end the sequence.  K1, K2, V (fp32) are updated in place.  Returns o [T][d_v]."""
+    then end the sequence (paperlayer §A.1: pairs accumulate until a chunk is ready).
+    K1, K2, V (fp32) are updated in place.  Returns o [T][d_v]."""
     q = np.asarray(q, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     g = np.asarray(g, dtype=np.float64)
