@@ -27,8 +27,13 @@
  *     enqueues work on it and returns; results are ready when the stream is.
  *   - Calls return a status and never throw.  Argument checks run synchronously
  *     before anything is enqueued (then nothing is enqueued).  Errors detected on
- *     the device are latched in a status word returned by fwpkm_sync() and by the
- *     next call on the same state.
+ *     the device (FWPKM_ERR_TIMEOUT, FWPKM_ERR_BAD_SLOT) are latched in a device
+ *     status word and in a copy of it in pinned host memory that the kernel writes
+ *     when it detects the error.  fwpkm_sync() waits for the stream and returns the
+ *     latched error, clearing it.  Every other call on the same handle first reads
+ *     the host copy without waiting: once the error has reached it, the call returns
+ *     that error and enqueues nothing, until fwpkm_sync() clears it.  (A call made
+ *     while the failing kernel is still running cannot know yet: it returns OK.)
  *   - Results are deterministic: the same inputs give bit-identical outputs.
  */
 #ifndef FWPKM_H
@@ -48,7 +53,8 @@ typedef enum {
   FWPKM_ERR_WORKSPACE = -3,   /* workspace smaller than fwpkm_workspace_size()         */
   FWPKM_ERR_CUDA = -4,        /* a CUDA runtime call failed                            */
   FWPKM_ERR_TIMEOUT = -5,     /* a bounded device-side wait gave up                    */
-  FWPKM_ERR_STATE = -6        /* call out of order (write_chunk without forward_chunk) */
+  FWPKM_ERR_STATE = -6,      /* call out of order (write_chunk without forward_chunk) */
+  FWPKM_ERR_BAD_SLOT = -7     /* the write met a slot index outside [0, n*n); that row was skipped */
 } fwpkm_status;
 
 typedef enum { FWPKM_F32 = 0, FWPKM_BF16 = 1 } fwpkm_dtype;
@@ -81,7 +87,8 @@ typedef struct {
 } fwpkm_config;
 
 /* Opaque host-side handle.  It records the caller's state pointers and the carved
- * workspace; it owns no device memory (only CUDA streams/events/graphs). */
+ * workspace; it owns no device memory (only CUDA streams/events/graphs and one word of
+ * pinned host memory, the host copy of the status word). */
 typedef struct fwpkm_state fwpkm_state;
 
 /* Bytes of device workspace needed for sequences of up to max_T tokens.
@@ -172,17 +179,20 @@ fwpkm_status fwpkm_stream_pending(const fwpkm_state* st, int* n_pending);
 /* One whole chunk step -- the read of fwpkm_forward_chunk followed by the write (and
  * key step) of fwpkm_write_chunk -- that allocates nothing and needs no workspace.
  * The paper has no counterpart: this exists for callers that cannot allocate device
- * memory (host callbacks, loops under a no-allocation rule, plugins whose host owns
- * the allocator, code that must not change the device memory map).  Arguments mean
- * what they mean in fwpkm_forward_chunk / fwpkm_write_chunk (K1, K2, V are the
- * caller's state, updated in place; v_next NULL = the chunk ends the sequence).
+ * memory (loops under a no-allocation rule, plugins whose host owns the allocator, code
+ * that must not change the device memory map).  It makes CUDA calls and launches
+ * kernels, so it must not be called from a CUDA host function (stream callback).
+ * Arguments mean what they mean in fwpkm_forward_chunk / fwpkm_write_chunk (K1, K2, V
+ * are the caller's state, updated in place; v_next NULL = the chunk ends the sequence).
+ * It runs the CUDA-core kernels of the chunk step, whatever the shape.
  * Scratch is a fixed 16 MiB array inside the library that every GPU loading the
- * library keeps until exit; shapes whose scratch for one chunk (fwpkm_workspace_size(cfg,
- * cfg->chunk) less the staging rows of token-at-a-time inference) exceeds it are rejected
- * with FWPKM_ERR_UNSUPPORTED.  The first call on a device
- * looks up that array's device address (make it before any stream capture).  All
- * calls share the array: calls that overlap on the GPU race and must be serialised
- * by the caller.  Device-side errors are not reported by this entry point. */
+ * library keeps until exit; shapes whose scratch for one chunk on the CUDA-core kernels
+ * (the workspace of one chunk without the tensor-core buffers and the staging rows of
+ * token-at-a-time inference) exceeds it are rejected with FWPKM_ERR_UNSUPPORTED.  The
+ * first call on a device looks up that array's device address (make it before any
+ * stream capture).  All calls share the array: calls that overlap on the GPU race and
+ * must be serialised by the caller.  Device-side errors are not reported by this entry
+ * point. */
 fwpkm_status fwpkm_chunk_step_noalloc(const fwpkm_config* cfg, float* K1, float* K2, float* V,
                                       const void* q, const void* v, const float* g, const void* v_next,
                                       int c_len, int seq_stride, float* o, void* stream);
@@ -254,11 +264,33 @@ fwpkm_status fwpkm_layer_in(fwpkm_layer* L, const void* h, int rows, void* q, vo
 fwpkm_status fwpkm_layer_out(fwpkm_layer* L, const float* o, int rows, void* o_out, void* stream);
 
 /* Wait for `stream` and return the handle's latched device status (a GEMM wait
- * that timed out gives FWPKM_ERR_TIMEOUT), clearing it. */
+ * that timed out gives FWPKM_ERR_TIMEOUT), clearing it.  As for fwpkm_state, the other
+ * calls on the handle return a latched error once its host copy shows it. */
 fwpkm_status fwpkm_layer_sync(fwpkm_layer* L, void* stream);
 
 /* Release the handle (the workspace is the caller's). */
 void fwpkm_layer_destroy(fwpkm_layer* L);
+
+/* The whole FwPKM layer ("快速权重积键值记忆 Fast-weight Product Key Memory" (rainbus
+ * summary), method steps 1-5) for M = cfg.num_mem sequences of one head each: method
+ * step 1 (fwpkm_layer_in on the M*T rows of h), the chunk-sequential memory loop over
+ * T tokens with n_iter passes (fwpkm_run_sequence), then the output projection of method
+ * step 3 (fwpkm_layer_out) on the final pass's o.  One call, stream-ordered.
+ *   L, st    the projections and the memory state; they must agree on d, d_v and the q/v
+ *            dtype, with M*T <= the layer's max_rows and T <= the state's max_T
+ *            (else FWPKM_ERR_INVALID_ARG).
+ *   h        device bf16 [M][T][d_model] (16-byte aligned); o_out device bf16
+ *            [M][T][d_model] (16-byte aligned).
+ *   scratch  device, 256-byte aligned, scratch_bytes >= fwpkm_run_layer_scratch_size()
+ *            (else FWPKM_ERR_WORKSPACE).  It receives, in this order, each part starting
+ *            on a 256-byte boundary: q [M][T][d] and v [M][T][d_v] (q/v dtype), g [M][T]
+ *            fp32 and o [M][T][d_v] fp32 -- the memory's inputs and output, readable once
+ *            the stream has passed the call.
+ * T = 0 is a no-op.  Errors are those of the three calls it makes (the first failing
+ * one is returned; nothing after it is enqueued). */
+fwpkm_status fwpkm_run_layer_scratch_size(const fwpkm_config* cfg, int T, size_t* bytes);
+fwpkm_status fwpkm_run_layer(fwpkm_layer* L, fwpkm_state* st, const void* h, int T, int n_iter, void* scratch,
+                             size_t scratch_bytes, void* o_out, void* stream);
 
 /* Copy the slot indices and softmax weights that the most recent call computed for
  * tokens [0, T) of every memory (final pass of fwpkm_run_sequence, the chunk of
@@ -305,8 +337,18 @@ fwpkm_status fwpkm_addressing_metrics(const int32_t* idx, int num_mem, int T, in
                                       void* stream);
 
 /* Wait for `stream` and return the latched device status (FWPKM_OK,
- * FWPKM_ERR_TIMEOUT, ...), clearing it. */
+ * FWPKM_ERR_TIMEOUT, FWPKM_ERR_BAD_SLOT), clearing it (device word and host copy). */
 fwpkm_status fwpkm_sync(fwpkm_state* st, void* stream);
+
+/* Test hook of the timeout path (no counterpart in the paper).  Each of the next
+ * `n_launches` tensor-core kernel launches made by this process (scoring, key step,
+ * projections) has its MMA-issuing thread first wait on a barrier that nothing
+ * completes.  That wait is bounded like every other wait in those kernels (0.2 s): it
+ * runs out, the kernel takes its abort path (in-flight copies drained, tensor memory
+ * freed, no further work) and latches FWPKM_ERR_TIMEOUT in the handle's status word.
+ * Nothing faults and the context stays usable.  n_launches = 0 cancels.  Launches
+ * captured into a CUDA graph keep the setting they were captured with. */
+void fwpkm_test_stall_waits(int n_launches);
 
 /* Release the handle (streams, events, graphs).  Caller buffers are untouched. */
 void fwpkm_destroy_state(fwpkm_state* st);

@@ -67,7 +67,7 @@ def _load():
         _lib.orc_chunk.argtypes = [ctypes.POINTER(Cfg), ctypes.c_int] + [P] * 12
         _lib.orc_run_sequence.argtypes = [ctypes.POINTER(Cfg), ctypes.c_int, ctypes.c_int] + [P] * 9
         _lib.orc_run_sequence_multi.argtypes = ([ctypes.POINTER(Cfg), ctypes.c_int, ctypes.c_int,
-                                                 ctypes.c_int] + [P] * 7 + [ctypes.c_int])
+                                                 ctypes.c_int] + [P] * 8 + [ctypes.c_int])
         _lib.orc_run_sequence_multi.restype = ctypes.c_int
     return _lib
 
@@ -147,13 +147,17 @@ def run_sequence(cfg: Cfg, q, v, g, K1, K2, V, n_iter=1):
     return o, I, w
 
 
-def run_sequence_multi(cfg: Cfg, q, v, g, K1, K2, V, n_iter=1, nthreads=1):
-    """M independent memories ([M][T][..] inputs, [M][..] state) on ``nthreads`` threads.
+def run_sequence_multi(cfg: Cfg, q, v, g, K1, K2, V, n_iter=1, nthreads=1, with_slots=False):
+    """M independent memories ([M][T][..] inputs, [M][..] state) on ``nthreads`` threads
+    (with more threads than memories, each memory splits its chunks' read phase over
+    nthreads // M threads).
 
-    Returns (o [M][T][d_v], threads used)."""
+    Returns (o [M][T][d_v], threads used), plus the final pass's slots I [M][T][k] when
+    ``with_slots``."""
     q = _f64(q); v = _f64(v); g = _f64(g)
     M, T = q.shape[0], q.shape[1]
     o = np.empty((M, T, cfg.d_v))
+    I = np.empty((M, T, cfg.k), np.int32) if with_slots else None
     used = _load().orc_run_sequence_multi(ctypes.byref(cfg), M, T, n_iter, _p(q), _p(v), _p(g),
-                                          _p(_f32(K1)), _p(_f32(K2)), _p(_f32(V)), _p(o), nthreads)
-    return o, used
+                                          _p(_f32(K1)), _p(_f32(K2)), _p(_f32(V)), _p(o), _p(I), nthreads)
+    return (o, used, I) if with_slots else (o, used)

@@ -193,9 +193,40 @@ static int pair_cmp(const void* x, const void* y) {
  *   forced [len][k] and force_mask [len] (both nullable): tokens whose mask is
  *   non-zero use the given slot list instead of the computed one.
  * ------------------------------------------------------------------------- */
-void orc_chunk(const orc_cfg* c, int len, const double* q, const double* v, const double* g,
-               const double* v_next, float* K1, float* K2, float* V, double* o, int32_t* I_out,
-               double* w_out, const int32_t* forced, const int32_t* force_mask) {
+/* Read phase of tokens [t0, t1) of a chunk ([R] steps 2-3): every token against the
+ * frozen state.  Tokens are independent, so any split of the range gives the same values. */
+typedef struct {
+  const orc_cfg* c;
+  int t0, t1;
+  const double *q, *v, *g;
+  const float *K1, *K2, *V;
+  double *D1, *D2, *S, *w, *vhat, *o;
+  int32_t* I;
+  const int32_t *forced, *force_mask;
+} orc_read_job;
+
+static void* orc_read_range(void* arg) {
+  const orc_read_job* j = (const orc_read_job*)arg;
+  const orc_cfg* c = j->c;
+  const int n = c->n, h = c->h, dv = c->d_v, k = c->k, d = 2 * h;
+  for (int t = j->t0; t < j->t1; ++t) {
+    orc_subkey_dist(c, j->q + (size_t)t * d, j->K1, j->D1 + (size_t)t * n);
+    orc_subkey_dist(c, j->q + (size_t)t * d + h, j->K2, j->D2 + (size_t)t * n);
+    const int32_t* f = (j->forced && j->force_mask && j->force_mask[t]) ? j->forced + (size_t)t * k : NULL;
+    orc_select(c, j->D1 + (size_t)t * n, j->D2 + (size_t)t * n, f, j->I + (size_t)t * k, j->S + (size_t)t * k,
+               j->w + (size_t)t * k);
+    orc_read_values(c, j->I + (size_t)t * k, j->w + (size_t)t * k, j->V, j->vhat + (size_t)t * dv);
+    for (int e = 0; e < dv; ++e)
+      j->o[(size_t)t * dv + e] = j->g[t] * j->vhat[(size_t)t * dv + e] + (1.0 - j->g[t]) * j->v[(size_t)t * dv + e];
+  }
+  return NULL;
+}
+
+/* One chunk with its read phase split over `read_threads` threads (token ranges); the
+ * write and the key step follow on the calling thread.  orc_chunk is the one-thread case. */
+static void orc_chunk_threads(const orc_cfg* c, int len, const double* q, const double* v, const double* g,
+                              const double* v_next, float* K1, float* K2, float* V, double* o, int32_t* I_out,
+                              double* w_out, const int32_t* forced, const int32_t* force_mask, int read_threads) {
   const int n = c->n, h = c->h, dv = c->d_v, k = c->k, d = 2 * h;
   double* D1 = (double*)malloc(sizeof(double) * (size_t)len * n);
   double* D2 = (double*)malloc(sizeof(double) * (size_t)len * n);
@@ -205,15 +236,21 @@ void orc_chunk(const orc_cfg* c, int len, const double* q, const double* v, cons
   double* vhat = (double*)malloc(sizeof(double) * (size_t)len * dv);
 
   /* ---- read phase: every token of the chunk against the frozen state ---- */
-  for (int t = 0; t < len; ++t) {
-    orc_subkey_dist(c, q + (size_t)t * d, K1, D1 + (size_t)t * n);
-    orc_subkey_dist(c, q + (size_t)t * d + h, K2, D2 + (size_t)t * n);
-    const int32_t* f = (forced && force_mask && force_mask[t]) ? forced + (size_t)t * k : NULL;
-    orc_select(c, D1 + (size_t)t * n, D2 + (size_t)t * n, f, I + (size_t)t * k, S + (size_t)t * k,
-               w + (size_t)t * k);
-    orc_read_values(c, I + (size_t)t * k, w + (size_t)t * k, V, vhat + (size_t)t * dv);
-    for (int e = 0; e < dv; ++e)
-      o[(size_t)t * dv + e] = g[t] * vhat[(size_t)t * dv + e] + (1.0 - g[t]) * v[(size_t)t * dv + e];
+  if (read_threads < 1) read_threads = 1;
+  if (read_threads > len) read_threads = len;
+  {
+    orc_read_job* jobs = (orc_read_job*)malloc(sizeof(orc_read_job) * (size_t)read_threads);
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)read_threads);
+    for (int i = 0; i < read_threads; ++i) {
+      orc_read_job jj = {c, (int)((long long)i * len / read_threads), (int)((long long)(i + 1) * len / read_threads),
+                         q, v, g, K1, K2, V, D1, D2, S, w, vhat, o, I, forced, force_mask};
+      jobs[i] = jj;
+    }
+    for (int i = 1; i < read_threads; ++i) pthread_create(&th[i], NULL, orc_read_range, &jobs[i]);
+    orc_read_range(&jobs[0]);
+    for (int i = 1; i < read_threads; ++i) pthread_join(th[i], NULL);
+    free(jobs);
+    free(th);
   }
   if (I_out) memcpy(I_out, I, sizeof(int32_t) * (size_t)len * k);
   if (w_out) memcpy(w_out, w, sizeof(double) * (size_t)len * k);
@@ -316,62 +353,79 @@ void orc_chunk(const orc_cfg* c, int len, const double* q, const double* v, cons
   free(r); free(tau); free(is_pair); free(pairs); free(G);
 }
 
+void orc_chunk(const orc_cfg* c, int len, const double* q, const double* v, const double* g,
+               const double* v_next, float* K1, float* K2, float* V, double* o, int32_t* I_out,
+               double* w_out, const int32_t* forced, const int32_t* force_mask) {
+  orc_chunk_threads(c, len, q, v, g, v_next, K1, K2, V, o, I_out, w_out, forced, force_mask, 1);
+}
+
 /* ---------------------------------------------------------------------------
  * Whole sequence of one memory, n_iter passes over the same input
  * ([P] §3.1 chunk-sequential schedule; [R] 技术新颖性 iterative memorization).
  * The state carries across chunks and passes.  o, I, w hold the final pass.
  * ------------------------------------------------------------------------- */
-void orc_run_sequence(const orc_cfg* c, int T, int n_iter, const double* q, const double* v,
-                      const double* g, float* K1, float* K2, float* V, double* o, int32_t* I,
-                      double* w) {
+static void orc_run_sequence_threads(const orc_cfg* c, int T, int n_iter, const double* q, const double* v,
+                                     const double* g, float* K1, float* K2, float* V, double* o, int32_t* I,
+                                     double* w, int read_threads) {
   const int d = 2 * c->h, dv = c->d_v, k = c->k;
   for (int pass = 0; pass < n_iter; ++pass) {
     for (int t0 = 0; t0 < T; t0 += c->chunk) {
       int len = T - t0 < c->chunk ? T - t0 : c->chunk;
       const double* v_next = (t0 + len < T) ? v + (size_t)(t0 + len) * dv : NULL;
-      orc_chunk(c, len, q + (size_t)t0 * d, v + (size_t)t0 * dv, g + t0, v_next, K1, K2, V,
-                o + (size_t)t0 * dv, I ? I + (size_t)t0 * k : NULL, w ? w + (size_t)t0 * k : NULL,
-                NULL, NULL);
+      orc_chunk_threads(c, len, q + (size_t)t0 * d, v + (size_t)t0 * dv, g + t0, v_next, K1, K2, V,
+                        o + (size_t)t0 * dv, I ? I + (size_t)t0 * k : NULL, w ? w + (size_t)t0 * k : NULL,
+                        NULL, NULL, read_threads);
     }
   }
 }
 
+void orc_run_sequence(const orc_cfg* c, int T, int n_iter, const double* q, const double* v,
+                      const double* g, float* K1, float* K2, float* V, double* o, int32_t* I,
+                      double* w) {
+  orc_run_sequence_threads(c, T, n_iter, q, v, g, K1, K2, V, o, I, w, 1);
+}
+
 /* Independent memories (sequence x head) in parallel threads: nothing is shared
- * between memories, so this is the same computation as one call per memory. */
+ * between memories, so this is the same computation as one call per memory.  With more
+ * threads than memories, each memory also splits the read phase of its chunks over
+ * nthreads / M threads (token ranges).  I (nullable) receives the final pass's slots. */
 typedef struct {
   const orc_cfg* c;
-  int T, n_iter, M, nthreads, tid;
+  int T, n_iter, M, nthreads, tid, read_threads;
   const double *q, *v, *g;
   float *K1, *K2, *V;
   double* o;
+  int32_t* I;
 } orc_job;
 
 static void* orc_worker(void* arg) {
   orc_job* j = (orc_job*)arg;
   const orc_cfg* c = j->c;
-  const size_t d = 2 * (size_t)c->h, dv = (size_t)c->d_v, n = (size_t)c->n, h = (size_t)c->h;
+  const size_t d = 2 * (size_t)c->h, dv = (size_t)c->d_v, n = (size_t)c->n, h = (size_t)c->h, k = (size_t)c->k;
   for (int m = j->tid; m < j->M; m += j->nthreads) {
-    orc_run_sequence(c, j->T, j->n_iter, j->q + (size_t)m * j->T * d, j->v + (size_t)m * j->T * dv,
-                     j->g + (size_t)m * j->T, j->K1 + (size_t)m * n * h, j->K2 + (size_t)m * n * h,
-                     j->V + (size_t)m * n * n * dv, j->o + (size_t)m * j->T * dv, NULL, NULL);
+    orc_run_sequence_threads(c, j->T, j->n_iter, j->q + (size_t)m * j->T * d, j->v + (size_t)m * j->T * dv,
+                             j->g + (size_t)m * j->T, j->K1 + (size_t)m * n * h, j->K2 + (size_t)m * n * h,
+                             j->V + (size_t)m * n * n * dv, j->o + (size_t)m * j->T * dv,
+                             j->I ? j->I + (size_t)m * j->T * k : NULL, NULL, j->read_threads);
   }
   return NULL;
 }
 
 int orc_run_sequence_multi(const orc_cfg* c, int M, int T, int n_iter, const double* q,
                            const double* v, const double* g, float* K1, float* K2, float* V,
-                           double* o, int nthreads) {
+                           double* o, int32_t* I, int nthreads) {
   if (nthreads < 1) nthreads = 1;
-  if (nthreads > M) nthreads = M;
-  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * nthreads);
-  orc_job* jobs = (orc_job*)malloc(sizeof(orc_job) * nthreads);
-  for (int i = 0; i < nthreads; ++i) {
-    orc_job jj = {c, T, n_iter, M, nthreads, i, q, v, g, K1, K2, V, o};
+  const int read_threads = nthreads > M ? nthreads / M : 1;
+  const int mem_threads = nthreads > M ? M : nthreads;
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * mem_threads);
+  orc_job* jobs = (orc_job*)malloc(sizeof(orc_job) * mem_threads);
+  for (int i = 0; i < mem_threads; ++i) {
+    orc_job jj = {c, T, n_iter, M, mem_threads, i, read_threads, q, v, g, K1, K2, V, o, I};
     jobs[i] = jj;
     pthread_create(&th[i], NULL, orc_worker, &jobs[i]);
   }
-  for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+  for (int i = 0; i < mem_threads; ++i) pthread_join(th[i], NULL);
   free(th);
   free(jobs);
-  return nthreads;
+  return mem_threads * read_threads;
 }

@@ -51,6 +51,10 @@ struct fwpkm_state {
   std::vector<cudaEvent_t> ev;
   int ev_used;
   int host_error;  // a launch could not be set up (e.g. tensor map encoding failed)
+  // host copy of the device status word (pinned, mapped: kernels that latch an error
+  // store it here too, so a later call sees it without waiting for the GPU)
+  int* hstat;
+  int* hstat_dev;
   // run_sequence schedule: internal streams, dependency events and the cached graph
   // Memories are split into `groups` contiguous groups; each group runs its own three
   // chains, so one group's latency-bound kernels overlap another's.
@@ -203,6 +207,15 @@ void count_launches(int n) { g_launches += (uint64_t)n; }
 thread_local int launch_priority = 0;
 thread_local bool launch_priority_set = false;
 
+static std::atomic<int> g_test_stalls{0};
+
+int take_test_stall() {
+  int n = g_test_stalls.load();
+  while (n > 0)
+    if (g_test_stalls.compare_exchange_weak(n, n - 1)) return 1;
+  return 0;
+}
+
 int pbar_slices() {
   static const int v = [] {
     const char* e = getenv("FWPKM_PBAR_SLICES");
@@ -238,7 +251,7 @@ int addressing_window(const Dims& d, int max_T) {
   return (int)wtok;
 }
 
-size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base, bool stream_stage) {
+size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base, bool stream_stage, bool allow_tc) {
   const size_t M = d.M, k = d.k, C = d.C, n = d.n, dv = d.dv;
   const size_t T = max_T;
   const size_t nch = (T + C - 1) / C;
@@ -252,6 +265,7 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base, bool strea
   x.max_T = max_T;
   x.max_chunks = (int)nch;
   x.status = (int*)take(sizeof(int));
+  x.hstat = nullptr;  // set by the handle that owns the carve
   x.A = (int32_t*)take(4 * M * 2 * T * k);
   x.Dsv = (float*)take(4 * M * 2 * T * k);
   x.idx = (int32_t*)take(4 * M * T * k);
@@ -260,7 +274,7 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base, bool strea
   x.npairs = (int32_t*)take(4 * M * nch);
   x.resid = (float*)take(4 * M * C * dv);
   const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
-  x.tc = use_tensor_cores(d) ? 1 : 0;
+  x.tc = (allow_tc && use_tensor_cores(d)) ? 1 : 0;
   x.drows = ku ? (int)C : (x.tc ? addressing_window(d, max_T) : 0);
   // with the key step the tensor-core path keeps two chunks of distance rows in flight
   const size_t dbufs = (ku && x.tc) ? 2 : 1;
@@ -343,11 +357,14 @@ const char* fwpkm_status_string(fwpkm_status s) {
     case FWPKM_ERR_CUDA: return "CUDA error";
     case FWPKM_ERR_TIMEOUT: return "device wait timed out";
     case FWPKM_ERR_STATE: return "call out of order";
+    case FWPKM_ERR_BAD_SLOT: return "slot index out of range in the write";
   }
   return "unknown status";
 }
 
 uint64_t fwpkm_launch_count(void) { return g_launches.load(); }
+
+void fwpkm_test_stall_waits(int n_launches) { g_test_stalls.store(n_launches > 0 ? n_launches : 0); }
 
 fwpkm_status fwpkm_workspace_size(const fwpkm_config* cfg, int max_T, size_t* bytes) {
   fwpkm_status s = check_cfg(cfg);
@@ -378,6 +395,8 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
   st->ev_used = 0;
   st->host_error = 0;
   st->ev_next = 0;
+  st->hstat = nullptr;
+  st->hstat_dev = nullptr;
   for (int i = 0; i < fwpkm_state::NGRAPH; ++i) {
     st->graph_exec[i] = nullptr;
     st->graph_kernels[i] = 0;
@@ -411,20 +430,29 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
     st->prio_S = (least + greatest) / 2;
     st->prio_V = least;
   }
-  bool ok = cudaStreamCreateWithFlags(&st->sCap, cudaStreamNonBlocking) == cudaSuccess;
+  bool ok = cudaHostAlloc((void**)&st->hstat, sizeof(int), cudaHostAllocMapped) == cudaSuccess &&
+            cudaHostGetDevicePointer((void**)&st->hstat_dev, st->hstat, 0) == cudaSuccess;
+  if (ok) {
+    *(volatile int*)st->hstat = DEV_OK;
+    st->wk.hstat = st->hstat_dev;
+  }
+  st->sCap = nullptr;
+  ok = ok && cudaStreamCreateWithFlags(&st->sCap, cudaStreamNonBlocking) == cudaSuccess;
   for (int gi = 0; gi < fwpkm_state::MAX_GROUPS; ++gi) st->sK[gi] = st->sS[gi] = st->sV[gi] = nullptr;
   for (int gi = 0; gi < st->groups && ok; ++gi)
     ok = cudaStreamCreateWithFlags(&st->sK[gi], cudaStreamNonBlocking) == cudaSuccess &&
          cudaStreamCreateWithFlags(&st->sS[gi], cudaStreamNonBlocking) == cudaSuccess &&
          cudaStreamCreateWithFlags(&st->sV[gi], cudaStreamNonBlocking) == cudaSuccess;
   if (!ok) {
+    cudaGetLastError();
     fwpkm_destroy_state(st);
     return FWPKM_ERR_CUDA;
   }
   if (cudaMemset(st->wk.status, 0, sizeof(int)) != cudaSuccess ||
       (st->wk.pbar_cnt &&
        cudaMemset(st->wk.pbar_cnt, 0, sizeof(int) * 2 * (size_t)dm.M * ((dm.n + 255) / 256)) != cudaSuccess)) {
-    delete st;
+    cudaGetLastError();
+    fwpkm_destroy_state(st);
     return FWPKM_ERR_CUDA;
   }
   *out = st;
@@ -443,12 +471,16 @@ void fwpkm_destroy_state(fwpkm_state* st) {
   }
   if (st->sCap) cudaStreamDestroy(st->sCap);
   for (cudaEvent_t e : st->ev) cudaEventDestroy(e);
+  if (st->hstat) cudaFreeHost(st->hstat);
   delete st;
 }
 
+// Before enqueueing anything: a device error that a kernel has already latched (its host
+// copy, read without waiting) is returned until fwpkm_sync clears it; then any pending
+// CUDA error of this thread.
 static fwpkm_status peek_status(fwpkm_state* st) {
-  // A latched device error is reported by the next call (non-blocking check).
-  (void)st;
+  const int h = st->hstat ? *(volatile int*)st->hstat : DEV_OK;
+  if (h != DEV_OK) return status_of_device(h);
   return last_cuda();
 }
 
@@ -488,6 +520,10 @@ fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream
   if (!st) return FWPKM_ERR_INVALID_ARG;
   if (!st->pending) return FWPKM_ERR_STATE;
   if (v_next && !aligned(v_next, 4)) return FWPKM_ERR_INVALID_ARG;
+  {
+    fwpkm_status ps = peek_status(st);
+    if (ps != FWPKM_OK) return ps;
+  }
   const Dims& d = st->dm;
   cudaStream_t s = (cudaStream_t)stream;
   const bool last_has_target = (v_next != nullptr) || !(d.flags & FWPKM_LOOKAHEAD);
@@ -846,8 +882,62 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
   return last_cuda();
 }
 
+// ---- the whole layer: projections in, the memory loop, projection out ----
+// Scratch parts: q, v (q/v dtype), g, o, each starting on a 256-byte boundary.
+static size_t run_layer_carve(const Dims& d, int T, char* base, void** q, void** v, float** g, float** o) {
+  const size_t rows = (size_t)d.M * T, es = qv_size(d);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return p;
+  };
+  void* pq = take(es * rows * d.d);
+  void* pv = take(es * rows * d.dv);
+  float* pg = (float*)take(4 * rows);
+  float* po = (float*)take(4 * rows * d.dv);
+  if (q) { *q = pq; *v = pv; *g = pg; *o = po; }
+  return off;
+}
+
+fwpkm_status fwpkm_run_layer_scratch_size(const fwpkm_config* cfg, int T, size_t* bytes) {
+  fwpkm_status s = check_cfg(cfg);
+  if (s != FWPKM_OK) return s;
+  if (!bytes || T < 0) return FWPKM_ERR_INVALID_ARG;
+  *bytes = run_layer_carve(make_dims(cfg), T, nullptr, nullptr, nullptr, nullptr, nullptr);
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_run_layer(fwpkm_layer* L, fwpkm_state* st, const void* h, int T, int n_iter, void* scratch,
+                             size_t scratch_bytes, void* o_out, void* stream) {
+  NvtxRange nvtx_range("fwpkm_run_layer");
+  const fwpkm_layer_config* lc = layer_config(L);
+  if (!lc || !st) return FWPKM_ERR_INVALID_ARG;
+  if (T == 0) return FWPKM_OK;
+  const Dims& d = st->dm;
+  if (!h || !scratch || !o_out || T < 0 || n_iter < 1 || T > st->wk.max_T) return FWPKM_ERR_INVALID_ARG;
+  if (lc->d != d.d || lc->d_v != d.dv || lc->qv_dtype != st->cfg.qv_dtype ||
+      (long long)d.M * T > (long long)lc->max_rows)
+    return FWPKM_ERR_INVALID_ARG;
+  if (!aligned(h, 16) || !aligned(o_out, 16) || !aligned(scratch, ALIGN)) return FWPKM_ERR_INVALID_ARG;
+  if (scratch_bytes < run_layer_carve(d, T, nullptr, nullptr, nullptr, nullptr, nullptr)) return FWPKM_ERR_WORKSPACE;
+  void *q, *v;
+  float *g, *o;
+  run_layer_carve(d, T, (char*)scratch, &q, &v, &g, &o);
+  const int rows = d.M * T;
+  fwpkm_status s = fwpkm_layer_in(L, h, rows, q, v, g, stream);
+  if (s != FWPKM_OK) return s;
+  s = fwpkm_run_sequence(st, q, v, g, T, n_iter, o, stream);
+  if (s != FWPKM_OK) return s;
+  return fwpkm_layer_out(L, o, rows, o_out, stream);
+}
+
 fwpkm_status fwpkm_last_addressing(fwpkm_state* st, int T, int32_t* idx_out, float* w_out, void* stream) {
   if (!st || T < 1 || T > st->wk.max_T) return FWPKM_ERR_INVALID_ARG;
+  {
+    fwpkm_status ps = peek_status(st);
+    if (ps != FWPKM_OK) return ps;
+  }
   const Dims& d = st->dm;
   cudaStream_t s = (cudaStream_t)stream;
   const size_t row = (size_t)T * d.k, src_pitch = (size_t)st->wk.max_T * d.k;
@@ -863,12 +953,20 @@ fwpkm_status fwpkm_last_addressing(fwpkm_state* st, int T, int32_t* idx_out, flo
 fwpkm_status fwpkm_sync(fwpkm_state* st, void* stream) {
   NvtxRange nvtx_range("fwpkm_sync");
   if (!st) return FWPKM_ERR_INVALID_ARG;
-  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return last_cuda() == FWPKM_OK ? FWPKM_ERR_CUDA : FWPKM_ERR_CUDA;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
+    last_cuda();
+    return FWPKM_ERR_CUDA;
+  }
   int h = 0;
-  if (cudaMemcpy(&h, st->wk.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FWPKM_ERR_CUDA;
+  if (cudaMemcpy(&h, st->wk.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return last_cuda();
+  const int hh = st->hstat ? *(volatile int*)st->hstat : DEV_OK;
+  if (h == DEV_OK) h = hh;
   if (h != DEV_OK) {
-    cudaMemset(st->wk.status, 0, sizeof(int));
-    return h == DEV_TIMEOUT ? FWPKM_ERR_TIMEOUT : FWPKM_ERR_CUDA;
+    // the word is cleared before the host copy, so a kernel still running on another
+    // stream can only leave both set again
+    if (cudaMemset(st->wk.status, 0, sizeof(int)) != cudaSuccess) return last_cuda();
+    if (st->hstat) *(volatile int*)st->hstat = DEV_OK;
+    return status_of_device(h);
   }
   return last_cuda();
 }

@@ -15,6 +15,28 @@ namespace fwpkm {
 // Device status word values (latched by kernels, read by fwpkm_sync).
 enum : int { DEV_OK = 0, DEV_BAD_SLOT = 1, DEV_TIMEOUT = 2 };
 
+// Latch a device-detected error: the device status word (read by the sync calls) and,
+// when the handle has one, its host-visible copy in mapped pinned host memory, which the
+// next host call reads without waiting for the GPU.
+__device__ __forceinline__ void raise_status(int* dev, int* host, int code) {
+  atomicExch(dev, code);
+  if (host) {
+    *reinterpret_cast<volatile int*>(host) = code;
+    __threadfence_system();
+  }
+}
+
+// Status of a device word value as returned by the C ABI.
+inline fwpkm_status status_of_device(int h) {
+  return h == DEV_OK ? FWPKM_OK : h == DEV_TIMEOUT ? FWPKM_ERR_TIMEOUT
+                              : h == DEV_BAD_SLOT ? FWPKM_ERR_BAD_SLOT : FWPKM_ERR_CUDA;
+}
+
+// Test hook of the timeout path (fwpkm_test_stall_waits): launches of the tensor-core
+// kernels that should wait once on a barrier that nothing completes.  Returns 1 (and
+// counts one down) while any remain.
+int take_test_stall();
+
 // Kernel kinds for the launch counter / per-kernel timing.
 enum KernelKind : int { KK_NONE = 0, KK_GATHER = 1, KK_WRITE = 2, KK_SCORE = 3, KK_CART = 4,
                         KK_SORT = 5, KK_ADDR = 6, KK_OTHER = 7, KK_TOPK = 8, KK_PREP = 9, KK_PBAR = 10,
@@ -45,6 +67,7 @@ struct Work {
   float* lp;         // [M][2][n]          key update: log pbar
   float* Lt;         // [M][2][C]          key update: sum_a P log pbar
   int* status;       // device status word
+  int* hstat;        // device view of the handle's mapped host copy of it (nullptr: none)
   // tensor-core path (bf16 q, d/2 in {64, 128})
   int tc;            // 1 if the tensor-core path is used
   int drows;         // rows of Dfull per problem (C with the key step, else the addressing window)
@@ -99,6 +122,8 @@ struct TcGemm {
   const float* rowscale; const float* bias;
   void* pout0; void* pout1; int split, ld0, ld1, out_bf16;
   int* status;
+  int* hstat;  // mapped host copy of the status word (nullptr: none)
+  int stall;   // test hook: the MMA issuer first waits on a barrier that nothing completes
 };
 
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z, uint64_t pitch_y,
@@ -106,7 +131,9 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t 
 int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g, int m_tiles, cudaStream_t s);
 
 // stream_stage: also carve the staging rows of token-at-a-time inference (at the end).
-size_t workspace_bytes(const Dims& d, int max_T, Work* carve, char* base, bool stream_stage = true);
+// allow_tc: false carves only what the CUDA-core kernels use (no tensor-core buffers).
+size_t workspace_bytes(const Dims& d, int max_T, Work* carve, char* base, bool stream_stage = true,
+                       bool allow_tc = true);
 // The carve `w` of all memories seen from memory m0 on (kernels index it from 0).
 Work group_work(const Dims& d, const Work& w, int m0);
 
@@ -204,6 +231,9 @@ struct NvtxRange {
   NvtxRange(const NvtxRange&) = delete;
   NvtxRange& operator=(const NvtxRange&) = delete;
 };
+
+// The configuration a layer handle was created with (nullptr for a null handle).
+const fwpkm_layer_config* layer_config(const fwpkm_layer* L);
 
 // Adds kernel launches made outside a state's schedule (layer projections, metrics) to
 // the count fwpkm_launch_count() reports.

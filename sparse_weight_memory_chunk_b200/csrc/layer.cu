@@ -28,6 +28,8 @@ struct fwpkm_layer {
   float* inv_rms;       // [max_rows]             per-row 1/rms scratch
   __nv_bfloat16* opc;   // [2][max_rows][d_v]     bf16 pieces of o
   int* status;          // device status word (GEMM wait timeouts)
+  int* hstat;           // its host copy (pinned, mapped), written by the kernel that latches
+  int* hstat_dev;       // device view of hstat
   float b_g;
   int qv_pieces, o_pieces;  // 1 when the norm weight is absent (folded weights exact in bf16)
   int have_params;
@@ -81,6 +83,12 @@ fwpkm_status cuda_status() {
     return FWPKM_ERR_CUDA;
   }
   return FWPKM_OK;
+}
+
+// A device error already latched in the handle's host copy (read without waiting).
+fwpkm_status layer_peek(const fwpkm_layer* L) {
+  const int h = L->hstat ? *(volatile int*)L->hstat : DEV_OK;
+  return h != DEV_OK ? status_of_device(h) : cuda_status();
 }
 
 }  // namespace
@@ -179,6 +187,10 @@ rms_split_kernel(const float* __restrict__ o, int rows, int dv, float eps, float
 
 }  // namespace fwpkm
 
+namespace fwpkm {
+const fwpkm_layer_config* layer_config(const fwpkm_layer* L) { return L ? &L->cfg : nullptr; }
+}  // namespace fwpkm
+
 extern "C" {
 
 fwpkm_status fwpkm_layer_workspace_size(const fwpkm_layer_config* cfg, size_t* bytes) {
@@ -198,10 +210,15 @@ fwpkm_status fwpkm_layer_init(const fwpkm_layer_config* cfg, void* workspace, si
   if (!L) return FWPKM_ERR_INVALID_ARG;
   L->cfg = *cfg;
   layer_carve(*cfg, L, (char*)workspace);
-  if (cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess) {
-    delete L;
-    return cuda_status() == FWPKM_OK ? FWPKM_ERR_CUDA : FWPKM_ERR_CUDA;
+  L->hstat = L->hstat_dev = nullptr;
+  if (cudaHostAlloc((void**)&L->hstat, sizeof(int), cudaHostAllocMapped) != cudaSuccess ||
+      cudaHostGetDevicePointer((void**)&L->hstat_dev, L->hstat, 0) != cudaSuccess ||
+      cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess) {
+    cuda_status();
+    fwpkm_layer_destroy(L);
+    return FWPKM_ERR_CUDA;
   }
+  *(volatile int*)L->hstat = DEV_OK;
   *out = L;
   return FWPKM_OK;
 }
@@ -213,15 +230,21 @@ fwpkm_status fwpkm_layer_sync(fwpkm_layer* L, void* stream) {
     return FWPKM_ERR_CUDA;
   }
   int h = 0;
-  if (cudaMemcpy(&h, L->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FWPKM_ERR_CUDA;
+  if (cudaMemcpy(&h, L->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_status();
+  if (h == DEV_OK && L->hstat) h = *(volatile int*)L->hstat;
   if (h != DEV_OK) {
-    cudaMemset(L->status, 0, sizeof(int));
-    return h == DEV_TIMEOUT ? FWPKM_ERR_TIMEOUT : FWPKM_ERR_CUDA;
+    if (cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess) return cuda_status();
+    if (L->hstat) *(volatile int*)L->hstat = DEV_OK;
+    return status_of_device(h);
   }
   return cuda_status();
 }
 
-void fwpkm_layer_destroy(fwpkm_layer* L) { delete L; }
+void fwpkm_layer_destroy(fwpkm_layer* L) {
+  if (!L) return;
+  if (L->hstat) cudaFreeHost(L->hstat);
+  delete L;
+}
 
 fwpkm_status fwpkm_layer_set_params(fwpkm_layer* L, const fwpkm_layer_params* p, void* stream) {
   NvtxRange nvtx_range("fwpkm_layer_set_params");
@@ -260,6 +283,10 @@ fwpkm_status fwpkm_layer_in(fwpkm_layer* L, const void* h, int rows, void* q, vo
   if (!h || !q || !v || !g || rows < 0 || rows > c.max_rows) return FWPKM_ERR_INVALID_ARG;
   if (!al(h, 16) || !al(q, 16) || !al(v, 16) || !al(g, 4)) return FWPKM_ERR_INVALID_ARG;
   if (!L->have_params) return FWPKM_ERR_STATE;
+  {
+    const fwpkm_status ps = layer_peek(L);
+    if (ps != FWPKM_OK) return ps;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   const int D = c.d_model, nqv = c.d + c.d_v;
   rms_gate_kernel<<<(rows + 7) / 8, LAYER_THREADS, 0, s>>>((const __nv_bfloat16*)h, rows, D, c.eps_rms, L->wg,
@@ -277,7 +304,9 @@ fwpkm_status fwpkm_layer_in(fwpkm_layer* L, const void* h, int rows, void* q, vo
   t.pout0 = q; t.ld0 = c.d; t.pout1 = v; t.ld1 = c.d_v; t.split = c.d;
   t.out_bf16 = c.qv_dtype == FWPKM_BF16;
   t.status = L->status;
-  launch_tc_gemm(A, B, t, (rows + 127) / 128, s);
+  t.hstat = L->hstat_dev;
+  t.stall = take_test_stall();
+  if (launch_tc_gemm(A, B, t, (rows + 127) / 128, s) < 0) return FWPKM_ERR_CUDA;
   count_launches(2);
   return cuda_status();
 }
@@ -290,6 +319,10 @@ fwpkm_status fwpkm_layer_out(fwpkm_layer* L, const float* o, int rows, void* o_o
   if (!o || !o_out || rows < 0 || rows > c.max_rows) return FWPKM_ERR_INVALID_ARG;
   if (!al(o, 16) || !al(o_out, 16)) return FWPKM_ERR_INVALID_ARG;
   if (!L->have_params) return FWPKM_ERR_STATE;
+  {
+    const fwpkm_status ps = layer_peek(L);
+    if (ps != FWPKM_OK) return ps;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   const int D = c.d_model, dv = c.d_v;
   const long long ops = (long long)c.max_rows * dv;
@@ -307,7 +340,9 @@ fwpkm_status fwpkm_layer_out(fwpkm_layer* L, const float* o, int rows, void* o_o
   t.pout0 = o_out; t.ld0 = D; t.pout1 = nullptr; t.ld1 = 0; t.split = D;
   t.out_bf16 = 1;
   t.status = L->status;
-  launch_tc_gemm(A, B, t, (rows + 127) / 128, s);
+  t.hstat = L->hstat_dev;
+  t.stall = take_test_stall();
+  if (launch_tc_gemm(A, B, t, (rows + 127) / 128, s) < 0) return FWPKM_ERR_CUDA;
   count_launches(2);
   return cuda_status();
 }

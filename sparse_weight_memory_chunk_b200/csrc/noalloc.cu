@@ -3,11 +3,16 @@
 // that cannot allocate device memory.
 //
 // Who needs it: code that runs where cudaMalloc is unavailable or forbidden -- a
-// host callback, a real-time or embedded loop with a no-allocation rule, a plugin
-// whose host process owns the device allocator, or a caller in the middle of
-// building a larger program that must not change the device memory map.  Every
-// other entry point takes its scratch from a caller-provided workspace; this one
-// takes nothing but its inputs, outputs and the state.
+// real-time or embedded loop with a no-allocation rule, a plugin whose host process
+// owns the device allocator, or a caller in the middle of building a larger program
+// that must not change the device memory map.  Every other entry point takes its
+// scratch from a caller-provided workspace; this one takes nothing but its inputs,
+// outputs and the state.  It makes CUDA runtime calls and launches kernels, so it must
+// not be called from a CUDA host function (a stream callback or cudaLaunchHostFunc),
+// where CUDA calls are not allowed.
+//
+// It runs the CUDA-core kernels of the chunk step (never the tensor-core ones), so its
+// scratch is sized for those alone.
 //
 // The scratch is the file-scope array g_scratch below (FWPKM_NOALLOC_SCRATCH_BYTES).
 // Every GPU that loads the library keeps it allocated until the process exits.
@@ -63,7 +68,8 @@ extern "C" fwpkm_status fwpkm_chunk_step_noalloc(const fwpkm_config* cfg, float*
   d.n = cfg->n; d.h = cfg->d / 2; d.d = cfg->d; d.dv = cfg->d_v; d.k = cfg->k; d.C = cfg->chunk;
   d.M = cfg->num_mem; d.N = (long long)cfg->n * cfg->n; d.qv_bf16 = cfg->qv_dtype == FWPKM_BF16;
   d.eps_idw = cfg->eps_idw; d.eps_norm = cfg->eps_norm; d.lr_key = cfg->lr_key; d.flags = cfg->flags;
-  need = workspace_bytes(d, cfg->chunk, nullptr, nullptr, false);  // no token-at-a-time staging
+  // no token-at-a-time staging and no tensor-core buffers: only what the kernels below use
+  need = workspace_bytes(d, cfg->chunk, nullptr, nullptr, false, false);
   if (need > FWPKM_NOALLOC_SCRATCH_BYTES) {
     fprintf(stderr, "fwpkm_chunk_step_noalloc: this shape needs %zu bytes of scratch; the built-in "
                     "array holds %u\n", need, FWPKM_NOALLOC_SCRATCH_BYTES);
@@ -79,15 +85,12 @@ extern "C" fwpkm_status fwpkm_chunk_step_noalloc(const fwpkm_config* cfg, float*
   if (s != FWPKM_OK) return s;
 
   Work w;
-  workspace_bytes(d, cfg->chunk, &w, (char*)base, false);
+  workspace_bytes(d, cfg->chunk, &w, (char*)base, false, false);
 
   cudaStream_t st = (cudaStream_t)stream;
-  // The array keeps the previous call's contents: only the status word is read
-  // before it is written, so it is the one thing cleared.
-  if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) {
-    cudaGetLastError();
-    return FWPKM_ERR_CUDA;
-  }
+  // The array keeps the previous call's contents.  Every buffer the kernels below read is
+  // written earlier in the same call, so nothing needs clearing (the status word a
+  // skipped bad slot would set is not read by this entry point).
   const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
   const bool last_has_target = (v_next != nullptr) || !(d.flags & FWPKM_LOOKAHEAD);
   bool ok = launch_score_topk(d, w, K1, K2, q, seq_stride, 0, c_len, ku, st) >= 0;

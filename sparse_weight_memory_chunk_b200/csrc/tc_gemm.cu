@@ -41,7 +41,8 @@ constexpr int TC_MAX_STAGES = 2;
 constexpr int TC_EPI_WARPS = 16;
 constexpr int TC_THREADS = (2 + TC_EPI_WARPS) * 32;
 constexpr uint32_t TC_TMEM_COLS = 256;
-constexpr uint64_t TC_TIMEOUT_NS = 200ull * 1000 * 1000;
+constexpr uint64_t TC_TIMEOUT_NS = 200ull * 1000 * 1000;  // every wait of the main loop
+constexpr uint64_t TC_DRAIN_NS = 200ull * 1000 * 1000;    // draining in-flight copies/MMAs on abort
 
 int tc_stages(int npieces, int kblocks_per_cta) {
   int st = (200 * 1024) / (npieces * TC_TILE_BYTES);
@@ -51,7 +52,7 @@ int tc_stages(int npieces, int kblocks_per_cta) {
 }
 
 size_t tc_smem_bytes(int npieces, int stages) {
-  return 1024 + (size_t)stages * npieces * TC_TILE_BYTES + 256;
+  return 1024 + (size_t)stages * npieces * TC_TILE_BYTES + 256;  // tiles + barriers and flags
 }
 
 __device__ __forceinline__ bool wait_deadline(uint64_t* bar, uint32_t parity, uint64_t deadline) {
@@ -80,7 +81,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* acce = accf + 2;
   uint64_t* drain = acce + 2;
   uint64_t* normbar = drain + 1;
-  uint32_t* tmem_slot = (uint32_t*)(normbar + 1);
+  uint64_t* stallbar = normbar + 1;  // test hook: a barrier that nothing completes
+  uint32_t* tmem_slot = (uint32_t*)(stallbar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   __shared__ float s_norm[4][TC_BM];
 
@@ -100,6 +102,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     mbar_init(drain, 1);
     mbar_init(normbar, TC_EPI_WARPS);
+    mbar_init(stallbar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -148,7 +151,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // ---------------- MMA issuer ----------------
     const uint32_t idesc = idesc_bf16_f32(TC_BM, TC_BN);
     int it = 0;
-    for (int j = 0; j < ntiles; ++j) {
+    // test hook of the timeout path: wait on a barrier that nothing completes; the bounded
+    // wait runs out and raises the abort flag, and every role unwinds as on a real timeout
+    const bool stalled = g.stall && !mbar_wait(stallbar, 0, abort_flag, deadline);
+    for (int j = 0; j < ntiles && !stalled; ++j) {
       const int b = j & 1;
       const uint32_t aph = (j >> 1) & 1;
       if (j >= 2 && !mbar_wait(&acce[b], aph ^ 1, abort_flag, deadline)) break;
@@ -178,7 +184,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       umma_commit(&accf[b]);
     }
     umma_commit(drain);  // completes once every MMA issued above has finished
-    wait_deadline(drain, 0, deadline + TC_TIMEOUT_NS);
+    wait_deadline(drain, 0, deadline + TC_DRAIN_NS);
   } else if (ntiles > 0 && warp >= 2) {
     // ---------------- epilogue: 16 warps; warp w reads TMEM lane quarter w%4 (tile rows
     // 32*(w%4)..+31, one per thread) and column group (w-2)/4 (32 columns) ----------------
@@ -356,7 +362,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 0 && lane == 0 && *abort_flag) {
     // let the copies this CTA issued land before its shared memory goes away
     for (int i = issued - S < 0 ? 0 : issued - S; i < issued; ++i)
-      wait_deadline(&full[i % S], (i / S) & 1, deadline + TC_TIMEOUT_NS);
+      wait_deadline(&full[i % S], (i / S) & 1, deadline + TC_DRAIN_NS);
   }
   tc_fence_before();
   __syncthreads();
@@ -364,7 +370,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tc_fence_after();
     tmem_dealloc(tmem, TC_TMEM_COLS);
   }
-  if (threadIdx.x == 0 && *abort_flag) atomicExch(g.status, DEV_TIMEOUT);
+  if (threadIdx.x == 0 && *abort_flag) raise_status(g.status, g.hstat, DEV_TIMEOUT);
 }
 
 // ---------------------------------------------------------------------------

@@ -302,6 +302,8 @@ int launch_tc_score(const Dims& d, const Work& w, const void* q_base, long long 
   g.colv = w.kn; g.colv_pstride = d.n;
   g.zpart = key_update ? w.zpart : nullptr; g.zpart_pstride = d.C; g.eps = d.eps_idw;
   g.status = w.status;
+  g.hstat = w.hstat;
+  g.stall = take_test_stall();
   return launch_tc_gemm(A, B, g, (len + 127) / 128, s);
 }
 
@@ -355,7 +357,9 @@ int launch_tc_keystep(const Dims& d, const Work& w, float* K1, float* K2, const 
   g.K1 = K1; g.K2 = K2; g.Kpc = w.Kpc; g.kn = w.kn; g.piece_P = w.P_all;
   g.wsum_part = w.wsum_part; g.wsum_tiles = ntb; g.lr = d.lr_key;
   g.status = w.status;
-  launch_tc_gemm(A, B, g, (d.n + 127) / 128, s);
+  g.hstat = w.hstat;
+  g.stall = take_test_stall();
+  if (launch_tc_gemm(A, B, g, (d.n + 127) / 128, s) < 0) return -1;
   return launched;
 }
 

@@ -303,7 +303,7 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
       if (!((heads >> gi) & 1u)) continue;
       const int slot = (int)(key0 >> 32);
       if (slot < 0 || (long long)slot >= dm.N) {
-        if (lane == 0) atomicExch(w.status, DEV_BAD_SLOT);
+        if (lane == 0) raise_status(w.status, w.hstat, DEV_BAD_SLOT);
         continue;
       }
       float4 Gs[VPL];

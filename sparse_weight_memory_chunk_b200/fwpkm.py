@@ -15,7 +15,8 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfwpkm.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_STATE = 0, -1, -2, -3, -4, -5, -6
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_STATE, ERR_BAD_SLOT = \
+    0, -1, -2, -3, -4, -5, -6, -7
 F32, BF16 = 0, 1
 KEY_UPDATE, TARGET_NORM, LOOKAHEAD, GATE_WEIGHT = 1, 2, 4, 8
 DEFAULT_FLAGS = TARGET_NORM | LOOKAHEAD | GATE_WEIGHT
@@ -99,6 +100,9 @@ def lib():
             "fwpkm_layer_out": ([_P, _P, ctypes.c_int, _P, _P], ctypes.c_int),
             "fwpkm_layer_sync": ([_P, _P], ctypes.c_int),
             "fwpkm_layer_destroy": ([_P], None),
+            "fwpkm_run_layer_scratch_size": ([C, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+            "fwpkm_run_layer": ([_P, _P, _P, ctypes.c_int, ctypes.c_int, _P, ctypes.c_size_t, _P, _P], ctypes.c_int),
+            "fwpkm_test_stall_waits": ([ctypes.c_int], None),
             "fwpkm_metrics_workspace_size": ([ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                               ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
             "fwpkm_addressing_metrics": ([_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -134,6 +138,37 @@ def status_string(status: int) -> str:
 
 def launch_count() -> int:
     return int(lib().fwpkm_launch_count())
+
+
+def test_stall_waits(n_launches: int):
+    """Test hook: the next n tensor-core launches wait once on a barrier that nothing
+    completes, so their bounded wait runs out (no fault; see include/fwpkm.h)."""
+    lib().fwpkm_test_stall_waits(int(n_launches))
+
+
+def run_layer_scratch_size(cfg: Config, T: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().fwpkm_run_layer_scratch_size(ctypes.byref(cfg), T, ctypes.byref(out)), "run_layer_scratch_size")
+    return out.value
+
+
+def run_layer_parts(cfg: Config, T: int, scratch):
+    """Views of the q, v, g, o that fwpkm_run_layer leaves in `scratch` (a uint8 tensor)."""
+    import torch
+    M, d, dv = cfg.num_mem, cfg.d, cfg.d_v
+    es = 2 if cfg.qv_dtype == BF16 else 4
+    qdt = torch.bfloat16 if cfg.qv_dtype == BF16 else torch.float32
+    al = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    sizes = [es * M * T * d, es * M * T * dv, 4 * M * T, 4 * M * T * dv]
+    offs, o = [], 0
+    for b in sizes:
+        offs.append(o)
+        o = al(o + b)
+    q = scratch[offs[0]:offs[0] + sizes[0]].view(qdt).view(M, T, d)
+    v = scratch[offs[1]:offs[1] + sizes[1]].view(qdt).view(M, T, dv)
+    g = scratch[offs[2]:offs[2] + sizes[2]].view(torch.float32).view(M, T)
+    ob = scratch[offs[3]:offs[3] + sizes[3]].view(torch.float32).view(M, T, dv)
+    return q, v, g, ob
 
 
 def workspace_size(cfg: Config, max_T: int) -> int:
@@ -308,6 +343,17 @@ class Layer:
 
     def sync(self, stream=None):
         _check(lib().fwpkm_layer_sync(self.handle, _stream(stream)), "layer_sync")
+
+    def run_layer(self, state, h, o_out, T=None, n_iter=1, scratch=None, stream=None):
+        """fwpkm_run_layer: h [M][T][d_model] bf16 -> o_out [M][T][d_model] bf16 through the
+        projections and the memory `state`.  Returns the scratch tensor (see run_layer_parts)."""
+        import torch
+        T = h.shape[1] if T is None else T
+        if scratch is None:
+            scratch = torch.empty(run_layer_scratch_size(state.cfg, T), dtype=torch.uint8, device=h.device)
+        _check(lib().fwpkm_run_layer(self.handle, state.handle, _ptr(h), T, n_iter, _ptr(scratch), scratch.numel(),
+                                     _ptr(o_out), _stream(stream)), "run_layer")
+        return scratch
 
     def destroy(self):
         if getattr(self, "handle", None):

@@ -169,23 +169,25 @@ def gen_needles(w: Workload, q: np.ndarray, v: np.ndarray):
     return pos, qpos, qs, vs
 
 
-def gen_layer(w: Workload, B: int | None = None, T: int | None = None):
+def gen_layer(w: Workload, B: int | None = None, T: int | None = None, clusters: int = 64, zipf: float = 1.1):
     """Hidden states and slow weights of the layer workload.
 
-    h [B][T][d_model] bf16 bits from 64 Gaussian clusters (centres N(0, I), cluster
-    weights proportional to j^-1.1, x = centre + 0.1 N(0, I)); RMSNorm gains = 1;
+    h [B][T][d_model] bf16 bits from `clusters` Gaussian clusters (centres N(0, I),
+    cluster weights proportional to j^-zipf, x = centre + 0.1 N(0, I)); RMSNorm gains = 1;
     W_q [d][d_model], W_v [d_v][d_model], w_g [d_model] and W_o [d_model][d_v]
-    ([out][in]) as bf16 bits drawn N(0, 1/fan_in); gate bias 0."""
+    ([out][in]) as bf16 bits drawn N(0, 1/fan_in); gate bias 0.  The workload itself is
+    64 clusters with s = 1.1; fewer clusters or a larger exponent give the hotter
+    variants that the skew tests use (same weights, same streams)."""
     B = w.B if B is None else B
     T = w.T if T is None else T
     ss = _streams(w.seed)
     kids = ss["layer"].spawn(6)
     gc = np.random.Generator(np.random.PCG64(kids[0]))
-    centres = gc.standard_normal((64, w.d_model), dtype=np.float32)
-    pz = np.arange(1, 65, dtype=np.float64) ** -1.1
+    centres = gc.standard_normal((clusters, w.d_model), dtype=np.float32)
+    pz = np.arange(1, clusters + 1, dtype=np.float64) ** -zipf
     pz /= pz.sum()
     ga = np.random.Generator(np.random.PCG64(kids[1]))
-    assign = ga.choice(64, size=(w.B, w.T), p=pz)[:B, :T]
+    assign = ga.choice(clusters, size=(w.B, w.T), p=pz)[:B, :T]
     gx = np.random.Generator(np.random.PCG64(kids[2]))
     noise = gx.standard_normal((w.B, w.T, w.d_model), dtype=np.float32)[:B, :T]
     hid = f32_to_bf16(centres[assign] + np.float32(0.1) * noise)

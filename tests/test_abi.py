@@ -43,6 +43,21 @@ def test_status_strings(lib):
     assert lib.status_string(0) == "ok"
     assert lib.status_string(-3) == "workspace too small"
     assert lib.status_string(-5) == "device wait timed out"
+    assert lib.status_string(lib.ERR_BAD_SLOT) == "slot index out of range in the write"
+
+
+def test_run_layer_scratch_and_checks(lib):
+    import ctypes as C
+    cfg = lib.make_config(n=512, d=256, d_v=256, k=32, chunk=256, num_mem=16, bf16=True, key_update=True)
+    rows = 16 * 4096
+    # q, v (bf16), g, o (fp32), each part on a 256-byte boundary
+    assert lib.run_layer_scratch_size(cfg, 4096) == 2 * rows * 256 * 2 + rows * 4 + rows * 256 * 4
+    so = lib.lib()
+    fake = C.c_void_p(1 << 20)
+    assert so.fwpkm_run_layer(None, None, fake, 16, 1, fake, 1 << 30, fake, None) == lib.ERR_INVALID_ARG
+    with pytest.raises(lib.FwpkmError):
+        lib.run_layer_scratch_size(cfg, -1)
+    lib.test_stall_waits(0)  # the timeout test hook is host-side state only
 
 
 def test_workspace_size_and_validation(lib):

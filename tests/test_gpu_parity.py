@@ -67,7 +67,12 @@ def streaming_vs_oracle(name, **flags):
     return compare_streaming(name, *make_case(name, **flags))
 
 
-def compare_streaming(name, w, data, gcfg, ocfg):
+def compare_streaming(name, w, data, gcfg, ocfg, n_iter=1):
+    """Chunk by chunk (n_iter passes over the sequence, the state carried across them):
+    forward_chunk + write_chunk on the GPU against the oracle's chunk from the GPU's own
+    pre-chunk state; o, weights, keys (and the key step itself) and value rows compared
+    after every chunk.  Returns the final GPU tensors, the near-tie count and every
+    chunk's slot lists (idx: list of [M][len][k] arrays, in order)."""
     q, v, g, K1, K2, V = data
     M, T, C, k, dv, N = w.M, w.T, w.C, w.k, w.d_v, w.N
     st, dev = device_state(w, data, gcfg, C)
@@ -77,47 +82,50 @@ def compare_streaming(name, w, data, gcfg, ocfg):
     small = N * dv <= (1 << 22)
     rng = np.random.default_rng(0)
     ties = 0
-    for t0 in range(0, T, C):
-        ln = min(C, T - t0)
-        K1pre, K2pre = dev["K1"].cpu().numpy().copy(), dev["K2"].cpu().numpy().copy()
-        idx_d = torch.empty(M, ln, k, dtype=torch.int32, device="cuda")
-        w_d = torch.empty(M, ln, k, device="cuda")
-        st.forward_chunk(dev["q"][:, t0:], dev["v"][:, t0:], dev["g"][:, t0:], o_d[:, t0:], ln, seq_stride=T,
-                         idx_out=idx_d, w_out=w_d)
-        has_next = t0 + ln < T
-        st.write_chunk(dev["v"][:, t0 + ln] if has_next else None)
-        st.sync()
-        idx_g, w_g = idx_d.cpu().numpy(), w_d.cpu().numpy()
-        o_g = o_d[:, t0:t0 + ln].cpu().numpy()
-        for m in range(M):
-            k1, k2 = K1pre[m].copy(), K2pre[m].copy()
-            vn = vf[m, t0 + ln] if has_next else None
-            o_o, I_o, w_o, nt = oracle_chunk_against_gpu(ocfg, qf[m, t0:t0 + ln], vf[m, t0:t0 + ln],
-                                                         g[m, t0:t0 + ln].astype(np.float64), vn, k1, k2,
-                                                         V_orc[m], idx_g[m])
-            ties += nt
-            assert_close(o_g[m], o_o, f"{name} chunk@{t0} mem {m}: o")
-            assert_close(w_g[m], w_o, f"{name} chunk@{t0} mem {m}: w", atol=1e-6)
-            if w.key_update:
-                K1g, K2g = dev["K1"][m].cpu().numpy(), dev["K2"][m].cpu().numpy()
-                assert_close(K1g, k1, f"{name} chunk@{t0} mem {m}: K1")
-                assert_close(K2g, k2, f"{name} chunk@{t0} mem {m}: K2")
-                # the step itself (tiny next to K) must agree, not just the keys
-                for Kg, Ko, Kp in ((K1g, k1, K1pre[m]), (K2g, k2, K2pre[m])):
-                    dg = Kg.astype(np.float64) - Kp
-                    do = Ko.astype(np.float64) - Kp
-                    ulp = np.spacing(np.abs(Ko)).astype(np.float64)
-                    assert np.all(np.abs(dg - do) <= 2 * ulp + 2e-3 * np.abs(do) + 1e-9), f"{name}: dK"
-            if small:
-                rows = np.arange(N)
-            else:
-                touched = np.unique(idx_g[m].reshape(-1))
-                rows = np.unique(np.concatenate([touched, rng.integers(0, N, 2048)]))
-            Vg = dev["V"][m][torch.from_numpy(rows).cuda()].cpu().numpy()
-            assert_close(Vg, V_orc[m][rows], f"{name} chunk@{t0} mem {m}: V")
+    idx_all = []
+    for _pass in range(n_iter):
+        for t0 in range(0, T, C):
+            ln = min(C, T - t0)
+            K1pre, K2pre = dev["K1"].cpu().numpy().copy(), dev["K2"].cpu().numpy().copy()
+            idx_d = torch.empty(M, ln, k, dtype=torch.int32, device="cuda")
+            w_d = torch.empty(M, ln, k, device="cuda")
+            st.forward_chunk(dev["q"][:, t0:], dev["v"][:, t0:], dev["g"][:, t0:], o_d[:, t0:], ln, seq_stride=T,
+                             idx_out=idx_d, w_out=w_d)
+            has_next = t0 + ln < T
+            st.write_chunk(dev["v"][:, t0 + ln] if has_next else None)
+            st.sync()
+            idx_g, w_g = idx_d.cpu().numpy(), w_d.cpu().numpy()
+            idx_all.append(idx_g)
+            o_g = o_d[:, t0:t0 + ln].cpu().numpy()
+            for m in range(M):
+                k1, k2 = K1pre[m].copy(), K2pre[m].copy()
+                vn = vf[m, t0 + ln] if has_next else None
+                o_o, I_o, w_o, nt = oracle_chunk_against_gpu(ocfg, qf[m, t0:t0 + ln], vf[m, t0:t0 + ln],
+                                                             g[m, t0:t0 + ln].astype(np.float64), vn, k1, k2,
+                                                             V_orc[m], idx_g[m])
+                ties += nt
+                assert_close(o_g[m], o_o, f"{name} chunk@{t0} mem {m}: o")
+                assert_close(w_g[m], w_o, f"{name} chunk@{t0} mem {m}: w", atol=1e-6)
+                if w.key_update:
+                    K1g, K2g = dev["K1"][m].cpu().numpy(), dev["K2"][m].cpu().numpy()
+                    assert_close(K1g, k1, f"{name} chunk@{t0} mem {m}: K1")
+                    assert_close(K2g, k2, f"{name} chunk@{t0} mem {m}: K2")
+                    # the step itself (tiny next to K) must agree, not just the keys
+                    for Kg, Ko, Kp in ((K1g, k1, K1pre[m]), (K2g, k2, K2pre[m])):
+                        dg = Kg.astype(np.float64) - Kp
+                        do = Ko.astype(np.float64) - Kp
+                        ulp = np.spacing(np.abs(Ko)).astype(np.float64)
+                        assert np.all(np.abs(dg - do) <= 2 * ulp + 2e-3 * np.abs(do) + 1e-9), f"{name}: dK"
+                if small:
+                    rows = np.arange(N)
+                else:
+                    touched = np.unique(idx_g[m].reshape(-1))
+                    rows = np.unique(np.concatenate([touched, rng.integers(0, N, 2048)]))
+                Vg = dev["V"][m][torch.from_numpy(rows).cuda()].cpu().numpy()
+                assert_close(Vg, V_orc[m][rows], f"{name} chunk@{t0} mem {m}: V")
     # full-size states stay on the device (8 GiB of V)
     return dict(o=o_d.cpu(), V=dev["V"].cpu() if small else dev["V"], K1=dev["K1"].cpu(), K2=dev["K2"].cpu(), ties=ties,
-                w=w, data=data, gcfg=gcfg)
+                w=w, data=data, gcfg=gcfg, idx=idx_all)
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -177,6 +185,28 @@ def test_passes_compose_and_determinism(name):
     st.sync()
     assert torch.equal(o.cpu(), outs[0][0]) and torch.equal(dev["V"].cpu(), outs[0][1])
     assert torch.equal(dev["K1"].cpu(), outs[0][2])
+
+
+def test_needle_stream_two_passes():
+    """The needle workload's shapes (N = 1,048,576 slots, C = 512, frozen keys) with its
+    planted (q*, v*) needle pairs, read in two passes over the same input (paperlayer §4.3
+    iterative reading): every chunk of both passes against the oracle, then
+    fwpkm_run_sequence(n_iter = 2) bit-for-bit against those chunk-by-chunk calls."""
+    from dataclasses import replace
+
+    from sparse_weight_memory_chunk_b200.inputs import gen_needles
+    w, data, gcfg, ocfg = make_case("needle_chunk")
+    w = replace(w, needles=64)
+    q, v, g, K1, K2, V = data
+    gen_needles(w, q, v)  # in place: 64 needles planted 3 times each, queried once late
+    res = compare_streaming("needle_2pass", w, (q, v, g, K1, K2, V), gcfg, ocfg, n_iter=2)
+    print(f"needle two passes: near-ties {res['ties']}")
+    st, dev = device_state(w, (q, v, g, K1, K2, V), gcfg, w.T)
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    st.run_sequence(dev["q"], dev["v"], dev["g"], o, n_iter=2)
+    st.sync()
+    assert torch.equal(o.cpu(), res["o"]), "run_sequence(n_iter=2) o differs from chunk-by-chunk"
+    assert torch.equal(dev["V"], res["V"]), "run_sequence(n_iter=2) V differs from chunk-by-chunk"
 
 
 def test_edge_cases():

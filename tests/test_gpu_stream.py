@@ -1,11 +1,12 @@
 """Token-at-a-time inference on the GPU (fwpkm_stream_tokens / fwpkm_stream_flush through
 the C ABI).
 
-Feeding a sequence in arbitrary groups of tokens, then flushing, must give the bits of the
-production entry point (fwpkm_run_sequence) on the same inputs: the reads are per token
-and the writes are the same kernels on the same chunk contents.  fwpkm_run_sequence is
-checked against the oracle chunk by chunk in test_gpu_parity.py, and the oracle's own
-token-at-a-time loop against its chunked loop in test_oracle_stream_pins.py.
+Feeding a sequence in arbitrary groups of tokens, then flushing, is compared directly
+with the oracle's own token-at-a-time loop (oracle/stream.py: each token read as it
+arrives, a chunk written when its lookahead arrives; "Fast-weight Product Key Memory"
+(paperlayer summary) §A.1), and must also give the bits of the production entry point
+(fwpkm_run_sequence) on the same inputs: the reads are per token and the writes are the
+same kernels on the same chunk contents.
 """
 import numpy as np
 import pytest
@@ -15,6 +16,8 @@ pytestmark = pytest.mark.gpu
 
 from sparse_weight_memory_chunk_b200 import fwpkm  # noqa: E402
 
+from oracle.stream import stream_sequence  # noqa: E402
+from parity import as_f64, assert_close  # noqa: E402
 from test_gpu_parity import device_state, make_case  # noqa: E402
 
 
@@ -56,6 +59,31 @@ def test_token_stream_gives_the_bits_of_run_sequence(name):
     assert torch.equal(o, o_ref), f"{name}: o differs from run_sequence"
     for key in ("V", "K1", "K2"):
         assert torch.equal(dev[key], dev_ref[key]), f"{name}: {key} differs from run_sequence"
+
+
+@pytest.mark.parametrize("name", ["tiny_key_ragged", "mid_key", "k1", "chunk1"])
+def test_token_stream_matches_oracle_stream(name):
+    """o of every token and the final V, K1, K2 against oracle.stream_sequence fed the same
+    arrival groups (parity tolerances: 1e-4 relative + 1e-5 absolute)."""
+    w, data, gcfg, ocfg = make_case(name)
+    q, v, g, K1, K2, V = data
+    st, dev = device_state(w, data, gcfg, w.C)
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    groups = groups_for(w.T, w.C, seed=7 + len(name))
+    t = 0
+    for n in groups:
+        st.stream_tokens(dev["q"][:, t:], dev["v"][:, t:], dev["g"][:, t:], o[:, t:], n_tok=n, seq_stride=w.T)
+        t += n
+    st.stream_flush()
+    st.sync()
+    qf, vf = as_f64(q, w.qv), as_f64(v, w.qv)
+    for m in range(w.M):
+        k1, k2, vv = K1[m].copy(), K2[m].copy(), V[m].copy()
+        o_o = stream_sequence(ocfg, qf[m], vf[m], g[m].astype(np.float64), k1, k2, vv, groups)
+        assert_close(o[m].cpu().numpy(), o_o, f"{name} mem {m}: o")
+        assert_close(dev["V"][m].cpu().numpy(), vv, f"{name} mem {m}: V")
+        assert_close(dev["K1"][m].cpu().numpy(), k1, f"{name} mem {m}: K1")
+        assert_close(dev["K2"][m].cpu().numpy(), k2, f"{name} mem {m}: K2")
 
 
 def test_one_token_at_a_time_and_state_rules():

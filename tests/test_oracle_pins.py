@@ -417,3 +417,32 @@ def test_single_token_and_lookahead_off():
     cfg2 = oracle.make_cfg(n=n, d=2 * h, d_v=dv, k=1, chunk=4, lookahead=False, target_norm=False)
     o, I, w = oracle.run_sequence(cfg2, q, v, np.ones(1), K1, K2, V)
     np.testing.assert_allclose(V[I[0, 0]], v[0], rtol=1e-7)
+
+
+@pytest.mark.parametrize("nthreads", [1, 2, 3, 7])
+def test_independent_memories_in_threads_equal_one_call_per_memory(nthreads):
+    """orc_run_sequence_multi (the CPU baseline's entry point: memories spread over
+    threads, each memory's inputs and state at its own stride; with more threads than
+    memories each chunk's read phase is split over token ranges) gives, bit for bit, the
+    outputs, slots and states of one orc_run_sequence per memory -- the memories share
+    nothing and the tokens of a chunk's read phase are independent."""
+    rng = np.random.default_rng(7)
+    n, h, dv, k, C, T, M = 16, 8, 8, 4, 5, 13, 3
+    cfg = oracle.make_cfg(n, 2 * h, dv, k, C, key_update=True, lr_key=10.0)
+    q = rng.normal(size=(M, T, 2 * h))
+    v = rng.normal(size=(M, T, dv))
+    g = rng.uniform(size=(M, T))
+    K1 = rng.normal(size=(M, n, h)).astype(np.float32)
+    K2 = rng.normal(size=(M, n, h)).astype(np.float32)
+    V = (0.02 * rng.normal(size=(M, n * n, dv))).astype(np.float32)
+    k1, k2, vv = K1.copy(), K2.copy(), V.copy()
+    o_multi, used, I_multi = oracle.run_sequence_multi(cfg, q, v, g, k1, k2, vv, n_iter=2, nthreads=nthreads,
+                                                       with_slots=True)
+    assert used == (nthreads if nthreads <= M else M * (nthreads // M))
+    for m in range(M):
+        a1, a2, av = K1[m].copy(), K2[m].copy(), V[m].copy()
+        o_m, I_m, _ = oracle.run_sequence(cfg, q[m], v[m], g[m], a1, a2, av, n_iter=2)
+        assert np.array_equal(o_multi[m], o_m), f"memory {m}: o"
+        assert np.array_equal(I_multi[m], I_m), f"memory {m}: slots"
+        assert np.array_equal(k1[m], a1) and np.array_equal(k2[m], a2), f"memory {m}: keys"
+        assert np.array_equal(vv[m], av), f"memory {m}: values"

@@ -24,9 +24,13 @@ def close(a, b):
     return bool(((a - b).abs() <= ATOL + RTOL * b.abs()).all())
 
 
-@pytest.mark.parametrize("qv,key_update", [("f32", True), ("bf16", False)])
-def test_noalloc_chunk_steps_match_workspace_entry_points(qv, key_update):
-    n, d, dv, k, C, M = (64, 64, 64, 8, 64, 2) if qv == "f32" else (256, 128, 128, 16, 128, 2)
+@pytest.mark.parametrize("qv,key_update,shape", [("f32", True, (64, 64, 64, 8, 64, 2)),
+                                                  ("bf16", False, (256, 128, 128, 16, 128, 2)),
+                                                  ("bf16", True, (64, 128, 64, 8, 32, 2))])
+def test_noalloc_chunk_steps_match_workspace_entry_points(qv, key_update, shape):
+    # the last case: bf16 queries with the key step, which this entry point runs on the
+    # CUDA-core kernels while the workspace entry points take the tensor-core path
+    n, d, dv, k, C, M = shape
     T = 2 * C
     w = Workload("noalloc", n, d, dv, k, T + 1, C, M, 1, qv, key_update, 21, "sigmoid", "normal002")
     q, v, g = gen_qvg(w)
