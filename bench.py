@@ -9,6 +9,12 @@ T=4096, bf16 q/v, fp32 state, key update on).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload paper|mid|tiny|needle|layer]
     python bench.py --impl reference ...   # the CPU oracle on a bounded sample
 
+The default run measures the paper-scale workload (the headline `value`) and then the
+other four workloads (tiny, mid, needle at n_iter = 1, 2 and 4 with its read-back, and
+the full layer), each reported under `configs` in the same JSON line with its own
+step time, throughput, roofline fractions, clocks and a selection check against the
+oracle.  `--workload X` measures X alone; `--no-configs` skips the other workloads.
+
 Multi-GPU (torchrun): every rank runs its own independent memories (different
 sequences); there is no collective on the data path ("scaling": "weak").
 """
@@ -33,10 +39,10 @@ from sparse_weight_memory_chunk_b200.inputs import (WORKLOADS, gen_keys, gen_lay
 BY_NAME = {w.name: (i, w) for i, w in WORKLOADS.items()}
 
 # DRAM bytes (read + write) per launch and per memory of the paper-scale kernels, from one
-# ncu capture of a 2-memory case of the paper shapes (profiles/kernel_counters_paper_workload_2mem.md
-# has the capture and its command): dram__bytes_read.sum + dram__bytes_write.sum of the
-# captured launch / 2; a full launch scales with the memories it processes (each memory's
-# work is the same).  A kernel changed since that capture is missing here and reports null.
+# ncu capture of a 2-memory case of the paper shapes (the capture and its command are kept
+# with the profiles): dram__bytes_read.sum + dram__bytes_write.sum of the captured launch
+# / 2; a full launch scales with the memories it processes (each memory's work is the
+# same).  A kernel changed since that capture is missing here and reports null.
 TRAFFIC = {
     "score": {"per_mem": (3_493_376 + 512) / 2},
     "pbar": {"per_mem": 4_345_856 / 2},
@@ -54,12 +60,15 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="paper", choices=["tiny", "mid", "paper", "needle", "layer"])
+    ap.add_argument("--workload", default=None, choices=["tiny", "mid", "paper", "needle", "layer"],
+                    help="measure this workload alone (default: paper, plus the others under `configs`)")
     ap.add_argument("--n-iter", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-metrics", action="store_true", help="skip the addressing-metrics measurement")
     ap.add_argument("--no-stream", action="store_true", help="skip the token-at-a-time measurement")
+    ap.add_argument("--no-configs", action="store_true", help="measure the headline workload only")
+    ap.add_argument("--config-steps", type=int, default=5, help="timed steps of each extra workload")
     ap.add_argument("--batch", type=int, default=None, help="override the number of sequences B (profiling)")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling)")
     ap.add_argument("--kernel", default=None,
@@ -81,49 +90,111 @@ def describe(w, n_iter):
 _SAMPLE_CACHE = {}
 
 
-def oracle_sample(w, n_chunks):
-    """Time the CPU oracle (as it stands) on sequence 0's H memories, first n_chunks chunks.
+def host_cpu():
+    """(hardware threads of this host, CPU model) for the CPU-baseline record."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
+
+
+def _oracle_inputs(w, seqs, T):
+    """fp64 inputs, initial fp32 state and (layer workload) W_o of sequences 0..seqs-1."""
+    from sparse_weight_memory_chunk_b200.inputs import bf16_to_f32
+    M = seqs * w.H
+    K1, K2 = gen_keys(w, M=M)
+    V = np.stack([gen_values(w, m) for m in range(M)])
+    if w.d_model:
+        # layer workload: the projections' oracle turns the hidden states into q, v, g
+        from oracle import layer as orc_layer
+        L = gen_layer(w, B=seqs, T=T)
+        ones = np.ones(w.d_model)
+        qs, vs, gs = [], [], []
+        for b in range(seqs):
+            qf, vf, gf = orc_layer.project_in(bf16_to_f32(L["h"][b]), ones, bf16_to_f32(L["Wq"]), None, ones,
+                                              bf16_to_f32(L["Wv"]), None, ones, bf16_to_f32(L["wg"]), 0.0)
+            qs.append(qf); vs.append(vf); gs.append(gf)
+        return np.stack(qs), np.stack(vs), np.stack(gs), K1, K2, V, bf16_to_f32(L["Wo"])
+    q, v, g = gen_qvg(w, M=M)
+    if w.needles:
+        gen_needles(w, q, v)  # planted over the whole stream, as on the GPU; the sample reads its head
+    q, v, g = q[:, :T], v[:, :T], g[:, :T]
+    qf = (bf16_to_f32(q) if w.qv == "bf16" else q).astype(np.float64)
+    vf = (bf16_to_f32(v) if w.qv == "bf16" else v).astype(np.float64)
+    return qf, vf, g.astype(np.float64), K1, K2, V, None
+
+
+def oracle_sample(w, n_chunks, seqs=None):
+    """CPU-baseline leg: time the oracle (as it stands) on sequences 0..seqs-1 (every head),
+    first n_chunks chunks, on all host threads (memories in parallel; with more threads
+    than memories each chunk's read phase is split over token ranges).
 
     The inputs are drawn once per process; every call starts from a fresh copy of the
     initial state (the oracle updates it in place)."""
     import oracle
-    from sparse_weight_memory_chunk_b200.inputs import bf16_to_f32
-    H = w.H
+    cores, model = host_cpu()
+    seqs = seqs or w.B
     T = min(w.T, n_chunks * w.C)
-    key = (w.name, T)
-    if key not in _SAMPLE_CACHE and w.d_model:
-        # layer workload: the projections' oracle turns sequence 0's hidden states into q, v, g
-        from oracle import layer as orc_layer
-        L = gen_layer(w, B=1, T=T)
-        hf = bf16_to_f32(L["h"][0])
-        ones = np.ones(w.d_model)
-        qf, vf, gf = orc_layer.project_in(hf, ones, bf16_to_f32(L["Wq"]), None, ones, bf16_to_f32(L["Wv"]), None,
-                                          ones, bf16_to_f32(L["wg"]), 0.0)
-        K1, K2 = gen_keys(w, M=H)
-        V = np.stack([gen_values(w, m) for m in range(H)])
-        _SAMPLE_CACHE[key] = (qf[None], vf[None], gf[None], K1, K2, V, bf16_to_f32(L["Wo"]))
-        oracle.build()
+    key = (w.name, T, seqs)
     if key not in _SAMPLE_CACHE:
-        q, v, g = gen_qvg(w, M=H)
-        q, v, g = q[:, :T], v[:, :T], g[:, :T]
-        K1, K2 = gen_keys(w, M=H)
-        V = np.stack([gen_values(w, m) for m in range(H)])
-        qf = (bf16_to_f32(q) if w.qv == "bf16" else q).astype(np.float64)
-        vf = (bf16_to_f32(v) if w.qv == "bf16" else v).astype(np.float64)
-        _SAMPLE_CACHE[key] = (qf, vf, g.astype(np.float64), K1, K2, V, None)
         oracle.build()
+        _SAMPLE_CACHE[key] = _oracle_inputs(w, seqs, T)
     qf, vf, gf, K1, K2, V, Wo = _SAMPLE_CACHE[key]
     k1, k2, vv = K1.copy(), K2.copy(), V.copy()
     cfg = oracle.make_cfg(w.n, w.d, w.d_v, w.k, w.C, key_update=w.key_update)
     t0 = time.perf_counter()
-    res, used = oracle.run_sequence_multi(cfg, qf, vf, gf, k1, k2, vv, 1, nthreads=H)
+    res, used = oracle.run_sequence_multi(cfg, qf, vf, gf, k1, k2, vv, 1, nthreads=cores)
     if Wo is not None:
         from oracle import layer as orc_layer
-        orc_layer.project_out(res[0], np.ones(w.d_v), Wo, None)
+        for b in range(seqs):
+            orc_layer.project_out(res[b], np.ones(w.d_v), Wo, None)
     dt = time.perf_counter() - t0
-    return dict(tokens=T, seconds=dt, threads=used,
-                sample=f"sequence 0 ({H} heads = {H} memories, full N={w.N:,} each), tokens 0..{T - 1} "
-                       f"({n_chunks} chunks), {used} threads")
+    M = seqs * w.H
+    return dict(tokens=seqs * T, seconds=dt, threads=used, cpu_model=model, host_threads=cores,
+                sample=f"sequences 0..{seqs - 1} ({M} memories of N={w.N:,} slots), tokens 0..{T - 1} "
+                       f"({n_chunks} chunks of {w.C}), {used} threads of {cores} on {model}")
+
+
+TIE_REL = 1e-6
+
+
+def selection_check(w, q_bits, K1, K2, idx):
+    """Part of the CPU-baseline leg: the GPU's slot lists of chunk 0 (initial keys) against
+    the oracle's, per token of memories 0..H-1 (sequence 0): exact, near-tie (at every rank
+    the GPU's slot score, recomputed in fp64, within 1e-6 max(1, |S|) of the oracle's) or
+    mismatch."""
+    import math
+
+    import oracle
+    from sparse_weight_memory_chunk_b200.inputs import bf16_to_f32
+    cfg = oracle.make_cfg(w.n, w.d, w.d_v, w.k, w.C)
+    h, n = w.h, w.n
+    out = {"tokens": 0, "exact": 0, "near_tie": 0, "mismatch": 0}
+    for m in range(idx.shape[0]):
+        qm = (bf16_to_f32(q_bits[m]) if q_bits.dtype == np.uint16 else q_bits[m]).astype(np.float64)
+        for t in range(idx.shape[1]):
+            D1 = oracle.subkey_dist(cfg, qm[t, :h], K1[m])
+            D2 = oracle.subkey_dist(cfg, qm[t, h:], K2[m])
+            I_o, S_o, _ = oracle.select(cfg, D1, D2)
+            out["tokens"] += 1
+            I_g = idx[m, t]
+            if np.array_equal(I_o, I_g):
+                out["exact"] += 1
+                continue
+            ok = len(set(I_g.tolist())) == w.k and I_g.min() >= 0 and I_g.max() < n * n
+            if ok:
+                S_g = np.array([-math.log(cfg.eps_idw + D1[s // n]) - math.log(cfg.eps_idw + D2[s % n]) for s in I_g])
+                ok = bool(np.all(np.abs(S_g - S_o) <= TIE_REL * np.maximum(1.0, np.abs(S_o))))
+            out["near_tie" if ok else "mismatch"] += 1
+    out["definition"] = ("chunk 0 of sequence 0's memories from the initial keys: GPU slot lists against the "
+                         "oracle's (exact; near-tie = scores within 1e-6 relative at every rank; mismatch)")
+    return out
 
 
 def run_reference(args, w, rank):
@@ -133,20 +204,23 @@ def run_reference(args, w, rank):
     times = []
     info = None
     for i in range(args.warmup + args.steps):
-        info = oracle_sample(w, n_chunks)
+        info = oracle_sample(w, n_chunks, seqs=None if w.name in ("paper", "mid", "tiny") else 1)
         if i >= args.warmup:
             times.append(info["seconds"])
     ms = 1000.0 * sum(times) / len(times)
     val = info["tokens"] / (ms / 1000.0)
-    line = {"metric": "FwPKM layer tokens/s (retrieve+chunk write) at 1M slots; % of HBM roofline",
-            "value": val, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": describe(w, 1), "sample": info["sample"]},
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": info["threads"], "kind": "oracle",
-                             "sample": info["sample"]},
+                             "sample": info["sample"], "host_threads": info["host_threads"],
+                             "cpu_model": info["cpu_model"]},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+METRIC = "FwPKM layer tokens/s (retrieve+chunk write) at 1M slots; % of HBM roofline"
 
 
 # --------------------------------------------------------------------------- clocks
@@ -234,27 +308,32 @@ def job_throughput(units_per_rank_step, world, ms_step):
     return units_per_rank_step * world / (ms_step / 1000.0)
 
 
-def run_ours(args, w, rank, world, local_rank):
-    import torch
-    import torch.distributed as dist
-
-    from sparse_weight_memory_chunk_b200 import build, fwpkm
-    build.build()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
+def load_peaks():
     peaks = {}
     pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(pp):
         peaks = json.load(open(pp))
-    hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
-    tc_peak = float(peaks.get("bf16_tflops_sustained", 1400.0))
-    peak_src = "measured" if peaks else "fallback"
+    return (float(peaks.get("hbm_gbs", 6650.0)), float(peaks.get("bf16_tflops_sustained", 1400.0)),
+            "measured" if peaks else "fallback", peaks)
+
+
+def measure(args, w, rank, world, local_rank, n_iter, steps, warmup, full):
+    """Measure one workload: `steps` timed steps after `warmup` (each step one call of the
+    public entry point over the whole batch: fwpkm_run_sequence, or fwpkm_run_layer for
+    the layer workload).  `full`: also the end-to-end, addressing-metrics and
+    token-at-a-time measurements and the CPU-baseline leg's timing.  Returns the line."""
+    import torch
+    import torch.distributed as dist
+
+    from sparse_weight_memory_chunk_b200 import fwpkm
+    dev = torch.device("cuda", local_rank)
+    hbm_peak, tc_peak, peak_src, peaks = load_peaks()
 
     # inputs (per-rank independent sequences: seed offset by rank)
     wr = rank_workload(w, rank)
     q, v, g = gen_qvg(wr)
     K1, K2 = gen_keys(wr)
-    needles = gen_needles(wr, q, v) if w.name == "needle" else None
+    needles = gen_needles(wr, q, v) if w.needles else None
 
     def to_dev(x):
         if x.dtype == np.uint16:
@@ -271,36 +350,34 @@ def run_ours(args, w, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     layer = None
     if w.d_model:
-        # full layer: h -> (RMSNorm + Linear) q, v, g -> memory -> (RMSNorm + Linear) o'
+        # full layer through fwpkm_run_layer: h -> (RMSNorm + Linear) q, v, g -> memory ->
+        # (RMSNorm + Linear) o'; the memory's q, v, g, o live in the call's scratch
         Ld = gen_layer(wr)
         hd = to_dev(Ld["h"])
         layer = fwpkm.Layer(w.d_model, w.d, w.d_v, w.M * w.T, qv_bf16=w.qv == "bf16", device=dev)
         lw = {k_: to_dev(Ld[k_]) for k_ in ("Wq", "Wv", "wg", "Wo")}
         layer.set_params(lw["Wq"], lw["Wv"], lw["wg"], lw["Wo"])
-        qdt = torch.bfloat16 if w.qv == "bf16" else torch.float32
-        qd = torch.empty(w.M, w.T, w.d, device=dev, dtype=qdt)
-        vd = torch.empty(w.M, w.T, w.d_v, device=dev, dtype=qdt)
-        gd = torch.empty(w.M, w.T, device=dev)
-        o_out = torch.empty(w.M * w.T, w.d_model, device=dev, dtype=torch.bfloat16)
+        scratch = torch.empty(fwpkm.run_layer_scratch_size(cfg, w.T), dtype=torch.uint8, device=dev)
+        qd, vd, gd, o = fwpkm.run_layer_parts(cfg, w.T, scratch)
+        o_out = torch.empty(w.M, w.T, w.d_model, device=dev, dtype=torch.bfloat16)
 
         def step():
-            layer.project_in(hd, qd, vd, gd, rows=w.M * w.T)
-            st.run_sequence(qd, vd, gd, o, n_iter=args.n_iter)
-            layer.project_out(o.view(-1, w.d_v), o_out)
+            layer.run_layer(st, hd, o_out, n_iter=n_iter, scratch=scratch)
     else:
         qd, vd, gd = to_dev(q), to_dev(v), to_dev(g)
 
         def step():
-            st.run_sequence(qd, vd, gd, o, n_iter=args.n_iter)
-    state0 = (K1d.clone(), K2d.clone(), Vd.clone()) if needles is not None else None
+            st.run_sequence(qd, vd, gd, o, n_iter=n_iter)
+    K1_init, K2_init = K1d.clone(), K2d.clone()
+    state0 = (Vd.clone(),) if needles is not None else None
 
     # warm-up; find the dominant kernel kind by timing each kind once
-    for _ in range(max(args.warmup, 1)):
+    for _ in range(max(warmup, 1)):
         step()
     kinds = {}
     if args.kernel is None:
-        for name in ("gather", "write", "score", "topk", "cartesian", "sort", "pbar", "wbuild", "address", "prep",
-                     "other"):
+        for name in ("gather", "write", "score", "topk", "cartesian", "sort", "pbar", "wbuild", "address", "fused",
+                     "prep", "other"):
             st.profile_kernel(name)
             step()
             ms, n = st.kernel_time()
@@ -326,8 +403,8 @@ def run_ours(args, w, rank, world, local_rank):
     l0 = fwpkm.launch_count()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
-    for s_ in range(args.steps):
-        if s_ == args.steps - 1:
+    for s_ in range(steps):
+        if s_ == steps - 1:
             st.profile_kernel(timed_kind)
         step()
     ev1.record(stream)
@@ -340,8 +417,10 @@ def run_ours(args, w, rank, world, local_rank):
     dom_ms, dom_n = st.kernel_time()
     st.profile_kernel(0)
     st.sync()
-    ms_step = max_over_ranks(ms_total / args.steps, world, dev)
-    tokens_per_step = w.B * w.T * args.n_iter
+    if layer is not None:
+        layer.sync()
+    ms_step = max_over_ranks(ms_total / steps, world, dev)
+    tokens_per_step = w.B * w.T * n_iter
     value = job_throughput(tokens_per_step, world, ms_step)
 
     # algorithmic traffic of the step (measured unique rows) and roofline
@@ -349,8 +428,8 @@ def run_ours(args, w, rank, world, local_rank):
     st.last_addressing(w.T, idx_out=idx)
     torch.cuda.synchronize()
     b_vk, gather_per_token, U = algorithmic_bytes(w, idx, w.T)
-    b_vk *= args.n_iter
-    flops = 2 * w.n * w.d * w.M * w.T * args.n_iter * (2 if w.key_update else 1)
+    b_vk *= n_iter
+    flops = 2 * w.n * w.d * w.M * w.T * n_iter * (2 if w.key_update else 1)
     if w.d_model:  # the slow-weight projections (in: q, v, gate; out: o')
         flops += 2 * w.M * w.T * w.d_model * (w.d + w.d_v + 1 + w.d_v)
     t_roof = max(b_vk / (hbm_peak * 1e9), flops / (tc_peak * 1e12))
@@ -372,6 +451,8 @@ def run_ours(args, w, rank, world, local_rank):
         "wbuild": ("hbm", 2 * w.n * 4 * tok * 2 + 2 * w.n * 2 * 2 * tok),  # rows read twice, 2 bf16 pieces written
         "sort": ("hbm", w.k * tok * (4 + 8)),                      # slots read, pair keys written
         "cartesian": ("alu", cand * 2 * tok),                      # one add + one compare per candidate
+        # the one-launch addressing step: scoring and (key update) key-step contractions
+        "fused": ("tensor", 2 * w.n * w.d * tok * (2 if w.key_update else 1)),
     }
 
     def kind_roofline(kind, ms, n):
@@ -385,8 +466,9 @@ def run_ours(args, w, rank, world, local_rank):
             ach, peak, unit, src = per_launch / avg_s / 1e12, tc_peak, "TFLOP/s", "bf16_tflops_sustained"
         else:
             ach, peak, unit, src = per_launch / avg_s / 1e12, alu_peak, "Tops/s", "148 SMs x 128 fp32 lanes x max clock"
+        traffic = TRAFFIC.get(kind, {}).get("per_mem", 0) * w.M if w.name == "paper" else 0
         return {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
-                "traffic": TRAFFIC.get(kind, {}).get("per_mem", 0) * w.M or None,
+                "traffic": traffic or None,
                 "kernel": kind, "peak_source": f"{peak_src if bound != 'alu' else 'derived'} ({src})",
                 "avg_launch_us": avg_s * 1e6, "launches_timed": n,
                 "algorithmic_per_launch": per_launch}
@@ -397,11 +479,10 @@ def run_ours(args, w, rank, world, local_rank):
                        "bound": r_["bound"] if r_ else None}
                   for k_, v_ in kinds.items()}
 
-    line = {"metric": "FwPKM layer tokens/s (retrieve+chunk write) at 1M slots; % of HBM roofline",
-            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": {"workload": describe(w, args.n_iter),
+            "config": {"workload": describe(w, n_iter),
                        "l2": "inputs larger than L2: V is 8 GiB per GPU and a step touches ~2.1 GB of V rows"
                              if w.name == "paper" else "V state larger than L2" if w.N * w.d_v * 4 * w.M > 126e6
                              else "L2-resident (tiny)",
@@ -412,9 +493,25 @@ def run_ours(args, w, rank, world, local_rank):
             "kernels_one_step": kind_table,
             "clocks": clk, "gpu_launches": int(launches)}
 
+    # chunk 0 of sequence 0's memories at the initial keys, for the selection check of the
+    # CPU-baseline leg (the selections do not depend on V)
+    chk = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cfg0 = fwpkm.make_config(w.n, w.d, w.d_v, w.k, w.C, w.H, w.qv == "bf16")
+        st0 = fwpkm.State(cfg0, K1_init[:w.H].contiguous(), K2_init[:w.H].contiguous(), Vd[:w.H], w.C)
+        idx0 = torch.empty(w.H, w.C, w.k, dtype=torch.int32, device=dev)
+        o0 = torch.empty(w.H, w.C, w.d_v, device=dev)
+        st0.forward_chunk(qd[:w.H], vd[:w.H], gd[:w.H], o0, w.C, seq_stride=qd.shape[1], idx_out=idx0)
+        st0.sync()
+        qb = qd[:w.H, :w.C]
+        q_bits = (qb.contiguous().view(torch.int16).cpu().numpy().view(np.uint16) if qb.dtype == torch.bfloat16
+                  else qb.cpu().numpy())
+        chk = (q_bits, K1_init[:w.H].cpu().numpy(), K2_init[:w.H].cpu().numpy(), idx0.cpu().numpy())
+        st0.destroy()
+
     # addressing metrics of the final pass's selections (windows of 32K tokens per memory),
     # timed apart from the step
-    if not args.no_metrics:
+    if full and not args.no_metrics:
         mwin = 32768
         mws = torch.empty(fwpkm.metrics_workspace_size(w.M, w.T, w.N, mwin), dtype=torch.uint8, device=dev)
         for _ in range(3):
@@ -439,7 +536,7 @@ def run_ours(args, w, rank, world, local_rank):
                          "definition": "selections read once + N 32-bit counters per window written and read once"}}
 
     # end to end through the public API with host buffers
-    if not args.no_e2e:
+    if full and not args.no_e2e:
         dev_in = [hd] if layer is not None else [qd, vd, gd]
         dev_out = o_out if layer is not None else o
         host_in = [torch.empty_like(x, device="cpu").pin_memory() for x in dev_in]
@@ -459,11 +556,11 @@ def run_ours(args, w, rank, world, local_rank):
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+        ems = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
         bi = sum(x.numel() * x.element_size() for x in host_in)
         line["e2e"] = {"value": job_throughput(tokens_per_step, world, ems), "unit": "tokens/s",
                        "h2d_bytes_per_step": bi, "d2h_bytes_per_step": host_out.numel() * host_out.element_size(),
@@ -473,7 +570,7 @@ def run_ours(args, w, rank, world, local_rank):
         # read-back: from the initial state, n_iter passes; vhat at each needle's query
         # position recovered from o = g vhat + (1 - g) v, against the normalised needle value
         from sparse_weight_memory_chunk_b200.inputs import bf16_to_f32
-        K1d.copy_(state0[0]); K2d.copy_(state0[1]); Vd.copy_(state0[2])
+        K1d.copy_(K1_init); K2d.copy_(K2_init); Vd.copy_(state0[0])
         step()
         st.sync()
         pos, qpos, _, vs = needles
@@ -486,12 +583,12 @@ def run_ours(args, w, rank, world, local_rank):
             vhat = (of[r] - (1.0 - gf[r]) * vf[r]) / gf[r]
             z = (vsf[i] - vsf[i].mean()) / np.sqrt(vsf[i].var() + 1e-5)
             cos.append(float(vhat @ z / (np.linalg.norm(vhat) * np.linalg.norm(z) + 1e-30)))
-        line["needle_readback"] = {"n_iter": args.n_iter, "mean_cos": float(np.mean(cos)),
+        line["needle_readback"] = {"n_iter": n_iter, "mean_cos": float(np.mean(cos)),
                                    "min_cos": float(np.min(cos)), "needles": len(cos),
                                    "definition": "cos(vhat_r, z(v*)) at each needle's query position r, final pass, "
                                                  "run from the initial state"}
 
-    if not args.no_stream:
+    if full and not args.no_stream and layer is None:
         # token-at-a-time inference: the first 2C + 1 tokens of every memory fed 1 (then 16)
         # per call through fwpkm_stream_tokens (two chunk writes, each when its lookahead
         # arrives), then a flush; timed with events on the launching stream
@@ -527,14 +624,49 @@ def run_ours(args, w, rank, world, local_rank):
                           "write (unique rows), all memories; latency-bound: a token's read is a chain of about "
                           "six dependent launches"}
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_chunks = 8 if w.name in ("paper", "needle") else 16
-        info = oracle_sample(w, n_chunks)
-        line["cpu_baseline"] = {"value": info["tokens"] / info["seconds"], "unit": "tokens/s",
-                                "cores": info["threads"], "kind": "oracle", "sample": info["sample"]}
+    st.destroy()
+    if layer is not None:
+        layer.destroy()
+    del Vd, K1d, K2d, o
+    torch.cuda.empty_cache()
+
+    # CPU-baseline leg (rank 0, one GPU): the oracle's selection check of chunk 0, and
+    # (full) the oracle timed on a bounded sample of the same workload
+    if chk is not None:
+        line["selection_check"] = selection_check(w, *chk)
+        if full:
+            n_chunks = 8 if w.name in ("paper", "needle") else 16
+            info = oracle_sample(w, n_chunks, seqs=None if w.name in ("paper", "mid") else 1)
+            line["cpu_baseline"] = {"value": info["tokens"] / info["seconds"], "unit": "tokens/s",
+                                    "cores": info["threads"], "kind": "oracle", "sample": info["sample"],
+                                    "host_threads": info["host_threads"], "cpu_model": info["cpu_model"]}
+    return line
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+
+    from sparse_weight_memory_chunk_b200 import build
+    build.build()
+    torch.cuda.set_device(local_rank)
+    line = measure(args, w, rank, world, local_rank, args.n_iter, args.steps, args.warmup, full=True)
+    if args.workload is None and not args.no_configs:
+        # the other workloads, each under `configs`: fewer timed steps, the same rules
+        configs = {}
+        for name, n_iter in (("tiny", 1), ("mid", 1), ("needle", 1), ("needle", 2), ("needle", 4), ("layer", 1)):
+            key = name if name != "needle" else f"needle_n{n_iter}"
+            _, wc = BY_NAME[name]
+            try:
+                sub = measure(args, wc, rank, world, local_rank, n_iter, max(1, args.config_steps),
+                              max(3, args.warmup), full=False)
+                keep = ("ms_per_step", "value", "unit", "steps", "warmup", "config", "roofline", "step_roofline",
+                        "kernels_one_step", "clocks", "gpu_launches", "selection_check", "needle_readback")
+                configs[key] = {k_: sub[k_] for k_ in keep if k_ in sub}
+            except Exception as e:  # one workload failing must not hide the others
+                configs[key] = {"error": f"{type(e).__name__}: {e}"}
+        line["configs"] = configs
     if rank == 0:
         print(json.dumps(line), flush=True)
-    st.destroy()
 
 
 def main():
@@ -542,7 +674,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    _, w = BY_NAME[args.workload]
+    _, w = BY_NAME[args.workload or "paper"]
     if args.batch or args.tokens:
         from dataclasses import replace
         w = replace(w, B=args.batch or w.B, T=args.tokens or w.T)
