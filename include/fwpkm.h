@@ -365,7 +365,8 @@ uint64_t fwpkm_launch_count(void);
  * 4 cartesian, 5 sort, 6 key-step GEMM (or the whole key step on the SIMT path),
  * 7 residual, 8 per-half top-k (on the tensor-core path fused with the Cartesian
  * search), 9 query/key prep, 10 usage marginals (pbar, log pbar),
- * 11 key-step weights W.  fwpkm_kernel_time() waits for the events and
+ * 11 key-step weights W, 12 the one-launch addressing step of a chunk (distances and,
+ * with the key update, the whole entropy step).  fwpkm_kernel_time() waits for the events and
  * returns the summed duration (ms) and the number of timed launches since the last
  * reset, then resets.  Graph replays overwrite their own events, so after graph
  * replays it covers the last replay. */

@@ -288,6 +288,7 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base, bool strea
   }
   x.Kpc = nullptr; x.kn = nullptr; x.qn = nullptr; x.zpart = nullptr; x.ppart = nullptr;
   x.Wt = nullptr; x.Qt = nullptr; x.wsum_part = nullptr; x.pbar_cnt = nullptr; x.qt_T = 0;
+  x.af_part = nullptr; x.af_cnt = nullptr;
   if (x.tc) {
     const size_t P = 2 * M, h = d.h, cpad = (C + 63) / 64 * 64, nt = (n + 127) / 128;
     x.Kpc = (__nv_bfloat16*)take(2 * 3 * P * n * h);
@@ -301,6 +302,10 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base, bool strea
       x.Qt = (__nv_bfloat16*)take(2 * P * h * (size_t)x.qt_T);
       x.wsum_part = (float*)take(4 * P * (cpad / 16) * n);
       x.pbar_cnt = (int*)take(4 * P * ((n + 255) / 256));
+      if (n % 128 == 0) {
+        x.af_part = (float*)take(4 * addr_fused_part_floats(d));
+        x.af_cnt = (int*)take(4 * P * 2);
+      }
     }
   }
   x.P_all = (int)(2 * M);
@@ -341,6 +346,8 @@ Work group_work(const Dims& d, const Work& w, int m0) {
   if (x.Qt) x.Qt += M0 * 2 * h * (size_t)w.qt_T;
   if (x.wsum_part) x.wsum_part += M0 * 2 * (cpad / 16) * n;
   if (x.pbar_cnt) x.pbar_cnt += M0 * 2 * ((n + 255) / 256);
+  if (x.af_part) x.af_part += M0 * 2 * (n / 128) * 2 * 256;
+  if (x.af_cnt) x.af_cnt += M0 * 2 * 2;
   return x;
 }
 
@@ -450,7 +457,8 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
   }
   if (cudaMemset(st->wk.status, 0, sizeof(int)) != cudaSuccess ||
       (st->wk.pbar_cnt &&
-       cudaMemset(st->wk.pbar_cnt, 0, sizeof(int) * 2 * (size_t)dm.M * ((dm.n + 255) / 256)) != cudaSuccess)) {
+       cudaMemset(st->wk.pbar_cnt, 0, sizeof(int) * 2 * (size_t)dm.M * ((dm.n + 255) / 256)) != cudaSuccess) ||
+      (st->wk.af_cnt && cudaMemset(st->wk.af_cnt, 0, sizeof(int) * 4 * (size_t)dm.M) != cudaSuccess)) {
     cudaGetLastError();
     fwpkm_destroy_state(st);
     return FWPKM_ERR_CUDA;
@@ -497,7 +505,18 @@ fwpkm_status fwpkm_forward_chunk(fwpkm_state* st, const void* q, const void* v, 
   cudaStream_t s = (cudaStream_t)stream;
   const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
   st->host_error = 0;
-  if (st->wk.tc) {
+  if (st->wk.tc && ku && use_fused_addressing(d)) {
+    // the chunk's whole addressing step in one launch: distances for the selection, then
+    // the entropy step on K1, K2 (it needs only this chunk's queries and the keys they
+    // were read with, so it is taken here; write_chunk then writes V)
+    run(st, KK_PREP, s, [&] { return launch_qnorm(d, st->wk, q, seq_stride, 0, c_len, s); });
+    run(st, KK_PREP, s, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, s); });
+    run(st, KK_PREP, s, [&] { return launch_qtrans(d, st->wk, q, seq_stride, 0, c_len, s); });
+    run(st, KK_FUSED, s, [&] {
+      return launch_addr_fused(d, st->wk, st->K1, st->K2, q, seq_stride, c_len, 0, 0, c_len, 0, false, s);
+    });
+    run(st, KK_TOPK, s, [&] { return launch_select(d, st->wk, 0, c_len, idx_out, w_out, s); });
+  } else if (st->wk.tc) {
     run(st, KK_PREP, s, [&] { return launch_qnorm(d, st->wk, q, seq_stride, 0, c_len, s); });
     run(st, KK_PREP, s, [&] { return launch_keyprep(d, st->wk, st->K1, st->K2, s); });
     run(st, KK_SCORE, s, [&] { return launch_tc_score(d, st->wk, q, seq_stride, c_len, 0, 0, c_len, ku, s); });
@@ -527,11 +546,13 @@ fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream
   const Dims& d = st->dm;
   cudaStream_t s = (cudaStream_t)stream;
   const bool last_has_target = (v_next != nullptr) || !(d.flags & FWPKM_LOOKAHEAD);
+  st->host_error = 0;
   run(st, KK_OTHER, s, [&] { return launch_resid(d, st->wk, st->v, st->g, st->stride, st->len, v_next, s); });
   run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, st->wk, 0, st->len, last_has_target, s); });
   run(st, KK_WRITE, s, [&] { return launch_write(d, st->wk, st->V, 0, s); });
-  st->host_error = 0;
-  if ((d.flags & FWPKM_KEY_UPDATE) && st->wk.tc) {
+  if ((d.flags & FWPKM_KEY_UPDATE) && st->wk.tc && use_fused_addressing(d)) {
+    // the key step was taken with the chunk's distances in fwpkm_forward_chunk
+  } else if ((d.flags & FWPKM_KEY_UPDATE) && st->wk.tc) {
     run(st, KK_PBAR, s, [&] { return launch_tc_pbar(d, st->wk, st->len, s); });
     run(st, KK_WBUILD, s, [&] { return launch_tc_wbuild(d, st->wk, st->len, s); });
     run(st, KK_ADDR, s, [&] {
@@ -565,8 +586,16 @@ static void stream_read(fwpkm_state* st, const void* v, const float* g, long lon
   const int p = st->spos;
   const void* qs = offs(wk.stage_q, (long long)p * d.d, es);
   if (wk.tc) {
+    // with the fused key step the reads take their distances from the same kernel (scoring
+    // only), so a token read here gets the bits it gets inside a whole chunk
+    const bool fused = (d.flags & FWPKM_KEY_UPDATE) && use_fused_addressing(d);
     run(st, KK_PREP, s, [&] { return launch_qnorm(d, wk, qs, d.C, p, len, s); });
-    run(st, KK_SCORE, s, [&] { return launch_tc_score(d, wk, wk.stage_q, d.C, d.C, p, p, len, false, s); });
+    if (fused)
+      run(st, KK_FUSED, s, [&] {
+        return launch_addr_fused(d, wk, st->K1, st->K2, wk.stage_q, d.C, d.C, p, p, len, 0, true, s);
+      });
+    else
+      run(st, KK_SCORE, s, [&] { return launch_tc_score(d, wk, wk.stage_q, d.C, d.C, p, p, len, false, s); });
     run(st, KK_TOPK, s, [&] { return launch_select(d, wk, p, len, nullptr, nullptr, s); });
   } else {
     run(st, KK_SCORE, s, [&] { return launch_score_topk(d, wk, st->K1, st->K2, qs, d.C, p, len, false, s); });
@@ -587,7 +616,14 @@ static void stream_write(fwpkm_state* st, bool has_next, cudaStream_t s) {
   run(st, KK_SORT, s, [&] { return launch_sort_pairs(d, wk, 0, len, last_has_target, s); });
   run(st, KK_WRITE, s, [&] { return launch_write(d, wk, st->V, 0, s); });
   if (d.flags & FWPKM_KEY_UPDATE) {
-    if (wk.tc) {
+    if (wk.tc && use_fused_addressing(d)) {
+      // distances recomputed from the staged queries and the key step, in one launch (it
+      // also leaves the new keys' bf16 pieces for the next chunk's reads)
+      run(st, KK_PREP, s, [&] { return launch_qtrans(d, wk, wk.stage_q, d.C, 0, len, s); });
+      run(st, KK_FUSED, s, [&] {
+        return launch_addr_fused(d, wk, st->K1, st->K2, wk.stage_q, d.C, d.C, 0, 0, len, 0, false, s);
+      });
+    } else if (wk.tc) {
       run(st, KK_SCORE, s, [&] { return launch_tc_score(d, wk, wk.stage_q, d.C, d.C, 0, 0, len, true, s); });
       run(st, KK_PBAR, s, [&] { return launch_tc_pbar(d, wk, len, s); });
       run(st, KK_WBUILD, s, [&] { return launch_tc_wbuild(d, wk, len, s); });
@@ -687,6 +723,9 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
   // the key step reads every chunk's half-queries from one feature-major copy made up front
   // (its TMA x offset, the chunk start, must be a multiple of 8 tokens)
   const bool qt_whole = tc && ku && C % 8 == 0;
+  // one launch per chunk for the whole addressing step (its half-queries need the
+  // feature-major copy: C % 16 == 0 keeps qt_whole)
+  const bool fused = tc && ku && use_fused_addressing(d);
   cudaStream_t sK = st->serial ? st->sK[0] : st->sK[gi];
   cudaStream_t sS = st->serial ? sK : st->sS[gi], sV = st->serial ? sK : st->sV[gi];
   auto dep = [&](cudaStream_t from, cudaStream_t to) {
@@ -751,6 +790,13 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
   } else {
     const size_t dbuf = (size_t)wk.dfull_buf;
     std::vector<cudaEvent_t> topk_done(2, nullptr), sel_done(nch, nullptr), val_done(nch, nullptr);
+    // FWPKM_SEL_FIRST=1: the addressing of chunk c+1 also waits for the selection of chunk c
+    // (the selection then runs beside the value kernels rather than beside the addressing)
+    static const bool sel_first = [] {
+      const char* e = getenv("FWPKM_SEL_FIRST");
+      return e && e[0] == '1';
+    }();
+    cudaEvent_t last_topk = nullptr;
     int cnt = 0;
     for (int pass = 0; pass < n_iter; ++pass) {
       for (int c = 0; c < nch; ++c, ++cnt) {
@@ -760,27 +806,32 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
         if (tc) wb.Dfull = wk.Dfull + (size_t)(cnt & 1) * dbuf;
         if (sel_done[c]) cudaStreamWaitEvent(sK, sel_done[c], 0);    // previous pass read A/Dsv
         if (topk_done[cnt & 1]) cudaStreamWaitEvent(sK, topk_done[cnt & 1], 0);  // buffer reuse
-        if (tc) {
+        if (sel_first && last_topk) cudaStreamWaitEvent(sK, last_topk, 0);
+        if (fused) {
+          // the chunk's whole addressing step in one launch; the selection needs its rows
+          run(st, KK_FUSED, sK, [&] {
+            return launch_addr_fused(d, wb, K1, K2, q, T, T, t0, t0, len, t0, false, sK);
+          });
+          cudaStreamWaitEvent(sS, mark(sK), 0);
+        } else if (tc) {
           run(st, KK_SCORE, sK, [&] { return launch_tc_score(d, wb, q, T, T, t0, t0, len, true, sK); });
-        } else {
-          run(st, KK_SCORE, sK, [&] { return launch_score_topk(d, wb, K1, K2, qc, T, t0, len, true, sK); });
-        }
-        // the selection needs the distance rows; on the tensor-core path it also waits for
-        // the usage marginals, so that pbar (on the critical addressing chain) does not share
-        // the GPU with it (1.606 against 1.628 ms per step)
-        if (!tc) cudaStreamWaitEvent(sS, mark(sK), 0);
-        if (tc) {
+          // the selection needs the distance rows; it also waits for the usage marginals, so
+          // that pbar (on the critical addressing chain) does not share the GPU with it
+          // (1.606 against 1.628 ms per step)
           run(st, KK_PBAR, sK, [&] { return launch_tc_pbar(d, wb, len, sK); });
           cudaStreamWaitEvent(sS, mark(sK), 0);
           run(st, KK_WBUILD, sK, [&] { return launch_tc_wbuild(d, wb, len, sK); });
           run(st, KK_ADDR, sK, [&] { return launch_tc_keystep(d, wb, K1, K2, qc, T, len, qt_whole ? t0 : -1, sK); });
         } else {
+          run(st, KK_SCORE, sK, [&] { return launch_score_topk(d, wb, K1, K2, qc, T, t0, len, true, sK); });
+          cudaStreamWaitEvent(sS, mark(sK), 0);
           run(st, KK_ADDR, sK, [&] { return launch_address(d, wb, K1, K2, qc, T, len, sK); });
         }
         if (val_done[c]) cudaStreamWaitEvent(sS, val_done[c], 0);     // previous pass wrote chunk c
         if (tc) {
           run(st, KK_TOPK, sS, [&] { return launch_select(d, wb, t0, len, nullptr, nullptr, sS); });
           topk_done[cnt & 1] = mark(sS);
+          last_topk = topk_done[cnt & 1];
         } else {
           run(st, KK_CART, sS, [&] { return launch_cartesian(d, wb, t0, len, nullptr, nullptr, sS); });
         }
@@ -965,6 +1016,10 @@ fwpkm_status fwpkm_sync(fwpkm_state* st, void* stream) {
     // the word is cleared before the host copy, so a kernel still running on another
     // stream can only leave both set again
     if (cudaMemset(st->wk.status, 0, sizeof(int)) != cudaSuccess) return last_cuda();
+    // a kernel that gave up may have left arrival counters between launches non-zero
+    if (h == DEV_TIMEOUT && st->wk.af_cnt &&
+        cudaMemset(st->wk.af_cnt, 0, sizeof(int) * 4 * (size_t)st->dm.M) != cudaSuccess)
+      return last_cuda();
     if (st->hstat) *(volatile int*)st->hstat = DEV_OK;
     return status_of_device(h);
   }

@@ -40,7 +40,7 @@ int take_test_stall();
 // Kernel kinds for the launch counter / per-kernel timing.
 enum KernelKind : int { KK_NONE = 0, KK_GATHER = 1, KK_WRITE = 2, KK_SCORE = 3, KK_CART = 4,
                         KK_SORT = 5, KK_ADDR = 6, KK_OTHER = 7, KK_TOPK = 8, KK_PREP = 9, KK_PBAR = 10,
-                        KK_WBUILD = 11, KK_LAST = 11 };
+                        KK_WBUILD = 11, KK_FUSED = 12, KK_LAST = 12 };
 
 struct Dims {
   int n, h, d, dv, k, C, M;
@@ -81,6 +81,8 @@ struct Work {
   int qt_T;          // token columns of Qt (a multiple of 64)
   float* wsum_part;  // [M*2][Cpad/16][n]  per-16-token-block sums of W
   int* pbar_cnt;     // [M*2][ceil(n/256)] arrival counters of the pbar column blocks (zero between launches)
+  float* af_part;    // [M*2][n/128][2][256] one-launch addressing: every CTA's partial Z_t and L_t
+  int* af_cnt;       // [M*2][2]           its arrival counters (zero between launches)
   // Every array above is memory-major except the bf16 pieces (Kpc, Wt), whose piece
   // stride is P_all problems; a Work for a group of memories is the same carve with its
   // pointers advanced to the group's first memory (see group_work).
@@ -203,6 +205,21 @@ int launch_tc_pbar(const Dims& d, const Work& w, int len, cudaStream_t s);
 int launch_tc_wbuild(const Dims& d, const Work& w, int len, cudaStream_t s);
 int launch_tc_keystep(const Dims& d, const Work& w, float* K1, float* K2, const void* q, long long q_stride, int len,
                       int qt_t0, cudaStream_t s);
+
+// ---- fused addressing (addr_fused.cu) ----
+// Whether the key-update path takes the one-launch addressing step of a chunk (bf16 q,
+// d/2 in {64, 128}, n a multiple of 128, C <= 256 and a multiple of 16, and the launch's
+// 2 M n / 128 CTAs no more than the GPU's SMs; FWPKM_FUSED_ADDR=0 turns it off).
+bool use_fused_addressing(const Dims& d);
+// Distances of `len` tokens (workspace tokens wt0.., half-query rows q_row0.. of a map over
+// q_base with q_extent rows per memory, q_stride tokens apart) into Dfull rows 0..len-1,
+// then (unless score_only) the whole entropy key step of those tokens: K1, K2, their bf16
+// pieces and squared norms updated in place.  The chunk's feature-major half-queries are
+// read from Qt columns qt_x0.. .  One launch of n/128 CTAs per problem (one per SM).
+int launch_addr_fused(const Dims& d, const Work& w, float* K1, float* K2, const void* q_base, long long q_stride,
+                      int q_extent, int q_row0, int wt0, int len, int qt_x0, bool score_only, cudaStream_t s);
+// Floats of the partial-sum buffer (af_part) for the memories of `d`.
+size_t addr_fused_part_floats(const Dims& d);
 
 // ---- launches ----
 // Whether kernels are launched with programmatic dependent launch (FWPKM_PDL=1; off by

@@ -222,9 +222,9 @@ int launch_cartesian(const Dims& d, const Work& w, int wt0, int len, int32_t* id
 // the bucket offsets), keeps the keys of its own share of the buckets in shared
 // memory, and one warp per bucket ranks each key by comparing it with every other key
 // of the bucket and stores it at its rank.  The scatter into buckets may land keys in
-// any order; ranking by the full unique key makes the output independent of it.  If a
-// bucket holds more than 128 keys (strongly skewed slot use), the first CTA sorts all
-// keys with a register bitonic network instead and the others do nothing.
+// any order; ranking by the full unique key makes the output independent of it.  A
+// bucket of more than 128 keys (strongly skewed slot use: a row read by many tokens) is
+// ranked by the whole CTA that owns it instead of one warp.
 // ---------------------------------------------------------------------------
 constexpr int SORT_THREADS = 1024;
 constexpr int SORT_SPLIT = 16;
@@ -238,7 +238,6 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
   pdl_trigger();
   extern __shared__ u64 s_keys[];
   __shared__ int s_cnt[512], s_off[513], s_cur[512];
-  __shared__ int s_max;
   const int m = blockIdx.y;
   const int cc = blockIdx.x / SORT_SPLIT, part = blockIdx.x % SORT_SPLIT;
   const int C = dm.C, k = dm.k;
@@ -276,75 +275,85 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
     x[u] = key;
   }
   __syncthreads();
-  if (warp == 0) {  // exclusive scan of the bucket sizes, and the largest bucket
-    int run = 0, mx = 0;
+  if (warp == 0) {  // exclusive scan of the bucket sizes
+    int run = 0;
     for (int b0 = 0; b0 < NB; b0 += 32) {
       const int v = b0 + lane < NB ? s_cnt[b0 + lane] : 0;
-      int incl = v, vm = v;
+      int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
-        vm = max(vm, __shfl_xor_sync(0xffffffffu, vm, o));
       }
       if (b0 + lane < NB) {
         s_off[b0 + lane] = run + incl - v;
         s_cur[b0 + lane] = run + incl - v;
       }
       run += __shfl_sync(0xffffffffu, incl, 31);
-      mx = max(mx, vm);
     }
-    if (lane == 0) {
-      s_off[NB] = run;
-      s_max = mx;
-    }
+    if (lane == 0) s_off[NB] = run;
   }
   __syncthreads();
   if (part == 0 && tid == 0) w.npairs[cbase] = P;
-  if (s_max <= SORT_BUCKET_CAP) {
-    // this CTA's buckets [b_lo, b_hi) occupy key positions [s_off[b_lo], s_off[b_hi])
-    const int base0 = s_off[b_lo];
+  // this CTA's buckets [b_lo, b_hi) occupy key positions [s_off[b_lo], s_off[b_hi])
+  const int base0 = s_off[b_lo];
 #pragma unroll
-    for (int u = 0; u < VPT; ++u)
-      if (bk[u] >= b_lo && bk[u] < b_hi) s_keys[atomicAdd(&s_cur[bk[u]], 1) - base0] = x[u];
-    __syncthreads();
-    for (int b = b_lo + warp; b < b_hi; b += SORT_THREADS / 32) {
-      const int base = s_off[b] - base0, cnt = s_off[b + 1] - s_off[b];
-      if (cnt == 0) continue;
-      u64 mine[SORT_BUCKET_CAP / 32];
-      int rk[SORT_BUCKET_CAP / 32];
+  for (int u = 0; u < VPT; ++u)
+    if (bk[u] >= b_lo && bk[u] < b_hi) s_keys[atomicAdd(&s_cur[bk[u]], 1) - base0] = x[u];
+  __syncthreads();
+  // buckets of up to SORT_BUCKET_CAP keys: one warp each, every key ranked against the others
+  for (int b = b_lo + warp; b < b_hi; b += SORT_THREADS / 32) {
+    const int base = s_off[b] - base0, cnt = s_off[b + 1] - s_off[b];
+    if (cnt == 0 || cnt > SORT_BUCKET_CAP) continue;
+    u64 mine[SORT_BUCKET_CAP / 32];
+    int rk[SORT_BUCKET_CAP / 32];
 #pragma unroll
-      for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j) {
-        const int i = lane + 32 * j;
+    for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j) {
+      const int i = lane + 32 * j;
+      mine[j] = i < cnt ? s_keys[base + i] : ~0ull;
+      rk[j] = 0;
+    }
+    if (cnt <= 64) {
+      for (int t = 0; t < cnt; ++t) {
+        const u64 o = s_keys[base + t];
+        rk[0] += o < mine[0] ? 1 : 0;
+        rk[1] += o < mine[1] ? 1 : 0;
+      }
+    } else {
+      for (int t = 0; t < cnt; ++t) {
+        const u64 o = s_keys[base + t];
+#pragma unroll
+        for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j) rk[j] += o < mine[j] ? 1 : 0;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j)
+      if (lane + 32 * j < cnt) out[s_off[b] + rk[j]] = mine[j];
+  }
+  // larger buckets (skewed slot use: a row read by many tokens of the chunk): the whole CTA
+  // ranks each one, every thread a strided share of its keys against all of them (the
+  // comparison reads are broadcasts); the output is the same as the warps' ranking
+  for (int b = b_lo; b < b_hi; ++b) {
+    const int base = s_off[b] - base0, cnt = s_off[b + 1] - s_off[b];
+    if (cnt <= SORT_BUCKET_CAP) continue;
+    for (int i0 = 0; i0 < cnt; i0 += 4 * SORT_THREADS) {
+      u64 mine[4];
+      int rk[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + tid + j * SORT_THREADS;
         mine[j] = i < cnt ? s_keys[base + i] : ~0ull;
         rk[j] = 0;
       }
-      if (cnt <= 64) {
-        for (int t = 0; t < cnt; ++t) {
-          const u64 o = s_keys[base + t];
-          rk[0] += o < mine[0] ? 1 : 0;
-          rk[1] += o < mine[1] ? 1 : 0;
-        }
-      } else {
-        for (int t = 0; t < cnt; ++t) {
-          const u64 o = s_keys[base + t];
+      for (int t = 0; t < cnt; ++t) {
+        const u64 o = s_keys[base + t];
 #pragma unroll
-          for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j) rk[j] += o < mine[j] ? 1 : 0;
-        }
+        for (int j = 0; j < 4; ++j) rk[j] += o < mine[j] ? 1 : 0;
       }
 #pragma unroll
-      for (int j = 0; j < SORT_BUCKET_CAP / 32; ++j)
-        if (lane + 32 * j < cnt) out[s_off[b] + rk[j]] = mine[j];
+      for (int j = 0; j < 4; ++j)
+        if (i0 + tid + j * SORT_THREADS < cnt) out[s_off[b] + rk[j]] = mine[j];
     }
-  } else if (part == 0) {
-    block_sort_asc<VPT>(x, s_keys, Ppad);
-    if (tid * VPT < Ppad)
-#pragma unroll
-      for (int u = 0; u < VPT; ++u)
-        if (tid * VPT + u < P) out[tid * VPT + u] = x[u];
-  } else {
-    // the skewed fallback is handled by the first CTA; nothing to do here (the bitonic
-    // sort needs every thread of its CTA, so it is taken as a whole or not at all)
   }
 }
 

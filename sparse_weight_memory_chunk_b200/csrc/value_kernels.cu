@@ -11,6 +11,7 @@
 // Rows are moved as 16-byte vectors: a warp covers 512 contiguous bytes per load.  Both
 // kernels are bound by HBM latency x bytes in flight, so each warp keeps many row loads
 // outstanding before it consumes any of them.
+#include <climits>
 #include <cstdlib>
 #include <mutex>
 
@@ -329,18 +330,177 @@ write_kernel(Dims dm, Work w, float* __restrict__ V, int wt0) {
         key = sk[p];
         if ((int)(key >> 32) != slot) break;
       }
-      const float nr = (float)(p - (pos0 + gi));
+      const float inv = 1.f / (float)(p - (pos0 + gi));
       float4* row = reinterpret_cast<float4*>(Vm + (size_t)slot * dm.dv);
 #pragma unroll
       for (int c = 0; c < VPL; ++c) {
         const int e4 = lane + 32 * c;
         if (e4 < dv4) {
           float4 x = Vr[gi][c];
-          x.x -= Gs[c].x / nr; x.y -= Gs[c].y / nr; x.z -= Gs[c].z / nr; x.w -= Gs[c].w / nr;
+          x.x = fmaf(-Gs[c].x, inv, x.x); x.y = fmaf(-Gs[c].y, inv, x.y);
+          x.z = fmaf(-Gs[c].z, inv, x.z); x.w = fmaf(-Gs[c].w, inv, x.w);
           row[e4] = x;
         }
       }
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Write, batched: each warp owns a contiguous range [r0, r1) of one memory's sorted pair
+// list and every segment (touched row) whose first pair lies in it, even where the
+// segment runs past r1; positions before its first head belong to a peer's segment.  The
+// warp reads the list in windows of 32 positions (one key per lane and the key before it,
+// in one round trip: a position is a segment head where the slot changes) and consumes
+// each window in batches of WB positions: it issues the residual-row and weight loads of
+// the batch's pairs and the V-row loads of the segments that start in it, all at once,
+// then accumulates G_i = sum s'_{t,i} r_t in list order (token order within a segment) and
+// stores V_i - G_i / N_read,i at each segment's last pair.  A segment still open at the end
+// of a window is carried (V row, partial sum, count) into the next window, so the additions
+// happen in the same order as in a serial walk of the segment.
+// ---------------------------------------------------------------------------
+constexpr int WR_WARPS = 4;
+
+template <int VPL>
+__device__ __forceinline__ void store_row(float* Vm, int slot, const Dims& dm, const float4 (&cv)[VPL],
+                                          const float4 (&acc)[VPL], int nr, int lane) {
+  float4* row = reinterpret_cast<float4*>(Vm + (size_t)slot * dm.dv);
+  // one reciprocal per row (exact for the common N_read = 1, 2, 4)
+  const float inv = 1.f / (float)nr;
+  const int dv4 = dm.dv >> 2;
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) {
+    const int e4 = lane + 32 * c;
+    if (e4 < dv4) {
+      float4 x = cv[c];
+      x.x = fmaf(-acc[c].x, inv, x.x); x.y = fmaf(-acc[c].y, inv, x.y);
+      x.z = fmaf(-acc[c].z, inv, x.z); x.w = fmaf(-acc[c].w, inv, x.w);
+      row[e4] = x;
+    }
+  }
+}
+
+template <int VPL, int WB>
+__global__ void __launch_bounds__(WR_WARPS * 32)
+write_batched_kernel(Dims dm, Work w, float* __restrict__ V, int wt0, int warps_per_mem) {
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * WR_WARPS + warp;
+  const int m = gw / warps_per_mem, wi = gw - m * warps_per_mem;
+  if (m >= dm.M) return;
+  const int C = dm.C, k = dm.k, dv4 = dm.dv >> 2;
+  const int kshift = (k & (k - 1)) == 0 ? __popc(k - 1) : -1;
+  const size_t cbase = (size_t)m * w.max_chunks + wt0 / C;
+  const int P = w.npairs[cbase];
+  const int r0 = (int)((long long)P * wi / warps_per_mem), r1 = (int)((long long)P * (wi + 1) / warps_per_mem);
+  if (r0 >= r1) return;
+  const unsigned long long* sk = w.sk + cbase * (size_t)(C * k);
+  const float* wrow = w.w + ((size_t)m * w.max_T + wt0) * k;
+  const float4* resid = reinterpret_cast<const float4*>(w.resid + (size_t)m * C * dm.dv);
+  float* Vm = V + (size_t)m * dm.N * dm.dv;
+  // the open segment: cur = its slot (-1: none open; -2: a slot outside [0, N), skipped),
+  // its V row cv, partial sum acc and pair count nr
+  int cur = -1, nr = 0;
+  float4 cv[VPL], acc[VPL];
+#pragma unroll
+  for (int c = 0; c < VPL; ++c) cv[c] = acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  bool started = false;
+  for (int pos0 = r0; pos0 < P; pos0 += 32) {
+    const int pos = pos0 + lane;
+    unsigned long long key = ~0ull, prv = ~0ull;
+    if (pos < P) {
+      key = sk[pos];
+      if (pos > 0) prv = sk[pos - 1];
+    }
+    const bool head = pos < P && (pos == 0 || (prv >> 32) != (key >> 32));
+    const unsigned hm = __ballot_sync(0xffffffffu, head);
+    // the segment carried from the previous window ends before this window's first head
+    if (cur != -1 && (hm & 1u)) {
+      if (cur >= 0) store_row<VPL>(Vm, cur, dm, cv, acc, nr, lane);
+      cur = -1;
+    }
+    // heads at positions >= r1 start peers' segments: the first of them ends this warp's work
+    const int rel = r1 - pos0;
+    const unsigned beyond = rel >= 32 ? 0u : (rel <= 0 ? 0xffffffffu : (0xffffffffu << rel));
+    const unsigned stop_heads = hm & beyond;
+    const int stop = stop_heads ? pos0 + __ffs(stop_heads) - 1 : P;  // first position not this warp's
+    int first = 0;
+    if (!started) {
+      if (!hm) {
+        if (rel <= 32) break;  // no head left in [r0, r1): the range is a peer's tail
+        continue;
+      }
+      first = __ffs(hm) - 1;
+      if (pos0 + first >= r1) break;  // likewise
+      started = true;
+    }
+    const int lim = stop - pos0 < 32 ? stop - pos0 : 32;  // positions [first, lim) of this window are ours
+#pragma unroll 1
+    for (int b0 = first; b0 < lim; b0 += WB) {
+      // ---- issue every load of the batch ----
+      float4 R[WB][VPL], Vh[WB][VPL];
+      float wt[WB];
+#pragma unroll
+      for (int u = 0; u < WB; ++u) {
+        const int l = b0 + u;
+        const bool in = l < lim;
+        const unsigned long long ku = __shfl_sync(0xffffffffu, key, l & 31);
+        const bool hd = in && ((hm >> (l & 31)) & 1u);
+        const uint32_t tr = (uint32_t)(ku & 0xffffffffu);
+        const int slot = (int)(ku >> 32);
+        const bool okslot = slot >= 0 && (long long)slot < dm.N;
+        const int t_local = kshift >= 0 ? (int)(tr >> kshift) : (int)(tr / (uint32_t)k);
+        wt[u] = in ? wrow[tr] : 0.f;
+        const float4* rr = resid + (size_t)(in ? t_local : 0) * dv4;
+        const float4* vr = reinterpret_cast<const float4*>(Vm + (size_t)(hd && okslot ? slot : 0) * dm.dv);
+#pragma unroll
+        for (int c = 0; c < VPL; ++c) {
+          const int e4 = lane + 32 * c;
+          R[u][c] = (in && e4 < dv4) ? rr[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+          Vh[u][c] = (hd && okslot && e4 < dv4) ? vr[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      // ---- accumulate in list order; a segment is stored at its last pair ----
+#pragma unroll
+      for (int u = 0; u < WB; ++u) {
+        const int l = b0 + u;
+        if (l >= lim) break;
+        if ((hm >> l) & 1u) {
+          const int slot = (int)(__shfl_sync(0xffffffffu, key, l) >> 32);
+          if (slot < 0 || (long long)slot >= dm.N) {
+            if (lane == 0) raise_status(w.status, w.hstat, DEV_BAD_SLOT);
+            cur = -2;
+          } else {
+            cur = slot;
+#pragma unroll
+            for (int c = 0; c < VPL; ++c) {
+              cv[c] = Vh[u][c];
+              acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            nr = 0;
+          }
+        }
+        if (cur >= 0) {
+          const float a = wt[u];
+#pragma unroll
+          for (int c = 0; c < VPL; ++c) {
+            acc[c].x = fmaf(a, R[u][c].x, acc[c].x); acc[c].y = fmaf(a, R[u][c].y, acc[c].y);
+            acc[c].z = fmaf(a, R[u][c].z, acc[c].z); acc[c].w = fmaf(a, R[u][c].w, acc[c].w);
+          }
+          ++nr;
+        }
+        // the segment ends at this pair if the next position starts another one or the list
+        // ends; at the window's last position the next head is only known in the next window
+        const int nx = pos0 + l + 1;
+        const bool ends = nx >= P || (l < 31 && ((hm >> (l + 1)) & 1u));
+        if (ends && cur != -1) {
+          if (cur >= 0) store_row<VPL>(Vm, cur, dm, cv, acc, nr, lane);
+          cur = -1;
+        }
+      }
+    }
+    if (lim < 32) break;  // a peer's head (or the list's end) was reached in this window
   }
 }
 
@@ -444,20 +604,14 @@ static int resident_ctas(const void* kern, int threads) {
   return v;
 }
 
-int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s) {
+// The per-position write (FWPKM_WRITE_V1=1): each warp walks whole segments from G list
+// positions with a dependent load per pair; kept to measure against the batched write.
+static int launch_write_v1(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s) {
   const int vpl = vpl_of(d.dv);
-  const int G = vpl <= 2 ? 4 : vpl == 4 ? 2 : 1;  // list positions per warp: ~8 float4 in flight per lane
-  const int need = (d.C * d.k + VAL_WARPS * G - 1) / (VAL_WARPS * G);  // CTAs per memory for one pass
-  // the grid is a fraction of one resident wave (FWPKM_WRITE_SHARE percent, default 50): the
-  // write runs beside the addressing chain of the next chunk, and a smaller footprint
-  // leaves that chain more of the GPU
-  static const int share = [] {
-    const char* e = getenv("FWPKM_WRITE_SHARE");
-    const int v = e ? atoi(e) : 50;
-    return v < 5 ? 5 : v > 100 ? 100 : v;
-  }();
+  const int G = vpl <= 2 ? 4 : vpl == 4 ? 2 : 1;
+  const int need = (d.C * d.k + VAL_WARPS * G - 1) / (VAL_WARPS * G);
   auto grid_for = [&](int resident) {
-    const int per_mem = ((long long)resident * share / 100 + d.M - 1) / d.M;
+    const int per_mem = (resident / 2 + d.M - 1) / d.M;
     return dim3(need < per_mem ? need : (per_mem < 1 ? 1 : per_mem), d.M);
   };
   switch (vpl) {
@@ -465,6 +619,38 @@ int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s
     case 2: launch_k(write_kernel<2, 4>, grid_for(resident_ctas((const void*)write_kernel<2, 4>, VAL_WARPS * 32)), VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
     case 4: launch_k(write_kernel<4, 2>, grid_for(resident_ctas((const void*)write_kernel<4, 2>, VAL_WARPS * 32)), VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
     default: launch_k(write_kernel<8, 1>, grid_for(resident_ctas((const void*)write_kernel<8, 1>, VAL_WARPS * 32)), VAL_WARPS * 32, 0, s, d, w, V, wt0); break;
+  }
+  return 1;
+}
+
+int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s) {
+  static const bool v1 = [] {
+    const char* e = getenv("FWPKM_WRITE_V1");
+    return e && e[0] == '1';
+  }();
+  if (v1) return launch_write_v1(d, w, V, wt0, s);
+  const int vpl = vpl_of(d.dv);
+  // one warp per ~32 positions of a memory's list at most, and no more warps than fit on the
+  // GPU at once (FWPKM_WRITE_SHARE percent of them, default 100)
+  static const int share = [] {
+    const char* e = getenv("FWPKM_WRITE_SHARE");
+    const int v = e ? atoi(e) : 100;
+    return v < 5 ? 5 : v > 100 ? 100 : v;
+  }();
+  auto go = [&](const void* kern, auto kfn) {
+    const int resident_warps = resident_ctas(kern, WR_WARPS * 32) * WR_WARPS;
+    int per_mem = (int)((long long)resident_warps * share / 100 / d.M);
+    const int most = (d.C * d.k + 31) / 32;
+    if (per_mem > most) per_mem = most;
+    if (per_mem < 1) per_mem = 1;
+    const int blocks = (d.M * per_mem + WR_WARPS - 1) / WR_WARPS;
+    launch_k(kfn, dim3((unsigned)blocks), WR_WARPS * 32, 0, s, d, w, V, wt0, per_mem);
+  };
+  switch (vpl) {
+    case 1: go((const void*)write_batched_kernel<1, 8>, write_batched_kernel<1, 8>); break;
+    case 2: go((const void*)write_batched_kernel<2, 4>, write_batched_kernel<2, 4>); break;
+    case 4: go((const void*)write_batched_kernel<4, 2>, write_batched_kernel<4, 2>); break;
+    default: go((const void*)write_batched_kernel<8, 1>, write_batched_kernel<8, 1>); break;
   }
   return 1;
 }

@@ -16,8 +16,9 @@ output projection.  Checked, element by element:
   * o' against the oracle's output projection of the call's o.
 Skewed slot use is what these inputs are for, so the test also asserts that it reached
 the two skew paths of the write: a chunk whose (slot, token) pairs overflow one hash
-bucket of the pair sort (more than 128 keys: the sort's single-CTA fallback), and, in
-the hot variant, a row read by at least half the chunk's tokens.
+bucket of the pair sort (more than 128 keys: ranked by a whole CTA instead of a warp),
+and, in the hot variant, a row read by at least half the chunk's tokens (one segment of
+the write carried across many batches and windows of its warp).
 """
 import numpy as np
 import pytest
@@ -113,7 +114,7 @@ def test_run_layer_matches_oracle_chain(variant):
             max_bucket = max(max_bucket, int(bucket_sizes(slots).max()))
             max_nread = max(max_nread, int(np.unique(slots, return_counts=True)[1].max()))
     print(f"layer chain ({variant}): largest sort bucket {max_bucket}, largest N_read {max_nread}")
-    assert max_bucket > SORT_BUCKET_CAP, "no chunk reached the pair sort's skewed fallback"
+    assert max_bucket > SORT_BUCKET_CAP, "no chunk reached the pair sort's oversized-bucket path"
     if variant == "hot":
         assert max_nread >= C // 2, "no row was read by half a chunk's tokens"
 
