@@ -14,8 +14,9 @@
 // [128c, 128c + 128) and every token of the chunk, so
 //   * the distance tile D^T[b][t] (128 sub-keys x len tokens, fp32) comes out of the
 //     scoring MMA (A = the keys' three bf16 pieces, B = the chunk's half-queries) into
-//     tensor memory; the first epilogue pass writes the distance rows for the selection and
-//     puts w = 1/(eps + D) back in the same tensor-memory columns for the later passes;
+//     tensor memory; the first epilogue pass stages it in shared memory for one TMA store
+//     into the rows the selection reads, and puts w = 1/(eps + D) back in the same
+//     tensor-memory columns for the later passes;
 //   * pbar, log pbar, W, sum_t W and the key update are local to the CTA (its sub-keys
 //     over all tokens); only Z_t and L_t are sums over all n sub-keys: each CTA reduces its
 //     128 across TMEM lanes (warp butterflies, then the four lane quarters in order),
@@ -27,7 +28,8 @@
 //     lands in tensor memory beside w.
 // The distance rows go to global memory once (the selection reads them); apart from two
 // small partial vectors per CTA nothing else of the step leaves the chip except the new
-// keys, their bf16 pieces and squared norms.
+// keys, their bf16 pieces and squared norms, staged in shared memory and written by
+// per-row bulk copies.
 //
 // Roles: warp 0 issues TMA loads, warp 1 owns tensor memory and issues the MMAs (one
 // thread), warps 2-17 are the epilogue: warp w reads TMEM lane quarter w % 4 (sub-keys
@@ -131,7 +133,7 @@ __device__ __forceinline__ void arrive_and_wait(int* cnt, int target, int et, vo
 
 __global__ void __launch_bounds__(AF_THREADS, 1)
 addr_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                  const __grid_constant__ CUtensorMap tmQt, AddrFused a) {
+                  const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmD, AddrFused a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   float* s_part = (float*)(smem + a.off_small);   // [4][AF_MAX_C] per-lane-quarter column sums
@@ -269,7 +271,9 @@ addr_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     int ok = lane == 0 ? (mbar_wait(accf, 0, abort_flag, deadline) ? 1 : 0) : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (ok) tc_fence_after();
-    float* Drow = a.Dfull + (size_t)p * a.d_pstride + b;
+    // the distance tile [npad][128] fp32, row-major, over the consumed scoring operands;
+    // one TMA store writes it to the rows the selection reads
+    float* sD = reinterpret_cast<float*>(smem);
 
     // pass 1: distances (rows for the selection), w back into tensor memory (0 past len),
     // and the CTA's partial Z_t
@@ -283,7 +287,7 @@ addr_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         for (int i = 0; i < 32; ++i) {
           const int t = 32 * g + i;
           const float D = fmaxf((s_qn[t] + knb) - 2.f * __uint_as_float(v[i]), 0.f);
-          if (t < len) Drow[(size_t)t * n] = D;
+          if (t < a.npad) sD[t * 128 + bl] = D;
           x[i] = t < len ? __fdividef(1.f, eps + D) : 0.f;
           v[i] = __float_as_uint(x[i]);
         }
@@ -297,8 +301,13 @@ addr_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       }
       if (!a.score_only) s_part[q * AF_MAX_C + 32 * g + lane] = col_sums32(x, lane);
     }
+    fence_async_smem();
+    epi_sync();
+    if (et == 0 && ok) {
+      tma_store_3d(&tmD, sD, 128 * c, 0, p);
+      bulk_commit();
+    }
     if (!a.score_only) {
-      epi_sync();
       for (int t = et; t < a.npad; t += AF_EPI_THREADS)
         part[t] = ((s_part[t] + s_part[AF_MAX_C + t]) + s_part[2 * AF_MAX_C + t]) + s_part[3 * AF_MAX_C + t];
       arrive_and_wait(cnt, ncl, et, abort_flag, deadline);  // every CTA's partial Z is published
@@ -350,6 +359,7 @@ addr_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           for (int r = 0; r < ncl; ++r) l += __ldcg(part_p + (size_t)r * 2 * AF_MAX_C + AF_MAX_C + t);
         s_L[t] = l * s_iz[t];
       }
+      if (et == 0) bulk_wait_read();  // the distance tile has been read: pass 4 writes over it
       epi_sync();
       // the problem's counters are read by every CTA before it arrives here: the last CTA
       // to arrive resets them for the next launch
@@ -455,28 +465,25 @@ addr_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         }
       }
       s_kn[cq * 128 + bl] = ss;
+      fence_async_smem();
       epi_sync();
       if (okg) {
-        // the CTA's 128 rows of K (128 h fp32) and of each piece (128 h bf16), consecutive
-        // threads on consecutive 16-byte words
-        float* Kt = (jh == 0 ? a.K1 : a.K2) + ((size_t)m * n + 128 * c) * h;
-        const int h4 = h >> 2, h8 = h >> 3;
-        for (int j = et; j < 128 * h4; j += AF_EPI_THREADS) {
-          const int r = j / h4, c4 = j - r * h4;
-          *reinterpret_cast<float4*>(Kt + (size_t)r * h + 4 * c4) =
-              *reinterpret_cast<const float4*>(sK + (size_t)r * kstr + 4 * c4);
+        // the CTA's 128 rows of K (h fp32 each) and of each bf16 piece (h each): one bulk
+        // copy per row, one row per epilogue thread
+        const int arr = et >> 7, r = et & 127;
+        if (arr == 0) {
+          float* Kt = (jh == 0 ? a.K1 : a.K2) + ((size_t)m * n + 128 * c + r) * h;
+          bulk_store(Kt, sK + (size_t)r * kstr, (uint32_t)(h * 4));
+        } else {
+          const size_t pstride = (size_t)a.P_all * n * h;
+          __nv_bfloat16* Pt = a.Kpc + (arr - 1) * pstride + ((size_t)p * n + 128 * c + r) * h;
+          bulk_store(Pt, sP + (size_t)((arr - 1) * 128 + r) * pstr, (uint32_t)(h * 2));
         }
-        const size_t pstride = (size_t)a.P_all * n * h;
-        __nv_bfloat16* Pt = a.Kpc + ((size_t)p * n + 128 * c) * h;
-        for (int j = et; j < 3 * 128 * h8; j += AF_EPI_THREADS) {
-          const int pc = j / (128 * h8), rem = j - pc * 128 * h8;
-          const int r = rem / h8, c8 = rem - r * h8;
-          *reinterpret_cast<uint4*>(Pt + pc * pstride + (size_t)r * h + 8 * c8) =
-              *reinterpret_cast<const uint4*>(sP + (size_t)(pc * 128 + r) * pstr + 8 * c8);
-        }
+        bulk_commit();
         if (cq == 0) a.kn[(size_t)p * n + b] = ((s_kn[bl] + s_kn[128 + bl]) + s_kn[256 + bl]) + s_kn[384 + bl];
       }
     }
+    bulk_wait_read();  // this thread's bulk stores have read shared memory (no-op if none)
   }
 
   // ---------------- teardown ----------------
@@ -559,6 +566,12 @@ int launch_addr_fused(const Dims& d, const Work& w, float* K1, float* K2, const 
   } else {
     tQt = tQ;  // unused
   }
+  // distance rows [P][drows][n] fp32: each CTA stores a box of 128 sub-keys x npad tokens
+  const int npad = (len + 15) / 16 * 16;
+  CUtensorMap tD;
+  if (!make_tmap_f32_3d(&tD, w.Dfull, d.n, w.drows, P, (uint64_t)d.n * 4, (uint64_t)w.drows * d.n * 4, 128,
+                        (uint32_t)npad))
+    return -1;
   AddrFused a = {};
   a.n = d.n; a.h = d.h; a.len = len;
   a.npad = (len + 15) / 16 * 16;
@@ -584,7 +597,7 @@ int launch_addr_fused(const Dims& d, const Work& w, float* K1, float* K2, const 
   a.status = w.status; a.hstat = w.hstat;
   a.stall = take_test_stall();
   if (!raise_smem_limit((const void*)addr_fused_kernel, smem)) return -1;
-  launch_k(addr_fused_kernel, dim3((unsigned)(d.n / 128), (unsigned)P, 1), AF_THREADS, smem, s, tK, tQ, tQt, a);
+  launch_k(addr_fused_kernel, dim3((unsigned)(d.n / 128), (unsigned)P, 1), AF_THREADS, smem, s, tK, tQ, tQt, tD, a);
   return 1;
 }
 

@@ -790,11 +790,12 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
   } else {
     const size_t dbuf = (size_t)wk.dfull_buf;
     std::vector<cudaEvent_t> topk_done(2, nullptr), sel_done(nch, nullptr), val_done(nch, nullptr);
-    // FWPKM_SEL_FIRST=1: the addressing of chunk c+1 also waits for the selection of chunk c
-    // (the selection then runs beside the value kernels rather than beside the addressing)
+    // The addressing of chunk c+1 also waits for the selection of chunk c, so the selection
+    // runs beside the value kernels rather than beside the addressing, which occupies most
+    // SMs (paper-scale step 1.453 against 1.555 ms); FWPKM_SEL_FIRST=0 lets them overlap.
     static const bool sel_first = [] {
       const char* e = getenv("FWPKM_SEL_FIRST");
-      return e && e[0] == '1';
+      return !(e && e[0] == '0');
     }();
     cudaEvent_t last_topk = nullptr;
     int cnt = 0;

@@ -130,6 +130,8 @@ struct TcGemm {
 
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z, uint64_t pitch_y,
                        uint64_t pitch_z);
+bool make_tmap_f32_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z, uint64_t pitch_y,
+                      uint64_t pitch_z, uint32_t box_x, uint32_t box_y);
 int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g, int m_tiles, cudaStream_t s);
 
 // stream_stage: also carve the staging rows of token-at-a-time inference (at the end).

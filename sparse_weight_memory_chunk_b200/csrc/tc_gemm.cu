@@ -409,6 +409,23 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
+// fp32 tensor [z][y][x] (pitches in bytes), box box_x x box_y x 1, no swizzle: the
+// shared-memory side of a copy is the dense box, row-major.
+bool make_tmap_f32_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z, uint64_t pitch_y,
+                      uint64_t pitch_z, uint32_t box_x, uint32_t box_y) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {x, y, z};
+  cuuint64_t strides[2] = {pitch_y, pitch_z};
+  cuuint32_t box[3] = {box_x, box_y, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) fprintf(stderr, "fwpkm: cuTensorMapEncodeTiled (fp32) failed (%d)\n", (int)r);
+  return r == CUDA_SUCCESS;
+}
+
 int launch_tc_gemm(const CUtensorMap& A, const CUtensorMap& B, const TcGemm& g0, int m_tiles, cudaStream_t s) {
   TcGemm g = g0;
   const int npc = g.a_pieces + g.b_pieces;

@@ -524,11 +524,11 @@ int launch_gather(const Dims& d, const Work& w, const float* V, const void* v, c
   if (len <= 0) return 0;
   dim3 grid((len + GATHER_TOK - 1) / GATHER_TOK, d.M);
   if (d.qv_bf16) {
-    FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(gather_kernel<__nv_bfloat16, VPL>, grid, VAL_WARPS * 32, 0, s, 
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(gather_kernel<__nv_bfloat16, VPL>, grid, VAL_WARPS * 32, 0, s,
         d, w, V, (const __nv_bfloat16*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0,
         (const __nv_bfloat16*)v_next));
   } else {
-    FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(gather_kernel<float, VPL>, grid, VAL_WARPS * 32, 0, s, 
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(gather_kernel<float, VPL>, grid, VAL_WARPS * 32, 0, s,
         d, w, V, (const float*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0, (const float*)v_next));
   }
   return 1;
