@@ -66,6 +66,7 @@ def _load():
         _lib.orc_target.argtypes = [ctypes.POINTER(Cfg), P, P]
         _lib.orc_chunk.argtypes = [ctypes.POINTER(Cfg), ctypes.c_int] + [P] * 12
         _lib.orc_run_sequence.argtypes = [ctypes.POINTER(Cfg), ctypes.c_int, ctypes.c_int] + [P] * 9
+        _lib.orc_chunk_heads.argtypes = [ctypes.POINTER(Cfg), ctypes.c_int, ctypes.c_int] + [P] * 12
         _lib.orc_run_sequence_multi.argtypes = ([ctypes.POINTER(Cfg), ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_int] + [P] * 8 + [ctypes.c_int])
         _lib.orc_run_sequence_multi.restype = ctypes.c_int
@@ -134,6 +135,38 @@ def chunk(cfg: Cfg, q, v, g, v_next, K1, K2, V, forced=None, force_mask=None):
     fm = None if force_mask is None else np.ascontiguousarray(force_mask, dtype=np.int32)
     _load().orc_chunk(ctypes.byref(cfg), length, _p(q), _p(v), _p(g), _p(vn), _p(_f32(K1)),
                       _p(_f32(K2)), _p(_f32(V)), _p(o), _p(I), _p(w), _p(f), _p(fm))
+    return o, I, w
+
+
+def chunk_heads(cfg: Cfg, q, v, g, v_next, K1, K2, V, forced=None, force_mask=None):
+    """One chunk of H heads sharing one value table (fwpkm_oracle.c, orc_chunk_heads).
+
+    q [H][len][d]; v [len][d_v], g [len], v_next [d_v] or None (the sequence's);
+    K1, K2 [H][n][h] and V [N][d_v] fp32, updated in place; forced [H][len][k] and
+    force_mask [H][len] optional.  Returns (o [len][d_v], I [H][len][k], w [H][len][k])."""
+    q = _f64(q); v = _f64(v); g = _f64(g)
+    vn = None if v_next is None else _f64(v_next)
+    H, length = q.shape[0], q.shape[1]
+    o = np.empty((length, cfg.d_v)); I = np.empty((H, length, cfg.k), np.int32)
+    w = np.empty((H, length, cfg.k))
+    f = None if forced is None else np.ascontiguousarray(forced, dtype=np.int32)
+    fm = None if force_mask is None else np.ascontiguousarray(force_mask, dtype=np.int32)
+    _load().orc_chunk_heads(ctypes.byref(cfg), H, length, _p(q), _p(v), _p(g), _p(vn), _p(_f32(K1)), _p(_f32(K2)),
+                            _p(_f32(V)), _p(o), _p(I), _p(w), _p(f), _p(fm))
+    return o, I, w
+
+
+def run_sequence_heads(cfg: Cfg, q, v, g, K1, K2, V, n_iter=1):
+    """A whole sequence of H heads sharing V: chunk after chunk (lookahead v_next = the next
+    chunk's first value), n_iter passes.  Returns the final pass's (o, I, w)."""
+    q = _f64(q); v = _f64(v); g = _f64(g)
+    H, T = q.shape[0], q.shape[1]
+    o = np.empty((T, cfg.d_v)); I = np.empty((H, T, cfg.k), np.int32); w = np.empty((H, T, cfg.k))
+    for _ in range(n_iter):
+        for t0 in range(0, T, cfg.chunk):
+            t1 = min(T, t0 + cfg.chunk)
+            vn = v[t1] if t1 < T else None
+            o[t0:t1], I[:, t0:t1], w[:, t0:t1] = chunk_heads(cfg, q[:, t0:t1], v[t0:t1], g[t0:t1], vn, K1, K2, V)
     return o, I, w
 
 

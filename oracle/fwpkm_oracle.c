@@ -222,6 +222,53 @@ static void* orc_read_range(void* arg) {
   return NULL;
 }
 
+/* ---------------------------------------------------------------------------
+ * Addressing step of one chunk of one memory ([R] step 5; [P] §3.4):
+ * L_addr = -H(pbar_1) - H(pbar_2) with pbar_j the chunk mean of
+ * P_j[t] = softmax_a(sigma_j[t][a]) over all n sub-keys, taken at the keys the chunk
+ * was read with (D1, D2: the chunk's distance rows).  One gradient step of size lr_key
+ * on K1, K2.
+ * ------------------------------------------------------------------------- */
+static void orc_key_step(const orc_cfg* c, int len, const double* q, const double* D1, const double* D2,
+                         float* K1, float* K2) {
+  const int n = c->n, h = c->h, d = 2 * h;
+  double* P = (double*)malloc(sizeof(double) * (size_t)len * n);
+  double* pbar = (double*)malloc(sizeof(double) * n);
+  double* lp = (double*)malloc(sizeof(double) * n);
+  double* gradK = (double*)malloc(sizeof(double) * (size_t)n * h);
+  for (int j = 0; j < 2; ++j) {
+    const double* Dj = j == 0 ? D1 : D2;
+    float* Kj = j == 0 ? K1 : K2;
+    for (int t = 0; t < len; ++t) {
+      double z = 0.0;
+      for (int a = 0; a < n; ++a) z += 1.0 / (c->eps_idw + Dj[(size_t)t * n + a]);
+      for (int a = 0; a < n; ++a) P[(size_t)t * n + a] = (1.0 / (c->eps_idw + Dj[(size_t)t * n + a])) / z;
+    }
+    for (int a = 0; a < n; ++a) {
+      double s = 0.0;
+      for (int t = 0; t < len; ++t) s += P[(size_t)t * n + a];
+      pbar[a] = s / len;
+      lp[a] = log(pbar[a]);
+    }
+    for (size_t x = 0; x < (size_t)n * h; ++x) gradK[x] = 0.0;
+    for (int t = 0; t < len; ++t) {
+      double Lt = 0.0;
+      for (int a = 0; a < n; ++a) Lt += P[(size_t)t * n + a] * lp[a];
+      const double* qj = q + (size_t)t * d + (size_t)j * h;
+      for (int b = 0; b < n; ++b) {
+        /* dL_addr/dsigma_j[t][b] */
+        double gam = P[(size_t)t * n + b] * (lp[b] - Lt) / len;
+        /* dsigma/dK[b] = 2 (q - K[b]) / (eps + D) */
+        double coef = gam * 2.0 / (c->eps_idw + Dj[(size_t)t * n + b]);
+        for (int e = 0; e < h; ++e)
+          gradK[(size_t)b * h + e] += coef * (qj[e] - (double)Kj[(size_t)b * h + e]);
+      }
+    }
+    for (size_t x = 0; x < (size_t)n * h; ++x) Kj[x] = (float)((double)Kj[x] - c->lr_key * gradK[x]);
+  }
+  free(P); free(pbar); free(lp); free(gradK);
+}
+
 /* One chunk with its read phase split over `read_threads` threads (token ranges); the
  * write and the key step follow on the calling thread.  orc_chunk is the one-thread case. */
 static void orc_chunk_threads(const orc_cfg* c, int len, const double* q, const double* v, const double* g,
@@ -307,47 +354,7 @@ static void orc_chunk_threads(const orc_cfg* c, int len, const double* q, const 
     s0 = s1;
   }
 
-  /* ---- addressing ([R] step 5; [P] §3.4) ----
-   * L_addr = -H(pbar_1) - H(pbar_2) with pbar_j the chunk mean of
-   * P_j[t] = softmax_a(sigma_j[t][a]) over all n sub-keys, taken at the keys
-   * the chunk was read with.  One gradient step of size lr_key on K1, K2. */
-  if (c->flags & ORC_KEY_UPDATE) {
-    double* P = (double*)malloc(sizeof(double) * (size_t)len * n);
-    double* pbar = (double*)malloc(sizeof(double) * n);
-    double* lp = (double*)malloc(sizeof(double) * n);
-    double* gradK = (double*)malloc(sizeof(double) * (size_t)n * h);
-    for (int j = 0; j < 2; ++j) {
-      const double* Dj = j == 0 ? D1 : D2;
-      float* Kj = j == 0 ? K1 : K2;
-      for (int t = 0; t < len; ++t) {
-        double z = 0.0;
-        for (int a = 0; a < n; ++a) z += 1.0 / (c->eps_idw + Dj[(size_t)t * n + a]);
-        for (int a = 0; a < n; ++a) P[(size_t)t * n + a] = (1.0 / (c->eps_idw + Dj[(size_t)t * n + a])) / z;
-      }
-      for (int a = 0; a < n; ++a) {
-        double s = 0.0;
-        for (int t = 0; t < len; ++t) s += P[(size_t)t * n + a];
-        pbar[a] = s / len;
-        lp[a] = log(pbar[a]);
-      }
-      for (size_t x = 0; x < (size_t)n * h; ++x) gradK[x] = 0.0;
-      for (int t = 0; t < len; ++t) {
-        double Lt = 0.0;
-        for (int a = 0; a < n; ++a) Lt += P[(size_t)t * n + a] * lp[a];
-        const double* qj = q + (size_t)t * d + (size_t)j * h;
-        for (int b = 0; b < n; ++b) {
-          /* dL_addr/dsigma_j[t][b] */
-          double gam = P[(size_t)t * n + b] * (lp[b] - Lt) / len;
-          /* dsigma/dK[b] = 2 (q - K[b]) / (eps + D) */
-          double coef = gam * 2.0 / (c->eps_idw + Dj[(size_t)t * n + b]);
-          for (int e = 0; e < h; ++e)
-            gradK[(size_t)b * h + e] += coef * (qj[e] - (double)Kj[(size_t)b * h + e]);
-        }
-      }
-      for (size_t x = 0; x < (size_t)n * h; ++x) Kj[x] = (float)((double)Kj[x] - c->lr_key * gradK[x]);
-    }
-    free(P); free(pbar); free(lp); free(gradK);
-  }
+  if (c->flags & ORC_KEY_UPDATE) orc_key_step(c, len, q, D1, D2, K1, K2);
 
   free(D1); free(D2); free(I); free(S); free(w); free(vhat);
   free(r); free(tau); free(is_pair); free(pairs); free(G);
@@ -357,6 +364,138 @@ void orc_chunk(const orc_cfg* c, int len, const double* q, const double* v, cons
                const double* v_next, float* K1, float* K2, float* V, double* o, int32_t* I_out,
                double* w_out, const int32_t* forced, const int32_t* force_mask) {
   orc_chunk_threads(c, len, q, v, g, v_next, K1, K2, V, o, I_out, w_out, forced, force_mask, 1);
+}
+
+/* ---------------------------------------------------------------------------
+ * One chunk of H heads that share one value table ([P] §D.1 ablates the head count
+ * with the slot count; §D.3: more heads raise the collision rate, i.e. heads read one
+ * table).  Readings where the pages are silent:
+ *   - head h has its own codebooks K1^h, K2^h and its own query q^h, and selects its own
+ *     k slots I^h_t with its own softmax weights s'^h_t (steps 1-4 per head);
+ *   - the memory's read is the mean of the heads' reads:
+ *       vhat_t = (1/H) sum_h sum_{i in I^h_t} s'^h_{t,i} V_i
+ *     (all H k weights sum to 1, as for one head reading H k slots), and
+ *     o_t = g_t vhat_t + (1 - g_t) v_t;
+ *   - the write is the gradient of L_mem = 1/2 sum_t g_t ||tau_t - vhat_t||^2 with
+ *     respect to the shared rows, G_i = sum_t sum_h [i in I^h_t] (s'^h_{t,i} / H) r_t,
+ *     divided by N_read,i = the number of the chunk's pair tokens that read row i
+ *     through at least one head; V_i -= G_i / N_read,i;
+ *   - each head's codebooks take their own addressing step (L_addr of that head).
+ *   q [H][len][2h], v [len][d_v], g [len], v_next [d_v] or NULL (per sequence)
+ *   K1, K2 [H][n][h] fp32 (updated), V [n*n][d_v] fp32 (shared, updated)
+ *   o [len][d_v]; I_out [H][len][k], w_out [H][len][k] (nullable)
+ *   forced [H][len][k] and force_mask [H][len] (both nullable): a head-token whose mask is
+ *   non-zero uses the given slot list (near-tie resynchronisation).
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int32_t slot;
+  int32_t t;
+  int32_t hd;
+  int32_t r;
+} orc_hpair;
+
+static int hpair_cmp(const void* x, const void* y) {
+  const orc_hpair* a = (const orc_hpair*)x;
+  const orc_hpair* b = (const orc_hpair*)y;
+  if (a->slot != b->slot) return a->slot < b->slot ? -1 : 1;
+  if (a->t != b->t) return a->t < b->t ? -1 : 1;
+  if (a->hd != b->hd) return a->hd < b->hd ? -1 : 1;
+  return 0;
+}
+
+void orc_chunk_heads(const orc_cfg* c, int H, int len, const double* q, const double* v, const double* g,
+                     const double* v_next, float* K1, float* K2, float* V, double* o, int32_t* I_out,
+                     double* w_out, const int32_t* forced, const int32_t* force_mask) {
+  const int n = c->n, h = c->h, dv = c->d_v, k = c->k, d = 2 * h;
+  const size_t nk = (size_t)n * h;
+  double* D1 = (double*)malloc(sizeof(double) * (size_t)H * len * n);
+  double* D2 = (double*)malloc(sizeof(double) * (size_t)H * len * n);
+  int32_t* I = (int32_t*)malloc(sizeof(int32_t) * (size_t)H * len * k);
+  double* S = (double*)malloc(sizeof(double) * (size_t)H * len * k);
+  double* w = (double*)malloc(sizeof(double) * (size_t)H * len * k);
+  double* vh = (double*)malloc(sizeof(double) * dv);
+  double* vhat = (double*)malloc(sizeof(double) * (size_t)len * dv);
+
+  /* ---- read phase: every head of every token against the frozen state ---- */
+  for (int t = 0; t < len; ++t) {
+    for (int e = 0; e < dv; ++e) vhat[(size_t)t * dv + e] = 0.0;
+    for (int hd = 0; hd < H; ++hd) {
+      const size_t ht = (size_t)hd * len + t;
+      const double* qt = q + ht * d;
+      orc_subkey_dist(c, qt, K1 + (size_t)hd * nk, D1 + ht * n);
+      orc_subkey_dist(c, qt + h, K2 + (size_t)hd * nk, D2 + ht * n);
+      const int32_t* f = (forced && force_mask && force_mask[ht]) ? forced + ht * k : NULL;
+      orc_select(c, D1 + ht * n, D2 + ht * n, f, I + ht * k, S + ht * k, w + ht * k);
+      orc_read_values(c, I + ht * k, w + ht * k, V, vh);
+      for (int e = 0; e < dv; ++e) vhat[(size_t)t * dv + e] += vh[e];
+    }
+    for (int e = 0; e < dv; ++e) {
+      vhat[(size_t)t * dv + e] /= H;
+      o[(size_t)t * dv + e] = g[t] * vhat[(size_t)t * dv + e] + (1.0 - g[t]) * v[(size_t)t * dv + e];
+    }
+  }
+  if (I_out) memcpy(I_out, I, sizeof(int32_t) * (size_t)H * len * k);
+  if (w_out) memcpy(w_out, w, sizeof(double) * (size_t)H * len * k);
+
+  /* ---- memorization: the gradient of the gated loss on the shared rows ---- */
+  double* r = (double*)malloc(sizeof(double) * (size_t)len * dv);
+  double* tau = (double*)malloc(sizeof(double) * dv);
+  char* is_pair = (char*)calloc((size_t)len, 1);
+  int npair_tok = 0;
+  for (int t = 0; t < len; ++t) {
+    const double* u;
+    if (c->flags & ORC_LOOKAHEAD) {
+      if (t + 1 < len) u = v + (size_t)(t + 1) * dv;
+      else if (v_next) u = v_next;
+      else continue; /* last token of the sequence: no lookahead target */
+    } else {
+      u = v + (size_t)t * dv;
+    }
+    is_pair[t] = 1;
+    ++npair_tok;
+    orc_target(c, u, tau);
+    double gw = (c->flags & ORC_GATE_WEIGHT) ? g[t] : 1.0;
+    for (int e = 0; e < dv; ++e) r[(size_t)t * dv + e] = gw * (vhat[(size_t)t * dv + e] - tau[e]);
+  }
+  orc_hpair* pairs = (orc_hpair*)malloc(sizeof(orc_hpair) * (size_t)(npair_tok > 0 ? npair_tok : 1) * H * k);
+  int np = 0;
+  for (int t = 0; t < len; ++t) {
+    if (!is_pair[t]) continue;
+    for (int hd = 0; hd < H; ++hd)
+      for (int rr = 0; rr < k; ++rr) {
+        pairs[np].slot = I[((size_t)hd * len + t) * k + rr];
+        pairs[np].t = t;
+        pairs[np].hd = hd;
+        pairs[np].r = rr;
+        ++np;
+      }
+  }
+  qsort(pairs, (size_t)np, sizeof(orc_hpair), hpair_cmp); /* (slot, t, head) keys are unique */
+  double* G = (double*)malloc(sizeof(double) * dv);
+  for (int s0 = 0; s0 < np;) {
+    int s1 = s0;
+    while (s1 < np && pairs[s1].slot == pairs[s0].slot) ++s1;
+    const int32_t slot = pairs[s0].slot;
+    int nread = 0;
+    for (int e = 0; e < dv; ++e) G[e] = 0.0;
+    for (int pp = s0; pp < s1; ++pp) { /* token order, then head order */
+      if (pp == s0 || pairs[pp].t != pairs[pp - 1].t) ++nread;
+      const double wt = w[((size_t)pairs[pp].hd * len + pairs[pp].t) * k + pairs[pp].r] / H;
+      for (int e = 0; e < dv; ++e) G[e] += wt * r[(size_t)pairs[pp].t * dv + e];
+    }
+    float* row = V + (size_t)slot * dv;
+    for (int e = 0; e < dv; ++e) row[e] = (float)((double)row[e] - G[e] / nread);
+    s0 = s1;
+  }
+
+  /* ---- addressing: each head's own step ---- */
+  if (c->flags & ORC_KEY_UPDATE)
+    for (int hd = 0; hd < H; ++hd)
+      orc_key_step(c, len, q + (size_t)hd * len * d, D1 + (size_t)hd * len * n, D2 + (size_t)hd * len * n,
+                   K1 + (size_t)hd * nk, K2 + (size_t)hd * nk);
+
+  free(D1); free(D2); free(I); free(S); free(w); free(vh); free(vhat);
+  free(r); free(tau); free(is_pair); free(pairs); free(G);
 }
 
 /* ---------------------------------------------------------------------------
