@@ -68,10 +68,23 @@ enum {
 };
 #define FWPKM_DEFAULT_FLAGS (FWPKM_TARGET_NORM | FWPKM_LOOKAHEAD | FWPKM_GATE_WEIGHT)
 
-/* Shape and hyper-parameters of M independent memories.
+/* Shape and hyper-parameters of M memories (heads).
  * Supported limits (else FWPKM_ERR_UNSUPPORTED):
  *   1 <= k <= 32, k <= n <= 4096, d even with 8 <= d <= 512, d_v % 4 == 0 with
- *   4 <= d_v <= 1024, 1 <= chunk <= 1024 with chunk*k <= 16384, num_mem >= 1. */
+ *   4 <= d_v <= 1024, 1 <= chunk <= 1024 with chunk*k*H <= 16384, num_mem >= 1;
+ *   with v_heads = H > 1: num_mem % H == 0 and k*H <= 64.
+ *
+ * Heads sharing one value table (v_heads = H > 1; "Fast-weight Product Key Memory"
+ * (paperlayer summary) §D.1 ablates the head count with the slot count, §D.3 notes that
+ * more heads raise the collision rate): the memories m = b*H + h (h < H) of sequence b
+ * have their own codebooks K1, K2 and queries q and select their own k slots, but read
+ * and write one table V_b.  The read is the mean of the heads' reads,
+ *   vhat_t = (1/H) sum_h sum_{i in I^h_t} s'^h_{t,i} V_b[i],
+ * the write is the gradient of the gated reconstruction loss on the shared rows divided
+ * by the number of the chunk's tokens that read a row through any head, and each head's
+ * codebooks take their own addressing step.  Then V is [M/H][n*n][d_v] and v, g, o are
+ * per sequence ([M/H][T][...]); q, K1, K2, idx_out, w_out stay per head.  Token-at-a-time
+ * inference, the allocation-free step and fwpkm_run_layer take v_heads <= 1 only. */
 typedef struct {
   int n;         /* sub-keys per codebook; the memory has N = n*n slots              */
   int d;         /* query width (two halves of d/2)                                  */
@@ -84,6 +97,7 @@ typedef struct {
   float eps_norm;/* z-score: (u - mean) / sqrt(var + eps_norm)                       */
   float lr_key;  /* step size of the key update                                      */
   unsigned flags;/* FWPKM_* flags                                                    */
+  int v_heads;   /* heads per value table (0 or 1: every memory has its own V)      */
 } fwpkm_config;
 
 /* Opaque host-side handle.  It records the caller's state pointers and the carved

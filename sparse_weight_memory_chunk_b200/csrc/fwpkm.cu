@@ -95,8 +95,11 @@ fwpkm_status check_cfg(const fwpkm_config* c) {
   if (!(c->eps_idw >= 0.f) || !(c->eps_norm >= 0.f)) return FWPKM_ERR_INVALID_ARG;
   if (c->d % 2 != 0 || c->d_v % 4 != 0) return FWPKM_ERR_INVALID_ARG;
   if (c->k > c->n) return FWPKM_ERR_INVALID_ARG;
+  if (c->v_heads < 0) return FWPKM_ERR_INVALID_ARG;
+  const int H = c->v_heads > 1 ? c->v_heads : 1;
+  if (c->num_mem % H != 0) return FWPKM_ERR_INVALID_ARG;
   if (c->k > 32 || c->n > 4096 || c->d < 8 || c->d > 512 || c->d_v > 1024 || c->chunk > 1024 ||
-      (long long)c->chunk * c->k > 16384)
+      (long long)c->chunk * c->k * H > 16384 || c->k * H > 64)
     return FWPKM_ERR_UNSUPPORTED;
   return FWPKM_OK;
 }
@@ -105,6 +108,8 @@ Dims make_dims(const fwpkm_config* c) {
   Dims d;
   d.n = c->n; d.h = c->d / 2; d.d = c->d; d.dv = c->d_v; d.k = c->k; d.C = c->chunk; d.M = c->num_mem;
   d.N = (long long)c->n * c->n;
+  d.H = c->v_heads > 1 ? c->v_heads : 1;
+  d.B = d.M / d.H;
   d.qv_bf16 = c->qv_dtype == FWPKM_BF16;
   d.eps_idw = c->eps_idw; d.eps_norm = c->eps_norm; d.lr_key = c->lr_key; d.flags = c->flags;
   return d;
@@ -426,6 +431,7 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
     if (e && atoi(e) > 0) gr = atoi(e);
     if (gr > dm.M) gr = dm.M;
     if (gr > fwpkm_state::MAX_GROUPS) gr = fwpkm_state::MAX_GROUPS;
+    if (dm.H > 1) gr = 1;  // the memories of a sequence share V: keep them in one group
     st->groups = gr < 1 ? 1 : gr;
   }
   {
@@ -647,7 +653,7 @@ fwpkm_status fwpkm_stream_tokens(fwpkm_state* st, const void* q, const void* v, 
   if (n_tok < 1 || seq_stride < n_tok) return FWPKM_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4)) return FWPKM_ERR_INVALID_ARG;
   if (st->pending) return FWPKM_ERR_STATE;
-  if (st->wk.max_T < d.C || !st->wk.stage_q) return FWPKM_ERR_UNSUPPORTED;
+  if (st->wk.max_T < d.C || !st->wk.stage_q || d.H > 1) return FWPKM_ERR_UNSUPPORTED;
   fwpkm_status ps = peek_status(st);
   if (ps != FWPKM_OK) return ps;
   cudaStream_t s = (cudaStream_t)stream;
@@ -865,6 +871,7 @@ static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, cons
     const int m0 = (int)((long long)gi * d.M / G), m1 = (int)((long long)(gi + 1) * d.M / G);
     Dims dg = d;
     dg.M = m1 - m0;
+    dg.B = dg.M / dg.H;  // one group when heads share V (dg.M = d.M)
     const Work wg = G == 1 ? st->wk : group_work(d, st->wk, m0);
     const size_t kh = (size_t)m0 * d.n * d.h;
     enqueue_group(st, gi, dg, wg, st->K1 + kh, st->K2 + kh, st->V + (size_t)m0 * d.N * d.dv,
@@ -968,6 +975,7 @@ fwpkm_status fwpkm_run_layer(fwpkm_layer* L, fwpkm_state* st, const void* h, int
   if (T == 0) return FWPKM_OK;
   const Dims& d = st->dm;
   if (!h || !scratch || !o_out || T < 0 || n_iter < 1 || T > st->wk.max_T) return FWPKM_ERR_INVALID_ARG;
+  if (d.H > 1) return FWPKM_ERR_UNSUPPORTED;
   if (lc->d != d.d || lc->d_v != d.dv || lc->qv_dtype != st->cfg.qv_dtype ||
       (long long)d.M * T > (long long)lc->max_rows)
     return FWPKM_ERR_INVALID_ARG;

@@ -44,6 +44,7 @@ enum KernelKind : int { KK_NONE = 0, KK_GATHER = 1, KK_WRITE = 2, KK_SCORE = 3, 
 
 struct Dims {
   int n, h, d, dv, k, C, M;
+  int H, B;  // heads per value table (1: independent memories) and value tables (M / H)
   long long N;
   int qv_bf16;
   float eps_idw, eps_norm, lr_key;

@@ -68,6 +68,8 @@ extern "C" fwpkm_status fwpkm_chunk_step_noalloc(const fwpkm_config* cfg, float*
   d.n = cfg->n; d.h = cfg->d / 2; d.d = cfg->d; d.dv = cfg->d_v; d.k = cfg->k; d.C = cfg->chunk;
   d.M = cfg->num_mem; d.N = (long long)cfg->n * cfg->n; d.qv_bf16 = cfg->qv_dtype == FWPKM_BF16;
   d.eps_idw = cfg->eps_idw; d.eps_norm = cfg->eps_norm; d.lr_key = cfg->lr_key; d.flags = cfg->flags;
+  d.H = 1; d.B = d.M;
+  if (cfg->v_heads > 1) return FWPKM_ERR_UNSUPPORTED;  // independent memories only
   // no token-at-a-time staging and no tensor-core buffers: only what the kernels below use
   need = workspace_bytes(d, cfg->chunk, nullptr, nullptr, false, false);
   if (need > FWPKM_NOALLOC_SCRATCH_BYTES) {

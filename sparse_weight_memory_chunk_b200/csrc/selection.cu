@@ -231,21 +231,23 @@ constexpr int SORT_SPLIT = 16;
 constexpr int SORT_BUCKET_KEYS = 64;   // average keys per bucket
 constexpr int SORT_BUCKET_CAP = 128;   // largest bucket the ranking path handles
 
-template <int VPT>
+// HEADS: the memories of a sequence share its value table (dm.H > 1); false compiles the
+// one-head kernel, whose pair i is offset i of the chunk's [C][k] slot block.
+template <int VPT, bool HEADS>
 __global__ void __launch_bounds__(SORT_THREADS)
 sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ u64 s_keys[];
   __shared__ int s_cnt[512], s_off[513], s_cur[512];
-  const int m = blockIdx.y;
+  const int m = blockIdx.y;  // the value table (sequence); its heads are memories m H .. m H + H - 1
   const int cc = blockIdx.x / SORT_SPLIT, part = blockIdx.x % SORT_SPLIT;
-  const int C = dm.C, k = dm.k;
+  const int C = dm.C, k = dm.k, H = HEADS ? dm.H : 1, kh = k * H;
   const int tc0 = cc * C;  // relative to wt0
   const int clen = min(C, total_len - tc0);
   int npair = clen;
   if (!last_has_target && tc0 + clen == total_len) npair = clen - 1;
-  const int P = npair * k;
+  const int P = npair * kh;
   int Ppad = 32 * VPT;
   while (Ppad < P) Ppad <<= 1;
   const int NB = Ppad / SORT_BUCKET_KEYS;  // a power of two, <= 512
@@ -253,21 +255,36 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
   const int b_lo = part * NB / SORT_SPLIT, b_hi = (part + 1) * NB / SORT_SPLIT;
   const int cslot = (wt0 + tc0) / C;
   const size_t cbase = (size_t)m * w.max_chunks + cslot;
-  u64* out = w.sk + cbase * (size_t)(C * k);
+  u64* out = w.sk + cbase * (size_t)(C * kh);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   for (int b = tid; b < NB; b += SORT_THREADS) s_cnt[b] = 0;
   __syncthreads();
   u64 x[VPT];
   int bk[VPT];
+  // every slot of this thread's pairs is loaded before the counting
+  unsigned sl[VPT];
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) {
+    const int i = tid * VPT + u;
+    sl[u] = 0u;
+    if (i < P) {
+      if (!HEADS) {
+        sl[u] = (unsigned)w.idx[((size_t)m * w.max_T + wt0 + tc0) * k + i];
+      } else {
+        // pair i = (t_local H + head) k + r: slot r of the head's selection for token t_local
+        const int t = i / kh, hr = i - t * kh, hd = hr / k, r = hr - hd * k;
+        sl[u] = (unsigned)w.idx[(((size_t)m * H + hd) * w.max_T + wt0 + tc0 + t) * k + r];
+      }
+    }
+  }
 #pragma unroll
   for (int u = 0; u < VPT; ++u) {
     const int i = tid * VPT + u;
     u64 key = ~0ull;
     bk[u] = -1;
     if (i < P) {
-      // pair i = t_local * k + r sits at offset i of the chunk's [C][k] slot block
-      const unsigned slot = (unsigned)w.idx[((size_t)m * w.max_T + wt0 + tc0) * k + i];
+      const unsigned slot = sl[u];
       key = ((u64)slot << 32) | (unsigned)i;
       bk[u] = NB > 1 ? (int)((slot * 2654435761u) >> (32 - nb_log2)) : 0;  // multiplicative hash
       atomicAdd(&s_cnt[bk[u]], 1);
@@ -361,21 +378,22 @@ int launch_sort_pairs(const Dims& d, const Work& w, int wt0, int total_len, bool
                       cudaStream_t s) {
   if (total_len <= 0) return 0;
   const int nchunks = (total_len + d.C - 1) / d.C;
-  const int P = d.C * d.k;
-  dim3 grid(nchunks * SORT_SPLIT, d.M);
-  if (P <= 8 * SORT_THREADS) {
-    int Ppad = 256;
+  const int P = d.C * d.k * d.H;
+  dim3 grid(nchunks * SORT_SPLIT, d.B);
+  auto go = [&](auto kern, int vpt) {
+    int Ppad = 32 * vpt;
     while (Ppad < P) Ppad <<= 1;
     const size_t smem = sizeof(u64) * (size_t)Ppad;
-    if (!raise_smem_limit((const void*)sort_pairs_kernel<8>, smem)) return -1;
-    launch_k(sort_pairs_kernel<8>, grid, SORT_THREADS, smem, s, d, w, wt0, total_len, last_has_target ? 1 : 0);
-  } else {
-    int Ppad = 512;
-    while (Ppad < P) Ppad <<= 1;
-    const size_t smem = sizeof(u64) * (size_t)Ppad;
-    if (!raise_smem_limit((const void*)sort_pairs_kernel<16>, smem)) return -1;
-    launch_k(sort_pairs_kernel<16>, grid, SORT_THREADS, smem, s, d, w, wt0, total_len, last_has_target ? 1 : 0);
-  }
+    if (!raise_smem_limit((const void*)kern, smem)) return -1;
+    launch_k(kern, grid, SORT_THREADS, smem, s, d, w, wt0, total_len, last_has_target ? 1 : 0);
+    return 1;
+  };
+  int rc;
+  if (P <= 8 * SORT_THREADS)
+    rc = d.H > 1 ? go(sort_pairs_kernel<8, true>, 8) : go(sort_pairs_kernel<8, false>, 8);
+  else
+    rc = d.H > 1 ? go(sort_pairs_kernel<16, true>, 16) : go(sort_pairs_kernel<16, false>, 16);
+  if (rc < 0) return -1;
   return 1;
 }
 

@@ -122,7 +122,9 @@ __device__ __forceinline__ const VT* target_src(const Dims& dm, const VT* v, con
 // overlaps the gather.
 // ---------------------------------------------------------------------------
 constexpr int GATHER_TOK = VAL_WARPS / 2;
-template <typename VT, int VPL>
+// HEADS: the memories of a sequence share its value table (dm.H > 1, up to 64 rows per
+// token); false compiles the one-head kernel (k <= 32 rows, one entry per lane).
+template <typename VT, int VPL, bool HEADS>
 __global__ void __launch_bounds__(VAL_WARPS * 32, 4)
 gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict__ v,
               const float* __restrict__ g, long long stride, int wt0, int len, float* __restrict__ o,
@@ -133,15 +135,31 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tl = warp >> 1, half = warp & 1;
   const int i = blockIdx.x * GATHER_TOK + tl;
-  const int m = blockIdx.y;
+  const int m = blockIdx.y;  // the value table (sequence); its heads are memories m H .. m H + H - 1
   const bool active = i < len;
-  const int k = dm.k, dv4 = dm.dv >> 2;
+  const int k = dm.k, dv4 = dm.dv >> 2, H = HEADS ? dm.H : 1;
+  const int R = H * k;       // rows read by the token: entry e = (head e / k, rank e % k)
   const long long tok = (long long)wt0 + i;
-  int myslot = 0;
-  float myw = 0.f;
-  if (active && lane < k) {
-    myslot = w.idx[((size_t)m * w.max_T + tok) * k + lane];
-    myw = w.w[((size_t)m * w.max_T + tok) * k + lane];
+  // lane l holds entries l and l + 32: slot and weight s'/H (H = 1: the weight itself)
+  int myslot = 0, myslot2 = 0;
+  float myw = 0.f, myw2 = 0.f;
+  const float invH = 1.f / (float)H;
+  if (active && !HEADS) {
+    if (lane < k) {
+      myslot = w.idx[((size_t)m * w.max_T + tok) * k + lane];
+      myw = w.w[((size_t)m * w.max_T + tok) * k + lane];
+    }
+  } else if (active) {
+    if (lane < R) {
+      const size_t o = (((size_t)m * H + lane / k) * w.max_T + tok) * k + lane % k;
+      myslot = w.idx[o];
+      myw = w.w[o] * invH;
+    }
+    if (lane + 32 < R) {
+      const size_t o = (((size_t)m * H + (lane + 32) / k) * w.max_T + tok) * k + (lane + 32) % k;
+      myslot2 = w.idx[o];
+      myw2 = w.w[o] * invH;
+    }
   }
   // half 0 prefetches the token's value row and gate
   float4 xv[VPL];
@@ -154,13 +172,15 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
   float4 acc[VPL];
 #pragma unroll
   for (int c = 0; c < VPL; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int r0 = half * 16, r1 = min(k, r0 + 16);
+  // warp half 0 sums entries [0, HALF), half 1 [HALF, R) (HALF = 16 when R <= 32)
+  const int HALF = R <= 32 ? 16 : (R + 1) / 2;
+  const int r0 = half * HALF, r1 = min(R, r0 + HALF);
   const uint64_t pol = evict_first_policy();
   if (active) {
 #pragma unroll 16
     for (int r = r0; r < r1; ++r) {
-      const int slot = __shfl_sync(0xffffffffu, myslot, r);
-      const float wr = __shfl_sync(0xffffffffu, myw, r);
+      const int slot = __shfl_sync(0xffffffffu, (!HEADS || r < 32) ? myslot : myslot2, r & 31);
+      const float wr = __shfl_sync(0xffffffffu, (!HEADS || r < 32) ? myw : myw2, r & 31);
       const float4* row = Vm + (size_t)slot * dv4;
 #pragma unroll
       for (int c = 0; c < VPL; ++c) {
@@ -380,28 +400,32 @@ __device__ __forceinline__ void store_row(float* Vm, int slot, const Dims& dm, c
   }
 }
 
-template <int VPL, int WB>
+// HEADS: the memories of a sequence share its value table (dm.H > 1): weights s'/H and
+// N_read counted in distinct tokens; false compiles the one-head kernel (N_read = pairs).
+template <int VPL, int WB, bool HEADS>
 __global__ void __launch_bounds__(WR_WARPS * 32)
 write_batched_kernel(Dims dm, Work w, float* __restrict__ V, int wt0, int warps_per_mem) {
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gw = blockIdx.x * WR_WARPS + warp;
-  const int m = gw / warps_per_mem, wi = gw - m * warps_per_mem;
-  if (m >= dm.M) return;
-  const int C = dm.C, k = dm.k, dv4 = dm.dv >> 2;
-  const int kshift = (k & (k - 1)) == 0 ? __popc(k - 1) : -1;
+  const int m = gw / warps_per_mem, wi = gw - m * warps_per_mem;  // m: the value table (sequence)
+  if (m >= dm.B) return;
+  const int C = dm.C, k = dm.k, dv4 = dm.dv >> 2, H = HEADS ? dm.H : 1, kh = k * H;
+  const int kshift = (kh & (kh - 1)) == 0 ? __popc(kh - 1) : -1;
+  const float invH = 1.f / (float)H;
   const size_t cbase = (size_t)m * w.max_chunks + wt0 / C;
   const int P = w.npairs[cbase];
   const int r0 = (int)((long long)P * wi / warps_per_mem), r1 = (int)((long long)P * (wi + 1) / warps_per_mem);
   if (r0 >= r1) return;
-  const unsigned long long* sk = w.sk + cbase * (size_t)(C * k);
-  const float* wrow = w.w + ((size_t)m * w.max_T + wt0) * k;
+  const unsigned long long* sk = w.sk + cbase * (size_t)(C * kh);
+  const float* wrow = w.w + ((size_t)m * w.max_T + wt0) * k;  // one head: pair t k + r at wrow[t k + r]
   const float4* resid = reinterpret_cast<const float4*>(w.resid + (size_t)m * C * dm.dv);
   float* Vm = V + (size_t)m * dm.N * dm.dv;
   // the open segment: cur = its slot (-1: none open; -2: a slot outside [0, N), skipped),
-  // its V row cv, partial sum acc and pair count nr
-  int cur = -1, nr = 0;
+  // its V row cv, partial sum acc, and N_read = the tokens it has met (a token may read
+  // the row through several heads; their pairs are adjacent) with the last of them
+  int cur = -1, nr = 0, last_t = -1;
   float4 cv[VPL], acc[VPL];
 #pragma unroll
   for (int c = 0; c < VPL; ++c) cv[c] = acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -441,6 +465,7 @@ write_batched_kernel(Dims dm, Work w, float* __restrict__ V, int wt0, int warps_
       // ---- issue every load of the batch ----
       float4 R[WB][VPL], Vh[WB][VPL];
       float wt[WB];
+      int tl_[HEADS ? WB : 1];
 #pragma unroll
       for (int u = 0; u < WB; ++u) {
         const int l = b0 + u;
@@ -450,8 +475,15 @@ write_batched_kernel(Dims dm, Work w, float* __restrict__ V, int wt0, int warps_
         const uint32_t tr = (uint32_t)(ku & 0xffffffffu);
         const int slot = (int)(ku >> 32);
         const bool okslot = slot >= 0 && (long long)slot < dm.N;
-        const int t_local = kshift >= 0 ? (int)(tr >> kshift) : (int)(tr / (uint32_t)k);
-        wt[u] = in ? wrow[tr] : 0.f;
+        // pair tr = (t_local H + head) k + r: weight s'/H of the head's rank r for the token
+        const int t_local = kshift >= 0 ? (int)(tr >> kshift) : (int)(tr / (uint32_t)kh);
+        if (HEADS) {
+          const int hr = (int)tr - t_local * kh, head = hr / k, rk = hr - head * k;
+          wt[u] = in ? w.w[(((size_t)m * H + head) * w.max_T + wt0 + t_local) * k + rk] * invH : 0.f;
+          tl_[u] = t_local;
+        } else {
+          wt[u] = in ? wrow[tr] : 0.f;
+        }
         const float4* rr = resid + (size_t)(in ? t_local : 0) * dv4;
         const float4* vr = reinterpret_cast<const float4*>(Vm + (size_t)(hd && okslot ? slot : 0) * dm.dv);
 #pragma unroll
@@ -479,6 +511,7 @@ write_batched_kernel(Dims dm, Work w, float* __restrict__ V, int wt0, int warps_
               acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
             nr = 0;
+            last_t = -1;
           }
         }
         if (cur >= 0) {
@@ -488,7 +521,12 @@ write_batched_kernel(Dims dm, Work w, float* __restrict__ V, int wt0, int warps_
             acc[c].x = fmaf(a, R[u][c].x, acc[c].x); acc[c].y = fmaf(a, R[u][c].y, acc[c].y);
             acc[c].z = fmaf(a, R[u][c].z, acc[c].z); acc[c].w = fmaf(a, R[u][c].w, acc[c].w);
           }
-          ++nr;
+          if (!HEADS) {
+            ++nr;
+          } else if (tl_[u] != last_t) {
+            ++nr;
+            last_t = tl_[u];
+          }
         }
         // the segment ends at this pair if the next position starts another one or the list
         // ends; at the window's last position the next head is only known in the next window
@@ -522,14 +560,17 @@ int launch_gather(const Dims& d, const Work& w, const float* V, const void* v, c
                   long long stride, int wt0, int len, float* o, bool fuse_resid, const void* v_next,
                   cudaStream_t s) {
   if (len <= 0) return 0;
-  dim3 grid((len + GATHER_TOK - 1) / GATHER_TOK, d.M);
+  dim3 grid((len + GATHER_TOK - 1) / GATHER_TOK, d.B);
+  const bool heads = d.H > 1;
   if (d.qv_bf16) {
-    FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(gather_kernel<__nv_bfloat16, VPL>, grid, VAL_WARPS * 32, 0, s,
-        d, w, V, (const __nv_bfloat16*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0,
-        (const __nv_bfloat16*)v_next));
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv),
+        launch_k(heads ? gather_kernel<__nv_bfloat16, VPL, true> : gather_kernel<__nv_bfloat16, VPL, false>, grid,
+                 VAL_WARPS * 32, 0, s, d, w, V, (const __nv_bfloat16*)v, g, stride, wt0, len, o,
+                 fuse_resid ? 1 : 0, (const __nv_bfloat16*)v_next));
   } else {
-    FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(gather_kernel<float, VPL>, grid, VAL_WARPS * 32, 0, s,
-        d, w, V, (const float*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0, (const float*)v_next));
+    FWPKM_VPL_DISPATCH(vpl_of(d.dv),
+        launch_k(heads ? gather_kernel<float, VPL, true> : gather_kernel<float, VPL, false>, grid, VAL_WARPS * 32, 0,
+                 s, d, w, V, (const float*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0, (const float*)v_next));
   }
   return 1;
 }
@@ -537,7 +578,7 @@ int launch_gather(const Dims& d, const Work& w, const float* V, const void* v, c
 int launch_resid(const Dims& d, const Work& w, const void* v, const float* g, long long stride, int len,
                  const void* v_next, cudaStream_t s) {
   if (len <= 0) return 0;
-  dim3 grid((len + VAL_WARPS - 1) / VAL_WARPS, d.M);
+  dim3 grid((len + VAL_WARPS - 1) / VAL_WARPS, d.B);
   if (d.qv_bf16) {
     FWPKM_VPL_DISPATCH(vpl_of(d.dv), launch_k(resid_kernel<__nv_bfloat16, VPL>, grid, VAL_WARPS * 32, 0, s, 
         d, w, (const __nv_bfloat16*)v, g, stride, len, (const __nv_bfloat16*)v_next));
@@ -628,7 +669,7 @@ int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s
     const char* e = getenv("FWPKM_WRITE_V1");
     return e && e[0] == '1';
   }();
-  if (v1) return launch_write_v1(d, w, V, wt0, s);
+  if (v1 && d.H == 1) return launch_write_v1(d, w, V, wt0, s);
   const int vpl = vpl_of(d.dv);
   // one warp per ~32 positions of a memory's list at most, and no more warps than fit on the
   // GPU at once (FWPKM_WRITE_SHARE percent of them, default 100)
@@ -639,19 +680,23 @@ int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s
   }();
   auto go = [&](const void* kern, auto kfn) {
     const int resident_warps = resident_ctas(kern, WR_WARPS * 32) * WR_WARPS;
-    int per_mem = (int)((long long)resident_warps * share / 100 / d.M);
-    const int most = (d.C * d.k + 31) / 32;
+    int per_mem = (int)((long long)resident_warps * share / 100 / d.B);
+    const int most = (d.C * d.k * d.H + 31) / 32;
     if (per_mem > most) per_mem = most;
     if (per_mem < 1) per_mem = 1;
-    const int blocks = (d.M * per_mem + WR_WARPS - 1) / WR_WARPS;
+    const int blocks = (d.B * per_mem + WR_WARPS - 1) / WR_WARPS;
     launch_k(kfn, dim3((unsigned)blocks), WR_WARPS * 32, 0, s, d, w, V, wt0, per_mem);
   };
+#define FWPKM_WRITE_GO(VPLV, WBV)                                                                      \
+  (d.H > 1 ? go((const void*)write_batched_kernel<VPLV, WBV, true>, write_batched_kernel<VPLV, WBV, true>) \
+           : go((const void*)write_batched_kernel<VPLV, WBV, false>, write_batched_kernel<VPLV, WBV, false>))
   switch (vpl) {
-    case 1: go((const void*)write_batched_kernel<1, 8>, write_batched_kernel<1, 8>); break;
-    case 2: go((const void*)write_batched_kernel<2, 4>, write_batched_kernel<2, 4>); break;
-    case 4: go((const void*)write_batched_kernel<4, 2>, write_batched_kernel<4, 2>); break;
-    default: go((const void*)write_batched_kernel<8, 1>, write_batched_kernel<8, 1>); break;
+    case 1: FWPKM_WRITE_GO(1, 8); break;
+    case 2: FWPKM_WRITE_GO(2, 4); break;
+    case 4: FWPKM_WRITE_GO(4, 2); break;
+    default: FWPKM_WRITE_GO(8, 1); break;
   }
+#undef FWPKM_WRITE_GO
   return 1;
 }
 

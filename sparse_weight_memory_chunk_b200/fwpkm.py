@@ -35,14 +35,14 @@ class Config(ctypes.Structure):
     _fields_ = [("n", ctypes.c_int), ("d", ctypes.c_int), ("d_v", ctypes.c_int), ("k", ctypes.c_int),
                 ("chunk", ctypes.c_int), ("num_mem", ctypes.c_int), ("qv_dtype", ctypes.c_int),
                 ("eps_idw", ctypes.c_float), ("eps_norm", ctypes.c_float), ("lr_key", ctypes.c_float),
-                ("flags", ctypes.c_uint)]
+                ("flags", ctypes.c_uint), ("v_heads", ctypes.c_int)]
 
 
 def make_config(n, d, d_v, k, chunk, num_mem, bf16, eps_idw=1e-3, eps_norm=1e-5, lr_key=1.0,
-                key_update=False, target_norm=True, lookahead=True, gate_weight=True) -> Config:
+                key_update=False, target_norm=True, lookahead=True, gate_weight=True, v_heads=1) -> Config:
     flags = ((KEY_UPDATE if key_update else 0) | (TARGET_NORM if target_norm else 0)
              | (LOOKAHEAD if lookahead else 0) | (GATE_WEIGHT if gate_weight else 0))
-    return Config(n, d, d_v, k, chunk, num_mem, BF16 if bf16 else F32, eps_idw, eps_norm, lr_key, flags)
+    return Config(n, d, d_v, k, chunk, num_mem, BF16 if bf16 else F32, eps_idw, eps_norm, lr_key, flags, v_heads)
 
 
 _lib = None
