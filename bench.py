@@ -44,13 +44,11 @@ BY_NAME = {w.name: (i, w) for i, w in WORKLOADS.items()}
 # / 2; a full launch scales with the memories it processes (each memory's work is the
 # same).  A kernel changed since that capture is missing here and reports null.
 TRAFFIC = {
-    "score": {"per_mem": (3_493_376 + 512) / 2},
-    "pbar": {"per_mem": 4_345_856 / 2},
-    "wbuild": {"per_mem": 4_244_736 / 2},
-    "address": {"per_mem": 6_880_000 / 2},
-    "topk": {"per_mem": 4_262_400 / 2},
-    "sort": {"per_mem": 107_008 / 2},
-    "write": {"per_mem": (16_262_656 + 8_704) / 2},
+    "fused": {"per_mem": (5_873_920 + 0) / 2},
+    "topk": {"per_mem": (4_266_240 + 0) / 2},
+    "sort": {"per_mem": (96_512 + 0) / 2},
+    "gather": {"per_mem": (15_792_128 + 0) / 2},
+    "write": {"per_mem": (16_094_464 + 0) / 2},
 }
 
 
@@ -377,7 +375,7 @@ def measure(args, w, rank, world, local_rank, n_iter, steps, warmup, full):
     kinds = {}
     if args.kernel is None:
         for name in ("gather", "write", "score", "topk", "cartesian", "sort", "pbar", "wbuild", "address", "fused",
-                     "prep", "other"):
+                     "value_loop", "prep", "other"):
             st.profile_kernel(name)
             step()
             ms, n = st.kernel_time()
@@ -435,31 +433,56 @@ def measure(args, w, rank, world, local_rank, n_iter, steps, warmup, full):
     t_roof = max(b_vk / (hbm_peak * 1e9), flops / (tc_peak * 1e12))
     step_frac = t_roof / (ms_step / 1000.0)
     nchunks = (w.T + w.C - 1) // w.C
-    U_chunk = U / max(1, nchunks)  # unique touched rows per chunk launch (all memories)
-    tok = w.M * w.C  # token-memories per chunk launch
-    # algorithmic work of one launch of each kernel kind (bytes against HBM, FLOPs against
-    # the tensor peak, ALU ops against the fp32 lanes)
+    # algorithmic work of one step of each kernel kind, as (bytes against HBM, FLOPs against
+    # the tensor peak, ALU ops against the fp32 lanes); a launch's share is the step's work
+    # over the kind's launches in the step.  The addressing of frozen keys runs once per
+    # call, the rest once per pass.
     alu_peak = 148 * 128 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12  # Tops/s
     cand = sum(w.k // (i + 1) for i in range(w.k))  # staircase candidates per token-memory
+    P, h = 2 * w.M, w.d // 2
+    es = 2 if w.qv == "bf16" else 4
+    tm_val = w.M * w.T * n_iter                                # token-memories through the value path
+    tm_adr = w.M * w.T * (n_iter if w.key_update else 1)       # token-memories addressed
+    gather_b = gather_per_token * tm_val
+    write_b = 2 * U * w.d_v * 4 * n_iter
+    tc = w.qv == "bf16" and h in (64, 128)                     # tensor-core scoring (else CUDA cores)
+    pieces = 3 * P * w.n * h * 2 if tc else 0                  # bf16 key pieces read per scoring launch
     work = {
-        "gather": ("hbm", gather_per_token * tok),
-        "write": ("hbm", 2 * U_chunk * w.d_v * 4),
-        "score": ("tensor", 2 * w.n * w.d * tok),
-        "address": ("tensor", 2 * w.n * w.d * tok),
-        "topk": ("hbm", 2 * w.n * 4 * tok),                       # distance rows read
-        "pbar": ("hbm", 2 * w.n * 4 * tok),                       # distance rows read
-        "wbuild": ("hbm", 2 * w.n * 4 * tok * 2 + 2 * w.n * 2 * 2 * tok),  # rows read twice, 2 bf16 pieces written
-        "sort": ("hbm", w.k * tok * (4 + 8)),                      # slots read, pair keys written
-        "cartesian": ("alu", cand * 2 * tok),                      # one add + one compare per candidate
-        # the one-launch addressing step: scoring and (key update) key-step contractions
-        "fused": ("tensor", 2 * w.n * w.d * tok * (2 if w.key_update else 1)),
+        "gather": (gather_b, 0, 0),
+        "write": (write_b, 0, 0),
+        # tensor cores: distance rows written + key pieces read per launch (added below), 2 n d
+        # FLOP per token-memory; CUDA cores (scoring fused with the per-half top-k): keys and
+        # queries read, the same products as fp32 FMAs
+        "score": ((2 * w.n * 4 * tm_adr, 2 * w.n * w.d * tm_adr, 0) if tc else
+                  (w.d * es * tm_adr, 0, 2 * w.n * w.d * tm_adr)),
+        "address": (0, 2 * w.n * w.d * tm_adr, 0),
+        "topk": (2 * w.n * 4 * tm_adr, 0, 0),                  # distance rows read
+        "pbar": (2 * w.n * 4 * tm_adr, 0, 0),                  # distance rows read
+        "wbuild": (2 * w.n * 4 * tm_adr * 2 + 2 * w.n * 2 * 2 * tm_adr, 0, 0),  # rows read twice, 2 bf16 pieces out
+        "sort": (w.k * tm_adr * (4 + 8), 0, 0),                # slots read, pair keys written
+        "cartesian": (0, 0, cand * 2 * tm_adr),                # one add + one compare per candidate
+        # one-launch addressing step: distance rows written, half-queries read (both layouts);
+        # per launch the key pieces read and, with the key step, keys read + written and
+        # their pieces rewritten; FLOPs of the scoring and key-step contractions
+        "fused": (2 * w.n * 4 * tm_adr + 2 * 2 * h * es * tm_adr,
+                  2 * w.n * w.d * tm_adr * (2 if w.key_update else 1), 0),
+        # the persistent value loop (frozen keys): every chunk's gather and write
+        "value_loop": (gather_b + write_b, 0, 0),
     }
+    per_launch_extra = {"score": pieces,
+                        "fused": pieces + ((2 * P * w.n * h * 4 + 3 * P * w.n * h * 2) if w.key_update else 0)}
 
     def kind_roofline(kind, ms, n):
         if kind not in work or n == 0:
             return None
-        bound, per_launch = work[kind]
+        b, f, a = work[kind]
+        b = b / n + per_launch_extra.get(kind, 0)
+        f, a = f / n, a / n
         avg_s = (ms / 1000.0) / n
+        # the bound is the roofline the launch's work takes longest on
+        t = {"hbm": b / (hbm_peak * 1e9), "tensor": f / (tc_peak * 1e12), "alu": a / (alu_peak * 1e12)}
+        bound = max(t, key=t.get)
+        per_launch = {"hbm": b, "tensor": f, "alu": a}[bound]
         if bound == "hbm":
             ach, peak, unit, src = per_launch / avg_s / 1e9, hbm_peak, "GB/s", "hbm_gbs"
         elif bound == "tensor":
@@ -471,7 +494,8 @@ def measure(args, w, rank, world, local_rank, n_iter, steps, warmup, full):
                 "traffic": traffic or None,
                 "kernel": kind, "peak_source": f"{peak_src if bound != 'alu' else 'derived'} ({src})",
                 "avg_launch_us": avg_s * 1e6, "launches_timed": n,
-                "algorithmic_per_launch": per_launch}
+                "algorithmic_per_launch": per_launch,
+                "roofline_us": {k_: round(v_ * 1e6, 3) for k_, v_ in t.items() if v_ > 0}}
 
     roof = kind_roofline(dominant, dom_ms, dom_n) or {"bound": None, "kernel": dominant}
     kind_table = {k_: {"ms_per_step": round(v_[0], 4),

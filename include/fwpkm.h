@@ -355,13 +355,16 @@ fwpkm_status fwpkm_addressing_metrics(const int32_t* idx, int num_mem, int T, in
 fwpkm_status fwpkm_sync(fwpkm_state* st, void* stream);
 
 /* Test hook of the timeout path (no counterpart in the paper).  Each of the next
- * `n_launches` tensor-core kernel launches made by this process (scoring, key step,
- * projections) has its MMA-issuing thread first wait on a barrier that nothing
- * completes.  That wait is bounded like every other wait in those kernels (0.2 s): it
- * runs out, the kernel takes its abort path (in-flight copies drained, tensor memory
- * freed, no further work) and latches FWPKM_ERR_TIMEOUT in the handle's status word.
- * Nothing faults and the context stays usable.  n_launches = 0 cancels.  Launches
- * captured into a CUDA graph keep the setting they were captured with. */
+ * `n_launches` launches made by this process of a kernel with a bounded wait (the
+ * tensor-core scoring, key step and projections; the one-launch addressing step; the
+ * persistent value loop of fwpkm_run_sequence with frozen keys) first waits on
+ * something that nothing completes: an mbarrier for the MMA-issuing thread, or an
+ * arrival count that no launch reaches for the value loop.  That wait is bounded like
+ * every other wait in those kernels (0.2 s): it runs out, the kernel takes its abort
+ * path (in-flight copies drained, tensor memory freed, no further work) and latches
+ * FWPKM_ERR_TIMEOUT in the handle's status word.  Nothing faults and the context stays
+ * usable.  n_launches = 0 cancels.  While a stall is pending fwpkm_run_sequence enqueues
+ * its launches directly instead of through its cached CUDA graph. */
 void fwpkm_test_stall_waits(int n_launches);
 
 /* Release the handle (streams, events, graphs).  Caller buffers are untouched. */

@@ -214,6 +214,8 @@ thread_local bool launch_priority_set = false;
 
 static std::atomic<int> g_test_stalls{0};
 
+bool test_stalls_pending() { return g_test_stalls.load() > 0; }
+
 int take_test_stall() {
   int n = g_test_stalls.load();
   while (n > 0)
@@ -294,6 +296,9 @@ size_t workspace_bytes(const Dims& d, int max_T, Work* w, char* base, bool strea
   x.Kpc = nullptr; x.kn = nullptr; x.qn = nullptr; x.zpart = nullptr; x.ppart = nullptr;
   x.Wt = nullptr; x.Qt = nullptr; x.wsum_part = nullptr; x.pbar_cnt = nullptr; x.qt_T = 0;
   x.af_part = nullptr; x.af_cnt = nullptr;
+  // frozen keys: the persistent value loop's counters (one pair per memory, so that each
+  // group of memories has its own)
+  x.vl_cnt = ku ? nullptr : (unsigned*)take(4 * M * 2);
   if (x.tc) {
     const size_t P = 2 * M, h = d.h, cpad = (C + 63) / 64 * 64, nt = (n + 127) / 128;
     x.Kpc = (__nv_bfloat16*)take(2 * 3 * P * n * h);
@@ -353,6 +358,7 @@ Work group_work(const Dims& d, const Work& w, int m0) {
   if (x.pbar_cnt) x.pbar_cnt += M0 * 2 * ((n + 255) / 256);
   if (x.af_part) x.af_part += M0 * 2 * (n / 128) * 2 * 256;
   if (x.af_cnt) x.af_cnt += M0 * 2 * 2;
+  if (x.vl_cnt) x.vl_cnt += M0 * 2;
   return x;
 }
 
@@ -464,7 +470,8 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
   if (cudaMemset(st->wk.status, 0, sizeof(int)) != cudaSuccess ||
       (st->wk.pbar_cnt &&
        cudaMemset(st->wk.pbar_cnt, 0, sizeof(int) * 2 * (size_t)dm.M * ((dm.n + 255) / 256)) != cudaSuccess) ||
-      (st->wk.af_cnt && cudaMemset(st->wk.af_cnt, 0, sizeof(int) * 4 * (size_t)dm.M) != cudaSuccess)) {
+      (st->wk.af_cnt && cudaMemset(st->wk.af_cnt, 0, sizeof(int) * 4 * (size_t)dm.M) != cudaSuccess) ||
+      (st->wk.vl_cnt && cudaMemset(st->wk.vl_cnt, 0, sizeof(unsigned) * 2 * (size_t)dm.M) != cudaSuccess)) {
     cudaGetLastError();
     fwpkm_destroy_state(st);
     return FWPKM_ERR_CUDA;
@@ -788,10 +795,19 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
       run(st, KK_SORT, sK, [&] { return launch_sort_pairs(d, wk, w0, wl, !la || (w0 + wl < T), sK); });
       ready.push_back(mark(sK));
     }
+    // the value loop: one persistent launch per addressing window in the first pass and
+    // one for all chunks in each later pass, else the chunks one by one
+    const bool vloop = value_loop_enabled() && wk.vl_cnt != nullptr;
+    const int wch = wtok >= T ? nch : wtok / C;  // chunks per window (wtok < T is whole chunks)
     for (int pass = 0; pass < n_iter; ++pass)
-      for (int c = 0; c < nch; ++c) {
-        if (pass == 0 && (c * C) % wtok == 0) cudaStreamWaitEvent(sV, ready[(c * C) / wtok], 0);
-        value_chunk(c);
+      for (int c = 0; c < nch; c += (pass == 0 ? wch : nch)) {
+        if (pass == 0) cudaStreamWaitEvent(sV, ready[c / wch], 0);
+        const int c1 = pass > 0 ? nch : (c + wch < nch ? c + wch : nch);
+        if (vloop) {
+          run(st, KK_VLOOP, sV, [&] { return launch_value_loop(d, wk, V, v, g, T, c, c1, o, sV); });
+        } else {
+          for (int cc = c; cc < c1; ++cc) value_chunk(cc);
+        }
       }
   } else {
     const size_t dbuf = (size_t)wk.dfull_buf;
@@ -893,7 +909,9 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
   st->pending = 0;
   st->host_error = 0;
   cudaStream_t user = (cudaStream_t)stream;
-  if (st->no_graph) {
+  // a pending test stall is taken at launch time, so such a call is not captured (the
+  // stall would stay in a cached graph)
+  if (st->no_graph || test_stalls_pending()) {
     enqueue_sequence(st, q, v, g, T, n_iter, o, user);
     if (st->host_error) return FWPKM_ERR_CUDA;
     return last_cuda();
@@ -1028,6 +1046,9 @@ fwpkm_status fwpkm_sync(fwpkm_state* st, void* stream) {
     // a kernel that gave up may have left arrival counters between launches non-zero
     if (h == DEV_TIMEOUT && st->wk.af_cnt &&
         cudaMemset(st->wk.af_cnt, 0, sizeof(int) * 4 * (size_t)st->dm.M) != cudaSuccess)
+      return last_cuda();
+    if (h == DEV_TIMEOUT && st->wk.vl_cnt &&
+        cudaMemset(st->wk.vl_cnt, 0, sizeof(unsigned) * 2 * (size_t)st->dm.M) != cudaSuccess)
       return last_cuda();
     if (st->hstat) *(volatile int*)st->hstat = DEV_OK;
     return status_of_device(h);

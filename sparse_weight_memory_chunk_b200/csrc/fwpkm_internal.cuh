@@ -36,11 +36,12 @@ inline fwpkm_status status_of_device(int h) {
 // kernels that should wait once on a barrier that nothing completes.  Returns 1 (and
 // counts one down) while any remain.
 int take_test_stall();
+bool test_stalls_pending();
 
 // Kernel kinds for the launch counter / per-kernel timing.
 enum KernelKind : int { KK_NONE = 0, KK_GATHER = 1, KK_WRITE = 2, KK_SCORE = 3, KK_CART = 4,
                         KK_SORT = 5, KK_ADDR = 6, KK_OTHER = 7, KK_TOPK = 8, KK_PREP = 9, KK_PBAR = 10,
-                        KK_WBUILD = 11, KK_FUSED = 12, KK_LAST = 12 };
+                        KK_WBUILD = 11, KK_FUSED = 12, KK_VLOOP = 13, KK_LAST = 13 };
 
 struct Dims {
   int n, h, d, dv, k, C, M;
@@ -84,6 +85,7 @@ struct Work {
   int* pbar_cnt;     // [M*2][ceil(n/256)] arrival counters of the pbar column blocks (zero between launches)
   float* af_part;    // [M*2][n/128][2][256] one-launch addressing: every CTA's partial Z_t and L_t
   int* af_cnt;       // [M*2][2]           its arrival counters (zero between launches)
+  unsigned* vl_cnt;  // [M][2]             persistent value loop: arrivals, exits (zero between launches)
   // Every array above is memory-major except the bf16 pieces (Kpc, Wt), whose piece
   // stride is P_all problems; a Work for a group of memories is the same carve with its
   // pointers advanced to the group's first memory (see group_work).
@@ -181,6 +183,13 @@ int launch_resid(const Dims& d, const Work& w, const void* v, const float* g, lo
                  int len, const void* v_next, cudaStream_t s);
 // One read-modify-write per touched row of the chunk starting at workspace token wt0.
 int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s);
+// Frozen keys: the read and write of chunks [c0, c1) of every table in one persistent
+// launch (v, g, o of stride T per table, as for launch_gather with the lookahead target).
+// Returns 0 (nothing launched) when the loop is switched off (FWPKM_VALUE_LOOP=0) or
+// the GPU cannot hold the grid; the caller then launches the chunks one by one.
+int launch_value_loop(const Dims& d, const Work& w, float* V, const void* v, const float* g, int T, int c0, int c1,
+                      float* o, cudaStream_t s);
+bool value_loop_enabled();
 // Entropy key step for the chunk whose distances are in Dfull/Z (`len` tokens).
 int launch_address(const Dims& d, const Work& w, float* K1, float* K2, const void* q,
                    long long q_stride, int len, cudaStream_t s);
@@ -285,6 +294,31 @@ inline void launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   cfg.numAttrs = na;
   set_carveout((const void*)kern);
   cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// A cooperative launch: every CTA of the grid is resident at once, which a kernel whose
+// CTAs wait for one another needs (no programmatic dependency: it starts after the
+// stream's previous kernel has completed).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_coop(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                               Args... args) {
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  attr[na].id = cudaLaunchAttributeCooperative;
+  attr[na++].val.cooperative = 1;
+  if (launch_priority_set) {
+    attr[na].id = cudaLaunchAttributePriority;
+    attr[na++].val.priority = launch_priority;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  set_carveout((const void*)kern);
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
 // Device side of programmatic dependent launch: wait until the preceding kernel of the

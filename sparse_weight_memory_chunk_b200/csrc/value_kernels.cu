@@ -43,12 +43,24 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
+// COHERENT: the row may have been written earlier in the same launch by another SM (the
+// persistent value loop), so the load goes to L2 (.cg) and never hits a stale L1 line.
+template <bool COHERENT>
 __device__ __forceinline__ float4 ld_stream(const float4* p, uint64_t pol) {
   float4 v;
-  asm volatile("ld.global.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "l"(p), "l"(pol));
+  if (COHERENT)
+    asm volatile("ld.global.cg.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(pol));
+  else
+    asm volatile("ld.global.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(pol));
   return v;
+}
+template <bool COHERENT>
+__device__ __forceinline__ float4 ld_row4(const float4* p) {
+  return COHERENT ? __ldcg(p) : *p;
 }
 // r = gw * (vhat - tau), tau = z(u) or u.  Shared by the fused and the streaming path
 // so both give the same bits.
@@ -124,19 +136,17 @@ __device__ __forceinline__ const VT* target_src(const Dims& dm, const VT* v, con
 constexpr int GATHER_TOK = VAL_WARPS / 2;
 // HEADS: the memories of a sequence share its value table (dm.H > 1, up to 64 rows per
 // token); false compiles the one-head kernel (k <= 32 rows, one entry per lane).
-template <typename VT, int VPL, bool HEADS>
-__global__ void __launch_bounds__(VAL_WARPS * 32, 4)
-gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict__ v,
-              const float* __restrict__ g, long long stride, int wt0, int len, float* __restrict__ o,
-              int fuse_resid, const VT* __restrict__ v_next) {
-  pdl_wait();
-  pdl_trigger();
-  __shared__ float4 s_part[GATHER_TOK][VPL][32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tl = warp >> 1, half = warp & 1;
-  const int i = blockIdx.x * GATHER_TOK + tl;
-  const int m = blockIdx.y;  // the value table (sequence); its heads are memories m H .. m H + H - 1
-  const bool active = i < len;
+//
+// gather_token is one token's read by its two warps (`half` 0 and 1): every thread of the
+// CTA calls it, inactive tokens too, since it holds a CTA barrier.  s_tok is the token's
+// slot of the CTA's partial-sum array.  m is the value table (sequence); its heads are
+// memories m H .. m H + H - 1.
+template <typename VT, int VPL, bool HEADS, bool COHERENT>
+__device__ __forceinline__ void gather_token(const Dims& dm, const Work& w, const float* __restrict__ V,
+                                             const VT* __restrict__ v, const float* __restrict__ g,
+                                             long long stride, int wt0, int len, float* __restrict__ o,
+                                             int fuse_resid, const VT* __restrict__ v_next, int m, int i,
+                                             bool active, int half, int lane, float4 (*s_tok)[32]) {
   const int k = dm.k, dv4 = dm.dv >> 2, H = HEADS ? dm.H : 1;
   const int R = H * k;       // rows read by the token: entry e = (head e / k, rank e % k)
   const long long tok = (long long)wt0 + i;
@@ -161,12 +171,15 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
       myw2 = w.w[o] * invH;
     }
   }
-  // half 0 prefetches the token's value row and gate
-  float4 xv[VPL];
+  // half 0 prefetches the token's value row, gate and write target (no V row is needed for
+  // them, so their loads overlap the gather instead of following it)
+  float4 xv[VPL], tv[VPL];
   float gt = 0.f;
+  const VT* u = (active && fuse_resid) ? target_src<VT>(dm, v, v_next, stride, m, i, len) : nullptr;
   if (active && half == 0) {
     gt = g[(long long)m * stride + i];
     load_row<VT, VPL>(dm, v + ((long long)m * stride + i) * dm.dv, xv, lane);
+    load_row<VT, VPL>(dm, u, tv, lane);
   }
   const float4* Vm = reinterpret_cast<const float4*>(V + (size_t)m * dm.N * dm.dv);
   float4 acc[VPL];
@@ -186,7 +199,7 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
       for (int c = 0; c < VPL; ++c) {
         int e4 = lane + 32 * c;
         if (e4 < dv4) {
-          float4 x = ld_stream(row + e4, pol);
+          float4 x = ld_stream<COHERENT>(row + e4, pol);
           acc[c].x = fmaf(wr, x.x, acc[c].x); acc[c].y = fmaf(wr, x.y, acc[c].y);
           acc[c].z = fmaf(wr, x.z, acc[c].z); acc[c].w = fmaf(wr, x.w, acc[c].w);
         }
@@ -195,13 +208,13 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
   }
   if (half == 1) {
 #pragma unroll
-    for (int c = 0; c < VPL; ++c) s_part[tl][c][lane] = acc[c];
+    for (int c = 0; c < VPL; ++c) s_tok[c][lane] = acc[c];
   }
   __syncthreads();
   if (half == 1 || !active) return;
 #pragma unroll
   for (int c = 0; c < VPL; ++c) {
-    const float4 b = s_part[tl][c][lane];
+    const float4 b = s_tok[c][lane];
     acc[c].x += b.x; acc[c].y += b.y; acc[c].z += b.z; acc[c].w += b.w;
   }
   float4* orow = reinterpret_cast<float4*>(o + ((long long)m * stride + i) * dm.dv);
@@ -219,11 +232,10 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
   // resid rows are chunk-local: a call may start inside a chunk (token-at-a-time reads)
   float4* rrow = reinterpret_cast<float4*>(w.resid + ((size_t)m * dm.C + wt0 % dm.C + i) * dm.dv);
   if (fuse_resid) {
-    const VT* u = target_src<VT>(dm, v, v_next, stride, m, i, len);
     if (u == nullptr) return;
     const float gw = (dm.flags & FWPKM_GATE_WEIGHT) ? gt : 1.f;
     float4 r[VPL];
-    residual<VT, VPL>(dm, acc, u, gw, r, lane);
+    residual_of<VPL>(dm, acc, tv, gw, r, lane);
 #pragma unroll
     for (int c = 0; c < VPL; ++c) {
       int e4 = lane + 32 * c;
@@ -236,6 +248,21 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
       if (e4 < dv4) rrow[e4] = acc[c];
     }
   }
+}
+
+template <typename VT, int VPL, bool HEADS>
+__global__ void __launch_bounds__(VAL_WARPS * 32, 4)
+gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict__ v,
+              const float* __restrict__ g, long long stride, int wt0, int len, float* __restrict__ o,
+              int fuse_resid, const VT* __restrict__ v_next) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float4 s_part[GATHER_TOK][VPL][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tl = warp >> 1;
+  const int i = blockIdx.x * GATHER_TOK + tl;
+  gather_token<VT, VPL, HEADS, false>(dm, w, V, v, g, stride, wt0, len, o, fuse_resid, v_next, blockIdx.y, i,
+                                      i < len, warp & 1, lane, s_part[tl]);
 }
 
 // Streaming path: resid holds vhat from the forward call; turn it into r_t in place.
@@ -402,15 +429,10 @@ __device__ __forceinline__ void store_row(float* Vm, int slot, const Dims& dm, c
 
 // HEADS: the memories of a sequence share its value table (dm.H > 1): weights s'/H and
 // N_read counted in distinct tokens; false compiles the one-head kernel (N_read = pairs).
-template <int VPL, int WB, bool HEADS>
-__global__ void __launch_bounds__(WR_WARPS * 32)
-write_batched_kernel(Dims dm, Work w, float* __restrict__ V, int wt0, int warps_per_mem) {
-  pdl_wait();
-  pdl_trigger();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * WR_WARPS + warp;
-  const int m = gw / warps_per_mem, wi = gw - m * warps_per_mem;  // m: the value table (sequence)
-  if (m >= dm.B) return;
+// write_warp is the work of warp wi of table m's warps_per_mem warps.
+template <int VPL, int WB, bool HEADS, bool COHERENT>
+__device__ __forceinline__ void write_warp(const Dims& dm, const Work& w, float* __restrict__ V, int wt0, int m,
+                                           int wi, int warps_per_mem, int lane) {
   const int C = dm.C, k = dm.k, dv4 = dm.dv >> 2, H = HEADS ? dm.H : 1, kh = k * H;
   const int kshift = (kh & (kh - 1)) == 0 ? __popc(kh - 1) : -1;
   const float invH = 1.f / (float)H;
@@ -489,8 +511,8 @@ write_batched_kernel(Dims dm, Work w, float* __restrict__ V, int wt0, int warps_
 #pragma unroll
         for (int c = 0; c < VPL; ++c) {
           const int e4 = lane + 32 * c;
-          R[u][c] = (in && e4 < dv4) ? rr[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
-          Vh[u][c] = (hd && okslot && e4 < dv4) ? vr[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+          R[u][c] = (in && e4 < dv4) ? ld_row4<COHERENT>(rr + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          Vh[u][c] = (hd && okslot && e4 < dv4) ? ld_row4<COHERENT>(vr + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
       // ---- accumulate in list order; a segment is stored at its last pair ----
@@ -539,6 +561,123 @@ write_batched_kernel(Dims dm, Work w, float* __restrict__ V, int wt0, int warps_
       }
     }
     if (lim < 32) break;  // a peer's head (or the list's end) was reached in this window
+  }
+}
+
+template <int VPL, int WB, bool HEADS>
+__global__ void __launch_bounds__(WR_WARPS * 32)
+write_batched_kernel(Dims dm, Work w, float* __restrict__ V, int wt0, int warps_per_mem) {
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * WR_WARPS + warp;
+  const int m = gw / warps_per_mem, wi = gw - m * warps_per_mem;  // m: the value table (sequence)
+  if (m >= dm.B) return;
+  write_warp<VPL, WB, HEADS, false>(dm, w, V, wt0, m, wi, warps_per_mem, lane);
+}
+
+// ---------------------------------------------------------------------------
+// Persistent value loop (frozen keys).  With the slot lists of a run of chunks already
+// made, one launch takes every chunk of the run through its read (gather_token, all tables)
+// and its write (write_warp, all tables) on every SM: no launch, ramp or drain per kernel.
+// Two grid-wide arrivals order the phases: the write of chunk c starts when every
+// residual of c is stored, the read of c+1 when every row of c's write is stored.  Rows
+// and residuals made inside the launch are read through L2 (COHERENT loads).  The grid is
+// launched cooperatively and never exceeds the CTAs that fit on the GPU, so each CTA it
+// waits for is resident; each wait is still bounded (VL_TIMEOUT_NS), after which the CTA
+// latches FWPKM_ERR_TIMEOUT and returns, leaving the counters for fwpkm_sync to clear.
+// The arithmetic is that of the per-chunk kernels, in the same order: the bits agree.
+// ---------------------------------------------------------------------------
+constexpr uint64_t VL_TIMEOUT_NS = 200ull * 1000 * 1000;
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t vl_clock() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Arrive on the grid counter and wait until `target` CTAs have arrived in total.  False:
+// this CTA gave up (the counter did not reach the target in time).
+__device__ __forceinline__ bool grid_arrive_wait(unsigned* cnt, unsigned target, const Work& w, int* s_abort) {
+  __syncthreads();  // this CTA's stores of the phase are issued
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(cnt, 1u);
+    const uint64_t deadline = vl_clock() + VL_TIMEOUT_NS;
+    uint32_t spins = 0;
+    while (ld_acquire_u32(cnt) < target) {
+      __nanosleep(32);
+      if ((++spins & 15u) == 0 && vl_clock() > deadline) {
+        raise_status(w.status, w.hstat, DEV_TIMEOUT);
+        *s_abort = 1;
+        break;
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return *s_abort == 0;
+}
+
+template <int VPL>
+struct VlOcc {  // CTAs per SM the loop is compiled for (the write holds up to ~176 registers)
+  static constexpr int value = VPL <= 4 ? 2 : 1;
+};
+
+template <typename VT, int VPL, int WB, bool HEADS>
+__global__ void __launch_bounds__(VAL_WARPS * 32, VlOcc<VPL>::value)
+value_loop_kernel(Dims dm, Work w, float* __restrict__ V, const VT* __restrict__ v, const float* __restrict__ g,
+                  int T, int c0, int c1, float* __restrict__ o, int warps_per_mem, int stall) {
+  __shared__ float4 s_part[GATHER_TOK][VPL][32];
+  __shared__ int s_abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tl = warp >> 1, half = warp & 1;
+  if (threadIdx.x == 0) s_abort = 0;
+  unsigned* arrivals = w.vl_cnt;
+  unsigned* exits = w.vl_cnt + 1;
+  const unsigned G = gridDim.x;
+  // test hook: the first wait's target is one no launch reaches
+  unsigned target = stall ? 0x40000000u : 0u;
+  const int C = dm.C, dv = dm.dv;
+  for (int c = c0; c < c1; ++c) {
+    const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
+    const VT* vc = v + (long long)t0 * dv;
+    const VT* vn = (t0 + len < T) ? v + (long long)(t0 + len) * dv : nullptr;
+    if (c > c0) {  // the previous chunk's rows are written
+      target += G;
+      if (!grid_arrive_wait(arrivals, target, w, &s_abort)) return;
+    }
+    const int ntok = dm.B * len;
+    for (int base = blockIdx.x * GATHER_TOK; base < ntok; base += G * GATHER_TOK) {
+      const int j = base + tl;
+      const bool active = j < ntok;
+      const int m = active ? j / len : 0, i = active ? j - m * len : 0;
+      gather_token<VT, VPL, HEADS, true>(dm, w, V, vc, g + t0, T, t0, len, o + (long long)t0 * dv, 1, vn, m, i,
+                                        active, half, lane, s_part[tl]);
+      __syncthreads();  // s_part is refilled by the next token
+    }
+    target += G;
+    if (!grid_arrive_wait(arrivals, target, w, &s_abort)) return;  // every residual of chunk c is stored
+    const int nvw = dm.B * warps_per_mem;
+    for (int vw = blockIdx.x * VAL_WARPS + warp; vw < nvw; vw += G * VAL_WARPS) {
+      const int m = vw / warps_per_mem;
+      write_warp<VPL, WB, HEADS, true>(dm, w, V, t0, m, vw - m * warps_per_mem, warps_per_mem, lane);
+    }
+  }
+  // the last CTA out (every CTA has passed every wait) zeroes the counters for the next launch
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(exits, 1u) == G - 1) {
+      *arrivals = 0;
+      *exits = 0;
+      __threadfence();
+    }
   }
 }
 
@@ -664,6 +803,17 @@ static int launch_write_v1(const Dims& d, const Work& w, float* V, int wt0, cuda
   return 1;
 }
 
+// The fewest list positions a write warp is given (FWPKM_WRITE_MINPOS, default 32): a
+// chunk's list is split over at most P / this many warps per table.
+static int write_min_positions() {
+  static const int v = [] {
+    const char* e = getenv("FWPKM_WRITE_MINPOS");
+    const int x = e ? atoi(e) : 32;
+    return x < 4 ? 4 : x > 256 ? 256 : x;
+  }();
+  return v;
+}
+
 int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s) {
   static const bool v1 = [] {
     const char* e = getenv("FWPKM_WRITE_V1");
@@ -681,7 +831,7 @@ int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s
   auto go = [&](const void* kern, auto kfn) {
     const int resident_warps = resident_ctas(kern, WR_WARPS * 32) * WR_WARPS;
     int per_mem = (int)((long long)resident_warps * share / 100 / d.B);
-    const int most = (d.C * d.k * d.H + 31) / 32;
+    const int most = (d.C * d.k * d.H + write_min_positions() - 1) / write_min_positions();
     if (per_mem > most) per_mem = most;
     if (per_mem < 1) per_mem = 1;
     const int blocks = (d.B * per_mem + WR_WARPS - 1) / WR_WARPS;
@@ -698,6 +848,75 @@ int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s
   }
 #undef FWPKM_WRITE_GO
   return 1;
+}
+
+// The same for the write phase of the persistent loop (FWPKM_LOOP_MINPOS, default 8): there
+// the grid's warps are resident anyway, and shorter ranges mean fewer dependent batches.
+static int loop_min_positions() {
+  static const int v = [] {
+    const char* e = getenv("FWPKM_LOOP_MINPOS");
+    const int x = e ? atoi(e) : 8;
+    return x < 4 ? 4 : x > 256 ? 256 : x;
+  }();
+  return v;
+}
+
+bool value_loop_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("FWPKM_VALUE_LOOP");
+    if (e && e[0] == '0') return false;
+    int dev = 0, coop = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    return coop != 0;
+  }();
+  return on;
+}
+
+int launch_value_loop(const Dims& d, const Work& w, float* V, const void* v, const float* g, int T, int c0, int c1,
+                      float* o, cudaStream_t s) {
+  if (c1 <= c0) return 0;
+  if (!value_loop_enabled() || w.vl_cnt == nullptr) return 0;
+  const int stall = take_test_stall();
+  auto go = [&](auto kfn, auto vt) -> int {
+    using VT = decltype(vt);
+    const int resident = resident_ctas((const void*)kfn, VAL_WARPS * 32);
+    // write warps per table: one per loop_min_positions() list positions, at most the grid's warps
+    int per_mem = (d.C * d.k * d.H + loop_min_positions() - 1) / loop_min_positions();
+    if ((long long)per_mem * d.B > (long long)resident * VAL_WARPS) per_mem = resident * VAL_WARPS / d.B;
+    if (per_mem < 1) per_mem = 1;
+    const int gather_ctas = (d.B * d.C + GATHER_TOK - 1) / GATHER_TOK;
+    const int write_ctas = (d.B * per_mem + VAL_WARPS - 1) / VAL_WARPS;
+    int grid = gather_ctas > write_ctas ? gather_ctas : write_ctas;
+    if (grid > resident) grid = resident;
+    const cudaError_t e = launch_coop(kfn, dim3((unsigned)grid), dim3(VAL_WARPS * 32), 0, s, d, w, V,
+                                      (const VT*)v, g, T, c0, c1, o, per_mem, stall);
+    return e == cudaSuccess ? 1 : -1;
+  };
+#define FWPKM_VLOOP_GO(VTT, VPLV, WBV)                                                     \
+  (d.H > 1 ? go(value_loop_kernel<VTT, VPLV, WBV, true>, VTT()) : go(value_loop_kernel<VTT, VPLV, WBV, false>, VTT()))
+  const int vpl = vpl_of(d.dv);
+  int r;
+  if (d.qv_bf16) {
+    switch (vpl) {
+      case 1: r = FWPKM_VLOOP_GO(__nv_bfloat16, 1, 8); break;
+      case 2: r = FWPKM_VLOOP_GO(__nv_bfloat16, 2, 4); break;
+      case 4: r = FWPKM_VLOOP_GO(__nv_bfloat16, 4, 2); break;
+      default: r = FWPKM_VLOOP_GO(__nv_bfloat16, 8, 1); break;
+    }
+  } else {
+    switch (vpl) {
+      case 1: r = FWPKM_VLOOP_GO(float, 1, 8); break;
+      case 2: r = FWPKM_VLOOP_GO(float, 2, 4); break;
+      case 4: r = FWPKM_VLOOP_GO(float, 4, 2); break;
+      default: r = FWPKM_VLOOP_GO(float, 8, 1); break;
+    }
+  }
+#undef FWPKM_VLOOP_GO
+  return r;
 }
 
 }  // namespace fwpkm

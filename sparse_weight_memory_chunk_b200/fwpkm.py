@@ -21,7 +21,7 @@ F32, BF16 = 0, 1
 KEY_UPDATE, TARGET_NORM, LOOKAHEAD, GATE_WEIGHT = 1, 2, 4, 8
 DEFAULT_FLAGS = TARGET_NORM | LOOKAHEAD | GATE_WEIGHT
 KIND = {"gather": 1, "write": 2, "score": 3, "cartesian": 4, "sort": 5, "address": 6, "other": 7, "topk": 8,
-        "prep": 9, "pbar": 10, "wbuild": 11, "fused": 12, "all": 100}
+        "prep": 9, "pbar": 10, "wbuild": 11, "fused": 12, "value_loop": 13, "all": 100}
 KIND_NAME = {v: k for k, v in KIND.items()}
 
 
