@@ -158,6 +158,25 @@ fwpkm_status fwpkm_write_chunk(fwpkm_state* st, const void* v_next, void* stream
 fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, const float* g,
                                 int T, int n_iter, float* o, void* stream);
 
+/* fwpkm_run_sequence from host memory (no counterpart in the paper: the end-to-end call).
+ * q, v, g, o are HOST buffers in the fwpkm_run_sequence layout (seq_stride = T), and
+ * must be page-locked (cudaHostAlloc, or cudaHostRegister'd): anything else returns
+ * FWPKM_ERR_INVALID_ARG.  The call copies chunk c's inputs to device scratch while
+ * earlier chunks compute (cudaMemcpy2DAsync on an internal stream; the tensor-core path
+ * also makes chunk c's query norms there), starts each chunk's kernels when its inputs
+ * (and the lookahead row after it) have landed, and copies each chunk's final-pass o back
+ * as soon as it is written, so the copies overlap the compute.  Everything is enqueued on
+ * `stream` (captured once into the state's cached graph, like fwpkm_run_sequence); the
+ * host buffers must stay valid, and o unread, until the stream passes the call.
+ *   scratch  device, 256-byte aligned, >= fwpkm_run_sequence_host_scratch_size(cfg, T)
+ *            bytes (device copies of q, v, g and o, each on a 256-byte boundary); too
+ *            small: FWPKM_ERR_WORKSPACE.
+ * Results are bit-identical to fwpkm_run_sequence on the same inputs. */
+fwpkm_status fwpkm_run_sequence_host_scratch_size(const fwpkm_config* cfg, int T, size_t* bytes);
+fwpkm_status fwpkm_run_sequence_host(fwpkm_state* st, const void* q, const void* v, const float* g,
+                                     int T, int n_iter, float* o, void* scratch, size_t scratch_bytes,
+                                     void* stream);
+
 /* Token-at-a-time inference ("Fast-weight Product Key Memory" (paperlayer summary),
  * §A.1: at inference the memory accumulates (q_t, v_{t+1}) pairs and writes once a
  * chunk's worth is ready).  Each call reads n_tok >= 1 new tokens of every memory at once,

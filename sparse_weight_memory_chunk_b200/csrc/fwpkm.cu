@@ -25,10 +25,21 @@ static std::atomic<uint64_t> g_launches{0};
 
 struct SeqKey {
   const void *q, *v, *g, *o;
+  const void *hq, *hv, *hg, *ho;  // host buffers of fwpkm_run_sequence_host (else null)
   int T, n_iter, prof_kind;
   bool operator==(const SeqKey& x) const {
-    return q == x.q && v == x.v && g == x.g && o == x.o && T == x.T && n_iter == x.n_iter && prof_kind == x.prof_kind;
+    return q == x.q && v == x.v && g == x.g && o == x.o && hq == x.hq && hv == x.hv && hg == x.hg && ho == x.ho &&
+           T == x.T && n_iter == x.n_iter && prof_kind == x.prof_kind;
   }
+};
+
+// Host inputs and output of fwpkm_run_sequence_host: page-locked buffers laid out like the
+// device ones, copied chunk by chunk beside the compute.
+struct HostIO {
+  const void* q;
+  const void* v;
+  const float* g;
+  float* o;
 };
 
 struct fwpkm_state {
@@ -61,6 +72,8 @@ struct fwpkm_state {
   static constexpr int MAX_GROUPS = 8;
   int groups;
   cudaStream_t sK[MAX_GROUPS], sS[MAX_GROUPS], sV[MAX_GROUPS], sCap;
+  // host-buffer calls: input copies, the query preparation of each chunk, output copies
+  cudaStream_t sH[MAX_GROUPS], sP[MAX_GROUPS], sD[MAX_GROUPS];
   // scheduling priorities of the kernels of the three chains (the addressing chain is the
   // critical path: highest); use_prio = 0 (FWPKM_PRIO=0) leaves them all at the default
   int use_prio, prio_K, prio_S, prio_V;
@@ -457,11 +470,15 @@ fwpkm_status fwpkm_init_state(const fwpkm_config* cfg, float* K1, float* K2, flo
   }
   st->sCap = nullptr;
   ok = ok && cudaStreamCreateWithFlags(&st->sCap, cudaStreamNonBlocking) == cudaSuccess;
-  for (int gi = 0; gi < fwpkm_state::MAX_GROUPS; ++gi) st->sK[gi] = st->sS[gi] = st->sV[gi] = nullptr;
+  for (int gi = 0; gi < fwpkm_state::MAX_GROUPS; ++gi)
+    st->sK[gi] = st->sS[gi] = st->sV[gi] = st->sH[gi] = st->sP[gi] = st->sD[gi] = nullptr;
   for (int gi = 0; gi < st->groups && ok; ++gi)
     ok = cudaStreamCreateWithFlags(&st->sK[gi], cudaStreamNonBlocking) == cudaSuccess &&
          cudaStreamCreateWithFlags(&st->sS[gi], cudaStreamNonBlocking) == cudaSuccess &&
-         cudaStreamCreateWithFlags(&st->sV[gi], cudaStreamNonBlocking) == cudaSuccess;
+         cudaStreamCreateWithFlags(&st->sV[gi], cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&st->sH[gi], cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&st->sP[gi], cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&st->sD[gi], cudaStreamNonBlocking) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     fwpkm_destroy_state(st);
@@ -489,6 +506,9 @@ void fwpkm_destroy_state(fwpkm_state* st) {
     if (st->sK[gi]) cudaStreamDestroy(st->sK[gi]);
     if (st->sS[gi]) cudaStreamDestroy(st->sS[gi]);
     if (st->sV[gi]) cudaStreamDestroy(st->sV[gi]);
+    if (st->sH[gi]) cudaStreamDestroy(st->sH[gi]);
+    if (st->sP[gi]) cudaStreamDestroy(st->sP[gi]);
+    if (st->sD[gi]) cudaStreamDestroy(st->sD[gi]);
   }
   if (st->sCap) cudaStreamDestroy(st->sCap);
   for (cudaEvent_t e : st->ev) cudaEventDestroy(e);
@@ -726,7 +746,7 @@ fwpkm_status fwpkm_stream_flush(fwpkm_state* st, void* stream) {
 // lists and weights are overwritten).
 static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk, float* K1, float* K2, float* V,
                           const void* q, const void* v, const float* g, int T, int n_iter, float* o,
-                          cudaStream_t origin) {
+                          const HostIO* hio, cudaStream_t origin) {
   const size_t es = qv_size(d);
   const int C = d.C;
   const bool ku = (d.flags & FWPKM_KEY_UPDATE) != 0;
@@ -755,6 +775,56 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
   dep(origin, sS);
   dep(origin, sV);
 
+  // Host buffers: chunk c's inputs are copied to the device on sH, in chunk order (copies
+  // only, so they run ahead of the compute); on the tensor-core path sP then makes the
+  // chunk's query norms and feature-major half-queries.  in_ready[c] marks both; each
+  // consumer waits only for the chunks it reads.  o goes back on sD as soon as the last
+  // pass's value work of a chunk (or window) has ended.
+  std::vector<cudaEvent_t> in_ready;
+  cudaStream_t sH = nullptr, sP = nullptr, sD = nullptr;
+  if (hio) {
+    sH = st->serial ? sK : st->sH[gi];
+    sP = st->serial ? sK : st->sP[gi];
+    sD = st->serial ? sK : st->sD[gi];
+    dep(origin, sH);
+    dep(origin, sP);
+    dep(origin, sD);
+    in_ready.resize(nch);
+    auto h2d = [&](const void* dst, const void* src, size_t row_bytes, size_t width, int rows) {
+      if (cudaMemcpy2DAsync(const_cast<void*>(dst), row_bytes, src, row_bytes, width, rows, cudaMemcpyHostToDevice,
+                            sH) != cudaSuccess)
+        st->host_error = 1;
+    };
+    for (int c = 0; c < nch; ++c) {
+      const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
+      h2d(offs(q, (long long)t0 * d.d, es), offs(hio->q, (long long)t0 * d.d, es), (size_t)T * d.d * es,
+          (size_t)len * d.d * es, d.M);
+      h2d(offs(v, (long long)t0 * d.dv, es), offs(hio->v, (long long)t0 * d.dv, es), (size_t)T * d.dv * es,
+          (size_t)len * d.dv * es, d.B);
+      h2d(g + t0, hio->g + t0, (size_t)T * 4, (size_t)len * 4, d.B);
+      in_ready[c] = mark(sH);
+      if (tc) {
+        cudaStreamWaitEvent(sP, in_ready[c], 0);
+        const void* qc = offs(q, (long long)t0 * d.d, es);
+        run(st, KK_PREP, sP, [&] { return launch_qnorm(d, wk, qc, T, t0, len, sP); });
+        if (qt_whole) run(st, KK_PREP, sP, [&] { return launch_qtrans(d, wk, qc, T, t0, len, sP); });
+        in_ready[c] = mark(sP);
+      }
+    }
+  }
+  auto wait_in = [&](cudaStream_t s, int c) {  // inputs of chunks <= c are on the device
+    if (hio) cudaStreamWaitEvent(s, in_ready[c < nch ? c : nch - 1], 0);
+  };
+  auto copy_out = [&](cudaStream_t from, int c0, int c1) {  // o of chunks [c0, c1) to the host
+    if (!hio) return;
+    cudaStreamWaitEvent(sD, mark(from), 0);
+    const long long t0 = (long long)c0 * C, t1 = (long long)c1 * C < T ? (long long)c1 * C : T;
+    const size_t pitch = (size_t)T * d.dv * 4;
+    if (cudaMemcpy2DAsync(hio->o + t0 * d.dv, pitch, o + t0 * d.dv, pitch, (size_t)(t1 - t0) * d.dv * 4, d.B,
+                          cudaMemcpyDeviceToHost, sD) != cudaSuccess)
+      st->host_error = 1;
+  };
+
   auto value_chunk = [&](int c) {
     const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
     const void* vc = offs(v, (long long)t0 * d.dv, es);
@@ -765,7 +835,7 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
     run(st, KK_WRITE, sV, [&] { return launch_write(d, wk, V, t0, sV); });
   };
 
-  if (tc) {
+  if (tc && !hio) {
     // the three per-call preparations are independent: query norms (selection stream),
     // query transpose (values stream) and key pieces (addressing stream) run side by side
     run(st, KK_PREP, sS, [&] { return launch_qnorm(d, wk, q, T, 0, T, sS); });
@@ -775,6 +845,8 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
     run(st, KK_PREP, sK, [&] { return launch_keyprep(d, wk, K1, K2, sK); });
     cudaStreamWaitEvent(sK, qn_done, 0);
     cudaStreamWaitEvent(sK, qt_done, 0);
+  } else if (tc) {
+    run(st, KK_PREP, sK, [&] { return launch_keyprep(d, wk, K1, K2, sK); });
   }
   if (!ku) {
     // frozen keys: address window by window on sK; the value loop of a window starts as
@@ -783,6 +855,7 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
     std::vector<cudaEvent_t> ready;
     for (int w0 = 0; w0 < T; w0 += wtok) {
       const int wl = T - w0 < wtok ? T - w0 : wtok;
+      wait_in(sK, (w0 + wl - 1) / C);
       if (tc) {
         run(st, KK_SCORE, sK, [&] { return launch_tc_score(d, wk, q, T, T, w0, w0, wl, false, sK); });
         run(st, KK_TOPK, sK, [&] { return launch_select(d, wk, w0, wl, nullptr, nullptr, sK); });
@@ -803,11 +876,13 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
       for (int c = 0; c < nch; c += (pass == 0 ? wch : nch)) {
         if (pass == 0) cudaStreamWaitEvent(sV, ready[c / wch], 0);
         const int c1 = pass > 0 ? nch : (c + wch < nch ? c + wch : nch);
+        if (pass == 0) wait_in(sV, c1);  // the window's v, g and the lookahead row after it
         if (vloop) {
           run(st, KK_VLOOP, sV, [&] { return launch_value_loop(d, wk, V, v, g, T, c, c1, o, sV); });
         } else {
           for (int cc = c; cc < c1; ++cc) value_chunk(cc);
         }
+        if (pass == n_iter - 1) copy_out(sV, c, c1);
       }
   } else {
     const size_t dbuf = (size_t)wk.dfull_buf;
@@ -830,6 +905,7 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
         if (sel_done[c]) cudaStreamWaitEvent(sK, sel_done[c], 0);    // previous pass read A/Dsv
         if (topk_done[cnt & 1]) cudaStreamWaitEvent(sK, topk_done[cnt & 1], 0);  // buffer reuse
         if (sel_first && last_topk) cudaStreamWaitEvent(sK, last_topk, 0);
+        if (pass == 0) wait_in(sK, c);
         if (fused) {
           // the chunk's whole addressing step in one launch; the selection needs its rows
           run(st, KK_FUSED, sK, [&] {
@@ -865,20 +941,27 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
         // made it overlap the scoring and key-step GEMMs, which slowed them (1.82 against
         // 1.62 ms per step)
         cudaStreamWaitEvent(sV, sel_done[c], 0);
+        if (pass == 0) wait_in(sV, c + 1);  // v, g of the chunk and its lookahead row
         value_chunk(c);
         val_done[c] = mark(sV);
+        if (pass == n_iter - 1) copy_out(sV, c, c + 1);
       }
     }
   }
   dep(sK, origin);
   dep(sS, origin);
   dep(sV, origin);
+  if (hio) {
+    dep(sH, origin);
+    dep(sP, origin);
+    dep(sD, origin);
+  }
 }
 
 // Split the memories into st->groups contiguous groups and enqueue each as its own set of
 // chains (all of them fork from and join back to `origin`).
 static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, const float* g, int T, int n_iter,
-                             float* o, cudaStream_t origin) {
+                             float* o, const HostIO* hio, cudaStream_t origin) {
   const Dims& d = st->dm;
   const size_t es = qv_size(d);
   st->ev_next = 0;
@@ -890,19 +973,23 @@ static void enqueue_sequence(fwpkm_state* st, const void* q, const void* v, cons
     dg.B = dg.M / dg.H;  // one group when heads share V (dg.M = d.M)
     const Work wg = G == 1 ? st->wk : group_work(d, st->wk, m0);
     const size_t kh = (size_t)m0 * d.n * d.h;
+    HostIO hg;
+    if (hio) {
+      hg.q = offs(hio->q, (long long)m0 * T * d.d, es);
+      hg.v = offs(hio->v, (long long)m0 * T * d.dv, es);
+      hg.g = hio->g + (size_t)m0 * T;
+      hg.o = hio->o + (size_t)m0 * T * d.dv;
+    }
     enqueue_group(st, gi, dg, wg, st->K1 + kh, st->K2 + kh, st->V + (size_t)m0 * d.N * d.dv,
                   offs(q, (long long)m0 * T * d.d, es), offs(v, (long long)m0 * T * d.dv, es), g + (size_t)m0 * T,
-                  T, n_iter, o + (size_t)m0 * T * d.dv, origin);
+                  T, n_iter, o + (size_t)m0 * T * d.dv, hio ? &hg : nullptr, origin);
   }
 }
 
-fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, const float* g, int T,
-                                int n_iter, float* o, void* stream) {
-  NvtxRange nvtx_range("fwpkm_run_sequence");
-  if (!st) return FWPKM_ERR_INVALID_ARG;
-  if (T == 0) return FWPKM_OK;
-  if (!q || !v || !g || !o || T < 0 || T > st->wk.max_T || n_iter < 1) return FWPKM_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4)) return FWPKM_ERR_INVALID_ARG;
+// The schedule of fwpkm_run_sequence (hio = nullptr) and fwpkm_run_sequence_host, captured
+// into a cached graph.  Arguments are checked by the callers.
+static fwpkm_status run_sequence_impl(fwpkm_state* st, const void* q, const void* v, const float* g, int T,
+                                      int n_iter, float* o, const HostIO* hio, void* stream) {
   if (st->spos) return FWPKM_ERR_STATE;  // token-at-a-time chunk pending
   fwpkm_status ps = peek_status(st);
   if (ps != FWPKM_OK) return ps;
@@ -912,13 +999,14 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
   // a pending test stall is taken at launch time, so such a call is not captured (the
   // stall would stay in a cached graph)
   if (st->no_graph || test_stalls_pending()) {
-    enqueue_sequence(st, q, v, g, T, n_iter, o, user);
+    enqueue_sequence(st, q, v, g, T, n_iter, o, hio, user);
     if (st->host_error) return FWPKM_ERR_CUDA;
     return last_cuda();
   }
   // One CUDA graph per distinct call (arguments and timing kind), replayed while they stay
   // the same; the last two are kept.
-  const SeqKey key = {q, v, g, o, T, n_iter, st->prof_kind};
+  const SeqKey key = {q, v, g, o, hio ? hio->q : nullptr, hio ? hio->v : nullptr, hio ? (const void*)hio->g : nullptr,
+                      hio ? (const void*)hio->o : nullptr, T, n_iter, st->prof_kind};
   int slot = -1;
   for (int i = 0; i < fwpkm_state::NGRAPH; ++i)
     if (st->graph_exec[i] && st->graph_key[i] == key) slot = i;
@@ -932,7 +1020,7 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
     }
     const uint64_t before = g_launches.load();
     if (cudaStreamBeginCapture(st->sCap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return last_cuda();
-    enqueue_sequence(st, q, v, g, T, n_iter, o, st->sCap);
+    enqueue_sequence(st, q, v, g, T, n_iter, o, hio, st->sCap);
     cudaGraph_t graph = nullptr;
     cudaError_t e = cudaStreamEndCapture(st->sCap, &graph);
     st->graph_kernels[slot] = g_launches.load() - before;
@@ -957,6 +1045,67 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
   g_launches += st->graph_kernels[slot];
   st->ev_used = st->graph_ev_used[slot];
   return last_cuda();
+}
+
+fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, const float* g, int T,
+                                int n_iter, float* o, void* stream) {
+  NvtxRange nvtx_range("fwpkm_run_sequence");
+  if (!st) return FWPKM_ERR_INVALID_ARG;
+  if (T == 0) return FWPKM_OK;
+  if (!q || !v || !g || !o || T < 0 || T > st->wk.max_T || n_iter < 1) return FWPKM_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(g, 4)) return FWPKM_ERR_INVALID_ARG;
+  return run_sequence_impl(st, q, v, g, T, n_iter, o, nullptr, stream);
+}
+
+// ---- host buffers: device copies of q, v, g, o in caller scratch ----
+static size_t host_io_carve(const Dims& d, int T, char* base, void** q, void** v, float** g, float** o) {
+  const size_t es = qv_size(d);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return p;
+  };
+  void* pq = take(es * (size_t)d.M * T * d.d);
+  void* pv = take(es * (size_t)d.B * T * d.dv);
+  float* pg = (float*)take(4 * (size_t)d.B * T);
+  float* po = (float*)take(4 * (size_t)d.B * T * d.dv);
+  if (q) { *q = pq; *v = pv; *g = pg; *o = po; }
+  return off;
+}
+
+static bool host_pinned(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
+fwpkm_status fwpkm_run_sequence_host_scratch_size(const fwpkm_config* cfg, int T, size_t* bytes) {
+  fwpkm_status s = check_cfg(cfg);
+  if (s != FWPKM_OK) return s;
+  if (!bytes || T < 0) return FWPKM_ERR_INVALID_ARG;
+  *bytes = host_io_carve(make_dims(cfg), T, nullptr, nullptr, nullptr, nullptr, nullptr);
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_run_sequence_host(fwpkm_state* st, const void* q, const void* v, const float* g, int T,
+                                     int n_iter, float* o, void* scratch, size_t scratch_bytes, void* stream) {
+  NvtxRange nvtx_range("fwpkm_run_sequence_host");
+  if (!st) return FWPKM_ERR_INVALID_ARG;
+  if (T == 0) return FWPKM_OK;
+  if (!q || !v || !g || !o || !scratch || T < 0 || T > st->wk.max_T || n_iter < 1) return FWPKM_ERR_INVALID_ARG;
+  if (!aligned(scratch, ALIGN)) return FWPKM_ERR_INVALID_ARG;
+  if (!host_pinned(q) || !host_pinned(v) || !host_pinned(g) || !host_pinned(o)) return FWPKM_ERR_INVALID_ARG;
+  const Dims& d = st->dm;
+  if (scratch_bytes < host_io_carve(d, T, nullptr, nullptr, nullptr, nullptr, nullptr)) return FWPKM_ERR_WORKSPACE;
+  void *dq, *dv;
+  float *dg, *dout;
+  host_io_carve(d, T, (char*)scratch, &dq, &dv, &dg, &dout);
+  const HostIO hio = {q, v, g, o};
+  return run_sequence_impl(st, dq, dv, dg, T, n_iter, dout, &hio, stream);
 }
 
 // ---- the whole layer: projections in, the memory loop, projection out ----

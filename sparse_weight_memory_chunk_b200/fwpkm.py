@@ -77,6 +77,10 @@ def lib():
             "fwpkm_forward_chunk": ([_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P], ctypes.c_int),
             "fwpkm_write_chunk": ([_P, _P, _P], ctypes.c_int),
             "fwpkm_run_sequence": ([_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P], ctypes.c_int),
+            "fwpkm_run_sequence_host_scratch_size": ([C, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)],
+                                                     ctypes.c_int),
+            "fwpkm_run_sequence_host": ([_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_size_t, _P],
+                                        ctypes.c_int),
             "fwpkm_last_addressing": ([_P, ctypes.c_int, _P, _P, _P], ctypes.c_int),
             "fwpkm_chunk_step_noalloc": ([C, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P],
                                          ctypes.c_int),
@@ -149,6 +153,13 @@ def test_stall_waits(n_launches: int):
 def run_layer_scratch_size(cfg: Config, T: int) -> int:
     out = ctypes.c_size_t(0)
     _check(lib().fwpkm_run_layer_scratch_size(ctypes.byref(cfg), T, ctypes.byref(out)), "run_layer_scratch_size")
+    return out.value
+
+
+def run_sequence_host_scratch_size(cfg: Config, T: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().fwpkm_run_sequence_host_scratch_size(ctypes.byref(cfg), T, ctypes.byref(out)),
+           "run_sequence_host_scratch_size")
     return out.value
 
 
@@ -251,6 +262,18 @@ class State:
         T = q.shape[1] if T is None else T
         _check(lib().fwpkm_run_sequence(self.handle, _ptr(q), _ptr(v), _ptr(g), T, n_iter, _ptr(o),
                                         _stream(stream)), "run_sequence")
+
+    def run_sequence_host(self, q, v, g, o, T=None, n_iter=1, scratch=None, stream=None):
+        """run_sequence on page-locked HOST tensors q, v, g, o (copies overlap the compute);
+        `scratch`: a device uint8 tensor of run_sequence_host_scratch_size bytes (made here if
+        None).  Returns the scratch so that repeated calls can reuse it."""
+        import torch
+        T = q.shape[1] if T is None else T
+        if scratch is None:
+            scratch = torch.empty(run_sequence_host_scratch_size(self.cfg, T), dtype=torch.uint8, device="cuda")
+        _check(lib().fwpkm_run_sequence_host(self.handle, _ptr(q), _ptr(v), _ptr(g), T, n_iter, _ptr(o),
+                                             _ptr(scratch), scratch.numel(), _stream(stream)), "run_sequence_host")
+        return scratch
 
     def stream_tokens(self, q, v, g, o, n_tok=None, seq_stride=None, stream=None):
         """Read n_tok new tokens of every memory ([M][seq_stride][..] rows); writes o for them."""
