@@ -130,18 +130,22 @@ __device__ __forceinline__ const VT* target_src(const Dims& dm, const VT* v, con
 // Gather: two warps per (memory, token), GATHER_TOK tokens per CTA.  Warp half h reads the
 // rows of ranks [16h, 16h + 16) with 16-byte loads, all in flight at once, and sums them in
 // rank order; warp half 0 adds half 1's sum (a fixed order), then forms o and the residual.
+// With at most 16 rows per token half 1 would read nothing, so one warp takes the token
+// (split = false: VAL_WARPS tokens per CTA); the sum is the same, since half 0 would only
+// have added half 1's +0.
 // The token's own value row and gate are loaded before the rows so that their latency
 // overlaps the gather.
 // ---------------------------------------------------------------------------
 constexpr int GATHER_TOK = VAL_WARPS / 2;
+__host__ __device__ __forceinline__ bool gather_split(const Dims& dm) { return dm.k * (dm.H > 1 ? dm.H : 1) > 16; }
 // HEADS: the memories of a sequence share its value table (dm.H > 1, up to 64 rows per
 // token); false compiles the one-head kernel (k <= 32 rows, one entry per lane).
 //
-// gather_token is one token's read by its two warps (`half` 0 and 1): every thread of the
-// CTA calls it, inactive tokens too, since it holds a CTA barrier.  s_tok is the token's
-// slot of the CTA's partial-sum array.  m is the value table (sequence); its heads are
-// memories m H .. m H + H - 1.
-template <typename VT, int VPL, bool HEADS, bool COHERENT>
+// gather_token is one token's read by its two warps (`half` 0 and 1; with split false by one
+// warp, half 0): every thread of the CTA calls it, inactive tokens too, since it holds a CTA
+// barrier when split.  s_tok is the token's slot of the CTA's partial-sum array.  m is the
+// value table (sequence); its heads are memories m H .. m H + H - 1.
+template <typename VT, int VPL, bool HEADS, bool COHERENT, bool SPLIT>
 __device__ __forceinline__ void gather_token(const Dims& dm, const Work& w, const float* __restrict__ V,
                                              const VT* __restrict__ v, const float* __restrict__ g,
                                              long long stride, int wt0, int len, float* __restrict__ o,
@@ -206,16 +210,20 @@ __device__ __forceinline__ void gather_token(const Dims& dm, const Work& w, cons
       }
     }
   }
-  if (half == 1) {
+  if (SPLIT) {
+    if (half == 1) {
 #pragma unroll
-    for (int c = 0; c < VPL; ++c) s_tok[c][lane] = acc[c];
-  }
-  __syncthreads();
-  if (half == 1 || !active) return;
+      for (int c = 0; c < VPL; ++c) s_tok[c][lane] = acc[c];
+    }
+    __syncthreads();
+    if (half == 1 || !active) return;
 #pragma unroll
-  for (int c = 0; c < VPL; ++c) {
-    const float4 b = s_tok[c][lane];
-    acc[c].x += b.x; acc[c].y += b.y; acc[c].z += b.z; acc[c].w += b.w;
+    for (int c = 0; c < VPL; ++c) {
+      const float4 b = s_tok[c][lane];
+      acc[c].x += b.x; acc[c].y += b.y; acc[c].z += b.z; acc[c].w += b.w;
+    }
+  } else if (!active) {
+    return;
   }
   float4* orow = reinterpret_cast<float4*>(o + ((long long)m * stride + i) * dm.dv);
 #pragma unroll
@@ -250,7 +258,7 @@ __device__ __forceinline__ void gather_token(const Dims& dm, const Work& w, cons
   }
 }
 
-template <typename VT, int VPL, bool HEADS>
+template <typename VT, int VPL, bool HEADS, bool SPLIT>
 __global__ void __launch_bounds__(VAL_WARPS * 32, 4)
 gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict__ v,
               const float* __restrict__ g, long long stride, int wt0, int len, float* __restrict__ o,
@@ -259,10 +267,10 @@ gather_kernel(Dims dm, Work w, const float* __restrict__ V, const VT* __restrict
   pdl_trigger();
   __shared__ float4 s_part[GATHER_TOK][VPL][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tl = warp >> 1;
-  const int i = blockIdx.x * GATHER_TOK + tl;
-  gather_token<VT, VPL, HEADS, false>(dm, w, V, v, g, stride, wt0, len, o, fuse_resid, v_next, blockIdx.y, i,
-                                      i < len, warp & 1, lane, s_part[tl]);
+  const int tl = SPLIT ? warp >> 1 : warp;
+  const int i = blockIdx.x * (SPLIT ? GATHER_TOK : VAL_WARPS) + tl;
+  gather_token<VT, VPL, HEADS, false, SPLIT>(dm, w, V, v, g, stride, wt0, len, o, fuse_resid, v_next, blockIdx.y, i,
+                                             i < len, SPLIT ? warp & 1 : 0, lane, s_part[SPLIT ? tl : 0]);
 }
 
 // Streaming path: resid holds vhat from the forward call; turn it into r_t in place.
@@ -629,14 +637,15 @@ struct VlOcc {  // CTAs per SM the loop is compiled for (the write holds up to ~
   static constexpr int value = VPL <= 4 ? 2 : 1;
 };
 
-template <typename VT, int VPL, int WB, bool HEADS>
+template <typename VT, int VPL, int WB, bool HEADS, bool SPLIT>
 __global__ void __launch_bounds__(VAL_WARPS * 32, VlOcc<VPL>::value)
 value_loop_kernel(Dims dm, Work w, float* __restrict__ V, const VT* __restrict__ v, const float* __restrict__ g,
                   int T, int c0, int c1, float* __restrict__ o, int warps_per_mem, int stall) {
   __shared__ float4 s_part[GATHER_TOK][VPL][32];
   __shared__ int s_abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tl = warp >> 1, half = warp & 1;
+  const int tpc = SPLIT ? GATHER_TOK : VAL_WARPS;  // tokens per CTA per iteration
+  const int tl = SPLIT ? warp >> 1 : warp, half = SPLIT ? warp & 1 : 0;
   if (threadIdx.x == 0) s_abort = 0;
   unsigned* arrivals = w.vl_cnt;
   unsigned* exits = w.vl_cnt + 1;
@@ -653,13 +662,13 @@ value_loop_kernel(Dims dm, Work w, float* __restrict__ V, const VT* __restrict__
       if (!grid_arrive_wait(arrivals, target, w, &s_abort)) return;
     }
     const int ntok = dm.B * len;
-    for (int base = blockIdx.x * GATHER_TOK; base < ntok; base += G * GATHER_TOK) {
+    for (int base = blockIdx.x * tpc; base < ntok; base += G * tpc) {
       const int j = base + tl;
       const bool active = j < ntok;
       const int m = active ? j / len : 0, i = active ? j - m * len : 0;
-      gather_token<VT, VPL, HEADS, true>(dm, w, V, vc, g + t0, T, t0, len, o + (long long)t0 * dv, 1, vn, m, i,
-                                        active, half, lane, s_part[tl]);
-      __syncthreads();  // s_part is refilled by the next token
+      gather_token<VT, VPL, HEADS, true, SPLIT>(dm, w, V, vc, g + t0, T, t0, len, o + (long long)t0 * dv, 1, vn, m,
+                                                i, active, half, lane, s_part[SPLIT ? tl : 0]);
+      if (SPLIT) __syncthreads();  // s_part is refilled by the next token
     }
     target += G;
     if (!grid_arrive_wait(arrivals, target, w, &s_abort)) return;  // every residual of chunk c is stored
@@ -699,18 +708,22 @@ int launch_gather(const Dims& d, const Work& w, const float* V, const void* v, c
                   long long stride, int wt0, int len, float* o, bool fuse_resid, const void* v_next,
                   cudaStream_t s) {
   if (len <= 0) return 0;
-  dim3 grid((len + GATHER_TOK - 1) / GATHER_TOK, d.B);
+  const bool split = gather_split(d);
+  const int tpc = split ? GATHER_TOK : VAL_WARPS;
+  dim3 grid((len + tpc - 1) / tpc, d.B);
   const bool heads = d.H > 1;
+#define FWPKM_GATHER_GO(VTT)                                                                                    \
+  FWPKM_VPL_DISPATCH(vpl_of(d.dv),                                                                              \
+      launch_k(heads ? (split ? gather_kernel<VTT, VPL, true, true> : gather_kernel<VTT, VPL, true, false>)     \
+                     : (split ? gather_kernel<VTT, VPL, false, true> : gather_kernel<VTT, VPL, false, false>),  \
+               grid, VAL_WARPS * 32, 0, s, d, w, V, (const VTT*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0, \
+               (const VTT*)v_next))
   if (d.qv_bf16) {
-    FWPKM_VPL_DISPATCH(vpl_of(d.dv),
-        launch_k(heads ? gather_kernel<__nv_bfloat16, VPL, true> : gather_kernel<__nv_bfloat16, VPL, false>, grid,
-                 VAL_WARPS * 32, 0, s, d, w, V, (const __nv_bfloat16*)v, g, stride, wt0, len, o,
-                 fuse_resid ? 1 : 0, (const __nv_bfloat16*)v_next));
+    FWPKM_GATHER_GO(__nv_bfloat16);
   } else {
-    FWPKM_VPL_DISPATCH(vpl_of(d.dv),
-        launch_k(heads ? gather_kernel<float, VPL, true> : gather_kernel<float, VPL, false>, grid, VAL_WARPS * 32, 0,
-                 s, d, w, V, (const float*)v, g, stride, wt0, len, o, fuse_resid ? 1 : 0, (const float*)v_next));
+    FWPKM_GATHER_GO(float);
   }
+#undef FWPKM_GATHER_GO
   return 1;
 }
 
@@ -888,7 +901,8 @@ int launch_value_loop(const Dims& d, const Work& w, float* V, const void* v, con
     int per_mem = (d.C * d.k * d.H + loop_min_positions() - 1) / loop_min_positions();
     if ((long long)per_mem * d.B > (long long)resident * VAL_WARPS) per_mem = resident * VAL_WARPS / d.B;
     if (per_mem < 1) per_mem = 1;
-    const int gather_ctas = (d.B * d.C + GATHER_TOK - 1) / GATHER_TOK;
+    const int tpc = gather_split(d) ? GATHER_TOK : VAL_WARPS;
+    const int gather_ctas = (d.B * d.C + tpc - 1) / tpc;
     const int write_ctas = (d.B * per_mem + VAL_WARPS - 1) / VAL_WARPS;
     int grid = gather_ctas > write_ctas ? gather_ctas : write_ctas;
     if (grid > resident) grid = resident;
@@ -896,8 +910,12 @@ int launch_value_loop(const Dims& d, const Work& w, float* V, const void* v, con
                                       (const VT*)v, g, T, c0, c1, o, per_mem, stall);
     return e == cudaSuccess ? 1 : -1;
   };
-#define FWPKM_VLOOP_GO(VTT, VPLV, WBV)                                                     \
-  (d.H > 1 ? go(value_loop_kernel<VTT, VPLV, WBV, true>, VTT()) : go(value_loop_kernel<VTT, VPLV, WBV, false>, VTT()))
+  const bool split = gather_split(d);
+#define FWPKM_VLOOP_GO(VTT, VPLV, WBV)                                                                   \
+  (d.H > 1 ? (split ? go(value_loop_kernel<VTT, VPLV, WBV, true, true>, VTT())                           \
+                    : go(value_loop_kernel<VTT, VPLV, WBV, true, false>, VTT()))                         \
+           : (split ? go(value_loop_kernel<VTT, VPLV, WBV, false, true>, VTT())                          \
+                    : go(value_loop_kernel<VTT, VPLV, WBV, false, false>, VTT())))
   const int vpl = vpl_of(d.dv);
   int r;
   if (d.qv_bf16) {
