@@ -894,6 +894,16 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
       const char* e = getenv("FWPKM_SEL_FIRST");
       return !(e && e[0] == '0');
     }();
+    // FWPKM_SEL_ON_SK=1 (with selection first and the one-launch addressing step) runs the
+    // selection on the addressing stream itself, so that addressing(c) -> selection(c) ->
+    // addressing(c+1) is stream order.  Measured slower (1.486 against 1.44 ms per step at
+    // the paper scale: the selection then meets the next chunk's gather), so off.
+    static const bool sel_on_k = [] {
+      const char* e = getenv("FWPKM_SEL_ON_SK");
+      return e && e[0] == '1';
+    }();
+    const bool selk = sel_first && sel_on_k && fused;
+    cudaStream_t sSel = selk ? sK : sS;
     cudaEvent_t last_topk = nullptr;
     int cnt = 0;
     for (int pass = 0; pass < n_iter; ++pass) {
@@ -926,11 +936,12 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
           cudaStreamWaitEvent(sS, mark(sK), 0);
           run(st, KK_ADDR, sK, [&] { return launch_address(d, wb, K1, K2, qc, T, len, sK); });
         }
-        if (val_done[c]) cudaStreamWaitEvent(sS, val_done[c], 0);     // previous pass wrote chunk c
+        if (val_done[c]) cudaStreamWaitEvent(sSel, val_done[c], 0);   // previous pass wrote chunk c
         if (tc) {
-          run(st, KK_TOPK, sS, [&] { return launch_select(d, wb, t0, len, nullptr, nullptr, sS); });
-          topk_done[cnt & 1] = mark(sS);
-          last_topk = topk_done[cnt & 1];
+          run(st, KK_TOPK, sSel, [&] { return launch_select(d, wb, t0, len, nullptr, nullptr, sSel); });
+          topk_done[cnt & 1] = mark(sSel);
+          last_topk = selk ? nullptr : topk_done[cnt & 1];  // on sK the order is the stream's
+          if (selk) cudaStreamWaitEvent(sS, topk_done[cnt & 1], 0);
         } else {
           run(st, KK_CART, sS, [&] { return launch_cartesian(d, wb, t0, len, nullptr, nullptr, sS); });
         }
