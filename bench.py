@@ -128,7 +128,7 @@ def _oracle_inputs(w, seqs, T):
     return qf, vf, g.astype(np.float64), K1, K2, V, None
 
 
-def oracle_sample(w, n_chunks, seqs=None):
+def oracle_sample(w, n_chunks, seqs=None, threads=None):
     """CPU-baseline leg: time the oracle (as it stands) on sequences 0..seqs-1 (every head),
     first n_chunks chunks, on all host threads (memories in parallel; with more threads
     than memories each chunk's read phase is split over token ranges).
@@ -147,7 +147,7 @@ def oracle_sample(w, n_chunks, seqs=None):
     k1, k2, vv = K1.copy(), K2.copy(), V.copy()
     cfg = oracle.make_cfg(w.n, w.d, w.d_v, w.k, w.C, key_update=w.key_update)
     t0 = time.perf_counter()
-    res, used = oracle.run_sequence_multi(cfg, qf, vf, gf, k1, k2, vv, 1, nthreads=cores)
+    res, used = oracle.run_sequence_multi(cfg, qf, vf, gf, k1, k2, vv, 1, nthreads=threads or cores)
     if Wo is not None:
         from oracle import layer as orc_layer
         for b in range(seqs):
@@ -667,12 +667,16 @@ def measure(args, w, rank, world, local_rank, n_iter, steps, warmup, full):
     # (full) the oracle timed on a bounded sample of the same workload
     if chk is not None:
         line["selection_check"] = selection_check(w, *chk)
-        if full:
-            n_chunks = 8 if w.name in ("paper", "needle") else 16
-            info = oracle_sample(w, n_chunks, seqs=None if w.name in ("paper", "mid") else 1)
-            line["cpu_baseline"] = {"value": info["tokens"] / info["seconds"], "unit": "tokens/s",
-                                    "cores": info["threads"], "kind": "oracle", "sample": info["sample"],
-                                    "host_threads": info["host_threads"], "cpu_model": info["cpu_model"]}
+        # the headline workload's sample is ~10-30 s of CPU work; the other workloads' are
+        # kept to a few seconds each (fewer chunks)
+        n_chunks = (8 if w.name in ("paper", "needle") else 16) if full else (2 if w.name == "needle" else 4)
+        info = oracle_sample(w, n_chunks, seqs=None if w.name in ("paper", "mid", "tiny") else 1)
+        line["cpu_baseline"] = {"value": info["tokens"] / info["seconds"], "unit": "tokens/s",
+                                "cores": info["threads"], "kind": "oracle", "sample": info["sample"],
+                                "host_threads": info["host_threads"], "cpu_model": info["cpu_model"]}
+        if w.name == "tiny":  # and one thread, for the single-memory workload
+            one = oracle_sample(w, n_chunks, threads=1)
+            line["cpu_baseline"]["one_thread"] = {"value": one["tokens"] / one["seconds"], "threads": one["threads"]}
     return line
 
 
@@ -693,7 +697,8 @@ def run_ours(args, w, rank, world, local_rank):
                 sub = measure(args, wc, rank, world, local_rank, n_iter, max(1, args.config_steps),
                               max(3, args.warmup), full=False)
                 keep = ("ms_per_step", "value", "unit", "steps", "warmup", "config", "roofline", "step_roofline",
-                        "kernels_one_step", "clocks", "gpu_launches", "selection_check", "needle_readback")
+                        "kernels_one_step", "clocks", "gpu_launches", "selection_check", "needle_readback",
+                        "cpu_baseline")
                 configs[key] = {k_: sub[k_] for k_ in keep if k_ in sub}
             except Exception as e:  # one workload failing must not hide the others
                 configs[key] = {"error": f"{type(e).__name__}: {e}"}
