@@ -218,9 +218,9 @@ int launch_cartesian(const Dims& d, const Work& w, int wt0, int len, int32_t* id
 // falls in exactly one bucket), laid out bucket after bucket, and ordered inside each
 // bucket by their full key.
 //
-// SORT_SPLIT CTAs share one (memory, chunk): each counts all buckets (so all agree on
-// the bucket offsets), keeps the keys of its own share of the buckets in shared
-// memory, and one warp per bucket ranks each key by comparing it with every other key
+// `split` CTAs (a power of two, at most SORT_SPLIT) share one (memory, chunk): each counts
+// all buckets (so all agree on the bucket offsets), keeps the keys of its own share of the
+// buckets in shared memory, and one warp per bucket ranks each key by comparing it with every other key
 // of the bucket and stores it at its rank.  The scatter into buckets may land keys in
 // any order; ranking by the full unique key makes the output independent of it.  A
 // bucket of more than 128 keys (strongly skewed slot use: a row read by many tokens) is
@@ -235,13 +235,13 @@ constexpr int SORT_BUCKET_CAP = 128;   // largest bucket the ranking path handle
 // one-head kernel, whose pair i is offset i of the chunk's [C][k] slot block.
 template <int VPT, bool HEADS>
 __global__ void __launch_bounds__(SORT_THREADS)
-sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) {
+sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target, int split) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ u64 s_keys[];
   __shared__ int s_cnt[512], s_off[513], s_cur[512];
   const int m = blockIdx.y;  // the value table (sequence); its heads are memories m H .. m H + H - 1
-  const int cc = blockIdx.x / SORT_SPLIT, part = blockIdx.x % SORT_SPLIT;
+  const int cc = blockIdx.x / split, part = blockIdx.x % split;
   const int C = dm.C, k = dm.k, H = HEADS ? dm.H : 1, kh = k * H;
   const int tc0 = cc * C;  // relative to wt0
   const int clen = min(C, total_len - tc0);
@@ -252,7 +252,7 @@ sort_pairs_kernel(Dims dm, Work w, int wt0, int total_len, int last_has_target) 
   while (Ppad < P) Ppad <<= 1;
   const int NB = Ppad / SORT_BUCKET_KEYS;  // a power of two, <= 512
   const int nb_log2 = 31 - __clz(NB);
-  const int b_lo = part * NB / SORT_SPLIT, b_hi = (part + 1) * NB / SORT_SPLIT;
+  const int b_lo = part * NB / split, b_hi = (part + 1) * NB / split;
   const int cslot = (wt0 + tc0) / C;
   const size_t cbase = (size_t)m * w.max_chunks + cslot;
   u64* out = w.sk + cbase * (size_t)(C * kh);
@@ -379,13 +379,33 @@ int launch_sort_pairs(const Dims& d, const Work& w, int wt0, int total_len, bool
   if (total_len <= 0) return 0;
   const int nchunks = (total_len + d.C - 1) / d.C;
   const int P = d.C * d.k * d.H;
-  dim3 grid(nchunks * SORT_SPLIT, d.B);
+  // CTAs per (table, chunk): about one wave of 1024-thread CTAs for the whole launch (each
+  // CTA counts all of its chunk's keys, so more CTAs than SMs only repeat that work);
+  // FWPKM_SORT_SPLIT overrides it
+  static const int forced = [] {
+    const char* e = getenv("FWPKM_SORT_SPLIT");
+    return e ? atoi(e) : 0;
+  }();
+  static const int sms = [] {
+    int dev = 0, v = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    return v;
+  }();
+  int split = 1;
+  const long long units = (long long)nchunks * d.B;
+  while (split < SORT_SPLIT && units * split * 2 <= sms) split <<= 1;
+  if (forced > 0) {
+    split = 1;
+    while (split < SORT_SPLIT && split * 2 <= forced) split <<= 1;
+  }
+  dim3 grid(nchunks * split, d.B);
   auto go = [&](auto kern, int vpt) {
     int Ppad = 32 * vpt;
     while (Ppad < P) Ppad <<= 1;
     const size_t smem = sizeof(u64) * (size_t)Ppad;
     if (!raise_smem_limit((const void*)kern, smem)) return -1;
-    launch_k(kern, grid, SORT_THREADS, smem, s, d, w, wt0, total_len, last_has_target ? 1 : 0);
+    launch_k(kern, grid, SORT_THREADS, smem, s, d, w, wt0, total_len, last_has_target ? 1 : 0, split);
     return 1;
   };
   int rc;
