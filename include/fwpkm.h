@@ -162,10 +162,9 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
  * q, v, g, o are HOST buffers in the fwpkm_run_sequence layout (seq_stride = T), and
  * must be page-locked (cudaHostAlloc, or cudaHostRegister'd): anything else returns
  * FWPKM_ERR_INVALID_ARG.  The call copies chunk c's inputs to device scratch while
- * earlier chunks compute (cudaMemcpy2DAsync on an internal stream; the tensor-core path
- * also makes chunk c's query norms there), starts each chunk's kernels when its inputs
- * (and the lookahead row after it) have landed, and copies each chunk's final-pass o back
- * as soon as it is written, so the copies overlap the compute.  Everything is enqueued on
+ * earlier chunks compute (cudaMemcpy2DAsync on an internal stream), starts each chunk's
+ * kernels when its inputs (and the lookahead row after it) have landed, and copies each
+ * chunk's final-pass o back as soon as it is written, so the copies overlap the compute.  Everything is enqueued on
  * `stream` (captured once into the state's cached graph, like fwpkm_run_sequence); the
  * host buffers must stay valid, and o unread, until the stream passes the call.
  *   scratch  device, 256-byte aligned, >= fwpkm_run_sequence_host_scratch_size(cfg, T)

@@ -776,12 +776,21 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
   dep(origin, sV);
 
   // Host buffers: chunk c's inputs are copied to the device on sH, in chunk order (copies
-  // only, so they run ahead of the compute); on the tensor-core path sP then makes the
-  // chunk's query norms and feature-major half-queries.  in_ready[c] marks both; each
-  // consumer waits only for the chunks it reads.  o goes back on sD as soon as the last
-  // pass's value work of a chunk (or window) has ended.
+  // only, so they run ahead of the compute), and in_ready[c] marks them; each consumer
+  // waits only for the chunks it reads.  On the tensor-core path the chunk's query norms and
+  // feature-major half-queries are made from the copy (see host_prep).  o goes back on sD
+  // as soon as the last pass's value work of a chunk (or window) has ended.
   std::vector<cudaEvent_t> in_ready;
   cudaStream_t sH = nullptr, sP = nullptr, sD = nullptr;
+  // where the query preparation of host-buffer calls runs (FWPKM_HOST_PREP): 'k' (default)
+  // per chunk on the addressing stream just before the chunk's addressing; 'p' per chunk on
+  // its own stream as soon as the chunk's copies land (its small kernels then take SMs the
+  // one-launch addressing kernel waits for: 1.93 against 1.58 ms per paper-scale call);
+  // 'w' once for the whole call after the last copy (2.25 ms)
+  static const char host_prep = [] {
+    const char* e = getenv("FWPKM_HOST_PREP");
+    return (e && (e[0] == 'p' || e[0] == 'w')) ? e[0] : 'k';
+  }();
   if (hio) {
     sH = st->serial ? sK : st->sH[gi];
     sP = st->serial ? sK : st->sP[gi];
@@ -803,7 +812,7 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
           (size_t)len * d.dv * es, d.B);
       h2d(g + t0, hio->g + t0, (size_t)T * 4, (size_t)len * 4, d.B);
       in_ready[c] = mark(sH);
-      if (tc) {
+      if (tc && host_prep == 'p') {
         cudaStreamWaitEvent(sP, in_ready[c], 0);
         const void* qc = offs(q, (long long)t0 * d.d, es);
         run(st, KK_PREP, sP, [&] { return launch_qnorm(d, wk, qc, T, t0, len, sP); });
@@ -811,7 +820,21 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
         in_ready[c] = mark(sP);
       }
     }
+    if (tc && host_prep == 'w') {  // one preparation over the whole call once every copy has landed
+      cudaStreamWaitEvent(sP, in_ready[nch - 1], 0);
+      run(st, KK_PREP, sP, [&] { return launch_qnorm(d, wk, q, T, 0, T, sP); });
+      if (qt_whole) run(st, KK_PREP, sP, [&] { return launch_qtrans(d, wk, q, T, 0, T, sP); });
+      const cudaEvent_t e = mark(sP);
+      for (int c = 0; c < nch; ++c) in_ready[c] = e;
+    }
   }
+  // the query preparation of tokens [t0, t0 + len) on stream s (host buffers, 'k' mode)
+  auto prep_on = [&](cudaStream_t s, int t0, int len) {
+    if (!(hio && tc && host_prep == 'k')) return;
+    const void* qc = offs(q, (long long)t0 * d.d, es);
+    run(st, KK_PREP, s, [&] { return launch_qnorm(d, wk, qc, T, t0, len, s); });
+    if (qt_whole) run(st, KK_PREP, s, [&] { return launch_qtrans(d, wk, qc, T, t0, len, s); });
+  };
   auto wait_in = [&](cudaStream_t s, int c) {  // inputs of chunks <= c are on the device
     if (hio) cudaStreamWaitEvent(s, in_ready[c < nch ? c : nch - 1], 0);
   };
@@ -856,6 +879,7 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
     for (int w0 = 0; w0 < T; w0 += wtok) {
       const int wl = T - w0 < wtok ? T - w0 : wtok;
       wait_in(sK, (w0 + wl - 1) / C);
+      prep_on(sK, w0, wl);
       if (tc) {
         run(st, KK_SCORE, sK, [&] { return launch_tc_score(d, wk, q, T, T, w0, w0, wl, false, sK); });
         run(st, KK_TOPK, sK, [&] { return launch_select(d, wk, w0, wl, nullptr, nullptr, sK); });
@@ -915,7 +939,10 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
         if (sel_done[c]) cudaStreamWaitEvent(sK, sel_done[c], 0);    // previous pass read A/Dsv
         if (topk_done[cnt & 1]) cudaStreamWaitEvent(sK, topk_done[cnt & 1], 0);  // buffer reuse
         if (sel_first && last_topk) cudaStreamWaitEvent(sK, last_topk, 0);
-        if (pass == 0) wait_in(sK, c);
+        if (pass == 0) {
+          wait_in(sK, c);
+          prep_on(sK, t0, len);
+        }
         if (fused) {
           // the chunk's whole addressing step in one launch; the selection needs its rows
           run(st, KK_FUSED, sK, [&] {
