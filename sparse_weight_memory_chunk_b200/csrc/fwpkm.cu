@@ -848,13 +848,15 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
       st->host_error = 1;
   };
 
-  auto value_chunk = [&](int c) {
+  // before_write: an event the write (not the gather) waits for (the pair sort), or null
+  auto value_chunk = [&](int c, cudaEvent_t before_write = nullptr) {
     const int t0 = c * C, len = T - t0 < C ? T - t0 : C;
     const void* vc = offs(v, (long long)t0 * d.dv, es);
     const void* vn = (t0 + len < T) ? offs(v, (long long)(t0 + len) * d.dv, es) : nullptr;
     run(st, KK_GATHER, sV, [&] {
       return launch_gather(d, wk, V, vc, g + t0, T, t0, len, o + (long long)t0 * d.dv, true, vn, sV);
     });
+    if (before_write) cudaStreamWaitEvent(sV, before_write, 0);
     run(st, KK_WRITE, sV, [&] { return launch_write(d, wk, V, t0, sV); });
   };
 
@@ -974,13 +976,18 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
         }
         run(st, KK_SORT, sS, [&] { return launch_sort_pairs(d, wb, t0, len, !la || (t0 + len < T), sS); });
         sel_done[c] = mark(sS);
-        // the values chain starts a chunk only once its whole selection (slots, weights and
-        // the pair sort) is done: starting the gather right after the slots were chosen
-        // made it overlap the scoring and key-step GEMMs, which slowed them (1.82 against
-        // 1.62 ms per step)
-        cudaStreamWaitEvent(sV, sel_done[c], 0);
+        // The gather of a chunk needs its slots and weights (the selection); only its write
+        // needs the pair sort, which then runs beside the gather (paper scale: 1.45 against
+        // 1.48 ms per step; FWPKM_GATHER_EARLY=0 waits for the sort, which with the
+        // four-kernel addressing chain had been the faster order, 1.62 against 1.82 ms).
+        static const bool gather_early = [] {
+          const char* e = getenv("FWPKM_GATHER_EARLY");
+          return !(e && e[0] == '0');
+        }();
+        const bool early = gather_early && tc && topk_done[cnt & 1];
+        cudaStreamWaitEvent(sV, early ? topk_done[cnt & 1] : sel_done[c], 0);
         if (pass == 0) wait_in(sV, c + 1);  // v, g of the chunk and its lookahead row
-        value_chunk(c);
+        value_chunk(c, early ? sel_done[c] : nullptr);
         val_done[c] = mark(sV);
         if (pass == n_iter - 1) copy_out(sV, c, c + 1);
       }
