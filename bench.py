@@ -46,7 +46,7 @@ BY_NAME = {w.name: (i, w) for i, w in WORKLOADS.items()}
 TRAFFIC = {
     "fused": {"per_mem": (5_873_920 + 0) / 2},
     "topk": {"per_mem": (4_266_240 + 0) / 2},
-    "sort": {"per_mem": (96_512 + 0) / 2},
+    "sort": {"per_mem": (97_024 + 0) / 2},
     "gather": {"per_mem": (15_792_128 + 0) / 2},
     "write": {"per_mem": (16_094_464 + 0) / 2},
 }
