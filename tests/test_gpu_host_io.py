@@ -68,6 +68,36 @@ def test_host_buffers_match_device_buffers(name, n_iter):
     assert torch.equal(oh2, oh) and torch.equal(dev_b2["V"], dev_a["V"])
 
 
+def test_host_buffers_heads_sharing_v():
+    """Heads sharing one value table: q per memory, v, g, o per sequence, copied through the
+    host-buffer call; bits of fwpkm_run_sequence on the same inputs."""
+    n, d, dv, k, C, B, H, T = 256, 128, 64, 8, 128, 2, 2, 300
+    for ku in (True, False):
+        w = Workload("heads_io", n, d, dv, k, T, C, B * H, 1, "bf16", ku, 9, "sigmoid", "normal002")
+        q, v_all, g_all = gen_qvg(w)
+        v, g = np.ascontiguousarray(v_all[:B]), np.ascontiguousarray(g_all[:B])
+        K1, K2 = gen_keys(w)
+        V = np.stack([gen_values(w, b) for b in range(B)])
+        cfg = fwpkm.make_config(n, d, dv, k, C, B * H, True, key_update=ku, v_heads=H)
+        qd, vd, gd = to_device(q, "bf16", torch), to_device(v, "bf16", torch), torch.from_numpy(g).cuda()
+        outs = []
+        for host in (False, True):
+            K1d, K2d, Vd = (torch.from_numpy(x).cuda() for x in (K1, K2, V))
+            st = fwpkm.State(cfg, K1d, K2d, Vd, T)
+            if host:
+                # the host buffers must outlive the asynchronous copies: keep references
+                qh, vh, gh = qd.cpu().pin_memory(), vd.cpu().pin_memory(), gd.cpu().pin_memory()
+                o = torch.zeros(B, T, dv).pin_memory()
+                st.run_sequence_host(qh, vh, gh, o)
+            else:
+                o = torch.zeros(B, T, dv, device="cuda")
+                st.run_sequence(qd, vd, gd, o)
+            st.sync()
+            torch.cuda.synchronize()
+            outs.append((o.cpu(), Vd.cpu(), K1d.cpu()))
+        assert all(torch.equal(a, b) for a, b in zip(*outs)), f"heads, key update {ku}: host-buffer call differs"
+
+
 def test_host_buffer_argument_checks():
     w, data, cfg = setup("key_update_tc")
     q, v, g = data[:3]

@@ -167,6 +167,21 @@ def test_flag_variants(flags):
     streaming_vs_oracle("tiny_key_ragged", **flags)
 
 
+@pytest.mark.parametrize("flags", [dict(lookahead=False), dict(target_norm=False), dict(gate_weight=False)])
+def test_flag_variants_frozen_keys(flags):
+    """The flag variants with frozen keys on the tensor-core shapes: chunk by chunk against
+    the oracle, then fwpkm_run_sequence (addressing windows and the persistent value loop)
+    bit-for-bit against those calls."""
+    res = streaming_vs_oracle("mid", **flags)
+    w, data, gcfg = res["w"], res["data"], res["gcfg"]
+    st, dev = device_state(w, data, gcfg, w.T)
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    st.run_sequence(dev["q"], dev["v"], dev["g"], o)
+    st.sync()
+    assert torch.equal(o.cpu(), res["o"]), f"{flags}: run_sequence o differs from chunk-by-chunk"
+    assert torch.equal(dev["V"].cpu(), res["V"].cpu()), f"{flags}: run_sequence V differs"
+
+
 @pytest.mark.parametrize("name", ["mid", "mid_key"])
 def test_passes_compose_and_determinism(name):
     w, data, gcfg, _ = make_case(name)
