@@ -224,6 +224,62 @@ def test_needle_stream_two_passes():
     assert torch.equal(dev["V"], res["V"]), "run_sequence(n_iter=2) V differs from chunk-by-chunk"
 
 
+def test_needle_workload_full_size_sampled():
+    """The needle workload at its full size and seed (N = 2^20 slots, T = 131,072, C = 512,
+    frozen keys, 64 planted needles): fwpkm_run_sequence, in the launch configuration the
+    benchmark times (addressing windows and the persistent value loop), bit-for-bit against
+    the chunk-by-chunk calls over all 256 chunks; every 16th of those chunks, and the last,
+    against the oracle from the GPU's own pre-chunk state (o, weights and every value row the
+    chunk writes)."""
+    from sparse_weight_memory_chunk_b200.inputs import WORKLOADS, gen_needles
+    w = WORKLOADS[4]
+    _, data, gcfg, ocfg = workload_case(w)
+    q, v, g, K1, K2, V = data
+    gen_needles(w, q, v)
+    M, T, C, k, dv = w.M, w.T, w.C, w.k, w.d_v
+    st, dev = device_state(w, (q, v, g, K1, K2, V), gcfg, C)
+    o_d = torch.zeros(M, T, dv, device="cuda")
+    qf, vf = as_f64(q, w.qv), as_f64(v, w.qv)
+    nch = (T + C - 1) // C
+    sampled = set(range(0, nch, 16)) | {nch - 1}
+    ties = 0
+    for ci in range(nch):
+        t0 = ci * C
+        ln = min(C, T - t0)
+        check = ci in sampled
+        if check:
+            st.sync()
+            Vpre = dev["V"][0].cpu().numpy().copy()
+            idx_d = torch.empty(M, ln, k, dtype=torch.int32, device="cuda")
+            w_d = torch.empty(M, ln, k, device="cuda")
+        st.forward_chunk(dev["q"][:, t0:], dev["v"][:, t0:], dev["g"][:, t0:], o_d[:, t0:], ln, seq_stride=T,
+                         idx_out=idx_d if check else None, w_out=w_d if check else None)
+        has_next = t0 + ln < T
+        st.write_chunk(dev["v"][:, t0 + ln] if has_next else None)
+        if check:
+            st.sync()
+            idx_g = idx_d.cpu().numpy()[0]
+            vn = vf[0, t0 + ln] if has_next else None
+            Vo = Vpre  # the oracle updates it in place
+            o_o, I_o, w_o, nt = oracle_chunk_against_gpu(ocfg, qf[0, t0:t0 + ln], vf[0, t0:t0 + ln],
+                                                         g[0, t0:t0 + ln].astype(np.float64), vn, K1[0].copy(),
+                                                         K2[0].copy(), Vo, idx_g)
+            ties += nt
+            assert_close(o_d[0, t0:t0 + ln].cpu().numpy(), o_o, f"needle chunk {ci}: o")
+            assert_close(w_d.cpu().numpy()[0], w_o, f"needle chunk {ci}: w", atol=1e-6)
+            rows = np.unique(idx_g.reshape(-1))
+            Vg = dev["V"][0][torch.from_numpy(rows).cuda()].cpu().numpy()
+            assert_close(Vg, Vo[rows], f"needle chunk {ci}: written V rows")
+    st.sync()
+    print(f"needle full size: {len(sampled)} chunks against the oracle, near-ties {ties}")
+    st2, dev2 = device_state(w, (q, v, g, K1, K2, V), gcfg, T)
+    o2 = torch.zeros(M, T, dv, device="cuda")
+    st2.run_sequence(dev2["q"], dev2["v"], dev2["g"], o2)
+    st2.sync()
+    assert torch.equal(o2, o_d), "needle full size: run_sequence o differs from chunk-by-chunk"
+    assert torch.equal(dev2["V"], dev["V"]), "needle full size: run_sequence V differs from chunk-by-chunk"
+
+
 def test_edge_cases():
     w, data, gcfg, ocfg = make_case("tiny_key_ragged")
     st, dev = device_state(w, data, gcfg, w.T)
