@@ -119,6 +119,58 @@ def test_run_layer_matches_oracle_chain(variant):
         assert max_nread >= C // 2, "no row was read by half a chunk's tokens"
 
 
+def test_run_layer_full_size():
+    """The layer workload at its full size and seed (B = 16 sequences, T = 4096, d_model =
+    2048, n = 512, 64 Zipf-weighted clusters), through fwpkm_run_layer as the benchmark
+    times it: q, v, g on 512 sampled rows against the oracle's projections, the memory chunk
+    by chunk against the oracle on the call's own q, v, g, the call's o and final state bit
+    for bit against that run, and o' on the sampled rows against the oracle's output
+    projection of the call's o."""
+    w5 = WORKLOADS[5]
+    B, T = w5.B, w5.T
+    L = gen_layer(w5, B=B, T=T)
+    K1, K2 = gen_keys(w5, M=B)
+    V = np.stack([gen_values(w5, m) for m in range(B)])
+    D, d, dv, C, k = w5.d_model, w5.d, w5.d_v, w5.C, w5.k
+    gcfg = fwpkm.make_config(w5.n, d, dv, k, C, B, True, key_update=True)
+    ocfg = oracle.make_cfg(w5.n, d, dv, k, C, key_update=True)
+    lay = fwpkm.Layer(D, d, dv, B * T, qv_bf16=True)
+    Wd = {name: bf16_dev(L[name]) for name in ("Wq", "Wv", "wg", "Wo")}
+    lay.set_params(Wd["Wq"], Wd["Wv"], Wd["wg"], Wd["Wo"])
+    K1d, K2d, Vd = (torch.from_numpy(x).cuda() for x in (K1, K2, V))
+    st = fwpkm.State(gcfg, K1d, K2d, Vd, T)
+    o_out = torch.empty(B, T, D, device="cuda", dtype=torch.bfloat16)
+    scratch = lay.run_layer(st, bf16_dev(L["h"]), o_out)
+    st.sync()
+    lay.sync()
+    q, v, g, o = (x.clone() for x in fwpkm.run_layer_parts(gcfg, T, scratch))
+
+    rows = np.random.default_rng(5).choice(B * T, 512, replace=False)
+    ri = torch.from_numpy(rows).cuda()
+    hf = bf16_to_f32(L["h"].reshape(B * T, D)[rows])
+    ones = np.ones(D)
+    Wq, Wv, wg, Wo = (bf16_to_f32(L[name]) for name in ("Wq", "Wv", "wg", "Wo"))
+    qo, vo, go = orc.project_in(hf, ones, Wq, None, ones, Wv, None, ones, wg, 0.0)
+    nrm = orc.rmsnorm(hf, ones, 1e-6)
+    assert_within(bf16_host(q.reshape(B * T, d)[ri]), qo, accum_bound(nrm, Wq), BF16_REL, "q")
+    assert_within(bf16_host(v.reshape(B * T, dv)[ri]), vo, accum_bound(nrm, Wv), BF16_REL, "v")
+    assert_within(g.reshape(-1).cpu().numpy()[rows], go, accum_bound(nrm, wg[None, :])[:, 0] * 0.25, RTOL, "g")
+
+    def bits(x):
+        return x.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+    w = Workload("layer_full", w5.n, d, dv, k, T, C, B, 1, "bf16", True, w5.seed, "sigmoid", "normal002")
+    res = compare_streaming("layer_full", w, (bits(q), bits(v), g.cpu().numpy(), K1, K2, V), gcfg, ocfg)
+    print(f"layer full size: near-ties {res['ties']}")
+    assert torch.equal(o.cpu(), res["o"]), "run_layer o differs from the chunk-by-chunk memory"
+    assert torch.equal(Vd, res["V"].cuda() if not res["V"].is_cuda else res["V"]), "run_layer V differs"
+    assert torch.equal(K1d.cpu(), res["K1"]) and torch.equal(K2d.cpu(), res["K2"])
+    of = o.reshape(B * T, dv)[ri].cpu().numpy()
+    want = orc.project_out(of, np.ones(dv), Wo, None)
+    assert_within(bf16_host(o_out.reshape(B * T, D)[ri]), want,
+                  accum_bound(orc.rmsnorm(of, np.ones(dv), 1e-6), Wo), BF16_REL, "o'")
+
+
 def test_run_layer_argument_checks():
     w5 = WORKLOADS[5]
     B, T = 1, 64

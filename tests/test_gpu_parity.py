@@ -162,6 +162,24 @@ def test_paper_workload_full_size():
     assert torch.equal(dev["K1"].cpu(), res["K1"]) and torch.equal(dev["K2"].cpu(), res["K2"])
 
 
+def test_mid_workload_full_size():
+    """The mid workload at its full size and seed (16 memories of 65,536 slots, T = 4096,
+    C = 128, frozen keys): every chunk's outputs, weights and sampled value rows against the
+    oracle, then fwpkm_run_sequence (two addressing windows, the persistent value loop) bit
+    for bit against the chunk-by-chunk run."""
+    from sparse_weight_memory_chunk_b200.inputs import WORKLOADS
+    w = WORKLOADS[2]
+    res = compare_streaming("mid_full", *workload_case(w))
+    print(f"mid full size: near-ties {res['ties']}")
+    data, gcfg = res["data"], res["gcfg"]
+    st, dev = device_state(w, data, gcfg, w.T)
+    o = torch.zeros(w.M, w.T, w.d_v, device="cuda")
+    st.run_sequence(dev["q"], dev["v"], dev["g"], o)
+    st.sync()
+    assert torch.equal(o.cpu(), res["o"]), "run_sequence o differs from chunk-by-chunk"
+    assert torch.equal(dev["V"], res["V"].cuda() if not res["V"].is_cuda else res["V"]), "run_sequence V differs"
+
+
 @pytest.mark.parametrize("flags", [dict(lookahead=False), dict(target_norm=False), dict(gate_weight=False)])
 def test_flag_variants(flags):
     streaming_vs_oracle("tiny_key_ragged", **flags)
