@@ -782,15 +782,18 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
   // as soon as the last pass's value work of a chunk (or window) has ended.
   std::vector<cudaEvent_t> in_ready;
   cudaStream_t sH = nullptr, sP = nullptr, sD = nullptr;
-  // where the query preparation of host-buffer calls runs (FWPKM_HOST_PREP): 'k' (default)
-  // per chunk on the addressing stream just before the chunk's addressing; 'p' per chunk on
-  // its own stream as soon as the chunk's copies land (its small kernels then take SMs the
-  // one-launch addressing kernel waits for: 1.93 against 1.58 ms per paper-scale call);
-  // 'w' once for the whole call after the last copy (2.25 ms)
+  // where the query preparation of host-buffer calls runs (FWPKM_HOST_PREP): 'a' (default)
+  // with the one-launch addressing step: chunk c+1's on its own stream once chunk c's
+  // addressing kernel has finished, so it runs beside chunk c's selection (else as 'k');
+  // 'k' per chunk on the addressing stream just before the chunk's addressing (on the
+  // critical chain: 1.58 ms per paper-scale call); 'p' per chunk on its own stream as soon as
+  // the chunk's copies land (its small kernels then take SMs the addressing kernel waits
+  // for: 1.93 ms); 'w' once for the whole call after the last copy (2.25 ms)
   static const char host_prep = [] {
     const char* e = getenv("FWPKM_HOST_PREP");
-    return (e && (e[0] == 'p' || e[0] == 'w')) ? e[0] : 'k';
+    return (e && (e[0] == 'p' || e[0] == 'w' || e[0] == 'k')) ? e[0] : 'a';
   }();
+  const bool prep_after = hio && tc && host_prep == 'a' && fused;
   if (hio) {
     sH = st->serial ? sK : st->sH[gi];
     sP = st->serial ? sK : st->sP[gi];
@@ -812,6 +815,13 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
           (size_t)len * d.dv * es, d.B);
       h2d(g + t0, hio->g + t0, (size_t)T * 4, (size_t)len * 4, d.B);
       in_ready[c] = mark(sH);
+      if (prep_after && c == 0) {  // the first chunk's preparation follows its copies
+        cudaStreamWaitEvent(sP, in_ready[0], 0);
+        const void* qc = offs(q, 0, es);
+        run(st, KK_PREP, sP, [&] { return launch_qnorm(d, wk, qc, T, 0, len, sP); });
+        if (qt_whole) run(st, KK_PREP, sP, [&] { return launch_qtrans(d, wk, qc, T, 0, len, sP); });
+        in_ready[0] = mark(sP);
+      }
       if (tc && host_prep == 'p') {
         cudaStreamWaitEvent(sP, in_ready[c], 0);
         const void* qc = offs(q, (long long)t0 * d.d, es);
@@ -830,7 +840,7 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
   }
   // the query preparation of tokens [t0, t0 + len) on stream s (host buffers, 'k' mode)
   auto prep_on = [&](cudaStream_t s, int t0, int len) {
-    if (!(hio && tc && host_prep == 'k')) return;
+    if (!(hio && tc && (host_prep == 'k' || (host_prep == 'a' && !prep_after)))) return;
     const void* qc = offs(q, (long long)t0 * d.d, es);
     run(st, KK_PREP, s, [&] { return launch_qnorm(d, wk, qc, T, t0, len, s); });
     if (qt_whole) run(st, KK_PREP, s, [&] { return launch_qtrans(d, wk, qc, T, t0, len, s); });
@@ -950,7 +960,18 @@ static void enqueue_group(fwpkm_state* st, int gi, const Dims& d, const Work& wk
           run(st, KK_FUSED, sK, [&] {
             return launch_addr_fused(d, wb, K1, K2, q, T, T, t0, t0, len, t0, false, sK);
           });
-          cudaStreamWaitEvent(sS, mark(sK), 0);
+          const cudaEvent_t addr_done = mark(sK);
+          cudaStreamWaitEvent(sS, addr_done, 0);
+          if (prep_after && pass == 0 && c + 1 < nch) {
+            // the next chunk's query preparation beside this chunk's selection
+            const int tn = t0 + C, ln = T - tn < C ? T - tn : C;
+            const void* qn = offs(q, (long long)tn * d.d, es);
+            cudaStreamWaitEvent(sP, in_ready[c + 1], 0);
+            cudaStreamWaitEvent(sP, addr_done, 0);
+            run(st, KK_PREP, sP, [&] { return launch_qnorm(d, wk, qn, T, tn, ln, sP); });
+            if (qt_whole) run(st, KK_PREP, sP, [&] { return launch_qtrans(d, wk, qn, T, tn, ln, sP); });
+            in_ready[c + 1] = mark(sP);
+          }
         } else if (tc) {
           run(st, KK_SCORE, sK, [&] { return launch_tc_score(d, wb, q, T, T, t0, t0, len, true, sK); });
           // the selection needs the distance rows; it also waits for the usage marginals, so
