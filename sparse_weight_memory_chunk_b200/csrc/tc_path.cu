@@ -43,39 +43,47 @@ qnorm_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long q_s
   }
 }
 
-// bf16 pieces and squared norm of every key: one thread per (problem, sub-key), features
-// in order (the key-step GEMM epilogue uses the same order, so both give the same bits).
+// bf16 pieces and squared norm of every key: four threads per (problem, sub-key), thread g
+// taking features [32 g, 32 g + 32) in order (adjacent threads read adjacent 128-byte
+// pieces of the row).  The squared norm is the four 32-feature partial sums combined in
+// order, exactly as the key-step epilogues form it, so both give the same bits.
 __global__ void __launch_bounds__(TP_THREADS)
 keyprep_kernel(Dims dm, Work w, const float* __restrict__ K1, const float* __restrict__ K2) {
   pdl_wait();
   pdl_trigger();
   const int P = dm.M * 2;
-  const long long idx = (long long)blockIdx.x * TP_THREADS + threadIdx.x;
-  if (idx >= (long long)P * dm.n) return;
-  const int p = (int)(idx / dm.n), b = (int)(idx - (long long)p * dm.n);
+  const long long gid = (long long)blockIdx.x * TP_THREADS + threadIdx.x;
+  const long long idx = gid >> 2;  // (problem, sub-key)
+  const int g = (int)(gid & 3);
+  const bool row_ok = idx < (long long)P * dm.n;
+  const int p = row_ok ? (int)(idx / dm.n) : 0, b = row_ok ? (int)(idx - (long long)p * dm.n) : 0;
   const int m = p >> 1, j = p & 1, h = dm.h;
-  const float* K = (j == 0 ? K1 : K2) + ((size_t)m * dm.n + b) * h;
-  const size_t pstride = (size_t)w.P_all * dm.n * h;
-  __nv_bfloat16* pc = w.Kpc + ((size_t)p * dm.n + b) * h;
-  // squared norm as four 32-feature partial sums combined in order, exactly as the
-  // key-step GEMM epilogue forms it
-  float part[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int e = 0; e < h; e += 8) {
-    float& ss = part[e >> 5];
-    float4 k0 = *reinterpret_cast<const float4*>(K + e);
-    float4 k1 = *reinterpret_cast<const float4*>(K + e + 4);
-    float kin[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-    __align__(16) __nv_bfloat16 hi[8], mid[8], lo[8];
+  float part = 0.f;
+  if (row_ok && 32 * g < h) {
+    const float* K = (j == 0 ? K1 : K2) + ((size_t)m * dm.n + b) * h + 32 * g;
+    const size_t pstride = (size_t)w.P_all * dm.n * h;
+    __nv_bfloat16* pc = w.Kpc + ((size_t)p * dm.n + b) * h + 32 * g;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      ss += kin[u] * kin[u];
-      split3_bf16(kin[u], hi[u], mid[u], lo[u]);
+    for (int e = 0; e < 32; e += 8) {
+      float4 k0 = *reinterpret_cast<const float4*>(K + e);
+      float4 k1 = *reinterpret_cast<const float4*>(K + e + 4);
+      float kin[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+      __align__(16) __nv_bfloat16 hi[8], mid[8], lo[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        part += kin[u] * kin[u];
+        split3_bf16(kin[u], hi[u], mid[u], lo[u]);
+      }
+      *reinterpret_cast<uint4*>(pc + e) = *reinterpret_cast<uint4*>(hi);
+      *reinterpret_cast<uint4*>(pc + pstride + e) = *reinterpret_cast<uint4*>(mid);
+      *reinterpret_cast<uint4*>(pc + 2 * pstride + e) = *reinterpret_cast<uint4*>(lo);
     }
-    *reinterpret_cast<uint4*>(pc + e) = *reinterpret_cast<uint4*>(hi);
-    *reinterpret_cast<uint4*>(pc + pstride + e) = *reinterpret_cast<uint4*>(mid);
-    *reinterpret_cast<uint4*>(pc + 2 * pstride + e) = *reinterpret_cast<uint4*>(lo);
   }
-  w.kn[(size_t)p * dm.n + b] = ((part[0] + part[1]) + part[2]) + part[3];
+  // the row's four partials sit in lanes 4r .. 4r + 3 of the warp
+  const int lane = threadIdx.x & 31, base = lane & ~3;
+  const float p0 = __shfl_sync(0xffffffffu, part, base), p1 = __shfl_sync(0xffffffffu, part, base + 1);
+  const float p2 = __shfl_sync(0xffffffffu, part, base + 2), p3 = __shfl_sync(0xffffffffu, part, base + 3);
+  if (row_ok && g == 0) w.kn[(size_t)p * dm.n + b] = ((p0 + p1) + p2) + p3;
 }
 
 // Partial column sums sum_t w[t][a] / Z_t over one token slice; also Z_t itself.  The
@@ -274,8 +282,8 @@ int launch_qnorm(const Dims& d, const Work& w, const void* q, long long q_stride
 }
 
 int launch_keyprep(const Dims& d, const Work& w, const float* K1, const float* K2, cudaStream_t s) {
-  const long long rows = (long long)d.M * 2 * d.n;
-  launch_k(keyprep_kernel, (unsigned)((rows + TP_THREADS - 1) / TP_THREADS), TP_THREADS, 0, s, d, w, K1, K2);
+  const long long threads = (long long)d.M * 2 * d.n * 4;
+  launch_k(keyprep_kernel, (unsigned)((threads + TP_THREADS - 1) / TP_THREADS), TP_THREADS, 0, s, d, w, K1, K2);
   return 1;
 }
 
