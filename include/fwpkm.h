@@ -176,6 +176,30 @@ fwpkm_status fwpkm_run_sequence_host(fwpkm_state* st, const void* q, const void*
                                      int T, int n_iter, float* o, void* scratch, size_t scratch_bytes,
                                      void* stream);
 
+/* The read path's backward: the gradient that reaches the slow weights' outputs q, v, g
+ * from an upstream dL/do ("Fast-weight Product Key Memory" (paperlayer summary) §2 /
+ * Figure 1: slow weights learn during training; §3.1-§3.2: the read o = g vhat + (1-g) v,
+ * vhat = sum_i s'_i V_i, s' = softmax over the selected slots of sigma_1 + sigma_2,
+ * sigma = -log(eps_idw + ||q_j - K_j||^2)).  The fast weights V, K1, K2 as they were when
+ * the tokens were read are constants (they learn only from their own chunk-local losses),
+ * and the discrete selection passes no gradient.  Per token with slots I (rank order):
+ *   dg = <dL/do, vhat - v>, dv = (1 - g) dL/do,
+ *   dq_j = sum_r dS_r (-2 / (eps_idw + D_j,r)) (q_j - K_j[row of slot r]),
+ *   dS = s' (ds - <s', ds>), ds_r = <g dL/do, V_{I_r}>;
+ * the distances and weights are recomputed from q, K1, K2 (direct form).  Stateless: no
+ * handle, no workspace.  cfg.v_heads > 1: FWPKM_ERR_UNSUPPORTED.
+ *   K1, K2, V   device fp32, the state the tokens were read with ([M][n][d/2], [M][n*n][d_v])
+ *   q, v, g     device, the forward_chunk layout (seq_stride >= len)
+ *   idx         device int32 [M][len][k]: the slots the forward read (forward_chunk's idx_out);
+ *               slots outside [0, N) contribute nothing
+ *   d_o         device fp32, (m, t, e) at d_o[(m*seq_stride + t)*d_v + e]
+ *   dq, dv, dg  device fp32 outputs in the q, v, g layouts (seq_stride)
+ * V, d_o and dv must be 16-byte aligned.  len = 0 is a no-op. */
+fwpkm_status fwpkm_read_backward(const fwpkm_config* cfg, const float* K1, const float* K2, const float* V,
+                                 const void* q, const void* v, const float* g, const int32_t* idx,
+                                 const float* d_o, int len, int seq_stride, float* dq, float* dv, float* dg,
+                                 void* stream);
+
 /* Token-at-a-time inference ("Fast-weight Product Key Memory" (paperlayer summary),
  * §A.1: at inference the memory accumulates (q_t, v_{t+1}) pairs and writes once a
  * chunk's worth is ready).  Each call reads n_tok >= 1 new tokens of every memory at once,

@@ -1123,6 +1123,27 @@ fwpkm_status fwpkm_run_sequence(fwpkm_state* st, const void* q, const void* v, c
   return run_sequence_impl(st, q, v, g, T, n_iter, o, nullptr, stream);
 }
 
+// ---- the read path's backward ----
+fwpkm_status fwpkm_read_backward(const fwpkm_config* cfg, const float* K1, const float* K2, const float* V,
+                                 const void* q, const void* v, const float* g, const int32_t* idx,
+                                 const float* d_o, int len, int seq_stride, float* dq, float* dv, float* dg,
+                                 void* stream) {
+  NvtxRange nvtx_range("fwpkm_read_backward");
+  fwpkm_status cs = check_cfg(cfg);
+  if (cs != FWPKM_OK) return cs;
+  if (cfg->v_heads > 1) return FWPKM_ERR_UNSUPPORTED;
+  if (len == 0) return FWPKM_OK;
+  if (len < 0 || seq_stride < len || !K1 || !K2 || !V || !q || !v || !g || !idx || !d_o || !dq || !dv || !dg)
+    return FWPKM_ERR_INVALID_ARG;
+  if (!aligned(V, 16) || !aligned(d_o, 16) || !aligned(dv, 16)) return FWPKM_ERR_INVALID_ARG;
+  const Dims d = make_dims(cfg);
+  cudaGetLastError();
+  const int nl = launch_read_backward(d, K1, K2, V, q, v, g, idx, d_o, len, seq_stride, dq, dv, dg,
+                                      (cudaStream_t)stream);
+  count_launches(nl);
+  return last_cuda();
+}
+
 // ---- host buffers: device copies of q, v, g, o in caller scratch ----
 static size_t host_io_carve(const Dims& d, int T, char* base, void** q, void** v, float** g, float** o) {
   const size_t es = qv_size(d);

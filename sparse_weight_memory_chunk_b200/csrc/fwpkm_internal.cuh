@@ -32,8 +32,8 @@ inline fwpkm_status status_of_device(int h) {
                               : h == DEV_BAD_SLOT ? FWPKM_ERR_BAD_SLOT : FWPKM_ERR_CUDA;
 }
 
-// Test hook of the timeout path (fwpkm_test_stall_waits): launches of the tensor-core
-// kernels that should wait once on a barrier that nothing completes.  Returns 1 (and
+// Test hook of the timeout path (fwpkm_test_stall_waits): launches of the kernels with
+// bounded waits that should wait once on something nothing completes.  Returns 1 (and
 // counts one down) while any remain.
 int take_test_stall();
 bool test_stalls_pending();
@@ -190,6 +190,10 @@ int launch_write(const Dims& d, const Work& w, float* V, int wt0, cudaStream_t s
 int launch_value_loop(const Dims& d, const Work& w, float* V, const void* v, const float* g, int T, int c0, int c1,
                       float* o, cudaStream_t s);
 bool value_loop_enabled();
+// The read path's backward (dq, dv, dg from dL/do) for `len` tokens of every memory.
+int launch_read_backward(const Dims& d, const float* K1, const float* K2, const float* V, const void* q,
+                         const void* v, const float* g, const int32_t* idx, const float* d_o, int len,
+                         long long stride, float* dq, float* dv, float* dg, cudaStream_t s);
 // Entropy key step for the chunk whose distances are in Dfull/Z (`len` tokens).
 int launch_address(const Dims& d, const Work& w, float* K1, float* K2, const void* q,
                    long long q_stride, int len, cudaStream_t s);

@@ -77,6 +77,8 @@ def lib():
             "fwpkm_forward_chunk": ([_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P], ctypes.c_int),
             "fwpkm_write_chunk": ([_P, _P, _P], ctypes.c_int),
             "fwpkm_run_sequence": ([_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P], ctypes.c_int),
+            "fwpkm_read_backward": ([C, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P],
+                                    ctypes.c_int),
             "fwpkm_run_sequence_host_scratch_size": ([C, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)],
                                                      ctypes.c_int),
             "fwpkm_run_sequence_host": ([_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, ctypes.c_size_t, _P],
@@ -154,6 +156,16 @@ def run_layer_scratch_size(cfg: Config, T: int) -> int:
     out = ctypes.c_size_t(0)
     _check(lib().fwpkm_run_layer_scratch_size(ctypes.byref(cfg), T, ctypes.byref(out)), "run_layer_scratch_size")
     return out.value
+
+
+def read_backward(cfg: Config, K1, K2, V, q, v, g, idx, d_o, dq, dv, dg, len_=None, seq_stride=None, stream=None):
+    """fwpkm_read_backward: dq, dv, dg (fp32, the q, v, g layouts) from d_o for the tokens
+    whose slots `idx` ([M][len][k]) the forward read with the state K1, K2, V."""
+    len_ = idx.shape[1] if len_ is None else len_
+    seq_stride = q.shape[1] if seq_stride is None else seq_stride
+    _check(lib().fwpkm_read_backward(ctypes.byref(cfg), _ptr(K1), _ptr(K2), _ptr(V), _ptr(q), _ptr(v), _ptr(g),
+                                     _ptr(idx), _ptr(d_o), len_, seq_stride, _ptr(dq), _ptr(dv), _ptr(dg),
+                                     _stream(stream)), "read_backward")
 
 
 def run_sequence_host_scratch_size(cfg: Config, T: int) -> int:
