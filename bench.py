@@ -559,6 +559,42 @@ def measure(args, w, rank, world, local_rank, n_iter, steps, warmup, full):
                          "frac": mbytes / (mms / 1e3) / 1e9 / hbm_peak, "algorithmic_bytes": mbytes,
                          "definition": "selections read once + N 32-bit counters per window written and read once"}}
 
+    # the read path's backward (dq, dv, dg from a seeded dL/do) for the first chunk of every
+    # memory, timed apart from the step; its slots are the final pass's
+    if full and layer is None and not args.no_metrics:
+        Cb = min(w.C, w.T)
+        idx_b = idx[:, :Cb].contiguous()
+        gen = torch.Generator(device=dev).manual_seed(5)
+        d_o = torch.randn(w.M, w.T, w.d_v, device=dev, generator=gen)
+        bq = torch.empty(w.M, w.T, w.d, device=dev)
+        bv = torch.empty(w.M, w.T, w.d_v, device=dev)
+        bg = torch.empty(w.M, w.T, device=dev)
+
+        def bwd():
+            fwpkm.read_backward(cfg, K1d, K2d, Vd, qd, vd, gd, idx_b, d_o, bq, bv, bg, len_=Cb, seq_stride=w.T,
+                                stream=stream)
+
+        for _ in range(3):
+            bwd()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        b0.record(stream)
+        for _ in range(reps):
+            bwd()
+        b1.record(stream)
+        torch.cuda.synchronize()
+        bms = b0.elapsed_time(b1) / reps
+        tm = w.M * Cb
+        es_b = 2 if w.qv == "bf16" else 4
+        bbytes = (tm * (w.k * w.d_v * 4 + w.k * 4 + (w.d + w.d_v) * es_b + 4 + w.d_v * 4 + (w.d + w.d_v + 1) * 4)
+                  + w.M * 2 * w.n * (w.d // 2) * 4)
+        line["read_backward"] = {
+            "token_memories": tm, "ms": bms, "token_memories_per_s": tm / (bms / 1e3),
+            "roofline": {"bound": "hbm", "achieved": bbytes / (bms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": bbytes / (bms / 1e3) / 1e9 / hbm_peak, "algorithmic_bytes": bbytes},
+            "definition": "fwpkm_read_backward over the first chunk of every memory: the selected V rows, q, v, g, "
+                          "slots and dL/do read once, dq, dv, dg written once, the keys read once per memory"}
+
     # end to end through the public API with host buffers: fwpkm_run_sequence_host (inputs
     # copied in and o copied out chunk by chunk, overlapped with the compute); the layer
     # workload copies h in and o' out around fwpkm_run_layer
