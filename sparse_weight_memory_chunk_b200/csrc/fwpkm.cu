@@ -244,12 +244,14 @@ int pbar_slices() {
   return v;
 }
 
+thread_local bool pdl_scope = false;
+
 bool pdl_enabled() {
-  static const bool on = [] {
+  static const int env = [] {  // 1: on everywhere, 0: off everywhere, -1: by scope
     const char* e = getenv("FWPKM_PDL");
-    return e && e[0] == '1';
+    return (e && e[0] == '1') ? 1 : (e && e[0] == '0') ? 0 : -1;
   }();
-  return on;
+  return env < 0 ? pdl_scope : env == 1;
 }
 
 // The tensor-core path needs bf16 queries (exact tcgen05 operands) and half widths that
@@ -687,6 +689,10 @@ fwpkm_status fwpkm_stream_tokens(fwpkm_state* st, const void* q, const void* v, 
   const size_t es = qv_size(d);
   const Work& wk = st->wk;
   st->host_error = 0;
+  // every kernel of the tensor-core path's reads and writes waits for its predecessor's
+  // results (griddepcontrol.wait) before it touches memory, so its launch may overlap
+  // the predecessor's tail
+  const PdlScope pdl(wk.tc);
   // bf16 pieces of the keys for the scoring GEMM: made at the start of every chunk (the
   // caller may change the keys between chunks, never inside one) and after a key step
   if (wk.tc && st->spos == 0) run(st, KK_PREP, s, [&] { return launch_keyprep(d, wk, st->K1, st->K2, s); });
@@ -729,6 +735,7 @@ fwpkm_status fwpkm_stream_flush(fwpkm_state* st, void* stream) {
   if (ps != FWPKM_OK) return ps;
   if (st->spos == 0) return FWPKM_OK;
   st->host_error = 0;
+  const PdlScope pdl(st->wk.tc);
   stream_write(st, false, (cudaStream_t)stream);
   if (st->host_error) return FWPKM_ERR_CUDA;
   return last_cuda();

@@ -238,10 +238,21 @@ int launch_addr_fused(const Dims& d, const Work& w, float* K1, float* K2, const 
 size_t addr_fused_part_floats(const Dims& d);
 
 // ---- launches ----
-// Whether kernels are launched with programmatic dependent launch (FWPKM_PDL=1; off by
-// default: on the paper-scale step the early-resident dependents held SM slots that the
-// other chains' kernels needed, 1.92 ms per step against 1.84 ms without).
+// Whether kernels are launched with programmatic dependent launch.  Off by default for the
+// chunk schedule (on the paper-scale step the early-resident dependents held SM slots that
+// the other chains' kernels needed: 1.53 ms per step against 1.42 ms without); on inside a
+// PdlScope, which the token-at-a-time calls on the tensor-core path open (their reads are
+// chains of small dependent launches on one stream: 26.8 us per token against 34.1 us at
+// one token per call).  FWPKM_PDL=1 turns it on everywhere, FWPKM_PDL=0 off everywhere.
 bool pdl_enabled();
+extern thread_local bool pdl_scope;
+struct PdlScope {
+  bool prev;
+  explicit PdlScope(bool on) : prev(pdl_scope) { pdl_scope = prev || on; }
+  ~PdlScope() { pdl_scope = prev; }
+  PdlScope(const PdlScope&) = delete;
+  PdlScope& operator=(const PdlScope&) = delete;
+};
 // With FWPKM_CARVEOUT=1, give `kern` the largest shared-memory carveout once per process,
 // so that an SM never has to drain to switch its L1/shared split before a CTA of another
 // kernel can start beside the running ones.  Off by default: the smaller L1 it leaves
