@@ -26,6 +26,7 @@ CASES = {
     "mid_bf16": (256, 128, 128, 16, 128, 2, 260, "bf16", False),
     "paper_shapes": (1024, 256, 256, 32, 256, 2, 300, "bf16", True),
     "odd_dims": (48, 40, 36, 5, 32, 2, 70, "f32", True),  # h = 20, d_v = 36: partial lanes
+    "k1_bf16": (64, 128, 64, 1, 32, 2, 70, "bf16", True),  # one slot: s' = 1, so dq = 0
 }
 
 
@@ -84,3 +85,46 @@ def test_read_backward_argument_checks():
         fwpkm.read_backward(heads, K1, K2, V, q, v, g, idx, d_o, *out, len_=C, seq_stride=T)
     assert e.value.status == fwpkm.ERR_UNSUPPORTED
     fwpkm.read_backward(cfg, K1, K2, V, q, v, g, idx, d_o, *out, len_=0, seq_stride=T)  # no-op
+
+
+def test_read_backward_drops_slots_outside_the_memory():
+    """Slots outside [0, N) contribute nothing: the token's softmax runs over its valid
+    slots only (the oracle is given just those), and a token with none has vhat = 0, so
+    dq = 0, dv = (1 - g) dL/do, dg = -<dL/do, v>."""
+    n, d, dv, k, C, M, T = 64, 64, 64, 8, 64, 2, 40
+    N = n * n
+    w = Workload("drop", n, d, dv, k, T, C, M, 1, "f32", False, 23, "sigmoid", "normal002")
+    q, v, g = gen_qvg(w)
+    K1, K2 = gen_keys(w)
+    V = np.stack([gen_values(w, m) for m in range(M)])
+    cfg = fwpkm.make_config(n, d, dv, k, C, M, False)
+    rng = np.random.default_rng(11)
+    I = np.stack([np.stack([rng.choice(N, size=k, replace=False) for _ in range(T)]) for _ in range(M)])
+    I = I.astype(np.int32)
+    drop = rng.random(I.shape) < 0.3
+    I[drop] = np.where(rng.random(int(drop.sum())) < 0.5, -1, N + 5).astype(np.int32)
+    I[0, 3, :] = -1                       # a token with no valid slot
+    I[1, 7, :] = N                        # another one, past the end
+    d_o = rng.normal(size=(M, T, dv)).astype(np.float32)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()  # noqa: E731
+    dq = torch.full((M, T, d), float("nan"), device="cuda")
+    dvv = torch.full((M, T, dv), float("nan"), device="cuda")
+    dg = torch.full((M, T), float("nan"), device="cuda")
+    fwpkm.read_backward(cfg, dev(K1), dev(K2), dev(V), dev(q), dev(v), dev(g), dev(I), dev(d_o),
+                        dq, dvv, dg, len_=T, seq_stride=T)
+    torch.cuda.synchronize()
+    dq, dvv, dg = dq.cpu().numpy(), dvv.cpu().numpy(), dg.cpu().numpy()
+    for m in range(M):
+        for t in range(T):
+            ok = I[m, t][(I[m, t] >= 0) & (I[m, t] < N)]
+            if ok.size == 0:
+                assert np.all(dq[m, t] == 0.0), f"mem {m} token {t}: dq"
+                assert np.array_equal(dvv[m, t], (np.float32(1.0) - g[m, t]) * d_o[m, t]), f"mem {m} token {t}: dv"
+                assert_close(np.array([dg[m, t]]), np.array([-np.dot(d_o[m, t].astype(np.float64), v[m, t])]),
+                             f"mem {m} token {t}: dg")
+                continue
+            rq, rv, rg = oracle_read_backward(n, cfg.eps_idw, q[m, t:t + 1], v[m, t:t + 1], g[m, t:t + 1],
+                                              K1[m], K2[m], V[m], ok[None, :], d_o[m, t:t + 1])
+            assert_close(dq[m, t:t + 1], rq, f"mem {m} token {t}: dq")
+            assert_close(dvv[m, t:t + 1], rv, f"mem {m} token {t}: dv")
+            assert_close(dg[m, t:t + 1], rg, f"mem {m} token {t}: dg")
