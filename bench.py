@@ -698,8 +698,8 @@ def measure(args, w, rank, world, local_rank, n_iter, steps, warmup, full):
             "definition": "tokens of the first 2C+1 positions of every sequence fed n per fwpkm_stream_tokens call, "
                           "then fwpkm_stream_flush; tokens/s counts sequence tokens (B per position); "
                           "hbm_bytes_per_token_max: gathered rows + the same rows read and written by the chunk "
-                          "write (unique rows), all memories; latency-bound: a token's read is a chain of about "
-                          "six dependent launches"}
+                          "write (unique rows), all memories; latency-bound: a token's read is a chain of four "
+                          "dependent launches (staging with the query norms, scoring, selection, gather)"}
 
     st.destroy()
     if layer is not None:

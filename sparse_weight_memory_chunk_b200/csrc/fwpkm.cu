@@ -622,9 +622,9 @@ static void stream_read(fwpkm_state* st, const void* v, const float* g, long lon
   const void* qs = offs(wk.stage_q, (long long)p * d.d, es);
   if (wk.tc) {
     // with the fused key step the reads take their distances from the same kernel (scoring
-    // only), so a token read here gets the bits it gets inside a whole chunk
+    // only), so a token read here gets the bits it gets inside a whole chunk; the staging
+    // launch has already written these tokens' query norms
     const bool fused = (d.flags & FWPKM_KEY_UPDATE) && use_fused_addressing(d);
-    run(st, KK_PREP, s, [&] { return launch_qnorm(d, wk, qs, d.C, p, len, s); });
     if (fused)
       run(st, KK_FUSED, s, [&] {
         return launch_addr_fused(d, wk, st->K1, st->K2, wk.stage_q, d.C, d.C, p, p, len, 0, true, s);
@@ -712,7 +712,11 @@ fwpkm_status fwpkm_stream_tokens(fwpkm_state* st, const void* q, const void* v, 
         {offs(q, (long long)j * d.d, es), wk.stage_q, seq_stride, d.C, (int)(d.d * es / 4)},
         {offs(v, (long long)j * d.dv, es), wk.stage_v, seq_stride, d.C + 1, (int)(d.dv * es / 4)},
         {g + j, wk.stage_g, seq_stride, d.C + 1, 1}};
-    run(st, KK_PREP, s, [&] { return launch_stage(d, in, st->spos, len, s); });
+    // on the tensor-core path the same launch writes the tokens' query norms
+    run(st, KK_PREP, s, [&] {
+      return wk.tc ? launch_stage(d, in, st->spos, len, s, &wk, offs(q, (long long)j * d.d, es), seq_stride)
+                   : launch_stage(d, in, st->spos, len, s);
+    });
     stream_read(st, offs(v, (long long)j * d.dv, es), g + j, seq_stride, len, o + (long long)j * d.dv, s);
     st->spos += len;
     j += len;

@@ -177,7 +177,10 @@ struct StageJob {
   long long src_stride, dst_stride;
   int words;
 };
-int launch_stage(const Dims& d, const StageJob (&jobs)[3], int r0, int len, cudaStream_t s);
+// With `qn_src` (bf16 queries of the staged tokens, per memory `qn_stride` rows apart), the
+// same launch also writes their squared half norms to w.qn at tokens r0.. (qnorm_row).
+int launch_stage(const Dims& d, const StageJob (&jobs)[3], int r0, int len, cudaStream_t s,
+                 const Work* w = nullptr, const void* qn_src = nullptr, long long qn_stride = 0);
 // Streaming write path: turn the stored vhat of a chunk into residuals.
 int launch_resid(const Dims& d, const Work& w, const void* v, const float* g, long long stride,
                  int len, const void* v_next, cudaStream_t s);
@@ -367,6 +370,23 @@ __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
+}
+
+// ||q_half||^2 of one bf16 query row (both halves) by one warp into w.qn[m][half][t]: each
+// lane sums its strided features in order, then a warp sum.  The chunk path's query-norm
+// kernel and the token-at-a-time staging kernel both use it, so their norms have the same
+// bits.
+__device__ __forceinline__ void qnorm_row(const Dims& dm, const Work& w, const __nv_bfloat16* __restrict__ row,
+                                          int m, long long t, int lane) {
+  for (int j = 0; j < 2; ++j) {
+    float s = 0.f;
+    for (int e = lane; e < dm.h; e += 32) {
+      float x = __bfloat162float(row[j * dm.h + e]);
+      s += x * x;
+    }
+    s = warp_sum(s);
+    if (lane == 0) w.qn[((size_t)m * 2 + j) * w.max_T + t] = s;
+  }
 }
 
 }  // namespace fwpkm

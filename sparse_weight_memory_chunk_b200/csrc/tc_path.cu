@@ -31,16 +31,7 @@ qnorm_kernel(Dims dm, Work w, const __nv_bfloat16* __restrict__ q, long long q_s
   const int i = blockIdx.x * (TP_THREADS / 32) + warp;
   const int m = blockIdx.y;
   if (i >= len) return;
-  const __nv_bfloat16* row = q + ((long long)m * q_stride + i) * dm.d;
-  for (int j = 0; j < 2; ++j) {
-    float s = 0.f;
-    for (int e = lane; e < dm.h; e += 32) {
-      float x = __bfloat162float(row[j * dm.h + e]);
-      s += x * x;
-    }
-    s = warp_sum(s);
-    if (lane == 0) w.qn[((size_t)m * 2 + j) * w.max_T + wt0 + i] = s;
-  }
+  qnorm_row(dm, w, q + ((long long)m * q_stride + i) * dm.d, m, (long long)wt0 + i, lane);
 }
 
 // bf16 pieces and squared norm of every key: four threads per (problem, sub-key), thread g

@@ -741,15 +741,25 @@ int launch_resid(const Dims& d, const Work& w, const void* v, const float* g, lo
   return 1;
 }
 
-// Token-at-a-time inference: copy rows of up to three inputs into the staging buffers.
+// Token-at-a-time inference: copy rows of up to three inputs into the staging buffers
+// (grid z = 0..2), and with `qn_src` the staged queries' half norms (grid z = 3, one warp
+// per token, read from the source rows).
 struct StageJobs {
   StageJob j[3];
   int r0, len;
+  const __nv_bfloat16* qn_src;
+  long long qn_stride;
 };
 
-__global__ void __launch_bounds__(256) stage_kernel(StageJobs jobs) {
+__global__ void __launch_bounds__(256) stage_kernel(StageJobs jobs, Dims dm, Work w) {
   pdl_wait();  // the previous chunk's write may still read the staging rows
   pdl_trigger();
+  if (blockIdx.z == 3) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, m = blockIdx.y;
+    for (int i = blockIdx.x * 8 + warp; i < jobs.len; i += gridDim.x * 8)
+      qnorm_row(dm, w, jobs.qn_src + ((long long)m * jobs.qn_stride + i) * dm.d, m, (long long)jobs.r0 + i, lane);
+    return;
+  }
   const StageJob& J = jobs.j[blockIdx.z];
   if (J.src == nullptr) return;
   const int m = blockIdx.y;
@@ -760,7 +770,8 @@ __global__ void __launch_bounds__(256) stage_kernel(StageJobs jobs) {
     dst[i] = src[i];
 }
 
-int launch_stage(const Dims& d, const StageJob (&jobs)[3], int r0, int len, cudaStream_t s) {
+int launch_stage(const Dims& d, const StageJob (&jobs)[3], int r0, int len, cudaStream_t s, const Work* w,
+                 const void* qn_src, long long qn_stride) {
   if (len <= 0) return 0;
   StageJobs J;
   int words = 1;
@@ -770,9 +781,12 @@ int launch_stage(const Dims& d, const StageJob (&jobs)[3], int r0, int len, cuda
   }
   J.r0 = r0;
   J.len = len;
+  const bool norms = w != nullptr && qn_src != nullptr;
+  J.qn_src = norms ? (const __nv_bfloat16*)qn_src : nullptr;
+  J.qn_stride = qn_stride;
   long long bx = ((long long)len * words + 255) / 256;
   if (bx > 64) bx = 64;
-  launch_k(stage_kernel, dim3((unsigned)bx, d.M, 3), 256, 0, s, J);
+  launch_k(stage_kernel, dim3((unsigned)bx, d.M, norms ? 4 : 3), 256, 0, s, J, d, norms ? *w : Work{});
   return 1;
 }
 
